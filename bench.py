@@ -1,0 +1,422 @@
+#!/usr/bin/env python
+"""Benchmark of the padding-free MoE layer hot path (forward + RBD plan + backward).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = moe_route -> pft_build -> moe_dispatch -> moe_expert_ffn -> moe_combine
+-> rbd_plan -> moe_backward over one batch of synthetic tokens, inputs and weights
+resident in HBM.  Rank 0 prints one JSON line.  With N > 1 (torchrun, one process
+per GPU) every rank runs an independent replica on its own tokens: the layer has no
+exchange step on one GPU, so there is no data-path collective; the timed region is
+bracketed by barriers and the reported time is the max over ranks.
+
+``--impl reference`` times the float64 CPU oracle (test infrastructure) on the
+host cores, on bounded token samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer fwd+bwd tokens/s; grouped-GEMM % of BF16 peak; dispatch/combine GB/s"
+DEFAULT_WORKLOAD = "dsmoe16b_bf16"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=512)
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "200"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------- algorithmic work per kernel
+def kernel_work(cfg, name):
+    """(kind, amount per launch): FLOPs for contractions, bytes for data movement."""
+    T, d, E, h, k, N = cfg.T, cfg.d, cfg.E, cfg.h, cfg.k, cfg.N
+    b = 2 if cfg.dtype == "bf16" else 4
+    flops = {
+        "ffn_gemm1_swiglu": 2.0 * N * d * 2 * h,
+        "ffn_gemm2": 2.0 * N * h * d,
+        "ffn_dgrad_act_swiglu_bwd": 2.0 * N * d * h,
+        "ffn_dgrad_x": 2.0 * N * 2 * h * d,
+        "ffn_wgrad_w1w3": 2.0 * N * d * 2 * h,
+        "ffn_wgrad_w2": 2.0 * N * h * d,
+        "gate_logits": 2.0 * T * d * E,
+        "gate_wgrad": 2.0 * T * d * E,
+    }
+    if name in flops:
+        return "tensor", flops[name]
+    bytes_ = {
+        "dispatch": (T + N) * d * b + 4 * N,
+        "combine": N * d * b + T * d * b + 8 * N,
+        "combine_bwd": T * d * b + 2 * N * d * b + 12 * N,
+        "token_grad": N * d * b + T * d * b + T * E * (4 + 2) + 16 * N,
+        "route_topk": T * E * 4 + 8 * N,
+        "pft_hist": 4 * N,
+        "pft_scatter": 8 * N + 16 * N,
+        "transpose": 2 * d * E * b,
+    }
+    if name in bytes_:
+        return "hbm", float(bytes_[name])
+    return None, None
+
+
+def gemm_names():
+    return ["ffn_gemm1_swiglu", "ffn_gemm2", "ffn_dgrad_act_swiglu_bwd", "ffn_dgrad_x", "ffn_wgrad_w1w3",
+            "ffn_wgrad_w2"]
+
+
+def traffic_for(kernel):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel source has not changed since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    ent = t.get(kernel)
+    if not ent:
+        return None
+    src = os.path.join(ROOT, ent["source"])
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    if sha != ent.get("source_sha256"):
+        return None
+    return ent["dram_bytes_per_launch"]
+
+
+# -------------------------------------------------------------- CPU oracle leg
+def oracle_sample(inp_cpu64, cfg, n_tok, seed=0):
+    """Time the float64 oracle's full layer (forward + backward) on n_tok tokens."""
+    import numpy as np
+    import oracle as O
+    rng = np.random.default_rng(seed)
+    toks = np.sort(rng.choice(cfg.T, size=min(n_tok, cfg.T), replace=False))
+    x, wg, bias, w1, w3, w2, dy = inp_cpu64
+    t0 = time.perf_counter()
+    f = O.layer_forward(x[toks], wg, bias, w1, w3, w2, cfg.k)
+    O.layer_backward(f, dy[toks], x[toks], wg, w1, w3, w2)
+    if cfg.has_rbd:
+        O.rbd_plan(f["ids"], cfg.E, cfg.rbd_epd, cfg.rbd_dpn)
+    return len(toks), time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def inputs_to_cpu64(inp):
+    import torch
+    cv = lambda t: None if t is None else t.detach().to("cpu").to(torch.float64).numpy()
+    return tuple(cv(t) for t in (inp.x, inp.wg, inp.bias, inp.w1, inp.w3, inp.w2, inp.dy))
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle as it stands, on bounded token samples of the workload."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from workloads import get_config, make_inputs
+    cfg = get_config(args.workload)
+    inp = make_inputs(cfg, seed=0, device="cpu")
+    cpu = inputs_to_cpu64(inp)
+    n_tok = max(1, min(args.cpu_sample_tokens // 4, cfg.T))
+    for _ in range(args.warmup):
+        oracle_sample(cpu, cfg, n_tok)
+    tot_tok, tot_s = 0, 0.0
+    for i in range(args.steps):
+        n, s = oracle_sample(cpu, cfg, n_tok, seed=i + 1)
+        tot_tok += n
+        tot_s += s
+    value = tot_tok / tot_s
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(cfg, world),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n_tok} random tokens of {cfg.name} per step through the float64 oracle "
+                                   f"(forward, RBD plan, backward)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(cfg, world):
+    return {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "h": cfg.h, "k": cfg.k,
+            "tokens_per_gpu": cfg.T, "global_batch": cfg.T * world,
+            "rbd_map": (f"{cfg.rbd_epd} experts/device, {cfg.rbd_dpn} devices/node" if cfg.has_rbd else None),
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "inputs larger than L2 (expert weights alone exceed 126 MB)"}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    rank, world, local_rank = dist_env()
+    import torch
+    import torch.distributed as dist
+    from padding_free_moe_b200 import _lib as L
+    from padding_free_moe_b200.layer import PFTMoELayer, Shape
+    from workloads import get_config, make_inputs
+    from workloads.generate import storage_dtype
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank)
+    cfg = get_config(args.workload)
+    inp = make_inputs(cfg, seed=1000 + rank, device=dev)
+    layer = PFTMoELayer(Shape(cfg.T, cfg.d, cfg.E, cfg.h, cfg.k, storage_dtype(cfg), cfg.rbd_epd, cfg.rbd_dpn), dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.step(inp.x, inp.wg, inp.bias, inp.w1, inp.w3, inp.w2, inp.dy, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    warm = max(3, args.warmup)
+    for _ in range(warm):
+        step()
+    torch.cuda.synchronize()
+    if layer.device_error() != 0:
+        raise RuntimeError(f"device error word {layer.device_error():#x} after warm-up")
+
+    # ---- device-timed region, inputs resident; per-kernel events live
+    clk = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                       int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    L.moe_profile_reset()
+    barrier()
+    torch.cuda.synchronize()
+    clk.start()
+    L.moe_profile_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    L.moe_profile_enable(False)
+    barrier()
+    clocks = clk.stop()
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1))
+    kern = L.moe_profile_read()
+    ms_step = ms_total / args.steps
+    value = world * cfg.T / (ms_step * 1e-3)
+
+    # ---- end to end through the public API: pinned host inputs in, results out, every step
+    x_h = inp.x.to("cpu").pin_memory()
+    dy_h = inp.dy.to("cpu").pin_memory()
+    y_h = torch.empty_like(layer.y, device="cpu").pin_memory()
+    dx_h = torch.empty_like(layer.dx, device="cpu").pin_memory()
+    x_d, dy_d = torch.empty_like(inp.x), torch.empty_like(inp.dy)
+    e2e_steps = max(3, min(args.steps, 10))
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        dy_d.copy_(dy_h, non_blocking=True)
+        layer.step(x_d, inp.wg, inp.bias, inp.w1, inp.w3, inp.w2, dy_d, stream)
+        y_h.copy_(layer.y, non_blocking=True)
+        dx_h.copy_(layer.dx, non_blocking=True)
+        stream.synchronize()
+
+    e2e_step()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+    h2d = x_h.numel() * x_h.element_size() + dy_h.numel() * dy_h.element_size()
+    d2h = y_h.numel() * y_h.element_size() + dx_h.numel() * dx_h.element_size()
+    if layer.device_error() != 0:
+        raise RuntimeError(f"device error word {layer.device_error():#x}")
+
+    # ---- roofline of the dominant kernel + per-kernel table
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
+    tc_peak = float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
+    kernels = {}
+    for nm, (n_launch, ms) in sorted(kern.items(), key=lambda kv: -kv[1][1]):
+        per_ms = ms / n_launch
+        kind, work = kernel_work(cfg, nm)
+        ent = {"launches": n_launch, "ms_per_launch": per_ms, "share": ms / sum(v[1] for v in kern.values())}
+        if kind == "tensor":
+            ent["tflops"] = work / (per_ms * 1e-3) / 1e12
+            ent["frac_of_peak"] = ent["tflops"] / tc_peak
+        elif kind == "hbm":
+            ent["gbs"] = work / (per_ms * 1e-3) / 1e9
+            ent["frac_of_peak"] = ent["gbs"] / hbm
+        kernels[nm] = ent
+    dom = max(kern.items(), key=lambda kv: kv[1][1])[0]
+    kind, work = kernel_work(cfg, dom)
+    dom_ms = kern[dom][1] / kern[dom][0]
+    if kind == "tensor":
+        ach = work / (dom_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": ach / tc_peak, "traffic": traffic_for(dom),
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+                "work_per_launch": work}
+    else:
+        ach = work / (dom_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                "traffic": traffic_for(dom), "peak_source": f"{peak_src} hbm_gbs", "work_per_launch": work}
+    gemm_ms = sum(kern[n][1] for n in gemm_names() if n in kern) / args.steps
+    gemm_flops = 18.0 * cfg.N * cfg.d * cfg.h
+    gemm_tflops = gemm_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
+
+    def gbs(nm):
+        return kernels.get(nm, {}).get("gbs")
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": warm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": config_block(cfg, world),
+        "clocks": clocks,
+        "e2e": {"value": world * cfg.T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": int(sum(v[0] for v in kern.values())),
+        "roofline": roof,
+        "grouped_gemm": {"tflops": gemm_tflops, "pct_of_bf16_peak": (100 * gemm_tflops / tc_peak) if gemm_tflops else None,
+                         "pct_of_burst_peak": (100 * gemm_tflops / float(peaks.get("bf16_tflops", 1590.0)))
+                         if gemm_tflops else None,
+                         "flops_per_step": gemm_flops, "ms_per_step": gemm_ms},
+        "dispatch_gbs": gbs("dispatch"), "combine_gbs": gbs("combine"),
+        "kernels": kernels,
+    }
+
+    # ---- CPU oracle baseline (rank 0, one GPU only)
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = inputs_to_cpu64(inp)
+        n, s = oracle_sample(cpu, cfg, args.cpu_sample_tokens)
+        line["cpu_baseline"] = {"value": n / s, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"{n} random tokens of {cfg.name} through the float64 oracle "
+                                          f"(forward, RBD plan, backward), {s:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

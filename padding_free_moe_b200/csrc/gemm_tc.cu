@@ -1,0 +1,802 @@
+// Persistent grouped GEMM on the 5th-generation tensor cores (sm_100a):
+// TMA -> shared memory ring -> tcgen05.mma (one issuing thread) -> TMEM
+// accumulators (double-buffered) -> register epilogue.
+//
+// D[M, N] = A[M, K] * B[N, K]^T, BF16 operands, FP32 accumulation.
+//
+// Two grouping modes cover every contraction of the padding-free MoE layer:
+//   RG (row-grouped): A's rows are split into expert segments [seg[g], seg[g+1])
+//      (the expert-sorted PFT rows, X-MoE article §2.1.2: one GEMM per expert
+//      over its unpadded rows).  Each segment uses its own weight matrix
+//      B_g (3-D tensor map, g = third coordinate).  M tiles of 128 rows may
+//      straddle the segment end; rows past it are computed but never stored.
+//   KG (K-grouped): the reduction dimension is split into segments (weight
+//      gradients dW_g = X_g^T dH_g); each group writes its own [M, N] output.
+//      K rows past the segment end are zeroed in shared memory before the MMA.
+//
+// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and
+// TMEM allocator), warps 2..5 = epilogue (one accumulator row per thread).
+// Every wait on an mbarrier is bounded (%globaltimer); on expiry the kernel
+// sets PFMOE_DEV_TIMEOUT, drains its own copies and MMAs, frees TMEM, returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+#include <type_traits>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace pfmoe {
+namespace tc {
+
+constexpr int BM = 128;          // MMA M (one CTA)
+constexpr int BK = 64;           // K elements per stage (one 128-byte swizzle row of BF16)
+constexpr int MAX_STAGES = 8;
+constexpr int THREADS = 192;
+constexpr int BOX_BYTES = 64 * 128;      // one 64 x 64 BF16 box (MN-major block)
+constexpr int A_BYTES = BM * BK * 2;     // 16 KB
+constexpr unsigned long long kTimeoutNs = 2000000000ull;
+
+enum Mode { RG = 0, KG = 1 };
+enum Epi { EPI_STORE_BF16 = 0, EPI_STORE_F32 = 1, EPI_SWIGLU_FWD = 2, EPI_SWIGLU_BWD = 3, EPI_SPLIT_BF16 = 4 };
+
+struct Params {
+  CUtensorMap tmA[2];
+  CUtensorMap tmB[2];
+  int mode;
+  int b_major;       // RG: 0 = K-major B (weights [G, N, K]), 1 = MN-major B (weights [G, K, N]); KG: 1
+  int bn;            // MMA N: multiple of 64, <= 256
+  int nsplit;        // 1: B tile columns [0, bn/2) come from tmB[0], [bn/2, bn) from tmB[1]
+  int M;             // KG: rows of each group's output
+  int Nout;          // output columns
+  int k0_blocks;     // RG: 64-wide K blocks read from source 0
+  int k1_blocks;     // RG: then from source 1 (K split; 0 = none)
+  const int* seg;    // [G+1] segment offsets, or null for one dense segment [0, dense_len)
+  const int* tiles;  // RG: [G+1] prefix of 128-row M tiles per group (null when dense)
+  int G;
+  int dense_len;
+  int stages;
+  void* D0;
+  void* D1;
+  void* D2;
+  const void* X0;    // SWIGLU_BWD: H1
+  const void* X1;    // SWIGLU_BWD: H3
+  const float* bias; // STORE_F32: optional per-column bias
+  long long ldd;     // output row stride (elements)
+  long long d_gstride;  // KG: elements between consecutive groups' outputs
+  int32_t* err;
+};
+
+struct Tile {
+  int g;
+  int row0;    // RG: first PFT row; KG: first output row (M)
+  int rows;    // valid rows (<= 128)
+  int n0;      // first output column
+  int nk;      // K blocks
+  int krow0;   // KG: first K row of the segment
+  int kvalid;  // KG: valid K rows in the last block
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ uint32_t mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok;
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait.  Returns false if the wait expired or another role aborted.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         int32_t* err, bool honour_abort = true) {
+  for (int i = 0; i < 128; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (honour_abort && *abort_flag) return false;
+    if (globaltimer() - t0 > kTimeoutNs) {
+      *abort_flag = 1;
+      dev_error(err, PFMOE_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, uint32_t bar, int c0, int c1,
+                                            int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* tm) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i gets lane (base lane + i).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format: version 1 at bit 46,
+// layout type 2 = SWIZZLE_128B at bits 61..63; addresses and offsets in 16-byte units).
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+// Instruction descriptor for kind::f16: D=F32, A=B=BF16, dense, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn) << 15) |
+         (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// ----------------------------------------------------------------- tile schedule
+__device__ __forceinline__ int n_step(const Params& p) { return p.nsplit ? p.bn / 2 : p.bn; }
+
+__device__ __forceinline__ int total_tiles(const Params& p) {
+  const int ns = n_step(p);
+  const int NT = (p.Nout + ns - 1) / ns;
+  if (p.mode == RG) {
+    const int mt = p.tiles ? p.tiles[p.G] : (p.dense_len + BM - 1) / BM;
+    return mt * NT;
+  }
+  return p.G * ((p.M + BM - 1) / BM) * NT;
+}
+
+__device__ __forceinline__ Tile decode(const Params& p, int t) {
+  Tile tl;
+  const int ns = n_step(p);
+  const int NT = (p.Nout + ns - 1) / ns;
+  if (p.mode == RG) {
+    int g = 0, tbase = 0, mtg, s0, s1;
+    if (p.tiles) {
+      int lo = 0, hi = p.G - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.tiles[mid] * NT <= t) lo = mid; else hi = mid - 1;
+      }
+      g = lo;
+      tbase = p.tiles[g] * NT;
+      mtg = p.tiles[g + 1] - p.tiles[g];
+      s0 = p.seg[g];
+      s1 = p.seg[g + 1];
+    } else {
+      mtg = (p.dense_len + BM - 1) / BM;
+      s0 = 0;
+      s1 = p.dense_len;
+    }
+    const int local = t - tbase;
+    const int n_idx = local / mtg;
+    const int m_loc = local - n_idx * mtg;
+    tl.g = g;
+    tl.row0 = s0 + m_loc * BM;
+    tl.rows = min(BM, s1 - tl.row0);
+    tl.n0 = n_idx * ns;
+    tl.nk = p.k0_blocks + p.k1_blocks;
+    tl.krow0 = 0;
+    tl.kvalid = BK;
+  } else {
+    const int MT = (p.M + BM - 1) / BM;
+    const int per = MT * NT;
+    const int g = t / per;
+    const int rem = t - g * per;
+    const int n_idx = rem / MT;
+    const int m_idx = rem - n_idx * MT;
+    const int s0 = p.seg ? p.seg[g] : 0;
+    const int s1 = p.seg ? p.seg[g + 1] : p.dense_len;
+    const int len = max(0, s1 - s0);
+    tl.g = g;
+    tl.row0 = m_idx * BM;
+    tl.rows = min(BM, p.M - tl.row0);
+    tl.n0 = n_idx * ns;
+    tl.nk = (len + BK - 1) / BK;
+    tl.krow0 = s0;
+    tl.kvalid = len - (tl.nk - 1) * BK;
+  }
+  return tl;
+}
+
+// -------------------------------------------------------------------- epilogue
+template <typename T>
+__device__ __forceinline__ void store_row_chunk(T* dst, const float* v, int ncols_valid) {
+  // Store up to 32 values of one row; ncols_valid is a multiple of 8 (BF16) or 4 (F32) or >= 32.
+  constexpr int VN = Vec<T>::n;
+#pragma unroll
+  for (int i = 0; i < 32; i += VN)
+    if (i < ncols_valid) store16<T>(dst + i, v + i);
+}
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, uint32_t tacc, int r) {
+  const bool row_ok = r < tl.rows;
+  const long long grow = static_cast<long long>(tl.row0) + r;
+  const bool zero = tl.nk == 0;
+  if constexpr (EPI == EPI_STORE_BF16 || EPI == EPI_STORE_F32) {
+    using T = typename std::conditional<EPI == EPI_STORE_F32, float, __nv_bfloat16>::type;
+    T* D = static_cast<T*>(p.D0) + (p.mode == KG ? tl.g * p.d_gstride : 0);
+    for (int c = 0; c < p.bn; c += 32) {
+      const int col = tl.n0 + c;
+      if (col >= p.Nout) break;
+      float v[32];
+      if (!zero) tmem_ld32(tacc + c, v);
+      else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      }
+      if (EPI == EPI_STORE_F32 && p.bias) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (col + i < p.Nout) v[i] += p.bias[col + i];
+      }
+      if (row_ok) store_row_chunk<T>(D + grow * p.ldd + col, v, p.Nout - col);
+    }
+  } else if constexpr (EPI == EPI_SWIGLU_FWD) {
+    // D columns [0, bn/2) = H1 tile, [bn/2, bn) = H3 tile for the same output columns.
+    const int half = p.bn / 2;
+    __nv_bfloat16* H1 = static_cast<__nv_bfloat16*>(p.D0);
+    __nv_bfloat16* H3 = static_cast<__nv_bfloat16*>(p.D1);
+    __nv_bfloat16* A = static_cast<__nv_bfloat16*>(p.D2);
+    for (int c = 0; c < half; c += 32) {
+      const int col = tl.n0 + c;
+      if (col >= p.Nout) break;
+      float h1[32], h3[32], a[32];
+      tmem_ld32(tacc + c, h1);
+      tmem_ld32(tacc + half + c, h3);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) a[i] = silu_f(h1[i]) * h3[i];
+      if (row_ok) {
+        const long long off = grow * p.ldd + col;
+        store_row_chunk(H1 + off, h1, p.Nout - col);
+        store_row_chunk(H3 + off, h3, p.Nout - col);
+        store_row_chunk(A + off, a, p.Nout - col);
+      }
+    }
+  } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+    // Accumulator = dA.  dH1 = dA * H3 * s * (1 + H1 (1 - s)), dH3 = dA * SiLU(H1), s = sigmoid(H1).
+    const __nv_bfloat16* H1 = static_cast<const __nv_bfloat16*>(p.X0);
+    const __nv_bfloat16* H3 = static_cast<const __nv_bfloat16*>(p.X1);
+    __nv_bfloat16* dH1 = static_cast<__nv_bfloat16*>(p.D0);
+    __nv_bfloat16* dH3 = static_cast<__nv_bfloat16*>(p.D1);
+    for (int c = 0; c < p.bn; c += 32) {
+      const int col = tl.n0 + c;
+      if (col >= p.Nout) break;
+      float da[32];
+      tmem_ld32(tacc + c, da);
+      if (row_ok) {
+        const long long off = grow * p.ldd + col;
+        const int nv = p.Nout - col;
+        float h1[32], h3[32], o1[32], o3[32];
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          if (i < nv) {
+            load16(H1 + off + i, h1 + i);
+            load16(H3 + off + i, h3 + i);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) h1[i + j] = h3[i + j] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float s = 1.0f / (1.0f + expf(-h1[i]));
+          o1[i] = da[i] * h3[i] * s * (1.0f + h1[i] * (1.0f - s));
+          o3[i] = da[i] * h1[i] * s;
+        }
+        store_row_chunk(dH1 + off, o1, nv);
+        store_row_chunk(dH3 + off, o3, nv);
+      }
+    }
+  } else if constexpr (EPI == EPI_SPLIT_BF16) {
+    // KG with nsplit: columns [0, bn/2) -> D0[g], [bn/2, bn) -> D1[g].
+    const int half = p.bn / 2;
+    __nv_bfloat16* D0 = static_cast<__nv_bfloat16*>(p.D0) + tl.g * p.d_gstride;
+    __nv_bfloat16* D1 = static_cast<__nv_bfloat16*>(p.D1) + tl.g * p.d_gstride;
+    for (int c = 0; c < half; c += 32) {
+      const int col = tl.n0 + c;
+      if (col >= p.Nout) break;
+      float v0[32], v1[32];
+      if (!zero) {
+        tmem_ld32(tacc + c, v0);
+        tmem_ld32(tacc + half + c, v1);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v0[i] = v1[i] = 0.f;
+      }
+      if (row_ok) {
+        const long long off = grow * p.ldd + col;
+        store_row_chunk(D0 + off, v0, p.Nout - col);
+        store_row_chunk(D1 + off, v1, p.Nout - col);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------- kernel
+template <int EPI>
+__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages;
+  const uint32_t b_bytes = static_cast<uint32_t>(p.bn) * BK * 2;
+  const uint32_t stage_bytes = A_BYTES + b_bytes;
+  uint8_t* bar_area = smem + S * stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
+  uint64_t* empty = full + MAX_STAGES;
+  uint64_t* acc_full = empty + MAX_STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t tmem_cols = p.bn * 2 <= 128 ? 128 : (p.bn * 2 <= 256 ? 256 : 512);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&acc_full[b]), 1);
+      mbar_init(smem_u32(&acc_empty[b]), 4 * 32);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&p.tmA[0]);
+    prefetch_tmap(&p.tmB[0]);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int ntiles = total_tiles(p);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t pending = 0;        // stages with an issued load
+      uint32_t pend_parity = 0;    // parity of that load's phase
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const Tile tl = decode(p, t);
+        for (int kb = 0; kb < tl.nk; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!wait_bar(smem_u32(&empty[s]), ph ^ 1, abort_flag, p.err)) { ok = false; break; }
+          const uint32_t fb = smem_u32(&full[s]);
+          mbar_expect_tx(fb, stage_bytes);
+          const uint32_t sa = smem_u32(smem + s * stage_bytes);
+          const uint32_t sb = sa + A_BYTES;
+          const int nb = p.bn / 64;
+          if (p.mode == RG) {
+            const int src = kb < p.k0_blocks ? 0 : 1;
+            const int kk = (src == 0 ? kb : kb - p.k0_blocks) * BK;
+            tma_load_3d(sa, &p.tmA[src], fb, kk, tl.row0, 0);
+            if (p.b_major == 0) {
+              if (p.nsplit) {
+                tma_load_3d(sb, &p.tmB[0], fb, kk, tl.n0, tl.g);
+                tma_load_3d(sb + (p.bn / 2) * 128, &p.tmB[1], fb, kk, tl.n0, tl.g);
+              } else {
+                tma_load_3d(sb, &p.tmB[src], fb, kk, tl.n0, tl.g);
+              }
+            } else {
+              for (int j = 0; j < nb; ++j) {
+                int which = src, nc = tl.n0 + 64 * j;
+                if (p.nsplit) {
+                  which = j < nb / 2 ? 0 : 1;
+                  nc = tl.n0 + 64 * (j < nb / 2 ? j : j - nb / 2);
+                }
+                tma_load_3d(sb + j * BOX_BYTES, &p.tmB[which], fb, nc, kk, tl.g);
+              }
+            }
+          } else {
+            const int krow = tl.krow0 + kb * BK;
+            tma_load_3d(sa, &p.tmA[0], fb, tl.row0, krow, 0);
+            tma_load_3d(sa + BOX_BYTES, &p.tmA[0], fb, tl.row0 + 64, krow, 0);
+            for (int j = 0; j < nb; ++j) {
+              int which = 0, nc = tl.n0 + 64 * j;
+              if (p.nsplit) {
+                which = j < nb / 2 ? 0 : 1;
+                nc = tl.n0 + 64 * (j < nb / 2 ? j : j - nb / 2);
+              }
+              tma_load_3d(sb + j * BOX_BYTES, &p.tmB[which], fb, nc, krow, 0);
+            }
+          }
+          pending |= 1u << s;
+          pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
+        }
+      }
+      // Drain: wait until every load this thread issued has landed.
+      for (int s = 0; s < S; ++s)
+        if (pending & (1u << s))
+          wait_bar(smem_u32(&full[s]), (pend_parity >> s) & 1, abort_flag, p.err, false);
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------------- MMA issuer
+    const int a_mn = p.mode == KG ? 1 : 0;
+    const int b_mn = p.mode == KG ? 1 : p.b_major;
+    const uint32_t idesc = idesc_bf16(BM, p.bn, a_mn, b_mn);
+    const uint32_t a_lbo = a_mn ? BOX_BYTES : 16, b_lbo = b_mn ? BOX_BYTES : 16;
+    const uint32_t a_step = a_mn ? 2048 : 32, b_step = b_mn ? 2048 : 32;
+    int it = 0, tcount = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
+      const Tile tl = decode(p, t);
+      const int buf = tcount & 1;
+      const uint32_t aph = (tcount >> 1) & 1;
+      ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&acc_empty[buf]), aph ^ 1, abort_flag, p.err));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tmem_d = tmem_base + buf * p.bn;
+      if (tl.nk == 0) {
+        if (lane == 0) mbar_arrive(smem_u32(&acc_full[buf]));
+        __syncwarp();
+        continue;
+      }
+      for (int kb = 0; kb < tl.nk; ++kb, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1;
+        ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&full[s]), ph, abort_flag, p.err));
+        if (!ok) break;
+        const uint32_t sa = smem_u32(smem + s * stage_bytes);
+        const uint32_t sb = sa + A_BYTES;
+        if (p.mode == KG && kb == tl.nk - 1 && tl.kvalid < BK) {
+          // Zero K rows past the segment end in every box of this stage (A: 2 boxes, B: bn/64).
+          const int nbox = 2 + p.bn / 64;
+          const int per_box = (BK - tl.kvalid) * 8;   // 16-byte chunks per box
+          for (int i = lane; i < nbox * per_box; i += 32) {
+            const int b = i / per_box, c = i - b * per_box;
+            const uint32_t addr = sa + b * BOX_BYTES + tl.kvalid * 128 + c * 16;
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0) : "memory");
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+        }
+        tc_fence_after();
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = sdesc(sa + kk * a_step, a_lbo, 1024);
+            const uint64_t bd = sdesc(sb + kk * b_step, b_lbo, 1024);
+            tc_mma(tmem_d, ad, bd, idesc, (kb | kk) != 0);
+          }
+          tc_commit(smem_u32(&empty[s]));
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) tc_commit(smem_u32(&acc_full[buf]));
+      __syncwarp();
+    }
+    // Drain: every MMA this thread issued has completed before TMEM is freed.
+    if (lane == 0) {
+      tc_commit(smem_u32(drain));
+      wait_bar(smem_u32(drain), 0, abort_flag, p.err, false);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;           // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;      // accumulator row held by this thread
+    int tcount = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
+      const Tile tl = decode(p, t);
+      const int buf = tcount & 1;
+      const uint32_t aph = (tcount >> 1) & 1;
+      if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&acc_full[buf]), aph, abort_flag, p.err))) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * p.bn;
+      epilogue_tile<EPI>(p, tl, tacc, r);
+      tc_fence_before();
+      mbar_arrive(smem_u32(&acc_empty[buf]));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+// ------------------------------------------------------------------------ host
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+static std::once_flag g_encode_once;
+
+static int get_encode() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return fail(PFMOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  return PFMOE_OK;
+}
+
+// 3-D BF16 tensor map over a row-major tensor [d2][d1][d0] with a box of b0 x b1 x 1, 128-byte swizzle.
+static int make_tmap(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+                     uint32_t b1, const char* what) {
+  PFMOE_TRY(get_encode());
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(PFMOE_ERR_CUDA, std::string("cuTensorMapEncodeTiled failed for ") + what + " (CUresult " +
+                                    std::to_string(static_cast<int>(r)) + ")");
+  return PFMOE_OK;
+}
+
+static int round_bn(int n) {
+  int bn = ((n + 63) / 64) * 64;
+  return bn > 256 ? 256 : bn;
+}
+
+static int pick_stages(int bn) {
+  const int stage = A_BYTES + bn * BK * 2;
+  int s = (200 * 1024) / stage;
+  return s > MAX_STAGES ? MAX_STAGES : s;
+}
+
+static size_t smem_bytes(int bn, int stages) {
+  return 1024 + static_cast<size_t>(stages) * (A_BYTES + bn * BK * 2) + 256;
+}
+
+template <int EPI>
+static int launch(Params& p, long long tile_upper_bound, const char* name, cudaStream_t stream) {
+  p.stages = pick_stages(p.bn);
+  const size_t smem = smem_bytes(p.bn, p.stages);
+  static bool attr_done = false;  // per template instance
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(227 * 1024)) != cudaSuccess)
+      return fail(PFMOE_ERR_CUDA, std::string("cudaFuncSetAttribute failed: ") +
+                                      cudaGetErrorString(cudaGetLastError()));
+    attr_done = true;
+  }
+  if (tile_upper_bound <= 0) return PFMOE_OK;
+  long long grid = num_sms();
+  if (tile_upper_bound < grid) grid = tile_upper_bound;
+  PFMOE_LAUNCH(name, stream,
+               grouped_gemm_kernel<EPI><<<static_cast<int>(grid), THREADS, smem, stream>>>(p));
+  return PFMOE_OK;
+}
+
+static Params base_params(int32_t* err) {
+  Params p;
+  memset(&p, 0, sizeof(p));
+  p.err = err;
+  return p;
+}
+
+}  // namespace tc
+
+using namespace tc;
+
+// Row-tile upper bound for expert-segmented rows: sum_e ceil(n_e / 128) <= N / 128 + E.
+static long long rg_tiles_ub(int N, int E, int Nout, int nstep) {
+  return (static_cast<long long>(N) / BM + E + 1) * ((Nout + nstep - 1) / nstep);
+}
+
+int tc_ffn_gemm1(const void* x_pft, const int* seg, const int* tiles, int N, int E, int d, int h,
+                 const void* w1, const void* w3, void* h1, void* h3, void* a, int32_t* err, cudaStream_t s) {
+  Params p = base_params(err);
+  p.mode = RG;
+  p.b_major = 1;
+  p.bn = h > 64 ? 256 : 128;
+  p.nsplit = 1;
+  p.Nout = h;
+  p.k0_blocks = (d + BK - 1) / BK;
+  p.seg = seg; p.tiles = tiles; p.G = E;
+  p.D0 = h1; p.D1 = h3; p.D2 = a; p.ldd = h;
+  PFMOE_TRY(make_tmap(&p.tmA[0], x_pft, d, N, 1, BK, BM, "x_pft"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], w1, h, d, E, 64, 64, "w1"));
+  PFMOE_TRY(make_tmap(&p.tmB[1], w3, h, d, E, 64, 64, "w3"));
+  return launch<EPI_SWIGLU_FWD>(p, rg_tiles_ub(N, E, h, p.bn / 2), "ffn_gemm1_swiglu", s);
+}
+
+int tc_ffn_gemm2(const void* a, const int* seg, const int* tiles, int N, int E, int d, int h, const void* w2,
+                 void* out, int32_t* err, cudaStream_t s) {
+  Params p = base_params(err);
+  p.mode = RG;
+  p.b_major = 1;
+  p.bn = round_bn(d);
+  p.Nout = d;
+  p.k0_blocks = (h + BK - 1) / BK;
+  p.seg = seg; p.tiles = tiles; p.G = E;
+  p.D0 = out; p.ldd = d;
+  PFMOE_TRY(make_tmap(&p.tmA[0], a, h, N, 1, BK, BM, "a"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], w2, d, h, E, 64, 64, "w2"));
+  return launch<EPI_STORE_BF16>(p, rg_tiles_ub(N, E, d, p.bn), "ffn_gemm2", s);
+}
+
+int tc_ffn_dgrad_act(const void* dO, const int* seg, const int* tiles, int N, int E, int d, int h, const void* w2,
+                     const void* h1, const void* h3, void* dh1, void* dh3, int32_t* err, cudaStream_t s) {
+  Params p = base_params(err);
+  p.mode = RG;
+  p.b_major = 0;              // W2_e [h, d]: rows = output columns (h), K = d contiguous
+  p.bn = round_bn(h);
+  p.Nout = h;
+  p.k0_blocks = (d + BK - 1) / BK;
+  p.seg = seg; p.tiles = tiles; p.G = E;
+  p.X0 = h1; p.X1 = h3; p.D0 = dh1; p.D1 = dh3; p.ldd = h;
+  PFMOE_TRY(make_tmap(&p.tmA[0], dO, d, N, 1, BK, BM, "dO"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], w2, d, h, E, BK, p.bn, "w2^T"));
+  return launch<EPI_SWIGLU_BWD>(p, rg_tiles_ub(N, E, h, p.bn), "ffn_dgrad_act_swiglu_bwd", s);
+}
+
+int tc_ffn_dgrad_x(const void* dh1, const void* dh3, const int* seg, const int* tiles, int N, int E, int d, int h,
+                   const void* w1, const void* w3, void* dx_pft, int32_t* err, cudaStream_t s) {
+  Params p = base_params(err);
+  p.mode = RG;
+  p.b_major = 0;              // W1_e [d, h]: rows = output columns (d), K = h contiguous
+  p.bn = round_bn(d);
+  p.Nout = d;
+  p.k0_blocks = (h + BK - 1) / BK;
+  p.k1_blocks = (h + BK - 1) / BK;
+  p.seg = seg; p.tiles = tiles; p.G = E;
+  p.D0 = dx_pft; p.ldd = d;
+  PFMOE_TRY(make_tmap(&p.tmA[0], dh1, h, N, 1, BK, BM, "dh1"));
+  PFMOE_TRY(make_tmap(&p.tmA[1], dh3, h, N, 1, BK, BM, "dh3"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], w1, h, d, E, BK, p.bn, "w1^T"));
+  PFMOE_TRY(make_tmap(&p.tmB[1], w3, h, d, E, BK, p.bn, "w3^T"));
+  return launch<EPI_STORE_BF16>(p, rg_tiles_ub(N, E, d, p.bn), "ffn_dgrad_x", s);
+}
+
+int tc_ffn_wgrad13(const void* x_pft, const void* dh1, const void* dh3, const int* seg, int N, int E, int d, int h,
+                   void* dw1, void* dw3, int32_t* err, cudaStream_t s) {
+  Params p = base_params(err);
+  p.mode = KG;
+  p.b_major = 1;
+  p.bn = h > 64 ? 256 : 128;
+  p.nsplit = 1;
+  p.M = d;
+  p.Nout = h;
+  p.seg = seg; p.G = E;
+  p.D0 = dw1; p.D1 = dw3; p.ldd = h; p.d_gstride = static_cast<long long>(d) * h;
+  PFMOE_TRY(make_tmap(&p.tmA[0], x_pft, d, N, 1, 64, 64, "x_pft^T"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], dh1, h, N, 1, 64, 64, "dh1"));
+  PFMOE_TRY(make_tmap(&p.tmB[1], dh3, h, N, 1, 64, 64, "dh3"));
+  const long long ub = static_cast<long long>(E) * ((d + BM - 1) / BM) * ((h + p.bn / 2 - 1) / (p.bn / 2));
+  return launch<EPI_SPLIT_BF16>(p, ub, "ffn_wgrad_w1w3", s);
+}
+
+int tc_ffn_wgrad2(const void* a, const void* dO, const int* seg, int N, int E, int d, int h, void* dw2,
+                  int32_t* err, cudaStream_t s) {
+  Params p = base_params(err);
+  p.mode = KG;
+  p.b_major = 1;
+  p.bn = round_bn(d);
+  p.M = h;
+  p.Nout = d;
+  p.seg = seg; p.G = E;
+  p.D0 = dw2; p.ldd = d; p.d_gstride = static_cast<long long>(h) * d;
+  PFMOE_TRY(make_tmap(&p.tmA[0], a, h, N, 1, 64, 64, "a^T"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], dO, d, N, 1, 64, 64, "dO"));
+  const long long ub = static_cast<long long>(E) * ((h + BM - 1) / BM) * ((d + p.bn - 1) / p.bn);
+  return launch<EPI_STORE_BF16>(p, ub, "ffn_wgrad_w2", s);
+}
+
+int tc_gate_logits(const void* x, const void* wg, const float* bias, int T, int d, int E, float* logits,
+                   int32_t* err, cudaStream_t s) {
+  Params p = base_params(err);
+  p.mode = RG;
+  p.b_major = 1;              // Wg [d, E]: K rows, E contiguous
+  p.bn = round_bn(E);
+  p.Nout = E;
+  p.k0_blocks = (d + BK - 1) / BK;
+  p.G = 1;
+  p.dense_len = T;
+  p.D0 = logits; p.bias = bias; p.ldd = E;
+  PFMOE_TRY(make_tmap(&p.tmA[0], x, d, T, 1, BK, BM, "x"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], wg, E, d, 1, 64, 64, "wg"));
+  const long long ub = static_cast<long long>((T + BM - 1) / BM) * ((E + p.bn - 1) / p.bn);
+  return launch<EPI_STORE_F32>(p, ub, "gate_logits", s);
+}
+
+int tc_gate_wgrad(const void* x, const void* dz_bf16, int T, int d, int E, float* dwg, int32_t* err,
+                  cudaStream_t s) {
+  Params p = base_params(err);
+  p.mode = KG;
+  p.b_major = 1;
+  p.bn = round_bn(E);
+  p.M = d;
+  p.Nout = E;
+  p.G = 1;
+  p.dense_len = T;
+  p.D0 = dwg; p.ldd = E; p.d_gstride = 0;
+  PFMOE_TRY(make_tmap(&p.tmA[0], x, d, T, 1, 64, 64, "x^T"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], dz_bf16, E, T, 1, 64, 64, "dz"));
+  const long long ub = static_cast<long long>((d + BM - 1) / BM) * ((E + p.bn - 1) / p.bn);
+  return launch<EPI_STORE_F32>(p, ub, "gate_wgrad", s);
+}
+
+}  // namespace pfmoe

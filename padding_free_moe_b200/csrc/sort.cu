@@ -1,0 +1,401 @@
+// Stable counting sort by small integer keys, and the two index structures
+// built on it: the padding-free token buffer (X-MoE article §2.1.1 "PFT数据结构创新")
+// and the redundancy-bypassing-dispatch pilot plan (§2.2.1 "分层冗余消除算法").
+//
+// Sort = three launches:
+//   1. chunk histograms: one warp per CHUNK consecutive keys, counts[c][key];
+//   2. one-CTA scan in (key, chunk) order -> per-key totals, key offsets and
+//      every chunk's base row for every key (plus the grouped-GEMM tile prefix);
+//   3. scatter: one warp per chunk walks its keys in order, 32 at a time;
+//      lanes holding the same key find each other with __match_any_sync and
+//      take consecutive rows in lane order -> the sort is stable.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace pfmoe {
+namespace {
+
+constexpr int CHUNK = 2048;
+constexpr int SCAN_THREADS = 1024;
+
+inline int warps_per_block(int K) {
+  int w = 12288 / (K > 0 ? K : 1);
+  return w < 1 ? 1 : (w > 8 ? 8 : w);
+}
+
+__device__ __forceinline__ long long dev_count(long long n, const int32_t* n_dev) {
+  return n_dev ? static_cast<long long>(*n_dev) : n;
+}
+
+__global__ void chunk_hist_kernel(const int32_t* __restrict__ keys, long long n, const int32_t* n_dev, int K,
+                                  int nchunks, int32_t* __restrict__ counts, int32_t* err) {
+  extern __shared__ int32_t sh[];
+  const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x * (blockDim.x >> 5) + wib;
+  int32_t* h = sh + wib * K;
+  for (int i = lane; i < K; i += 32) h[i] = 0;
+  __syncwarp();
+  if (chunk >= nchunks) return;
+  const long long nn = dev_count(n, n_dev);
+  const long long b = static_cast<long long>(chunk) * CHUNK;
+  const long long e = min(b + CHUNK, nn);
+  bool bad = false;
+  for (long long i = b + lane; i < e; i += 32) {
+    const int key = keys[i];
+    if (static_cast<unsigned>(key) < static_cast<unsigned>(K)) atomicAdd(&h[key], 1);
+    else bad = true;
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) dev_error(err, PFMOE_DEV_BAD_EXPERT_ID);
+  __syncwarp();
+  for (int i = lane; i < K; i += 32) counts[static_cast<long long>(chunk) * K + i] = h[i];
+}
+
+// Block-wide exclusive scan of one int per thread; returns the exclusive prefix, *total = block sum.
+__device__ int block_excl_scan(int v, int* tmp /*[32]*/, int* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) tmp[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    int s = lane < nw ? tmp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    tmp[lane] = s;  // inclusive warp sums
+  }
+  __syncthreads();
+  const int warp_off = wid > 0 ? tmp[wid - 1] : 0;
+  *total = tmp[nw - 1];
+  __syncthreads();
+  return warp_off + x - v;
+}
+
+// counts [C][K] -> totals [K], offsets [K+1], base [C][K]; optional tiles [K+1] = prefix of ceil(total/tile_rows).
+__global__ void __launch_bounds__(SCAN_THREADS) chunk_scan_kernel(const int32_t* __restrict__ counts, int C, int K,
+                                                                  int32_t* totals, int32_t* offsets,
+                                                                  int32_t* __restrict__ base, int32_t* tiles,
+                                                                  int tile_rows) {
+  __shared__ int tmp[32];
+  int carry = 0, tcarry = 0;
+  for (int k0 = 0; k0 < K; k0 += SCAN_THREADS) {
+    const int key = k0 + threadIdx.x;
+    int tot = 0;
+    if (key < K)
+      for (int c = 0; c < C; ++c) tot += counts[static_cast<long long>(c) * K + key];
+    int blk;
+    const int excl = block_excl_scan(tot, tmp, &blk) + carry;
+    int tblk;
+    const int nt = tile_rows > 0 ? (tot + tile_rows - 1) / tile_rows : 0;
+    const int texcl = block_excl_scan(nt, tmp, &tblk) + tcarry;
+    if (key < K) {
+      if (totals) totals[key] = tot;
+      offsets[key] = excl;
+      if (tiles) tiles[key] = texcl;
+      int run = excl;
+      for (int c = 0; c < C; ++c) {
+        const long long idx = static_cast<long long>(c) * K + key;
+        const int cnt = counts[idx];
+        base[idx] = run;
+        run += cnt;
+      }
+    }
+    carry += blk;
+    tcarry += tblk;
+  }
+  if (threadIdx.x == 0) {
+    offsets[K] = carry;
+    if (tiles) tiles[K] = tcarry;
+  }
+}
+
+// Stable scatter; Sink(i, p, key) records that element i lands at sorted position p.
+template <class Sink>
+__global__ void chunk_scatter_kernel(const int32_t* __restrict__ keys, long long n, const int32_t* n_dev, int K,
+                                     int nchunks, const int32_t* __restrict__ base, Sink sink) {
+  extern __shared__ int32_t sh[];
+  const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x * (blockDim.x >> 5) + wib;
+  if (chunk >= nchunks) return;
+  int32_t* ctr = sh + wib * K;
+  for (int i = lane; i < K; i += 32) ctr[i] = base[static_cast<long long>(chunk) * K + i];
+  __syncwarp();
+  const long long nn = dev_count(n, n_dev);
+  const long long b = static_cast<long long>(chunk) * CHUNK;
+  const long long e = min(b + CHUNK, nn);
+  for (long long i0 = b; i0 < e; i0 += 32) {
+    const long long i = i0 + lane;
+    const int key = i < e ? keys[i] : -1;
+    const bool ok = i < e && static_cast<unsigned>(key) < static_cast<unsigned>(K);
+    const unsigned peers = __match_any_sync(0xffffffffu, ok ? key : K + lane);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int cnt = ok ? ctr[key] : 0;
+    __syncwarp();
+    if (ok && rank == 0) ctr[key] = cnt + __popc(peers);
+    __syncwarp();
+    if (ok) sink(i, cnt + rank, key);
+  }
+}
+
+struct PftSink {
+  const float* w;
+  int k;
+  int32_t* pos;
+  int32_t* token_ids;
+  int32_t* expert_ids;
+  float* cw;
+  __device__ void operator()(long long i, int p, int key) const {
+    pos[i] = p;
+    token_ids[p] = static_cast<int32_t>(i / k);
+    expert_ids[p] = key;
+    cw[p] = w[i];
+  }
+};
+
+// Single-CTA exclusive scan of n (device or host count) ints: out[0..n], out[n] = sum.
+__global__ void __launch_bounds__(SCAN_THREADS) excl_scan_kernel(const int32_t* __restrict__ in, long long n,
+                                                                 const int32_t* n_dev, int32_t* __restrict__ out) {
+  __shared__ int tmp[32];
+  const long long nn = dev_count(n, n_dev);
+  int carry = 0;
+  for (long long i0 = 0; i0 < nn; i0 += SCAN_THREADS) {
+    const long long i = i0 + threadIdx.x;
+    const int v = i < nn ? in[i] : 0;
+    int blk;
+    const int ex = block_excl_scan(v, tmp, &blk);
+    if (i < nn) out[i] = carry + ex;
+    carry += blk;
+  }
+  if (threadIdx.x == 0) out[nn] = carry;
+}
+
+// ------------------------------------------------------------------------- RBD
+// Per token (one warp; lane j < k holds expert e_j): rank experts by (e, lane);
+// a lane "leads" its node (device) when no earlier-ranked lane shares it.
+struct TokView {
+  int e, node, dev;
+  bool valid;
+  bool node_lead, dev_lead;
+  int node_rank;   // index of this lane's node among the token's distinct nodes (ascending)
+  int within;      // rank of e among the token's experts on the same node
+  int same_node;   // experts of this token on this lane's node
+};
+
+__device__ __forceinline__ TokView token_view(const int32_t* ids, int t, int k, int E, int epd, int epn,
+                                              int32_t* err) {
+  const int lane = threadIdx.x & 31;
+  TokView v;
+  v.valid = lane < k;
+  int e = v.valid ? ids[static_cast<long long>(t) * k + lane] : 0;
+  if (v.valid && static_cast<unsigned>(e) >= static_cast<unsigned>(E)) {
+    dev_error(err, PFMOE_DEV_BAD_EXPERT_ID);
+    e = 0;
+  }
+  v.e = e;
+  v.node = e / epn;
+  v.dev = e / epd;
+  int node_before = 0, dev_before = 0, within = 0, same = 0;
+  for (int j = 0; j < k; ++j) {
+    const int oe = __shfl_sync(0xffffffffu, e, j);
+    const bool earlier = oe < e || (oe == e && j < lane);
+    const int onode = oe / epn, odev = oe / epd;
+    if (onode == v.node) {
+      ++same;
+      if (earlier) { ++node_before; ++within; }
+    }
+    if (odev == v.dev && earlier) ++dev_before;
+  }
+  v.node_lead = v.valid && node_before == 0;
+  v.dev_lead = v.valid && dev_before == 0;
+  v.within = within;
+  v.same_node = same;
+  const unsigned leads = __ballot_sync(0xffffffffu, v.node_lead);
+  int rank = 0;
+  for (int j = 0; j < k; ++j) {
+    const int onode = __shfl_sync(0xffffffffu, v.node, j);
+    if (((leads >> j) & 1u) && onode < v.node) ++rank;
+  }
+  v.node_rank = rank;
+  return v;
+}
+
+__global__ void rbd_count_kernel(const int32_t* ids, int T, int k, int E, int epd, int epn, int32_t* ucount,
+                                 int32_t* dcount, int32_t* err) {
+  const int lane = threadIdx.x & 31;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nw) {
+    const TokView v = token_view(ids, t, k, E, epd, epn, err);
+    const int u = __popc(__ballot_sync(0xffffffffu, v.node_lead));
+    const int dd = __popc(__ballot_sync(0xffffffffu, v.dev_lead));
+    if (lane == 0) { ucount[t] = u; dcount[t] = dd; }
+  }
+}
+
+// Scan of per-token pilot counts; counts[0] = P, counts[1] = sum of distinct (token, device) pairs.
+__global__ void __launch_bounds__(SCAN_THREADS) rbd_scan_kernel(const int32_t* ucount, const int32_t* dcount, int T,
+                                                                int32_t* pilot_base, int32_t* counts) {
+  __shared__ int tmp[32];
+  int carry = 0, dcarry = 0;
+  for (int i0 = 0; i0 < T; i0 += SCAN_THREADS) {
+    const int i = i0 + threadIdx.x;
+    const int u = i < T ? ucount[i] : 0;
+    const int dd = i < T ? dcount[i] : 0;
+    int blk, dblk;
+    const int ex = block_excl_scan(u, tmp, &blk);
+    block_excl_scan(dd, tmp, &dblk);
+    if (i < T) pilot_base[i] = carry + ex;
+    carry += blk;
+    dcarry += dblk;
+  }
+  if (threadIdx.x == 0) { counts[0] = carry; counts[1] = dcarry; }
+}
+
+// Token-major pilot list: key = node, token, replica count.
+__global__ void rbd_emit_kernel(const int32_t* ids, int T, int k, int E, int epd, int epn, const int32_t* pilot_base,
+                                int32_t* pkey, int32_t* ptoken, int32_t* prc, int32_t* err) {
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nw) {
+    const TokView v = token_view(ids, t, k, E, epd, epn, err);
+    if (v.node_lead) {
+      const int i = pilot_base[t] + v.node_rank;
+      pkey[i] = v.node;
+      ptoken[i] = t;
+      prc[i] = v.same_node;
+    }
+  }
+}
+
+struct RbdSink {
+  const int32_t* ptoken;
+  const int32_t* prc;
+  int32_t* pilot_token;
+  int32_t* pilot_node;
+  int32_t* rc_sorted;
+  int32_t* psorted;
+  __device__ void operator()(long long i, int p, int key) const {
+    pilot_token[p] = ptoken[i];
+    pilot_node[p] = key;
+    rc_sorted[p] = prc[i];
+    psorted[i] = p;
+  }
+};
+
+__global__ void rbd_final_kernel(const int32_t* ids, int T, int k, int E, int epd, int epn,
+                                 const int32_t* pilot_base, const int32_t* psorted, const int32_t* replica_offsets,
+                                 int32_t* assign_pilot, int32_t* replica_expert, int32_t* pilot_device,
+                                 int32_t* err) {
+  const int lane = threadIdx.x & 31;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nw) {
+    const TokView v = token_view(ids, t, k, E, epd, epn, err);
+    if (v.valid) {
+      const int q = psorted[pilot_base[t] + v.node_rank];
+      assign_pilot[static_cast<long long>(t) * k + lane] = q;
+      replica_expert[replica_offsets[q] + v.within] = v.e;
+      if (v.within == 0) pilot_device[q] = v.dev;
+    }
+  }
+}
+
+int rows_grid(long long rows, int warps_per_blk = 8) {
+  long long b = (rows + warps_per_blk - 1) / warps_per_blk;
+  const long long cap = static_cast<long long>(num_sms()) * 16;
+  if (b > cap) b = cap;
+  return static_cast<int>(b < 1 ? 1 : b);
+}
+
+struct CsortWs {
+  int32_t* counts;
+  int32_t* base;
+};
+
+}  // namespace
+
+size_t csort_ws_bytes(long long n_max, int K) {
+  const long long C = (n_max + CHUNK - 1) / CHUNK;
+  return static_cast<size_t>(2 * (C > 0 ? C : 1) * static_cast<long long>(K)) * sizeof(int32_t);
+}
+
+int pft_build_impl(const int32_t* ids, const float* w, int T, int E, int k, int32_t* tpe, int32_t* offsets,
+                   int32_t* token_ids, int32_t* expert_ids, float* cw, int32_t* pos, int32_t* tile_offsets,
+                   void* ws, int32_t* err, cudaStream_t s) {
+  const long long N = static_cast<long long>(T) * k;
+  const int C = static_cast<int>((N + CHUNK - 1) / CHUNK);
+  int32_t* counts = static_cast<int32_t*>(ws);
+  int32_t* base = counts + static_cast<long long>(C) * E;
+  const int wpb = warps_per_block(E);
+  const int blocks = (C + wpb - 1) / wpb;
+  const size_t sm = static_cast<size_t>(wpb) * E * sizeof(int32_t);
+  if (C > 0)
+    PFMOE_LAUNCH("pft_hist", s, chunk_hist_kernel<<<blocks, wpb * 32, sm, s>>>(ids, N, nullptr, E, C, counts, err));
+  PFMOE_LAUNCH("pft_scan", s,
+               chunk_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(counts, C, E, tpe, offsets, base, tile_offsets, 128));
+  PftSink sink{w, k, pos, token_ids, expert_ids, cw};
+  if (C > 0)
+    PFMOE_LAUNCH("pft_scatter", s,
+                 chunk_scatter_kernel<PftSink><<<blocks, wpb * 32, sm, s>>>(ids, N, nullptr, E, C, base, sink));
+  return PFMOE_OK;
+}
+
+size_t rbd_ws_bytes(int T, int k, int n_nodes) {
+  const long long pmax = static_cast<long long>(T) * (k < n_nodes ? k : n_nodes);
+  const size_t ints = 3 * static_cast<size_t>(T) + 5 * static_cast<size_t>(pmax) + 64;
+  return ints * sizeof(int32_t) + csort_ws_bytes(pmax, n_nodes) + 256;
+}
+
+int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int32_t* pilots_per_node,
+                  int32_t* node_offsets, int32_t* pilot_token, int32_t* pilot_node, int32_t* pilot_device,
+                  int32_t* replica_offsets, int32_t* replica_expert, int32_t* assign_pilot, int32_t* counts,
+                  void* ws, int32_t* err, cudaStream_t s) {
+  const int epn = epd * dpn;
+  const int n_nodes = E / epn;
+  const long long pmax = static_cast<long long>(T) * (k < n_nodes ? k : n_nodes);
+  int32_t* p = static_cast<int32_t*>(ws);
+  int32_t* ucount = p; p += T;
+  int32_t* dcount = p; p += T;
+  int32_t* pbase = p; p += T;
+  int32_t* pkey = p; p += pmax;
+  int32_t* ptoken = p; p += pmax;
+  int32_t* prc = p; p += pmax;
+  int32_t* psorted = p; p += pmax;
+  int32_t* rc_sorted = p; p += pmax;
+  p += 64 - ((p - static_cast<int32_t*>(ws)) & 63);   // keep 256-byte alignment
+  const int C = static_cast<int>((pmax + CHUNK - 1) / CHUNK);
+  int32_t* ccounts = p; p += static_cast<long long>(C > 0 ? C : 1) * n_nodes;
+  int32_t* cbase = p;
+
+  const int g = rows_grid(T);
+  PFMOE_LAUNCH("rbd_count", s, rbd_count_kernel<<<g, 256, 0, s>>>(ids, T, k, E, epd, epn, ucount, dcount, err));
+  PFMOE_LAUNCH("rbd_scan_tokens", s, rbd_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(ucount, dcount, T, pbase, counts));
+  PFMOE_LAUNCH("rbd_emit", s, rbd_emit_kernel<<<g, 256, 0, s>>>(ids, T, k, E, epd, epn, pbase, pkey, ptoken, prc, err));
+  const int wpb = warps_per_block(n_nodes);
+  const int blocks = (C + wpb - 1) / wpb;
+  const size_t sm = static_cast<size_t>(wpb) * n_nodes * sizeof(int32_t);
+  if (C > 0) {
+    PFMOE_LAUNCH("rbd_hist", s,
+                 chunk_hist_kernel<<<blocks, wpb * 32, sm, s>>>(pkey, pmax, counts, n_nodes, C, ccounts, err));
+  }
+  PFMOE_LAUNCH("rbd_scan_nodes", s,
+               chunk_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(ccounts, C, n_nodes, pilots_per_node, node_offsets,
+                                                            cbase, nullptr, 0));
+  if (C > 0) {
+    RbdSink sink{ptoken, prc, pilot_token, pilot_node, rc_sorted, psorted};
+    PFMOE_LAUNCH("rbd_scatter", s,
+                 chunk_scatter_kernel<RbdSink><<<blocks, wpb * 32, sm, s>>>(pkey, pmax, counts, n_nodes, C, cbase,
+                                                                             sink));
+  }
+  PFMOE_LAUNCH("rbd_scan_replicas", s,
+               excl_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(rc_sorted, pmax, counts, replica_offsets));
+  PFMOE_LAUNCH("rbd_final", s,
+               rbd_final_kernel<<<g, 256, 0, s>>>(ids, T, k, E, epd, epn, pbase, psorted, replica_offsets,
+                                                   assign_pilot, replica_expert, pilot_device, err));
+  return PFMOE_OK;
+}
+
+}  // namespace pfmoe

@@ -1,0 +1,102 @@
+"""Edge cases of the CUDA path: no tokens, out-of-range indices reported through
+the device error word (nothing traps), and argument errors from a live context."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from padding_free_moe_b200 import _lib as L
+from workloads import get_config, make_inputs
+
+from tests.parity import i64, make_layer, run_step
+
+
+@pytest.mark.gpu
+def test_zero_tokens():
+    cfg = get_config("small_bf16").with_(T=0)
+    layer = make_layer(cfg)
+    inp = make_inputs(cfg, seed=0, device="cuda")
+    for t in (layer.expert_offsets, layer.tile_offsets, layer.tokens_per_expert, layer.node_offsets,
+              layer.pilots_per_node, layer.rbd_counts, layer.replica_offsets):
+        t.fill_(-7)
+    layer.dw1.fill_(3.0); layer.dw3.fill_(3.0); layer.dw2.fill_(3.0); layer.dwg.fill_(3.0)
+    assert run_step(layer, inp) == 0
+    for t in (layer.expert_offsets, layer.tile_offsets, layer.tokens_per_expert, layer.node_offsets,
+              layer.pilots_per_node, layer.rbd_counts):
+        assert not t.any()
+    assert int(layer.replica_offsets[0]) == 0
+    for t in (layer.dw1, layer.dw3, layer.dw2, layer.dwg):
+        assert not t.any()
+
+
+@pytest.mark.gpu
+def test_bad_expert_ids_set_error_bit():
+    T, E, k = 50, 16, 2
+    ids = torch.randint(0, E, (T, k), device="cuda", dtype=torch.int32)
+    ids[7, 1] = E          # out of range
+    ids[9, 0] = -3
+    w = torch.full((T, k), 0.5, device="cuda")
+    out = {n: torch.zeros(sz, device="cuda", dtype=torch.int32) for n, sz in
+           (("tpe", E), ("off", E + 1), ("tok", T * k), ("eid", T * k), ("pos", T * k), ("tiles", E + 1))}
+    cw = torch.zeros(T * k, device="cuda")
+    ws_b = L.pft_build_workspace_size(T, E, k)
+    ws = torch.empty(ws_b, device="cuda", dtype=torch.uint8)
+    err = torch.zeros(1, device="cuda", dtype=torch.int32)
+    L.pft_build(ids, w, T, E, k, out["tpe"], out["off"], out["tok"], out["eid"], cw, out["pos"], out["tiles"], ws,
+                ws_b, err)
+    torch.cuda.synchronize()
+    assert int(err) & L.DEV_BAD_EXPERT_ID
+    # the valid assignments are all counted
+    assert int(out["tpe"].sum()) == T * k - 2
+
+
+@pytest.mark.gpu
+def test_bad_pos_sets_error_bit():
+    T, k, d = 10, 2, 64
+    o = torch.randn(T * k, d, device="cuda").to(torch.bfloat16)
+    pos = torch.arange(T * k, device="cuda", dtype=torch.int32).view(T, k).contiguous()
+    pos[3, 1] = T * k + 5
+    w = torch.full((T, k), 0.5, device="cuda")
+    y = torch.zeros(T, d, device="cuda", dtype=torch.bfloat16)
+    err = torch.zeros(1, device="cuda", dtype=torch.int32)
+    L.moe_combine(o, pos, w, T, k, d, L.PFMOE_BF16, y, err)
+    torch.cuda.synchronize()
+    assert int(err) & L.DEV_BAD_POS
+    assert not y[3].any()          # the bad token was skipped
+
+
+@pytest.mark.gpu
+def test_argument_error_message():
+    x = torch.zeros(4, 64, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(L.PFMoEError, match="k <= E"):
+        L.moe_route(x, x, None, 4, 64, 8, 9, L.PFMOE_BF16, x, x, x)
+
+
+@pytest.mark.gpu
+def test_rbd_stress_shape_matches_oracle():
+    # A large index-only shape (no expert maths): 2^17 tokens, 256 experts, k = 8, 8 nodes.
+    from workloads.generate import make_topk_ids
+    T, E, k, epd, dpn = 1 << 17, 256, 8, 8, 4
+    ids = make_topk_ids(T, E, k, seed=5, device="cuda")
+    n_nodes = E // (epd * dpn)
+    pmax = T * min(k, n_nodes)
+    i32 = dict(device="cuda", dtype=torch.int32)
+    o = dict(ppn=torch.empty(n_nodes, **i32), noff=torch.empty(n_nodes + 1, **i32), ptok=torch.empty(pmax, **i32),
+             pnode=torch.empty(pmax, **i32), pdev=torch.empty(pmax, **i32), roff=torch.empty(pmax + 1, **i32),
+             rexp=torch.empty(T * k, **i32), ap=torch.empty(T, k, **i32), cnt=torch.empty(2, **i32))
+    ws_b = L.rbd_plan_workspace_size(T, k, E, epd, dpn)
+    ws = torch.empty(ws_b, device="cuda", dtype=torch.uint8)
+    err = torch.zeros(1, **i32)
+    L.rbd_plan(ids, T, k, E, epd, dpn, o["ppn"], o["noff"], o["ptok"], o["pnode"], o["pdev"], o["roff"], o["rexp"],
+               o["ap"], o["cnt"], ws, ws_b, err)
+    torch.cuda.synchronize()
+    assert int(err) == 0
+    r = O.rbd_plan(i64(ids), E, epd, dpn)
+    P = r["num_pilots"]
+    assert int(o["cnt"][0]) == P
+    assert np.array_equal(i64(o["ptok"][:P]), r["pilot_token"])
+    assert np.array_equal(i64(o["pnode"][:P]), r["pilot_node"])
+    assert np.array_equal(i64(o["roff"][:P + 1]), r["replica_offsets"])
+    assert np.array_equal(i64(o["rexp"]), r["replica_expert"])
+    assert np.array_equal(i64(o["ap"]), r["assign_pilot"])
+    assert np.array_equal(i64(o["pdev"][:P]), r["pilot_device"])

@@ -67,13 +67,13 @@ CONFIGS = {
 # BF16 tensor-core path with several M tiles per expert, ragged segment tails,
 # h and d that are not multiples of the N tile, empty experts and k = E.
 SMALL = {
-    "small_bf16": LayerConfig("small_bf16", T=300, d=256, E=12, h=192, k=3, dtype="bf16",
+    "small_bf16": LayerConfig("small_bf16", T=300, d=256, E=16, h=192, k=3, dtype="bf16",
                               rbd_epd=2, rbd_dpn=2),
-    "small_ragged_bf16": LayerConfig("small_ragged_bf16", T=517, d=200, E=7, h=136, k=2, dtype="bf16",
-                                     rbd_epd=7, rbd_dpn=1),
+    "small_ragged_bf16": LayerConfig("small_ragged_bf16", T=517, d=200, E=24, h=136, k=5, dtype="bf16",
+                                     rbd_epd=3, rbd_dpn=2),
     "small_skew_bf16": LayerConfig("small_skew_bf16", T=700, d=320, E=16, h=256, k=4, dtype="bf16",
                                    zipf_c=1.5, rbd_epd=2, rbd_dpn=4),
-    "small_kE_bf16": LayerConfig("small_kE_bf16", T=130, d=128, E=4, h=64, k=4, dtype="bf16",
+    "small_kE_bf16": LayerConfig("small_kE_bf16", T=130, d=128, E=8, h=64, k=8, dtype="bf16",
                                  rbd_epd=1, rbd_dpn=2),
     "small_f32": LayerConfig("small_f32", T=333, d=96, E=9, h=40, k=3, dtype="f32",
                              rbd_epd=3, rbd_dpn=1),
