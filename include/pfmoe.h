@@ -101,6 +101,30 @@ PFMOE_API int pft_build(const int32_t* topk_ids, const float* topk_w, int T, int
               void* ws, size_t ws_bytes, int32_t* err, void* stream);
 
 /*
+ * pft_build_no_ws -- pft_build for callers that cannot allocate device memory.
+ *   No counterpart in the X-MoE pages: this is a service of this library.
+ *   Some callers cannot hand pft_build a workspace -- for example a process whose
+ *   device memory is all carved out by another pool at start-up, or a fixed C
+ *   interface that passes only input and output pointers.  This entry point takes
+ *   the same inputs and outputs as pft_build and gives the same results, but
+ *   uses a scratch array built into the library (PFMOE_PFT_NO_WS_SCRATCH_BYTES
+ *   bytes of device memory that every GPU loading the library holds until the
+ *   process exits).  It allocates nothing.
+ *   Limit: pft_build_workspace_size(T, E, k) must not exceed
+ *   PFMOE_PFT_NO_WS_SCRATCH_BYTES (for example T*k up to 262144 with E up to 1024);
+ *   larger shapes return PFMOE_ERR_UNSUPPORTED with a message naming both sizes.
+ *   The first call on a device looks up the array's device address (once, with
+ *   that device current); make that first call before any stream capture.
+ *   All calls on a device share the array and it keeps the last call's contents
+ *   (nothing has to start at zero); calls that overlap on the GPU race on it.
+ */
+#define PFMOE_PFT_NO_WS_SCRATCH_BYTES (1u << 20)
+PFMOE_API int pft_build_no_ws(const int32_t* topk_ids, const float* topk_w, int T, int E, int k,
+                              int32_t* tokens_per_expert, int32_t* expert_offsets, int32_t* token_ids,
+                              int32_t* expert_ids, float* combine_weights, int32_t* pos, int32_t* tile_offsets,
+                              int32_t* err, void* stream);
+
+/*
  * moe_dispatch -- PFT.x ([A] §2.1.2 gather): row pos[t,j] of x_pft [T*k, d]
  *   receives token row x[t].  Equivalent to x_pft[r] = x[token_ids[r]]; it is
  *   computed token-major so that every x row is read once.

@@ -19,6 +19,7 @@ PFMOE_OK, PFMOE_ERR_ARG, PFMOE_ERR_UNSUPPORTED, PFMOE_ERR_CUDA = 0, 1, 2, 3
 PFMOE_F32, PFMOE_BF16 = 0, 1
 DEV_BAD_EXPERT_ID, DEV_BAD_POS, DEV_TIMEOUT, DEV_NONFINITE = 1, 2, 4, 8
 TILE_ROWS = 128
+PFT_NO_WS_SCRATCH_BYTES = 1 << 20
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -31,6 +32,7 @@ SIGNATURES = {
     "moe_route": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
     "pft_build_workspace_size": (_Z, [_I, _I, _I]),
     "pft_build": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _P]),
+    "pft_build_no_ws": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "moe_expert_ffn": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
@@ -122,6 +124,15 @@ def pft_build(topk_ids, topk_w, T, E, k, tokens_per_expert, expert_offsets, toke
                                         _ptr(expert_offsets), _ptr(token_ids), _ptr(expert_ids),
                                         _ptr(combine_weights), _ptr(pos), _ptr(tile_offsets), _ptr(ws), ws_bytes,
                                         _ptr(err), _stream(stream)))
+
+
+def pft_build_no_ws(topk_ids, topk_w, T, E, k, tokens_per_expert, expert_offsets, token_ids, expert_ids,
+                    combine_weights, pos, tile_offsets, err=None, stream=None):
+    """pft_build without a workspace argument: for callers that cannot allocate device memory,
+    the scratch comes from an array built into the library (PFT_NO_WS_SCRATCH_BYTES bytes)."""
+    _check("pft_build_no_ws", lib().pft_build_no_ws(
+        _ptr(topk_ids), _ptr(topk_w), T, E, k, _ptr(tokens_per_expert), _ptr(expert_offsets), _ptr(token_ids),
+        _ptr(expert_ids), _ptr(combine_weights), _ptr(pos), _ptr(tile_offsets), _ptr(err), _stream(stream)))
 
 
 def moe_dispatch(x, pos, T, k, d, dtype, x_pft, err=None, stream=None):

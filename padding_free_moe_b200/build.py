@@ -22,7 +22,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libpfmoe.so")
 
-SOURCES = ["api.cu", "gemm_tc.cu", "gemm_simt.cu", "route.cu", "sort.cu", "rows.cu"]
+SOURCES = ["api.cu", "gemm_tc.cu", "gemm_simt.cu", "route.cu", "sort.cu", "rows.cu", "pft_noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
