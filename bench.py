@@ -37,7 +37,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
@@ -77,7 +77,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                                          "-i", str(self.gpu), "-lms", "200"], stdout=subprocess.PIPE,
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=subprocess.PIPE,
                                          stderr=subprocess.DEVNULL, text=True)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -142,9 +142,15 @@ def kernel_work(cfg, name):
         "token_grad": N * d * b + T * d * b + T * E * (4 + 2) + 16 * N,
         "route_topk": T * E * 4 + 8 * N,
         "pft_hist": 4 * N,
+        "pft_scan": 8 * E,
         "pft_scatter": 8 * N + 16 * N,
         "transpose": 2 * d * E * b,
     }
+    if cfg.has_rbd:   # RBD plan kernels: ids in, pilot / replica lists out (P <= N)
+        P = T * min(k, E // (cfg.rbd_epd * cfg.rbd_dpn))
+        bytes_.update({"rbd_count": 4 * N + 8 * T, "rbd_scan_tokens": 12 * T, "rbd_emit": 4 * N + 16 * P,
+                       "rbd_hist": 4 * P, "rbd_scan_nodes": 8 * T, "rbd_scatter": 24 * P,
+                       "rbd_scan_replicas": 8 * P, "rbd_final": 12 * N + 8 * T})
     if name in bytes_:
         return "hbm", float(bytes_[name])
     return None, None
@@ -359,7 +365,8 @@ def run_ours(args):
             ent["gbs"] = work / (per_ms * 1e-3) / 1e9
             ent["frac_of_peak"] = ent["gbs"] / hbm
         kernels[nm] = ent
-    dom = max(kern.items(), key=lambda kv: kv[1][1])[0]
+    known = {nm: v for nm, v in kern.items() if kernel_work(cfg, nm)[0] is not None}
+    dom = max((known or kern).items(), key=lambda kv: kv[1][1])[0]
     kind, work = kernel_work(cfg, dom)
     dom_ms = kern[dom][1] / kern[dom][0]
     if kind == "tensor":
