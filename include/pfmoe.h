@@ -76,10 +76,15 @@ PFMOE_API int moe_abi_version(void);
  *     logits are ordered by the lower expert index.  Selection is decided on the
  *     float32 logits written to `logits`.
  *   topk_w [T,k] float32 out: softmax over the k selected logits (sums to 1).
- *   Requires 1 <= k <= E, k <= 32, E <= 1024, T >= 1.
+ *   ws (nullable): moe_route_workspace_size(...) bytes.  With it, the BF16 gate GEMM
+ *   splits its K dimension over more SMs and sums the parts in a fixed order (the
+ *   result does not depend on the split); without it the GEMM runs unsplit.
+ *   Requires 1 <= k <= E, k <= 32, E <= 1024.
  */
+PFMOE_API size_t moe_route_workspace_size(int T, int d, int E, int k, int dtype);
 PFMOE_API int moe_route(const void* x, const void* wg, const float* bias, int T, int d, int E, int k, int dtype,
-              float* logits, int32_t* topk_ids, float* topk_w, int32_t* err, void* stream);
+                        float* logits, int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes, int32_t* err,
+                        void* stream);
 
 /*
  * pft_build -- the padding-free token buffer's index fields ([A] §2.1.1).

@@ -29,7 +29,8 @@ _Z = ctypes.c_size_t
 SIGNATURES = {
     "moe_last_error": (ctypes.c_char_p, []),
     "moe_abi_version": (_I, []),
-    "moe_route": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "moe_route_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
+    "moe_route": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _Z, _P, _P]),
     "pft_build_workspace_size": (_Z, [_I, _I, _I]),
     "pft_build": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _P]),
     "pft_build_no_ws": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
@@ -109,9 +110,14 @@ def moe_abi_version() -> int:
     return lib().moe_abi_version()
 
 
-def moe_route(x, wg, bias, T, d, E, k, dtype, logits, topk_ids, topk_w, err=None, stream=None):
+def moe_route_workspace_size(T, d, E, k, dtype) -> int:
+    return lib().moe_route_workspace_size(T, d, E, k, dtype)
+
+
+def moe_route(x, wg, bias, T, d, E, k, dtype, logits, topk_ids, topk_w, ws=None, ws_bytes=0, err=None, stream=None):
     _check("moe_route", lib().moe_route(_ptr(x), _ptr(wg), _ptr(bias), T, d, E, k, dtype, _ptr(logits),
-                                        _ptr(topk_ids), _ptr(topk_w), _ptr(err), _stream(stream)))
+                                        _ptr(topk_ids), _ptr(topk_w), _ptr(ws), ws_bytes, _ptr(err),
+                                        _stream(stream)))
 
 
 def pft_build_workspace_size(T, E, k) -> int:

@@ -139,6 +139,8 @@ struct BwdWs {
   void* dx_pft;
   void* wgT;
   void* dz_bf16;  // BF16 path only
+  void* dwg_parts;  // BF16 path only: split-K partial sums of dWg
+  size_t dwg_parts_bytes;
   size_t bytes;
 };
 
@@ -155,6 +157,8 @@ BwdWs carve_bwd(void* base, int T, int d, int E, int h, int k, int dtype) {
   w.dx_pft = c.take(N * d * es);
   w.wgT = c.take(static_cast<size_t>(E) * d * es);
   w.dz_bf16 = dtype == PFMOE_BF16 ? c.take(static_cast<size_t>(T) * E * 2) : nullptr;
+  w.dwg_parts_bytes = dtype == PFMOE_BF16 && T > 0 ? tc_gate_wgrad_ws(T, d, E) : 0;
+  w.dwg_parts = w.dwg_parts_bytes ? c.take(w.dwg_parts_bytes) : nullptr;
   w.bytes = c.used;
   return w;
 }
@@ -175,10 +179,15 @@ extern "C" {
 
 const char* moe_last_error(void) { return g_last_error.c_str(); }
 
-int moe_abi_version(void) { return 1; }
+int moe_abi_version(void) { return 2; }
+
+size_t moe_route_workspace_size(int T, int d, int E, int k, int dtype) {
+  if (T <= 0 || d <= 0 || E <= 0 || k <= 0 || dtype != PFMOE_BF16) return 0;
+  return align256(tc_gate_logits_ws(T, d, E));
+}
 
 int moe_route(const void* x, const void* wg, const float* bias, int T, int d, int E, int k, int dtype, float* logits,
-              int32_t* topk_ids, float* topk_w, int32_t* err, void* stream) {
+              int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes, int32_t* err, void* stream) {
   set_error("");
   PFMOE_TRY(need_dtype(dtype));
   PFMOE_TRY(need_tk(T, k, E));
@@ -192,9 +201,11 @@ int moe_route(const void* x, const void* wg, const float* bias, int T, int d, in
   PFMOE_TRY(need_ptr(logits, "logits"));
   PFMOE_TRY(need_ptr(topk_ids, "topk_ids"));
   PFMOE_TRY(need_ptr(topk_w, "topk_w"));
+  PFMOE_TRY(need_ptr(ws, "ws", true));
+  if (ws && ws_bytes < moe_route_workspace_size(T, d, E, k, dtype)) return fail(PFMOE_ERR_ARG, "workspace too small");
   cudaStream_t s = st(stream);
   if (dtype == PFMOE_BF16) {
-    PFMOE_TRY(tc_gate_logits(x, wg, bias, T, d, E, logits, err, s));
+    PFMOE_TRY(tc_gate_logits(x, wg, bias, T, d, E, logits, ws, ws_bytes, err, s));
   } else {
     SimtGemm g{};
     g.A = static_cast<const float*>(x); g.sam = d; g.sak = 1;
@@ -349,7 +360,7 @@ int moe_backward(const void* dy, const void* x, const void* wg, const float* top
     PFMOE_TRY(launch_transpose(wg, d, E, dtype, w.wgT, s));
     PFMOE_TRY(launch_token_grad(w.dx_pft, pos, w.g, topk_w, topk_ids, w.wgT, T, k, d, E, dtype, dx, dlogits,
                                 w.dz_bf16, err, s));
-    return tc_gate_wgrad(x, w.dz_bf16, T, d, E, dwg, err, s);
+    return tc_gate_wgrad(x, w.dz_bf16, T, d, E, dwg, w.dwg_parts, w.dwg_parts_bytes, err, s);
   }
   // FP32 path on the CUDA cores.
   const long long dh = static_cast<long long>(d) * h;

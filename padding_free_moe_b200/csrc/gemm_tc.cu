@@ -58,6 +58,8 @@ struct Params {
   int G;
   int dense_len;
   int stages;
+  int ksplit;        // dense problems only: K is cut into ksplit parts, part s writes output slice s
+  int kchunk;        // KG dense: K rows per part (multiple of BK)
   void* D0;
   void* D1;
   void* D2;
@@ -77,6 +79,8 @@ struct Tile {
   int nk;      // K blocks
   int krow0;   // KG: first K row of the segment
   int kvalid;  // KG: valid K rows in the last block
+  int kb0;     // RG: first K block (split-K)
+  int split;   // RG: split-K part (output slice)
 };
 
 // ------------------------------------------------------------------ PTX wrappers
@@ -205,22 +209,24 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
 // ----------------------------------------------------------------- tile schedule
 __device__ __forceinline__ int n_step(const Params& p) { return p.nsplit ? p.bn / 2 : p.bn; }
 
+template <int MODE>
 __device__ __forceinline__ int total_tiles(const Params& p) {
   const int ns = n_step(p);
   const int NT = (p.Nout + ns - 1) / ns;
-  if (p.mode == RG) {
-    const int mt = p.tiles ? p.tiles[p.G] : (p.dense_len + BM - 1) / BM;
+  if constexpr (MODE == RG) {
+    const int mt = p.tiles ? p.tiles[p.G] : (p.dense_len + BM - 1) / BM * p.ksplit;
     return mt * NT;
   }
   return p.G * ((p.M + BM - 1) / BM) * NT;
 }
 
+template <int MODE>
 __device__ __forceinline__ Tile decode(const Params& p, int t) {
   Tile tl;
   const int ns = n_step(p);
   const int NT = (p.Nout + ns - 1) / ns;
-  if (p.mode == RG) {
-    int g = 0, tbase = 0, mtg, s0, s1;
+  if constexpr (MODE == RG) {
+    int g = 0, tbase = 0, mtg, s0, s1, split = 0;
     if (p.tiles) {
       int lo = 0, hi = p.G - 1;
       while (lo < hi) {
@@ -236,6 +242,8 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
       mtg = (p.dense_len + BM - 1) / BM;
       s0 = 0;
       s1 = p.dense_len;
+      split = t / (mtg * NT);
+      tbase = split * mtg * NT;
     }
     const int local = t - tbase;
     const int n_idx = local / mtg;
@@ -244,7 +252,11 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
     tl.row0 = s0 + m_loc * BM;
     tl.rows = min(BM, s1 - tl.row0);
     tl.n0 = n_idx * ns;
-    tl.nk = p.k0_blocks + p.k1_blocks;
+    const int nk_all = p.k0_blocks + p.k1_blocks;
+    const int kbs = (nk_all + p.ksplit - 1) / p.ksplit;
+    tl.split = split;
+    tl.kb0 = split * kbs;
+    tl.nk = max(0, min(kbs, nk_all - tl.kb0));
     tl.krow0 = 0;
     tl.kvalid = BK;
   } else {
@@ -254,9 +266,11 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
     const int rem = t - g * per;
     const int n_idx = rem / MT;
     const int m_idx = rem - n_idx * MT;
-    const int s0 = p.seg ? p.seg[g] : 0;
-    const int s1 = p.seg ? p.seg[g + 1] : p.dense_len;
+    const int s0 = p.seg ? p.seg[g] : g * p.kchunk;
+    const int s1 = p.seg ? p.seg[g + 1] : min(p.dense_len, s0 + p.kchunk);
     const int len = max(0, s1 - s0);
+    tl.split = 0;
+    tl.kb0 = 0;
     tl.g = g;
     tl.row0 = m_idx * BM;
     tl.rows = min(BM, p.M - tl.row0);
@@ -268,7 +282,11 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
   return tl;
 }
 
-// -------------------------------------------------------------------- epilogue
+// ------------------------------------------------------------- direct epilogue
+// Row-grouped tiles: each thread stores its own row straight from registers (16-byte
+// vectors).  These tiles have long K loops, so the epilogue hides behind the next
+// tile's mainloop, and measured faster than staging through shared memory, which
+// competes with the operand traffic of the mainloop.
 template <typename T>
 __device__ __forceinline__ void store_row_chunk(T* dst, const float* v, int ncols_valid) {
   // Store up to 32 values of one row; ncols_valid is a multiple of 8 (BF16) or 4 (F32) or >= 32.
@@ -279,13 +297,13 @@ __device__ __forceinline__ void store_row_chunk(T* dst, const float* v, int ncol
 }
 
 template <int EPI>
-__device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, uint32_t tacc, int r) {
+__device__ __forceinline__ void epilogue_tile_direct(const Params& p, const Tile& tl, uint32_t tacc, int r) {
   const bool row_ok = r < tl.rows;
   const long long grow = static_cast<long long>(tl.row0) + r;
   const bool zero = tl.nk == 0;
   if constexpr (EPI == EPI_STORE_BF16 || EPI == EPI_STORE_F32) {
     using T = typename std::conditional<EPI == EPI_STORE_F32, float, __nv_bfloat16>::type;
-    T* D = static_cast<T*>(p.D0) + (p.mode == KG ? tl.g * p.d_gstride : 0);
+    T* D = static_cast<T*>(p.D0) + (p.mode == KG ? tl.g : tl.split) * p.d_gstride;
     for (int c = 0; c < p.bn; c += 32) {
       const int col = tl.n0 + c;
       if (col >= p.Nout) break;
@@ -383,15 +401,235 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, u
   }
 }
 
-// ---------------------------------------------------------------------- kernel
+// -------------------------------------------------------- staged epilogue
+// Each epilogue warp owns a 32-row slab of the 128-row accumulator (its TMEM lane
+// quarter).  Values leave TMEM one row per thread; they are written to a per-warp
+// 32 x 128-byte staging buffer in shared memory (16-byte chunks swizzled by row so
+// both the row-wise writes and the column-wise reads are bank-conflict free) and
+// copied to global memory four rows per instruction, eight lanes per 128-byte row
+// segment.  Every global store is then part of a full 128-byte line.  Used for
+// K-grouped (weight-gradient) tiles, whose short K loops leave the epilogue exposed.
+constexpr int STAGE_BYTES_PER_WARP = 32 * 128;
+
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+// 64 consecutive accumulator columns of this thread's row (two loads, one wait).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+  tmem_ld32_async(taddr, r);
+  tmem_ld32_async(taddr + 32, r + 32);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ uint32_t stg_addr(uint32_t stg, int row, int chunk) {
+  return stg + row * 128 + ((chunk ^ (row & 7)) << 4);
+}
+__device__ __forceinline__ void st_shared16(uint32_t addr, uint4 u) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(u.x), "r"(u.y), "r"(u.z), "r"(u.w)
+               : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared16(uint32_t addr) {
+  uint4 u;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(addr)
+               : "memory");
+  return u;
+}
+
+// Thread `lane` writes row `lane` of the slab: 64 BF16 values (or 32 FP32 values) = 128 bytes.
+template <typename T>
+__device__ __forceinline__ void stage_row(uint32_t stg, int lane, const float* v) {
+  constexpr int VN = Vec<T>::n;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint4 u;
+    if constexpr (sizeof(T) == 4) {
+      u.x = __float_as_uint(v[4 * c]); u.y = __float_as_uint(v[4 * c + 1]);
+      u.z = __float_as_uint(v[4 * c + 2]); u.w = __float_as_uint(v[4 * c + 3]);
+    } else {
+      __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[VN * c + 2 * i], v[VN * c + 2 * i + 1]);
+    }
+    st_shared16(stg_addr(stg, lane, c), u);
+  }
+}
+
+// Thread `lane` reads back row `lane` of the slab as 64 BF16 values.
+__device__ __forceinline__ void unstage_row_bf16(uint32_t stg, int lane, float* v) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint4 u = ld_shared16(stg_addr(stg, lane, c));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      v[8 * c + 2 * i] = f.x;
+      v[8 * c + 2 * i + 1] = f.y;
+    }
+  }
+}
+
+// Staged slab -> global rows base + row * stride (bytes); rows >= rows_valid and bytes >= bytes_valid are skipped.
+__device__ __forceinline__ void copy_out(uint32_t stg, int lane, char* base, long long stride, int rows_valid,
+                                         int bytes_valid) {
+  const int chunk = lane & 7;
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int row = it * 4 + (lane >> 3);
+    const uint4 u = ld_shared16(stg_addr(stg, row, chunk));
+    if (row < rows_valid && chunk * 16 < bytes_valid)
+      *reinterpret_cast<uint4*>(base + row * stride + chunk * 16) = u;
+  }
+}
+
+// Global rows -> staged slab (coalesced); missing rows / bytes read as zero.
+__device__ __forceinline__ void copy_in(uint32_t stg, int lane, const char* base, long long stride, int rows_valid,
+                                        int bytes_valid) {
+  const int chunk = lane & 7;
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int row = it * 4 + (lane >> 3);
+    uint4 u = make_uint4(0, 0, 0, 0);
+    if (row < rows_valid && chunk * 16 < bytes_valid)
+      u = __ldg(reinterpret_cast<const uint4*>(base + row * stride + chunk * 16));
+    st_shared16(stg_addr(stg, row, chunk), u);
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void emit(uint32_t stg, int lane, const float* v, T* dst_row0, long long ldd,
+                                     int rows_valid, int cols_valid) {
+  __syncwarp();
+  stage_row<T>(stg, lane, v);
+  __syncwarp();
+  copy_out(stg, lane, reinterpret_cast<char*>(dst_row0), ldd * static_cast<long long>(sizeof(T)), rows_valid,
+           min(128, cols_valid * static_cast<int>(sizeof(T))));
+}
+
 template <int EPI>
+__device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, uint32_t tacc, int q, int lane,
+                                              uint32_t stg) {
+  const int slab0 = q * 32;
+  const int rows_valid = max(0, min(32, tl.rows - slab0));
+  const long long grow0 = static_cast<long long>(tl.row0) + slab0;
+  const bool zero = tl.nk == 0;
+  if constexpr (EPI == EPI_STORE_BF16 || EPI == EPI_SPLIT_BF16) {
+    const int nparts = EPI == EPI_SPLIT_BF16 ? 2 : 1;
+    const int width = EPI == EPI_SPLIT_BF16 ? p.bn / 2 : p.bn;
+    const long long goff = p.mode == KG ? tl.g * p.d_gstride : 0;
+    for (int part = 0; part < nparts; ++part) {
+      __nv_bfloat16* D = static_cast<__nv_bfloat16*>(part == 0 ? p.D0 : p.D1) + goff;
+      for (int c = 0; c < width; c += 64) {
+        const int col = tl.n0 + c;
+        if (col >= p.Nout) break;
+        float v[64];
+        if (!zero) tmem_ld64(tacc + part * width + c, v);
+        else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) v[i] = 0.f;
+        }
+        emit(stg, lane, v, D + grow0 * p.ldd + col, p.ldd, rows_valid, p.Nout - col);
+      }
+    }
+  } else if constexpr (EPI == EPI_STORE_F32) {
+    float* D = static_cast<float*>(p.D0) + (p.mode == KG ? tl.g * p.d_gstride : 0);
+    for (int c = 0; c < p.bn; c += 32) {
+      const int col = tl.n0 + c;
+      if (col >= p.Nout) break;
+      float v[32];
+      if (!zero) {
+        uint32_t r[32];
+        tmem_ld32_async(tacc + c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      }
+      if (p.bias) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (col + i < p.Nout) v[i] += p.bias[col + i];
+      }
+      emit(stg, lane, v, D + grow0 * p.ldd + col, p.ldd, rows_valid, p.Nout - col);
+    }
+  } else if constexpr (EPI == EPI_SWIGLU_FWD) {
+    // D columns [0, bn/2) = H1 tile, [bn/2, bn) = H3 tile for the same output columns.
+    const int half = p.bn / 2;
+    __nv_bfloat16* H1 = static_cast<__nv_bfloat16*>(p.D0);
+    __nv_bfloat16* H3 = static_cast<__nv_bfloat16*>(p.D1);
+    __nv_bfloat16* A = static_cast<__nv_bfloat16*>(p.D2);
+    for (int c = 0; c < half; c += 64) {
+      const int col = tl.n0 + c;
+      if (col >= p.Nout) break;
+      const long long off = grow0 * p.ldd + col;
+      float h1[64], h3[64];
+      tmem_ld64(tacc + c, h1);
+      tmem_ld64(tacc + half + c, h3);
+      emit(stg, lane, h1, H1 + off, p.ldd, rows_valid, p.Nout - col);
+      emit(stg, lane, h3, H3 + off, p.ldd, rows_valid, p.Nout - col);
+#pragma unroll
+      for (int i = 0; i < 64; ++i) h1[i] = silu_f(h1[i]) * h3[i];
+      emit(stg, lane, h1, A + off, p.ldd, rows_valid, p.Nout - col);
+    }
+  } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+    // Accumulator = dA.  dH1 = dA * H3 * s * (1 + H1 (1 - s)), dH3 = dA * SiLU(H1), s = sigmoid(H1).
+    const char* H1 = static_cast<const char*>(p.X0);
+    const char* H3 = static_cast<const char*>(p.X1);
+    __nv_bfloat16* dH1 = static_cast<__nv_bfloat16*>(p.D0);
+    __nv_bfloat16* dH3 = static_cast<__nv_bfloat16*>(p.D1);
+    const long long stride = p.ldd * 2;
+    for (int c = 0; c < p.bn; c += 64) {
+      const int col = tl.n0 + c;
+      if (col >= p.Nout) break;
+      const long long off = grow0 * p.ldd + col;
+      const int bytes_valid = min(128, (p.Nout - col) * 2);
+      float da[64], h1[64], h3[64];
+      tmem_ld64(tacc + c, da);
+      __syncwarp();
+      copy_in(stg, lane, H1 + off * 2, stride, rows_valid, bytes_valid);
+      __syncwarp();
+      unstage_row_bf16(stg, lane, h1);
+      __syncwarp();
+      copy_in(stg, lane, H3 + off * 2, stride, rows_valid, bytes_valid);
+      __syncwarp();
+      unstage_row_bf16(stg, lane, h3);
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float s = 1.0f / (1.0f + expf(-h1[i]));
+        const float d1 = da[i] * h3[i] * s * (1.0f + h1[i] * (1.0f - s));
+        h1[i] = da[i] * h1[i] * s;
+        da[i] = d1;
+      }
+      emit(stg, lane, da, dH1 + off, p.ldd, rows_valid, p.Nout - col);
+      emit(stg, lane, h1, dH3 + off, p.ldd, rows_valid, p.Nout - col);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------- kernel
+template <int EPI, int MODE>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages;
   const uint32_t b_bytes = static_cast<uint32_t>(p.bn) * BK * 2;
   const uint32_t stage_bytes = A_BYTES + b_bytes;
-  uint8_t* bar_area = smem + S * stage_bytes;
+  uint8_t* stage_area = smem + S * stage_bytes;                       // epilogue staging (K-grouped only)
+  uint8_t* bar_area = stage_area + (MODE == KG ? 4 * STAGE_BYTES_PER_WARP : 0);
   uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
   uint64_t* empty = full + MAX_STAGES;
   uint64_t* acc_full = empty + MAX_STAGES;
@@ -430,7 +668,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int ntiles = total_tiles(p);
+  const int ntiles = total_tiles<MODE>(p);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -440,7 +678,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const Tile tl = decode(p, t);
+        const Tile tl = decode<MODE>(p, t);
         for (int kb = 0; kb < tl.nk; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
@@ -450,9 +688,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
           const uint32_t sa = smem_u32(smem + s * stage_bytes);
           const uint32_t sb = sa + A_BYTES;
           const int nb = p.bn / 64;
-          if (p.mode == RG) {
-            const int src = kb < p.k0_blocks ? 0 : 1;
-            const int kk = (src == 0 ? kb : kb - p.k0_blocks) * BK;
+          if constexpr (MODE == RG) {
+            const int kbg = tl.kb0 + kb;
+            const int src = kbg < p.k0_blocks ? 0 : 1;
+            const int kk = (src == 0 ? kbg : kbg - p.k0_blocks) * BK;
             tma_load_3d(sa, &p.tmA[src], fb, kk, tl.row0, 0);
             if (p.b_major == 0) {
               if (p.nsplit) {
@@ -495,15 +734,15 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     }
   } else if (warp == 1) {
     // -------------------------------------------------------------- MMA issuer
-    const int a_mn = p.mode == KG ? 1 : 0;
-    const int b_mn = p.mode == KG ? 1 : p.b_major;
+    const int a_mn = MODE == KG ? 1 : 0;
+    const int b_mn = MODE == KG ? 1 : p.b_major;
     const uint32_t idesc = idesc_bf16(BM, p.bn, a_mn, b_mn);
     const uint32_t a_lbo = a_mn ? BOX_BYTES : 16, b_lbo = b_mn ? BOX_BYTES : 16;
     const uint32_t a_step = a_mn ? 2048 : 32, b_step = b_mn ? 2048 : 32;
     int it = 0, tcount = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
-      const Tile tl = decode(p, t);
+      const Tile tl = decode<MODE>(p, t);
       const int buf = tcount & 1;
       const uint32_t aph = (tcount >> 1) & 1;
       ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&acc_empty[buf]), aph ^ 1, abort_flag, p.err));
@@ -522,22 +761,25 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         if (!ok) break;
         const uint32_t sa = smem_u32(smem + s * stage_bytes);
         const uint32_t sb = sa + A_BYTES;
-        if (p.mode == KG && kb == tl.nk - 1 && tl.kvalid < BK) {
-          // Zero K rows past the segment end in every box of this stage (A: 2 boxes, B: bn/64).
-          const int nbox = 2 + p.bn / 64;
-          const int per_box = (BK - tl.kvalid) * 8;   // 16-byte chunks per box
-          for (int i = lane; i < nbox * per_box; i += 32) {
-            const int b = i / per_box, c = i - b * per_box;
-            const uint32_t addr = sa + b * BOX_BYTES + tl.kvalid * 128 + c * 16;
-            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0) : "memory");
+        int kk_count = BK / 16;
+        if (MODE == KG && kb == tl.nk - 1 && tl.kvalid < BK) {
+          // Last block of a segment: MMAs stop at the 16-row step holding the segment end, and the
+          // rows of that step past the end are zeroed in every box (A: 2 boxes, B: bn/64).
+          const int kv16 = (tl.kvalid + 15) & ~15;
+          kk_count = kv16 / 16;
+          const int per_box = (kv16 - tl.kvalid) * 8;   // 16-byte chunks to clear per box
+          if (per_box > 0) {
+            const int nbox = 2 + p.bn / 64;
+            for (int b = 0; b < nbox; ++b)
+              for (int i = lane; i < per_box; i += 32)
+                st_shared16(sa + b * BOX_BYTES + tl.kvalid * 128 + i * 16, make_uint4(0, 0, 0, 0));
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           __syncwarp();
         }
         tc_fence_after();
         if (lane == 0) {
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
+          for (int kk = 0; kk < kk_count; ++kk) {
             const uint64_t ad = sdesc(sa + kk * a_step, a_lbo, 1024);
             const uint64_t bd = sdesc(sb + kk * b_step, b_lbo, 1024);
             tc_mma(tmem_d, ad, bd, idesc, (kb | kk) != 0);
@@ -558,17 +800,18 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
-    const int q = warp & 3;           // TMEM lane quarter this warp may access
-    const int r = q * 32 + lane;      // accumulator row held by this thread
+    const int q = warp & 3;           // TMEM lane quarter this warp may access: rows 32q .. 32q+31
+    const uint32_t stg = smem_u32(stage_area + (warp - 2) * STAGE_BYTES_PER_WARP);
     int tcount = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
-      const Tile tl = decode(p, t);
+      const Tile tl = decode<MODE>(p, t);
       const int buf = tcount & 1;
       const uint32_t aph = (tcount >> 1) & 1;
       if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&acc_full[buf]), aph, abort_flag, p.err))) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * p.bn;
-      epilogue_tile<EPI>(p, tl, tacc, r);
+      if constexpr (MODE == KG) epilogue_tile<EPI>(p, tl, tacc, q, lane, stg);
+      else epilogue_tile_direct<EPI>(p, tl, tacc, q * 32 + lane);
       tc_fence_before();
       mbar_arrive(smem_u32(&acc_empty[buf]));
     }
@@ -620,23 +863,29 @@ static int round_bn(int n) {
   return bn > 256 ? 256 : bn;
 }
 
-static int pick_stages(int bn) {
+constexpr int SMEM_LIMIT = 227 * 1024;
+// Alignment slack + barriers, plus the epilogue staging buffers when the launch uses them (K-grouped).
+static int smem_fixed(bool staged) { return 1024 + 256 + (staged ? 4 * STAGE_BYTES_PER_WARP : 0); }
+
+static int pick_stages(int bn, bool staged) {
   const int stage = A_BYTES + bn * BK * 2;
-  int s = (200 * 1024) / stage;
+  int s = (SMEM_LIMIT - smem_fixed(staged)) / stage;
   return s > MAX_STAGES ? MAX_STAGES : s;
 }
 
-static size_t smem_bytes(int bn, int stages) {
-  return 1024 + static_cast<size_t>(stages) * (A_BYTES + bn * BK * 2) + 256;
+static size_t smem_bytes(int bn, int stages, bool staged) {
+  return smem_fixed(staged) + static_cast<size_t>(stages) * (A_BYTES + bn * BK * 2);
 }
 
-template <int EPI>
+template <int EPI, int MODE>
 static int launch(Params& p, long long tile_upper_bound, const char* name, cudaStream_t stream) {
-  p.stages = pick_stages(p.bn);
-  const size_t smem = smem_bytes(p.bn, p.stages);
+  p.mode = MODE;
+  const bool staged = p.mode == KG;
+  p.stages = pick_stages(p.bn, staged);
+  const size_t smem = smem_bytes(p.bn, p.stages, staged);
   static bool attr_done = false;  // per template instance
   if (!attr_done) {
-    if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(227 * 1024)) != cudaSuccess)
       return fail(PFMOE_ERR_CUDA, std::string("cudaFuncSetAttribute failed: ") +
                                       cudaGetErrorString(cudaGetLastError()));
@@ -646,7 +895,7 @@ static int launch(Params& p, long long tile_upper_bound, const char* name, cudaS
   long long grid = num_sms();
   if (tile_upper_bound < grid) grid = tile_upper_bound;
   PFMOE_LAUNCH(name, stream,
-               grouped_gemm_kernel<EPI><<<static_cast<int>(grid), THREADS, smem, stream>>>(p));
+               (grouped_gemm_kernel<EPI, MODE><<<static_cast<int>(grid), THREADS, smem, stream>>>(p)));
   return PFMOE_OK;
 }
 
@@ -654,7 +903,51 @@ static Params base_params(int32_t* err) {
   Params p;
   memset(&p, 0, sizeof(p));
   p.err = err;
+  p.ksplit = 1;
   return p;
+}
+
+// Split-K for the dense gate GEMMs, which have too few output tiles to fill the GPU:
+// enough parts for about one wave on a 148-SM B200, at least 4 K blocks per part,
+// every part non-empty.  Depends only on the shape, so workspace sizes are host-computable.
+static int choose_ksplit(long long tiles, int nk) {
+  long long ks = (148 + tiles - 1) / tiles;
+  if (ks > 8) ks = 8;
+  const long long cap = nk / 4 > 1 ? nk / 4 : 1;
+  if (ks > cap) ks = cap;
+  if (ks < 1) ks = 1;
+  const long long kbs = (nk + ks - 1) / ks;
+  return static_cast<int>((nk + kbs - 1) / kbs);
+}
+
+__global__ void split_reduce_kernel(const float* __restrict__ parts, int nparts, long long n,
+                                    const float* __restrict__ bias, int ncols, float* __restrict__ out) {
+  // out = parts[0] + parts[1] + ... (fixed order) + bias[column]; n and ncols are multiples of 4.
+  const long long n4 = n / 4;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float4 acc = reinterpret_cast<const float4*>(parts)[i];
+    for (int s = 1; s < nparts; ++s) {
+      const float4 v = reinterpret_cast<const float4*>(parts + s * n)[i];
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    if (bias) {
+      const int c = static_cast<int>((i * 4) % ncols);
+      acc.x += bias[c]; acc.y += bias[c + 1]; acc.z += bias[c + 2]; acc.w += bias[c + 3];
+    }
+    reinterpret_cast<float4*>(out)[i] = acc;
+  }
+}
+
+static int launch_split_reduce(const float* parts, int nparts, long long n, const float* bias, int ncols, float* out,
+                               cudaStream_t s) {
+  long long blocks = (n / 4 + 255) / 256;
+  const long long cap = static_cast<long long>(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  PFMOE_LAUNCH("gate_split_reduce", s,
+               split_reduce_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(parts, nparts, n, bias, ncols, out));
+  return PFMOE_OK;
 }
 
 }  // namespace tc
@@ -680,7 +973,7 @@ int tc_ffn_gemm1(const void* x_pft, const int* seg, const int* tiles, int N, int
   PFMOE_TRY(make_tmap(&p.tmA[0], x_pft, d, N, 1, BK, BM, "x_pft"));
   PFMOE_TRY(make_tmap(&p.tmB[0], w1, h, d, E, 64, 64, "w1"));
   PFMOE_TRY(make_tmap(&p.tmB[1], w3, h, d, E, 64, 64, "w3"));
-  return launch<EPI_SWIGLU_FWD>(p, rg_tiles_ub(N, E, h, p.bn / 2), "ffn_gemm1_swiglu", s);
+  return launch<EPI_SWIGLU_FWD, RG>(p, rg_tiles_ub(N, E, h, p.bn / 2), "ffn_gemm1_swiglu", s);
 }
 
 int tc_ffn_gemm2(const void* a, const int* seg, const int* tiles, int N, int E, int d, int h, const void* w2,
@@ -695,7 +988,7 @@ int tc_ffn_gemm2(const void* a, const int* seg, const int* tiles, int N, int E, 
   p.D0 = out; p.ldd = d;
   PFMOE_TRY(make_tmap(&p.tmA[0], a, h, N, 1, BK, BM, "a"));
   PFMOE_TRY(make_tmap(&p.tmB[0], w2, d, h, E, 64, 64, "w2"));
-  return launch<EPI_STORE_BF16>(p, rg_tiles_ub(N, E, d, p.bn), "ffn_gemm2", s);
+  return launch<EPI_STORE_BF16, RG>(p, rg_tiles_ub(N, E, d, p.bn), "ffn_gemm2", s);
 }
 
 int tc_ffn_dgrad_act(const void* dO, const int* seg, const int* tiles, int N, int E, int d, int h, const void* w2,
@@ -710,7 +1003,7 @@ int tc_ffn_dgrad_act(const void* dO, const int* seg, const int* tiles, int N, in
   p.X0 = h1; p.X1 = h3; p.D0 = dh1; p.D1 = dh3; p.ldd = h;
   PFMOE_TRY(make_tmap(&p.tmA[0], dO, d, N, 1, BK, BM, "dO"));
   PFMOE_TRY(make_tmap(&p.tmB[0], w2, d, h, E, BK, p.bn, "w2^T"));
-  return launch<EPI_SWIGLU_BWD>(p, rg_tiles_ub(N, E, h, p.bn), "ffn_dgrad_act_swiglu_bwd", s);
+  return launch<EPI_SWIGLU_BWD, RG>(p, rg_tiles_ub(N, E, h, p.bn), "ffn_dgrad_act_swiglu_bwd", s);
 }
 
 int tc_ffn_dgrad_x(const void* dh1, const void* dh3, const int* seg, const int* tiles, int N, int E, int d, int h,
@@ -728,7 +1021,7 @@ int tc_ffn_dgrad_x(const void* dh1, const void* dh3, const int* seg, const int* 
   PFMOE_TRY(make_tmap(&p.tmA[1], dh3, h, N, 1, BK, BM, "dh3"));
   PFMOE_TRY(make_tmap(&p.tmB[0], w1, h, d, E, BK, p.bn, "w1^T"));
   PFMOE_TRY(make_tmap(&p.tmB[1], w3, h, d, E, BK, p.bn, "w3^T"));
-  return launch<EPI_STORE_BF16>(p, rg_tiles_ub(N, E, d, p.bn), "ffn_dgrad_x", s);
+  return launch<EPI_STORE_BF16, RG>(p, rg_tiles_ub(N, E, d, p.bn), "ffn_dgrad_x", s);
 }
 
 int tc_ffn_wgrad13(const void* x_pft, const void* dh1, const void* dh3, const int* seg, int N, int E, int d, int h,
@@ -746,7 +1039,7 @@ int tc_ffn_wgrad13(const void* x_pft, const void* dh1, const void* dh3, const in
   PFMOE_TRY(make_tmap(&p.tmB[0], dh1, h, N, 1, 64, 64, "dh1"));
   PFMOE_TRY(make_tmap(&p.tmB[1], dh3, h, N, 1, 64, 64, "dh3"));
   const long long ub = static_cast<long long>(E) * ((d + BM - 1) / BM) * ((h + p.bn / 2 - 1) / (p.bn / 2));
-  return launch<EPI_SPLIT_BF16>(p, ub, "ffn_wgrad_w1w3", s);
+  return launch<EPI_SPLIT_BF16, KG>(p, ub, "ffn_wgrad_w1w3", s);
 }
 
 int tc_ffn_wgrad2(const void* a, const void* dO, const int* seg, int N, int E, int d, int h, void* dw2,
@@ -762,11 +1055,31 @@ int tc_ffn_wgrad2(const void* a, const void* dO, const int* seg, int N, int E, i
   PFMOE_TRY(make_tmap(&p.tmA[0], a, h, N, 1, 64, 64, "a^T"));
   PFMOE_TRY(make_tmap(&p.tmB[0], dO, d, N, 1, 64, 64, "dO"));
   const long long ub = static_cast<long long>(E) * ((h + BM - 1) / BM) * ((d + p.bn - 1) / p.bn);
-  return launch<EPI_STORE_BF16>(p, ub, "ffn_wgrad_w2", s);
+  return launch<EPI_STORE_BF16, KG>(p, ub, "ffn_wgrad_w2", s);
 }
 
-int tc_gate_logits(const void* x, const void* wg, const float* bias, int T, int d, int E, float* logits,
-                   int32_t* err, cudaStream_t s) {
+static int gate_logits_split(int T, int d, int E) {
+  const int bn = round_bn(E);
+  return choose_ksplit(static_cast<long long>((T + BM - 1) / BM) * ((E + bn - 1) / bn), (d + BK - 1) / BK);
+}
+
+static int gate_wgrad_split(int T, int d, int E) {
+  const int bn = round_bn(E);
+  return choose_ksplit(static_cast<long long>((d + BM - 1) / BM) * ((E + bn - 1) / bn), (T + BK - 1) / BK);
+}
+
+size_t tc_gate_logits_ws(int T, int d, int E) {
+  const int ks = gate_logits_split(T, d, E);
+  return ks > 1 ? static_cast<size_t>(ks) * T * E * sizeof(float) : 0;
+}
+
+size_t tc_gate_wgrad_ws(int T, int d, int E) {
+  const int ks = gate_wgrad_split(T, d, E);
+  return ks > 1 ? static_cast<size_t>(ks) * d * E * sizeof(float) : 0;
+}
+
+int tc_gate_logits(const void* x, const void* wg, const float* bias, int T, int d, int E, float* logits, void* ws,
+                   size_t ws_bytes, int32_t* err, cudaStream_t s) {
   Params p = base_params(err);
   p.mode = RG;
   p.b_major = 1;              // Wg [d, E]: K rows, E contiguous
@@ -775,28 +1088,56 @@ int tc_gate_logits(const void* x, const void* wg, const float* bias, int T, int 
   p.k0_blocks = (d + BK - 1) / BK;
   p.G = 1;
   p.dense_len = T;
-  p.D0 = logits; p.bias = bias; p.ldd = E;
+  p.ldd = E;
+  int ks = gate_logits_split(T, d, E);
+  if (ws_bytes < tc_gate_logits_ws(T, d, E) || !ws) ks = 1;
+  p.ksplit = ks;
+  if (ks > 1) {
+    p.D0 = ws;
+    p.d_gstride = static_cast<long long>(T) * E;
+  } else {
+    p.D0 = logits;
+    p.bias = bias;
+  }
   PFMOE_TRY(make_tmap(&p.tmA[0], x, d, T, 1, BK, BM, "x"));
   PFMOE_TRY(make_tmap(&p.tmB[0], wg, E, d, 1, 64, 64, "wg"));
-  const long long ub = static_cast<long long>((T + BM - 1) / BM) * ((E + p.bn - 1) / p.bn);
-  return launch<EPI_STORE_F32>(p, ub, "gate_logits", s);
+  const long long ub = static_cast<long long>((T + BM - 1) / BM) * ((E + p.bn - 1) / p.bn) * ks;
+  PFMOE_TRY((launch<EPI_STORE_F32, RG>(p, ub, "gate_logits", s)));
+  if (ks > 1)
+    PFMOE_TRY(launch_split_reduce(static_cast<const float*>(ws), ks, static_cast<long long>(T) * E, bias, E, logits, s));
+  return PFMOE_OK;
 }
 
-int tc_gate_wgrad(const void* x, const void* dz_bf16, int T, int d, int E, float* dwg, int32_t* err,
-                  cudaStream_t s) {
+int tc_gate_wgrad(const void* x, const void* dz_bf16, int T, int d, int E, float* dwg, void* ws, size_t ws_bytes,
+                  int32_t* err, cudaStream_t s) {
   Params p = base_params(err);
   p.mode = KG;
   p.b_major = 1;
   p.bn = round_bn(E);
   p.M = d;
   p.Nout = E;
-  p.G = 1;
   p.dense_len = T;
-  p.D0 = dwg; p.ldd = E; p.d_gstride = 0;
+  p.ldd = E;
+  int ks = gate_wgrad_split(T, d, E);
+  if (ws_bytes < tc_gate_wgrad_ws(T, d, E) || !ws) ks = 1;
+  const int nk = (T + BK - 1) / BK;
+  const int kbs = (nk + ks - 1) / ks;
+  p.kchunk = kbs * BK;
+  p.G = ks;
+  if (ks > 1) {
+    p.D0 = ws;
+    p.d_gstride = static_cast<long long>(d) * E;
+  } else {
+    p.D0 = dwg;
+    p.d_gstride = 0;
+  }
   PFMOE_TRY(make_tmap(&p.tmA[0], x, d, T, 1, 64, 64, "x^T"));
   PFMOE_TRY(make_tmap(&p.tmB[0], dz_bf16, E, T, 1, 64, 64, "dz"));
-  const long long ub = static_cast<long long>((d + BM - 1) / BM) * ((E + p.bn - 1) / p.bn);
-  return launch<EPI_STORE_F32>(p, ub, "gate_wgrad", s);
+  const long long ub = static_cast<long long>(ks) * ((d + BM - 1) / BM) * ((E + p.bn - 1) / p.bn);
+  PFMOE_TRY((launch<EPI_STORE_F32, KG>(p, ub, "gate_wgrad", s)));
+  if (ks > 1)
+    PFMOE_TRY(launch_split_reduce(static_cast<const float*>(ws), ks, static_cast<long long>(d) * E, nullptr, E, dwg, s));
+  return PFMOE_OK;
 }
 
 }  // namespace pfmoe

@@ -20,10 +20,13 @@ int tc_ffn_wgrad13(const void* x_pft, const void* dh1, const void* dh3, const in
                    void* dw1, void* dw3, int32_t* err, cudaStream_t s);
 int tc_ffn_wgrad2(const void* a, const void* dO, const int* seg, int N, int E, int d, int h, void* dw2,
                   int32_t* err, cudaStream_t s);
-int tc_gate_logits(const void* x, const void* wg, const float* bias, int T, int d, int E, float* logits,
-                   int32_t* err, cudaStream_t s);
-int tc_gate_wgrad(const void* x, const void* dz_bf16, int T, int d, int E, float* dwg, int32_t* err,
-                  cudaStream_t s);
+// Dense gate GEMMs split K over a workspace (sizes below; 0 = no split) and reduce deterministically.
+size_t tc_gate_logits_ws(int T, int d, int E);
+size_t tc_gate_wgrad_ws(int T, int d, int E);
+int tc_gate_logits(const void* x, const void* wg, const float* bias, int T, int d, int E, float* logits, void* ws,
+                   size_t ws_bytes, int32_t* err, cudaStream_t s);
+int tc_gate_wgrad(const void* x, const void* dz_bf16, int T, int d, int E, float* dwg, void* ws, size_t ws_bytes,
+                  int32_t* err, cudaStream_t s);
 
 // ---- FP32 SIMT grouped GEMM, gemm_simt.cu
 // D(m, n) = beta * D(m, n) + sum_k A(m, k) B(n, k) (+ bias[n]).

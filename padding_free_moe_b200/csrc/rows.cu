@@ -66,7 +66,8 @@ __global__ void __launch_bounds__(WARPS * 32) dispatch_kernel(const T* __restric
 }
 
 // y[t] = sum_j w[t, j] * O[pos[t, j]] in slot order, float32 accumulation, one rounding.
-template <typename T>
+// Each lane carries U 16-byte column chunks so that U*k row loads are in flight per warp.
+template <typename T, int U>
 __global__ void __launch_bounds__(WARPS * 32) combine_kernel(const T* __restrict__ O, const int32_t* __restrict__ pos,
                                                              const float* __restrict__ w, int Tn, int k, int d,
                                                              T* __restrict__ y, int32_t* err) {
@@ -78,24 +79,32 @@ __global__ void __launch_bounds__(WARPS * 32) combine_kernel(const T* __restrict
     int my_pos;
     if (!load_pos(pos, t, k, N, lane, my_pos, err)) continue;
     const float my_w = lane < k ? w[static_cast<long long>(t) * k + lane] : 0.f;
-    for (int base = 0; base < d; base += 32 * VN) {   // warp-uniform trip count
-      const int c0 = base + lane * VN;
-      const bool act = c0 < d;
-      float acc[VN];
+    for (int base = 0; base < d; base += 32 * VN * U) {   // warp-uniform trip count
+      float acc[U][VN];
 #pragma unroll
-      for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int i = 0; i < VN; ++i) acc[u][i] = 0.f;
 #pragma unroll 4
       for (int j = 0; j < k; ++j) {
         const long long p = __shfl_sync(0xffffffffu, my_pos, j);
         const float wj = __shfl_sync(0xffffffffu, my_w, j);
-        if (act) {
-          float o[VN];
-          load16(O + p * d + c0, o);
 #pragma unroll
-          for (int i = 0; i < VN; ++i) acc[i] = fmaf(wj, o[i], acc[i]);
+        for (int u = 0; u < U; ++u) {
+          const int c0 = base + (u * 32 + lane) * VN;
+          if (c0 < d) {
+            float o[VN];
+            load16(O + p * d + c0, o);
+#pragma unroll
+            for (int i = 0; i < VN; ++i) acc[u][i] = fmaf(wj, o[i], acc[u][i]);
+          }
         }
       }
-      if (act) store16(y + static_cast<long long>(t) * d + c0, acc);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c0 = base + (u * 32 + lane) * VN;
+        if (c0 < d) store16(y + static_cast<long long>(t) * d + c0, acc[u]);
+      }
     }
   }
 }
@@ -247,11 +256,11 @@ int launch_combine(const void* out, const int32_t* pos, const float* w, int T, i
   const int g = token_grid(T);
   if (dtype == PFMOE_BF16) {
     PFMOE_LAUNCH("combine", s,
-                 combine_kernel<__nv_bfloat16><<<g, WARPS * 32, 0, s>>>(
+                 combine_kernel<__nv_bfloat16, 2><<<g, WARPS * 32, 0, s>>>(
                      static_cast<const __nv_bfloat16*>(out), pos, w, T, k, d, static_cast<__nv_bfloat16*>(y), err));
   } else {
     PFMOE_LAUNCH("combine", s,
-                 combine_kernel<float><<<g, WARPS * 32, 0, s>>>(static_cast<const float*>(out), pos, w, T, k, d,
+                 combine_kernel<float, 2><<<g, WARPS * 32, 0, s>>>(static_cast<const float*>(out), pos, w, T, k, d,
                                                                 static_cast<float*>(y), err));
   }
   return PFMOE_OK;

@@ -2,52 +2,55 @@
 // built on it: the padding-free token buffer (X-MoE article §2.1.1 "PFT数据结构创新")
 // and the redundancy-bypassing-dispatch pilot plan (§2.2.1 "分层冗余消除算法").
 //
-// Sort = three launches:
-//   1. chunk histograms: one warp per CHUNK consecutive keys, counts[c][key];
+// Sort = three launches over chunks of W * 256 consecutive keys (one CTA of W warps
+// per chunk, W = 8 unless the per-warp counters would not fit in shared memory):
+//   1. chunk histograms counts[c][key];
 //   2. one-CTA scan in (key, chunk) order -> per-key totals, key offsets and
 //      every chunk's base row for every key (plus the grouped-GEMM tile prefix);
-//   3. scatter: one warp per chunk walks its keys in order, 32 at a time;
-//      lanes holding the same key find each other with __match_any_sync and
-//      take consecutive rows in lane order -> the sort is stable.
+//   3. scatter: warp w of a chunk owns keys [256w, 256w + 256) of it; the warps count
+//      their keys per key, take an exclusive prefix over warps, then walk their keys in
+//      order, 32 at a time; lanes holding the same key find each other with
+//      __match_any_sync and take consecutive rows in lane order -> the sort is stable.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace pfmoe {
 namespace {
 
-constexpr int CHUNK = 2048;
+constexpr int KEYS_PER_WARP = 256;   // 8 per lane
 constexpr int SCAN_THREADS = 1024;
 
+// Warps per chunk CTA: up to 8, while the scatter's per-warp counters (W * K ints) fit in 48 KB.
 inline int warps_per_block(int K) {
   int w = 12288 / (K > 0 ? K : 1);
   return w < 1 ? 1 : (w > 8 ? 8 : w);
 }
+inline long long chunk_keys(int K) { return static_cast<long long>(warps_per_block(K)) * KEYS_PER_WARP; }
 
 __device__ __forceinline__ long long dev_count(long long n, const int32_t* n_dev) {
   return n_dev ? static_cast<long long>(*n_dev) : n;
 }
 
+// One CTA per chunk: shared histogram of the chunk's keys -> counts[chunk][key].
 __global__ void chunk_hist_kernel(const int32_t* __restrict__ keys, long long n, const int32_t* n_dev, int K,
                                   int nchunks, int32_t* __restrict__ counts, int32_t* err) {
   extern __shared__ int32_t sh[];
-  const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk = blockIdx.x * (blockDim.x >> 5) + wib;
-  int32_t* h = sh + wib * K;
-  for (int i = lane; i < K; i += 32) h[i] = 0;
-  __syncwarp();
-  if (chunk >= nchunks) return;
+  const int chunk = blockIdx.x;
+  for (int i = threadIdx.x; i < K; i += blockDim.x) sh[i] = 0;
+  __syncthreads();
   const long long nn = dev_count(n, n_dev);
-  const long long b = static_cast<long long>(chunk) * CHUNK;
-  const long long e = min(b + CHUNK, nn);
+  const long long b = static_cast<long long>(chunk) * blockDim.x / 32 * KEYS_PER_WARP;
+  const long long e = min(b + static_cast<long long>(blockDim.x / 32) * KEYS_PER_WARP, nn);
   bool bad = false;
-  for (long long i = b + lane; i < e; i += 32) {
+  for (long long i = b + threadIdx.x; i < e; i += blockDim.x) {
     const int key = keys[i];
-    if (static_cast<unsigned>(key) < static_cast<unsigned>(K)) atomicAdd(&h[key], 1);
+    if (static_cast<unsigned>(key) < static_cast<unsigned>(K)) atomicAdd(&sh[key], 1);
     else bad = true;
   }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) dev_error(err, PFMOE_DEV_BAD_EXPERT_ID);
-  __syncwarp();
-  for (int i = lane; i < K; i += 32) counts[static_cast<long long>(chunk) * K + i] = h[i];
+  if (bad) dev_error(err, PFMOE_DEV_BAD_EXPERT_ID);
+  __syncthreads();
+  if (chunk < nchunks)
+    for (int i = threadIdx.x; i < K; i += blockDim.x) counts[static_cast<long long>(chunk) * K + i] = sh[i];
 }
 
 // Block-wide exclusive scan of one int per thread; returns the exclusive prefix, *total = block sum.
@@ -119,27 +122,53 @@ __global__ void __launch_bounds__(SCAN_THREADS) chunk_scan_kernel(const int32_t*
 template <class Sink>
 __global__ void chunk_scatter_kernel(const int32_t* __restrict__ keys, long long n, const int32_t* n_dev, int K,
                                      int nchunks, const int32_t* __restrict__ base, Sink sink) {
-  extern __shared__ int32_t sh[];
-  const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk = blockIdx.x * (blockDim.x >> 5) + wib;
-  if (chunk >= nchunks) return;
-  int32_t* ctr = sh + wib * K;
-  for (int i = lane; i < K; i += 32) ctr[i] = base[static_cast<long long>(chunk) * K + i];
-  __syncwarp();
+  extern __shared__ int32_t sh[];   // [warps][K]: per-warp counts, then per-warp first rows
+  const int nw = blockDim.x >> 5;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x;
+  for (int i = threadIdx.x; i < nw * K; i += blockDim.x) sh[i] = 0;
+  __syncthreads();
   const long long nn = dev_count(n, n_dev);
-  const long long b = static_cast<long long>(chunk) * CHUNK;
-  const long long e = min(b + CHUNK, nn);
-  for (long long i0 = b; i0 < e; i0 += 32) {
-    const long long i = i0 + lane;
-    const int key = i < e ? keys[i] : -1;
-    const bool ok = i < e && static_cast<unsigned>(key) < static_cast<unsigned>(K);
-    const unsigned peers = __match_any_sync(0xffffffffu, ok ? key : K + lane);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    const int cnt = ok ? ctr[key] : 0;
+  const long long b = (static_cast<long long>(chunk) * nw + w) * KEYS_PER_WARP;
+  int32_t* cnt = sh + w * K;
+  constexpr int IT = KEYS_PER_WARP / 32;
+  int key[IT];
+  unsigned peers[IT];
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const long long i = b + it * 32 + lane;
+    key[it] = i < nn ? keys[i] : -1;
+  }
+  // pass 1: per-warp counts (one shared update per distinct key per 32 keys)
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const bool ok = static_cast<unsigned>(key[it]) < static_cast<unsigned>(K);
+    peers[it] = __match_any_sync(0xffffffffu, ok ? key[it] : K + lane);
+    if (ok && (peers[it] & ((1u << lane) - 1u)) == 0) cnt[key[it]] += __popc(peers[it]);
     __syncwarp();
-    if (ok && rank == 0) ctr[key] = cnt + __popc(peers);
+  }
+  __syncthreads();
+  // exclusive prefix over the warps of this chunk, starting at the chunk's base row of each key
+  if (chunk < nchunks)
+    for (int k = threadIdx.x; k < K; k += blockDim.x) {
+      int run = base[static_cast<long long>(chunk) * K + k];
+      for (int w2 = 0; w2 < nw; ++w2) {
+        const int c = sh[w2 * K + k];
+        sh[w2 * K + k] = run;
+        run += c;
+      }
+    }
+  __syncthreads();
+  // pass 2: rows in key order within the warp
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const bool ok = static_cast<unsigned>(key[it]) < static_cast<unsigned>(K);
+    const int rank = __popc(peers[it] & ((1u << lane) - 1u));
+    const int c0 = ok ? cnt[key[it]] : 0;
     __syncwarp();
-    if (ok) sink(i, cnt + rank, key);
+    if (ok && rank == 0) cnt[key[it]] = c0 + __popc(peers[it]);
+    __syncwarp();
+    if (ok) sink(b + it * 32 + lane, c0 + rank, key[it]);
   }
 }
 
@@ -318,7 +347,7 @@ struct CsortWs {
 }  // namespace
 
 size_t csort_ws_bytes(long long n_max, int K) {
-  const long long C = (n_max + CHUNK - 1) / CHUNK;
+  const long long C = (n_max + chunk_keys(K) - 1) / chunk_keys(K);
   return static_cast<size_t>(2 * (C > 0 ? C : 1) * static_cast<long long>(K)) * sizeof(int32_t);
 }
 
@@ -326,14 +355,15 @@ int pft_build_impl(const int32_t* ids, const float* w, int T, int E, int k, int3
                    int32_t* token_ids, int32_t* expert_ids, float* cw, int32_t* pos, int32_t* tile_offsets,
                    void* ws, int32_t* err, cudaStream_t s) {
   const long long N = static_cast<long long>(T) * k;
-  const int C = static_cast<int>((N + CHUNK - 1) / CHUNK);
+  const int C = static_cast<int>((N + chunk_keys(E) - 1) / chunk_keys(E));
   int32_t* counts = static_cast<int32_t*>(ws);
   int32_t* base = counts + static_cast<long long>(C) * E;
   const int wpb = warps_per_block(E);
-  const int blocks = (C + wpb - 1) / wpb;
+  const int blocks = C;
   const size_t sm = static_cast<size_t>(wpb) * E * sizeof(int32_t);
   if (C > 0)
-    PFMOE_LAUNCH("pft_hist", s, chunk_hist_kernel<<<blocks, wpb * 32, sm, s>>>(ids, N, nullptr, E, C, counts, err));
+    PFMOE_LAUNCH("pft_hist", s,
+                 chunk_hist_kernel<<<blocks, wpb * 32, E * sizeof(int32_t), s>>>(ids, N, nullptr, E, C, counts, err));
   PFMOE_LAUNCH("pft_scan", s,
                chunk_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(counts, C, E, tpe, offsets, base, tile_offsets, 128));
   PftSink sink{w, k, pos, token_ids, expert_ids, cw};
@@ -366,7 +396,7 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
   int32_t* psorted = p; p += pmax;
   int32_t* rc_sorted = p; p += pmax;
   p += 64 - ((p - static_cast<int32_t*>(ws)) & 63);   // keep 256-byte alignment
-  const int C = static_cast<int>((pmax + CHUNK - 1) / CHUNK);
+  const int C = static_cast<int>((pmax + chunk_keys(n_nodes) - 1) / chunk_keys(n_nodes));
   int32_t* ccounts = p; p += static_cast<long long>(C > 0 ? C : 1) * n_nodes;
   int32_t* cbase = p;
 
@@ -375,11 +405,12 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
   PFMOE_LAUNCH("rbd_scan_tokens", s, rbd_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(ucount, dcount, T, pbase, counts));
   PFMOE_LAUNCH("rbd_emit", s, rbd_emit_kernel<<<g, 256, 0, s>>>(ids, T, k, E, epd, epn, pbase, pkey, ptoken, prc, err));
   const int wpb = warps_per_block(n_nodes);
-  const int blocks = (C + wpb - 1) / wpb;
+  const int blocks = C;
   const size_t sm = static_cast<size_t>(wpb) * n_nodes * sizeof(int32_t);
   if (C > 0) {
     PFMOE_LAUNCH("rbd_hist", s,
-                 chunk_hist_kernel<<<blocks, wpb * 32, sm, s>>>(pkey, pmax, counts, n_nodes, C, ccounts, err));
+                 chunk_hist_kernel<<<blocks, wpb * 32, n_nodes * sizeof(int32_t), s>>>(pkey, pmax, counts, n_nodes, C,
+                                                                                     ccounts, err));
   }
   PFMOE_LAUNCH("rbd_scan_nodes", s,
                chunk_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(ccounts, C, n_nodes, pilots_per_node, node_offsets,

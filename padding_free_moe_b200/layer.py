@@ -44,6 +44,8 @@ class PFTMoELayer:
         self.logits = e(T, E, dtype=f32)
         self.topk_ids = e(T, k, dtype=i32)
         self.topk_w = e(T, k, dtype=f32)
+        self.route_ws_bytes = L.moe_route_workspace_size(T, d, E, k, self.code)
+        self.route_ws = e(max(self.route_ws_bytes, 256), dtype=torch.uint8)
         self.tokens_per_expert = e(E, dtype=i32)
         self.expert_offsets = e(E + 1, dtype=i32)
         self.token_ids = e(max(N, 1), dtype=i32)
@@ -91,8 +93,8 @@ class PFTMoELayer:
     # ------------------------------------------------------------------ steps
     def route(self, x, wg, bias=None, stream=None):
         s = self.s
-        L.moe_route(x, wg, bias, s.T, s.d, s.E, s.k, self.code, self.logits, self.topk_ids, self.topk_w, self.err,
-                    stream)
+        L.moe_route(x, wg, bias, s.T, s.d, s.E, s.k, self.code, self.logits, self.topk_ids, self.topk_w,
+                    self.route_ws, self.route_ws_bytes, self.err, stream)
 
     def build_pft(self, stream=None):
         s = self.s

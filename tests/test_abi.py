@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
     for n in names:
         assert hasattr(lib, n), n
         assert n in L.SIGNATURES, f"binding lacks {n}"
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == 2
 
 
 FAKE = 1 << 20     # an aligned, never-dereferenced pointer value (validation fails before any use)
@@ -49,7 +49,7 @@ def test_route_argument_errors(lib):
                  w=FAKE)
         a.update(kw)
         return lib.moe_route(a["x"], a["wg"], a["bias"], a["T"], a["d"], a["E"], a["k"], a["dtype"], a["logits"],
-                             a["ids"], a["w"], None, None)
+                             a["ids"], a["w"], None, 0, None, None)
     assert call(k=9) == L.PFMOE_ERR_ARG                     # k > E
     assert b"k <= E" in lib.moe_last_error()
     assert call(k=0) == L.PFMOE_ERR_ARG
