@@ -877,6 +877,337 @@ static size_t smem_bytes(int bn, int stages, bool staged) {
   return smem_fixed(staged) + static_cast<size_t>(stages) * (A_BYTES + bn * BK * 2);
 }
 
+// ============================================================================
+// Two-SM variant for row-grouped problems (tcgen05 cta_group::2).
+//
+// A cluster of two CTAs on one TPC computes a 256-row x bn-column tile with one
+// M=256 MMA issued by the even CTA.  CTA v loads its own 128 rows of A and
+// columns [v*bn/2, (v+1)*bn/2) of B; the tensor cores read the other half of B
+// from the peer.  Per FLOP this moves 1.5x fewer operand bytes through L2 and
+// shared memory than two independent 128-row tiles.  Each CTA keeps its 128
+// accumulator rows in its own TMEM and runs the same epilogue as the one-SM
+// kernel.  A 256-row tile covers rows [256p, 256p+256) of one expert segment
+// (rows past the segment end are computed but never stored).  With N-split
+// (SwiGLU pairing) CTA 0 loads the W1 block and CTA 1 the W3 block.
+//
+// Synchronisation: both CTAs' TMA loads complete on the even CTA's full[s]
+// barrier; the MMA's commits arrive on both CTAs' empty[s] / acc_full[b]
+// (multicast commit); both CTAs' epilogues arrive on the even CTA's acc_empty[b].
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ uint32_t mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok;
+}
+__device__ __forceinline__ bool wait_bar2(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* err,
+                                          bool honour_abort = true) {
+  for (int i = 0; i < 128; ++i)
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (honour_abort && *abort_flag) return false;
+    if (globaltimer() - t0 > kTimeoutNs) {
+      *abort_flag = 1;
+      dev_error(err, PFMOE_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* tm, uint32_t bar_cluster, int c0,
+                                                 int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc2(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_mma2(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Commit arriving on the barrier at the same offset in both CTAs of the pair.
+__device__ __forceinline__ void tc_commit2_both(uint32_t bar) {
+  const uint16_t mask = 3;
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                   bar),
+               "h"(mask)
+               : "memory");
+}
+
+struct PairTile {
+  int g, row0, rows, n0, nk, kb0, split;
+};
+
+// Pair tiles of a row-grouped problem: expert g has ceil(n_g / 256) of them (prefix in pair_off).
+__device__ __forceinline__ int total_pair_tiles(const Params& p, const int* pair_off) {
+  const int ns = n_step(p);
+  const int NT = (p.Nout + ns - 1) / ns;
+  const int np = p.tiles ? pair_off[p.G] : (p.dense_len + 2 * BM - 1) / (2 * BM) * p.ksplit;
+  return np * NT;
+}
+
+__device__ __forceinline__ PairTile decode_pair(const Params& p, const int* pair_off, int t, uint32_t rank) {
+  PairTile tl;
+  const int ns = n_step(p);
+  const int NT = (p.Nout + ns - 1) / ns;
+  int g = 0, tbase = 0, npg, s0, s1, split = 0;
+  if (p.tiles) {
+    int lo = 0, hi = p.G - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pair_off[mid] * NT <= t) lo = mid; else hi = mid - 1;
+    }
+    g = lo;
+    tbase = pair_off[g] * NT;
+    npg = pair_off[g + 1] - pair_off[g];
+    s0 = p.seg[g];
+    s1 = p.seg[g + 1];
+  } else {
+    npg = (p.dense_len + 2 * BM - 1) / (2 * BM);
+    s0 = 0;
+    s1 = p.dense_len;
+    split = t / (npg * NT);
+    tbase = split * npg * NT;
+  }
+  const int local = t - tbase;
+  const int n_idx = local / npg;
+  const int pr = local - n_idx * npg;
+  tl.g = g;
+  tl.row0 = s0 + pr * 2 * BM + static_cast<int>(rank) * BM;
+  tl.rows = max(0, min(BM, s1 - tl.row0));
+  tl.n0 = n_idx * ns;
+  const int nk_all = p.k0_blocks + p.k1_blocks;
+  const int kbs = (nk_all + p.ksplit - 1) / p.ksplit;
+  tl.split = split;
+  tl.kb0 = split * kbs;
+  tl.nk = max(0, min(kbs, nk_all - tl.kb0));
+  return tl;
+}
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    grouped_gemm_2sm_kernel(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages;
+  const int bh = p.bn / 2;                         // B columns held by this CTA
+  const uint32_t b_bytes = static_cast<uint32_t>(bh) * BK * 2;
+  const uint32_t stage_bytes = A_BYTES + b_bytes;
+  int* pair_off = reinterpret_cast<int*>(smem + S * stage_bytes);
+  const int poff_ints = p.tiles ? ((p.G + 1 + 63) & ~63) : 0;
+  uint8_t* bar_area = reinterpret_cast<uint8_t*>(pair_off + poff_ints);
+  uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
+  uint64_t* empty = full + MAX_STAGES;
+  uint64_t* acc_full = empty + MAX_STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const uint32_t tmem_cols = p.bn * 2 <= 128 ? 128 : (p.bn * 2 <= 256 ? 256 : 512);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&acc_full[b]), 1);
+      mbar_init(smem_u32(&acc_empty[b]), 2 * 4 * 32);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  // Prefix over experts of ceil(n_g / 256) pair tiles (from the 128-row tile prefix).
+  if (p.tiles && warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < p.G; base += 32) {
+      const int e = base + lane;
+      const int np = e < p.G ? (p.tiles[e + 1] - p.tiles[e] + 1) / 2 : 0;
+      int x = np;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (e < p.G) pair_off[e] = carry + x - np;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) pair_off[p.G] = carry;
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&p.tmA[0]);
+    prefetch_tmap(&p.tmB[0]);
+  }
+  if (warp == 1) {
+    tmem_alloc2(smem_u32(tmem_slot), tmem_cols);
+    tmem_relinquish2();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int ntiles = total_pair_tiles(p, pair_off);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      uint32_t pending = 0, pend_parity = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = pair; t < ntiles && ok; t += npairs) {
+        const PairTile tl = decode_pair(p, pair_off, t, rank);
+        for (int kb = 0; kb < tl.nk; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!wait_bar2(smem_u32(&empty[s]), ph ^ 1, abort_flag, p.err)) { ok = false; break; }
+          const uint32_t fb_local = smem_u32(&full[s]);
+          if (leader) mbar_expect_tx(fb_local, 2 * stage_bytes);
+          const uint32_t fb = mapa_shared(fb_local, 0);
+          const uint32_t sa = smem_u32(smem + s * stage_bytes);
+          const uint32_t sb = sa + A_BYTES;
+          const int kbg = tl.kb0 + kb;
+          const int src = kbg < p.k0_blocks ? 0 : 1;
+          const int kk = (src == 0 ? kbg : kbg - p.k0_blocks) * BK;
+          tma_load_3d_pair(sa, &p.tmA[src], fb, kk, tl.row0, 0);
+          const CUtensorMap* tb = &p.tmB[p.nsplit ? static_cast<int>(rank) : src];
+          const int ncol = p.nsplit ? tl.n0 : tl.n0 + static_cast<int>(rank) * bh;
+          if (p.b_major == 0) {
+            tma_load_3d_pair(sb, tb, fb, kk, ncol, tl.g);
+          } else {
+            for (int j = 0; j < bh / 64; ++j) tma_load_3d_pair(sb + j * BOX_BYTES, tb, fb, ncol + 64 * j, kk, tl.g);
+          }
+          pending |= 1u << s;
+          pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
+        }
+      }
+      // Drain: a stage's empty barrier completes only after the MMA consumed it, so its loads landed.
+      for (int s = 0; s < S; ++s)
+        if (pending & (1u << s))
+          wait_bar2(smem_u32(&empty[s]), (pend_parity >> s) & 1, abort_flag, p.err, false);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (leader) {
+      const uint32_t idesc = idesc_bf16(2 * BM, p.bn, 0, p.b_major);
+      const uint32_t b_lbo = p.b_major ? BOX_BYTES : 16;
+      const uint32_t b_step = p.b_major ? 2048 : 32;
+      int it = 0, tcount = 0;
+      bool ok = true;
+      for (int t = pair; t < ntiles && ok; t += npairs, ++tcount) {
+        const PairTile tl = decode_pair(p, pair_off, t, rank);
+        const int buf = tcount & 1;
+        const uint32_t aph = (tcount >> 1) & 1;
+        ok = __all_sync(0xffffffffu, wait_bar2(smem_u32(&acc_empty[buf]), aph ^ 1, abort_flag, p.err));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tmem_d = tmem_base + buf * p.bn;
+        for (int kb = 0; kb < tl.nk; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          ok = __all_sync(0xffffffffu, wait_bar2(smem_u32(&full[s]), ph, abort_flag, p.err));
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * stage_bytes);
+          const uint32_t sb = sa + A_BYTES;
+          if (lane == 0) {
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = sdesc(sa + kk * 32, 16, 1024);
+              const uint64_t bd = sdesc(sb + kk * b_step, b_lbo, 1024);
+              tc_mma2(tmem_d, ad, bd, idesc, (kb | kk) != 0);
+            }
+            tc_commit2_both(smem_u32(&empty[s]));
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        if (lane == 0) tc_commit2_both(smem_u32(&acc_full[buf]));
+        __syncwarp();
+      }
+      if (lane == 0) {
+        tc_commit2_both(smem_u32(drain));
+        wait_bar2(smem_u32(drain), 0, abort_flag, p.err, false);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
+    const uint32_t acc_empty_leader1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
+    int tcount = 0;
+    for (int t = pair; t < ntiles; t += npairs, ++tcount) {
+      const PairTile pt = decode_pair(p, pair_off, t, rank);
+      const int buf = tcount & 1;
+      const uint32_t aph = (tcount >> 1) & 1;
+      if (!__all_sync(0xffffffffu, wait_bar2(smem_u32(&acc_full[buf]), aph, abort_flag, p.err))) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * p.bn;
+      Tile tl;
+      tl.g = pt.g; tl.row0 = pt.row0; tl.rows = pt.rows; tl.n0 = pt.n0; tl.nk = pt.nk;
+      tl.krow0 = 0; tl.kvalid = BK; tl.kb0 = pt.kb0; tl.split = pt.split;
+      epilogue_tile_direct<EPI>(p, tl, tacc, q * 32 + lane);
+      tc_fence_before();
+      mbar_arrive_cluster(buf ? acc_empty_leader1 : acc_empty_leader0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc2(tmem_base, tmem_cols);
+  }
+}
+
 template <int EPI, int MODE>
 static int launch(Params& p, long long tile_upper_bound, const char* name, cudaStream_t stream) {
   p.mode = MODE;
@@ -898,6 +1229,51 @@ static int launch(Params& p, long long tile_upper_bound, const char* name, cudaS
                (grouped_gemm_kernel<EPI, MODE><<<static_cast<int>(grid), THREADS, smem, stream>>>(p)));
   return PFMOE_OK;
 }
+
+
+// Two-SM launcher for row-grouped problems.
+static int max_pairs() {
+  static int cached = -1;
+  if (cached < 0) {
+    int n = num_sms() / 2;
+    cached = n > 0 ? n : 1;
+  }
+  return cached;
+}
+
+template <int EPI>
+static int launch2(Params& p, long long pair_tile_upper_bound, const char* name, cudaStream_t stream) {
+  p.mode = RG;
+  const int stage = A_BYTES + (p.bn / 2) * BK * 2;
+  const int poff = p.tiles ? ((p.G + 1 + 63) & ~63) * 4 : 0;
+  const int fixed = 1024 + 256 + poff;
+  int st = (SMEM_LIMIT - fixed) / stage;
+  p.stages = st > MAX_STAGES ? MAX_STAGES : st;
+  const size_t smem = fixed + static_cast<size_t>(p.stages) * stage;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(grouped_gemm_2sm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(227 * 1024)) != cudaSuccess)
+      return fail(PFMOE_ERR_CUDA, std::string("cudaFuncSetAttribute failed: ") +
+                                      cudaGetErrorString(cudaGetLastError()));
+    attr_done = true;
+  }
+  if (pair_tile_upper_bound <= 0) return PFMOE_OK;
+  long long pairs = max_pairs();
+  if (pair_tile_upper_bound < pairs) pairs = pair_tile_upper_bound;
+  PFMOE_LAUNCH(name, stream,
+               (grouped_gemm_2sm_kernel<EPI><<<static_cast<int>(2 * pairs), THREADS, smem, stream>>>(p)));
+  return PFMOE_OK;
+}
+
+// Pair-tile upper bound: sum_e ceil(n_e / 256) <= N / 256 + E.
+static long long rg_pairs_ub(int N, int E, int Nout, int nstep) {
+  return (static_cast<long long>(N) / (2 * BM) + E + 1) * ((Nout + nstep - 1) / nstep);
+}
+
+// The two-SM kernel pays for half-empty pair tiles on small expert segments; use it when the
+// average segment holds at least one full 256-row pair tile.
+static bool use_pairs(int N, int E) { return N >= 2 * BM * E; }
 
 static Params base_params(int32_t* err) {
   Params p;
@@ -973,6 +1349,7 @@ int tc_ffn_gemm1(const void* x_pft, const int* seg, const int* tiles, int N, int
   PFMOE_TRY(make_tmap(&p.tmA[0], x_pft, d, N, 1, BK, BM, "x_pft"));
   PFMOE_TRY(make_tmap(&p.tmB[0], w1, h, d, E, 64, 64, "w1"));
   PFMOE_TRY(make_tmap(&p.tmB[1], w3, h, d, E, 64, 64, "w3"));
+  if (use_pairs(N, E)) return launch2<EPI_SWIGLU_FWD>(p, rg_pairs_ub(N, E, h, p.bn / 2), "ffn_gemm1_swiglu", s);
   return launch<EPI_SWIGLU_FWD, RG>(p, rg_tiles_ub(N, E, h, p.bn / 2), "ffn_gemm1_swiglu", s);
 }
 
@@ -988,6 +1365,7 @@ int tc_ffn_gemm2(const void* a, const int* seg, const int* tiles, int N, int E, 
   p.D0 = out; p.ldd = d;
   PFMOE_TRY(make_tmap(&p.tmA[0], a, h, N, 1, BK, BM, "a"));
   PFMOE_TRY(make_tmap(&p.tmB[0], w2, d, h, E, 64, 64, "w2"));
+  if (use_pairs(N, E)) return launch2<EPI_STORE_BF16>(p, rg_pairs_ub(N, E, d, p.bn), "ffn_gemm2", s);
   return launch<EPI_STORE_BF16, RG>(p, rg_tiles_ub(N, E, d, p.bn), "ffn_gemm2", s);
 }
 
@@ -1001,8 +1379,11 @@ int tc_ffn_dgrad_act(const void* dO, const int* seg, const int* tiles, int N, in
   p.k0_blocks = (d + BK - 1) / BK;
   p.seg = seg; p.tiles = tiles; p.G = E;
   p.X0 = h1; p.X1 = h3; p.D0 = dh1; p.D1 = dh3; p.ldd = h;
+  const bool pairs = use_pairs(N, E);
+  const uint32_t brows = pairs ? p.bn / 2 : p.bn;   // B rows loaded per CTA
   PFMOE_TRY(make_tmap(&p.tmA[0], dO, d, N, 1, BK, BM, "dO"));
-  PFMOE_TRY(make_tmap(&p.tmB[0], w2, d, h, E, BK, p.bn, "w2^T"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], w2, d, h, E, BK, brows, "w2^T"));
+  if (pairs) return launch2<EPI_SWIGLU_BWD>(p, rg_pairs_ub(N, E, h, p.bn), "ffn_dgrad_act_swiglu_bwd", s);
   return launch<EPI_SWIGLU_BWD, RG>(p, rg_tiles_ub(N, E, h, p.bn), "ffn_dgrad_act_swiglu_bwd", s);
 }
 
@@ -1017,10 +1398,13 @@ int tc_ffn_dgrad_x(const void* dh1, const void* dh3, const int* seg, const int* 
   p.k1_blocks = (h + BK - 1) / BK;
   p.seg = seg; p.tiles = tiles; p.G = E;
   p.D0 = dx_pft; p.ldd = d;
+  const bool pairs = use_pairs(N, E);
+  const uint32_t brows = pairs ? p.bn / 2 : p.bn;   // B rows loaded per CTA
   PFMOE_TRY(make_tmap(&p.tmA[0], dh1, h, N, 1, BK, BM, "dh1"));
   PFMOE_TRY(make_tmap(&p.tmA[1], dh3, h, N, 1, BK, BM, "dh3"));
-  PFMOE_TRY(make_tmap(&p.tmB[0], w1, h, d, E, BK, p.bn, "w1^T"));
-  PFMOE_TRY(make_tmap(&p.tmB[1], w3, h, d, E, BK, p.bn, "w3^T"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], w1, h, d, E, BK, brows, "w1^T"));
+  PFMOE_TRY(make_tmap(&p.tmB[1], w3, h, d, E, BK, brows, "w3^T"));
+  if (pairs) return launch2<EPI_STORE_BF16>(p, rg_pairs_ub(N, E, d, p.bn), "ffn_dgrad_x", s);
   return launch<EPI_STORE_BF16, RG>(p, rg_tiles_ub(N, E, d, p.bn), "ffn_dgrad_x", s);
 }
 

@@ -11,7 +11,7 @@ from workloads import get_config, make_inputs
 from tests.parity import LOGIT_TOL, TOL, check_index_parity, f64, i64, make_layer, rel_err, run_step
 
 SMALL = ["small_bf16", "small_ragged_bf16", "small_skew_bf16", "small_kE_bf16", "small_f32", "one_token_bf16",
-         "tiny_fp32"]
+         "tiny_fp32", "small_pairs_bf16"]
 
 
 @pytest.mark.gpu

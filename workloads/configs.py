@@ -79,6 +79,11 @@ SMALL = {
                              rbd_epd=3, rbd_dpn=1),
     "one_token_bf16": LayerConfig("one_token_bf16", T=1, d=64, E=8, h=64, k=2, dtype="bf16",
                                   rbd_epd=2, rbd_dpn=2),
+    # >= 256 rows per expert on average: exercises the two-SM (256-row pair tile) GEMMs,
+    # with ragged segment ends, pair tiles whose second half is empty, and d, h that are
+    # not multiples of the N tile.
+    "small_pairs_bf16": LayerConfig("small_pairs_bf16", T=1100, d=320, E=8, h=136, k=2, dtype="bf16",
+                                    rbd_epd=2, rbd_dpn=2),
 }
 
 
