@@ -282,6 +282,10 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
   return tl;
 }
 
+// Sigmoid for the BF16 epilogues: fast exponential and division (relative error ~1e-6,
+// far below the 2^-9 rounding of the BF16 results they feed).
+__device__ __forceinline__ float sigmoid_fast(float u) { return __fdividef(1.0f, 1.0f + __expf(-u)); }
+
 // ------------------------------------------------------------- direct epilogue
 // Row-grouped tiles: each thread stores its own row straight from registers (16-byte
 // vectors).  These tiles have long K loops, so the epilogue hides behind the next
@@ -333,7 +337,7 @@ __device__ __forceinline__ void epilogue_tile_direct(const Params& p, const Tile
       tmem_ld32(tacc + c, h1);
       tmem_ld32(tacc + half + c, h3);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) a[i] = silu_f(h1[i]) * h3[i];
+      for (int i = 0; i < 32; ++i) a[i] = h1[i] * sigmoid_fast(h1[i]) * h3[i];
       if (row_ok) {
         const long long off = grow * p.ldd + col;
         store_row_chunk(H1 + off, h1, p.Nout - col);
@@ -368,7 +372,7 @@ __device__ __forceinline__ void epilogue_tile_direct(const Params& p, const Tile
         }
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float s = 1.0f / (1.0f + expf(-h1[i]));
+          const float s = sigmoid_fast(h1[i]);
           o1[i] = da[i] * h3[i] * s * (1.0f + h1[i] * (1.0f - s));
           o3[i] = da[i] * h1[i] * s;
         }
@@ -582,7 +586,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, u
       emit(stg, lane, h1, H1 + off, p.ldd, rows_valid, p.Nout - col);
       emit(stg, lane, h3, H3 + off, p.ldd, rows_valid, p.Nout - col);
 #pragma unroll
-      for (int i = 0; i < 64; ++i) h1[i] = silu_f(h1[i]) * h3[i];
+      for (int i = 0; i < 64; ++i) h1[i] = h1[i] * sigmoid_fast(h1[i]) * h3[i];
       emit(stg, lane, h1, A + off, p.ldd, rows_valid, p.Nout - col);
     }
   } else if constexpr (EPI == EPI_SWIGLU_BWD) {
@@ -609,7 +613,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, u
       unstage_row_bf16(stg, lane, h3);
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
-        const float s = 1.0f / (1.0f + expf(-h1[i]));
+        const float s = sigmoid_fast(h1[i]);
         const float d1 = da[i] * h3[i] * s * (1.0f + h1[i] * (1.0f - s));
         h1[i] = da[i] * h1[i] * s;
         da[i] = d1;
@@ -1021,6 +1025,10 @@ __device__ __forceinline__ PairTile decode_pair(const Params& p, const int* pair
   return tl;
 }
 
+// Epilogue of the two-SM kernel: staged through shared memory (full-line stores, coalesced
+// reads of the SwiGLU-backward inputs) or direct per-row stores.
+constexpr bool kStaged2sm = true;
+
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     grouped_gemm_2sm_kernel(const __grid_constant__ Params p) {
@@ -1030,7 +1038,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int bh = p.bn / 2;                         // B columns held by this CTA
   const uint32_t b_bytes = static_cast<uint32_t>(bh) * BK * 2;
   const uint32_t stage_bytes = A_BYTES + b_bytes;
-  int* pair_off = reinterpret_cast<int*>(smem + S * stage_bytes);
+  uint8_t* stage_area = smem + S * stage_bytes;
+  int* pair_off = reinterpret_cast<int*>(stage_area + (kStaged2sm ? 4 * STAGE_BYTES_PER_WARP : 0));
   const int poff_ints = p.tiles ? ((p.G + 1 + 63) & ~63) : 0;
   uint8_t* bar_area = reinterpret_cast<uint8_t*>(pair_off + poff_ints);
   uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
@@ -1193,7 +1202,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       Tile tl;
       tl.g = pt.g; tl.row0 = pt.row0; tl.rows = pt.rows; tl.n0 = pt.n0; tl.nk = pt.nk;
       tl.krow0 = 0; tl.kvalid = BK; tl.kb0 = pt.kb0; tl.split = pt.split;
-      epilogue_tile_direct<EPI>(p, tl, tacc, q * 32 + lane);
+      if constexpr (kStaged2sm)
+        epilogue_tile<EPI>(p, tl, tacc, q, lane, smem_u32(stage_area + (warp - 2) * STAGE_BYTES_PER_WARP));
+      else
+        epilogue_tile_direct<EPI>(p, tl, tacc, q * 32 + lane);
       tc_fence_before();
       mbar_arrive_cluster(buf ? acc_empty_leader1 : acc_empty_leader0);
     }
@@ -1246,7 +1258,7 @@ static int launch2(Params& p, long long pair_tile_upper_bound, const char* name,
   p.mode = RG;
   const int stage = A_BYTES + (p.bn / 2) * BK * 2;
   const int poff = p.tiles ? ((p.G + 1 + 63) & ~63) * 4 : 0;
-  const int fixed = 1024 + 256 + poff;
+  const int fixed = 1024 + 256 + poff + (kStaged2sm ? 4 * STAGE_BYTES_PER_WARP : 0);
   int st = (SMEM_LIMIT - fixed) / stage;
   p.stages = st > MAX_STAGES ? MAX_STAGES : st;
   const size_t smem = fixed + static_cast<size_t>(p.stages) * stage;
