@@ -45,6 +45,8 @@ enum Epi { EPI_STORE_BF16 = 0, EPI_STORE_F32 = 1, EPI_SWIGLU_FWD = 2, EPI_SWIGLU
 struct Params {
   CUtensorMap tmA[2];
   CUtensorMap tmB[2];
+  CUtensorMap tmD[3];  // output maps for TMA stores from the staged epilogue (box 128 B x 32 rows)
+  int tma_store;       // 1: tmD[] are valid
   int mode;
   int b_major;       // RG: 0 = K-major B (weights [G, N, K]), 1 = MN-major B (weights [G, K, N]); KG: 1
   int bn;            // MMA N: multiple of 64, <= 256
@@ -413,7 +415,8 @@ __device__ __forceinline__ void epilogue_tile_direct(const Params& p, const Tile
 // copied to global memory four rows per instruction, eight lanes per 128-byte row
 // segment.  Every global store is then part of a full 128-byte line.  Used for
 // K-grouped (weight-gradient) tiles, whose short K loops leave the epilogue exposed.
-constexpr int STAGE_BYTES_PER_WARP = 32 * 128;
+constexpr int STAGE_BYTES_PER_WARP = 32 * 128;   // one 32-row x 128-byte slab
+constexpr int STAGE_BUFS = 2;                     // per warp: ping-pong so a TMA store overlaps the next slab
 
 __device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t* r) {
   asm volatile(
@@ -512,23 +515,61 @@ __device__ __forceinline__ void copy_in(uint32_t stg, int lane, const char* base
   }
 }
 
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* tm, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tm)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
+// Per-warp staging state: two 4 KB slabs used alternately.
+struct Stager {
+  uint32_t base;
+  int seq;
+};
+
+// Stage one 32-row x 128-byte slab and write it out: a full slab goes out as one TMA store
+// (the staging layout is the TMA 128-byte swizzle; the store clips at the tensor bounds);
+// a slab with missing rows goes out with masked vector stores.  One bulk group is committed
+// per slab, so "at most one group pending" means the slab about to be reused is free.
 template <typename T>
-__device__ __forceinline__ void emit(uint32_t stg, int lane, const float* v, T* dst_row0, long long ldd,
-                                     int rows_valid, int cols_valid) {
+__device__ __forceinline__ void emit(Stager& st, int lane, const float* v, const CUtensorMap* tm, int c0, int c1,
+                                     int c2, T* dst_row0, long long ldd, int rows_valid, int cols_valid) {
+  const uint32_t buf = st.base + (st.seq & 1) * STAGE_BYTES_PER_WARP;
+  ++st.seq;
+  if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
   __syncwarp();
-  stage_row<T>(stg, lane, v);
+  stage_row<T>(buf, lane, v);
+  if (tm && rows_valid == 32) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) tma_store_3d(tm, buf, c0, c1, c2);
+  } else {
+    __syncwarp();
+    copy_out(buf, lane, reinterpret_cast<char*>(dst_row0), ldd * static_cast<long long>(sizeof(T)), rows_valid,
+             min(128, cols_valid * static_cast<int>(sizeof(T))));
+  }
+  if (lane == 0) asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until every TMA store this warp issued has written global memory.
+__device__ __forceinline__ void emit_drain(int lane) {
+  if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   __syncwarp();
-  copy_out(stg, lane, reinterpret_cast<char*>(dst_row0), ldd * static_cast<long long>(sizeof(T)), rows_valid,
-           min(128, cols_valid * static_cast<int>(sizeof(T))));
+}
+
+__device__ __forceinline__ const CUtensorMap* tmd(const Params& p, int i) {
+  return p.tma_store ? &p.tmD[i] : nullptr;
 }
 
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, uint32_t tacc, int q, int lane,
-                                              uint32_t stg) {
+                                              Stager& stg) {
   const int slab0 = q * 32;
   const int rows_valid = max(0, min(32, tl.rows - slab0));
   const long long grow0 = static_cast<long long>(tl.row0) + slab0;
   const bool zero = tl.nk == 0;
+  const int tz = p.mode == KG ? tl.g : 0;   // third output coordinate: expert / split part
   if constexpr (EPI == EPI_STORE_BF16 || EPI == EPI_SPLIT_BF16) {
     const int nparts = EPI == EPI_SPLIT_BF16 ? 2 : 1;
     const int width = EPI == EPI_SPLIT_BF16 ? p.bn / 2 : p.bn;
@@ -544,7 +585,8 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, u
 #pragma unroll
           for (int i = 0; i < 64; ++i) v[i] = 0.f;
         }
-        emit(stg, lane, v, D + grow0 * p.ldd + col, p.ldd, rows_valid, p.Nout - col);
+        emit(stg, lane, v, tmd(p, part), col, static_cast<int>(grow0), tz, D + grow0 * p.ldd + col, p.ldd, rows_valid,
+             p.Nout - col);
       }
     }
   } else if constexpr (EPI == EPI_STORE_F32) {
@@ -568,7 +610,8 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, u
         for (int i = 0; i < 32; ++i)
           if (col + i < p.Nout) v[i] += p.bias[col + i];
       }
-      emit(stg, lane, v, D + grow0 * p.ldd + col, p.ldd, rows_valid, p.Nout - col);
+      emit(stg, lane, v, tmd(p, 0), col, static_cast<int>(grow0), tz, D + grow0 * p.ldd + col, p.ldd, rows_valid,
+           p.Nout - col);
     }
   } else if constexpr (EPI == EPI_SWIGLU_FWD) {
     // D columns [0, bn/2) = H1 tile, [bn/2, bn) = H3 tile for the same output columns.
@@ -583,11 +626,11 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, u
       float h1[64], h3[64];
       tmem_ld64(tacc + c, h1);
       tmem_ld64(tacc + half + c, h3);
-      emit(stg, lane, h1, H1 + off, p.ldd, rows_valid, p.Nout - col);
-      emit(stg, lane, h3, H3 + off, p.ldd, rows_valid, p.Nout - col);
+      emit(stg, lane, h1, tmd(p, 0), col, static_cast<int>(grow0), 0, H1 + off, p.ldd, rows_valid, p.Nout - col);
+      emit(stg, lane, h3, tmd(p, 1), col, static_cast<int>(grow0), 0, H3 + off, p.ldd, rows_valid, p.Nout - col);
 #pragma unroll
       for (int i = 0; i < 64; ++i) h1[i] = h1[i] * sigmoid_fast(h1[i]) * h3[i];
-      emit(stg, lane, h1, A + off, p.ldd, rows_valid, p.Nout - col);
+      emit(stg, lane, h1, tmd(p, 2), col, static_cast<int>(grow0), 0, A + off, p.ldd, rows_valid, p.Nout - col);
     }
   } else if constexpr (EPI == EPI_SWIGLU_BWD) {
     // Accumulator = dA.  dH1 = dA * H3 * s * (1 + H1 (1 - s)), dH3 = dA * SiLU(H1), s = sigmoid(H1).
@@ -603,14 +646,18 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, u
       const int bytes_valid = min(128, (p.Nout - col) * 2);
       float da[64], h1[64], h3[64];
       tmem_ld64(tacc + c, da);
+      // Read H1 / H3 through the slab the next emit will use (no store of ours is pending on it
+      // once at most one bulk group is outstanding).
+      const uint32_t ibuf = stg.base + (stg.seq & 1) * STAGE_BYTES_PER_WARP;
+      if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
       __syncwarp();
-      copy_in(stg, lane, H1 + off * 2, stride, rows_valid, bytes_valid);
+      copy_in(ibuf, lane, H1 + off * 2, stride, rows_valid, bytes_valid);
       __syncwarp();
-      unstage_row_bf16(stg, lane, h1);
+      unstage_row_bf16(ibuf, lane, h1);
       __syncwarp();
-      copy_in(stg, lane, H3 + off * 2, stride, rows_valid, bytes_valid);
+      copy_in(ibuf, lane, H3 + off * 2, stride, rows_valid, bytes_valid);
       __syncwarp();
-      unstage_row_bf16(stg, lane, h3);
+      unstage_row_bf16(ibuf, lane, h3);
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
         const float s = sigmoid_fast(h1[i]);
@@ -618,8 +665,8 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, u
         h1[i] = da[i] * h1[i] * s;
         da[i] = d1;
       }
-      emit(stg, lane, da, dH1 + off, p.ldd, rows_valid, p.Nout - col);
-      emit(stg, lane, h1, dH3 + off, p.ldd, rows_valid, p.Nout - col);
+      emit(stg, lane, da, tmd(p, 0), col, static_cast<int>(grow0), 0, dH1 + off, p.ldd, rows_valid, p.Nout - col);
+      emit(stg, lane, h1, tmd(p, 1), col, static_cast<int>(grow0), 0, dH3 + off, p.ldd, rows_valid, p.Nout - col);
     }
   }
 }
@@ -633,7 +680,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   const uint32_t b_bytes = static_cast<uint32_t>(p.bn) * BK * 2;
   const uint32_t stage_bytes = A_BYTES + b_bytes;
   uint8_t* stage_area = smem + S * stage_bytes;                       // epilogue staging (K-grouped only)
-  uint8_t* bar_area = stage_area + (MODE == KG ? 4 * STAGE_BYTES_PER_WARP : 0);
+  uint8_t* bar_area = stage_area + (MODE == KG ? 4 * STAGE_BUFS * STAGE_BYTES_PER_WARP : 0);
   uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
   uint64_t* empty = full + MAX_STAGES;
   uint64_t* acc_full = empty + MAX_STAGES;
@@ -805,7 +852,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   } else {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;           // TMEM lane quarter this warp may access: rows 32q .. 32q+31
-    const uint32_t stg = smem_u32(stage_area + (warp - 2) * STAGE_BYTES_PER_WARP);
+    Stager stg{smem_u32(stage_area + (warp - 2) * STAGE_BUFS * STAGE_BYTES_PER_WARP), 0};
     int tcount = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
       const Tile tl = decode<MODE>(p, t);
@@ -819,6 +866,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       tc_fence_before();
       mbar_arrive(smem_u32(&acc_empty[buf]));
     }
+    emit_drain(lane);
   }
 
   tc_fence_before();
@@ -845,21 +893,34 @@ static int get_encode() {
   return PFMOE_OK;
 }
 
-// 3-D BF16 tensor map over a row-major tensor [d2][d1][d0] with a box of b0 x b1 x 1, 128-byte swizzle.
-static int make_tmap(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
-                     uint32_t b1, const char* what) {
+// 3-D tensor map over a row-major tensor [d2][d1][d0] (BF16 or FP32) with a box of
+// b0 x b1 x 1 elements and 128-byte swizzle (b0 * element size must be 128 bytes or less).
+static int make_tmap_t(CUtensorMap* m, const void* ptr, bool f32, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+                       uint32_t b1, const char* what) {
   PFMOE_TRY(get_encode());
+  const uint64_t es = f32 ? 4 : 2;
   cuuint64_t dims[3] = {d0, d1, d2};
-  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint64_t strides[2] = {d0 * es, d0 * d1 * es};
   cuuint32_t box[3] = {b0, b1, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = g_encode(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                        const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(PFMOE_ERR_CUDA, std::string("cuTensorMapEncodeTiled failed for ") + what + " (CUresult " +
                                     std::to_string(static_cast<int>(r)) + ")");
   return PFMOE_OK;
+}
+
+static int make_tmap(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+                     uint32_t b1, const char* what) {
+  return make_tmap_t(m, ptr, false, d0, d1, d2, b0, b1, what);
+}
+
+// Output map for TMA stores of 32-row slabs: BF16 outputs [d2][rows][cols] in 64-column slabs.
+static int make_out_map(CUtensorMap* m, void* ptr, uint64_t cols, uint64_t rows, uint64_t d2, const char* what) {
+  return make_tmap_t(m, ptr, false, cols, rows, d2, 64, 32, what);
 }
 
 static int round_bn(int n) {
@@ -869,7 +930,7 @@ static int round_bn(int n) {
 
 constexpr int SMEM_LIMIT = 227 * 1024;
 // Alignment slack + barriers, plus the epilogue staging buffers when the launch uses them (K-grouped).
-static int smem_fixed(bool staged) { return 1024 + 256 + (staged ? 4 * STAGE_BYTES_PER_WARP : 0); }
+static int smem_fixed(bool staged) { return 1024 + 256 + (staged ? 4 * STAGE_BUFS * STAGE_BYTES_PER_WARP : 0); }
 
 static int pick_stages(int bn, bool staged) {
   const int stage = A_BYTES + bn * BK * 2;
@@ -1039,7 +1100,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const uint32_t b_bytes = static_cast<uint32_t>(bh) * BK * 2;
   const uint32_t stage_bytes = A_BYTES + b_bytes;
   uint8_t* stage_area = smem + S * stage_bytes;
-  int* pair_off = reinterpret_cast<int*>(stage_area + (kStaged2sm ? 4 * STAGE_BYTES_PER_WARP : 0));
+  int* pair_off = reinterpret_cast<int*>(stage_area + (kStaged2sm ? 4 * STAGE_BUFS * STAGE_BYTES_PER_WARP : 0));
   const int poff_ints = p.tiles ? ((p.G + 1 + 63) & ~63) : 0;
   uint8_t* bar_area = reinterpret_cast<uint8_t*>(pair_off + poff_ints);
   uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
@@ -1191,6 +1252,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int q = warp & 3;
     const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
     const uint32_t acc_empty_leader1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
+    Stager stg{smem_u32(stage_area + (warp - 2) * STAGE_BUFS * STAGE_BYTES_PER_WARP), 0};
     int tcount = 0;
     for (int t = pair; t < ntiles; t += npairs, ++tcount) {
       const PairTile pt = decode_pair(p, pair_off, t, rank);
@@ -1203,12 +1265,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       tl.g = pt.g; tl.row0 = pt.row0; tl.rows = pt.rows; tl.n0 = pt.n0; tl.nk = pt.nk;
       tl.krow0 = 0; tl.kvalid = BK; tl.kb0 = pt.kb0; tl.split = pt.split;
       if constexpr (kStaged2sm)
-        epilogue_tile<EPI>(p, tl, tacc, q, lane, smem_u32(stage_area + (warp - 2) * STAGE_BYTES_PER_WARP));
+        epilogue_tile<EPI>(p, tl, tacc, q, lane, stg);
       else
         epilogue_tile_direct<EPI>(p, tl, tacc, q * 32 + lane);
       tc_fence_before();
       mbar_arrive_cluster(buf ? acc_empty_leader1 : acc_empty_leader0);
     }
+    emit_drain(lane);
   }
 
   tc_fence_before();
@@ -1258,7 +1321,7 @@ static int launch2(Params& p, long long pair_tile_upper_bound, const char* name,
   p.mode = RG;
   const int stage = A_BYTES + (p.bn / 2) * BK * 2;
   const int poff = p.tiles ? ((p.G + 1 + 63) & ~63) * 4 : 0;
-  const int fixed = 1024 + 256 + poff + (kStaged2sm ? 4 * STAGE_BYTES_PER_WARP : 0);
+  const int fixed = 1024 + 256 + poff + (kStaged2sm ? 4 * STAGE_BUFS * STAGE_BYTES_PER_WARP : 0);
   int st = (SMEM_LIMIT - fixed) / stage;
   p.stages = st > MAX_STAGES ? MAX_STAGES : st;
   const size_t smem = fixed + static_cast<size_t>(p.stages) * stage;
@@ -1361,7 +1424,13 @@ int tc_ffn_gemm1(const void* x_pft, const int* seg, const int* tiles, int N, int
   PFMOE_TRY(make_tmap(&p.tmA[0], x_pft, d, N, 1, BK, BM, "x_pft"));
   PFMOE_TRY(make_tmap(&p.tmB[0], w1, h, d, E, 64, 64, "w1"));
   PFMOE_TRY(make_tmap(&p.tmB[1], w3, h, d, E, 64, 64, "w3"));
-  if (use_pairs(N, E)) return launch2<EPI_SWIGLU_FWD>(p, rg_pairs_ub(N, E, h, p.bn / 2), "ffn_gemm1_swiglu", s);
+  if (use_pairs(N, E)) {
+    PFMOE_TRY(make_out_map(&p.tmD[0], h1, h, N, 1, "h1 out"));
+    PFMOE_TRY(make_out_map(&p.tmD[1], h3, h, N, 1, "h3 out"));
+    PFMOE_TRY(make_out_map(&p.tmD[2], a, h, N, 1, "a out"));
+    p.tma_store = 1;
+    return launch2<EPI_SWIGLU_FWD>(p, rg_pairs_ub(N, E, h, p.bn / 2), "ffn_gemm1_swiglu", s);
+  }
   return launch<EPI_SWIGLU_FWD, RG>(p, rg_tiles_ub(N, E, h, p.bn / 2), "ffn_gemm1_swiglu", s);
 }
 
@@ -1377,7 +1446,11 @@ int tc_ffn_gemm2(const void* a, const int* seg, const int* tiles, int N, int E, 
   p.D0 = out; p.ldd = d;
   PFMOE_TRY(make_tmap(&p.tmA[0], a, h, N, 1, BK, BM, "a"));
   PFMOE_TRY(make_tmap(&p.tmB[0], w2, d, h, E, 64, 64, "w2"));
-  if (use_pairs(N, E)) return launch2<EPI_STORE_BF16>(p, rg_pairs_ub(N, E, d, p.bn), "ffn_gemm2", s);
+  if (use_pairs(N, E)) {
+    PFMOE_TRY(make_out_map(&p.tmD[0], out, d, N, 1, "out"));
+    p.tma_store = 1;
+    return launch2<EPI_STORE_BF16>(p, rg_pairs_ub(N, E, d, p.bn), "ffn_gemm2", s);
+  }
   return launch<EPI_STORE_BF16, RG>(p, rg_tiles_ub(N, E, d, p.bn), "ffn_gemm2", s);
 }
 
@@ -1395,7 +1468,12 @@ int tc_ffn_dgrad_act(const void* dO, const int* seg, const int* tiles, int N, in
   const uint32_t brows = pairs ? p.bn / 2 : p.bn;   // B rows loaded per CTA
   PFMOE_TRY(make_tmap(&p.tmA[0], dO, d, N, 1, BK, BM, "dO"));
   PFMOE_TRY(make_tmap(&p.tmB[0], w2, d, h, E, BK, brows, "w2^T"));
-  if (pairs) return launch2<EPI_SWIGLU_BWD>(p, rg_pairs_ub(N, E, h, p.bn), "ffn_dgrad_act_swiglu_bwd", s);
+  if (pairs) {
+    PFMOE_TRY(make_out_map(&p.tmD[0], dh1, h, N, 1, "dh1 out"));
+    PFMOE_TRY(make_out_map(&p.tmD[1], dh3, h, N, 1, "dh3 out"));
+    p.tma_store = 1;
+    return launch2<EPI_SWIGLU_BWD>(p, rg_pairs_ub(N, E, h, p.bn), "ffn_dgrad_act_swiglu_bwd", s);
+  }
   return launch<EPI_SWIGLU_BWD, RG>(p, rg_tiles_ub(N, E, h, p.bn), "ffn_dgrad_act_swiglu_bwd", s);
 }
 
@@ -1416,7 +1494,11 @@ int tc_ffn_dgrad_x(const void* dh1, const void* dh3, const int* seg, const int* 
   PFMOE_TRY(make_tmap(&p.tmA[1], dh3, h, N, 1, BK, BM, "dh3"));
   PFMOE_TRY(make_tmap(&p.tmB[0], w1, h, d, E, BK, brows, "w1^T"));
   PFMOE_TRY(make_tmap(&p.tmB[1], w3, h, d, E, BK, brows, "w3^T"));
-  if (pairs) return launch2<EPI_STORE_BF16>(p, rg_pairs_ub(N, E, d, p.bn), "ffn_dgrad_x", s);
+  if (pairs) {
+    PFMOE_TRY(make_out_map(&p.tmD[0], dx_pft, d, N, 1, "dx_pft out"));
+    p.tma_store = 1;
+    return launch2<EPI_STORE_BF16>(p, rg_pairs_ub(N, E, d, p.bn), "ffn_dgrad_x", s);
+  }
   return launch<EPI_STORE_BF16, RG>(p, rg_tiles_ub(N, E, d, p.bn), "ffn_dgrad_x", s);
 }
 
@@ -1434,6 +1516,9 @@ int tc_ffn_wgrad13(const void* x_pft, const void* dh1, const void* dh3, const in
   PFMOE_TRY(make_tmap(&p.tmA[0], x_pft, d, N, 1, 64, 64, "x_pft^T"));
   PFMOE_TRY(make_tmap(&p.tmB[0], dh1, h, N, 1, 64, 64, "dh1"));
   PFMOE_TRY(make_tmap(&p.tmB[1], dh3, h, N, 1, 64, 64, "dh3"));
+  PFMOE_TRY(make_out_map(&p.tmD[0], dw1, h, d, E, "dw1 out"));
+  PFMOE_TRY(make_out_map(&p.tmD[1], dw3, h, d, E, "dw3 out"));
+  p.tma_store = 1;
   const long long ub = static_cast<long long>(E) * ((d + BM - 1) / BM) * ((h + p.bn / 2 - 1) / (p.bn / 2));
   return launch<EPI_SPLIT_BF16, KG>(p, ub, "ffn_wgrad_w1w3", s);
 }
@@ -1450,6 +1535,8 @@ int tc_ffn_wgrad2(const void* a, const void* dO, const int* seg, int N, int E, i
   p.D0 = dw2; p.ldd = d; p.d_gstride = static_cast<long long>(h) * d;
   PFMOE_TRY(make_tmap(&p.tmA[0], a, h, N, 1, 64, 64, "a^T"));
   PFMOE_TRY(make_tmap(&p.tmB[0], dO, d, N, 1, 64, 64, "dO"));
+  PFMOE_TRY(make_out_map(&p.tmD[0], dw2, d, h, E, "dw2 out"));
+  p.tma_store = 1;
   const long long ub = static_cast<long long>(E) * ((h + BM - 1) / BM) * ((d + p.bn - 1) / p.bn);
   return launch<EPI_STORE_BF16, KG>(p, ub, "ffn_wgrad_w2", s);
 }
@@ -1529,6 +1616,8 @@ int tc_gate_wgrad(const void* x, const void* dz_bf16, int T, int d, int E, float
   }
   PFMOE_TRY(make_tmap(&p.tmA[0], x, d, T, 1, 64, 64, "x^T"));
   PFMOE_TRY(make_tmap(&p.tmB[0], dz_bf16, E, T, 1, 64, 64, "dz"));
+  PFMOE_TRY(make_tmap_t(&p.tmD[0], p.D0, true, E, d, ks, 32, 32, "dwg out"));
+  p.tma_store = 1;
   const long long ub = static_cast<long long>(ks) * ((d + BM - 1) / BM) * ((E + p.bn - 1) / p.bn);
   PFMOE_TRY((launch<EPI_STORE_F32, KG>(p, ub, "gate_wgrad", s)));
   if (ks > 1)
