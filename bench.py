@@ -46,11 +46,6 @@ def parse():
     return ap.parse_args()
 
 
-def dist_env():
-    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
-            int(os.environ.get("LOCAL_RANK", 0)))
-
-
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -214,7 +209,9 @@ def inputs_to_cpu64(inp):
 
 def run_reference(args):
     """Reference arm: the CPU oracle as it stands, on bounded token samples of the workload."""
-    rank, world, _ = dist_env()
+    from padding_free_moe_b200 import replicas
+    info = replicas.rank_info()
+    rank, world = info.rank, info.world
     if rank != 0:
         return 0
     from workloads import get_config, make_inputs
@@ -255,20 +252,18 @@ def config_block(cfg, world):
 
 # ------------------------------------------------------------------ our arm
 def run_ours(args):
-    rank, world, local_rank = dist_env()
     import torch
-    import torch.distributed as dist
     from padding_free_moe_b200 import _lib as L
+    from padding_free_moe_b200 import replicas
     from padding_free_moe_b200.layer import PFTMoELayer, Shape
     from workloads import get_config, make_inputs
     from workloads.generate import storage_dtype
 
+    info = replicas.rank_info()
+    rank, world, local_rank = info.rank, info.world, info.local_rank
     torch.cuda.set_device(local_rank)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local_rank))
     dev = torch.device("cuda", local_rank)
+    replicas.init(info, "nccl", timeout_s=120, device=dev)
     cfg = get_config(args.workload)
     inp = make_inputs(cfg, seed=1000 + rank, device=dev)
     layer = PFTMoELayer(Shape(cfg.T, cfg.d, cfg.E, cfg.h, cfg.k, storage_dtype(cfg), cfg.rbd_epd, cfg.rbd_dpn), dev)
@@ -278,15 +273,10 @@ def run_ours(args):
         layer.step(inp.x, inp.wg, inp.bias, inp.w1, inp.w3, inp.w2, inp.dy, stream)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        replicas.barrier(info)
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(v, info, device=dev)
 
     warm = max(3, args.warmup)
     for _ in range(warm):
@@ -296,8 +286,7 @@ def run_ours(args):
         raise RuntimeError(f"device error word {layer.device_error():#x} after warm-up")
 
     # ---- device-timed region, inputs resident; per-kernel events live
-    clk = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
-                       int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    clk = ClockSampler(replicas.physical_gpu_index(local_rank))
     L.moe_profile_reset()
     barrier()
     torch.cuda.synchronize()
@@ -413,8 +402,7 @@ def run_ours(args):
                                           f"(forward, RBD plan, backward), {s:.1f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    replicas.finish(info)
     return 0
 
 
