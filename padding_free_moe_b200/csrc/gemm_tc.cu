@@ -47,8 +47,6 @@ struct Params {
   CUtensorMap tmB[2];
   CUtensorMap tmD[3];  // output maps for TMA stores from the staged epilogue (box 128 B x 32 rows)
   int tma_store;       // 1: tmD[] are valid
-  const char* pf_base[2];   // two-SM row-grouped: per-expert weight matrices prefetched into L2 ...
-  long long pf_bytes;       // ... one wave of tiles ahead (bytes per expert; 0 = off)
   int mode;
   int b_major;       // RG: 0 = K-major B (weights [G, N, K]), 1 = MN-major B (weights [G, K, N]); KG: 1
   int bn;            // MMA N: multiple of 64, <= 256
@@ -1002,10 +1000,6 @@ __device__ __forceinline__ bool wait_bar2(uint32_t bar, uint32_t parity, volatil
     }
   }
 }
-__device__ __forceinline__ void bulk_prefetch_l2(const void* gptr, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(gptr)), "r"(bytes)
-               : "memory");
-}
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* tm, uint32_t bar_cluster, int c0,
                                                  int c1, int c2) {
   asm volatile(
@@ -1179,17 +1173,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       bool ok = true;
       for (int t = pair; t < ntiles && ok; t += npairs) {
         const PairTile tl = decode_pair(p, pair_off, t, rank);
-        if (leader && p.pf_bytes > 0 && t + npairs < ntiles) {
-          // The tile one wave ahead opens a new expert: pull that expert's weights into L2 now,
-          // so the weight stream from HBM overlaps the current wave instead of stalling it.
-          const PairTile nx = decode_pair(p, pair_off, t + npairs, 0);
-          if (nx.n0 == 0 && nx.row0 == p.seg[nx.g] && nx.kb0 == 0)
-            for (int i = 0; i < 2; ++i)
-              if (p.pf_base[i])
-                for (long long off = 0; off < p.pf_bytes; off += (1ll << 30))
-                  bulk_prefetch_l2(p.pf_base[i] + nx.g * p.pf_bytes + off,
-                                   static_cast<uint32_t>(min(p.pf_bytes - off, 1ll << 30)));
-        }
         for (int kb = 0; kb < tl.nk; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
@@ -1446,9 +1429,6 @@ int tc_ffn_gemm1(const void* x_pft, const int* seg, const int* tiles, int N, int
     PFMOE_TRY(make_out_map(&p.tmD[1], h3, h, N, 1, "h3 out"));
     PFMOE_TRY(make_out_map(&p.tmD[2], a, h, N, 1, "a out"));
     p.tma_store = 1;
-    p.pf_base[0] = static_cast<const char*>(w1);
-    p.pf_base[1] = static_cast<const char*>(w3);
-    p.pf_bytes = static_cast<long long>(d) * h * 2;
     return launch2<EPI_SWIGLU_FWD>(p, rg_pairs_ub(N, E, h, p.bn / 2), "ffn_gemm1_swiglu", s);
   }
   return launch<EPI_SWIGLU_FWD, RG>(p, rg_tiles_ub(N, E, h, p.bn / 2), "ffn_gemm1_swiglu", s);
@@ -1469,8 +1449,6 @@ int tc_ffn_gemm2(const void* a, const int* seg, const int* tiles, int N, int E, 
   if (use_pairs(N, E)) {
     PFMOE_TRY(make_out_map(&p.tmD[0], out, d, N, 1, "out"));
     p.tma_store = 1;
-    p.pf_base[0] = static_cast<const char*>(w2);
-    p.pf_bytes = static_cast<long long>(d) * h * 2;
     return launch2<EPI_STORE_BF16>(p, rg_pairs_ub(N, E, d, p.bn), "ffn_gemm2", s);
   }
   return launch<EPI_STORE_BF16, RG>(p, rg_tiles_ub(N, E, d, p.bn), "ffn_gemm2", s);
@@ -1494,8 +1472,6 @@ int tc_ffn_dgrad_act(const void* dO, const int* seg, const int* tiles, int N, in
     PFMOE_TRY(make_out_map(&p.tmD[0], dh1, h, N, 1, "dh1 out"));
     PFMOE_TRY(make_out_map(&p.tmD[1], dh3, h, N, 1, "dh3 out"));
     p.tma_store = 1;
-    p.pf_base[0] = static_cast<const char*>(w2);
-    p.pf_bytes = static_cast<long long>(d) * h * 2;
     return launch2<EPI_SWIGLU_BWD>(p, rg_pairs_ub(N, E, h, p.bn), "ffn_dgrad_act_swiglu_bwd", s);
   }
   return launch<EPI_SWIGLU_BWD, RG>(p, rg_tiles_ub(N, E, h, p.bn), "ffn_dgrad_act_swiglu_bwd", s);
@@ -1521,9 +1497,6 @@ int tc_ffn_dgrad_x(const void* dh1, const void* dh3, const int* seg, const int* 
   if (pairs) {
     PFMOE_TRY(make_out_map(&p.tmD[0], dx_pft, d, N, 1, "dx_pft out"));
     p.tma_store = 1;
-    p.pf_base[0] = static_cast<const char*>(w1);
-    p.pf_base[1] = static_cast<const char*>(w3);
-    p.pf_bytes = static_cast<long long>(d) * h * 2;
     return launch2<EPI_STORE_BF16>(p, rg_pairs_ub(N, E, d, p.bn), "ffn_dgrad_x", s);
   }
   return launch<EPI_STORE_BF16, RG>(p, rg_tiles_ub(N, E, d, p.bn), "ffn_dgrad_x", s);
