@@ -46,9 +46,14 @@ struct Params {
   CUtensorMap tmA[2];
   CUtensorMap tmB[2];
   CUtensorMap tmD[3];  // output maps for TMA stores from the staged epilogue (box 128 B x 32 rows)
+  CUtensorMap tmB32[2];  // token-as-N kernel: the token maps of tmB[] with 32-row boxes (ragged tiles)
   int tma_store;       // 1: tmD[] are valid
   int mode;
   int b_major;       // RG: 0 = K-major B (weights [G, N, K]), 1 = MN-major B (weights [G, K, N]); KG: 1
+  int a_major;       // token-as-N kernel: 0 = K-major weights [G, F, K], 1 = MN-major weights [G, K, F]
+  int a_merged;      // MN-major A map is the 4-D block view (one copy fetches every 64-wide block of a stage)
+  int b_merged;      // same for the MN-major B maps
+  int fstep;         // token-as-N kernel: output features per pair tile (256, or 128 with nsplit)
   int bn;            // MMA N: multiple of 64, <= 256
   int nsplit;        // 1: B tile columns [0, bn/2) come from tmB[0], [bn/2, bn) from tmB[1]
   int M;             // KG: rows of each group's output
@@ -138,6 +143,15 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm,
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
           dst),
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+// 4-D form for the block view of an MN-major tensor: coordinates (0, k, block, group).
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm, uint32_t bar, int c0, int c1, int c2,
+                                            int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* tm) {
@@ -763,15 +777,28 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
             }
           } else {
             const int krow = tl.krow0 + kb * BK;
-            tma_load_3d(sa, &p.tmA[0], fb, tl.row0, krow, 0);
-            tma_load_3d(sa + BOX_BYTES, &p.tmA[0], fb, tl.row0 + 64, krow, 0);
-            for (int j = 0; j < nb; ++j) {
-              int which = 0, nc = tl.n0 + 64 * j;
+            if (p.a_merged) {
+              tma_load_4d(sa, &p.tmA[0], fb, 0, krow, tl.row0 / 64, 0);
+            } else {
+              tma_load_3d(sa, &p.tmA[0], fb, tl.row0, krow, 0);
+              tma_load_3d(sa + BOX_BYTES, &p.tmA[0], fb, tl.row0 + 64, krow, 0);
+            }
+            if (p.b_merged) {
               if (p.nsplit) {
-                which = j < nb / 2 ? 0 : 1;
-                nc = tl.n0 + 64 * (j < nb / 2 ? j : j - nb / 2);
+                tma_load_4d(sb, &p.tmB[0], fb, 0, krow, tl.n0 / 64, 0);
+                tma_load_4d(sb + (nb / 2) * BOX_BYTES, &p.tmB[1], fb, 0, krow, tl.n0 / 64, 0);
+              } else {
+                tma_load_4d(sb, &p.tmB[0], fb, 0, krow, tl.n0 / 64, 0);
               }
-              tma_load_3d(sb + j * BOX_BYTES, &p.tmB[which], fb, nc, krow, 0);
+            } else {
+              for (int j = 0; j < nb; ++j) {
+                int which = 0, nc = tl.n0 + 64 * j;
+                if (p.nsplit) {
+                  which = j < nb / 2 ? 0 : 1;
+                  nc = tl.n0 + 64 * (j < nb / 2 ? j : j - nb / 2);
+                }
+                tma_load_3d(sb + j * BOX_BYTES, &p.tmB[which], fb, nc, krow, 0);
+              }
             }
           }
           pending |= 1u << s;
@@ -896,7 +923,7 @@ static int get_encode() {
 // 3-D tensor map over a row-major tensor [d2][d1][d0] (BF16 or FP32) with a box of
 // b0 x b1 x 1 elements and 128-byte swizzle (b0 * element size must be 128 bytes or less).
 static int make_tmap_t(CUtensorMap* m, const void* ptr, bool f32, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
-                       uint32_t b1, const char* what) {
+                       uint32_t b1, const char* what, bool swizzle = true) {
   PFMOE_TRY(get_encode());
   const uint64_t es = f32 ? 4 : 2;
   cuuint64_t dims[3] = {d0, d1, d2};
@@ -905,7 +932,8 @@ static int make_tmap_t(CUtensorMap* m, const void* ptr, bool f32, uint64_t d0, u
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                         const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(PFMOE_ERR_CUDA, std::string("cuTensorMapEncodeTiled failed for ") + what + " (CUresult " +
@@ -923,10 +951,39 @@ static int make_out_map(CUtensorMap* m, void* ptr, uint64_t cols, uint64_t rows,
   return make_tmap_t(m, ptr, false, cols, rows, d2, 64, 32, what);
 }
 
+// Block view of an MN-major BF16 tensor [g][k][mn] (mn a multiple of 64): a 4-D map over
+// (64, k, mn / 64, g) whose box {64, box_k, nblk, 1} lands in shared memory as nblk
+// consecutive 64-wide blocks of box_k 128-byte rows -- the same layout as nblk separate
+// {64, box_k} boxes, fetched by one copy.  TMA delivery per copy has a fixed cost, so one
+// 16-32 KB copy moves operands markedly faster than two to four 8 KB copies.
+static int make_tmap_mn(CUtensorMap* m, const void* ptr, uint64_t mn, uint64_t k, uint64_t g, uint32_t box_k,
+                        uint32_t nblk, const char* what) {
+  PFMOE_TRY(get_encode());
+  cuuint64_t dims[4] = {64, k, mn / 64, g};
+  cuuint64_t strides[3] = {mn * 2, 128, k * mn * 2};
+  cuuint32_t box[4] = {64, box_k, nblk, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(PFMOE_ERR_CUDA, std::string("cuTensorMapEncodeTiled (block view) failed for ") + what + " (CUresult " +
+                                    std::to_string(static_cast<int>(r)) + ")");
+  return PFMOE_OK;
+}
+
+// Output map for the token-as-N kernel: BF16 [rows][cols], 32 x 32 boxes, unswizzled 64-byte rows.
+static int make_out_map_tn(CUtensorMap* m, void* ptr, uint64_t cols, uint64_t rows, const char* what) {
+  return make_tmap_t(m, ptr, false, cols, rows, 1, 32, 32, what, false);
+}
+
 static int round_bn(int n) {
   int bn = ((n + 63) / 64) * 64;
   return bn > 256 ? 256 : bn;
 }
+
+// MMA N for the two-SM kernel: each CTA of the pair holds half of it in whole 64-column boxes.
+static int round_bn_pair(int n) { return n > 128 ? 256 : 128; }
 
 constexpr int SMEM_LIMIT = 227 * 1024;
 // Alignment slack + barriers, plus the epilogue staging buffers when the launch uses them (K-grouped).
@@ -1008,6 +1065,14 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const CUtensorMap* tm, uint32_t bar_cluster, int c0,
+                                                 int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_alloc2(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
                : "memory");
@@ -1037,15 +1102,44 @@ __device__ __forceinline__ void tc_commit2_both(uint32_t bar) {
 }
 
 struct PairTile {
-  int g, row0, rows, n0, nk, kb0, split;
+  int g, row0, rows, n0, nk, kb0, split, krow0, kvalid;
 };
 
 // Pair tiles of a row-grouped problem: expert g has ceil(n_g / 256) of them (prefix in pair_off).
+// K-grouped: every group has ceil(M / 256) x NT output tiles.
+template <int MODE>
 __device__ __forceinline__ int total_pair_tiles(const Params& p, const int* pair_off) {
   const int ns = n_step(p);
   const int NT = (p.Nout + ns - 1) / ns;
+  if constexpr (MODE == KG) return p.G * ((p.M + 2 * BM - 1) / (2 * BM)) * NT;
   const int np = p.tiles ? pair_off[p.G] : (p.dense_len + 2 * BM - 1) / (2 * BM) * p.ksplit;
   return np * NT;
+}
+
+// K-grouped pair tile: rows [256 mp + 128 rank, +128) of group g's [M, Nout] output, K = the group's segment.
+__device__ __forceinline__ PairTile decode_pair_kg(const Params& p, int t, uint32_t rank) {
+  PairTile tl;
+  const int ns = n_step(p);
+  const int NT = (p.Nout + ns - 1) / ns;
+  const int MP = (p.M + 2 * BM - 1) / (2 * BM);
+  const int per = MP * NT;
+  const int g = t / per;
+  const int rem = t - g * per;
+  const int n_idx = rem / MP;
+  const int mp = rem - n_idx * MP;
+  const int s0 = p.seg ? p.seg[g] : g * p.kchunk;
+  const int s1 = p.seg ? p.seg[g + 1] : min(p.dense_len, s0 + p.kchunk);
+  const int len = max(0, s1 - s0);
+  tl.g = g;
+  tl.row0 = mp * 2 * BM + static_cast<int>(rank) * BM;
+  tl.rows = max(0, min(BM, p.M - tl.row0));
+  tl.n0 = n_idx * ns;
+  tl.nk = (len + BK - 1) / BK;
+  tl.kb0 = 0;
+  tl.split = 0;
+  tl.krow0 = s0;
+  tl.kvalid = len - (tl.nk - 1) * BK;
+  return tl;
 }
 
 __device__ __forceinline__ PairTile decode_pair(const Params& p, const int* pair_off, int t, uint32_t rank) {
@@ -1083,14 +1177,28 @@ __device__ __forceinline__ PairTile decode_pair(const Params& p, const int* pair
   tl.split = split;
   tl.kb0 = split * kbs;
   tl.nk = max(0, min(kbs, nk_all - tl.kb0));
+  tl.krow0 = 0;
+  tl.kvalid = BK;
   return tl;
+}
+
+template <int MODE>
+__device__ __forceinline__ PairTile decode_pair_any(const Params& p, const int* pair_off, int t, uint32_t rank) {
+  if constexpr (MODE == KG) return decode_pair_kg(p, t, rank);
+  else return decode_pair(p, pair_off, t, rank);
+}
+
+__device__ __forceinline__ void st_cluster16(uint32_t addr, uint4 u) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(u.x), "r"(u.y), "r"(u.z),
+               "r"(u.w)
+               : "memory");
 }
 
 // Epilogue of the two-SM kernel: staged through shared memory (full-line stores, coalesced
 // reads of the SwiGLU-backward inputs) or direct per-row stores.
 constexpr bool kStaged2sm = true;
 
-template <int EPI>
+template <int EPI, int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     grouped_gemm_2sm_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -1163,7 +1271,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int ntiles = total_pair_tiles(p, pair_off);
+  const int ntiles = total_pair_tiles<MODE>(p, pair_off);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -1172,7 +1280,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int it = 0;
       bool ok = true;
       for (int t = pair; t < ntiles && ok; t += npairs) {
-        const PairTile tl = decode_pair(p, pair_off, t, rank);
+        const PairTile tl = decode_pair_any<MODE>(p, pair_off, t, rank);
         for (int kb = 0; kb < tl.nk; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
@@ -1182,6 +1290,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           const uint32_t fb = mapa_shared(fb_local, 0);
           const uint32_t sa = smem_u32(smem + s * stage_bytes);
           const uint32_t sb = sa + A_BYTES;
+          if constexpr (MODE == KG) {
+            // A = X^T (MN-major): this CTA's 128 output rows; B (MN-major): its bh output columns.
+            const int krow = tl.krow0 + kb * BK;
+            if (p.a_merged) {
+              tma_load_4d_pair(sa, &p.tmA[0], fb, 0, krow, tl.row0 / 64, 0);
+            } else {
+              tma_load_3d_pair(sa, &p.tmA[0], fb, tl.row0, krow, 0);
+              tma_load_3d_pair(sa + BOX_BYTES, &p.tmA[0], fb, tl.row0 + 64, krow, 0);
+            }
+            const CUtensorMap* tb = &p.tmB[p.nsplit ? static_cast<int>(rank) : 0];
+            const int ncol = p.nsplit ? tl.n0 : tl.n0 + static_cast<int>(rank) * bh;
+            if (p.b_merged) {
+              tma_load_4d_pair(sb, tb, fb, 0, krow, ncol / 64, 0);
+            } else {
+              for (int j = 0; j < bh / 64; ++j) tma_load_3d_pair(sb + j * BOX_BYTES, tb, fb, ncol + 64 * j, krow, 0);
+            }
+            pending |= 1u << s;
+            pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
+            continue;
+          }
           const int kbg = tl.kb0 + kb;
           const int src = kbg < p.k0_blocks ? 0 : 1;
           const int kk = (src == 0 ? kbg : kbg - p.k0_blocks) * BK;
@@ -1205,13 +1333,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (leader) {
-      const uint32_t idesc = idesc_bf16(2 * BM, p.bn, 0, p.b_major);
-      const uint32_t b_lbo = p.b_major ? BOX_BYTES : 16;
-      const uint32_t b_step = p.b_major ? 2048 : 32;
+      const int a_mn = MODE == KG ? 1 : 0;
+      const int b_mn = MODE == KG ? 1 : p.b_major;
+      const uint32_t idesc = idesc_bf16(2 * BM, p.bn, a_mn, b_mn);
+      const uint32_t a_lbo = a_mn ? BOX_BYTES : 16, b_lbo = b_mn ? BOX_BYTES : 16;
+      const uint32_t a_step = a_mn ? 2048 : 32, b_step = b_mn ? 2048 : 32;
       int it = 0, tcount = 0;
       bool ok = true;
       for (int t = pair; t < ntiles && ok; t += npairs, ++tcount) {
-        const PairTile tl = decode_pair(p, pair_off, t, rank);
+        const PairTile tl = decode_pair_any<MODE>(p, pair_off, t, rank);
         const int buf = tcount & 1;
         const uint32_t aph = (tcount >> 1) & 1;
         ok = __all_sync(0xffffffffu, wait_bar2(smem_u32(&acc_empty[buf]), aph ^ 1, abort_flag, p.err));
@@ -1223,13 +1353,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           const uint32_t ph = (it / S) & 1;
           ok = __all_sync(0xffffffffu, wait_bar2(smem_u32(&full[s]), ph, abort_flag, p.err));
           if (!ok) break;
-          tc_fence_after();
           const uint32_t sa = smem_u32(smem + s * stage_bytes);
           const uint32_t sb = sa + A_BYTES;
+          int kk_count = BK / 16;
+          if (MODE == KG && kb == tl.nk - 1 && tl.kvalid < BK) {
+            // Last block of a segment: MMAs stop at the 16-row step holding the segment end, and the
+            // rows of that step past the end are zeroed in every box of both CTAs (the peer's over DSMEM).
+            const int kv16 = (tl.kvalid + 15) & ~15;
+            kk_count = kv16 / 16;
+            const int per_box = (kv16 - tl.kvalid) * 8;   // 16-byte chunks to clear per box
+            if (per_box > 0) {
+              const int nbox = 2 + bh / 64;
+              for (int b = 0; b < nbox; ++b)
+                for (int i = lane; i < per_box; i += 32) {
+                  const uint32_t a = sa + b * BOX_BYTES + tl.kvalid * 128 + i * 16;
+                  st_shared16(a, make_uint4(0, 0, 0, 0));
+                  st_cluster16(mapa_shared(a, 1), make_uint4(0, 0, 0, 0));
+                }
+              asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+            }
+            __syncwarp();
+          }
+          tc_fence_after();
           if (lane == 0) {
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-              const uint64_t ad = sdesc(sa + kk * 32, 16, 1024);
+            for (int kk = 0; kk < kk_count; ++kk) {
+              const uint64_t ad = sdesc(sa + kk * a_step, a_lbo, 1024);
               const uint64_t bd = sdesc(sb + kk * b_step, b_lbo, 1024);
               tc_mma2(tmem_d, ad, bd, idesc, (kb | kk) != 0);
             }
@@ -1238,7 +1386,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           __syncwarp();
         }
         if (!ok) break;
-        if (lane == 0) tc_commit2_both(smem_u32(&acc_full[buf]));
+        if (lane == 0) tc_commit2_both(smem_u32(&acc_full[buf]));   // also for nk == 0 (zero tile)
         __syncwarp();
       }
       if (lane == 0) {
@@ -1255,7 +1403,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     Stager stg{smem_u32(stage_area + (warp - 2) * STAGE_BUFS * STAGE_BYTES_PER_WARP), 0};
     int tcount = 0;
     for (int t = pair; t < ntiles; t += npairs, ++tcount) {
-      const PairTile pt = decode_pair(p, pair_off, t, rank);
+      const PairTile pt = decode_pair_any<MODE>(p, pair_off, t, rank);
       const int buf = tcount & 1;
       const uint32_t aph = (tcount >> 1) & 1;
       if (!__all_sync(0xffffffffu, wait_bar2(smem_u32(&acc_full[buf]), aph, abort_flag, p.err))) break;
@@ -1263,13 +1411,525 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * p.bn;
       Tile tl;
       tl.g = pt.g; tl.row0 = pt.row0; tl.rows = pt.rows; tl.n0 = pt.n0; tl.nk = pt.nk;
-      tl.krow0 = 0; tl.kvalid = BK; tl.kb0 = pt.kb0; tl.split = pt.split;
+      tl.krow0 = pt.krow0; tl.kvalid = pt.kvalid; tl.kb0 = pt.kb0; tl.split = pt.split;
       if constexpr (kStaged2sm)
         epilogue_tile<EPI>(p, tl, tacc, q, lane, stg);
       else
         epilogue_tile_direct<EPI>(p, tl, tacc, q * 32 + lane);
       tc_fence_before();
       mbar_arrive_cluster(buf ? acc_empty_leader1 : acc_empty_leader0);
+    }
+    emit_drain(lane);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc2(tmem_base, tmem_cols);
+  }
+}
+
+// ============================================================================
+// Token-as-N two-SM kernel for row-grouped problems.
+//
+// The expert's weights are the MMA's A operand and its tokens the B operand:
+// D^T[f, t] = sum_k W_g[f, k] X[t, k], so TMEM lanes hold output features and
+// TMEM columns hold tokens.  A pair tile is M = 256 weight rows (128 per CTA)
+// by N = the tile's token count rounded up to 32 (at most 256; CTA v loads
+// token columns [vN/2, (v+1)N/2)).  A ragged expert segment therefore costs at
+// most 31 spare MMA columns, where 256-row tiles over tokens compute up to 255
+// spare rows; on MoE layers with a few hundred tokens per expert that is a
+// quarter of the row-major kernel's tensor work.  The epilogue transposes
+// 32 x 32 blocks through shared memory and stores [token, feature] rows.
+//
+// With nsplit (SwiGLU forward) a pair tile covers 128 features: CTA v holds
+// rows [64v, 64v + 64) of W1^T in TMEM lanes 0..63 and the same rows of W3^T in
+// lanes 64..127, so the H1 and H3 values of one (token, feature) sit in the
+// same lane of epilogue warps q and q + 2; warp q + 2 hands its FP32 H3 block
+// to warp q through shared memory (bounded mbarrier handshake).
+constexpr int TN_TOK = 256;             // tokens per pair tile
+constexpr int TN_SLAB = 32 * 64;        // one 32-token x 32-feature BF16 block (64-byte rows)
+constexpr int TN_XBUF = 32 * 32 * 4;    // one 32 x 32 FP32 block
+
+__host__ __device__ constexpr int tn_aux_bytes(int epi) {
+  return epi == EPI_SWIGLU_FWD ? 2 * 2 * TN_XBUF : (epi == EPI_SWIGLU_BWD ? 4 * 2 * TN_SLAB : 0);
+}
+
+struct TnTile {
+  int g, tok0, ntok, nmma, f0, nk;
+};
+
+__device__ __forceinline__ int tn_feature_tiles(const Params& p) { return (p.Nout + p.fstep - 1) / p.fstep; }
+
+// Pair tiles: expert g has ceil(n_g / 256) token tiles (prefix in pair_off) per feature tile;
+// token tiles are the fastest index, so neighbouring CTAs share the same weight block.
+__device__ __forceinline__ TnTile decode_tn(const Params& p, const int* pair_off, int t) {
+  const int FT = tn_feature_tiles(p);
+  int lo = 0, hi = p.G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pair_off[mid] * FT <= t) lo = mid; else hi = mid - 1;
+  }
+  TnTile tl;
+  const int npg = max(1, pair_off[lo + 1] - pair_off[lo]);   // >= 1 whenever tiles[] matches seg[]
+  const int local = t - pair_off[lo] * FT;
+  const int fi = local / npg;
+  const int j = local - fi * npg;
+  tl.g = lo;
+  tl.tok0 = p.seg[lo] + j * TN_TOK;
+  tl.ntok = max(0, min(TN_TOK, p.seg[lo + 1] - tl.tok0));
+  tl.nmma = max(32, (tl.ntok + 31) & ~31);                  // a valid MMA shape even for an empty tile
+  tl.f0 = fi * p.fstep;
+  tl.nk = p.k0_blocks + p.k1_blocks;
+  return tl;
+}
+
+// Tile order of one pair.  Unit order: the pair takes (expert, feature block) units
+// u = pair, pair + npairs, ... and runs all token tiles of a unit back to back, so the
+// unit's weight block is fetched into this die's L2 once and re-read from there.  Wave
+// order: wave k holds pair tiles [k P, (k + 1) P) as numbered by decode_tn (P pairs), and
+// pair p takes tile k P + p in even waves and k P + P - 1 - p in odd ones.  Neighbouring
+// tiles (the full and the ragged token tile of one weight block) thus alternate between
+// pairs instead of always landing on pairs of the same parity.
+constexpr bool kTnUnitOrder = false;
+// Ragged token tiles load their token columns in 32-row boxes instead of one 128-row box.
+constexpr bool kTnRaggedBoxes = false;
+
+struct TnCursor {
+  int u, j, t;   // unit order: unit u, token tile j; wave order: wave u, pair t
+};
+
+__device__ __forceinline__ bool tn_next(const Params& p, const int* pair_off, int npairs, TnCursor& c, TnTile& tl) {
+  const int FT = tn_feature_tiles(p);
+  if constexpr (kTnUnitOrder) {
+    const int nunits = p.G * FT;
+    while (c.u < nunits) {
+      const int g = c.u / FT;
+      const int npg = pair_off[g + 1] - pair_off[g];
+      if (c.j < npg) {
+        tl.g = g;
+        tl.tok0 = p.seg[g] + c.j * TN_TOK;
+        tl.ntok = max(0, min(TN_TOK, p.seg[g + 1] - tl.tok0));
+        tl.nmma = max(32, (tl.ntok + 31) & ~31);
+        tl.f0 = (c.u - g * FT) * p.fstep;
+        tl.nk = p.k0_blocks + p.k1_blocks;
+        ++c.j;
+        return true;
+      }
+      c.u += npairs;
+      c.j = 0;
+    }
+    return false;
+  } else {
+    // c.u = wave index, c.t = this pair's index
+    const int t = c.u * npairs + ((c.u & 1) ? npairs - 1 - c.t : c.t);
+    if (t >= pair_off[p.G] * FT) return false;
+    tl = decode_tn(p, pair_off, t);
+    ++c.u;
+    return true;
+  }
+}
+
+__device__ __forceinline__ void st_shared32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_shared32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// Transposes between a thread-per-feature register block (v[j] = token j of feature `lane`)
+// and a [token][feature] BF16 slab with 64-byte rows.  Neighbouring lanes swap one value so
+// every shared access is a 32-bit word holding two adjacent features; even lanes touch row j
+// and odd lanes row j + 1, which sit in opposite halves of the 32 banks.
+__device__ __forceinline__ void stage_t_write(uint32_t slab, int lane, const float* v) {
+  const int odd = lane & 1;
+  const uint32_t col = static_cast<uint32_t>(lane & ~1) * 2;
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    const float send = odd ? v[j] : v[j + 1];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+    __nv_bfloat162 b = __floats2bfloat162_rn(odd ? recv : v[j], odd ? v[j + 1] : recv);
+    st_shared32(slab + (j + odd) * 64 + col, *reinterpret_cast<uint32_t*>(&b));
+  }
+}
+
+__device__ __forceinline__ void stage_t_read(uint32_t slab, int lane, float* v) {
+  const int odd = lane & 1;
+  const uint32_t col = static_cast<uint32_t>(lane & ~1) * 2;
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    const uint32_t w = ld_shared32(slab + (j + odd) * 64 + col);
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+    const float recv = __shfl_xor_sync(0xffffffffu, odd ? f.x : f.y, 1);
+    v[j] = odd ? recv : f.x;
+    v[j + 1] = odd ? f.y : recv;
+  }
+}
+
+// Slab <-> global rows (32 rows of up to 64 bytes; eight rows per instruction, 16 bytes a lane).
+// Rows >= rows_valid and bytes >= bytes_valid are skipped on the way out and read as zero on the way in.
+__device__ __forceinline__ void copy_out_t(uint32_t slab, int lane, char* base, long long stride, int rows_valid,
+                                           int bytes_valid) {
+  const int chunk = lane & 3;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int row = it * 8 + (lane >> 2);
+    const uint4 u = ld_shared16(slab + row * 64 + chunk * 16);
+    if (row < rows_valid && chunk * 16 < bytes_valid)
+      *reinterpret_cast<uint4*>(base + row * stride + chunk * 16) = u;
+  }
+}
+__device__ __forceinline__ void load_t(uint4 (&u)[4], int lane, const char* base, long long stride, int rows_valid,
+                                       int bytes_valid) {
+  const int chunk = lane & 3;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int row = it * 8 + (lane >> 2);
+    u[it] = make_uint4(0, 0, 0, 0);
+    if (row < rows_valid && chunk * 16 < bytes_valid)
+      u[it] = __ldg(reinterpret_cast<const uint4*>(base + row * stride + chunk * 16));
+  }
+}
+__device__ __forceinline__ void put_t(uint32_t slab, int lane, const uint4 (&u)[4]) {
+  const int chunk = lane & 3;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) st_shared16(slab + (it * 8 + (lane >> 2)) * 64 + chunk * 16, u[it]);
+}
+
+// Transpose one 32 x 32 block into the next staging slab and write it out: a block of 32 valid
+// tokens goes out as one TMA store (clipped at the feature bound); a partial block with masked
+// vector stores, so tokens of the next expert segment are never touched.
+__device__ __forceinline__ void emit_t(Stager& st, int lane, const float* v, const CUtensorMap* tm, int f, int tok,
+                                       __nv_bfloat16* dst, long long ldd, int rows_valid, int fvalid) {
+  const uint32_t buf = st.base + (st.seq & 1) * TN_SLAB;
+  ++st.seq;
+  if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+  __syncwarp();
+  stage_t_write(buf, lane, v);
+  if (tm && rows_valid == 32) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) tma_store_3d(tm, buf, f, tok, 0);
+  } else {
+    __syncwarp();
+    copy_out_t(buf, lane, reinterpret_cast<char*>(dst), ldd * 2, rows_valid, min(64, fvalid * 2));
+  }
+  if (lane == 0) asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Epilogue of one pair tile for epilogue warp q (TMEM lanes 32q..32q+31).  `xn` counts the H3
+// hand-offs of this warp pair (SwiGLU forward).  Returns false if a hand-off wait gave up.
+template <int EPI>
+__device__ __forceinline__ bool epilogue_tn(const Params& p, const TnTile& tl, uint32_t tacc, int q, int lane,
+                                            uint32_t rank, Stager& st, uint32_t aux, uint64_t* xfull,
+                                            uint64_t* xempty, int& xn, volatile int* abort_flag) {
+  const int nch = (tl.ntok + 31) / 32;
+  const long long ldd = p.ldd;
+  if constexpr (EPI == EPI_SWIGLU_FWD) {
+    const int pid = q & 1;
+    const bool h3_warp = q >= 2;
+    const int fw = tl.f0 + 64 * static_cast<int>(rank) + 32 * pid;
+    const int fvalid = min(32, p.Nout - fw);
+    if (fvalid <= 0) return true;   // both warps of the pair skip together
+    __nv_bfloat16* H1 = static_cast<__nv_bfloat16*>(p.D0);
+    __nv_bfloat16* H3 = static_cast<__nv_bfloat16*>(p.D1);
+    __nv_bfloat16* A = static_cast<__nv_bfloat16*>(p.D2);
+    for (int c = 0; c < nch; ++c, ++xn) {
+      const int tok = tl.tok0 + 32 * c;
+      const int rv = min(32, tl.ntok - 32 * c);
+      const long long off = static_cast<long long>(tok) * ldd + fw;
+      const int b = xn & 1;
+      const uint32_t ph = (xn >> 1) & 1;
+      const uint32_t xb = aux + (pid * 2 + b) * TN_XBUF;
+      float v[32];
+      tmem_ld32(tacc + 32 * c, v);
+      if (h3_warp) {
+        emit_t(st, lane, v, tmd(p, 1), fw, tok, H3 + off, ldd, rv, fvalid);
+        if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&xempty[pid * 2 + b]), ph ^ 1, abort_flag, p.err)))
+          return false;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) st_shared32(xb + (j * 32 + lane) * 4, __float_as_uint(v[j]));
+        mbar_arrive(smem_u32(&xfull[pid * 2 + b]));
+      } else {
+        emit_t(st, lane, v, tmd(p, 0), fw, tok, H1 + off, ldd, rv, fvalid);
+        if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&xfull[pid * 2 + b]), ph, abort_flag, p.err)))
+          return false;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float h3 = __uint_as_float(ld_shared32(xb + (j * 32 + lane) * 4));
+          v[j] = v[j] * sigmoid_fast(v[j]) * h3;
+        }
+        mbar_arrive(smem_u32(&xempty[pid * 2 + b]));
+        emit_t(st, lane, v, tmd(p, 2), fw, tok, A + off, ldd, rv, fvalid);
+      }
+    }
+  } else if constexpr (EPI == EPI_STORE_BF16) {
+    const int fw = tl.f0 + 128 * static_cast<int>(rank) + 32 * q;
+    const int fvalid = min(32, p.Nout - fw);
+    if (fvalid <= 0) return true;
+    __nv_bfloat16* D = static_cast<__nv_bfloat16*>(p.D0);
+    for (int c = 0; c < nch; ++c) {
+      const int tok = tl.tok0 + 32 * c;
+      float v[32];
+      tmem_ld32(tacc + 32 * c, v);
+      emit_t(st, lane, v, tmd(p, 0), fw, tok, D + static_cast<long long>(tok) * ldd + fw, ldd,
+             min(32, tl.ntok - 32 * c), fvalid);
+    }
+  } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+    // Accumulator = dA^T.  dH1 = dA * H3 * s * (1 + H1 (1 - s)), dH3 = dA * SiLU(H1), s = sigmoid(H1).
+    // The H1 / H3 blocks of chunk c + 1 are fetched into registers while chunk c is computed.
+    const int fw = tl.f0 + 128 * static_cast<int>(rank) + 32 * q;
+    const int fvalid = min(32, p.Nout - fw);
+    if (fvalid <= 0) return true;
+    const char* H1 = static_cast<const char*>(p.X0);
+    const char* H3 = static_cast<const char*>(p.X1);
+    __nv_bfloat16* dH1 = static_cast<__nv_bfloat16*>(p.D0);
+    __nv_bfloat16* dH3 = static_cast<__nv_bfloat16*>(p.D1);
+    const uint32_t in1 = aux + q * 2 * TN_SLAB;
+    const uint32_t in3 = in1 + TN_SLAB;
+    const int bv = min(64, fvalid * 2);
+    uint4 r1[4], r3[4];
+    {
+      const long long boff = (static_cast<long long>(tl.tok0) * ldd + fw) * 2;
+      load_t(r1, lane, H1 + boff, ldd * 2, min(32, tl.ntok), bv);
+      load_t(r3, lane, H3 + boff, ldd * 2, min(32, tl.ntok), bv);
+    }
+    for (int c = 0; c < nch; ++c) {
+      const int tok = tl.tok0 + 32 * c;
+      const int rv = min(32, tl.ntok - 32 * c);
+      __syncwarp();
+      put_t(in1, lane, r1);
+      put_t(in3, lane, r3);
+      if (c + 1 < nch) {
+        const long long boff = (static_cast<long long>(tok + 32) * ldd + fw) * 2;
+        load_t(r1, lane, H1 + boff, ldd * 2, min(32, tl.ntok - 32 * (c + 1)), bv);
+        load_t(r3, lane, H3 + boff, ldd * 2, min(32, tl.ntok - 32 * (c + 1)), bv);
+      }
+      __syncwarp();
+      float da[32], h1[32], h3[32];
+      stage_t_read(in1, lane, h1);
+      stage_t_read(in3, lane, h3);
+      tmem_ld32(tacc + 32 * c, da);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float s = sigmoid_fast(h1[i]);
+        const float d1 = da[i] * h3[i] * s * (1.0f + h1[i] * (1.0f - s));
+        h1[i] = da[i] * h1[i] * s;
+        da[i] = d1;
+      }
+      const long long off = static_cast<long long>(tok) * ldd + fw;
+      emit_t(st, lane, da, tmd(p, 0), fw, tok, dH1 + off, ldd, rv, fvalid);
+      emit_t(st, lane, h1, tmd(p, 1), fw, tok, dH3 + off, ldd, rv, fvalid);
+    }
+  }
+  return true;
+}
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    grouped_gemm_tn_kernel(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages;
+  constexpr uint32_t stage_bytes = A_BYTES + 128 * BK * 2;   // 128 weight rows + 128 token rows
+  uint8_t* stage_area = smem + S * stage_bytes;               // 4 warps x 2 staging slabs
+  uint8_t* aux_area = stage_area + 4 * 2 * TN_SLAB;
+  int* pair_off = reinterpret_cast<int*>(aux_area + tn_aux_bytes(EPI));
+  const int poff_ints = (p.G + 1 + 63) & ~63;
+  uint8_t* bar_area = reinterpret_cast<uint8_t*>(pair_off + poff_ints);
+  uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
+  uint64_t* empty = full + MAX_STAGES;
+  uint64_t* acc_full = empty + MAX_STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint64_t* xfull = drain + 1;
+  uint64_t* xempty = xfull + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xempty + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  constexpr uint32_t tmem_cols = 2 * TN_TOK;   // two 256-column accumulators
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&acc_full[b]), 1);
+      mbar_init(smem_u32(&acc_empty[b]), 2 * 4 * 32);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(smem_u32(&xfull[i]), 32);
+      mbar_init(smem_u32(&xempty[i]), 32);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  // Prefix over experts of ceil(n_g / 256) token tiles (from the 128-row tile prefix).
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < p.G; base += 32) {
+      const int e = base + lane;
+      const int np = e < p.G ? (p.tiles[e + 1] - p.tiles[e] + 1) / 2 : 0;
+      int x = np;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (e < p.G) pair_off[e] = carry + x - np;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) pair_off[p.G] = carry;
+    if (lane == 0) {
+      prefetch_tmap(&p.tmA[0]);
+      prefetch_tmap(&p.tmB[0]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc2(smem_u32(tmem_slot), tmem_cols);
+    tmem_relinquish2();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      uint32_t pending = 0, pend_parity = 0;
+      int it = 0;
+      bool ok = true;
+      TnCursor cur{kTnUnitOrder ? pair : 0, 0, pair};
+      TnTile tl;
+      while (ok && tn_next(p, pair_off, npairs, cur, tl)) {
+        const int half = tl.nmma / 2;                                     // token columns per CTA
+        const int tokc = tl.tok0 + static_cast<int>(rank) * half;
+        const int nb32 = (!kTnRaggedBoxes || half == 128) ? 0 : (half + 31) / 32;
+        const uint32_t tx = 2 * (A_BYTES + (nb32 ? nb32 * 32 : 128) * BK * 2);
+        for (int kb = 0; kb < tl.nk; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!wait_bar2(smem_u32(&empty[s]), ph ^ 1, abort_flag, p.err)) { ok = false; break; }
+          const uint32_t fb_local = smem_u32(&full[s]);
+          if (leader) mbar_expect_tx(fb_local, tx);
+          const uint32_t fb = mapa_shared(fb_local, 0);
+          const uint32_t sa = smem_u32(smem + s * stage_bytes);
+          const uint32_t sb = sa + A_BYTES;
+          const int src = kb < p.k0_blocks ? 0 : 1;
+          const int kk = (src == 0 ? kb : kb - p.k0_blocks) * BK;
+          if (p.a_major) {
+            if (p.nsplit) {
+              const int f = tl.f0 + 64 * static_cast<int>(rank);
+              tma_load_3d_pair(sa, &p.tmA[0], fb, f, kk, tl.g);
+              tma_load_3d_pair(sa + BOX_BYTES, &p.tmA[1], fb, f, kk, tl.g);
+            } else {
+              const int f = tl.f0 + 128 * static_cast<int>(rank);
+              if (p.a_merged) {
+                tma_load_4d_pair(sa, &p.tmA[src], fb, 0, kk, f / 64, tl.g);
+              } else {
+                tma_load_3d_pair(sa, &p.tmA[src], fb, f, kk, tl.g);
+                tma_load_3d_pair(sa + BOX_BYTES, &p.tmA[src], fb, f + 64, kk, tl.g);
+              }
+            }
+          } else {
+            tma_load_3d_pair(sa, &p.tmA[src], fb, kk, tl.f0 + 128 * static_cast<int>(rank), tl.g);
+          }
+          const int bsrc = p.nsplit ? 0 : src;
+          if (nb32 == 0) {
+            tma_load_3d_pair(sb, &p.tmB[bsrc], fb, kk, tokc, 0);
+          } else {
+            for (int j = 0; j < nb32; ++j) tma_load_3d_pair(sb + j * 32 * 128, &p.tmB32[bsrc], fb, kk, tokc + 32 * j, 0);
+          }
+          pending |= 1u << s;
+          pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
+        }
+      }
+      // Drain: a stage's empty barrier completes only after the MMA consumed it, so its loads landed.
+      for (int s = 0; s < S; ++s)
+        if (pending & (1u << s))
+          wait_bar2(smem_u32(&empty[s]), (pend_parity >> s) & 1, abort_flag, p.err, false);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (leader) {
+      const uint32_t a_lbo = p.a_major ? BOX_BYTES : 16;
+      const uint32_t a_step = p.a_major ? 2048 : 32;
+      int it = 0, tcount = 0;
+      bool ok = true;
+      TnCursor cur{kTnUnitOrder ? pair : 0, 0, pair};
+      TnTile tl;
+      for (; ok && tn_next(p, pair_off, npairs, cur, tl); ++tcount) {
+        const uint32_t idesc = idesc_bf16(2 * BM, tl.nmma, p.a_major, 0);
+        const int buf = tcount & 1;
+        const uint32_t aph = (tcount >> 1) & 1;
+        ok = __all_sync(0xffffffffu, wait_bar2(smem_u32(&acc_empty[buf]), aph ^ 1, abort_flag, p.err));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tmem_d = tmem_base + buf * TN_TOK;
+        for (int kb = 0; kb < tl.nk; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          ok = __all_sync(0xffffffffu, wait_bar2(smem_u32(&full[s]), ph, abort_flag, p.err));
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * stage_bytes);
+          const uint32_t sb = sa + A_BYTES;
+          if (lane == 0) {
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = sdesc(sa + kk * a_step, a_lbo, 1024);
+              const uint64_t bd = sdesc(sb + kk * 32, 16, 1024);
+              tc_mma2(tmem_d, ad, bd, idesc, (kb | kk) != 0);
+            }
+            tc_commit2_both(smem_u32(&empty[s]));
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        if (lane == 0) tc_commit2_both(smem_u32(&acc_full[buf]));   // also for nk == 0 (zero tile)
+        __syncwarp();
+      }
+      if (lane == 0) {
+        tc_commit2_both(smem_u32(drain));
+        wait_bar2(smem_u32(drain), 0, abort_flag, p.err, false);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
+    const uint32_t acc_empty_leader1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
+    Stager stg{smem_u32(stage_area + q * 2 * TN_SLAB), 0};
+    const uint32_t aux = smem_u32(aux_area);
+    int tcount = 0, xn = 0;
+    TnCursor cur{kTnUnitOrder ? pair : 0, 0, pair};
+    TnTile tl;
+    for (; tn_next(p, pair_off, npairs, cur, tl); ++tcount) {
+      const int buf = tcount & 1;
+      const uint32_t aph = (tcount >> 1) & 1;
+      if (!__all_sync(0xffffffffu, wait_bar2(smem_u32(&acc_full[buf]), aph, abort_flag, p.err))) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * TN_TOK;
+      const bool ok = epilogue_tn<EPI>(p, tl, tacc, q, lane, rank, stg, aux, xfull, xempty, xn, abort_flag);
+      tc_fence_before();
+      mbar_arrive_cluster(buf ? acc_empty_leader1 : acc_empty_leader0);
+      if (!ok) break;
     }
     emit_drain(lane);
   }
@@ -1316,9 +1976,13 @@ static int max_pairs() {
   return cached;
 }
 
-template <int EPI>
+template <int EPI, int MODE = RG>
 static int launch2(Params& p, long long pair_tile_upper_bound, const char* name, cudaStream_t stream) {
-  p.mode = RG;
+  p.mode = MODE;
+  // Each CTA loads bn/2 B columns: in 64-column boxes (MN-major), or rows of a bn/2-row box (K-major),
+  // and the stage's expected byte count assumes exactly that.
+  if (p.bn % 128 != 0 || p.bn > 256)
+    return fail(PFMOE_ERR_UNSUPPORTED, std::string(name) + ": two-SM tiles need bn in {128, 256}");
   const int stage = A_BYTES + (p.bn / 2) * BK * 2;
   const int poff = p.tiles ? ((p.G + 1 + 63) & ~63) * 4 : 0;
   const int fixed = 1024 + 256 + poff + (kStaged2sm ? 4 * STAGE_BUFS * STAGE_BYTES_PER_WARP : 0);
@@ -1327,7 +1991,7 @@ static int launch2(Params& p, long long pair_tile_upper_bound, const char* name,
   const size_t smem = fixed + static_cast<size_t>(p.stages) * stage;
   static bool attr_done = false;
   if (!attr_done) {
-    if (cudaFuncSetAttribute(grouped_gemm_2sm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(grouped_gemm_2sm_kernel<EPI, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(227 * 1024)) != cudaSuccess)
       return fail(PFMOE_ERR_CUDA, std::string("cudaFuncSetAttribute failed: ") +
                                       cudaGetErrorString(cudaGetLastError()));
@@ -1337,9 +2001,47 @@ static int launch2(Params& p, long long pair_tile_upper_bound, const char* name,
   long long pairs = max_pairs();
   if (pair_tile_upper_bound < pairs) pairs = pair_tile_upper_bound;
   PFMOE_LAUNCH(name, stream,
-               (grouped_gemm_2sm_kernel<EPI><<<static_cast<int>(2 * pairs), THREADS, smem, stream>>>(p)));
+               (grouped_gemm_2sm_kernel<EPI, MODE><<<static_cast<int>(2 * pairs), THREADS, smem, stream>>>(p)));
   return PFMOE_OK;
 }
+
+// Token-as-N launcher (expert-segmented rows only).
+template <int EPI>
+static int launch_tn(Params& p, long long pair_tile_upper_bound, const char* name, cudaStream_t stream) {
+  p.mode = RG;
+  const int stage = A_BYTES + 128 * BK * 2;
+  const int poff = ((p.G + 1 + 63) & ~63) * 4;
+  const int fixed = 1024 + 512 + poff + 4 * 2 * TN_SLAB + tn_aux_bytes(EPI);
+  const int st = (SMEM_LIMIT - fixed) / stage;
+  if (st < 2) return fail(PFMOE_ERR_UNSUPPORTED, std::string(name) + ": too many experts for the shared-memory plan");
+  p.stages = st > MAX_STAGES ? MAX_STAGES : st;
+  const size_t smem = fixed + static_cast<size_t>(p.stages) * stage;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(grouped_gemm_tn_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(227 * 1024)) != cudaSuccess)
+      return fail(PFMOE_ERR_CUDA, std::string("cudaFuncSetAttribute failed: ") +
+                                      cudaGetErrorString(cudaGetLastError()));
+    attr_done = true;
+  }
+  if (pair_tile_upper_bound <= 0) return PFMOE_OK;
+  long long pairs = max_pairs();
+  if (pair_tile_upper_bound < pairs) pairs = pair_tile_upper_bound;
+  PFMOE_LAUNCH(name, stream,
+               (grouped_gemm_tn_kernel<EPI><<<static_cast<int>(2 * pairs), THREADS, smem, stream>>>(p)));
+  return PFMOE_OK;
+}
+
+// Token-tile upper bound of the token-as-N kernel: sum_e ceil(n_e / 256) <= N / 256 + E.
+static long long tn_tiles_ub(int N, int E, int F, int fstep) {
+  return (static_cast<long long>(N) / TN_TOK + E + 1) * ((F + fstep - 1) / fstep);
+}
+
+// Row-grouped expert GEMMs run on the token-as-N kernel (no spare rows on ragged segments).
+constexpr bool kTokenAsN = true;
+// Expert weight gradients run on the two-SM kernel (256-row output tiles: 1.5x fewer operand
+// bytes per FLOP than one-SM 128-row tiles).
+constexpr bool kPairWgrad = false;
 
 // Pair-tile upper bound: sum_e ceil(n_e / 256) <= N / 256 + E.
 static long long rg_pairs_ub(int N, int E, int Nout, int nstep) {
@@ -1421,6 +2123,19 @@ int tc_ffn_gemm1(const void* x_pft, const int* seg, const int* tiles, int N, int
   p.k0_blocks = (d + BK - 1) / BK;
   p.seg = seg; p.tiles = tiles; p.G = E;
   p.D0 = h1; p.D1 = h3; p.D2 = a; p.ldd = h;
+  if (kTokenAsN) {
+    p.a_major = 1;            // W1_e, W3_e [d, h]: K rows, features contiguous
+    p.fstep = 128;            // 64 features of W1 and the same 64 of W3 per CTA
+    PFMOE_TRY(make_tmap(&p.tmA[0], w1, h, d, E, 64, 64, "w1"));
+    PFMOE_TRY(make_tmap(&p.tmA[1], w3, h, d, E, 64, 64, "w3"));
+    PFMOE_TRY(make_tmap(&p.tmB[0], x_pft, d, N, 1, BK, 128, "x_pft"));
+    PFMOE_TRY(make_tmap(&p.tmB32[0], x_pft, d, N, 1, BK, 32, "x_pft"));
+    PFMOE_TRY(make_out_map_tn(&p.tmD[0], h1, h, N, "h1 out"));
+    PFMOE_TRY(make_out_map_tn(&p.tmD[1], h3, h, N, "h3 out"));
+    PFMOE_TRY(make_out_map_tn(&p.tmD[2], a, h, N, "a out"));
+    p.tma_store = 1;
+    return launch_tn<EPI_SWIGLU_FWD>(p, tn_tiles_ub(N, E, h, p.fstep), "ffn_gemm1_swiglu", s);
+  }
   PFMOE_TRY(make_tmap(&p.tmA[0], x_pft, d, N, 1, BK, BM, "x_pft"));
   PFMOE_TRY(make_tmap(&p.tmB[0], w1, h, d, E, 64, 64, "w1"));
   PFMOE_TRY(make_tmap(&p.tmB[1], w3, h, d, E, 64, 64, "w3"));
@@ -1444,6 +2159,18 @@ int tc_ffn_gemm2(const void* a, const int* seg, const int* tiles, int N, int E, 
   p.k0_blocks = (h + BK - 1) / BK;
   p.seg = seg; p.tiles = tiles; p.G = E;
   p.D0 = out; p.ldd = d;
+  if (kTokenAsN) {
+    p.a_major = 1;            // W2_e [h, d]: K rows, features contiguous
+    p.fstep = 2 * BM;
+    p.a_merged = d % 64 == 0;
+    if (p.a_merged) PFMOE_TRY(make_tmap_mn(&p.tmA[0], w2, d, h, E, BK, 2, "w2"));
+    else PFMOE_TRY(make_tmap(&p.tmA[0], w2, d, h, E, 64, 64, "w2"));
+    PFMOE_TRY(make_tmap(&p.tmB[0], a, h, N, 1, BK, 128, "a"));
+    PFMOE_TRY(make_tmap(&p.tmB32[0], a, h, N, 1, BK, 32, "a"));
+    PFMOE_TRY(make_out_map_tn(&p.tmD[0], out, d, N, "out"));
+    p.tma_store = 1;
+    return launch_tn<EPI_STORE_BF16>(p, tn_tiles_ub(N, E, d, p.fstep), "ffn_gemm2", s);
+  }
   PFMOE_TRY(make_tmap(&p.tmA[0], a, h, N, 1, BK, BM, "a"));
   PFMOE_TRY(make_tmap(&p.tmB[0], w2, d, h, E, 64, 64, "w2"));
   if (use_pairs(N, E)) {
@@ -1464,6 +2191,17 @@ int tc_ffn_dgrad_act(const void* dO, const int* seg, const int* tiles, int N, in
   p.k0_blocks = (d + BK - 1) / BK;
   p.seg = seg; p.tiles = tiles; p.G = E;
   p.X0 = h1; p.X1 = h3; p.D0 = dh1; p.D1 = dh3; p.ldd = h;
+  if (kTokenAsN) {
+    p.a_major = 0;            // W2_e [h, d]: feature rows, K = d contiguous
+    p.fstep = 2 * BM;
+    PFMOE_TRY(make_tmap(&p.tmA[0], w2, d, h, E, BK, 128, "w2^T"));
+    PFMOE_TRY(make_tmap(&p.tmB[0], dO, d, N, 1, BK, 128, "dO"));
+    PFMOE_TRY(make_tmap(&p.tmB32[0], dO, d, N, 1, BK, 32, "dO"));
+    PFMOE_TRY(make_out_map_tn(&p.tmD[0], dh1, h, N, "dh1 out"));
+    PFMOE_TRY(make_out_map_tn(&p.tmD[1], dh3, h, N, "dh3 out"));
+    p.tma_store = 1;
+    return launch_tn<EPI_SWIGLU_BWD>(p, tn_tiles_ub(N, E, h, p.fstep), "ffn_dgrad_act_swiglu_bwd", s);
+  }
   const bool pairs = use_pairs(N, E);
   const uint32_t brows = pairs ? p.bn / 2 : p.bn;   // B rows loaded per CTA
   PFMOE_TRY(make_tmap(&p.tmA[0], dO, d, N, 1, BK, BM, "dO"));
@@ -1488,6 +2226,19 @@ int tc_ffn_dgrad_x(const void* dh1, const void* dh3, const int* seg, const int* 
   p.k1_blocks = (h + BK - 1) / BK;
   p.seg = seg; p.tiles = tiles; p.G = E;
   p.D0 = dx_pft; p.ldd = d;
+  if (kTokenAsN) {
+    p.a_major = 0;            // W1_e, W3_e [d, h]: feature rows, K = h contiguous
+    p.fstep = 2 * BM;
+    PFMOE_TRY(make_tmap(&p.tmA[0], w1, h, d, E, BK, 128, "w1^T"));
+    PFMOE_TRY(make_tmap(&p.tmA[1], w3, h, d, E, BK, 128, "w3^T"));
+    PFMOE_TRY(make_tmap(&p.tmB[0], dh1, h, N, 1, BK, 128, "dh1"));
+    PFMOE_TRY(make_tmap(&p.tmB[1], dh3, h, N, 1, BK, 128, "dh3"));
+    PFMOE_TRY(make_tmap(&p.tmB32[0], dh1, h, N, 1, BK, 32, "dh1"));
+    PFMOE_TRY(make_tmap(&p.tmB32[1], dh3, h, N, 1, BK, 32, "dh3"));
+    PFMOE_TRY(make_out_map_tn(&p.tmD[0], dx_pft, d, N, "dx_pft out"));
+    p.tma_store = 1;
+    return launch_tn<EPI_STORE_BF16>(p, tn_tiles_ub(N, E, d, p.fstep), "ffn_dgrad_x", s);
+  }
   const bool pairs = use_pairs(N, E);
   const uint32_t brows = pairs ? p.bn / 2 : p.bn;   // B rows loaded per CTA
   PFMOE_TRY(make_tmap(&p.tmA[0], dh1, h, N, 1, BK, BM, "dh1"));
@@ -1513,12 +2264,25 @@ int tc_ffn_wgrad13(const void* x_pft, const void* dh1, const void* dh3, const in
   p.Nout = h;
   p.seg = seg; p.G = E;
   p.D0 = dw1; p.D1 = dw3; p.ldd = h; p.d_gstride = static_cast<long long>(d) * h;
-  PFMOE_TRY(make_tmap(&p.tmA[0], x_pft, d, N, 1, 64, 64, "x_pft^T"));
-  PFMOE_TRY(make_tmap(&p.tmB[0], dh1, h, N, 1, 64, 64, "dh1"));
-  PFMOE_TRY(make_tmap(&p.tmB[1], dh3, h, N, 1, 64, 64, "dh3"));
+  p.a_merged = d % 64 == 0;
+  p.b_merged = h % 64 == 0;
+  const uint32_t bblk = (p.bn / 2) / 64;   // 64-wide blocks of dH1 (and of dH3) per tile
+  if (p.a_merged) PFMOE_TRY(make_tmap_mn(&p.tmA[0], x_pft, d, N, 1, BK, 2, "x_pft^T"));
+  else PFMOE_TRY(make_tmap(&p.tmA[0], x_pft, d, N, 1, 64, 64, "x_pft^T"));
+  if (p.b_merged) {
+    PFMOE_TRY(make_tmap_mn(&p.tmB[0], dh1, h, N, 1, BK, bblk, "dh1"));
+    PFMOE_TRY(make_tmap_mn(&p.tmB[1], dh3, h, N, 1, BK, bblk, "dh3"));
+  } else {
+    PFMOE_TRY(make_tmap(&p.tmB[0], dh1, h, N, 1, 64, 64, "dh1"));
+    PFMOE_TRY(make_tmap(&p.tmB[1], dh3, h, N, 1, 64, 64, "dh3"));
+  }
   PFMOE_TRY(make_out_map(&p.tmD[0], dw1, h, d, E, "dw1 out"));
   PFMOE_TRY(make_out_map(&p.tmD[1], dw3, h, d, E, "dw3 out"));
   p.tma_store = 1;
+  if (kPairWgrad) {
+    const long long ub = static_cast<long long>(E) * ((d + 2 * BM - 1) / (2 * BM)) * ((h + p.bn / 2 - 1) / (p.bn / 2));
+    return launch2<EPI_SPLIT_BF16, KG>(p, ub, "ffn_wgrad_w1w3", s);
+  }
   const long long ub = static_cast<long long>(E) * ((d + BM - 1) / BM) * ((h + p.bn / 2 - 1) / (p.bn / 2));
   return launch<EPI_SPLIT_BF16, KG>(p, ub, "ffn_wgrad_w1w3", s);
 }
@@ -1528,15 +2292,25 @@ int tc_ffn_wgrad2(const void* a, const void* dO, const int* seg, int N, int E, i
   Params p = base_params(err);
   p.mode = KG;
   p.b_major = 1;
-  p.bn = round_bn(d);
+  p.bn = kPairWgrad ? round_bn_pair(d) : round_bn(d);
   p.M = h;
   p.Nout = d;
   p.seg = seg; p.G = E;
   p.D0 = dw2; p.ldd = d; p.d_gstride = static_cast<long long>(h) * d;
-  PFMOE_TRY(make_tmap(&p.tmA[0], a, h, N, 1, 64, 64, "a^T"));
-  PFMOE_TRY(make_tmap(&p.tmB[0], dO, d, N, 1, 64, 64, "dO"));
+  p.a_merged = h % 64 == 0;
+  p.b_merged = d % 64 == 0;
+  // one-SM tiles load all bn columns of B; two-SM tiles bn / 2 per CTA
+  const uint32_t bblk2 = (kPairWgrad ? p.bn / 2 : p.bn) / 64;
+  if (p.a_merged) PFMOE_TRY(make_tmap_mn(&p.tmA[0], a, h, N, 1, BK, 2, "a^T"));
+  else PFMOE_TRY(make_tmap(&p.tmA[0], a, h, N, 1, 64, 64, "a^T"));
+  if (p.b_merged) PFMOE_TRY(make_tmap_mn(&p.tmB[0], dO, d, N, 1, BK, bblk2, "dO"));
+  else PFMOE_TRY(make_tmap(&p.tmB[0], dO, d, N, 1, 64, 64, "dO"));
   PFMOE_TRY(make_out_map(&p.tmD[0], dw2, d, h, E, "dw2 out"));
   p.tma_store = 1;
+  if (kPairWgrad) {
+    const long long ub = static_cast<long long>(E) * ((h + 2 * BM - 1) / (2 * BM)) * ((d + p.bn - 1) / p.bn);
+    return launch2<EPI_STORE_BF16, KG>(p, ub, "ffn_wgrad_w2", s);
+  }
   const long long ub = static_cast<long long>(E) * ((h + BM - 1) / BM) * ((d + p.bn - 1) / p.bn);
   return launch<EPI_STORE_BF16, KG>(p, ub, "ffn_wgrad_w2", s);
 }
