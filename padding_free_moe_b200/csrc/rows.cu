@@ -1,9 +1,11 @@
 // Row-movement kernels of the padding-free layer: dispatch (PFT.x), combine,
 // combine backward, token-gradient gather-sum with the gate's backward, and a
-// small transpose.  All are HBM-bound: one warp owns one token and moves its
-// rows with 16-byte vector loads/stores, so every warp access is a coalesced
-// 512-byte run of one row.  Nothing uses atomics; every sum runs over the k
-// slots in slot order, so results are deterministic.
+// small transpose.  All are HBM-bound and move rows with 16-byte vector
+// loads/stores, so every warp access is a coalesced 512-byte run of one row
+// (BF16).  Dispatch gives a warp one token; the gather-sums give a warp one
+// (token, column chunk) or one PFT row, which keeps many more row loads in
+// flight.  Nothing uses atomics; every sum runs over the k slots in slot
+// order, so results are deterministic.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -18,6 +20,9 @@ inline int token_grid(long long T) {
   if (b > cap) b = cap;
   return static_cast<int>(b < 1 ? 1 : b);
 }
+
+// Grid for `items` one-warp work items (grid-stride beyond 16 blocks of 8 warps per SM).
+inline int item_grid(long long items) { return token_grid(items); }
 
 // Lane j < k loads pos[t, j]; returns false (and flags) if any row index is out of range.
 __device__ __forceinline__ bool load_pos(const int32_t* pos, long long t, int k, long long N, int lane, int& my_pos,
@@ -65,51 +70,50 @@ __global__ void __launch_bounds__(WARPS * 32) dispatch_kernel(const T* __restric
   }
 }
 
-// y[t] = sum_j w[t, j] * O[pos[t, j]] in slot order, float32 accumulation, one rounding.
-// Each lane carries U 16-byte column chunks so that U*k row loads are in flight per warp.
-template <typename T, int U>
+// The gather-sum kernels below take one work item per warp: a (token, column chunk) pair, the
+// chunk being the 32 * VN columns one warp covers with one 16-byte vector per lane.  Every lane
+// then has all k row loads of its chunk in flight at once, and a token's chunks sit on
+// neighbouring warps (its pos / weight rows stay in L1).  Sums still run over the k slots in
+// slot order with float32 accumulation, so results do not depend on the launch shape.
+template <typename T>
+__host__ __device__ inline int chunk_cols() { return 32 * Vec<T>::n; }
+
+// y[t] = sum_j w[t, j] * O[pos[t, j]].
+template <typename T>
 __global__ void __launch_bounds__(WARPS * 32) combine_kernel(const T* __restrict__ O, const int32_t* __restrict__ pos,
                                                              const float* __restrict__ w, int Tn, int k, int d,
                                                              T* __restrict__ y, int32_t* err) {
   constexpr int VN = Vec<T>::n;
   const int lane = threadIdx.x & 31;
-  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   const long long N = static_cast<long long>(Tn) * k;
-  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < Tn; t += nw) {
+  const int C = (d + chunk_cols<T>() - 1) / chunk_cols<T>();
+  const long long items = static_cast<long long>(Tn) * C;
+  for (long long it = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; it < items; it += nw) {
+    const long long t = it / C;
+    const int c0 = static_cast<int>(it - t * C) * chunk_cols<T>() + lane * VN;
     int my_pos;
     if (!load_pos(pos, t, k, N, lane, my_pos, err)) continue;
-    const float my_w = lane < k ? w[static_cast<long long>(t) * k + lane] : 0.f;
-    for (int base = 0; base < d; base += 32 * VN * U) {   // warp-uniform trip count
-      float acc[U][VN];
+    const float my_w = lane < k ? w[t * k + lane] : 0.f;
+    float acc[VN];
 #pragma unroll
-      for (int u = 0; u < U; ++u)
+    for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < k; ++j) {
+      const long long p = __shfl_sync(0xffffffffu, my_pos, j);
+      const float wj = __shfl_sync(0xffffffffu, my_w, j);
+      if (c0 < d) {
+        float o[VN];
+        load16(O + p * d + c0, o);
 #pragma unroll
-        for (int i = 0; i < VN; ++i) acc[u][i] = 0.f;
-#pragma unroll 4
-      for (int j = 0; j < k; ++j) {
-        const long long p = __shfl_sync(0xffffffffu, my_pos, j);
-        const float wj = __shfl_sync(0xffffffffu, my_w, j);
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int c0 = base + (u * 32 + lane) * VN;
-          if (c0 < d) {
-            float o[VN];
-            load16(O + p * d + c0, o);
-#pragma unroll
-            for (int i = 0; i < VN; ++i) acc[u][i] = fmaf(wj, o[i], acc[u][i]);
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int c0 = base + (u * 32 + lane) * VN;
-        if (c0 < d) store16(y + static_cast<long long>(t) * d + c0, acc[u]);
+        for (int i = 0; i < VN; ++i) acc[i] = fmaf(wj, o[i], acc[i]);
       }
     }
+    if (c0 < d) store16(y + t * d + c0, acc);
   }
 }
 
-// dO[pos[t, j]] = w[t, j] * dY[t];  g[t, j] = <dY[t], O[pos[t, j]]>.
+// One warp per PFT row r = (t, j): dO[pos[t, j]] = w[t, j] * dY[t];  g[t, j] = <dY[t], O[pos[t, j]]>.
 template <typename T>
 __global__ void __launch_bounds__(WARPS * 32) combine_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ O,
                                                                  const int32_t* __restrict__ pos,
@@ -118,36 +122,40 @@ __global__ void __launch_bounds__(WARPS * 32) combine_bwd_kernel(const T* __rest
                                                                  int32_t* err) {
   constexpr int VN = Vec<T>::n;
   const int lane = threadIdx.x & 31;
-  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   const long long N = static_cast<long long>(Tn) * k;
-  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < Tn; t += nw) {
-    int my_pos;
-    if (!load_pos(pos, t, k, N, lane, my_pos, err)) continue;
-    const float my_w = lane < k ? w[static_cast<long long>(t) * k + lane] : 0.f;
-    const T* dyr = dy + static_cast<long long>(t) * d;
-    for (int j = 0; j < k; ++j) {
-      const long long p = __shfl_sync(0xffffffffu, my_pos, j);
-      const float wj = __shfl_sync(0xffffffffu, my_w, j);
-      float part = 0.f;
-      for (int c0 = lane * VN; c0 < d; c0 += 32 * VN) {
-        float a[VN], o[VN];
-        load16(dyr + c0, a);
-        load16(O + p * d + c0, o);
-#pragma unroll
-        for (int i = 0; i < VN; ++i) {
-          part = fmaf(a[i], o[i], part);
-          a[i] *= wj;
-        }
-        store16(dO + p * d + c0, a);
-      }
-      part = warp_sum(part);
-      if (lane == 0) g[static_cast<long long>(t) * k + j] = part;
+  for (long long r = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < N; r += nw) {
+    const long long t = r / k;
+    const long long p = pos[r];
+    if (p < 0 || p >= N) {
+      if (lane == 0) dev_error(err, PFMOE_DEV_BAD_POS);
+      continue;
     }
+    const float wj = w[r];
+    const T* dyr = dy + t * d;
+    const T* orow = O + p * d;
+    T* drow = dO + p * d;
+    float part = 0.f;
+#pragma unroll 2
+    for (int c0 = lane * VN; c0 < d; c0 += 32 * VN) {
+      float a[VN], o[VN];
+      load16(dyr + c0, a);
+      load16(orow + c0, o);
+#pragma unroll
+      for (int i = 0; i < VN; ++i) {
+        part = fmaf(a[i], o[i], part);
+        a[i] *= wj;
+      }
+      store16(drow + c0, a);
+    }
+    part = warp_sum(part);
+    if (lane == 0) g[r] = part;
   }
 }
 
 // dz_{t, ids[t,j]} = w_j (g_j - sum_l w_l g_l) (zero elsewhere);
 // dx[t] = sum_j dX_pft[pos[t, j]] + sum_j dz_j * Wg^T[ids[t, j]].
+// The dense dlogits row (and its BF16 copy for the dWg GEMM) is written by the token's chunk-0 item.
 template <typename T>
 __global__ void __launch_bounds__(WARPS * 32) token_grad_kernel(const T* __restrict__ dxp, const int32_t* __restrict__ pos,
                                                                 const float* __restrict__ g, const float* __restrict__ w,
@@ -157,12 +165,17 @@ __global__ void __launch_bounds__(WARPS * 32) token_grad_kernel(const T* __restr
                                                                 __nv_bfloat16* __restrict__ dz_bf16, int32_t* err) {
   constexpr int VN = Vec<T>::n;
   const int lane = threadIdx.x & 31;
-  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   const long long N = static_cast<long long>(Tn) * k;
-  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < Tn; t += nw) {
+  const int C = (d + chunk_cols<T>() - 1) / chunk_cols<T>();
+  const long long items = static_cast<long long>(Tn) * C;
+  for (long long it = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; it < items; it += nw) {
+    const long long t = it / C;
+    const int ch = static_cast<int>(it - t * C);
+    const int c0 = ch * chunk_cols<T>() + lane * VN;
     int my_pos;
     if (!load_pos(pos, t, k, N, lane, my_pos, err)) continue;
-    const long long tk = static_cast<long long>(t) * k;
+    const long long tk = t * k;
     const float my_w = lane < k ? w[tk + lane] : 0.f;
     const float my_g = lane < k ? g[tk + lane] : 0.f;
     int my_id = lane < k ? ids[tk + lane] : 0;
@@ -172,49 +185,47 @@ __global__ void __launch_bounds__(WARPS * 32) token_grad_kernel(const T* __restr
     }
     const float inner = warp_sum(my_w * my_g);
     const float my_dz = lane < k ? my_w * (my_g - inner) : 0.f;
-    // dense dlogits row (and its BF16 copy for the dWg GEMM)
-    for (int e0 = 0; e0 < E; e0 += 32) {
-      const int e = e0 + lane;
-      float val = 0.f;
-      for (int j = 0; j < k; ++j) {
-        const int idj = __shfl_sync(0xffffffffu, my_id, j);
-        const float dzj = __shfl_sync(0xffffffffu, my_dz, j);
-        if (idj == e) val = dzj;
-      }
-      if (e < E) {
-        dlogits[static_cast<long long>(t) * E + e] = val;
-        if (dz_bf16) dz_bf16[static_cast<long long>(t) * E + e] = __float2bfloat16_rn(val);
-      }
-    }
-    for (int base = 0; base < d; base += 32 * VN) {   // warp-uniform trip count
-      const int c0 = base + lane * VN;
-      const bool act = c0 < d;
-      float acc[VN];
-#pragma unroll
-      for (int i = 0; i < VN; ++i) acc[i] = 0.f;
-#pragma unroll 4
-      for (int j = 0; j < k; ++j) {
-        const long long p = __shfl_sync(0xffffffffu, my_pos, j);
-        if (act) {
-          float v[VN];
-          load16(dxp + p * d + c0, v);
-#pragma unroll
-          for (int i = 0; i < VN; ++i) acc[i] += v[i];
+    if (ch == 0) {
+      for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        float val = 0.f;
+        for (int j = 0; j < k; ++j) {
+          const int idj = __shfl_sync(0xffffffffu, my_id, j);
+          const float dzj = __shfl_sync(0xffffffffu, my_dz, j);
+          if (idj == e) val = dzj;
+        }
+        if (e < E) {
+          dlogits[t * E + e] = val;
+          if (dz_bf16) dz_bf16[t * E + e] = __float2bfloat16_rn(val);
         }
       }
-#pragma unroll 4
-      for (int j = 0; j < k; ++j) {
-        const long long idj = __shfl_sync(0xffffffffu, my_id, j);
-        const float dzj = __shfl_sync(0xffffffffu, my_dz, j);
-        if (act) {
-          float v[VN];
-          load16(wgT + idj * d + c0, v);
-#pragma unroll
-          for (int i = 0; i < VN; ++i) acc[i] = fmaf(dzj, v[i], acc[i]);
-        }
-      }
-      if (act) store16(dx + static_cast<long long>(t) * d + c0, acc);
     }
+    const bool act = c0 < d;
+    float acc[VN];
+#pragma unroll
+    for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < k; ++j) {
+      const long long p = __shfl_sync(0xffffffffu, my_pos, j);
+      if (act) {
+        float v[VN];
+        load16(dxp + p * d + c0, v);
+#pragma unroll
+        for (int i = 0; i < VN; ++i) acc[i] += v[i];
+      }
+    }
+#pragma unroll 8
+    for (int j = 0; j < k; ++j) {
+      const long long idj = __shfl_sync(0xffffffffu, my_id, j);
+      const float dzj = __shfl_sync(0xffffffffu, my_dz, j);
+      if (act) {
+        float v[VN];
+        load16(wgT + idj * d + c0, v);
+#pragma unroll
+        for (int i = 0; i < VN; ++i) acc[i] = fmaf(dzj, v[i], acc[i]);
+      }
+    }
+    if (act) store16(dx + t * d + c0, acc);
   }
 }
 
@@ -253,14 +264,15 @@ int launch_dispatch(const void* x, const int32_t* pos, int T, int k, int d, int 
 
 int launch_combine(const void* out, const int32_t* pos, const float* w, int T, int k, int d, int dtype, void* y,
                    int32_t* err, cudaStream_t s) {
-  const int g = token_grid(T);
+  const int vn = dtype == PFMOE_BF16 ? 8 : 4;
+  const int g = item_grid(static_cast<long long>(T) * ((d + 32 * vn - 1) / (32 * vn)));
   if (dtype == PFMOE_BF16) {
     PFMOE_LAUNCH("combine", s,
-                 combine_kernel<__nv_bfloat16, 2><<<g, WARPS * 32, 0, s>>>(
+                 combine_kernel<__nv_bfloat16><<<g, WARPS * 32, 0, s>>>(
                      static_cast<const __nv_bfloat16*>(out), pos, w, T, k, d, static_cast<__nv_bfloat16*>(y), err));
   } else {
     PFMOE_LAUNCH("combine", s,
-                 combine_kernel<float, 2><<<g, WARPS * 32, 0, s>>>(static_cast<const float*>(out), pos, w, T, k, d,
+                 combine_kernel<float><<<g, WARPS * 32, 0, s>>>(static_cast<const float*>(out), pos, w, T, k, d,
                                                                 static_cast<float*>(y), err));
   }
   return PFMOE_OK;
@@ -268,7 +280,7 @@ int launch_combine(const void* out, const int32_t* pos, const float* w, int T, i
 
 int launch_combine_bwd(const void* dy, const void* out, const int32_t* pos, const float* w, int T, int k, int d,
                        int dtype, void* dO, float* g, int32_t* err, cudaStream_t s) {
-  const int gr = token_grid(T);
+  const int gr = item_grid(static_cast<long long>(T) * k);
   if (dtype == PFMOE_BF16) {
     PFMOE_LAUNCH("combine_bwd", s,
                  combine_bwd_kernel<__nv_bfloat16><<<gr, WARPS * 32, 0, s>>>(
@@ -300,7 +312,8 @@ int launch_transpose(const void* in, int rows, int cols, int dtype, void* out, c
 int launch_token_grad(const void* dx_pft, const int32_t* pos, const float* g, const float* w, const int32_t* ids,
                       const void* wgT, int T, int k, int d, int E, int dtype, void* dx, float* dlogits,
                       void* dz_bf16, int32_t* err, cudaStream_t s) {
-  const int gr = token_grid(T);
+  const int vn = dtype == PFMOE_BF16 ? 8 : 4;
+  const int gr = item_grid(static_cast<long long>(T) * ((d + 32 * vn - 1) / (32 * vn)));
   if (dtype == PFMOE_BF16) {
     PFMOE_LAUNCH("token_grad", s,
                  token_grad_kernel<__nv_bfloat16><<<gr, WARPS * 32, 0, s>>>(

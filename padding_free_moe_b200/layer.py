@@ -89,6 +89,13 @@ class PFTMoELayer:
             self.rbd_counts = e(2, dtype=i32)
             self.rbd_ws_bytes = L.rbd_plan_workspace_size(T, k, E, s.rbd_epd, s.rbd_dpn)
             self.rbd_ws = e(max(self.rbd_ws_bytes, 256), dtype=torch.uint8)
+            # The RBD plan reads only the routing ids, so step() runs it on a side stream next
+            # to dispatch / experts / backward; these events fork it after routing and join it
+            # back before the step ends (so the next step's routing cannot overwrite ids in use).
+            if self.device.type == "cuda":
+                self.side = torch.cuda.Stream(device=self.device)
+                self.ev_routed = torch.cuda.Event()
+                self.ev_rbd_done = torch.cuda.Event()
 
     # ------------------------------------------------------------------ steps
     def route(self, x, wg, bias=None, stream=None):
@@ -140,11 +147,24 @@ class PFTMoELayer:
                    self.assign_pilot, self.rbd_counts, self.rbd_ws, self.rbd_ws_bytes, self.err, stream)
 
     def step(self, x, wg, bias, w1, w3, w2, dy, stream=None):
-        """One pass of the whole hot path: forward, RBD plan (if mapped), backward."""
-        self.forward(x, wg, bias, w1, w3, w2, stream)
+        """One pass of the whole hot path: forward, RBD plan (if mapped), backward.
+
+        With an RBD map the plan runs on a side stream forked after routing and joined
+        before return, overlapping the PFT build, the expert GEMMs and the backward."""
+        main = stream if stream is not None else torch.cuda.current_stream(self.device)
+        self.route(x, wg, bias, main)
         if self.has_rbd:
-            self.rbd(stream)
-        self.backward(dy, x, wg, w1, w3, w2, stream)
+            self.ev_routed.record(main)
+            self.side.wait_event(self.ev_routed)
+            self.rbd(self.side)
+            self.ev_rbd_done.record(self.side)
+        self.build_pft(main)
+        self.dispatch(x, main)
+        self.experts(w1, w3, w2, main)
+        self.combine(main)
+        self.backward(dy, x, wg, w1, w3, w2, main)
+        if self.has_rbd:
+            main.wait_event(self.ev_rbd_done)
 
     def device_error(self) -> int:
         """Read (synchronously) and return the device error word; 0 means no device-side fault."""
