@@ -4,11 +4,16 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 One step = moe_route -> pft_build -> moe_dispatch -> moe_expert_ffn -> moe_combine
--> rbd_plan -> moe_backward over one batch of synthetic tokens, inputs and weights
-resident in HBM.  Rank 0 prints one JSON line.  With N > 1 (torchrun, one process
-per GPU) every rank runs an independent replica on its own tokens: the layer has no
-exchange step on one GPU, so there is no data-path collective; the timed region is
-bracketed by barriers and the reported time is the max over ranks.
+-> moe_backward over one batch of synthetic tokens, with rbd_plan on a side stream
+after routing (PFTMoELayer.step); inputs and weights resident in HBM.  Rank 0 prints
+one JSON line.  ``value`` comes from K timed steps with no per-kernel events; a second
+pass of the same K steps records a CUDA event pair around every launch for the
+per-kernel table and the roofline.  ``e2e`` runs the same steps with each step's
+inputs copied from pinned host memory and its results copied back (double-buffered
+on copy streams).  With N > 1 (torchrun, one process per GPU) every rank runs an
+independent replica on its own tokens: the layer has no exchange step on one GPU,
+so there is no data-path collective; the timed region is bracketed by barriers and
+the reported time is the max over ranks.
 
 ``--impl reference`` times the float64 CPU oracle (test infrastructure) on the
 host cores, on bounded token samples of the same workload.
@@ -285,56 +290,105 @@ def run_ours(args):
     if layer.device_error() != 0:
         raise RuntimeError(f"device error word {layer.device_error():#x} after warm-up")
 
-    # ---- device-timed region, inputs resident; per-kernel events live
+    # ---- device-timed region, inputs resident (no per-kernel events in it)
     clk = ClockSampler(replicas.physical_gpu_index(local_rank))
-    L.moe_profile_reset()
     barrier()
     torch.cuda.synchronize()
     clk.start()
-    L.moe_profile_enable(True)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     for _ in range(args.steps):
         step()
     ev1.record(stream)
     torch.cuda.synchronize()
-    L.moe_profile_enable(False)
     barrier()
     clocks = clk.stop()
     ms_total = max_over_ranks(ev0.elapsed_time(ev1))
-    kern = L.moe_profile_read()
     ms_step = ms_total / args.steps
     value = world * cfg.T / (ms_step * 1e-3)
 
-    # ---- end to end through the public API: pinned host inputs in, results out, every step
+    # ---- the same steps again with a CUDA event pair around every kernel launch (on the
+    # stream it is launched on): per-kernel durations for the roofline and launch counts.
+    # Kept out of the headline pass because the events add host-side gaps between kernels.
+    L.moe_profile_reset()
+    barrier()
+    torch.cuda.synchronize()
+    L.moe_profile_enable(True)
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    L.moe_profile_enable(False)
+    barrier()
+    kern = L.moe_profile_read()
+
+    # ---- end to end through the public API: every step copies its inputs (x, dY) from pinned
+    # host memory and reads its results (y, dx) back to pinned host memory.  Copies run on
+    # their own streams, double-buffered, so step i+1's inputs travel while step i computes;
+    # the timed region ends when the last step's results are on the host.
     x_h = inp.x.to("cpu").pin_memory()
     dy_h = inp.dy.to("cpu").pin_memory()
-    y_h = torch.empty_like(layer.y, device="cpu").pin_memory()
-    dx_h = torch.empty_like(layer.dx, device="cpu").pin_memory()
-    x_d, dy_d = torch.empty_like(inp.x), torch.empty_like(inp.dy)
-    e2e_steps = max(3, min(args.steps, 10))
+    x_d = [torch.empty_like(inp.x) for _ in range(2)]
+    dy_d = [torch.empty_like(inp.dy) for _ in range(2)]
+    y_st = [torch.empty_like(layer.y) for _ in range(2)]
+    dx_st = [torch.empty_like(layer.dx) for _ in range(2)]
+    y_h = [torch.empty_like(layer.y, device="cpu").pin_memory() for _ in range(2)]
+    dx_h = [torch.empty_like(layer.dx, device="cpu").pin_memory() for _ in range(2)]
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of buffer b on the device
+    ev_used = [torch.cuda.Event() for _ in range(2)]   # the step reading buffer b has finished
+    ev_out = [torch.cuda.Event() for _ in range(2)]    # results of buffer b staged
+    ev_read = [torch.cuda.Event() for _ in range(2)]   # staged results of buffer b on the host
+    e2e_steps = max(3, min(args.steps, 50))
 
-    def e2e_step():
-        x_d.copy_(x_h, non_blocking=True)
-        dy_d.copy_(dy_h, non_blocking=True)
-        layer.step(x_d, inp.wg, inp.bias, inp.w1, inp.w3, inp.w2, dy_d, stream)
-        y_h.copy_(layer.y, non_blocking=True)
-        dx_h.copy_(layer.dx, non_blocking=True)
-        stream.synchronize()
+    def run_e2e(n, start_event=None):
+        if start_event is not None:
+            h2d_s.wait_event(start_event)
 
-    e2e_step()
+        def h2d(i):
+            b = i % 2
+            if i >= 2:
+                h2d_s.wait_event(ev_used[b])
+            with torch.cuda.stream(h2d_s):
+                x_d[b].copy_(x_h, non_blocking=True)
+                dy_d[b].copy_(dy_h, non_blocking=True)
+            ev_in[b].record(h2d_s)
+
+        h2d(0)
+        for i in range(n):
+            b = i % 2
+            if i + 1 < n:
+                h2d(i + 1)
+            stream.wait_event(ev_in[b])
+            layer.step(x_d[b], inp.wg, inp.bias, inp.w1, inp.w3, inp.w2, dy_d[b], stream)
+            if i >= 2:
+                stream.wait_event(ev_read[b])
+            with torch.cuda.stream(stream):
+                y_st[b].copy_(layer.y)
+                dx_st[b].copy_(layer.dx)
+            ev_used[b].record(stream)
+            ev_out[b].record(stream)
+            d2h_s.wait_event(ev_out[b])
+            with torch.cuda.stream(d2h_s):
+                y_h[b].copy_(y_st[b], non_blocking=True)
+                dx_h[b].copy_(dx_st[b], non_blocking=True)
+            ev_read[b].record(d2h_s)
+        stream.wait_event(ev_read[(n - 1) % 2])
+
+    run_e2e(3)
+    torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    run_e2e(e2e_steps, start_event=e0)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
     h2d = x_h.numel() * x_h.element_size() + dy_h.numel() * dy_h.element_size()
-    d2h = y_h.numel() * y_h.element_size() + dx_h.numel() * dx_h.element_size()
+    d2h = y_h[0].numel() * y_h[0].element_size() + dx_h[0].numel() * dx_h[0].element_size()
+    if not (torch.equal(y_h[(e2e_steps - 1) % 2], layer.y.cpu()) and torch.equal(dx_h[(e2e_steps - 1) % 2], layer.dx.cpu())):
+        raise RuntimeError("end-to-end results read back to the host differ from the device results")
     if layer.device_error() != 0:
         raise RuntimeError(f"device error word {layer.device_error():#x}")
 

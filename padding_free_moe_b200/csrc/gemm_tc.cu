@@ -1,23 +1,29 @@
-// Persistent grouped GEMM on the 5th-generation tensor cores (sm_100a):
-// TMA -> shared memory ring -> tcgen05.mma (one issuing thread) -> TMEM
-// accumulators (double-buffered) -> register epilogue.
+// Persistent GEMMs on the 5th-generation tensor cores (sm_100a):
+// TMA -> shared-memory ring -> tcgen05.mma (one issuing thread) -> TMEM
+// accumulators (double-buffered) -> epilogue warps.  BF16 operands, FP32
+// accumulation.  Two kernels cover every contraction of the padding-free layer:
 //
-// D[M, N] = A[M, K] * B[N, K]^T, BF16 operands, FP32 accumulation.
+// grouped_gemm_tn_kernel (two-SM, cta_group::2) -- the row-grouped expert GEMMs
+//   (H1/H3/A = SwiGLU(X W1, X W3), O = A W2, dA = dO W2^T, dX = dH1 W1^T + dH3 W3^T).
+//   The PFT rows of expert g are the segment [seg[g], seg[g+1]) (X-MoE article
+//   §2.1.2: one GEMM per expert over its unpadded rows).  The expert's weights
+//   are the MMA's A operand (256 output features per CTA pair) and its tokens the
+//   B operand (N = the tile's token count rounded up to 32), and the epilogue
+//   transposes back to [token, feature] rows.
 //
-// Two grouping modes cover every contraction of the padding-free MoE layer:
-//   RG (row-grouped): A's rows are split into expert segments [seg[g], seg[g+1])
-//      (the expert-sorted PFT rows, X-MoE article §2.1.2: one GEMM per expert
-//      over its unpadded rows).  Each segment uses its own weight matrix
-//      B_g (3-D tensor map, g = third coordinate).  M tiles of 128 rows may
-//      straddle the segment end; rows past it are computed but never stored.
-//   KG (K-grouped): the reduction dimension is split into segments (weight
-//      gradients dW_g = X_g^T dH_g); each group writes its own [M, N] output.
-//      K rows past the segment end are zeroed in shared memory before the MMA.
+// grouped_gemm_kernel (one-SM) in two modes:
+//   KG (K-grouped): the reduction runs over a segment (weight gradients
+//      dW_g = X_g^T dH_g, and the gate's dWg split along T); each group writes its
+//      own [M, N] output.  K rows past the segment end are zeroed in shared memory
+//      by a dedicated warp before the MMA reads the block.
+//   RG (row-grouped, dense): the gate logits X Wg, split along K when the output
+//      has too few tiles to fill the GPU.
 //
-// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer (and
-// TMEM allocator), warps 2..5 = epilogue (one accumulator row per thread).
-// Every wait on an mbarrier is bounded (%globaltimer); on expiry the kernel
-// sets PFMOE_DEV_TIMEOUT, drains its own copies and MMAs, frees TMEM, returns.
+// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM allocator),
+// warps 2..5 = epilogue (TMEM lane quarter q = warp % 4), warp 6 (K-grouped
+// launches only) = K-tail zeroing.  Every wait on an mbarrier is bounded
+// (%globaltimer); on expiry the kernel sets PFMOE_DEV_TIMEOUT, drains its own
+// copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -35,6 +41,7 @@ constexpr int BM = 128;          // MMA M (one CTA)
 constexpr int BK = 64;           // K elements per stage (one 128-byte swizzle row of BF16)
 constexpr int MAX_STAGES = 8;
 constexpr int THREADS = 192;
+constexpr int THREADS_KG = 224;          // K-grouped launches add a seventh warp: the K-tail zeroing warp
 constexpr int BOX_BYTES = 64 * 128;      // one 64 x 64 BF16 box (MN-major block)
 constexpr int A_BYTES = BM * BK * 2;     // 16 KB
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
@@ -46,7 +53,6 @@ struct Params {
   CUtensorMap tmA[2];
   CUtensorMap tmB[2];
   CUtensorMap tmD[3];  // output maps for TMA stores from the staged epilogue (box 128 B x 32 rows)
-  CUtensorMap tmB32[2];  // token-as-N kernel: the token maps of tmB[] with 32-row boxes (ragged tiles)
   int tma_store;       // 1: tmD[] are valid
   int mode;
   int b_major;       // RG: 0 = K-major B (weights [G, N, K]), 1 = MN-major B (weights [G, K, N]); KG: 1
@@ -229,10 +235,7 @@ template <int MODE>
 __device__ __forceinline__ int total_tiles(const Params& p) {
   const int ns = n_step(p);
   const int NT = (p.Nout + ns - 1) / ns;
-  if constexpr (MODE == RG) {
-    const int mt = p.tiles ? p.tiles[p.G] : (p.dense_len + BM - 1) / BM * p.ksplit;
-    return mt * NT;
-  }
+  if constexpr (MODE == RG) return (p.dense_len + BM - 1) / BM * p.ksplit * NT;
   return p.G * ((p.M + BM - 1) / BM) * NT;
 }
 
@@ -242,31 +245,15 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
   const int ns = n_step(p);
   const int NT = (p.Nout + ns - 1) / ns;
   if constexpr (MODE == RG) {
-    int g = 0, tbase = 0, mtg, s0, s1, split = 0;
-    if (p.tiles) {
-      int lo = 0, hi = p.G - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (p.tiles[mid] * NT <= t) lo = mid; else hi = mid - 1;
-      }
-      g = lo;
-      tbase = p.tiles[g] * NT;
-      mtg = p.tiles[g + 1] - p.tiles[g];
-      s0 = p.seg[g];
-      s1 = p.seg[g + 1];
-    } else {
-      mtg = (p.dense_len + BM - 1) / BM;
-      s0 = 0;
-      s1 = p.dense_len;
-      split = t / (mtg * NT);
-      tbase = split * mtg * NT;
-    }
-    const int local = t - tbase;
+    // dense rows [0, dense_len), optionally split along K into ksplit output slices
+    const int mtg = (p.dense_len + BM - 1) / BM;
+    const int split = t / (mtg * NT);
+    const int local = t - split * mtg * NT;
     const int n_idx = local / mtg;
     const int m_loc = local - n_idx * mtg;
-    tl.g = g;
-    tl.row0 = s0 + m_loc * BM;
-    tl.rows = min(BM, s1 - tl.row0);
+    tl.g = 0;
+    tl.row0 = m_loc * BM;
+    tl.rows = min(BM, p.dense_len - tl.row0);
     tl.n0 = n_idx * ns;
     const int nk_all = p.k0_blocks + p.k1_blocks;
     const int kbs = (nk_all + p.ksplit - 1) / p.ksplit;
@@ -303,10 +290,8 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
 __device__ __forceinline__ float sigmoid_fast(float u) { return __fdividef(1.0f, 1.0f + __expf(-u)); }
 
 // ------------------------------------------------------------- direct epilogue
-// Row-grouped tiles: each thread stores its own row straight from registers (16-byte
-// vectors).  These tiles have long K loops, so the epilogue hides behind the next
-// tile's mainloop, and measured faster than staging through shared memory, which
-// competes with the operand traffic of the mainloop.
+// Row-grouped (dense gate) tiles: each thread stores its own FP32 row straight from
+// registers (16-byte vectors); the tiles are few and their K loops long.
 template <typename T>
 __device__ __forceinline__ void store_row_chunk(T* dst, const float* v, int ncols_valid) {
   // Store up to 32 values of one row; ncols_valid is a multiple of 8 (BF16) or 4 (F32) or >= 32.
@@ -339,84 +324,6 @@ __device__ __forceinline__ void epilogue_tile_direct(const Params& p, const Tile
           if (col + i < p.Nout) v[i] += p.bias[col + i];
       }
       if (row_ok) store_row_chunk<T>(D + grow * p.ldd + col, v, p.Nout - col);
-    }
-  } else if constexpr (EPI == EPI_SWIGLU_FWD) {
-    // D columns [0, bn/2) = H1 tile, [bn/2, bn) = H3 tile for the same output columns.
-    const int half = p.bn / 2;
-    __nv_bfloat16* H1 = static_cast<__nv_bfloat16*>(p.D0);
-    __nv_bfloat16* H3 = static_cast<__nv_bfloat16*>(p.D1);
-    __nv_bfloat16* A = static_cast<__nv_bfloat16*>(p.D2);
-    for (int c = 0; c < half; c += 32) {
-      const int col = tl.n0 + c;
-      if (col >= p.Nout) break;
-      float h1[32], h3[32], a[32];
-      tmem_ld32(tacc + c, h1);
-      tmem_ld32(tacc + half + c, h3);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) a[i] = h1[i] * sigmoid_fast(h1[i]) * h3[i];
-      if (row_ok) {
-        const long long off = grow * p.ldd + col;
-        store_row_chunk(H1 + off, h1, p.Nout - col);
-        store_row_chunk(H3 + off, h3, p.Nout - col);
-        store_row_chunk(A + off, a, p.Nout - col);
-      }
-    }
-  } else if constexpr (EPI == EPI_SWIGLU_BWD) {
-    // Accumulator = dA.  dH1 = dA * H3 * s * (1 + H1 (1 - s)), dH3 = dA * SiLU(H1), s = sigmoid(H1).
-    const __nv_bfloat16* H1 = static_cast<const __nv_bfloat16*>(p.X0);
-    const __nv_bfloat16* H3 = static_cast<const __nv_bfloat16*>(p.X1);
-    __nv_bfloat16* dH1 = static_cast<__nv_bfloat16*>(p.D0);
-    __nv_bfloat16* dH3 = static_cast<__nv_bfloat16*>(p.D1);
-    for (int c = 0; c < p.bn; c += 32) {
-      const int col = tl.n0 + c;
-      if (col >= p.Nout) break;
-      float da[32];
-      tmem_ld32(tacc + c, da);
-      if (row_ok) {
-        const long long off = grow * p.ldd + col;
-        const int nv = p.Nout - col;
-        float h1[32], h3[32], o1[32], o3[32];
-#pragma unroll
-        for (int i = 0; i < 32; i += 8) {
-          if (i < nv) {
-            load16(H1 + off + i, h1 + i);
-            load16(H3 + off + i, h3 + i);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) h1[i + j] = h3[i + j] = 0.f;
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float s = sigmoid_fast(h1[i]);
-          o1[i] = da[i] * h3[i] * s * (1.0f + h1[i] * (1.0f - s));
-          o3[i] = da[i] * h1[i] * s;
-        }
-        store_row_chunk(dH1 + off, o1, nv);
-        store_row_chunk(dH3 + off, o3, nv);
-      }
-    }
-  } else if constexpr (EPI == EPI_SPLIT_BF16) {
-    // KG with nsplit: columns [0, bn/2) -> D0[g], [bn/2, bn) -> D1[g].
-    const int half = p.bn / 2;
-    __nv_bfloat16* D0 = static_cast<__nv_bfloat16*>(p.D0) + tl.g * p.d_gstride;
-    __nv_bfloat16* D1 = static_cast<__nv_bfloat16*>(p.D1) + tl.g * p.d_gstride;
-    for (int c = 0; c < half; c += 32) {
-      const int col = tl.n0 + c;
-      if (col >= p.Nout) break;
-      float v0[32], v1[32];
-      if (!zero) {
-        tmem_ld32(tacc + c, v0);
-        tmem_ld32(tacc + half + c, v1);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v0[i] = v1[i] = 0.f;
-      }
-      if (row_ok) {
-        const long long off = grow * p.ldd + col;
-        store_row_chunk(D0 + off, v0, p.Nout - col);
-        store_row_chunk(D1 + off, v1, p.Nout - col);
-      }
     }
   }
 }
@@ -487,21 +394,6 @@ __device__ __forceinline__ void stage_row(uint32_t stg, int lane, const float* v
   }
 }
 
-// Thread `lane` reads back row `lane` of the slab as 64 BF16 values.
-__device__ __forceinline__ void unstage_row_bf16(uint32_t stg, int lane, float* v) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint4 u = ld_shared16(stg_addr(stg, lane, c));
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __bfloat1622float2(h[i]);
-      v[8 * c + 2 * i] = f.x;
-      v[8 * c + 2 * i + 1] = f.y;
-    }
-  }
-}
-
 // Staged slab -> global rows base + row * stride (bytes); rows >= rows_valid and bytes >= bytes_valid are skipped.
 __device__ __forceinline__ void copy_out(uint32_t stg, int lane, char* base, long long stride, int rows_valid,
                                          int bytes_valid) {
@@ -512,20 +404,6 @@ __device__ __forceinline__ void copy_out(uint32_t stg, int lane, char* base, lon
     const uint4 u = ld_shared16(stg_addr(stg, row, chunk));
     if (row < rows_valid && chunk * 16 < bytes_valid)
       *reinterpret_cast<uint4*>(base + row * stride + chunk * 16) = u;
-  }
-}
-
-// Global rows -> staged slab (coalesced); missing rows / bytes read as zero.
-__device__ __forceinline__ void copy_in(uint32_t stg, int lane, const char* base, long long stride, int rows_valid,
-                                        int bytes_valid) {
-  const int chunk = lane & 7;
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int row = it * 4 + (lane >> 3);
-    uint4 u = make_uint4(0, 0, 0, 0);
-    if (row < rows_valid && chunk * 16 < bytes_valid)
-      u = __ldg(reinterpret_cast<const uint4*>(base + row * stride + chunk * 16));
-    st_shared16(stg_addr(stg, row, chunk), u);
   }
 }
 
@@ -627,67 +505,12 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, u
       emit(stg, lane, v, tmd(p, 0), col, static_cast<int>(grow0), tz, D + grow0 * p.ldd + col, p.ldd, rows_valid,
            p.Nout - col);
     }
-  } else if constexpr (EPI == EPI_SWIGLU_FWD) {
-    // D columns [0, bn/2) = H1 tile, [bn/2, bn) = H3 tile for the same output columns.
-    const int half = p.bn / 2;
-    __nv_bfloat16* H1 = static_cast<__nv_bfloat16*>(p.D0);
-    __nv_bfloat16* H3 = static_cast<__nv_bfloat16*>(p.D1);
-    __nv_bfloat16* A = static_cast<__nv_bfloat16*>(p.D2);
-    for (int c = 0; c < half; c += 64) {
-      const int col = tl.n0 + c;
-      if (col >= p.Nout) break;
-      const long long off = grow0 * p.ldd + col;
-      float h1[64], h3[64];
-      tmem_ld64(tacc + c, h1);
-      tmem_ld64(tacc + half + c, h3);
-      emit(stg, lane, h1, tmd(p, 0), col, static_cast<int>(grow0), 0, H1 + off, p.ldd, rows_valid, p.Nout - col);
-      emit(stg, lane, h3, tmd(p, 1), col, static_cast<int>(grow0), 0, H3 + off, p.ldd, rows_valid, p.Nout - col);
-#pragma unroll
-      for (int i = 0; i < 64; ++i) h1[i] = h1[i] * sigmoid_fast(h1[i]) * h3[i];
-      emit(stg, lane, h1, tmd(p, 2), col, static_cast<int>(grow0), 0, A + off, p.ldd, rows_valid, p.Nout - col);
-    }
-  } else if constexpr (EPI == EPI_SWIGLU_BWD) {
-    // Accumulator = dA.  dH1 = dA * H3 * s * (1 + H1 (1 - s)), dH3 = dA * SiLU(H1), s = sigmoid(H1).
-    const char* H1 = static_cast<const char*>(p.X0);
-    const char* H3 = static_cast<const char*>(p.X1);
-    __nv_bfloat16* dH1 = static_cast<__nv_bfloat16*>(p.D0);
-    __nv_bfloat16* dH3 = static_cast<__nv_bfloat16*>(p.D1);
-    const long long stride = p.ldd * 2;
-    for (int c = 0; c < p.bn; c += 64) {
-      const int col = tl.n0 + c;
-      if (col >= p.Nout) break;
-      const long long off = grow0 * p.ldd + col;
-      const int bytes_valid = min(128, (p.Nout - col) * 2);
-      float da[64], h1[64], h3[64];
-      tmem_ld64(tacc + c, da);
-      // Read H1 / H3 through the slab the next emit will use (no store of ours is pending on it
-      // once at most one bulk group is outstanding).
-      const uint32_t ibuf = stg.base + (stg.seq & 1) * STAGE_BYTES_PER_WARP;
-      if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-      __syncwarp();
-      copy_in(ibuf, lane, H1 + off * 2, stride, rows_valid, bytes_valid);
-      __syncwarp();
-      unstage_row_bf16(ibuf, lane, h1);
-      __syncwarp();
-      copy_in(ibuf, lane, H3 + off * 2, stride, rows_valid, bytes_valid);
-      __syncwarp();
-      unstage_row_bf16(ibuf, lane, h3);
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float s = sigmoid_fast(h1[i]);
-        const float d1 = da[i] * h3[i] * s * (1.0f + h1[i] * (1.0f - s));
-        h1[i] = da[i] * h1[i] * s;
-        da[i] = d1;
-      }
-      emit(stg, lane, da, tmd(p, 0), col, static_cast<int>(grow0), 0, dH1 + off, p.ldd, rows_valid, p.Nout - col);
-      emit(stg, lane, h1, tmd(p, 1), col, static_cast<int>(grow0), 0, dH3 + off, p.ldd, rows_valid, p.Nout - col);
-    }
   }
 }
 
 // ---------------------------------------------------------------------- kernel
 template <int EPI, int MODE>
-__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_gemm_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages;
@@ -700,7 +523,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
   uint64_t* acc_full = empty + MAX_STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* ready = drain + 1;   // K-grouped: stage s landed and its segment-tail rows are zero
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ready + MAX_STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -717,6 +541,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       mbar_init(smem_u32(&acc_empty[b]), 4 * 32);
     }
     mbar_init(smem_u32(drain), 1);
+    for (int z = 0; z < MAX_STAGES; ++z) mbar_init(smem_u32(&ready[z]), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -754,27 +579,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
           const uint32_t sb = sa + A_BYTES;
           const int nb = p.bn / 64;
           if constexpr (MODE == RG) {
-            const int kbg = tl.kb0 + kb;
-            const int src = kbg < p.k0_blocks ? 0 : 1;
-            const int kk = (src == 0 ? kbg : kbg - p.k0_blocks) * BK;
-            tma_load_3d(sa, &p.tmA[src], fb, kk, tl.row0, 0);
-            if (p.b_major == 0) {
-              if (p.nsplit) {
-                tma_load_3d(sb, &p.tmB[0], fb, kk, tl.n0, tl.g);
-                tma_load_3d(sb + (p.bn / 2) * 128, &p.tmB[1], fb, kk, tl.n0, tl.g);
-              } else {
-                tma_load_3d(sb, &p.tmB[src], fb, kk, tl.n0, tl.g);
-              }
-            } else {
-              for (int j = 0; j < nb; ++j) {
-                int which = src, nc = tl.n0 + 64 * j;
-                if (p.nsplit) {
-                  which = j < nb / 2 ? 0 : 1;
-                  nc = tl.n0 + 64 * (j < nb / 2 ? j : j - nb / 2);
-                }
-                tma_load_3d(sb + j * BOX_BYTES, &p.tmB[which], fb, nc, kk, tl.g);
-              }
-            }
+            // dense gate GEMM: A = X rows (K-major), B = Wg [K, N] (MN-major 64-column boxes)
+            const int kk = (tl.kb0 + kb) * BK;
+            tma_load_3d(sa, &p.tmA[0], fb, kk, tl.row0, 0);
+            for (int j = 0; j < nb; ++j) tma_load_3d(sb + j * BOX_BYTES, &p.tmB[0], fb, tl.n0 + 64 * j, kk, 0);
           } else {
             const int krow = tl.krow0 + kb * BK;
             if (p.a_merged) {
@@ -835,26 +643,15 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       for (int kb = 0; kb < tl.nk; ++kb, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
-        ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&full[s]), ph, abort_flag, p.err));
+        int kk_count = BK / 16;
+        // K-grouped: the zeroing warp passes every stage on through ready[s] (one phase per ring
+        // round, like full[s]) after clearing a segment's tail rows; MMAs of a segment's last block
+        // stop at the 16-row step that holds the segment end.
+        if (MODE == KG && kb == tl.nk - 1 && tl.kvalid < BK) kk_count = ((tl.kvalid + 15) & ~15) / 16;
+        ok = __all_sync(0xffffffffu, wait_bar(smem_u32(MODE == KG ? &ready[s] : &full[s]), ph, abort_flag, p.err));
         if (!ok) break;
         const uint32_t sa = smem_u32(smem + s * stage_bytes);
         const uint32_t sb = sa + A_BYTES;
-        int kk_count = BK / 16;
-        if (MODE == KG && kb == tl.nk - 1 && tl.kvalid < BK) {
-          // Last block of a segment: MMAs stop at the 16-row step holding the segment end, and the
-          // rows of that step past the end are zeroed in every box (A: 2 boxes, B: bn/64).
-          const int kv16 = (tl.kvalid + 15) & ~15;
-          kk_count = kv16 / 16;
-          const int per_box = (kv16 - tl.kvalid) * 8;   // 16-byte chunks to clear per box
-          if (per_box > 0) {
-            const int nbox = 2 + p.bn / 64;
-            for (int b = 0; b < nbox; ++b)
-              for (int i = lane; i < per_box; i += 32)
-                st_shared16(sa + b * BOX_BYTES + tl.kvalid * 128 + i * 16, make_uint4(0, 0, 0, 0));
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          }
-          __syncwarp();
-        }
         tc_fence_after();
         if (lane == 0) {
           for (int kk = 0; kk < kk_count; ++kk) {
@@ -876,6 +673,33 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
       wait_bar(smem_u32(drain), 0, abort_flag, p.err, false);
     }
     __syncwarp();
+  } else if (MODE == KG && warp == 6) {
+    // ---------------------------------------------------- K-tail zeroing (K-grouped only)
+    // Walks every K block in ring order: waits for it to land (full[s]), clears the rows of a
+    // segment's last 16-row step past the segment end in every box (A: 2, B: bn/64), and hands
+    // the stage to the MMA warp (ready[s]).  Taking part in every round keeps its parity waits
+    // unambiguous: it can be at most one phase ahead on any stage.
+    int it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      const Tile tl = decode<MODE>(p, t);
+      for (int kb = 0; kb < tl.nk; ++kb, ++it) {
+        const int s = it % S;
+        ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&full[s]), (it / S) & 1, abort_flag, p.err));
+        if (!ok) break;
+        if (kb == tl.nk - 1 && tl.kvalid < BK) {
+          const uint32_t sa = smem_u32(smem + s * stage_bytes);
+          const int per_box = (((tl.kvalid + 15) & ~15) - tl.kvalid) * 8;   // 16-byte chunks per box
+          const int nbox = 2 + p.bn / 64;
+          for (int b = 0; b < nbox; ++b)
+            for (int i = lane; i < per_box; i += 32)
+              st_shared16(sa + b * BOX_BYTES + tl.kvalid * 128 + i * 16, make_uint4(0, 0, 0, 0));
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&ready[s]));
+      }
+    }
   } else {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;           // TMEM lane quarter this warp may access: rows 32q .. 32q+31
@@ -982,12 +806,10 @@ static int round_bn(int n) {
   return bn > 256 ? 256 : bn;
 }
 
-// MMA N for the two-SM kernel: each CTA of the pair holds half of it in whole 64-column boxes.
-static int round_bn_pair(int n) { return n > 128 ? 256 : 128; }
 
 constexpr int SMEM_LIMIT = 227 * 1024;
-// Alignment slack + barriers, plus the epilogue staging buffers when the launch uses them (K-grouped).
-static int smem_fixed(bool staged) { return 1024 + 256 + (staged ? 4 * STAGE_BUFS * STAGE_BYTES_PER_WARP : 0); }
+// Alignment slack + barriers (512 B), plus the epilogue staging buffers when the launch uses them (K-grouped).
+static int smem_fixed(bool staged) { return 1024 + 512 + (staged ? 4 * STAGE_BUFS * STAGE_BYTES_PER_WARP : 0); }
 
 static int pick_stages(int bn, bool staged) {
   const int stage = A_BYTES + bn * BK * 2;
@@ -1000,21 +822,14 @@ static size_t smem_bytes(int bn, int stages, bool staged) {
 }
 
 // ============================================================================
-// Two-SM variant for row-grouped problems (tcgen05 cta_group::2).
+// Two-SM (tcgen05 cta_group::2) building blocks.
 //
-// A cluster of two CTAs on one TPC computes a 256-row x bn-column tile with one
-// M=256 MMA issued by the even CTA.  CTA v loads its own 128 rows of A and
-// columns [v*bn/2, (v+1)*bn/2) of B; the tensor cores read the other half of B
-// from the peer.  Per FLOP this moves 1.5x fewer operand bytes through L2 and
-// shared memory than two independent 128-row tiles.  Each CTA keeps its 128
-// accumulator rows in its own TMEM and runs the same epilogue as the one-SM
-// kernel.  A 256-row tile covers rows [256p, 256p+256) of one expert segment
-// (rows past the segment end are computed but never stored).  With N-split
-// (SwiGLU pairing) CTA 0 loads the W1 block and CTA 1 the W3 block.
-//
-// Synchronisation: both CTAs' TMA loads complete on the even CTA's full[s]
-// barrier; the MMA's commits arrive on both CTAs' empty[s] / acc_full[b]
-// (multicast commit); both CTAs' epilogues arrive on the even CTA's acc_empty[b].
+// A cluster of two CTAs on one TPC computes one M = 256 tile with MMAs issued by
+// the even CTA: each CTA holds 128 rows of A and half of B's columns in its own
+// shared memory, and keeps its 128 accumulator rows in its own TMEM.  Both CTAs'
+// TMA loads complete on the even CTA's full[s] barrier; the MMA's commits arrive
+// on both CTAs' barriers (multicast commit); both CTAs' epilogues arrive on the
+// even CTA's acc_empty[b].
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -1101,336 +916,6 @@ __device__ __forceinline__ void tc_commit2_both(uint32_t bar) {
                : "memory");
 }
 
-struct PairTile {
-  int g, row0, rows, n0, nk, kb0, split, krow0, kvalid;
-};
-
-// Pair tiles of a row-grouped problem: expert g has ceil(n_g / 256) of them (prefix in pair_off).
-// K-grouped: every group has ceil(M / 256) x NT output tiles.
-template <int MODE>
-__device__ __forceinline__ int total_pair_tiles(const Params& p, const int* pair_off) {
-  const int ns = n_step(p);
-  const int NT = (p.Nout + ns - 1) / ns;
-  if constexpr (MODE == KG) return p.G * ((p.M + 2 * BM - 1) / (2 * BM)) * NT;
-  const int np = p.tiles ? pair_off[p.G] : (p.dense_len + 2 * BM - 1) / (2 * BM) * p.ksplit;
-  return np * NT;
-}
-
-// K-grouped pair tile: rows [256 mp + 128 rank, +128) of group g's [M, Nout] output, K = the group's segment.
-__device__ __forceinline__ PairTile decode_pair_kg(const Params& p, int t, uint32_t rank) {
-  PairTile tl;
-  const int ns = n_step(p);
-  const int NT = (p.Nout + ns - 1) / ns;
-  const int MP = (p.M + 2 * BM - 1) / (2 * BM);
-  const int per = MP * NT;
-  const int g = t / per;
-  const int rem = t - g * per;
-  const int n_idx = rem / MP;
-  const int mp = rem - n_idx * MP;
-  const int s0 = p.seg ? p.seg[g] : g * p.kchunk;
-  const int s1 = p.seg ? p.seg[g + 1] : min(p.dense_len, s0 + p.kchunk);
-  const int len = max(0, s1 - s0);
-  tl.g = g;
-  tl.row0 = mp * 2 * BM + static_cast<int>(rank) * BM;
-  tl.rows = max(0, min(BM, p.M - tl.row0));
-  tl.n0 = n_idx * ns;
-  tl.nk = (len + BK - 1) / BK;
-  tl.kb0 = 0;
-  tl.split = 0;
-  tl.krow0 = s0;
-  tl.kvalid = len - (tl.nk - 1) * BK;
-  return tl;
-}
-
-__device__ __forceinline__ PairTile decode_pair(const Params& p, const int* pair_off, int t, uint32_t rank) {
-  PairTile tl;
-  const int ns = n_step(p);
-  const int NT = (p.Nout + ns - 1) / ns;
-  int g = 0, tbase = 0, npg, s0, s1, split = 0;
-  if (p.tiles) {
-    int lo = 0, hi = p.G - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (pair_off[mid] * NT <= t) lo = mid; else hi = mid - 1;
-    }
-    g = lo;
-    tbase = pair_off[g] * NT;
-    npg = pair_off[g + 1] - pair_off[g];
-    s0 = p.seg[g];
-    s1 = p.seg[g + 1];
-  } else {
-    npg = (p.dense_len + 2 * BM - 1) / (2 * BM);
-    s0 = 0;
-    s1 = p.dense_len;
-    split = t / (npg * NT);
-    tbase = split * npg * NT;
-  }
-  const int local = t - tbase;
-  const int n_idx = local / npg;
-  const int pr = local - n_idx * npg;
-  tl.g = g;
-  tl.row0 = s0 + pr * 2 * BM + static_cast<int>(rank) * BM;
-  tl.rows = max(0, min(BM, s1 - tl.row0));
-  tl.n0 = n_idx * ns;
-  const int nk_all = p.k0_blocks + p.k1_blocks;
-  const int kbs = (nk_all + p.ksplit - 1) / p.ksplit;
-  tl.split = split;
-  tl.kb0 = split * kbs;
-  tl.nk = max(0, min(kbs, nk_all - tl.kb0));
-  tl.krow0 = 0;
-  tl.kvalid = BK;
-  return tl;
-}
-
-template <int MODE>
-__device__ __forceinline__ PairTile decode_pair_any(const Params& p, const int* pair_off, int t, uint32_t rank) {
-  if constexpr (MODE == KG) return decode_pair_kg(p, t, rank);
-  else return decode_pair(p, pair_off, t, rank);
-}
-
-__device__ __forceinline__ void st_cluster16(uint32_t addr, uint4 u) {
-  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(u.x), "r"(u.y), "r"(u.z),
-               "r"(u.w)
-               : "memory");
-}
-
-// Epilogue of the two-SM kernel: staged through shared memory (full-line stores, coalesced
-// reads of the SwiGLU-backward inputs) or direct per-row stores.
-constexpr bool kStaged2sm = true;
-
-template <int EPI, int MODE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-    grouped_gemm_2sm_kernel(const __grid_constant__ Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int S = p.stages;
-  const int bh = p.bn / 2;                         // B columns held by this CTA
-  const uint32_t b_bytes = static_cast<uint32_t>(bh) * BK * 2;
-  const uint32_t stage_bytes = A_BYTES + b_bytes;
-  uint8_t* stage_area = smem + S * stage_bytes;
-  int* pair_off = reinterpret_cast<int*>(stage_area + (kStaged2sm ? 4 * STAGE_BUFS * STAGE_BYTES_PER_WARP : 0));
-  const int poff_ints = p.tiles ? ((p.G + 1 + 63) & ~63) : 0;
-  uint8_t* bar_area = reinterpret_cast<uint8_t*>(pair_off + poff_ints);
-  uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
-  uint64_t* empty = full + MAX_STAGES;
-  uint64_t* acc_full = empty + MAX_STAGES;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_rank();
-  const bool leader = rank == 0;
-  const int pair = blockIdx.x >> 1;
-  const int npairs = gridDim.x >> 1;
-  const uint32_t tmem_cols = p.bn * 2 <= 128 ? 128 : (p.bn * 2 <= 256 ? 256 : 512);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&empty[s]), 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&acc_full[b]), 1);
-      mbar_init(smem_u32(&acc_empty[b]), 2 * 4 * 32);
-    }
-    mbar_init(smem_u32(drain), 1);
-    *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  }
-  // Prefix over experts of ceil(n_g / 256) pair tiles (from the 128-row tile prefix).
-  if (p.tiles && warp == 0) {
-    int carry = 0;
-    for (int base = 0; base < p.G; base += 32) {
-      const int e = base + lane;
-      const int np = e < p.G ? (p.tiles[e + 1] - p.tiles[e] + 1) / 2 : 0;
-      int x = np;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      if (e < p.G) pair_off[e] = carry + x - np;
-      carry += __shfl_sync(0xffffffffu, x, 31);
-    }
-    if (lane == 0) pair_off[p.G] = carry;
-  }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&p.tmA[0]);
-    prefetch_tmap(&p.tmB[0]);
-  }
-  if (warp == 1) {
-    tmem_alloc2(smem_u32(tmem_slot), tmem_cols);
-    tmem_relinquish2();
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  const int ntiles = total_pair_tiles<MODE>(p, pair_off);
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (both CTAs)
-    if (lane == 0) {
-      uint32_t pending = 0, pend_parity = 0;
-      int it = 0;
-      bool ok = true;
-      for (int t = pair; t < ntiles && ok; t += npairs) {
-        const PairTile tl = decode_pair_any<MODE>(p, pair_off, t, rank);
-        for (int kb = 0; kb < tl.nk; ++kb, ++it) {
-          const int s = it % S;
-          const uint32_t ph = (it / S) & 1;
-          if (!wait_bar2(smem_u32(&empty[s]), ph ^ 1, abort_flag, p.err)) { ok = false; break; }
-          const uint32_t fb_local = smem_u32(&full[s]);
-          if (leader) mbar_expect_tx(fb_local, 2 * stage_bytes);
-          const uint32_t fb = mapa_shared(fb_local, 0);
-          const uint32_t sa = smem_u32(smem + s * stage_bytes);
-          const uint32_t sb = sa + A_BYTES;
-          if constexpr (MODE == KG) {
-            // A = X^T (MN-major): this CTA's 128 output rows; B (MN-major): its bh output columns.
-            const int krow = tl.krow0 + kb * BK;
-            if (p.a_merged) {
-              tma_load_4d_pair(sa, &p.tmA[0], fb, 0, krow, tl.row0 / 64, 0);
-            } else {
-              tma_load_3d_pair(sa, &p.tmA[0], fb, tl.row0, krow, 0);
-              tma_load_3d_pair(sa + BOX_BYTES, &p.tmA[0], fb, tl.row0 + 64, krow, 0);
-            }
-            const CUtensorMap* tb = &p.tmB[p.nsplit ? static_cast<int>(rank) : 0];
-            const int ncol = p.nsplit ? tl.n0 : tl.n0 + static_cast<int>(rank) * bh;
-            if (p.b_merged) {
-              tma_load_4d_pair(sb, tb, fb, 0, krow, ncol / 64, 0);
-            } else {
-              for (int j = 0; j < bh / 64; ++j) tma_load_3d_pair(sb + j * BOX_BYTES, tb, fb, ncol + 64 * j, krow, 0);
-            }
-            pending |= 1u << s;
-            pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
-            continue;
-          }
-          const int kbg = tl.kb0 + kb;
-          const int src = kbg < p.k0_blocks ? 0 : 1;
-          const int kk = (src == 0 ? kbg : kbg - p.k0_blocks) * BK;
-          tma_load_3d_pair(sa, &p.tmA[src], fb, kk, tl.row0, 0);
-          const CUtensorMap* tb = &p.tmB[p.nsplit ? static_cast<int>(rank) : src];
-          const int ncol = p.nsplit ? tl.n0 : tl.n0 + static_cast<int>(rank) * bh;
-          if (p.b_major == 0) {
-            tma_load_3d_pair(sb, tb, fb, kk, ncol, tl.g);
-          } else {
-            for (int j = 0; j < bh / 64; ++j) tma_load_3d_pair(sb + j * BOX_BYTES, tb, fb, ncol + 64 * j, kk, tl.g);
-          }
-          pending |= 1u << s;
-          pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
-        }
-      }
-      // Drain: a stage's empty barrier completes only after the MMA consumed it, so its loads landed.
-      for (int s = 0; s < S; ++s)
-        if (pending & (1u << s))
-          wait_bar2(smem_u32(&empty[s]), (pend_parity >> s) & 1, abort_flag, p.err, false);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (even CTA)
-    if (leader) {
-      const int a_mn = MODE == KG ? 1 : 0;
-      const int b_mn = MODE == KG ? 1 : p.b_major;
-      const uint32_t idesc = idesc_bf16(2 * BM, p.bn, a_mn, b_mn);
-      const uint32_t a_lbo = a_mn ? BOX_BYTES : 16, b_lbo = b_mn ? BOX_BYTES : 16;
-      const uint32_t a_step = a_mn ? 2048 : 32, b_step = b_mn ? 2048 : 32;
-      int it = 0, tcount = 0;
-      bool ok = true;
-      for (int t = pair; t < ntiles && ok; t += npairs, ++tcount) {
-        const PairTile tl = decode_pair_any<MODE>(p, pair_off, t, rank);
-        const int buf = tcount & 1;
-        const uint32_t aph = (tcount >> 1) & 1;
-        ok = __all_sync(0xffffffffu, wait_bar2(smem_u32(&acc_empty[buf]), aph ^ 1, abort_flag, p.err));
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t tmem_d = tmem_base + buf * p.bn;
-        for (int kb = 0; kb < tl.nk; ++kb, ++it) {
-          const int s = it % S;
-          const uint32_t ph = (it / S) & 1;
-          ok = __all_sync(0xffffffffu, wait_bar2(smem_u32(&full[s]), ph, abort_flag, p.err));
-          if (!ok) break;
-          const uint32_t sa = smem_u32(smem + s * stage_bytes);
-          const uint32_t sb = sa + A_BYTES;
-          int kk_count = BK / 16;
-          if (MODE == KG && kb == tl.nk - 1 && tl.kvalid < BK) {
-            // Last block of a segment: MMAs stop at the 16-row step holding the segment end, and the
-            // rows of that step past the end are zeroed in every box of both CTAs (the peer's over DSMEM).
-            const int kv16 = (tl.kvalid + 15) & ~15;
-            kk_count = kv16 / 16;
-            const int per_box = (kv16 - tl.kvalid) * 8;   // 16-byte chunks to clear per box
-            if (per_box > 0) {
-              const int nbox = 2 + bh / 64;
-              for (int b = 0; b < nbox; ++b)
-                for (int i = lane; i < per_box; i += 32) {
-                  const uint32_t a = sa + b * BOX_BYTES + tl.kvalid * 128 + i * 16;
-                  st_shared16(a, make_uint4(0, 0, 0, 0));
-                  st_cluster16(mapa_shared(a, 1), make_uint4(0, 0, 0, 0));
-                }
-              asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
-            }
-            __syncwarp();
-          }
-          tc_fence_after();
-          if (lane == 0) {
-            for (int kk = 0; kk < kk_count; ++kk) {
-              const uint64_t ad = sdesc(sa + kk * a_step, a_lbo, 1024);
-              const uint64_t bd = sdesc(sb + kk * b_step, b_lbo, 1024);
-              tc_mma2(tmem_d, ad, bd, idesc, (kb | kk) != 0);
-            }
-            tc_commit2_both(smem_u32(&empty[s]));
-          }
-          __syncwarp();
-        }
-        if (!ok) break;
-        if (lane == 0) tc_commit2_both(smem_u32(&acc_full[buf]));   // also for nk == 0 (zero tile)
-        __syncwarp();
-      }
-      if (lane == 0) {
-        tc_commit2_both(smem_u32(drain));
-        wait_bar2(smem_u32(drain), 0, abort_flag, p.err, false);
-      }
-      __syncwarp();
-    }
-  } else {
-    // ------------------------------------------------------------ epilogue (both CTAs)
-    const int q = warp & 3;
-    const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
-    const uint32_t acc_empty_leader1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
-    Stager stg{smem_u32(stage_area + (warp - 2) * STAGE_BUFS * STAGE_BYTES_PER_WARP), 0};
-    int tcount = 0;
-    for (int t = pair; t < ntiles; t += npairs, ++tcount) {
-      const PairTile pt = decode_pair_any<MODE>(p, pair_off, t, rank);
-      const int buf = tcount & 1;
-      const uint32_t aph = (tcount >> 1) & 1;
-      if (!__all_sync(0xffffffffu, wait_bar2(smem_u32(&acc_full[buf]), aph, abort_flag, p.err))) break;
-      tc_fence_after();
-      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * p.bn;
-      Tile tl;
-      tl.g = pt.g; tl.row0 = pt.row0; tl.rows = pt.rows; tl.n0 = pt.n0; tl.nk = pt.nk;
-      tl.krow0 = pt.krow0; tl.kvalid = pt.kvalid; tl.kb0 = pt.kb0; tl.split = pt.split;
-      if constexpr (kStaged2sm)
-        epilogue_tile<EPI>(p, tl, tacc, q, lane, stg);
-      else
-        epilogue_tile_direct<EPI>(p, tl, tacc, q * 32 + lane);
-      tc_fence_before();
-      mbar_arrive_cluster(buf ? acc_empty_leader1 : acc_empty_leader0);
-    }
-    emit_drain(lane);
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc2(tmem_base, tmem_cols);
-  }
-}
-
 // ============================================================================
 // Token-as-N two-SM kernel for row-grouped problems.
 //
@@ -1486,50 +971,18 @@ __device__ __forceinline__ TnTile decode_tn(const Params& p, const int* pair_off
   return tl;
 }
 
-// Tile order of one pair.  Unit order: the pair takes (expert, feature block) units
-// u = pair, pair + npairs, ... and runs all token tiles of a unit back to back, so the
-// unit's weight block is fetched into this die's L2 once and re-read from there.  Wave
-// order: wave k holds pair tiles [k P, (k + 1) P) as numbered by decode_tn (P pairs), and
-// pair p takes tile k P + p in even waves and k P + P - 1 - p in odd ones.  Neighbouring
-// tiles (the full and the ragged token tile of one weight block) thus alternate between
-// pairs instead of always landing on pairs of the same parity.
-constexpr bool kTnUnitOrder = false;
-// Ragged token tiles load their token columns in 32-row boxes instead of one 128-row box.
-constexpr bool kTnRaggedBoxes = false;
-
-struct TnCursor {
-  int u, j, t;   // unit order: unit u, token tile j; wave order: wave u, pair t
-};
-
-__device__ __forceinline__ bool tn_next(const Params& p, const int* pair_off, int npairs, TnCursor& c, TnTile& tl) {
-  const int FT = tn_feature_tiles(p);
-  if constexpr (kTnUnitOrder) {
-    const int nunits = p.G * FT;
-    while (c.u < nunits) {
-      const int g = c.u / FT;
-      const int npg = pair_off[g + 1] - pair_off[g];
-      if (c.j < npg) {
-        tl.g = g;
-        tl.tok0 = p.seg[g] + c.j * TN_TOK;
-        tl.ntok = max(0, min(TN_TOK, p.seg[g + 1] - tl.tok0));
-        tl.nmma = max(32, (tl.ntok + 31) & ~31);
-        tl.f0 = (c.u - g * FT) * p.fstep;
-        tl.nk = p.k0_blocks + p.k1_blocks;
-        ++c.j;
-        return true;
-      }
-      c.u += npairs;
-      c.j = 0;
-    }
-    return false;
-  } else {
-    // c.u = wave index, c.t = this pair's index
-    const int t = c.u * npairs + ((c.u & 1) ? npairs - 1 - c.t : c.t);
-    if (t >= pair_off[p.G] * FT) return false;
-    tl = decode_tn(p, pair_off, t);
-    ++c.u;
-    return true;
-  }
+// Tile order of one pair (P pairs): wave k holds pair tiles [k P, (k + 1) P) as numbered by
+// decode_tn, and pair p takes tile k P + p in even waves and k P + P - 1 - p in odd ones.
+// Neighbouring tiles (the full and the ragged token tile of one weight block) thus alternate
+// between pairs instead of always landing on pairs of the same parity, and the two token tiles
+// of a weight block run at the same time, so the block is read from L2 for the second one.
+__device__ __forceinline__ bool tn_next(const Params& p, const int* pair_off, int npairs, int pair, int& wave,
+                                        TnTile& tl) {
+  const int t = wave * npairs + ((wave & 1) ? npairs - 1 - pair : pair);
+  if (t >= pair_off[p.G] * tn_feature_tiles(p)) return false;
+  tl = decode_tn(p, pair_off, t);
+  ++wave;
+  return true;
 }
 
 __device__ __forceinline__ void st_shared32(uint32_t addr, uint32_t v) {
@@ -1814,13 +1267,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       uint32_t pending = 0, pend_parity = 0;
       int it = 0;
       bool ok = true;
-      TnCursor cur{kTnUnitOrder ? pair : 0, 0, pair};
+      int wave = 0;
       TnTile tl;
-      while (ok && tn_next(p, pair_off, npairs, cur, tl)) {
-        const int half = tl.nmma / 2;                                     // token columns per CTA
-        const int tokc = tl.tok0 + static_cast<int>(rank) * half;
-        const int nb32 = (!kTnRaggedBoxes || half == 128) ? 0 : (half + 31) / 32;
-        const uint32_t tx = 2 * (A_BYTES + (nb32 ? nb32 * 32 : 128) * BK * 2);
+      while (ok && tn_next(p, pair_off, npairs, pair, wave, tl)) {
+        // This CTA's token columns [tokc, tokc + nmma / 2), loaded as one 128-row box (rows past
+        // them are not read by the MMA).  Smaller boxes for ragged tiles measured slower: TMA
+        // delivery per copy has a fixed cost.
+        const int tokc = tl.tok0 + static_cast<int>(rank) * (tl.nmma / 2);
+        const uint32_t tx = 2 * stage_bytes;
         for (int kb = 0; kb < tl.nk; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
@@ -1849,12 +1303,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           } else {
             tma_load_3d_pair(sa, &p.tmA[src], fb, kk, tl.f0 + 128 * static_cast<int>(rank), tl.g);
           }
-          const int bsrc = p.nsplit ? 0 : src;
-          if (nb32 == 0) {
-            tma_load_3d_pair(sb, &p.tmB[bsrc], fb, kk, tokc, 0);
-          } else {
-            for (int j = 0; j < nb32; ++j) tma_load_3d_pair(sb + j * 32 * 128, &p.tmB32[bsrc], fb, kk, tokc + 32 * j, 0);
-          }
+          tma_load_3d_pair(sb, &p.tmB[p.nsplit ? 0 : src], fb, kk, tokc, 0);
           pending |= 1u << s;
           pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
         }
@@ -1871,9 +1320,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const uint32_t a_step = p.a_major ? 2048 : 32;
       int it = 0, tcount = 0;
       bool ok = true;
-      TnCursor cur{kTnUnitOrder ? pair : 0, 0, pair};
+      int wave = 0;
       TnTile tl;
-      for (; ok && tn_next(p, pair_off, npairs, cur, tl); ++tcount) {
+      for (; ok && tn_next(p, pair_off, npairs, pair, wave, tl); ++tcount) {
         const uint32_t idesc = idesc_bf16(2 * BM, tl.nmma, p.a_major, 0);
         const int buf = tcount & 1;
         const uint32_t aph = (tcount >> 1) & 1;
@@ -1918,9 +1367,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     Stager stg{smem_u32(stage_area + q * 2 * TN_SLAB), 0};
     const uint32_t aux = smem_u32(aux_area);
     int tcount = 0, xn = 0;
-    TnCursor cur{kTnUnitOrder ? pair : 0, 0, pair};
+    int wave = 0;
     TnTile tl;
-    for (; tn_next(p, pair_off, npairs, cur, tl); ++tcount) {
+    for (; tn_next(p, pair_off, npairs, pair, wave, tl); ++tcount) {
       const int buf = tcount & 1;
       const uint32_t aph = (tcount >> 1) & 1;
       if (!__all_sync(0xffffffffu, wait_bar2(smem_u32(&acc_full[buf]), aph, abort_flag, p.err))) break;
@@ -1961,7 +1410,8 @@ static int launch(Params& p, long long tile_upper_bound, const char* name, cudaS
   long long grid = num_sms();
   if (tile_upper_bound < grid) grid = tile_upper_bound;
   PFMOE_LAUNCH(name, stream,
-               (grouped_gemm_kernel<EPI, MODE><<<static_cast<int>(grid), THREADS, smem, stream>>>(p)));
+               (grouped_gemm_kernel<EPI, MODE><<<static_cast<int>(grid), MODE == KG ? THREADS_KG : THREADS, smem,
+                                                 stream>>>(p)));
   return PFMOE_OK;
 }
 
@@ -1974,35 +1424,6 @@ static int max_pairs() {
     cached = n > 0 ? n : 1;
   }
   return cached;
-}
-
-template <int EPI, int MODE = RG>
-static int launch2(Params& p, long long pair_tile_upper_bound, const char* name, cudaStream_t stream) {
-  p.mode = MODE;
-  // Each CTA loads bn/2 B columns: in 64-column boxes (MN-major), or rows of a bn/2-row box (K-major),
-  // and the stage's expected byte count assumes exactly that.
-  if (p.bn % 128 != 0 || p.bn > 256)
-    return fail(PFMOE_ERR_UNSUPPORTED, std::string(name) + ": two-SM tiles need bn in {128, 256}");
-  const int stage = A_BYTES + (p.bn / 2) * BK * 2;
-  const int poff = p.tiles ? ((p.G + 1 + 63) & ~63) * 4 : 0;
-  const int fixed = 1024 + 256 + poff + (kStaged2sm ? 4 * STAGE_BUFS * STAGE_BYTES_PER_WARP : 0);
-  int st = (SMEM_LIMIT - fixed) / stage;
-  p.stages = st > MAX_STAGES ? MAX_STAGES : st;
-  const size_t smem = fixed + static_cast<size_t>(p.stages) * stage;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(grouped_gemm_2sm_kernel<EPI, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(227 * 1024)) != cudaSuccess)
-      return fail(PFMOE_ERR_CUDA, std::string("cudaFuncSetAttribute failed: ") +
-                                      cudaGetErrorString(cudaGetLastError()));
-    attr_done = true;
-  }
-  if (pair_tile_upper_bound <= 0) return PFMOE_OK;
-  long long pairs = max_pairs();
-  if (pair_tile_upper_bound < pairs) pairs = pair_tile_upper_bound;
-  PFMOE_LAUNCH(name, stream,
-               (grouped_gemm_2sm_kernel<EPI, MODE><<<static_cast<int>(2 * pairs), THREADS, smem, stream>>>(p)));
-  return PFMOE_OK;
 }
 
 // Token-as-N launcher (expert-segmented rows only).
@@ -2037,20 +1458,6 @@ static long long tn_tiles_ub(int N, int E, int F, int fstep) {
   return (static_cast<long long>(N) / TN_TOK + E + 1) * ((F + fstep - 1) / fstep);
 }
 
-// Row-grouped expert GEMMs run on the token-as-N kernel (no spare rows on ragged segments).
-constexpr bool kTokenAsN = true;
-// Expert weight gradients run on the two-SM kernel (256-row output tiles: 1.5x fewer operand
-// bytes per FLOP than one-SM 128-row tiles).
-constexpr bool kPairWgrad = false;
-
-// Pair-tile upper bound: sum_e ceil(n_e / 256) <= N / 256 + E.
-static long long rg_pairs_ub(int N, int E, int Nout, int nstep) {
-  return (static_cast<long long>(N) / (2 * BM) + E + 1) * ((Nout + nstep - 1) / nstep);
-}
-
-// The two-SM kernel pays for half-empty pair tiles on small expert segments; use it when the
-// average segment holds at least one full 256-row pair tile.
-static bool use_pairs(int N, int E) { return N >= 2 * BM * E; }
 
 static Params base_params(int32_t* err) {
   Params p;
@@ -2107,152 +1514,88 @@ static int launch_split_reduce(const float* parts, int nparts, long long n, cons
 
 using namespace tc;
 
-// Row-tile upper bound for expert-segmented rows: sum_e ceil(n_e / 128) <= N / 128 + E.
-static long long rg_tiles_ub(int N, int E, int Nout, int nstep) {
-  return (static_cast<long long>(N) / BM + E + 1) * ((Nout + nstep - 1) / nstep);
-}
+// Expert GEMMs over the PFT rows (token-as-N kernel).  seg = expert_offsets, tiles = the
+// 128-row tile prefix from pft_build (the kernel derives its 256-token tile counts from it).
 
+// H1 = X_pft W1_e, H3 = X_pft W3_e, A = SiLU(H1) * H3 (X-MoE article §2.1.2, SwiGLU expert).
 int tc_ffn_gemm1(const void* x_pft, const int* seg, const int* tiles, int N, int E, int d, int h,
                  const void* w1, const void* w3, void* h1, void* h3, void* a, int32_t* err, cudaStream_t s) {
   Params p = base_params(err);
-  p.mode = RG;
-  p.b_major = 1;
-  p.bn = h > 64 ? 256 : 128;
   p.nsplit = 1;
   p.Nout = h;
   p.k0_blocks = (d + BK - 1) / BK;
   p.seg = seg; p.tiles = tiles; p.G = E;
   p.D0 = h1; p.D1 = h3; p.D2 = a; p.ldd = h;
-  if (kTokenAsN) {
-    p.a_major = 1;            // W1_e, W3_e [d, h]: K rows, features contiguous
-    p.fstep = 128;            // 64 features of W1 and the same 64 of W3 per CTA
-    PFMOE_TRY(make_tmap(&p.tmA[0], w1, h, d, E, 64, 64, "w1"));
-    PFMOE_TRY(make_tmap(&p.tmA[1], w3, h, d, E, 64, 64, "w3"));
-    PFMOE_TRY(make_tmap(&p.tmB[0], x_pft, d, N, 1, BK, 128, "x_pft"));
-    PFMOE_TRY(make_tmap(&p.tmB32[0], x_pft, d, N, 1, BK, 32, "x_pft"));
-    PFMOE_TRY(make_out_map_tn(&p.tmD[0], h1, h, N, "h1 out"));
-    PFMOE_TRY(make_out_map_tn(&p.tmD[1], h3, h, N, "h3 out"));
-    PFMOE_TRY(make_out_map_tn(&p.tmD[2], a, h, N, "a out"));
-    p.tma_store = 1;
-    return launch_tn<EPI_SWIGLU_FWD>(p, tn_tiles_ub(N, E, h, p.fstep), "ffn_gemm1_swiglu", s);
-  }
-  PFMOE_TRY(make_tmap(&p.tmA[0], x_pft, d, N, 1, BK, BM, "x_pft"));
-  PFMOE_TRY(make_tmap(&p.tmB[0], w1, h, d, E, 64, 64, "w1"));
-  PFMOE_TRY(make_tmap(&p.tmB[1], w3, h, d, E, 64, 64, "w3"));
-  if (use_pairs(N, E)) {
-    PFMOE_TRY(make_out_map(&p.tmD[0], h1, h, N, 1, "h1 out"));
-    PFMOE_TRY(make_out_map(&p.tmD[1], h3, h, N, 1, "h3 out"));
-    PFMOE_TRY(make_out_map(&p.tmD[2], a, h, N, 1, "a out"));
-    p.tma_store = 1;
-    return launch2<EPI_SWIGLU_FWD>(p, rg_pairs_ub(N, E, h, p.bn / 2), "ffn_gemm1_swiglu", s);
-  }
-  return launch<EPI_SWIGLU_FWD, RG>(p, rg_tiles_ub(N, E, h, p.bn / 2), "ffn_gemm1_swiglu", s);
+  p.a_major = 1;            // W1_e, W3_e [d, h]: K rows, features contiguous
+  p.fstep = 128;            // 64 features of W1 and the same 64 of W3 per CTA
+  PFMOE_TRY(make_tmap(&p.tmA[0], w1, h, d, E, 64, 64, "w1"));
+  PFMOE_TRY(make_tmap(&p.tmA[1], w3, h, d, E, 64, 64, "w3"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], x_pft, d, N, 1, BK, 128, "x_pft"));
+  PFMOE_TRY(make_out_map_tn(&p.tmD[0], h1, h, N, "h1 out"));
+  PFMOE_TRY(make_out_map_tn(&p.tmD[1], h3, h, N, "h3 out"));
+  PFMOE_TRY(make_out_map_tn(&p.tmD[2], a, h, N, "a out"));
+  p.tma_store = 1;
+  return launch_tn<EPI_SWIGLU_FWD>(p, tn_tiles_ub(N, E, h, p.fstep), "ffn_gemm1_swiglu", s);
 }
 
+// O = A W2_e.
 int tc_ffn_gemm2(const void* a, const int* seg, const int* tiles, int N, int E, int d, int h, const void* w2,
                  void* out, int32_t* err, cudaStream_t s) {
   Params p = base_params(err);
-  p.mode = RG;
-  p.b_major = 1;
-  p.bn = round_bn(d);
   p.Nout = d;
   p.k0_blocks = (h + BK - 1) / BK;
   p.seg = seg; p.tiles = tiles; p.G = E;
   p.D0 = out; p.ldd = d;
-  if (kTokenAsN) {
-    p.a_major = 1;            // W2_e [h, d]: K rows, features contiguous
-    p.fstep = 2 * BM;
-    p.a_merged = d % 64 == 0;
-    if (p.a_merged) PFMOE_TRY(make_tmap_mn(&p.tmA[0], w2, d, h, E, BK, 2, "w2"));
-    else PFMOE_TRY(make_tmap(&p.tmA[0], w2, d, h, E, 64, 64, "w2"));
-    PFMOE_TRY(make_tmap(&p.tmB[0], a, h, N, 1, BK, 128, "a"));
-    PFMOE_TRY(make_tmap(&p.tmB32[0], a, h, N, 1, BK, 32, "a"));
-    PFMOE_TRY(make_out_map_tn(&p.tmD[0], out, d, N, "out"));
-    p.tma_store = 1;
-    return launch_tn<EPI_STORE_BF16>(p, tn_tiles_ub(N, E, d, p.fstep), "ffn_gemm2", s);
-  }
-  PFMOE_TRY(make_tmap(&p.tmA[0], a, h, N, 1, BK, BM, "a"));
-  PFMOE_TRY(make_tmap(&p.tmB[0], w2, d, h, E, 64, 64, "w2"));
-  if (use_pairs(N, E)) {
-    PFMOE_TRY(make_out_map(&p.tmD[0], out, d, N, 1, "out"));
-    p.tma_store = 1;
-    return launch2<EPI_STORE_BF16>(p, rg_pairs_ub(N, E, d, p.bn), "ffn_gemm2", s);
-  }
-  return launch<EPI_STORE_BF16, RG>(p, rg_tiles_ub(N, E, d, p.bn), "ffn_gemm2", s);
+  p.a_major = 1;            // W2_e [h, d]: K rows, features contiguous
+  p.fstep = 2 * BM;
+  p.a_merged = d % 64 == 0;
+  if (p.a_merged) PFMOE_TRY(make_tmap_mn(&p.tmA[0], w2, d, h, E, BK, 2, "w2"));
+  else PFMOE_TRY(make_tmap(&p.tmA[0], w2, d, h, E, 64, 64, "w2"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], a, h, N, 1, BK, 128, "a"));
+  PFMOE_TRY(make_out_map_tn(&p.tmD[0], out, d, N, "out"));
+  p.tma_store = 1;
+  return launch_tn<EPI_STORE_BF16>(p, tn_tiles_ub(N, E, d, p.fstep), "ffn_gemm2", s);
 }
 
+// dA = dO W2_e^T, then dH1 = dA * H3 * s * (1 + H1 (1 - s)), dH3 = dA * SiLU(H1) in the epilogue.
 int tc_ffn_dgrad_act(const void* dO, const int* seg, const int* tiles, int N, int E, int d, int h, const void* w2,
                      const void* h1, const void* h3, void* dh1, void* dh3, int32_t* err, cudaStream_t s) {
   Params p = base_params(err);
-  p.mode = RG;
-  p.b_major = 0;              // W2_e [h, d]: rows = output columns (h), K = d contiguous
-  p.bn = round_bn(h);
   p.Nout = h;
   p.k0_blocks = (d + BK - 1) / BK;
   p.seg = seg; p.tiles = tiles; p.G = E;
   p.X0 = h1; p.X1 = h3; p.D0 = dh1; p.D1 = dh3; p.ldd = h;
-  if (kTokenAsN) {
-    p.a_major = 0;            // W2_e [h, d]: feature rows, K = d contiguous
-    p.fstep = 2 * BM;
-    PFMOE_TRY(make_tmap(&p.tmA[0], w2, d, h, E, BK, 128, "w2^T"));
-    PFMOE_TRY(make_tmap(&p.tmB[0], dO, d, N, 1, BK, 128, "dO"));
-    PFMOE_TRY(make_tmap(&p.tmB32[0], dO, d, N, 1, BK, 32, "dO"));
-    PFMOE_TRY(make_out_map_tn(&p.tmD[0], dh1, h, N, "dh1 out"));
-    PFMOE_TRY(make_out_map_tn(&p.tmD[1], dh3, h, N, "dh3 out"));
-    p.tma_store = 1;
-    return launch_tn<EPI_SWIGLU_BWD>(p, tn_tiles_ub(N, E, h, p.fstep), "ffn_dgrad_act_swiglu_bwd", s);
-  }
-  const bool pairs = use_pairs(N, E);
-  const uint32_t brows = pairs ? p.bn / 2 : p.bn;   // B rows loaded per CTA
-  PFMOE_TRY(make_tmap(&p.tmA[0], dO, d, N, 1, BK, BM, "dO"));
-  PFMOE_TRY(make_tmap(&p.tmB[0], w2, d, h, E, BK, brows, "w2^T"));
-  if (pairs) {
-    PFMOE_TRY(make_out_map(&p.tmD[0], dh1, h, N, 1, "dh1 out"));
-    PFMOE_TRY(make_out_map(&p.tmD[1], dh3, h, N, 1, "dh3 out"));
-    p.tma_store = 1;
-    return launch2<EPI_SWIGLU_BWD>(p, rg_pairs_ub(N, E, h, p.bn), "ffn_dgrad_act_swiglu_bwd", s);
-  }
-  return launch<EPI_SWIGLU_BWD, RG>(p, rg_tiles_ub(N, E, h, p.bn), "ffn_dgrad_act_swiglu_bwd", s);
+  p.a_major = 0;            // W2_e [h, d]: feature rows, K = d contiguous
+  p.fstep = 2 * BM;
+  PFMOE_TRY(make_tmap(&p.tmA[0], w2, d, h, E, BK, 128, "w2^T"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], dO, d, N, 1, BK, 128, "dO"));
+  PFMOE_TRY(make_out_map_tn(&p.tmD[0], dh1, h, N, "dh1 out"));
+  PFMOE_TRY(make_out_map_tn(&p.tmD[1], dh3, h, N, "dh3 out"));
+  p.tma_store = 1;
+  return launch_tn<EPI_SWIGLU_BWD>(p, tn_tiles_ub(N, E, h, p.fstep), "ffn_dgrad_act_swiglu_bwd", s);
 }
 
+// dX_pft = dH1 W1_e^T + dH3 W3_e^T (one K loop over both sources).
 int tc_ffn_dgrad_x(const void* dh1, const void* dh3, const int* seg, const int* tiles, int N, int E, int d, int h,
                    const void* w1, const void* w3, void* dx_pft, int32_t* err, cudaStream_t s) {
   Params p = base_params(err);
-  p.mode = RG;
-  p.b_major = 0;              // W1_e [d, h]: rows = output columns (d), K = h contiguous
-  p.bn = round_bn(d);
   p.Nout = d;
   p.k0_blocks = (h + BK - 1) / BK;
   p.k1_blocks = (h + BK - 1) / BK;
   p.seg = seg; p.tiles = tiles; p.G = E;
   p.D0 = dx_pft; p.ldd = d;
-  if (kTokenAsN) {
-    p.a_major = 0;            // W1_e, W3_e [d, h]: feature rows, K = h contiguous
-    p.fstep = 2 * BM;
-    PFMOE_TRY(make_tmap(&p.tmA[0], w1, h, d, E, BK, 128, "w1^T"));
-    PFMOE_TRY(make_tmap(&p.tmA[1], w3, h, d, E, BK, 128, "w3^T"));
-    PFMOE_TRY(make_tmap(&p.tmB[0], dh1, h, N, 1, BK, 128, "dh1"));
-    PFMOE_TRY(make_tmap(&p.tmB[1], dh3, h, N, 1, BK, 128, "dh3"));
-    PFMOE_TRY(make_tmap(&p.tmB32[0], dh1, h, N, 1, BK, 32, "dh1"));
-    PFMOE_TRY(make_tmap(&p.tmB32[1], dh3, h, N, 1, BK, 32, "dh3"));
-    PFMOE_TRY(make_out_map_tn(&p.tmD[0], dx_pft, d, N, "dx_pft out"));
-    p.tma_store = 1;
-    return launch_tn<EPI_STORE_BF16>(p, tn_tiles_ub(N, E, d, p.fstep), "ffn_dgrad_x", s);
-  }
-  const bool pairs = use_pairs(N, E);
-  const uint32_t brows = pairs ? p.bn / 2 : p.bn;   // B rows loaded per CTA
-  PFMOE_TRY(make_tmap(&p.tmA[0], dh1, h, N, 1, BK, BM, "dh1"));
-  PFMOE_TRY(make_tmap(&p.tmA[1], dh3, h, N, 1, BK, BM, "dh3"));
-  PFMOE_TRY(make_tmap(&p.tmB[0], w1, h, d, E, BK, brows, "w1^T"));
-  PFMOE_TRY(make_tmap(&p.tmB[1], w3, h, d, E, BK, brows, "w3^T"));
-  if (pairs) {
-    PFMOE_TRY(make_out_map(&p.tmD[0], dx_pft, d, N, 1, "dx_pft out"));
-    p.tma_store = 1;
-    return launch2<EPI_STORE_BF16>(p, rg_pairs_ub(N, E, d, p.bn), "ffn_dgrad_x", s);
-  }
-  return launch<EPI_STORE_BF16, RG>(p, rg_tiles_ub(N, E, d, p.bn), "ffn_dgrad_x", s);
+  p.a_major = 0;            // W1_e, W3_e [d, h]: feature rows, K = h contiguous
+  p.fstep = 2 * BM;
+  PFMOE_TRY(make_tmap(&p.tmA[0], w1, h, d, E, BK, 128, "w1^T"));
+  PFMOE_TRY(make_tmap(&p.tmA[1], w3, h, d, E, BK, 128, "w3^T"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], dh1, h, N, 1, BK, 128, "dh1"));
+  PFMOE_TRY(make_tmap(&p.tmB[1], dh3, h, N, 1, BK, 128, "dh3"));
+  PFMOE_TRY(make_out_map_tn(&p.tmD[0], dx_pft, d, N, "dx_pft out"));
+  p.tma_store = 1;
+  return launch_tn<EPI_STORE_BF16>(p, tn_tiles_ub(N, E, d, p.fstep), "ffn_dgrad_x", s);
 }
 
+// dW1_e = X_e^T dH1_e, dW3_e = X_e^T dH3_e (K-grouped over the expert's PFT rows).
 int tc_ffn_wgrad13(const void* x_pft, const void* dh1, const void* dh3, const int* seg, int N, int E, int d, int h,
                    void* dw1, void* dw3, int32_t* err, cudaStream_t s) {
   Params p = base_params(err);
@@ -2279,38 +1622,29 @@ int tc_ffn_wgrad13(const void* x_pft, const void* dh1, const void* dh3, const in
   PFMOE_TRY(make_out_map(&p.tmD[0], dw1, h, d, E, "dw1 out"));
   PFMOE_TRY(make_out_map(&p.tmD[1], dw3, h, d, E, "dw3 out"));
   p.tma_store = 1;
-  if (kPairWgrad) {
-    const long long ub = static_cast<long long>(E) * ((d + 2 * BM - 1) / (2 * BM)) * ((h + p.bn / 2 - 1) / (p.bn / 2));
-    return launch2<EPI_SPLIT_BF16, KG>(p, ub, "ffn_wgrad_w1w3", s);
-  }
   const long long ub = static_cast<long long>(E) * ((d + BM - 1) / BM) * ((h + p.bn / 2 - 1) / (p.bn / 2));
   return launch<EPI_SPLIT_BF16, KG>(p, ub, "ffn_wgrad_w1w3", s);
 }
 
+// dW2_e = A_e^T dO_e.
 int tc_ffn_wgrad2(const void* a, const void* dO, const int* seg, int N, int E, int d, int h, void* dw2,
                   int32_t* err, cudaStream_t s) {
   Params p = base_params(err);
   p.mode = KG;
   p.b_major = 1;
-  p.bn = kPairWgrad ? round_bn_pair(d) : round_bn(d);
+  p.bn = round_bn(d);
   p.M = h;
   p.Nout = d;
   p.seg = seg; p.G = E;
   p.D0 = dw2; p.ldd = d; p.d_gstride = static_cast<long long>(h) * d;
   p.a_merged = h % 64 == 0;
   p.b_merged = d % 64 == 0;
-  // one-SM tiles load all bn columns of B; two-SM tiles bn / 2 per CTA
-  const uint32_t bblk2 = (kPairWgrad ? p.bn / 2 : p.bn) / 64;
   if (p.a_merged) PFMOE_TRY(make_tmap_mn(&p.tmA[0], a, h, N, 1, BK, 2, "a^T"));
   else PFMOE_TRY(make_tmap(&p.tmA[0], a, h, N, 1, 64, 64, "a^T"));
-  if (p.b_merged) PFMOE_TRY(make_tmap_mn(&p.tmB[0], dO, d, N, 1, BK, bblk2, "dO"));
+  if (p.b_merged) PFMOE_TRY(make_tmap_mn(&p.tmB[0], dO, d, N, 1, BK, p.bn / 64, "dO"));
   else PFMOE_TRY(make_tmap(&p.tmB[0], dO, d, N, 1, 64, 64, "dO"));
   PFMOE_TRY(make_out_map(&p.tmD[0], dw2, d, h, E, "dw2 out"));
   p.tma_store = 1;
-  if (kPairWgrad) {
-    const long long ub = static_cast<long long>(E) * ((h + 2 * BM - 1) / (2 * BM)) * ((d + p.bn - 1) / p.bn);
-    return launch2<EPI_STORE_BF16, KG>(p, ub, "ffn_wgrad_w2", s);
-  }
   const long long ub = static_cast<long long>(E) * ((h + BM - 1) / BM) * ((d + p.bn - 1) / p.bn);
   return launch<EPI_STORE_BF16, KG>(p, ub, "ffn_wgrad_w2", s);
 }

@@ -78,8 +78,14 @@ __global__ void __launch_bounds__(WARPS * 32) dispatch_kernel(const T* __restric
 template <typename T>
 __host__ __device__ inline int chunk_cols() { return 32 * Vec<T>::n; }
 
-// y[t] = sum_j w[t, j] * O[pos[t, j]].
-template <typename T>
+// Items per token when each item covers U column chunks.
+__host__ __device__ inline int items_per_token(int d, int vn, int U) {
+  const int C = (d + 32 * vn - 1) / (32 * vn);
+  return (C + U - 1) / U;
+}
+
+// y[t] = sum_j w[t, j] * O[pos[t, j]].  An item covers U consecutive column chunks.
+template <typename T, int U>
 __global__ void __launch_bounds__(WARPS * 32) combine_kernel(const T* __restrict__ O, const int32_t* __restrict__ pos,
                                                              const float* __restrict__ w, int Tn, int k, int d,
                                                              T* __restrict__ y, int32_t* err) {
@@ -87,29 +93,39 @@ __global__ void __launch_bounds__(WARPS * 32) combine_kernel(const T* __restrict
   const int lane = threadIdx.x & 31;
   const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   const long long N = static_cast<long long>(Tn) * k;
-  const int C = (d + chunk_cols<T>() - 1) / chunk_cols<T>();
-  const long long items = static_cast<long long>(Tn) * C;
+  const int CU = items_per_token(d, VN, U);
+  const long long items = static_cast<long long>(Tn) * CU;
   for (long long it = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; it < items; it += nw) {
-    const long long t = it / C;
-    const int c0 = static_cast<int>(it - t * C) * chunk_cols<T>() + lane * VN;
+    const long long t = it / CU;
+    const int cb = static_cast<int>(it - t * CU) * U * chunk_cols<T>() + lane * VN;
     int my_pos;
     if (!load_pos(pos, t, k, N, lane, my_pos, err)) continue;
     const float my_w = lane < k ? w[t * k + lane] : 0.f;
-    float acc[VN];
+    float acc[U][VN];
 #pragma unroll
-    for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int i = 0; i < VN; ++i) acc[u][i] = 0.f;
 #pragma unroll 8
     for (int j = 0; j < k; ++j) {
       const long long p = __shfl_sync(0xffffffffu, my_pos, j);
       const float wj = __shfl_sync(0xffffffffu, my_w, j);
-      if (c0 < d) {
-        float o[VN];
-        load16(O + p * d + c0, o);
 #pragma unroll
-        for (int i = 0; i < VN; ++i) acc[i] = fmaf(wj, o[i], acc[i]);
+      for (int u = 0; u < U; ++u) {
+        const int c0 = cb + u * chunk_cols<T>();
+        if (c0 < d) {
+          float o[VN];
+          load16(O + p * d + c0, o);
+#pragma unroll
+          for (int i = 0; i < VN; ++i) acc[u][i] = fmaf(wj, o[i], acc[u][i]);
+        }
       }
     }
-    if (c0 < d) store16(y + t * d + c0, acc);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c0 = cb + u * chunk_cols<T>();
+      if (c0 < d) store16(y + t * d + c0, acc[u]);
+    }
   }
 }
 
@@ -156,7 +172,7 @@ __global__ void __launch_bounds__(WARPS * 32) combine_bwd_kernel(const T* __rest
 // dz_{t, ids[t,j]} = w_j (g_j - sum_l w_l g_l) (zero elsewhere);
 // dx[t] = sum_j dX_pft[pos[t, j]] + sum_j dz_j * Wg^T[ids[t, j]].
 // The dense dlogits row (and its BF16 copy for the dWg GEMM) is written by the token's chunk-0 item.
-template <typename T>
+template <typename T, int U>
 __global__ void __launch_bounds__(WARPS * 32) token_grad_kernel(const T* __restrict__ dxp, const int32_t* __restrict__ pos,
                                                                 const float* __restrict__ g, const float* __restrict__ w,
                                                                 const int32_t* __restrict__ ids,
@@ -167,12 +183,12 @@ __global__ void __launch_bounds__(WARPS * 32) token_grad_kernel(const T* __restr
   const int lane = threadIdx.x & 31;
   const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   const long long N = static_cast<long long>(Tn) * k;
-  const int C = (d + chunk_cols<T>() - 1) / chunk_cols<T>();
-  const long long items = static_cast<long long>(Tn) * C;
+  const int CU = items_per_token(d, VN, U);
+  const long long items = static_cast<long long>(Tn) * CU;
   for (long long it = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; it < items; it += nw) {
-    const long long t = it / C;
-    const int ch = static_cast<int>(it - t * C);
-    const int c0 = ch * chunk_cols<T>() + lane * VN;
+    const long long t = it / CU;
+    const int ch = static_cast<int>(it - t * CU);
+    const int cb = ch * U * chunk_cols<T>() + lane * VN;
     int my_pos;
     if (!load_pos(pos, t, k, N, lane, my_pos, err)) continue;
     const long long tk = t * k;
@@ -200,32 +216,45 @@ __global__ void __launch_bounds__(WARPS * 32) token_grad_kernel(const T* __restr
         }
       }
     }
-    const bool act = c0 < d;
-    float acc[VN];
+    float acc[U][VN];
 #pragma unroll
-    for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int i = 0; i < VN; ++i) acc[u][i] = 0.f;
 #pragma unroll 8
     for (int j = 0; j < k; ++j) {
       const long long p = __shfl_sync(0xffffffffu, my_pos, j);
-      if (act) {
-        float v[VN];
-        load16(dxp + p * d + c0, v);
 #pragma unroll
-        for (int i = 0; i < VN; ++i) acc[i] += v[i];
+      for (int u = 0; u < U; ++u) {
+        const int c0 = cb + u * chunk_cols<T>();
+        if (c0 < d) {
+          float v[VN];
+          load16(dxp + p * d + c0, v);
+#pragma unroll
+          for (int i = 0; i < VN; ++i) acc[u][i] += v[i];
+        }
       }
     }
 #pragma unroll 8
     for (int j = 0; j < k; ++j) {
       const long long idj = __shfl_sync(0xffffffffu, my_id, j);
       const float dzj = __shfl_sync(0xffffffffu, my_dz, j);
-      if (act) {
-        float v[VN];
-        load16(wgT + idj * d + c0, v);
 #pragma unroll
-        for (int i = 0; i < VN; ++i) acc[i] = fmaf(dzj, v[i], acc[i]);
+      for (int u = 0; u < U; ++u) {
+        const int c0 = cb + u * chunk_cols<T>();
+        if (c0 < d) {
+          float v[VN];
+          load16(wgT + idj * d + c0, v);
+#pragma unroll
+          for (int i = 0; i < VN; ++i) acc[u][i] = fmaf(dzj, v[i], acc[u][i]);
+        }
       }
     }
-    if (act) store16(dx + t * d + c0, acc);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c0 = cb + u * chunk_cols<T>();
+      if (c0 < d) store16(dx + t * d + c0, acc[u]);
+    }
   }
 }
 
@@ -262,18 +291,25 @@ int launch_dispatch(const void* x, const int32_t* pos, int T, int k, int d, int 
   return PFMOE_OK;
 }
 
+// Column chunks per work item: one for rows of up to 16 chunks (d <= 4096 BF16), else 4, which
+// keeps the per-token prologue (pos / weight loads, dlogits row) off wide rows.
+static int chunks_per_item(int d, int vn) { return (d + 32 * vn - 1) / (32 * vn) > 16 ? 4 : 1; }
+
 int launch_combine(const void* out, const int32_t* pos, const float* w, int T, int k, int d, int dtype, void* y,
                    int32_t* err, cudaStream_t s) {
   const int vn = dtype == PFMOE_BF16 ? 8 : 4;
-  const int g = item_grid(static_cast<long long>(T) * ((d + 32 * vn - 1) / (32 * vn)));
+  const int U = chunks_per_item(d, vn);
+  const int g = item_grid(static_cast<long long>(T) * items_per_token(d, vn, U));
   if (dtype == PFMOE_BF16) {
-    PFMOE_LAUNCH("combine", s,
-                 combine_kernel<__nv_bfloat16><<<g, WARPS * 32, 0, s>>>(
-                     static_cast<const __nv_bfloat16*>(out), pos, w, T, k, d, static_cast<__nv_bfloat16*>(y), err));
+    const auto* o = static_cast<const __nv_bfloat16*>(out);
+    auto* yy = static_cast<__nv_bfloat16*>(y);
+    if (U == 4) PFMOE_LAUNCH("combine", s, (combine_kernel<__nv_bfloat16, 4><<<g, WARPS * 32, 0, s>>>(o, pos, w, T, k, d, yy, err)));
+    else PFMOE_LAUNCH("combine", s, (combine_kernel<__nv_bfloat16, 1><<<g, WARPS * 32, 0, s>>>(o, pos, w, T, k, d, yy, err)));
   } else {
-    PFMOE_LAUNCH("combine", s,
-                 combine_kernel<float><<<g, WARPS * 32, 0, s>>>(static_cast<const float*>(out), pos, w, T, k, d,
-                                                                static_cast<float*>(y), err));
+    const auto* o = static_cast<const float*>(out);
+    auto* yy = static_cast<float*>(y);
+    if (U == 4) PFMOE_LAUNCH("combine", s, (combine_kernel<float, 4><<<g, WARPS * 32, 0, s>>>(o, pos, w, T, k, d, yy, err)));
+    else PFMOE_LAUNCH("combine", s, (combine_kernel<float, 1><<<g, WARPS * 32, 0, s>>>(o, pos, w, T, k, d, yy, err)));
   }
   return PFMOE_OK;
 }
@@ -313,18 +349,29 @@ int launch_token_grad(const void* dx_pft, const int32_t* pos, const float* g, co
                       const void* wgT, int T, int k, int d, int E, int dtype, void* dx, float* dlogits,
                       void* dz_bf16, int32_t* err, cudaStream_t s) {
   const int vn = dtype == PFMOE_BF16 ? 8 : 4;
-  const int gr = item_grid(static_cast<long long>(T) * ((d + 32 * vn - 1) / (32 * vn)));
+  const int U = chunks_per_item(d, vn);
+  const int gr = item_grid(static_cast<long long>(T) * items_per_token(d, vn, U));
+  auto* dzb = static_cast<__nv_bfloat16*>(dz_bf16);
   if (dtype == PFMOE_BF16) {
-    PFMOE_LAUNCH("token_grad", s,
-                 token_grad_kernel<__nv_bfloat16><<<gr, WARPS * 32, 0, s>>>(
-                     static_cast<const __nv_bfloat16*>(dx_pft), pos, g, w, ids,
-                     static_cast<const __nv_bfloat16*>(wgT), T, k, d, E, static_cast<__nv_bfloat16*>(dx), dlogits,
-                     static_cast<__nv_bfloat16*>(dz_bf16), err));
+    const auto* a = static_cast<const __nv_bfloat16*>(dx_pft);
+    const auto* wt = static_cast<const __nv_bfloat16*>(wgT);
+    auto* o = static_cast<__nv_bfloat16*>(dx);
+    if (U == 4)
+      PFMOE_LAUNCH("token_grad", s, (token_grad_kernel<__nv_bfloat16, 4><<<gr, WARPS * 32, 0, s>>>(
+                                         a, pos, g, w, ids, wt, T, k, d, E, o, dlogits, dzb, err)));
+    else
+      PFMOE_LAUNCH("token_grad", s, (token_grad_kernel<__nv_bfloat16, 1><<<gr, WARPS * 32, 0, s>>>(
+                                         a, pos, g, w, ids, wt, T, k, d, E, o, dlogits, dzb, err)));
   } else {
-    PFMOE_LAUNCH("token_grad", s,
-                 token_grad_kernel<float><<<gr, WARPS * 32, 0, s>>>(
-                     static_cast<const float*>(dx_pft), pos, g, w, ids, static_cast<const float*>(wgT), T, k, d, E,
-                     static_cast<float*>(dx), dlogits, static_cast<__nv_bfloat16*>(dz_bf16), err));
+    const auto* a = static_cast<const float*>(dx_pft);
+    const auto* wt = static_cast<const float*>(wgT);
+    auto* o = static_cast<float*>(dx);
+    if (U == 4)
+      PFMOE_LAUNCH("token_grad", s, (token_grad_kernel<float, 4><<<gr, WARPS * 32, 0, s>>>(
+                                         a, pos, g, w, ids, wt, T, k, d, E, o, dlogits, dzb, err)));
+    else
+      PFMOE_LAUNCH("token_grad", s, (token_grad_kernel<float, 1><<<gr, WARPS * 32, 0, s>>>(
+                                         a, pos, g, w, ids, wt, T, k, d, E, o, dlogits, dzb, err)));
   }
   return PFMOE_OK;
 }

@@ -79,11 +79,14 @@ SMALL = {
                              rbd_epd=3, rbd_dpn=1),
     "one_token_bf16": LayerConfig("one_token_bf16", T=1, d=64, E=8, h=64, k=2, dtype="bf16",
                                   rbd_epd=2, rbd_dpn=2),
-    # >= 256 rows per expert on average: exercises the two-SM (256-row pair tile) GEMMs,
-    # with ragged segment ends, pair tiles whose second half is empty, and d, h that are
-    # not multiples of the N tile.
+    # >= 256 rows per expert on average: full 256-token tiles of the token-as-N GEMMs next to
+    # ragged tails, and d, h that are not multiples of the feature tile.
     "small_pairs_bf16": LayerConfig("small_pairs_bf16", T=1100, d=320, E=8, h=136, k=2, dtype="bf16",
                                     rbd_epd=2, rbd_dpn=2),
+    # rows wider than 16 column chunks: the gather-sum kernels take 4 chunks per work item,
+    # and the last item of every row is partial (17 and 18 chunks).
+    "wide_d_bf16": LayerConfig("wide_d_bf16", T=96, d=4160, E=8, h=64, k=3, dtype="bf16"),
+    "wide_d_f32": LayerConfig("wide_d_f32", T=40, d=2200, E=6, h=40, k=2, dtype="f32"),
 }
 
 
