@@ -309,13 +309,14 @@ def run_ours(args):
 
     # ---- the same steps again with a CUDA event pair around every kernel launch (on the
     # stream it is launched on): per-kernel durations for the roofline and launch counts.
-    # Kept out of the headline pass because the events add host-side gaps between kernels.
+    # Kept out of the headline pass because the events add host-side gaps between kernels;
+    # the RBD plan runs in line here so that each event pair times one kernel's own work.
     L.moe_profile_reset()
     barrier()
     torch.cuda.synchronize()
     L.moe_profile_enable(True)
     for _ in range(args.steps):
-        step()
+        layer.step(inp.x, inp.wg, inp.bias, inp.w1, inp.w3, inp.w2, inp.dy, stream, overlap_rbd=False)
     torch.cuda.synchronize()
     L.moe_profile_enable(False)
     barrier()

@@ -146,14 +146,17 @@ class PFTMoELayer:
                    self.pilot_token, self.pilot_node, self.pilot_device, self.replica_offsets, self.replica_expert,
                    self.assign_pilot, self.rbd_counts, self.rbd_ws, self.rbd_ws_bytes, self.err, stream)
 
-    def step(self, x, wg, bias, w1, w3, w2, dy, stream=None):
+    def step(self, x, wg, bias, w1, w3, w2, dy, stream=None, overlap_rbd=True):
         """One pass of the whole hot path: forward, RBD plan (if mapped), backward.
 
         With an RBD map the plan runs on a side stream forked after routing and joined
-        before return, overlapping the PFT build, the expert GEMMs and the backward."""
+        before return, overlapping the PFT build, the expert GEMMs and the backward
+        (overlap_rbd=False runs it in line after routing instead)."""
         main = stream if stream is not None else torch.cuda.current_stream(self.device)
         self.route(x, wg, bias, main)
-        if self.has_rbd:
+        if self.has_rbd and not overlap_rbd:
+            self.rbd(main)
+        elif self.has_rbd:
             self.ev_routed.record(main)
             self.side.wait_event(self.ev_routed)
             self.rbd(self.side)
@@ -163,7 +166,7 @@ class PFTMoELayer:
         self.experts(w1, w3, w2, main)
         self.combine(main)
         self.backward(dy, x, wg, w1, w3, w2, main)
-        if self.has_rbd:
+        if self.has_rbd and overlap_rbd:
             main.wait_event(self.ev_rbd_done)
 
     def device_error(self) -> int:
