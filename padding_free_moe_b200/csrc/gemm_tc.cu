@@ -935,12 +935,19 @@ __device__ __forceinline__ void tc_commit2_both(uint32_t bar) {
 // same lane of epilogue warps q and q + 2; warp q + 2 hands its FP32 H3 block
 // to warp q through shared memory (bounded mbarrier handshake).
 constexpr int TN_TOK = 256;             // tokens per pair tile
+// K depth of one ring stage: two 64-element sub-blocks, so each mbarrier handshake feeds eight
+// K16 MMAs.  Measured on this part: back-to-back M=256 N=256 pair MMAs take ~130 cycles each, and
+// a handshake every four of them costs ~30 % of that rate, one every eight none.
+constexpr int TN_BK = 2 * BK;
+constexpr int TN_SUB = 128 * BK * 2;    // one 64-deep sub-block of 128 rows (16 KB)
+constexpr int TN_STAGE = 4 * TN_SUB;    // A: 2 sub-blocks (or 2 feature blocks), B: 2 sub-blocks
 constexpr int TN_SLAB = 32 * 64;        // one 32-token x 32-feature BF16 block (64-byte rows)
 constexpr int TN_XBUF = 32 * 32 * 4;    // one 32 x 32 FP32 block
 
-__host__ __device__ constexpr int tn_aux_bytes(int epi) {
-  return epi == EPI_SWIGLU_FWD ? 2 * 2 * TN_XBUF : (epi == EPI_SWIGLU_BWD ? 4 * 2 * TN_SLAB : 0);
-}
+// SwiGLU forward: one FP32 hand-off block per warp pair.  (The SwiGLU backward reads its H1 / H3
+// blocks through the epilogue warp's own staging slabs.)
+__host__ __device__ constexpr int tn_aux_bytes(int epi) { return epi == EPI_SWIGLU_FWD ? 2 * TN_XBUF : 0; }
+constexpr int TN_STAGING = 4 * 2 * TN_SLAB;   // epilogue staging: 2 slabs per epilogue warp
 
 struct TnTile {
   int g, tok0, ntok, nmma, f0, nk;
@@ -1095,28 +1102,27 @@ __device__ __forceinline__ bool epilogue_tn(const Params& p, const TnTile& tl, u
       const int tok = tl.tok0 + 32 * c;
       const int rv = min(32, tl.ntok - 32 * c);
       const long long off = static_cast<long long>(tok) * ldd + fw;
-      const int b = xn & 1;
-      const uint32_t ph = (xn >> 1) & 1;
-      const uint32_t xb = aux + (pid * 2 + b) * TN_XBUF;
+      const uint32_t ph = xn & 1;                 // one hand-off buffer per pair: one phase per chunk
+      const uint32_t xb = aux + pid * TN_XBUF;
       float v[32];
       tmem_ld32(tacc + 32 * c, v);
       if (h3_warp) {
         emit_t(st, lane, v, tmd(p, 1), fw, tok, H3 + off, ldd, rv, fvalid);
-        if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&xempty[pid * 2 + b]), ph ^ 1, abort_flag, p.err)))
+        if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&xempty[pid]), ph ^ 1, abort_flag, p.err)))
           return false;
 #pragma unroll
         for (int j = 0; j < 32; ++j) st_shared32(xb + (j * 32 + lane) * 4, __float_as_uint(v[j]));
-        mbar_arrive(smem_u32(&xfull[pid * 2 + b]));
+        mbar_arrive(smem_u32(&xfull[pid]));
       } else {
         emit_t(st, lane, v, tmd(p, 0), fw, tok, H1 + off, ldd, rv, fvalid);
-        if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&xfull[pid * 2 + b]), ph, abort_flag, p.err)))
+        if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&xfull[pid]), ph, abort_flag, p.err)))
           return false;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const float h3 = __uint_as_float(ld_shared32(xb + (j * 32 + lane) * 4));
           v[j] = v[j] * sigmoid_fast(v[j]) * h3;
         }
-        mbar_arrive(smem_u32(&xempty[pid * 2 + b]));
+        mbar_arrive(smem_u32(&xempty[pid]));
         emit_t(st, lane, v, tmd(p, 2), fw, tok, A + off, ldd, rv, fvalid);
       }
     }
@@ -1142,8 +1148,10 @@ __device__ __forceinline__ bool epilogue_tn(const Params& p, const TnTile& tl, u
     const char* H3 = static_cast<const char*>(p.X1);
     __nv_bfloat16* dH1 = static_cast<__nv_bfloat16*>(p.D0);
     __nv_bfloat16* dH3 = static_cast<__nv_bfloat16*>(p.D1);
-    const uint32_t in1 = aux + q * 2 * TN_SLAB;
-    const uint32_t in3 = in1 + TN_SLAB;
+    // H1 / H3 blocks pass through this warp's two staging slabs, once the TMA stores that last
+    // used them have read them out.
+    const uint32_t in1 = st.base;
+    const uint32_t in3 = st.base + TN_SLAB;
     const int bv = min(64, fvalid * 2);
     uint4 r1[4], r3[4];
     {
@@ -1154,6 +1162,7 @@ __device__ __forceinline__ bool epilogue_tn(const Params& p, const TnTile& tl, u
     for (int c = 0; c < nch; ++c) {
       const int tok = tl.tok0 + 32 * c;
       const int rv = min(32, tl.ntok - 32 * c);
+      if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
       __syncwarp();
       put_t(in1, lane, r1);
       put_t(in3, lane, r3);
@@ -1166,6 +1175,7 @@ __device__ __forceinline__ bool epilogue_tn(const Params& p, const TnTile& tl, u
       float da[32], h1[32], h3[32];
       stage_t_read(in1, lane, h1);
       stage_t_read(in3, lane, h3);
+      __syncwarp();   // every lane has read the slabs before the first emit reuses one
       tmem_ld32(tacc + 32 * c, da);
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -1188,9 +1198,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages;
-  constexpr uint32_t stage_bytes = A_BYTES + 128 * BK * 2;   // 128 weight rows + 128 token rows
+  constexpr uint32_t stage_bytes = TN_STAGE;   // 128 weight rows + 128 token rows, 128 deep in K
   uint8_t* stage_area = smem + S * stage_bytes;               // 4 warps x 2 staging slabs
-  uint8_t* aux_area = stage_area + 4 * 2 * TN_SLAB;
+  uint8_t* aux_area = stage_area + TN_STAGING;
   int* pair_off = reinterpret_cast<int*>(aux_area + tn_aux_bytes(EPI));
   const int poff_ints = (p.G + 1 + 63) & ~63;
   uint8_t* bar_area = reinterpret_cast<uint8_t*>(pair_off + poff_ints);
@@ -1283,27 +1293,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           if (leader) mbar_expect_tx(fb_local, tx);
           const uint32_t fb = mapa_shared(fb_local, 0);
           const uint32_t sa = smem_u32(smem + s * stage_bytes);
-          const uint32_t sb = sa + A_BYTES;
+          const uint32_t sb = sa + 2 * TN_SUB;
           const int src = kb < p.k0_blocks ? 0 : 1;
-          const int kk = (src == 0 ? kb : kb - p.k0_blocks) * BK;
+          const int kk = (src == 0 ? kb : kb - p.k0_blocks) * TN_BK;
           if (p.a_major) {
+            // MN-major weights: 64-feature blocks of 128 K rows ([block][K row][128 B])
             if (p.nsplit) {
               const int f = tl.f0 + 64 * static_cast<int>(rank);
               tma_load_3d_pair(sa, &p.tmA[0], fb, f, kk, tl.g);
-              tma_load_3d_pair(sa + BOX_BYTES, &p.tmA[1], fb, f, kk, tl.g);
+              tma_load_3d_pair(sa + TN_SUB, &p.tmA[1], fb, f, kk, tl.g);
             } else {
               const int f = tl.f0 + 128 * static_cast<int>(rank);
               if (p.a_merged) {
                 tma_load_4d_pair(sa, &p.tmA[src], fb, 0, kk, f / 64, tl.g);
               } else {
                 tma_load_3d_pair(sa, &p.tmA[src], fb, f, kk, tl.g);
-                tma_load_3d_pair(sa + BOX_BYTES, &p.tmA[src], fb, f + 64, kk, tl.g);
+                tma_load_3d_pair(sa + TN_SUB, &p.tmA[src], fb, f + 64, kk, tl.g);
               }
             }
           } else {
-            tma_load_3d_pair(sa, &p.tmA[src], fb, kk, tl.f0 + 128 * static_cast<int>(rank), tl.g);
+            // K-major weights: two 64-deep sub-blocks of 128 feature rows ([sub-block][row][128 B])
+            const int f = tl.f0 + 128 * static_cast<int>(rank);
+            tma_load_3d_pair(sa, &p.tmA[src], fb, kk, f, tl.g);
+            tma_load_3d_pair(sa + TN_SUB, &p.tmA[src], fb, kk + BK, f, tl.g);
           }
-          tma_load_3d_pair(sb, &p.tmB[p.nsplit ? 0 : src], fb, kk, tokc, 0);
+          const CUtensorMap* tb = &p.tmB[p.nsplit ? 0 : src];
+          tma_load_3d_pair(sb, tb, fb, kk, tokc, 0);
+          tma_load_3d_pair(sb + TN_SUB, tb, fb, kk + BK, tokc, 0);
           pending |= 1u << s;
           pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
         }
@@ -1316,8 +1332,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (leader) {
-      const uint32_t a_lbo = p.a_major ? BOX_BYTES : 16;
-      const uint32_t a_step = p.a_major ? 2048 : 32;
+      const uint32_t a_lbo = p.a_major ? TN_SUB : 16;   // MN-major: stride between 64-feature blocks
       int it = 0, tcount = 0;
       bool ok = true;
       int wave = 0;
@@ -1337,12 +1352,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + s * stage_bytes);
-          const uint32_t sb = sa + A_BYTES;
+          const uint32_t sb = sa + 2 * TN_SUB;
           if (lane == 0) {
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-              const uint64_t ad = sdesc(sa + kk * a_step, a_lbo, 1024);
-              const uint64_t bd = sdesc(sb + kk * 32, 16, 1024);
+            for (int kk = 0; kk < TN_BK / 16; ++kk) {
+              // K-major operands: sub-block kk / 4, +32 B per K16 step inside it; MN-major: +16 rows
+              const uint32_t koff = (kk >> 2) * TN_SUB + (kk & 3) * 32;
+              const uint64_t ad = sdesc(sa + (p.a_major ? kk * 2048 : koff), a_lbo, 1024);
+              const uint64_t bd = sdesc(sb + koff, 16, 1024);
               tc_mma2(tmem_d, ad, bd, idesc, (kb | kk) != 0);
             }
             tc_commit2_both(smem_u32(&empty[s]));
@@ -1430,9 +1447,9 @@ static int max_pairs() {
 template <int EPI>
 static int launch_tn(Params& p, long long pair_tile_upper_bound, const char* name, cudaStream_t stream) {
   p.mode = RG;
-  const int stage = A_BYTES + 128 * BK * 2;
+  const int stage = TN_STAGE;
   const int poff = ((p.G + 1 + 63) & ~63) * 4;
-  const int fixed = 1024 + 512 + poff + 4 * 2 * TN_SLAB + tn_aux_bytes(EPI);
+  const int fixed = 1024 + 512 + poff + TN_STAGING + tn_aux_bytes(EPI);
   const int st = (SMEM_LIMIT - fixed) / stage;
   if (st < 2) return fail(PFMOE_ERR_UNSUPPORTED, std::string(name) + ": too many experts for the shared-memory plan");
   p.stages = st > MAX_STAGES ? MAX_STAGES : st;
@@ -1523,13 +1540,13 @@ int tc_ffn_gemm1(const void* x_pft, const int* seg, const int* tiles, int N, int
   Params p = base_params(err);
   p.nsplit = 1;
   p.Nout = h;
-  p.k0_blocks = (d + BK - 1) / BK;
+  p.k0_blocks = (d + TN_BK - 1) / TN_BK;
   p.seg = seg; p.tiles = tiles; p.G = E;
   p.D0 = h1; p.D1 = h3; p.D2 = a; p.ldd = h;
   p.a_major = 1;            // W1_e, W3_e [d, h]: K rows, features contiguous
   p.fstep = 128;            // 64 features of W1 and the same 64 of W3 per CTA
-  PFMOE_TRY(make_tmap(&p.tmA[0], w1, h, d, E, 64, 64, "w1"));
-  PFMOE_TRY(make_tmap(&p.tmA[1], w3, h, d, E, 64, 64, "w3"));
+  PFMOE_TRY(make_tmap(&p.tmA[0], w1, h, d, E, 64, TN_BK, "w1"));
+  PFMOE_TRY(make_tmap(&p.tmA[1], w3, h, d, E, 64, TN_BK, "w3"));
   PFMOE_TRY(make_tmap(&p.tmB[0], x_pft, d, N, 1, BK, 128, "x_pft"));
   PFMOE_TRY(make_out_map_tn(&p.tmD[0], h1, h, N, "h1 out"));
   PFMOE_TRY(make_out_map_tn(&p.tmD[1], h3, h, N, "h3 out"));
@@ -1543,14 +1560,14 @@ int tc_ffn_gemm2(const void* a, const int* seg, const int* tiles, int N, int E, 
                  void* out, int32_t* err, cudaStream_t s) {
   Params p = base_params(err);
   p.Nout = d;
-  p.k0_blocks = (h + BK - 1) / BK;
+  p.k0_blocks = (h + TN_BK - 1) / TN_BK;
   p.seg = seg; p.tiles = tiles; p.G = E;
   p.D0 = out; p.ldd = d;
   p.a_major = 1;            // W2_e [h, d]: K rows, features contiguous
   p.fstep = 2 * BM;
   p.a_merged = d % 64 == 0;
-  if (p.a_merged) PFMOE_TRY(make_tmap_mn(&p.tmA[0], w2, d, h, E, BK, 2, "w2"));
-  else PFMOE_TRY(make_tmap(&p.tmA[0], w2, d, h, E, 64, 64, "w2"));
+  if (p.a_merged) PFMOE_TRY(make_tmap_mn(&p.tmA[0], w2, d, h, E, TN_BK, 2, "w2"));
+  else PFMOE_TRY(make_tmap(&p.tmA[0], w2, d, h, E, 64, TN_BK, "w2"));
   PFMOE_TRY(make_tmap(&p.tmB[0], a, h, N, 1, BK, 128, "a"));
   PFMOE_TRY(make_out_map_tn(&p.tmD[0], out, d, N, "out"));
   p.tma_store = 1;
@@ -1562,7 +1579,7 @@ int tc_ffn_dgrad_act(const void* dO, const int* seg, const int* tiles, int N, in
                      const void* h1, const void* h3, void* dh1, void* dh3, int32_t* err, cudaStream_t s) {
   Params p = base_params(err);
   p.Nout = h;
-  p.k0_blocks = (d + BK - 1) / BK;
+  p.k0_blocks = (d + TN_BK - 1) / TN_BK;
   p.seg = seg; p.tiles = tiles; p.G = E;
   p.X0 = h1; p.X1 = h3; p.D0 = dh1; p.D1 = dh3; p.ldd = h;
   p.a_major = 0;            // W2_e [h, d]: feature rows, K = d contiguous
@@ -1580,8 +1597,8 @@ int tc_ffn_dgrad_x(const void* dh1, const void* dh3, const int* seg, const int* 
                    const void* w1, const void* w3, void* dx_pft, int32_t* err, cudaStream_t s) {
   Params p = base_params(err);
   p.Nout = d;
-  p.k0_blocks = (h + BK - 1) / BK;
-  p.k1_blocks = (h + BK - 1) / BK;
+  p.k0_blocks = (h + TN_BK - 1) / TN_BK;
+  p.k1_blocks = (h + TN_BK - 1) / TN_BK;
   p.seg = seg; p.tiles = tiles; p.G = E;
   p.D0 = dx_pft; p.ldd = d;
   p.a_major = 0;            // W1_e, W3_e [d, h]: feature rows, K = h contiguous
