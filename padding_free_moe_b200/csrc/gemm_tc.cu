@@ -562,7 +562,10 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // Two issuing lanes (per-SM TMA delivery rises a few percent with two issuers): lane 0 posts
+    // the stage's byte count and loads A, lane 1 loads B.  The stage's phase completes only after
+    // lane 0's arrival and all bytes, so the order of the two lanes' copies does not matter.
+    if (lane < 2) {
       uint32_t pending = 0;        // stages with an issued load
       uint32_t pend_parity = 0;    // parity of that load's phase
       int it = 0;
@@ -574,24 +577,27 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
           const uint32_t ph = (it / S) & 1;
           if (!wait_bar(smem_u32(&empty[s]), ph ^ 1, abort_flag, p.err)) { ok = false; break; }
           const uint32_t fb = smem_u32(&full[s]);
-          mbar_expect_tx(fb, stage_bytes);
+          if (lane == 0) mbar_expect_tx(fb, stage_bytes);
           const uint32_t sa = smem_u32(smem + s * stage_bytes);
           const uint32_t sb = sa + A_BYTES;
           const int nb = p.bn / 64;
+          pending |= 1u << s;
+          pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
           if constexpr (MODE == RG) {
             // dense gate GEMM: A = X rows (K-major), B = Wg [K, N] (MN-major 64-column boxes)
             const int kk = (tl.kb0 + kb) * BK;
-            tma_load_3d(sa, &p.tmA[0], fb, kk, tl.row0, 0);
-            for (int j = 0; j < nb; ++j) tma_load_3d(sb + j * BOX_BYTES, &p.tmB[0], fb, tl.n0 + 64 * j, kk, 0);
+            if (lane == 0) tma_load_3d(sa, &p.tmA[0], fb, kk, tl.row0, 0);
+            else for (int j = 0; j < nb; ++j) tma_load_3d(sb + j * BOX_BYTES, &p.tmB[0], fb, tl.n0 + 64 * j, kk, 0);
           } else {
             const int krow = tl.krow0 + kb * BK;
-            if (p.a_merged) {
-              tma_load_4d(sa, &p.tmA[0], fb, 0, krow, tl.row0 / 64, 0);
-            } else {
-              tma_load_3d(sa, &p.tmA[0], fb, tl.row0, krow, 0);
-              tma_load_3d(sa + BOX_BYTES, &p.tmA[0], fb, tl.row0 + 64, krow, 0);
-            }
-            if (p.b_merged) {
+            if (lane == 0) {
+              if (p.a_merged) {
+                tma_load_4d(sa, &p.tmA[0], fb, 0, krow, tl.row0 / 64, 0);
+              } else {
+                tma_load_3d(sa, &p.tmA[0], fb, tl.row0, krow, 0);
+                tma_load_3d(sa + BOX_BYTES, &p.tmA[0], fb, tl.row0 + 64, krow, 0);
+              }
+            } else if (p.b_merged) {
               if (p.nsplit) {
                 tma_load_4d(sb, &p.tmB[0], fb, 0, krow, tl.n0 / 64, 0);
                 tma_load_4d(sb + (nb / 2) * BOX_BYTES, &p.tmB[1], fb, 0, krow, tl.n0 / 64, 0);
@@ -609,11 +615,9 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
               }
             }
           }
-          pending |= 1u << s;
-          pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
         }
       }
-      // Drain: wait until every load this thread issued has landed.
+      // Drain: wait until every load of this stage ring has landed (both lanes wait the same phases).
       for (int s = 0; s < S; ++s)
         if (pending & (1u << s))
           wait_bar(smem_u32(&full[s]), (pend_parity >> s) & 1, abort_flag, p.err, false);
@@ -1273,7 +1277,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
-    if (lane == 0) {
+    // Two issuing lanes, as in the one-SM kernel: lane 0 posts the byte count (even CTA) and
+    // loads A, lane 1 loads B.
+    if (lane < 2) {
       uint32_t pending = 0, pend_parity = 0;
       int it = 0;
       bool ok = true;
@@ -1290,12 +1296,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           const uint32_t ph = (it / S) & 1;
           if (!wait_bar2(smem_u32(&empty[s]), ph ^ 1, abort_flag, p.err)) { ok = false; break; }
           const uint32_t fb_local = smem_u32(&full[s]);
-          if (leader) mbar_expect_tx(fb_local, tx);
+          if (leader && lane == 0) mbar_expect_tx(fb_local, tx);
           const uint32_t fb = mapa_shared(fb_local, 0);
           const uint32_t sa = smem_u32(smem + s * stage_bytes);
           const uint32_t sb = sa + 2 * TN_SUB;
           const int src = kb < p.k0_blocks ? 0 : 1;
           const int kk = (src == 0 ? kb : kb - p.k0_blocks) * TN_BK;
+          pending |= 1u << s;
+          pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
+          if (lane == 1) {
+            const CUtensorMap* tb = &p.tmB[p.nsplit ? 0 : src];
+            tma_load_3d_pair(sb, tb, fb, kk, tokc, 0);
+            tma_load_3d_pair(sb + TN_SUB, tb, fb, kk + BK, tokc, 0);
+            continue;
+          }
           if (p.a_major) {
             // MN-major weights: 64-feature blocks of 128 K rows ([block][K row][128 B])
             if (p.nsplit) {
@@ -1317,11 +1331,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             tma_load_3d_pair(sa, &p.tmA[src], fb, kk, f, tl.g);
             tma_load_3d_pair(sa + TN_SUB, &p.tmA[src], fb, kk + BK, f, tl.g);
           }
-          const CUtensorMap* tb = &p.tmB[p.nsplit ? 0 : src];
-          tma_load_3d_pair(sb, tb, fb, kk, tokc, 0);
-          tma_load_3d_pair(sb + TN_SUB, tb, fb, kk + BK, tokc, 0);
-          pending |= 1u << s;
-          pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
         }
       }
       // Drain: a stage's empty barrier completes only after the MMA consumed it, so its loads landed.
