@@ -44,9 +44,15 @@ constexpr int THREADS = 192;
 constexpr int THREADS_KG = 224;          // K-grouped launches add a seventh warp: the K-tail zeroing warp
 constexpr int BOX_BYTES = 64 * 128;      // one 64 x 64 BF16 box (MN-major block)
 constexpr int A_BYTES = BM * BK * 2;     // 16 KB
+
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 
 enum Mode { RG = 0, KG = 1 };
+// K depth of one ring stage of the one-SM kernel (template argument KBK): 128 where three or more
+// stages still fit (gate dWg: bn = 64), which doubles the operand copies and halves the MMA
+// issuer's barrier handshakes; 64 for the 256-wide expert weight-gradient tiles, where a
+// 128-deep stage leaves room for only two stages and measured slower.
+constexpr int KG_BK = 2 * BK;
 enum Epi { EPI_STORE_BF16 = 0, EPI_STORE_F32 = 1, EPI_SWIGLU_FWD = 2, EPI_SWIGLU_BWD = 3, EPI_SPLIT_BF16 = 4 };
 
 struct Params {
@@ -72,7 +78,7 @@ struct Params {
   int dense_len;
   int stages;
   int ksplit;        // dense problems only: K is cut into ksplit parts, part s writes output slice s
-  int kchunk;        // KG dense: K rows per part (multiple of BK)
+  int kchunk;        // KG dense: K rows per part (multiple of KG_BK)
   void* D0;
   void* D1;
   void* D2;
@@ -239,7 +245,7 @@ __device__ __forceinline__ int total_tiles(const Params& p) {
   return p.G * ((p.M + BM - 1) / BM) * NT;
 }
 
-template <int MODE>
+template <int MODE, int KBK>
 __device__ __forceinline__ Tile decode(const Params& p, int t) {
   Tile tl;
   const int ns = n_step(p);
@@ -278,9 +284,9 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
     tl.row0 = m_idx * BM;
     tl.rows = min(BM, p.M - tl.row0);
     tl.n0 = n_idx * ns;
-    tl.nk = (len + BK - 1) / BK;
+    tl.nk = (len + KBK - 1) / KBK;
     tl.krow0 = s0;
-    tl.kvalid = len - (tl.nk - 1) * BK;
+    tl.kvalid = len - (tl.nk - 1) * KBK;
   }
   return tl;
 }
@@ -509,13 +515,15 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, u
 }
 
 // ---------------------------------------------------------------------- kernel
-template <int EPI, int MODE>
+template <int EPI, int MODE, int KBK>
 __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_gemm_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages;
-  const uint32_t b_bytes = static_cast<uint32_t>(p.bn) * BK * 2;
-  const uint32_t stage_bytes = A_BYTES + b_bytes;
+  constexpr uint32_t a_bytes = BM * KBK * 2;
+  constexpr uint32_t blk = KBK * 128;        // one MN-major block: 64 columns x KBK K rows
+  const uint32_t b_bytes = static_cast<uint32_t>(p.bn) * KBK * 2;
+  const uint32_t stage_bytes = a_bytes + b_bytes;
   uint8_t* stage_area = smem + S * stage_bytes;                       // epilogue staging (K-grouped only)
   uint8_t* bar_area = stage_area + (MODE == KG ? 4 * STAGE_BUFS * STAGE_BYTES_PER_WARP : 0);
   uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
@@ -571,7 +579,7 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const Tile tl = decode<MODE>(p, t);
+        const Tile tl = decode<MODE, KBK>(p, t);
         for (int kb = 0; kb < tl.nk; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
@@ -579,7 +587,7 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
           const uint32_t fb = smem_u32(&full[s]);
           if (lane == 0) mbar_expect_tx(fb, stage_bytes);
           const uint32_t sa = smem_u32(smem + s * stage_bytes);
-          const uint32_t sb = sa + A_BYTES;
+          const uint32_t sb = sa + a_bytes;
           const int nb = p.bn / 64;
           pending |= 1u << s;
           pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
@@ -589,18 +597,18 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
             if (lane == 0) tma_load_3d(sa, &p.tmA[0], fb, kk, tl.row0, 0);
             else for (int j = 0; j < nb; ++j) tma_load_3d(sb + j * BOX_BYTES, &p.tmB[0], fb, tl.n0 + 64 * j, kk, 0);
           } else {
-            const int krow = tl.krow0 + kb * BK;
+            const int krow = tl.krow0 + kb * KBK;
             if (lane == 0) {
               if (p.a_merged) {
                 tma_load_4d(sa, &p.tmA[0], fb, 0, krow, tl.row0 / 64, 0);
               } else {
                 tma_load_3d(sa, &p.tmA[0], fb, tl.row0, krow, 0);
-                tma_load_3d(sa + BOX_BYTES, &p.tmA[0], fb, tl.row0 + 64, krow, 0);
+                tma_load_3d(sa + blk, &p.tmA[0], fb, tl.row0 + 64, krow, 0);
               }
             } else if (p.b_merged) {
               if (p.nsplit) {
                 tma_load_4d(sb, &p.tmB[0], fb, 0, krow, tl.n0 / 64, 0);
-                tma_load_4d(sb + (nb / 2) * BOX_BYTES, &p.tmB[1], fb, 0, krow, tl.n0 / 64, 0);
+                tma_load_4d(sb + (nb / 2) * blk, &p.tmB[1], fb, 0, krow, tl.n0 / 64, 0);
               } else {
                 tma_load_4d(sb, &p.tmB[0], fb, 0, krow, tl.n0 / 64, 0);
               }
@@ -611,7 +619,7 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
                   which = j < nb / 2 ? 0 : 1;
                   nc = tl.n0 + 64 * (j < nb / 2 ? j : j - nb / 2);
                 }
-                tma_load_3d(sb + j * BOX_BYTES, &p.tmB[which], fb, nc, krow, 0);
+                tma_load_3d(sb + j * blk, &p.tmB[which], fb, nc, krow, 0);
               }
             }
           }
@@ -627,12 +635,12 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
     const int a_mn = MODE == KG ? 1 : 0;
     const int b_mn = MODE == KG ? 1 : p.b_major;
     const uint32_t idesc = idesc_bf16(BM, p.bn, a_mn, b_mn);
-    const uint32_t a_lbo = a_mn ? BOX_BYTES : 16, b_lbo = b_mn ? BOX_BYTES : 16;
+    const uint32_t a_lbo = a_mn ? blk : 16, b_lbo = b_mn ? blk : 16;   // MN-major: stride between 64-wide blocks
     const uint32_t a_step = a_mn ? 2048 : 32, b_step = b_mn ? 2048 : 32;
     int it = 0, tcount = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tcount) {
-      const Tile tl = decode<MODE>(p, t);
+      const Tile tl = decode<MODE, KBK>(p, t);
       const int buf = tcount & 1;
       const uint32_t aph = (tcount >> 1) & 1;
       ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&acc_empty[buf]), aph ^ 1, abort_flag, p.err));
@@ -647,15 +655,15 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
       for (int kb = 0; kb < tl.nk; ++kb, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
-        int kk_count = BK / 16;
+        int kk_count = KBK / 16;
         // K-grouped: the zeroing warp passes every stage on through ready[s] (one phase per ring
         // round, like full[s]) after clearing a segment's tail rows; MMAs of a segment's last block
         // stop at the 16-row step that holds the segment end.
-        if (MODE == KG && kb == tl.nk - 1 && tl.kvalid < BK) kk_count = ((tl.kvalid + 15) & ~15) / 16;
+        if (MODE == KG && kb == tl.nk - 1 && tl.kvalid < KBK) kk_count = ((tl.kvalid + 15) & ~15) / 16;
         ok = __all_sync(0xffffffffu, wait_bar(smem_u32(MODE == KG ? &ready[s] : &full[s]), ph, abort_flag, p.err));
         if (!ok) break;
         const uint32_t sa = smem_u32(smem + s * stage_bytes);
-        const uint32_t sb = sa + A_BYTES;
+        const uint32_t sb = sa + a_bytes;
         tc_fence_after();
         if (lane == 0) {
           for (int kk = 0; kk < kk_count; ++kk) {
@@ -686,18 +694,18 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
     int it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-      const Tile tl = decode<MODE>(p, t);
+      const Tile tl = decode<MODE, KBK>(p, t);
       for (int kb = 0; kb < tl.nk; ++kb, ++it) {
         const int s = it % S;
         ok = __all_sync(0xffffffffu, wait_bar(smem_u32(&full[s]), (it / S) & 1, abort_flag, p.err));
         if (!ok) break;
-        if (kb == tl.nk - 1 && tl.kvalid < BK) {
+        if (kb == tl.nk - 1 && tl.kvalid < KBK) {
           const uint32_t sa = smem_u32(smem + s * stage_bytes);
           const int per_box = (((tl.kvalid + 15) & ~15) - tl.kvalid) * 8;   // 16-byte chunks per box
           const int nbox = 2 + p.bn / 64;
           for (int b = 0; b < nbox; ++b)
             for (int i = lane; i < per_box; i += 32)
-              st_shared16(sa + b * BOX_BYTES + tl.kvalid * 128 + i * 16, make_uint4(0, 0, 0, 0));
+              st_shared16(sa + b * blk + tl.kvalid * 128 + i * 16, make_uint4(0, 0, 0, 0));
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
         __syncwarp();
@@ -710,7 +718,7 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
     Stager stg{smem_u32(stage_area + (warp - 2) * STAGE_BUFS * STAGE_BYTES_PER_WARP), 0};
     int tcount = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
-      const Tile tl = decode<MODE>(p, t);
+      const Tile tl = decode<MODE, KBK>(p, t);
       const int buf = tcount & 1;
       const uint32_t aph = (tcount >> 1) & 1;
       if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&acc_full[buf]), aph, abort_flag, p.err))) break;
@@ -815,14 +823,15 @@ constexpr int SMEM_LIMIT = 227 * 1024;
 // Alignment slack + barriers (512 B), plus the epilogue staging buffers when the launch uses them (K-grouped).
 static int smem_fixed(bool staged) { return 1024 + 512 + (staged ? 4 * STAGE_BUFS * STAGE_BYTES_PER_WARP : 0); }
 
-static int pick_stages(int bn, bool staged) {
-  const int stage = A_BYTES + bn * BK * 2;
-  int s = (SMEM_LIMIT - smem_fixed(staged)) / stage;
+static int stage_size(int bn, int kbk) { return (BM + bn) * kbk * 2; }
+
+static int pick_stages(int bn, bool staged, int kbk) {
+  int s = (SMEM_LIMIT - smem_fixed(staged)) / stage_size(bn, kbk);
   return s > MAX_STAGES ? MAX_STAGES : s;
 }
 
-static size_t smem_bytes(int bn, int stages, bool staged) {
-  return smem_fixed(staged) + static_cast<size_t>(stages) * (A_BYTES + bn * BK * 2);
+static size_t smem_bytes(int bn, int stages, bool staged, int kbk) {
+  return smem_fixed(staged) + static_cast<size_t>(stages) * stage_size(bn, kbk);
 }
 
 // ============================================================================
@@ -1418,15 +1427,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int EPI, int MODE>
+template <int EPI, int MODE, int KBK = BK>
 static int launch(Params& p, long long tile_upper_bound, const char* name, cudaStream_t stream) {
   p.mode = MODE;
   const bool staged = p.mode == KG;
-  p.stages = pick_stages(p.bn, staged);
-  const size_t smem = smem_bytes(p.bn, p.stages, staged);
+  p.stages = pick_stages(p.bn, staged, KBK);
+  if (p.stages < 2) return fail(PFMOE_ERR_UNSUPPORTED, std::string(name) + ": shared-memory plan needs two stages");
+  const size_t smem = smem_bytes(p.bn, p.stages, staged, KBK);
   static bool attr_done = false;  // per template instance
   if (!attr_done) {
-    if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI, MODE, KBK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(227 * 1024)) != cudaSuccess)
       return fail(PFMOE_ERR_CUDA, std::string("cudaFuncSetAttribute failed: ") +
                                       cudaGetErrorString(cudaGetLastError()));
@@ -1436,7 +1446,7 @@ static int launch(Params& p, long long tile_upper_bound, const char* name, cudaS
   long long grid = num_sms();
   if (tile_upper_bound < grid) grid = tile_upper_bound;
   PFMOE_LAUNCH(name, stream,
-               (grouped_gemm_kernel<EPI, MODE><<<static_cast<int>(grid), MODE == KG ? THREADS_KG : THREADS, smem,
+               (grouped_gemm_kernel<EPI, MODE, KBK><<<static_cast<int>(grid), MODE == KG ? THREADS_KG : THREADS, smem,
                                                  stream>>>(p)));
   return PFMOE_OK;
 }
@@ -1637,13 +1647,13 @@ int tc_ffn_wgrad13(const void* x_pft, const void* dh1, const void* dh3, const in
   p.b_merged = h % 64 == 0;
   const uint32_t bblk = (p.bn / 2) / 64;   // 64-wide blocks of dH1 (and of dH3) per tile
   if (p.a_merged) PFMOE_TRY(make_tmap_mn(&p.tmA[0], x_pft, d, N, 1, BK, 2, "x_pft^T"));
-  else PFMOE_TRY(make_tmap(&p.tmA[0], x_pft, d, N, 1, 64, 64, "x_pft^T"));
+  else PFMOE_TRY(make_tmap(&p.tmA[0], x_pft, d, N, 1, 64, BK, "x_pft^T"));
   if (p.b_merged) {
     PFMOE_TRY(make_tmap_mn(&p.tmB[0], dh1, h, N, 1, BK, bblk, "dh1"));
     PFMOE_TRY(make_tmap_mn(&p.tmB[1], dh3, h, N, 1, BK, bblk, "dh3"));
   } else {
-    PFMOE_TRY(make_tmap(&p.tmB[0], dh1, h, N, 1, 64, 64, "dh1"));
-    PFMOE_TRY(make_tmap(&p.tmB[1], dh3, h, N, 1, 64, 64, "dh3"));
+    PFMOE_TRY(make_tmap(&p.tmB[0], dh1, h, N, 1, 64, BK, "dh1"));
+    PFMOE_TRY(make_tmap(&p.tmB[1], dh3, h, N, 1, 64, BK, "dh3"));
   }
   PFMOE_TRY(make_out_map(&p.tmD[0], dw1, h, d, E, "dw1 out"));
   PFMOE_TRY(make_out_map(&p.tmD[1], dw3, h, d, E, "dw3 out"));
@@ -1666,9 +1676,9 @@ int tc_ffn_wgrad2(const void* a, const void* dO, const int* seg, int N, int E, i
   p.a_merged = h % 64 == 0;
   p.b_merged = d % 64 == 0;
   if (p.a_merged) PFMOE_TRY(make_tmap_mn(&p.tmA[0], a, h, N, 1, BK, 2, "a^T"));
-  else PFMOE_TRY(make_tmap(&p.tmA[0], a, h, N, 1, 64, 64, "a^T"));
+  else PFMOE_TRY(make_tmap(&p.tmA[0], a, h, N, 1, 64, BK, "a^T"));
   if (p.b_merged) PFMOE_TRY(make_tmap_mn(&p.tmB[0], dO, d, N, 1, BK, p.bn / 64, "dO"));
-  else PFMOE_TRY(make_tmap(&p.tmB[0], dO, d, N, 1, 64, 64, "dO"));
+  else PFMOE_TRY(make_tmap(&p.tmB[0], dO, d, N, 1, 64, BK, "dO"));
   PFMOE_TRY(make_out_map(&p.tmD[0], dw2, d, h, E, "dw2 out"));
   p.tma_store = 1;
   const long long ub = static_cast<long long>(E) * ((h + BM - 1) / BM) * ((d + p.bn - 1) / p.bn);
@@ -1682,7 +1692,7 @@ static int gate_logits_split(int T, int d, int E) {
 
 static int gate_wgrad_split(int T, int d, int E) {
   const int bn = round_bn(E);
-  return choose_ksplit(static_cast<long long>((d + BM - 1) / BM) * ((E + bn - 1) / bn), (T + BK - 1) / BK);
+  return choose_ksplit(static_cast<long long>((d + BM - 1) / BM) * ((E + bn - 1) / bn), (T + KG_BK - 1) / KG_BK);
 }
 
 size_t tc_gate_logits_ws(int T, int d, int E) {
@@ -1737,9 +1747,9 @@ int tc_gate_wgrad(const void* x, const void* dz_bf16, int T, int d, int E, float
   p.ldd = E;
   int ks = gate_wgrad_split(T, d, E);
   if (ws_bytes < tc_gate_wgrad_ws(T, d, E) || !ws) ks = 1;
-  const int nk = (T + BK - 1) / BK;
+  const int nk = (T + KG_BK - 1) / KG_BK;
   const int kbs = (nk + ks - 1) / ks;
-  p.kchunk = kbs * BK;
+  p.kchunk = kbs * KG_BK;
   p.G = ks;
   if (ks > 1) {
     p.D0 = ws;
@@ -1748,12 +1758,12 @@ int tc_gate_wgrad(const void* x, const void* dz_bf16, int T, int d, int E, float
     p.D0 = dwg;
     p.d_gstride = 0;
   }
-  PFMOE_TRY(make_tmap(&p.tmA[0], x, d, T, 1, 64, 64, "x^T"));
-  PFMOE_TRY(make_tmap(&p.tmB[0], dz_bf16, E, T, 1, 64, 64, "dz"));
+  PFMOE_TRY(make_tmap(&p.tmA[0], x, d, T, 1, 64, KG_BK, "x^T"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], dz_bf16, E, T, 1, 64, KG_BK, "dz"));
   PFMOE_TRY(make_tmap_t(&p.tmD[0], p.D0, true, E, d, ks, 32, 32, "dwg out"));
   p.tma_store = 1;
   const long long ub = static_cast<long long>(ks) * ((d + BM - 1) / BM) * ((E + p.bn - 1) / p.bn);
-  PFMOE_TRY((launch<EPI_STORE_F32, KG>(p, ub, "gate_wgrad", s)));
+  PFMOE_TRY((launch<EPI_STORE_F32, KG, KG_BK>(p, ub, "gate_wgrad", s)));
   if (ks > 1)
     PFMOE_TRY(launch_split_reduce(static_cast<const float*>(ws), ks, static_cast<long long>(d) * E, nullptr, E, dwg, s));
   return PFMOE_OK;
