@@ -204,8 +204,9 @@ int moe_route(const void* x, const void* wg, const float* bias, int T, int d, in
   PFMOE_TRY(need_ptr(ws, "ws", true));
   if (ws && ws_bytes < moe_route_workspace_size(T, d, E, k, dtype)) return fail(PFMOE_ERR_ARG, "workspace too small");
   cudaStream_t s = st(stream);
+  int nparts = 1;
   if (dtype == PFMOE_BF16) {
-    PFMOE_TRY(tc_gate_logits(x, wg, bias, T, d, E, logits, ws, ws_bytes, err, s));
+    PFMOE_TRY(tc_gate_logits(x, wg, bias, T, d, E, logits, ws, ws_bytes, &nparts, err, s));
   } else {
     SimtGemm g{};
     g.A = static_cast<const float*>(x); g.sam = d; g.sak = 1;
@@ -214,7 +215,9 @@ int moe_route(const void* x, const void* wg, const float* bias, int T, int d, in
     g.bias = bias; g.G = 1; g.M = T; g.N = E; g.K = d; g.mode = 0;
     PFMOE_TRY(simt_gemm_f32(g, err, s, "gate_logits_f32"));
   }
-  return launch_topk(logits, T, E, k, topk_ids, topk_w, err, s);
+  if (nparts > 1)   // split-K gate GEMM: the top-k kernel forms the logits from the K parts in ws
+    return launch_topk(logits, static_cast<const float*>(ws), nparts, bias, T, E, k, topk_ids, topk_w, err, s);
+  return launch_topk(logits, nullptr, 1, nullptr, T, E, k, topk_ids, topk_w, err, s);
 }
 
 size_t pft_build_workspace_size(int T, int E, int k) {

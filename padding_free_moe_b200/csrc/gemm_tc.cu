@@ -1706,7 +1706,7 @@ size_t tc_gate_wgrad_ws(int T, int d, int E) {
 }
 
 int tc_gate_logits(const void* x, const void* wg, const float* bias, int T, int d, int E, float* logits, void* ws,
-                   size_t ws_bytes, int32_t* err, cudaStream_t s) {
+                   size_t ws_bytes, int* nparts, int32_t* err, cudaStream_t s) {
   Params p = base_params(err);
   p.mode = RG;
   p.b_major = 1;              // Wg [d, E]: K rows, E contiguous
@@ -1730,8 +1730,7 @@ int tc_gate_logits(const void* x, const void* wg, const float* bias, int T, int 
   PFMOE_TRY(make_tmap(&p.tmB[0], wg, E, d, 1, 64, 64, "wg"));
   const long long ub = static_cast<long long>((T + BM - 1) / BM) * ((E + p.bn - 1) / p.bn) * ks;
   PFMOE_TRY((launch<EPI_STORE_F32, RG>(p, ub, "gate_logits", s)));
-  if (ks > 1)
-    PFMOE_TRY(launch_split_reduce(static_cast<const float*>(ws), ks, static_cast<long long>(T) * E, bias, E, logits, s));
+  *nparts = ks;   // ks > 1: the top-k kernel sums the parts (and adds the bias)
   return PFMOE_OK;
 }
 

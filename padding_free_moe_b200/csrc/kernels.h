@@ -23,8 +23,11 @@ int tc_ffn_wgrad2(const void* a, const void* dO, const int* seg, int N, int E, i
 // Dense gate GEMMs split K over a workspace (sizes below; 0 = no split) and reduce deterministically.
 size_t tc_gate_logits_ws(int T, int d, int E);
 size_t tc_gate_wgrad_ws(int T, int d, int E);
+// Gate logits X Wg (+ bias).  When the GEMM is split along K (ws large enough), the K parts are
+// left in ws ([*nparts][T][E] FP32) for launch_topk to sum; otherwise *nparts = 1 and logits holds
+// the result.
 int tc_gate_logits(const void* x, const void* wg, const float* bias, int T, int d, int E, float* logits, void* ws,
-                   size_t ws_bytes, int32_t* err, cudaStream_t s);
+                   size_t ws_bytes, int* nparts, int32_t* err, cudaStream_t s);
 int tc_gate_wgrad(const void* x, const void* dz_bf16, int T, int d, int E, float* dwg, void* ws, size_t ws_bytes,
                   int32_t* err, cudaStream_t s);
 
@@ -49,7 +52,10 @@ int simt_swiglu_bwd_f32(const float* da, const float* h1, const float* h3, float
                         cudaStream_t s);
 
 // ---- routing, route.cu
-int launch_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w, int32_t* err, cudaStream_t s);
+// Top-k softmax over logits [T][E].  With parts != null the logits are first formed as
+// parts[0] + ... + parts[nparts-1] (+ bias), in that order, and written to logits.
+int launch_topk(float* logits, const float* parts, int nparts, const float* bias, int T, int E, int k, int32_t* ids,
+                float* w, int32_t* err, cudaStream_t s);
 
 // ---- stable counting sort, PFT, RBD: sort.cu
 // Stable counting sort of n keys in [0, K): chunk histograms + scan.  n may be read

@@ -21,14 +21,19 @@ __device__ __forceinline__ bool before(float va, int ea, float vb, int eb) {
   return va > vb || (va == vb && ea < eb);
 }
 
+// With parts != null the logits row is first formed from the split-K parts of the gate GEMM
+// (sum in part order, then the bias: the same float operations as a separate reduce) and
+// written out, so the logits take one pass instead of two.
 template <int VPT>
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+__global__ void __launch_bounds__(256) topk_kernel(float* __restrict__ logits, const float* __restrict__ parts,
+                                                   int nparts, const float* __restrict__ bias, int T, int E, int k,
                                                    int32_t* __restrict__ ids, float* __restrict__ w,
                                                    int32_t* err) {
   const int lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const long long pstride = static_cast<long long>(T) * E;
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
-    const float* z = logits + static_cast<long long>(t) * E;
+    float* z = logits + static_cast<long long>(t) * E;
     float v[VPT];
     uint32_t taken = 0;
     bool nan_seen = false;
@@ -36,7 +41,16 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     for (int i = 0; i < VPT; ++i) {
       const int e = lane + 32 * i;
       if (e < E) {
-        float x = z[e];
+        float x;
+        if (parts) {
+          const float* pp = parts + static_cast<long long>(t) * E + e;
+          x = pp[0];
+          for (int sp = 1; sp < nparts; ++sp) x += pp[sp * pstride];
+          if (bias) x += bias[e];
+          z[e] = x;
+        } else {
+          x = z[e];
+        }
         if (x != x) { nan_seen = true; x = -INFINITY; }
         v[i] = x;
       } else {
@@ -73,23 +87,27 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 }
 
 template <int VPT>
-int launch_vpt(const float* logits, int T, int E, int k, int32_t* ids, float* w, int32_t* err, cudaStream_t s) {
+int launch_vpt(float* logits, const float* parts, int nparts, const float* bias, int T, int E, int k, int32_t* ids,
+               float* w, int32_t* err, cudaStream_t s) {
   long long blocks = (static_cast<long long>(T) * 32 + 255) / 256;
   const long long cap = static_cast<long long>(num_sms()) * 8;
   if (blocks > cap) blocks = cap;
-  PFMOE_LAUNCH("route_topk", s, topk_kernel<VPT><<<static_cast<int>(blocks), 256, 0, s>>>(logits, T, E, k, ids, w, err));
+  PFMOE_LAUNCH("route_topk", s,
+               topk_kernel<VPT><<<static_cast<int>(blocks), 256, 0, s>>>(logits, parts, nparts, bias, T, E, k, ids, w,
+                                                                         err));
   return PFMOE_OK;
 }
 
 }  // namespace
 
-int launch_topk(const float* logits, int T, int E, int k, int32_t* ids, float* w, int32_t* err, cudaStream_t s) {
-  if (E <= 32) return launch_vpt<1>(logits, T, E, k, ids, w, err, s);
-  if (E <= 64) return launch_vpt<2>(logits, T, E, k, ids, w, err, s);
-  if (E <= 128) return launch_vpt<4>(logits, T, E, k, ids, w, err, s);
-  if (E <= 256) return launch_vpt<8>(logits, T, E, k, ids, w, err, s);
-  if (E <= 512) return launch_vpt<16>(logits, T, E, k, ids, w, err, s);
-  return launch_vpt<32>(logits, T, E, k, ids, w, err, s);
+int launch_topk(float* logits, const float* parts, int nparts, const float* bias, int T, int E, int k, int32_t* ids,
+                float* w, int32_t* err, cudaStream_t s) {
+  if (E <= 32) return launch_vpt<1>(logits, parts, nparts, bias, T, E, k, ids, w, err, s);
+  if (E <= 64) return launch_vpt<2>(logits, parts, nparts, bias, T, E, k, ids, w, err, s);
+  if (E <= 128) return launch_vpt<4>(logits, parts, nparts, bias, T, E, k, ids, w, err, s);
+  if (E <= 256) return launch_vpt<8>(logits, parts, nparts, bias, T, E, k, ids, w, err, s);
+  if (E <= 512) return launch_vpt<16>(logits, parts, nparts, bias, T, E, k, ids, w, err, s);
+  return launch_vpt<32>(logits, parts, nparts, bias, T, E, k, ids, w, err, s);
 }
 
 }  // namespace pfmoe
