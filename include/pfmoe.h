@@ -206,6 +206,17 @@ PFMOE_API int moe_profile_enable(int on);
 PFMOE_API void moe_profile_reset(void);
 PFMOE_API int moe_profile_read(char* names, int name_stride, int max_entries, double* total_ms, int* launches);
 
+/*
+ * Test support, not part of the layer (the X-MoE pages have no counterpart).
+ * moe_selftest_wait_timeout launches one warp that waits, with the bounded mbarrier wait
+ * every GEMM of this library uses, on a barrier nothing ever arrives at.  After limit_ns
+ * nanoseconds (1 ms .. 5 s) the wait gives up, ORs PFMOE_DEV_TIMEOUT into *err (device
+ * memory) and the kernel returns; the CUDA context stays usable.  This lets a test drive
+ * the timeout path without faulting or hanging the GPU.  Asynchronous on `stream`.
+ * Errors: PFMOE_ERR_ARG for a null err or a limit outside the range.
+ */
+PFMOE_API int moe_selftest_wait_timeout(int32_t* err, unsigned long long limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

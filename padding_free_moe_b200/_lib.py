@@ -44,6 +44,7 @@ SIGNATURES = {
     "moe_profile_enable": (_I, [_I]),
     "moe_profile_reset": (None, []),
     "moe_profile_read": (_I, [_P, _I, _I, _P, _P]),
+    "moe_selftest_wait_timeout": (_I, [_P, ctypes.c_ulonglong, _P]),
 }
 
 
@@ -207,3 +208,10 @@ def moe_profile_read(max_entries: int = 64):
         nm = names.raw[i * stride:(i + 1) * stride].split(b"\0", 1)[0].decode()
         out[nm] = (cnt[i], ms[i])
     return out
+
+
+def moe_selftest_wait_timeout(err, limit_ns: int, stream=None):
+    """Test support: a one-warp kernel whose bounded mbarrier wait must give up after limit_ns and
+    set DEV_TIMEOUT in the device error word `err` (the context stays usable)."""
+    _check("moe_selftest_wait_timeout", lib().moe_selftest_wait_timeout(_ptr(err), int(limit_ns), _stream(stream)))
+

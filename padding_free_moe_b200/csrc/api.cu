@@ -503,4 +503,11 @@ int moe_profile_read(char* names, int name_stride, int max_entries, double* tota
   return n;
 }
 
+int moe_selftest_wait_timeout(int32_t* err, unsigned long long limit_ns, void* stream) {
+  set_error("");
+  PFMOE_TRY(need_ptr(err, "err"));
+  if (limit_ns < 1000000ull || limit_ns > 5000000000ull) return fail(PFMOE_ERR_ARG, "limit_ns must be in [1e6, 5e9]");
+  return tc_wait_selftest(err, limit_ns, st(stream));
+}
+
 }  // extern "C"

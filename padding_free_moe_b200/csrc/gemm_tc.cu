@@ -134,14 +134,15 @@ __device__ __forceinline__ unsigned long long globaltimer() {
 
 // Bounded wait.  Returns false if the wait expired or another role aborted.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                         int32_t* err, bool honour_abort = true) {
+                                         int32_t* err, bool honour_abort = true,
+                                         unsigned long long limit_ns = kTimeoutNs) {
   for (int i = 0; i < 128; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (honour_abort && *abort_flag) return false;
-    if (globaltimer() - t0 > kTimeoutNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort_flag = 1;
       dev_error(err, PFMOE_DEV_TIMEOUT);
       return false;
@@ -1546,9 +1547,29 @@ static int launch_split_reduce(const float* parts, int nparts, long long n, cons
   return PFMOE_OK;
 }
 
+// Self-test of the bounded wait: one warp waits on an mbarrier nothing ever arrives at.  The wait
+// must give up after limit_ns, OR PFMOE_DEV_TIMEOUT into *err and let the kernel return, leaving
+// the context usable.
+__global__ void wait_selftest_kernel(int32_t* err, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  wait_bar(smem_u32(&bar), 0, &abort_flag, err, true, limit_ns);
+}
+
 }  // namespace tc
 
 using namespace tc;
+
+int tc_wait_selftest(int32_t* err, unsigned long long limit_ns, cudaStream_t s) {
+  PFMOE_LAUNCH("wait_selftest", s, (wait_selftest_kernel<<<1, 32, 0, s>>>(err, limit_ns)));
+  return PFMOE_OK;
+}
 
 // Expert GEMMs over the PFT rows (token-as-N kernel).  seg = expert_offsets, tiles = the
 // 128-row tile prefix from pft_build (the kernel derives its 256-token tile counts from it).

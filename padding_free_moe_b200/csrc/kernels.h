@@ -54,6 +54,7 @@ int simt_swiglu_bwd_f32(const float* da, const float* h1, const float* h3, float
 // ---- routing, route.cu
 // Top-k softmax over logits [T][E].  With parts != null the logits are first formed as
 // parts[0] + ... + parts[nparts-1] (+ bias), in that order, and written to logits.
+int tc_wait_selftest(int32_t* err, unsigned long long limit_ns, cudaStream_t s);
 int launch_topk(float* logits, const float* parts, int nparts, const float* bias, int T, int E, int k, int32_t* ids,
                 float* w, int32_t* err, cudaStream_t s);
 

@@ -78,6 +78,13 @@ def test_other_argument_errors(lib):
     assert lib.rbd_plan_workspace_size(4, 2, 12, 4, 2) == 0
 
 
+def test_wait_selftest_argument_errors(lib):
+    assert lib.moe_selftest_wait_timeout(None, 50_000_000, None) == L.PFMOE_ERR_ARG
+    assert lib.moe_selftest_wait_timeout(FAKE, 10, None) == L.PFMOE_ERR_ARG          # below 1 ms
+    assert lib.moe_selftest_wait_timeout(FAKE, 10 ** 10, None) == L.PFMOE_ERR_ARG    # above 5 s
+    assert b"limit_ns" in lib.moe_last_error()
+
+
 def test_empty_inputs_are_noops(lib):
     # T = 0: nothing to launch for these steps, so they succeed without a GPU.
     assert lib.moe_dispatch(None, None, 0, 2, 64, L.PFMOE_BF16, None, None, None) == L.PFMOE_OK

@@ -1,5 +1,6 @@
 """Edge cases of the CUDA path: no tokens, out-of-range indices reported through
-the device error word (nothing traps), and argument errors from a live context."""
+the device error word (nothing traps), a bounded wait that runs out, and argument
+errors from a live context."""
 import numpy as np
 import pytest
 import torch
@@ -100,3 +101,23 @@ def test_rbd_stress_shape_matches_oracle():
     assert np.array_equal(i64(o["rexp"]), r["replica_expert"])
     assert np.array_equal(i64(o["ap"]), r["assign_pilot"])
     assert np.array_equal(i64(o["pdev"][:P]), r["pilot_device"])
+
+
+@pytest.mark.gpu
+def test_bounded_wait_gives_up_and_context_survives():
+    # One warp waits, with the GEMMs' bounded mbarrier wait, on a barrier nothing arrives at:
+    # after the 50 ms limit it reports PFMOE_DEV_TIMEOUT through the error word and returns.
+    err = torch.zeros(1, device="cuda", dtype=torch.int32)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    L.moe_selftest_wait_timeout(err, 50_000_000)
+    ev1.record()
+    torch.cuda.synchronize()
+    assert int(err) == L.DEV_TIMEOUT
+    assert 40.0 <= ev0.elapsed_time(ev1) < 2000.0       # it waited about the limit, then returned
+    # the context is still usable: a full layer step runs clean afterwards
+    cfg = get_config("small_bf16")
+    layer = make_layer(cfg)
+    inp = make_inputs(cfg, seed=3, device="cuda")
+    assert run_step(layer, inp) == 0
+
