@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--no-sort-stress", action="store_true", help="skip the PFT / RBD stress-shape timing")
     ap.add_argument("--cpu-sample-tokens", type=int, default=512)
     return ap.parse_args()
 
@@ -256,6 +257,59 @@ def config_block(cfg, world):
 
 
 # ------------------------------------------------------------------ our arm
+def stress_sort(L, torch, dev, stream, hbm_gbs, reps=20):
+    """PFT build and RBD plan on a scaled shape (T = 2^20, E = 256, k = 8, RBD map 8 experts per
+    device, 4 devices per node): at the layer configs these kernels are launch-latency bound, so
+    their HBM efficiency is measured here.  Synthetic ids, distinct per token: (r_t + 37 j) mod E.
+    Algorithmic bytes: PFT reads ids + weights (8Tk) and writes token_ids, expert_ids, weights,
+    pos (16Tk) plus 8E of counts; the RBD plan reads ids (4Tk) and writes its lists (about 36Tk)."""
+    T, E, k, epd, dpn = 1 << 20, 256, 8, 8, 4
+    N = T * k
+    g = torch.Generator(device=dev).manual_seed(11)
+    r = torch.randint(0, E, (T, 1), generator=g, device=dev, dtype=torch.int64)
+    ids = ((r + 37 * torch.arange(k, device=dev)) % E).to(torch.int32).contiguous()
+    w = torch.full((T, k), 1.0 / k, device=dev)
+    i32 = dict(device=dev, dtype=torch.int32)
+    tpe, off, tiles = torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(E + 1, **i32)
+    tok, eid, pos = torch.empty(N, **i32), torch.empty(N, **i32), torch.empty(N, **i32)
+    cw = torch.empty(N, device=dev)
+    err = torch.zeros(1, **i32)
+    pws_b = L.pft_build_workspace_size(T, E, k)
+    pws = torch.empty(max(pws_b, 256), device=dev, dtype=torch.uint8)
+    n_nodes = E // (epd * dpn)
+    P = T * min(k, n_nodes)
+    ppn, noff = torch.empty(n_nodes, **i32), torch.empty(n_nodes + 1, **i32)
+    ptok, pnode, pdev = torch.empty(P, **i32), torch.empty(P, **i32), torch.empty(P, **i32)
+    roff, rexp, apil, cnt = torch.empty(P + 1, **i32), torch.empty(N, **i32), torch.empty(N, **i32), torch.empty(2, **i32)
+    rws_b = L.rbd_plan_workspace_size(T, k, E, epd, dpn)
+    rws = torch.empty(max(rws_b, 256), device=dev, dtype=torch.uint8)
+
+    def pft():
+        L.pft_build(ids, w, T, E, k, tpe, off, tok, eid, cw, pos, tiles, pws, pws_b, err, stream)
+
+    def rbd():
+        L.rbd_plan(ids, T, k, E, epd, dpn, ppn, noff, ptok, pnode, pdev, roff, rexp, apil, cnt, rws, rws_b, err,
+                   stream)
+
+    out = {}
+    for name, fn, alg in (("pft_build", pft, 24 * N + 8 * E), ("rbd_plan", rbd, 40 * N)):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / reps * 1000
+        gbs = alg / (us * 1e-6) / 1e9
+        out[name] = {"T": T, "E": E, "k": k, "us": us, "algorithmic_bytes": alg, "gbs": gbs, "frac": gbs / hbm_gbs}
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item()):#x} in the PFT / RBD stress shape")
+    out["rbd_plan"]["pilots"] = int(cnt[0].item())
+    return out
+
+
 def run_ours(args):
     import torch
     from padding_free_moe_b200 import _lib as L
@@ -445,6 +499,7 @@ def run_ours(args):
                          if gemm_tflops else None,
                          "flops_per_step": gemm_flops, "ms_per_step": gemm_ms},
         "dispatch_gbs": gbs("dispatch"), "combine_gbs": gbs("combine"),
+        "sort_stress": None if args.no_sort_stress else stress_sort(L, torch, dev, stream, hbm),
         "kernels": kernels,
     }
 
