@@ -303,7 +303,15 @@ def stress_sort(L, torch, dev, stream, hbm_gbs, reps=20):
         torch.cuda.synchronize()
         us = e0.elapsed_time(e1) / reps * 1000
         gbs = alg / (us * 1e-6) / 1e9
-        out[name] = {"T": T, "E": E, "k": k, "us": us, "algorithmic_bytes": alg, "gbs": gbs, "frac": gbs / hbm_gbs}
+        # one more pass with per-kernel events: where the time goes inside the plan
+        L.moe_profile_reset()
+        L.moe_profile_enable(True)
+        fn()
+        torch.cuda.synchronize()
+        L.moe_profile_enable(False)
+        kern = {nm: round(ms * 1000, 1) for nm, (c, ms) in L.moe_profile_read().items()}
+        out[name] = {"T": T, "E": E, "k": k, "us": us, "algorithmic_bytes": alg, "gbs": gbs, "frac": gbs / hbm_gbs,
+                     "kernel_us": kern}
     if int(err.item()) != 0:
         raise RuntimeError(f"device error word {int(err.item()):#x} in the PFT / RBD stress shape")
     out["rbd_plan"]["pilots"] = int(cnt[0].item())

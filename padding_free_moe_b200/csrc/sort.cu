@@ -80,7 +80,9 @@ __device__ int block_excl_scan(int v, int* tmp /*[32]*/, int* total) {
   return warp_off + x - v;
 }
 
-// counts [C][K] -> totals [K], offsets [K+1], base [C][K]; optional tiles [K+1] = prefix of ceil(total/tile_rows).
+// counts [C][K] -> totals [K], offsets [K+1], base [C][K] = rows of key k in chunks before c (relative
+// to the key's first row; the scatter adds offsets[k]); optional tiles [K+1] = prefix of
+// ceil(total/tile_rows).  One CTA: used while C is small (launch latency dominates there).
 __global__ void __launch_bounds__(SCAN_THREADS) chunk_scan_kernel(const int32_t* __restrict__ counts, int C, int K,
                                                                   int32_t* totals, int32_t* offsets,
                                                                   int32_t* __restrict__ base, int32_t* tiles,
@@ -101,7 +103,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) chunk_scan_kernel(const int32_t*
       if (totals) totals[key] = tot;
       offsets[key] = excl;
       if (tiles) tiles[key] = texcl;
-      int run = excl;
+      int run = 0;
       for (int c = 0; c < C; ++c) {
         const long long idx = static_cast<long long>(c) * K + key;
         const int cnt = counts[idx];
@@ -118,10 +120,57 @@ __global__ void __launch_bounds__(SCAN_THREADS) chunk_scan_kernel(const int32_t*
   }
 }
 
+// Many chunks: one CTA per key scans that key's column of chunk counts (exclusive, relative
+// bases) and writes the key's total; key_scan_kernel then forms the key offsets.
+__global__ void __launch_bounds__(SCAN_THREADS) col_scan_kernel(const int32_t* __restrict__ counts, int C, int K,
+                                                                int32_t* __restrict__ base, int32_t* totals) {
+  __shared__ int tmp[32];
+  const int key = blockIdx.x;
+  int carry = 0;
+  for (int c0 = 0; c0 < C; c0 += SCAN_THREADS) {
+    const int c = c0 + threadIdx.x;
+    const long long idx = static_cast<long long>(c) * K + key;
+    const int v = c < C ? counts[idx] : 0;
+    int blk;
+    const int ex = block_excl_scan(v, tmp, &blk);
+    if (c < C) base[idx] = carry + ex;
+    carry += blk;
+  }
+  if (threadIdx.x == 0) totals[key] = carry;
+}
+
+// Key totals -> offsets [K+1], optional tiles [K+1] (prefix of ceil(total/tile_rows)), optional copy of totals.
+__global__ void __launch_bounds__(SCAN_THREADS) key_scan_kernel(const int32_t* __restrict__ totals, int K,
+                                                                int32_t* totals_out, int32_t* offsets, int32_t* tiles,
+                                                                int tile_rows) {
+  __shared__ int tmp[32];
+  int carry = 0, tcarry = 0;
+  for (int k0 = 0; k0 < K; k0 += SCAN_THREADS) {
+    const int key = k0 + threadIdx.x;
+    const int tot = key < K ? totals[key] : 0;
+    int blk, tblk;
+    const int excl = block_excl_scan(tot, tmp, &blk) + carry;
+    const int nt = tile_rows > 0 ? (tot + tile_rows - 1) / tile_rows : 0;
+    const int texcl = block_excl_scan(nt, tmp, &tblk) + tcarry;
+    if (key < K) {
+      if (totals_out) totals_out[key] = tot;
+      offsets[key] = excl;
+      if (tiles) tiles[key] = texcl;
+    }
+    carry += blk;
+    tcarry += tblk;
+  }
+  if (threadIdx.x == 0) {
+    offsets[K] = carry;
+    if (tiles) tiles[K] = tcarry;
+  }
+}
+
 // Stable scatter; Sink(i, p, key) records that element i lands at sorted position p.
 template <class Sink>
 __global__ void chunk_scatter_kernel(const int32_t* __restrict__ keys, long long n, const int32_t* n_dev, int K,
-                                     int nchunks, const int32_t* __restrict__ base, Sink sink) {
+                                     int nchunks, const int32_t* __restrict__ base,
+                                     const int32_t* __restrict__ key_offsets, Sink sink) {
   extern __shared__ int32_t sh[];   // [warps][K]: per-warp counts, then per-warp first rows
   const int nw = blockDim.x >> 5;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -151,7 +200,7 @@ __global__ void chunk_scatter_kernel(const int32_t* __restrict__ keys, long long
   // exclusive prefix over the warps of this chunk, starting at the chunk's base row of each key
   if (chunk < nchunks)
     for (int k = threadIdx.x; k < K; k += blockDim.x) {
-      int run = base[static_cast<long long>(chunk) * K + k];
+      int run = key_offsets[k] + base[static_cast<long long>(chunk) * K + k];
       for (int w2 = 0; w2 < nw; ++w2) {
         const int c = sh[w2 * K + k];
         sh[w2 * K + k] = run;
@@ -202,6 +251,90 @@ __global__ void __launch_bounds__(SCAN_THREADS) excl_scan_kernel(const int32_t* 
     carry += blk;
   }
   if (threadIdx.x == 0) out[nn] = carry;
+}
+
+// Long scans (tokens, pilots): three launches instead of one CTA walking the whole array.
+//   tile_sum: per 8192-element tile, the sums of a (and of b);
+//   tile_offsets: one CTA scans the tile sums in place and writes the totals;
+//   tile_scan: each tile's exclusive scan plus its offset (each thread scans 8 consecutive values).
+constexpr int TILE_PT = 8;
+constexpr int SCAN_TILE = SCAN_THREADS * TILE_PT;
+
+__global__ void __launch_bounds__(SCAN_THREADS) tile_sum_kernel(const int32_t* __restrict__ a,
+                                                                const int32_t* __restrict__ b, long long n,
+                                                                const int32_t* n_dev, int32_t* sum_a, int32_t* sum_b) {
+  __shared__ int tmp[32];
+  const long long nn = dev_count(n, n_dev);
+  const long long t0 = static_cast<long long>(blockIdx.x) * SCAN_TILE;
+  int va = 0, vb = 0;
+#pragma unroll
+  for (int i = 0; i < TILE_PT; ++i) {
+    const long long idx = t0 + threadIdx.x + static_cast<long long>(i) * SCAN_THREADS;
+    if (idx < nn) {
+      va += a[idx];
+      if (b) vb += b[idx];
+    }
+  }
+  int tot;
+  block_excl_scan(va, tmp, &tot);
+  if (threadIdx.x == 0) sum_a[blockIdx.x] = tot;
+  if (b) {
+    block_excl_scan(vb, tmp, &tot);
+    if (threadIdx.x == 0) sum_b[blockIdx.x] = tot;
+  }
+}
+
+// sum_a[0..ntiles) -> exclusive prefix in place; the sum goes to *total_a and/or to out_end[n] (n = the
+// device count when n_dev is given); *total_b = sum of sum_b (if given).
+__global__ void __launch_bounds__(SCAN_THREADS) tile_offsets_kernel(int32_t* sum_a, const int32_t* sum_b, int ntiles,
+                                                                    int32_t* total_a, int32_t* total_b,
+                                                                    int32_t* out_end, long long n,
+                                                                    const int32_t* n_dev) {
+  __shared__ int tmp[32];
+  int carry = 0, bcarry = 0;
+  for (int i0 = 0; i0 < ntiles; i0 += SCAN_THREADS) {
+    const int i = i0 + threadIdx.x;
+    const int v = i < ntiles ? sum_a[i] : 0;
+    int blk;
+    const int ex = block_excl_scan(v, tmp, &blk);
+    if (i < ntiles) sum_a[i] = carry + ex;
+    carry += blk;
+    if (sum_b) {
+      int bblk;
+      block_excl_scan(i < ntiles ? sum_b[i] : 0, tmp, &bblk);
+      bcarry += bblk;
+    }
+  }
+  if (threadIdx.x == 0) {
+    if (total_a) *total_a = carry;
+    if (total_b) *total_b = bcarry;
+    if (out_end) out_end[dev_count(n, n_dev)] = carry;
+  }
+}
+
+__global__ void __launch_bounds__(SCAN_THREADS) tile_scan_kernel(const int32_t* __restrict__ a, long long n,
+                                                                 const int32_t* n_dev,
+                                                                 const int32_t* __restrict__ tile_off,
+                                                                 int32_t* __restrict__ out) {
+  __shared__ int tmp[32];
+  const long long nn = dev_count(n, n_dev);
+  const long long t0 = static_cast<long long>(blockIdx.x) * SCAN_TILE;
+  if (t0 >= nn) return;   // uniform per CTA
+  const long long i0 = t0 + static_cast<long long>(threadIdx.x) * TILE_PT;
+  int v[TILE_PT];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < TILE_PT; ++i) {
+    v[i] = i0 + i < nn ? a[i0 + i] : 0;
+    sum += v[i];
+  }
+  int blk;
+  int run = block_excl_scan(sum, tmp, &blk) + tile_off[blockIdx.x];
+#pragma unroll
+  for (int i = 0; i < TILE_PT; ++i) {
+    if (i0 + i < nn) out[i0 + i] = run;
+    run += v[i];
+  }
 }
 
 // ------------------------------------------------------------------------- RBD
@@ -339,16 +472,31 @@ int rows_grid(long long rows, int warps_per_blk = 8) {
   return static_cast<int>(b < 1 ? 1 : b);
 }
 
-struct CsortWs {
-  int32_t* counts;
-  int32_t* base;
-};
+// Chunk counts -> relative bases + key totals/offsets/tiles: one CTA while the chunks are few, else a
+// CTA per key (col_scan) and a key scan.  key_tot receives the totals on the many-chunk path.
+constexpr int SMALL_CHUNKS = 64;
+
+int sort_scan(const int32_t* counts, int C, int K, int32_t* totals, int32_t* offsets, int32_t* base, int32_t* tiles,
+              int tile_rows, int32_t* key_tot, const char* name, cudaStream_t s) {
+  if (C <= SMALL_CHUNKS) {
+    PFMOE_LAUNCH(name, s,
+                 chunk_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(counts, C, K, totals, offsets, base, tiles, tile_rows));
+    return PFMOE_OK;
+  }
+  PFMOE_LAUNCH(name, s, col_scan_kernel<<<K, SCAN_THREADS, 0, s>>>(counts, C, K, base, key_tot));
+  PFMOE_LAUNCH(name, s, key_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(key_tot, K, totals, offsets, tiles, tile_rows));
+  return PFMOE_OK;
+}
+
+// Tiles of the three-launch long scan for n_max elements (the tile sums need 2 * this many ints).
+inline long long long_scan_tiles(long long n_max) { return (n_max + SCAN_TILE - 1) / SCAN_TILE; }
+constexpr long long LONG_SCAN_MIN = 4LL * SCAN_TILE;   // below this one CTA scans the array
 
 }  // namespace
 
 size_t csort_ws_bytes(long long n_max, int K) {
   const long long C = (n_max + chunk_keys(K) - 1) / chunk_keys(K);
-  return static_cast<size_t>(2 * (C > 0 ? C : 1) * static_cast<long long>(K)) * sizeof(int32_t);
+  return static_cast<size_t>(2 * (C > 0 ? C : 1) * static_cast<long long>(K) + K) * sizeof(int32_t);
 }
 
 int pft_build_impl(const int32_t* ids, const float* w, int T, int E, int k, int32_t* tpe, int32_t* offsets,
@@ -364,18 +512,20 @@ int pft_build_impl(const int32_t* ids, const float* w, int T, int E, int k, int3
   if (C > 0)
     PFMOE_LAUNCH("pft_hist", s,
                  chunk_hist_kernel<<<blocks, wpb * 32, E * sizeof(int32_t), s>>>(ids, N, nullptr, E, C, counts, err));
-  PFMOE_LAUNCH("pft_scan", s,
-               chunk_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(counts, C, E, tpe, offsets, base, tile_offsets, 128));
+  int32_t* key_tot = base + static_cast<long long>(C) * E;
+  PFMOE_TRY(sort_scan(counts, C, E, tpe, offsets, base, tile_offsets, 128, key_tot, "pft_scan", s));
   PftSink sink{w, k, pos, token_ids, expert_ids, cw};
   if (C > 0)
     PFMOE_LAUNCH("pft_scatter", s,
-                 chunk_scatter_kernel<PftSink><<<blocks, wpb * 32, sm, s>>>(ids, N, nullptr, E, C, base, sink));
+                 chunk_scatter_kernel<PftSink><<<blocks, wpb * 32, sm, s>>>(ids, N, nullptr, E, C, base, offsets,
+                                                                             sink));
   return PFMOE_OK;
 }
 
 size_t rbd_ws_bytes(int T, int k, int n_nodes) {
   const long long pmax = static_cast<long long>(T) * (k < n_nodes ? k : n_nodes);
-  const size_t ints = 3 * static_cast<size_t>(T) + 5 * static_cast<size_t>(pmax) + 64;
+  const long long lt = long_scan_tiles(pmax > T ? pmax : T);
+  const size_t ints = 3 * static_cast<size_t>(T) + 5 * static_cast<size_t>(pmax) + 2 * static_cast<size_t>(lt) + 128;
   return ints * sizeof(int32_t) + csort_ws_bytes(pmax, n_nodes) + 256;
 }
 
@@ -395,6 +545,9 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
   int32_t* prc = p; p += pmax;
   int32_t* psorted = p; p += pmax;
   int32_t* rc_sorted = p; p += pmax;
+  const long long lt = long_scan_tiles(pmax > T ? pmax : T);
+  int32_t* tsum_a = p; p += lt;
+  int32_t* tsum_b = p; p += lt;
   p += 64 - ((p - static_cast<int32_t*>(ws)) & 63);   // keep 256-byte alignment
   const int C = static_cast<int>((pmax + chunk_keys(n_nodes) - 1) / chunk_keys(n_nodes));
   int32_t* ccounts = p; p += static_cast<long long>(C > 0 ? C : 1) * n_nodes;
@@ -402,7 +555,17 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
 
   const int g = rows_grid(T);
   PFMOE_LAUNCH("rbd_count", s, rbd_count_kernel<<<g, 256, 0, s>>>(ids, T, k, E, epd, epn, ucount, dcount, err));
-  PFMOE_LAUNCH("rbd_scan_tokens", s, rbd_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(ucount, dcount, T, pbase, counts));
+  if (T < LONG_SCAN_MIN) {
+    PFMOE_LAUNCH("rbd_scan_tokens", s, rbd_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(ucount, dcount, T, pbase, counts));
+  } else {
+    const int nt = static_cast<int>(long_scan_tiles(T));
+    PFMOE_LAUNCH("rbd_scan_tokens", s,
+                 tile_sum_kernel<<<nt, SCAN_THREADS, 0, s>>>(ucount, dcount, T, nullptr, tsum_a, tsum_b));
+    PFMOE_LAUNCH("rbd_scan_tokens", s,
+                 tile_offsets_kernel<<<1, SCAN_THREADS, 0, s>>>(tsum_a, tsum_b, nt, counts, counts + 1, nullptr, 0,
+                                                                nullptr));
+    PFMOE_LAUNCH("rbd_scan_tokens", s, tile_scan_kernel<<<nt, SCAN_THREADS, 0, s>>>(ucount, T, nullptr, tsum_a, pbase));
+  }
   PFMOE_LAUNCH("rbd_emit", s, rbd_emit_kernel<<<g, 256, 0, s>>>(ids, T, k, E, epd, epn, pbase, pkey, ptoken, prc, err));
   const int wpb = warps_per_block(n_nodes);
   const int blocks = C;
@@ -412,17 +575,29 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
                  chunk_hist_kernel<<<blocks, wpb * 32, n_nodes * sizeof(int32_t), s>>>(pkey, pmax, counts, n_nodes, C,
                                                                                      ccounts, err));
   }
-  PFMOE_LAUNCH("rbd_scan_nodes", s,
-               chunk_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(ccounts, C, n_nodes, pilots_per_node, node_offsets,
-                                                            cbase, nullptr, 0));
+  int32_t* node_tot = cbase + static_cast<long long>(C > 0 ? C : 1) * n_nodes;
+  PFMOE_TRY(sort_scan(ccounts, C, n_nodes, pilots_per_node, node_offsets, cbase, nullptr, 0, node_tot,
+                      "rbd_scan_nodes", s));
   if (C > 0) {
     RbdSink sink{ptoken, prc, pilot_token, pilot_node, rc_sorted, psorted};
     PFMOE_LAUNCH("rbd_scatter", s,
                  chunk_scatter_kernel<RbdSink><<<blocks, wpb * 32, sm, s>>>(pkey, pmax, counts, n_nodes, C, cbase,
-                                                                             sink));
+                                                                             node_offsets, sink));
   }
-  PFMOE_LAUNCH("rbd_scan_replicas", s,
-               excl_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(rc_sorted, pmax, counts, replica_offsets));
+  if (pmax < LONG_SCAN_MIN) {
+    PFMOE_LAUNCH("rbd_scan_replicas", s,
+                 excl_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(rc_sorted, pmax, counts, replica_offsets));
+  } else {
+    // P = counts[0] lives on the device: tiles past it sum to zero and write nothing
+    const int nt = static_cast<int>(long_scan_tiles(pmax));
+    PFMOE_LAUNCH("rbd_scan_replicas", s,
+                 tile_sum_kernel<<<nt, SCAN_THREADS, 0, s>>>(rc_sorted, nullptr, pmax, counts, tsum_a, nullptr));
+    PFMOE_LAUNCH("rbd_scan_replicas", s,
+                 tile_offsets_kernel<<<1, SCAN_THREADS, 0, s>>>(tsum_a, nullptr, nt, nullptr, nullptr, replica_offsets,
+                                                                pmax, counts));
+    PFMOE_LAUNCH("rbd_scan_replicas", s,
+                 tile_scan_kernel<<<nt, SCAN_THREADS, 0, s>>>(rc_sorted, pmax, counts, tsum_a, replica_offsets));
+  }
   PFMOE_LAUNCH("rbd_final", s,
                rbd_final_kernel<<<g, 256, 0, s>>>(ids, T, k, E, epd, epn, pbase, psorted, replica_offsets,
                                                    assign_pilot, replica_expert, pilot_device, err));
