@@ -338,8 +338,9 @@ __global__ void __launch_bounds__(SCAN_THREADS) tile_scan_kernel(const int32_t* 
 }
 
 // ------------------------------------------------------------------------- RBD
-// Per token (one warp; lane j < k holds expert e_j): rank experts by (e, lane);
-// a lane "leads" its node (device) when no earlier-ranked lane shares it.
+// Per token (a group of G lanes, G = 8, 16 or 32 >= k, so one warp serves 32 / G tokens; lane j < k
+// of the group holds expert e_j): rank experts by (e, lane); a lane "leads" its node (device) when
+// no earlier-ranked lane of the group shares it.
 struct TokView {
   int e, node, dev;
   bool valid;
@@ -347,14 +348,17 @@ struct TokView {
   int node_rank;   // index of this lane's node among the token's distinct nodes (ascending)
   int within;      // rank of e among the token's experts on the same node
   int same_node;   // experts of this token on this lane's node
+  int sub;         // lane index within the token's group
 };
 
-__device__ __forceinline__ TokView token_view(const int32_t* ids, int t, int k, int E, int epd, int epn,
-                                              int32_t* err) {
+template <int G>
+__device__ __forceinline__ TokView token_view(const int32_t* ids, long long t, bool tvalid, int k, int E, int epd,
+                                              int epn, int32_t* err) {
   const int lane = threadIdx.x & 31;
   TokView v;
-  v.valid = lane < k;
-  int e = v.valid ? ids[static_cast<long long>(t) * k + lane] : 0;
+  v.sub = lane & (G - 1);
+  v.valid = tvalid && v.sub < k;
+  int e = v.valid ? ids[t * k + v.sub] : 0;
   if (v.valid && static_cast<unsigned>(e) >= static_cast<unsigned>(E)) {
     dev_error(err, PFMOE_DEV_BAD_EXPERT_ID);
     e = 0;
@@ -364,8 +368,8 @@ __device__ __forceinline__ TokView token_view(const int32_t* ids, int t, int k, 
   v.dev = e / epd;
   int node_before = 0, dev_before = 0, within = 0, same = 0;
   for (int j = 0; j < k; ++j) {
-    const int oe = __shfl_sync(0xffffffffu, e, j);
-    const bool earlier = oe < e || (oe == e && j < lane);
+    const int oe = __shfl_sync(0xffffffffu, e, j, G);
+    const bool earlier = oe < e || (oe == e && j < v.sub);
     const int onode = oe / epn, odev = oe / epd;
     if (onode == v.node) {
       ++same;
@@ -377,25 +381,38 @@ __device__ __forceinline__ TokView token_view(const int32_t* ids, int t, int k, 
   v.dev_lead = v.valid && dev_before == 0;
   v.within = within;
   v.same_node = same;
-  const unsigned leads = __ballot_sync(0xffffffffu, v.node_lead);
+  const unsigned gmask = G == 32 ? 0xffffffffu : ((1u << G) - 1u);
+  const unsigned leads = (__ballot_sync(0xffffffffu, v.node_lead) >> (lane & ~(G - 1))) & gmask;
   int rank = 0;
   for (int j = 0; j < k; ++j) {
-    const int onode = __shfl_sync(0xffffffffu, v.node, j);
+    const int onode = __shfl_sync(0xffffffffu, v.node, j, G);
     if (((leads >> j) & 1u) && onode < v.node) ++rank;
   }
   v.node_rank = rank;
   return v;
 }
 
+// Token of this lane's group, for grid-stride loops over groups of G lanes.
+template <int G>
+__device__ __forceinline__ long long group_token(long long step) {
+  const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  return (warp + step) * (32 / G) + ((threadIdx.x & 31) / G);
+}
+
+template <int G>
 __global__ void rbd_count_kernel(const int32_t* ids, int T, int k, int E, int epd, int epn, int32_t* ucount,
                                  int32_t* dcount, int32_t* err) {
   const int lane = threadIdx.x & 31;
-  const int nw = (gridDim.x * blockDim.x) >> 5;
-  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nw) {
-    const TokView v = token_view(ids, t, k, E, epd, epn, err);
-    const int u = __popc(__ballot_sync(0xffffffffu, v.node_lead));
-    const int dd = __popc(__ballot_sync(0xffffffffu, v.dev_lead));
-    if (lane == 0) { ucount[t] = u; dcount[t] = dd; }
+  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long step = 0;; step += nw) {
+    const long long t = group_token<G>(step);
+    if (__all_sync(0xffffffffu, t >= T)) break;
+    const TokView v = token_view<G>(ids, t, t < T, k, E, epd, epn, err);
+    const unsigned gmask = G == 32 ? 0xffffffffu : ((1u << G) - 1u);
+    const int shift = lane & ~(G - 1);
+    const int u = __popc((__ballot_sync(0xffffffffu, v.node_lead) >> shift) & gmask);
+    const int dd = __popc((__ballot_sync(0xffffffffu, v.dev_lead) >> shift) & gmask);
+    if (v.sub == 0 && t < T) { ucount[t] = u; dcount[t] = dd; }
   }
 }
 
@@ -419,15 +436,18 @@ __global__ void __launch_bounds__(SCAN_THREADS) rbd_scan_kernel(const int32_t* u
 }
 
 // Token-major pilot list: key = node, token, replica count.
+template <int G>
 __global__ void rbd_emit_kernel(const int32_t* ids, int T, int k, int E, int epd, int epn, const int32_t* pilot_base,
                                 int32_t* pkey, int32_t* ptoken, int32_t* prc, int32_t* err) {
-  const int nw = (gridDim.x * blockDim.x) >> 5;
-  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nw) {
-    const TokView v = token_view(ids, t, k, E, epd, epn, err);
+  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long step = 0;; step += nw) {
+    const long long t = group_token<G>(step);
+    if (__all_sync(0xffffffffu, t >= T)) break;
+    const TokView v = token_view<G>(ids, t, t < T, k, E, epd, epn, err);
     if (v.node_lead) {
       const int i = pilot_base[t] + v.node_rank;
       pkey[i] = v.node;
-      ptoken[i] = t;
+      ptoken[i] = static_cast<int32_t>(t);
       prc[i] = v.same_node;
     }
   }
@@ -448,22 +468,34 @@ struct RbdSink {
   }
 };
 
+template <int G>
 __global__ void rbd_final_kernel(const int32_t* ids, int T, int k, int E, int epd, int epn,
                                  const int32_t* pilot_base, const int32_t* psorted, const int32_t* replica_offsets,
                                  int32_t* assign_pilot, int32_t* replica_expert, int32_t* pilot_device,
                                  int32_t* err) {
-  const int lane = threadIdx.x & 31;
-  const int nw = (gridDim.x * blockDim.x) >> 5;
-  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nw) {
-    const TokView v = token_view(ids, t, k, E, epd, epn, err);
+  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long step = 0;; step += nw) {
+    const long long t = group_token<G>(step);
+    if (__all_sync(0xffffffffu, t >= T)) break;
+    const TokView v = token_view<G>(ids, t, t < T, k, E, epd, epn, err);
     if (v.valid) {
       const int q = psorted[pilot_base[t] + v.node_rank];
-      assign_pilot[static_cast<long long>(t) * k + lane] = q;
+      assign_pilot[t * k + v.sub] = q;
       replica_expert[replica_offsets[q] + v.within] = v.e;
       if (v.within == 0) pilot_device[q] = v.dev;
     }
   }
 }
+
+// Launch one of the per-token RBD kernels with the smallest lane group that holds k experts.
+#define PFMOE_RBD_LAUNCH(NAME, KERNEL, T_, k_, s_, ...)                                                       \
+  do {                                                                                                       \
+    const int gsz = (k_) <= 8 ? 8 : ((k_) <= 16 ? 16 : 32);                                                  \
+    const int grid = rows_grid((static_cast<long long>(T_) * gsz + 31) / 32);                                 \
+    if (gsz == 8) PFMOE_LAUNCH(NAME, s_, (KERNEL<8><<<grid, 256, 0, s_>>>(__VA_ARGS__)));                     \
+    else if (gsz == 16) PFMOE_LAUNCH(NAME, s_, (KERNEL<16><<<grid, 256, 0, s_>>>(__VA_ARGS__)));              \
+    else PFMOE_LAUNCH(NAME, s_, (KERNEL<32><<<grid, 256, 0, s_>>>(__VA_ARGS__)));                             \
+  } while (0)
 
 int rows_grid(long long rows, int warps_per_blk = 8) {
   long long b = (rows + warps_per_blk - 1) / warps_per_blk;
@@ -553,8 +585,7 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
   int32_t* ccounts = p; p += static_cast<long long>(C > 0 ? C : 1) * n_nodes;
   int32_t* cbase = p;
 
-  const int g = rows_grid(T);
-  PFMOE_LAUNCH("rbd_count", s, rbd_count_kernel<<<g, 256, 0, s>>>(ids, T, k, E, epd, epn, ucount, dcount, err));
+  PFMOE_RBD_LAUNCH("rbd_count", rbd_count_kernel, T, k, s, ids, T, k, E, epd, epn, ucount, dcount, err);
   if (T < LONG_SCAN_MIN) {
     PFMOE_LAUNCH("rbd_scan_tokens", s, rbd_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(ucount, dcount, T, pbase, counts));
   } else {
@@ -566,7 +597,7 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
                                                                 nullptr));
     PFMOE_LAUNCH("rbd_scan_tokens", s, tile_scan_kernel<<<nt, SCAN_THREADS, 0, s>>>(ucount, T, nullptr, tsum_a, pbase));
   }
-  PFMOE_LAUNCH("rbd_emit", s, rbd_emit_kernel<<<g, 256, 0, s>>>(ids, T, k, E, epd, epn, pbase, pkey, ptoken, prc, err));
+  PFMOE_RBD_LAUNCH("rbd_emit", rbd_emit_kernel, T, k, s, ids, T, k, E, epd, epn, pbase, pkey, ptoken, prc, err);
   const int wpb = warps_per_block(n_nodes);
   const int blocks = C;
   const size_t sm = static_cast<size_t>(wpb) * n_nodes * sizeof(int32_t);
@@ -598,9 +629,8 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
     PFMOE_LAUNCH("rbd_scan_replicas", s,
                  tile_scan_kernel<<<nt, SCAN_THREADS, 0, s>>>(rc_sorted, pmax, counts, tsum_a, replica_offsets));
   }
-  PFMOE_LAUNCH("rbd_final", s,
-               rbd_final_kernel<<<g, 256, 0, s>>>(ids, T, k, E, epd, epn, pbase, psorted, replica_offsets,
-                                                   assign_pilot, replica_expert, pilot_device, err));
+  PFMOE_RBD_LAUNCH("rbd_final", rbd_final_kernel, T, k, s, ids, T, k, E, epd, epn, pbase, psorted, replica_offsets,
+                   assign_pilot, replica_expert, pilot_device, err);
   return PFMOE_OK;
 }
 
