@@ -116,7 +116,7 @@ PFMOE_API int pft_build(const int32_t* topk_ids, const float* topk_w, int T, int
  *   bytes of device memory that every GPU loading the library holds until the
  *   process exits).  It allocates nothing.
  *   Limit: pft_build_workspace_size(T, E, k) must not exceed
- *   PFMOE_PFT_NO_WS_SCRATCH_BYTES (for example T*k up to 262144 with E up to 1024);
+ *   PFMOE_PFT_NO_WS_SCRATCH_BYTES (for example T*k up to 260096 with E = 1024, 1046528 with E = 256);
  *   larger shapes return PFMOE_ERR_UNSUPPORTED with a message naming both sizes.
  *   The first call on a device looks up the array's device address (once, with
  *   that device current); make that first call before any stream capture.
