@@ -1,7 +1,7 @@
 """CUDA path vs the CPU oracle, element by element, on layers the oracle runs in
 full: several tiles per expert, ragged segment tails, d and h that are not
-multiples of the GEMM tiles, empty experts, k = E, a single token, rows wider
-than 16 column chunks, FP32."""
+multiples of the GEMM tiles, empty experts, k = E, k > 16, a single token, rows
+wider than 16 column chunks, FP32."""
 import numpy as np
 import pytest
 import torch
@@ -12,7 +12,7 @@ from workloads import get_config, make_inputs
 from tests.parity import LOGIT_TOL, TOL, check_index_parity, f64, i64, make_layer, rel_err, run_step
 
 SMALL = ["small_bf16", "small_ragged_bf16", "small_skew_bf16", "small_kE_bf16", "small_f32", "one_token_bf16",
-         "tiny_fp32", "small_pairs_bf16", "wide_d_bf16", "wide_d_f32"]
+         "tiny_fp32", "small_pairs_bf16", "wide_d_bf16", "wide_d_f32", "big_k_bf16"]
 
 
 @pytest.mark.gpu

@@ -87,6 +87,8 @@ SMALL = {
     # and the last item of every row is partial (17 and 18 chunks).
     "wide_d_bf16": LayerConfig("wide_d_bf16", T=96, d=4160, E=8, h=64, k=3, dtype="bf16"),
     "wide_d_f32": LayerConfig("wide_d_f32", T=40, d=2200, E=6, h=40, k=2, dtype="f32"),
+    # k > 16: the RBD per-token kernels use whole 32-lane groups; 8 nodes of 8 experts.
+    "big_k_bf16": LayerConfig("big_k_bf16", T=96, d=64, E=64, h=64, k=20, dtype="bf16", rbd_epd=4, rbd_dpn=2),
 }
 
 
