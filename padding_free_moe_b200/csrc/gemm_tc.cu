@@ -66,6 +66,7 @@ struct Params {
   int a_merged;      // MN-major A map is the 4-D block view (one copy fetches every 64-wide block of a stage)
   int b_merged;      // same for the MN-major B maps
   int fstep;         // token-as-N kernel: output features per pair tile (256, or 128 with nsplit)
+  int tn_nb;         // token-as-N kernel: epilogue chunk buffers (2; 1 where shared memory is short)
   int bn;            // MMA N: multiple of 64, <= 256
   int nsplit;        // 1: B tile columns [0, bn/2) come from tmB[0], [bn/2, bn) from tmB[1]
   int M;             // KG: rows of each group's output
@@ -809,9 +810,10 @@ static int make_tmap_mn(CUtensorMap* m, const void* ptr, uint64_t mn, uint64_t k
   return PFMOE_OK;
 }
 
-// Output map for the token-as-N kernel: BF16 [rows][cols], 32 x 32 boxes, unswizzled 64-byte rows.
+// Output map for the token-as-N kernel: BF16 [rows][cols], boxes of 32 rows x 64 columns with the
+// 128-byte swizzle (one staged epilogue block).
 static int make_out_map_tn(CUtensorMap* m, void* ptr, uint64_t cols, uint64_t rows, const char* what) {
-  return make_tmap_t(m, ptr, false, cols, rows, 1, 32, 32, what, false);
+  return make_tmap_t(m, ptr, false, cols, rows, 1, 64, 32, what, true);
 }
 
 static int round_bn(int n) {
@@ -940,14 +942,17 @@ __device__ __forceinline__ void tc_commit2_both(uint32_t bar) {
 // token columns [vN/2, (v+1)N/2)).  A ragged expert segment therefore costs at
 // most 31 spare MMA columns, where 256-row tiles over tokens compute up to 255
 // spare rows; on MoE layers with a few hundred tokens per expert that is a
-// quarter of the row-major kernel's tensor work.  The epilogue transposes
-// 32 x 32 blocks through shared memory and stores [token, feature] rows.
+// quarter of the row-major kernel's tensor work.  The epilogue transposes the
+// accumulator through shared memory into [token, feature] rows: the four
+// epilogue warps of a CTA fill 32-token x 64-feature blocks together and one
+// thread writes each block with a single TMA store (fewer, larger copies: the
+// per-copy cost of TMA is shared with the operand loads).
 //
 // With nsplit (SwiGLU forward) a pair tile covers 128 features: CTA v holds
 // rows [64v, 64v + 64) of W1^T in TMEM lanes 0..63 and the same rows of W3^T in
-// lanes 64..127, so the H1 and H3 values of one (token, feature) sit in the
-// same lane of epilogue warps q and q + 2; warp q + 2 hands its FP32 H3 block
-// to warp q through shared memory (bounded mbarrier handshake).
+// lanes 64..127.  Warps q and q + 2 stage the H1 and H3 bands of one block
+// pair; after a barrier all four warps form the A block element-wise from the
+// two staged BF16 blocks, so A = SiLU(H1) * H3 of the values that are stored.
 constexpr int TN_TOK = 256;             // tokens per pair tile
 // K depth of one ring stage: two 64-element sub-blocks, so each mbarrier handshake feeds eight
 // K16 MMAs.  Measured on this part: back-to-back M=256 N=256 pair MMAs take ~130 cycles each, and
@@ -955,13 +960,15 @@ constexpr int TN_TOK = 256;             // tokens per pair tile
 constexpr int TN_BK = 2 * BK;
 constexpr int TN_SUB = 128 * BK * 2;    // one 64-deep sub-block of 128 rows (16 KB)
 constexpr int TN_STAGE = 4 * TN_SUB;    // A: 2 sub-blocks (or 2 feature blocks), B: 2 sub-blocks
-constexpr int TN_SLAB = 32 * 64;        // one 32-token x 32-feature BF16 block (64-byte rows)
-constexpr int TN_XBUF = 32 * 32 * 4;    // one 32 x 32 FP32 block
+constexpr int TN_BLK = 32 * 128;        // one 32-token x 64-feature BF16 block (128-byte rows)
 
-// SwiGLU forward: one FP32 hand-off block per warp pair.  (The SwiGLU backward reads its H1 / H3
-// blocks through the epilogue warp's own staging slabs.)
-__host__ __device__ constexpr int tn_aux_bytes(int epi) { return epi == EPI_SWIGLU_FWD ? 2 * TN_XBUF : 0; }
-constexpr int TN_STAGING = 4 * 2 * TN_SLAB;   // epilogue staging: 2 slabs per epilogue warp
+// Epilogue blocks per 32-token chunk: H1, H3, A (SwiGLU forward); dH1 and dH3, two 64-feature
+// halves each (SwiGLU backward); two 64-feature halves (plain store).  nb chunk buffers are used
+// in turn.
+__host__ __device__ constexpr int tn_blocks(int epi) {
+  return epi == EPI_SWIGLU_FWD ? 3 : (epi == EPI_SWIGLU_BWD ? 4 : 2);
+}
+__host__ __device__ constexpr int tn_staging_bytes(int epi, int nb) { return nb * tn_blocks(epi) * TN_BLK; }
 
 struct TnTile {
   int g, tok0, ntok, nmma, f0, nk;
@@ -1015,181 +1022,245 @@ __device__ __forceinline__ uint32_t ld_shared32(uint32_t addr) {
   return v;
 }
 
-// Transposes between a thread-per-feature register block (v[j] = token j of feature `lane`)
-// and a [token][feature] BF16 slab with 64-byte rows.  Neighbouring lanes swap one value so
-// every shared access is a 32-bit word holding two adjacent features; even lanes touch row j
-// and odd lanes row j + 1, which sit in opposite halves of the 32 banks.
-__device__ __forceinline__ void stage_t_write(uint32_t slab, int lane, const float* v) {
+// A staged block is [32 tokens][64 features] BF16 with 128-byte rows; 16-byte chunk c of row t
+// sits at chunk position c ^ (t & 7) (the TMA 128-byte swizzle).  Epilogue warp q owns the
+// 32-feature band (q & 1) of a block: chunks 4 band .. 4 band + 3.
+__device__ __forceinline__ uint32_t blk_addr(uint32_t blk, int t, int chunk) {
+  return blk + static_cast<uint32_t>(t * 128 + ((chunk ^ (t & 7)) << 4));
+}
+
+// Register block (v[j] = token j of feature `lane` of the band) -> staged block.  Lanes 2i and
+// 2i + 1 swap one value so that each shared access is a 32-bit word with features 2i, 2i + 1 of
+// one token: the even lane writes token j and the odd lane token j + 4, whose swizzled chunk
+// lies in the other half of the banks.
+__device__ __forceinline__ void blk_write(uint32_t blk, int band, int lane, const float* v) {
   const int odd = lane & 1;
-  const uint32_t col = static_cast<uint32_t>(lane & ~1) * 2;
+  const int i = lane >> 1;
+  const int chunk = 4 * band + (i >> 2);
+  const uint32_t w = (i & 3) * 4;
 #pragma unroll
-  for (int j = 0; j < 32; j += 2) {
-    const float send = odd ? v[j] : v[j + 1];
+  for (int jj = 0; jj < 16; ++jj) {
+    const int j = (jj & 3) + 8 * (jj >> 2);
+    const float send = odd ? v[j] : v[j + 4];
     const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-    __nv_bfloat162 b = __floats2bfloat162_rn(odd ? recv : v[j], odd ? v[j + 1] : recv);
-    st_shared32(slab + (j + odd) * 64 + col, *reinterpret_cast<uint32_t*>(&b));
+    const __nv_bfloat162 b = __floats2bfloat162_rn(odd ? recv : v[j], odd ? v[j + 4] : recv);
+    st_shared32(blk_addr(blk, j + 4 * odd, chunk) + w, *reinterpret_cast<const uint32_t*>(&b));
   }
 }
 
-__device__ __forceinline__ void stage_t_read(uint32_t slab, int lane, float* v) {
+// Staged block -> register block (the inverse of blk_write).
+__device__ __forceinline__ void blk_read(uint32_t blk, int band, int lane, float* v) {
   const int odd = lane & 1;
-  const uint32_t col = static_cast<uint32_t>(lane & ~1) * 2;
+  const int i = lane >> 1;
+  const int chunk = 4 * band + (i >> 2);
+  const uint32_t w = (i & 3) * 4;
 #pragma unroll
-  for (int j = 0; j < 32; j += 2) {
-    const uint32_t w = ld_shared32(slab + (j + odd) * 64 + col);
-    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+  for (int jj = 0; jj < 16; ++jj) {
+    const int j = (jj & 3) + 8 * (jj >> 2);
+    const uint32_t word = ld_shared32(blk_addr(blk, j + 4 * odd, chunk) + w);
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&word));
     const float recv = __shfl_xor_sync(0xffffffffu, odd ? f.x : f.y, 1);
     v[j] = odd ? recv : f.x;
-    v[j + 1] = odd ? f.y : recv;
+    v[j + 4] = odd ? f.y : recv;
   }
 }
 
-// Slab <-> global rows (32 rows of up to 64 bytes; eight rows per instruction, 16 bytes a lane).
-// Rows >= rows_valid and bytes >= bytes_valid are skipped on the way out and read as zero on the way in.
-__device__ __forceinline__ void copy_out_t(uint32_t slab, int lane, char* base, long long stride, int rows_valid,
-                                           int bytes_valid) {
-  const int chunk = lane & 3;
+// One band's 32 rows x 64 bytes <-> global rows, 16 bytes a lane.  Lanes 8g .. 8g + 3 take row
+// 8 it + g and lanes 8g + 4 .. 8g + 7 row 8 it + g + 4, so each group of eight lanes covers all
+// 32 banks.  Rows >= rows_valid and bytes >= bytes_valid are skipped (loaded as zero).
+__device__ __forceinline__ int band_row(int it, int lane) { return 8 * it + (lane >> 3) + 4 * ((lane >> 2) & 1); }
+
+__device__ __forceinline__ void band_load(uint4 (&u)[4], int lane, const char* base, long long stride, int rows_valid,
+                                          int bytes_valid) {
+  const int c = lane & 3;
 #pragma unroll
   for (int it = 0; it < 4; ++it) {
-    const int row = it * 8 + (lane >> 2);
-    const uint4 u = ld_shared16(slab + row * 64 + chunk * 16);
-    if (row < rows_valid && chunk * 16 < bytes_valid)
-      *reinterpret_cast<uint4*>(base + row * stride + chunk * 16) = u;
-  }
-}
-__device__ __forceinline__ void load_t(uint4 (&u)[4], int lane, const char* base, long long stride, int rows_valid,
-                                       int bytes_valid) {
-  const int chunk = lane & 3;
-#pragma unroll
-  for (int it = 0; it < 4; ++it) {
-    const int row = it * 8 + (lane >> 2);
+    const int r = band_row(it, lane);
     u[it] = make_uint4(0, 0, 0, 0);
-    if (row < rows_valid && chunk * 16 < bytes_valid)
-      u[it] = __ldg(reinterpret_cast<const uint4*>(base + row * stride + chunk * 16));
+    if (r < rows_valid && c * 16 < bytes_valid)
+      u[it] = __ldg(reinterpret_cast<const uint4*>(base + r * stride + c * 16));
   }
 }
-__device__ __forceinline__ void put_t(uint32_t slab, int lane, const uint4 (&u)[4]) {
-  const int chunk = lane & 3;
+__device__ __forceinline__ void band_put(uint32_t blk, int band, int lane, const uint4 (&u)[4]) {
+  const int c = 4 * band + (lane & 3);
 #pragma unroll
-  for (int it = 0; it < 4; ++it) st_shared16(slab + (it * 8 + (lane >> 2)) * 64 + chunk * 16, u[it]);
+  for (int it = 0; it < 4; ++it) st_shared16(blk_addr(blk, band_row(it, lane), c), u[it]);
 }
-
-// Transpose one 32 x 32 block into the next staging slab and write it out: a block of 32 valid
-// tokens goes out as one TMA store (clipped at the feature bound); a partial block with masked
-// vector stores, so tokens of the next expert segment are never touched.
-__device__ __forceinline__ void emit_t(Stager& st, int lane, const float* v, const CUtensorMap* tm, int f, int tok,
-                                       __nv_bfloat16* dst, long long ldd, int rows_valid, int fvalid) {
-  const uint32_t buf = st.base + (st.seq & 1) * TN_SLAB;
-  ++st.seq;
-  if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-  __syncwarp();
-  stage_t_write(buf, lane, v);
-  if (tm && rows_valid == 32) {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncwarp();
-    if (lane == 0) tma_store_3d(tm, buf, f, tok, 0);
-  } else {
-    __syncwarp();
-    copy_out_t(buf, lane, reinterpret_cast<char*>(dst), ldd * 2, rows_valid, min(64, fvalid * 2));
+__device__ __forceinline__ void band_copy_out(uint32_t blk, int band, int lane, char* base, long long stride,
+                                              int rows_valid, int bytes_valid) {
+  const int c = lane & 3;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int r = band_row(it, lane);
+    const uint4 u = ld_shared16(blk_addr(blk, r, 4 * band + c));
+    if (r < rows_valid && c * 16 < bytes_valid) *reinterpret_cast<uint4*>(base + r * stride + c * 16) = u;
   }
-  if (lane == 0) asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
-// Epilogue of one pair tile for epilogue warp q (TMEM lanes 32q..32q+31).  `xn` counts the H3
-// hand-offs of this warp pair (SwiGLU forward).  Returns false if a hand-off wait gave up.
+// The four epilogue warps (128 threads) synchronise on named barrier 1.
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ bool epi_all(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred))
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void store_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Two BF16 SwiGLU products SiLU(h1) * h3 of a packed pair.
+__device__ __forceinline__ uint32_t swiglu_bf16x2(uint32_t h1w, uint32_t h3w) {
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h1w));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h3w));
+  const __nv_bfloat162 r = __floats2bfloat162_rn(a.x * sigmoid_fast(a.x) * b.x, a.y * sigmoid_fast(a.y) * b.y);
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// Epilogue of one pair tile for epilogue warp q (TMEM lanes 32q .. 32q + 31).
+//
+// Every 32-token chunk takes the same barrier steps in all four warps (the chunk count and the
+// early return depend only on the tile and the CTA), so no warp is ever left at a barrier.  A
+// chunk of 32 valid tokens leaves as TMA stores of whole blocks, issued by one thread
+// (`issuer`); a ragged last chunk leaves with masked vector stores by each band's owner, so
+// rows of the next expert segment are never touched.  `seq` counts the CTA's chunks and picks
+// the chunk buffer; before each barrier after which a buffer is written again, the issuer waits
+// until the stores that read that buffer have read it.
 template <int EPI>
-__device__ __forceinline__ bool epilogue_tn(const Params& p, const TnTile& tl, uint32_t tacc, int q, int lane,
-                                            uint32_t rank, Stager& st, uint32_t aux, uint64_t* xfull,
-                                            uint64_t* xempty, int& xn, volatile int* abort_flag) {
+__device__ __forceinline__ void epilogue_tn(const Params& p, const TnTile& tl, uint32_t tacc, int q, int lane,
+                                            uint32_t rank, uint32_t staging, int& seq, bool issuer) {
   const int nch = (tl.ntok + 31) / 32;
   const long long ldd = p.ldd;
+  const int band = q & 1;
   if constexpr (EPI == EPI_SWIGLU_FWD) {
-    const int pid = q & 1;
-    const bool h3_warp = q >= 2;
-    const int fw = tl.f0 + 64 * static_cast<int>(rank) + 32 * pid;
-    const int fvalid = min(32, p.Nout - fw);
-    if (fvalid <= 0) return true;   // both warps of the pair skip together
-    __nv_bfloat16* H1 = static_cast<__nv_bfloat16*>(p.D0);
-    __nv_bfloat16* H3 = static_cast<__nv_bfloat16*>(p.D1);
-    __nv_bfloat16* A = static_cast<__nv_bfloat16*>(p.D2);
-    for (int c = 0; c < nch; ++c, ++xn) {
+    const int fc = tl.f0 + 64 * static_cast<int>(rank);   // this CTA's 64 features
+    if (fc >= p.Nout) return;
+    const int fw = fc + 32 * band;
+    const int bytes = max(0, min(64, (p.Nout - fw) * 2));
+    const int own = q >> 1;                                 // 0: H1 band, 1: H3 band
+    char* Hown = static_cast<char*>(own ? p.D1 : p.D0);
+    char* A = static_cast<char*>(p.D2);
+    for (int c = 0; c < nch; ++c, ++seq) {
       const int tok = tl.tok0 + 32 * c;
       const int rv = min(32, tl.ntok - 32 * c);
-      const long long off = static_cast<long long>(tok) * ldd + fw;
-      const uint32_t ph = xn & 1;                 // one hand-off buffer per pair: one phase per chunk
-      const uint32_t xb = aux + pid * TN_XBUF;
+      const bool full = rv == 32 && p.tma_store;
+      const uint32_t buf = staging + (seq & 1) * 3 * TN_BLK;
       float v[32];
       tmem_ld32(tacc + 32 * c, v);
-      if (h3_warp) {
-        emit_t(st, lane, v, tmd(p, 1), fw, tok, H3 + off, ldd, rv, fvalid);
-        if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&xempty[pid]), ph ^ 1, abort_flag, p.err)))
-          return false;
+      blk_write(buf + own * TN_BLK, band, lane, v);
+      if (full) fence_async_smem();
+      epi_sync();                                           // H1 and H3 blocks complete
+      if (full && issuer) {
+        tma_store_3d(tmd(p, 0), buf, fc, tok, 0);
+        tma_store_3d(tmd(p, 1), buf + TN_BLK, fc, tok, 0);
+        store_commit();
+      }
+      // A block, element-wise: warp q takes bytes [1024 q, 1024 q + 1024) of the three blocks.
 #pragma unroll
-        for (int j = 0; j < 32; ++j) st_shared32(xb + (j * 32 + lane) * 4, __float_as_uint(v[j]));
-        mbar_arrive(smem_u32(&xfull[pid]));
-      } else {
-        emit_t(st, lane, v, tmd(p, 0), fw, tok, H1 + off, ldd, rv, fvalid);
-        if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&xfull[pid]), ph, abort_flag, p.err)))
-          return false;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float h3 = __uint_as_float(ld_shared32(xb + (j * 32 + lane) * 4));
-          v[j] = v[j] * sigmoid_fast(v[j]) * h3;
+      for (int it = 0; it < 2; ++it) {
+        const uint32_t off = q * 1024 + it * 512 + lane * 16;
+        const uint4 h1 = ld_shared16(buf + off);
+        const uint4 h3 = ld_shared16(buf + TN_BLK + off);
+        const uint4 a = make_uint4(swiglu_bf16x2(h1.x, h3.x), swiglu_bf16x2(h1.y, h3.y), swiglu_bf16x2(h1.z, h3.z),
+                                   swiglu_bf16x2(h1.w, h3.w));
+        st_shared16(buf + 2 * TN_BLK + off, a);
+      }
+      if (full) fence_async_smem();
+      // Chunk buffers alternate: the next chunk's H1 / H3 go where the previous chunk's did, so
+      // every store but this chunk's H1 / H3 pair must have read its block.
+      if (issuer) {
+        if (full) store_wait_read<1>(); else store_wait_read<0>();
+      }
+      epi_sync();                                           // A block complete
+      if (full) {
+        if (issuer) {
+          tma_store_3d(tmd(p, 2), buf + 2 * TN_BLK, fc, tok, 0);
+          store_commit();
         }
-        mbar_arrive(smem_u32(&xempty[pid]));
-        emit_t(st, lane, v, tmd(p, 2), fw, tok, A + off, ldd, rv, fvalid);
+      } else if (bytes > 0) {
+        const long long off = (static_cast<long long>(tok) * ldd + fw) * 2;
+        band_copy_out(buf + own * TN_BLK, band, lane, Hown + off, ldd * 2, rv, bytes);
+        if (own == 0) band_copy_out(buf + 2 * TN_BLK, band, lane, A + off, ldd * 2, rv, bytes);
       }
     }
   } else if constexpr (EPI == EPI_STORE_BF16) {
-    const int fw = tl.f0 + 128 * static_cast<int>(rank) + 32 * q;
-    const int fvalid = min(32, p.Nout - fw);
-    if (fvalid <= 0) return true;
-    __nv_bfloat16* D = static_cast<__nv_bfloat16*>(p.D0);
-    for (int c = 0; c < nch; ++c) {
+    const int fc = tl.f0 + 128 * static_cast<int>(rank);  // this CTA's 128 features: two blocks
+    if (fc >= p.Nout) return;
+    const int fw = fc + 32 * q;
+    const int bytes = max(0, min(64, (p.Nout - fw) * 2));
+    const bool second = fc + 64 < p.Nout;
+    char* D = static_cast<char*>(p.D0);
+    for (int c = 0; c < nch; ++c, ++seq) {
       const int tok = tl.tok0 + 32 * c;
+      const int rv = min(32, tl.ntok - 32 * c);
+      const bool full = rv == 32 && p.tma_store;
+      const uint32_t buf = staging + (seq & 1) * 2 * TN_BLK;
       float v[32];
       tmem_ld32(tacc + 32 * c, v);
-      emit_t(st, lane, v, tmd(p, 0), fw, tok, D + static_cast<long long>(tok) * ldd + fw, ldd,
-             min(32, tl.ntok - 32 * c), fvalid);
+      blk_write(buf + (q >> 1) * TN_BLK, band, lane, v);
+      if (full) fence_async_smem();
+      if (issuer) store_wait_read<0>();                     // the previous chunk's buffer is free
+      epi_sync();
+      if (full) {
+        if (issuer) {
+          tma_store_3d(tmd(p, 0), buf, fc, tok, 0);
+          if (second) tma_store_3d(tmd(p, 0), buf + TN_BLK, fc + 64, tok, 0);
+          store_commit();
+        }
+      } else if (bytes > 0) {
+        band_copy_out(buf + (q >> 1) * TN_BLK, band, lane, D + (static_cast<long long>(tok) * ldd + fw) * 2, ldd * 2,
+                      rv, bytes);
+      }
     }
   } else if constexpr (EPI == EPI_SWIGLU_BWD) {
     // Accumulator = dA^T.  dH1 = dA * H3 * s * (1 + H1 (1 - s)), dH3 = dA * SiLU(H1), s = sigmoid(H1).
-    // The H1 / H3 blocks of chunk c + 1 are fetched into registers while chunk c is computed.
-    const int fw = tl.f0 + 128 * static_cast<int>(rank) + 32 * q;
-    const int fvalid = min(32, p.Nout - fw);
-    if (fvalid <= 0) return true;
+    // Each warp brings its H1 / H3 bands in through its own bands of the dH1 / dH3 blocks (rows
+    // fetched into registers one chunk ahead), then overwrites them with the results.
+    const int fc = tl.f0 + 128 * static_cast<int>(rank);
+    if (fc >= p.Nout) return;
+    const int fw = fc + 32 * q;
+    const int bytes = max(0, min(64, (p.Nout - fw) * 2));
+    const bool second = fc + 64 < p.Nout;
+    const int nb = p.tn_nb;
     const char* H1 = static_cast<const char*>(p.X0);
     const char* H3 = static_cast<const char*>(p.X1);
-    __nv_bfloat16* dH1 = static_cast<__nv_bfloat16*>(p.D0);
-    __nv_bfloat16* dH3 = static_cast<__nv_bfloat16*>(p.D1);
-    // H1 / H3 blocks pass through this warp's two staging slabs, once the TMA stores that last
-    // used them have read them out.
-    const uint32_t in1 = st.base;
-    const uint32_t in3 = st.base + TN_SLAB;
-    const int bv = min(64, fvalid * 2);
+    char* dH1 = static_cast<char*>(p.D0);
+    char* dH3 = static_cast<char*>(p.D1);
     uint4 r1[4], r3[4];
     {
       const long long boff = (static_cast<long long>(tl.tok0) * ldd + fw) * 2;
-      load_t(r1, lane, H1 + boff, ldd * 2, min(32, tl.ntok), bv);
-      load_t(r3, lane, H3 + boff, ldd * 2, min(32, tl.ntok), bv);
+      band_load(r1, lane, H1 + boff, ldd * 2, min(32, tl.ntok), bytes);
+      band_load(r3, lane, H3 + boff, ldd * 2, min(32, tl.ntok), bytes);
     }
-    for (int c = 0; c < nch; ++c) {
+    for (int c = 0; c < nch; ++c, ++seq) {
       const int tok = tl.tok0 + 32 * c;
       const int rv = min(32, tl.ntok - 32 * c);
-      if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-      __syncwarp();
-      put_t(in1, lane, r1);
-      put_t(in3, lane, r3);
+      const bool full = rv == 32 && p.tma_store;
+      const uint32_t buf = staging + (nb == 2 ? (seq & 1) : 0) * 4 * TN_BLK;
+      const uint32_t b1 = buf + (q >> 1) * TN_BLK;          // dH1 half holding this warp's band
+      const uint32_t b3 = b1 + 2 * TN_BLK;                  // dH3 half
+      if (nb == 1) {                                        // one buffer: the last chunk's stores first
+        if (issuer) store_wait_read<0>();
+        epi_sync();
+      }
+      band_put(b1, band, lane, r1);
+      band_put(b3, band, lane, r3);
       if (c + 1 < nch) {
         const long long boff = (static_cast<long long>(tok + 32) * ldd + fw) * 2;
-        load_t(r1, lane, H1 + boff, ldd * 2, min(32, tl.ntok - 32 * (c + 1)), bv);
-        load_t(r3, lane, H3 + boff, ldd * 2, min(32, tl.ntok - 32 * (c + 1)), bv);
+        band_load(r1, lane, H1 + boff, ldd * 2, min(32, tl.ntok - 32 * (c + 1)), bytes);
+        band_load(r3, lane, H3 + boff, ldd * 2, min(32, tl.ntok - 32 * (c + 1)), bytes);
       }
       __syncwarp();
       float da[32], h1[32], h3[32];
-      stage_t_read(in1, lane, h1);
-      stage_t_read(in3, lane, h3);
-      __syncwarp();   // every lane has read the slabs before the first emit reuses one
+      blk_read(b1, band, lane, h1);
+      blk_read(b3, band, lane, h3);
+      __syncwarp();                                         // every lane has read the bands
       tmem_ld32(tacc + 32 * c, da);
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -1198,12 +1269,26 @@ __device__ __forceinline__ bool epilogue_tn(const Params& p, const TnTile& tl, u
         h1[i] = da[i] * h1[i] * s;
         da[i] = d1;
       }
-      const long long off = static_cast<long long>(tok) * ldd + fw;
-      emit_t(st, lane, da, tmd(p, 0), fw, tok, dH1 + off, ldd, rv, fvalid);
-      emit_t(st, lane, h1, tmd(p, 1), fw, tok, dH3 + off, ldd, rv, fvalid);
+      blk_write(b1, band, lane, da);
+      blk_write(b3, band, lane, h1);
+      if (full) fence_async_smem();
+      if (issuer && nb == 2) store_wait_read<0>();
+      epi_sync();
+      if (full) {
+        if (issuer) {
+          tma_store_3d(tmd(p, 0), buf, fc, tok, 0);
+          if (second) tma_store_3d(tmd(p, 0), buf + TN_BLK, fc + 64, tok, 0);
+          tma_store_3d(tmd(p, 1), buf + 2 * TN_BLK, fc, tok, 0);
+          if (second) tma_store_3d(tmd(p, 1), buf + 3 * TN_BLK, fc + 64, tok, 0);
+          store_commit();
+        }
+      } else if (bytes > 0) {
+        const long long off = (static_cast<long long>(tok) * ldd + fw) * 2;
+        band_copy_out(b1, band, lane, dH1 + off, ldd * 2, rv, bytes);
+        band_copy_out(b3, band, lane, dH3 + off, ldd * 2, rv, bytes);
+      }
     }
   }
-  return true;
 }
 
 template <int EPI>
@@ -1213,9 +1298,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages;
   constexpr uint32_t stage_bytes = TN_STAGE;   // 128 weight rows + 128 token rows, 128 deep in K
-  uint8_t* stage_area = smem + S * stage_bytes;               // 4 warps x 2 staging slabs
-  uint8_t* aux_area = stage_area + TN_STAGING;
-  int* pair_off = reinterpret_cast<int*>(aux_area + tn_aux_bytes(EPI));
+  uint8_t* stage_area = smem + S * stage_bytes;               // epilogue chunk buffers
+  int* pair_off = reinterpret_cast<int*>(stage_area + tn_staging_bytes(EPI, p.tn_nb));
   const int poff_ints = (p.G + 1 + 63) & ~63;
   uint8_t* bar_area = reinterpret_cast<uint8_t*>(pair_off + poff_ints);
   uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
@@ -1223,9 +1307,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint64_t* acc_full = empty + MAX_STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint64_t* xfull = drain + 1;
-  uint64_t* xempty = xfull + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xempty + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -1244,10 +1326,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&acc_full[b]), 1);
       mbar_init(smem_u32(&acc_empty[b]), 2 * 4 * 32);
-    }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(smem_u32(&xfull[i]), 32);
-      mbar_init(smem_u32(&xempty[i]), 32);
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
@@ -1400,21 +1478,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int q = warp & 3;
     const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
     const uint32_t acc_empty_leader1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
-    Stager stg{smem_u32(stage_area + q * 2 * TN_SLAB), 0};
-    const uint32_t aux = smem_u32(aux_area);
-    int tcount = 0, xn = 0;
+    const uint32_t staging = smem_u32(stage_area);
+    const bool issuer = q == 0 && lane == 0;
+    int tcount = 0, seq = 0;
     int wave = 0;
     TnTile tl;
     for (; tn_next(p, pair_off, npairs, pair, wave, tl); ++tcount) {
       const int buf = tcount & 1;
       const uint32_t aph = (tcount >> 1) & 1;
-      if (!__all_sync(0xffffffffu, wait_bar2(smem_u32(&acc_full[buf]), aph, abort_flag, p.err))) break;
+      const bool got = __all_sync(0xffffffffu, wait_bar2(smem_u32(&acc_full[buf]), aph, abort_flag, p.err));
+      if (!epi_all(got)) break;   // the four warps leave together, so none waits at a barrier
       tc_fence_after();
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * TN_TOK;
-      const bool ok = epilogue_tn<EPI>(p, tl, tacc, q, lane, rank, stg, aux, xfull, xempty, xn, abort_flag);
+      epilogue_tn<EPI>(p, tl, tacc, q, lane, rank, staging, seq, issuer);
       tc_fence_before();
       mbar_arrive_cluster(buf ? acc_empty_leader1 : acc_empty_leader0);
-      if (!ok) break;
     }
     emit_drain(lane);
   }
@@ -1469,7 +1547,11 @@ static int launch_tn(Params& p, long long pair_tile_upper_bound, const char* nam
   p.mode = RG;
   const int stage = TN_STAGE;
   const int poff = ((p.G + 1 + 63) & ~63) * 4;
-  const int fixed = 1024 + 512 + poff + TN_STAGING + tn_aux_bytes(EPI);
+  // Two epilogue chunk buffers, unless that costs the SwiGLU backward (four blocks a chunk) its
+  // third ring stage; it then runs with one buffer and a second barrier per chunk.
+  p.tn_nb = 2;
+  if (EPI == EPI_SWIGLU_BWD && (SMEM_LIMIT - (1024 + 512 + poff + tn_staging_bytes(EPI, 2))) / stage < 3) p.tn_nb = 1;
+  const int fixed = 1024 + 512 + poff + tn_staging_bytes(EPI, p.tn_nb);
   const int st = (SMEM_LIMIT - fixed) / stage;
   if (st < 2) return fail(PFMOE_ERR_UNSUPPORTED, std::string(name) + ": too many experts for the shared-memory plan");
   p.stages = st > MAX_STAGES ? MAX_STAGES : st;
