@@ -23,7 +23,10 @@
 // warps 2..5 = epilogue (TMEM lane quarter q = warp % 4), warp 6 (K-grouped
 // launches only) = K-tail zeroing.  Every wait on an mbarrier is bounded
 // (%globaltimer); on expiry the kernel sets PFMOE_DEV_TIMEOUT, drains its own
-// copies and MMAs, frees TMEM and returns.
+// copies and MMAs, frees TMEM and returns.  The token-as-N epilogue warps also
+// meet at a named barrier once or twice per 32-token chunk; all four take the
+// same barrier steps and leave their tile loop together through a barrier vote,
+// so none waits at a barrier that another has left.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
