@@ -166,20 +166,40 @@ __global__ void __launch_bounds__(SCAN_THREADS) key_scan_kernel(const int32_t* _
   }
 }
 
-// Stable scatter; Sink(i, p, key) records that element i lands at sorted position p.
+// Stable scatter.  Pass 1 counts each warp's keys.  Pass 2 gives every element its sorted row p
+// (its key's first row in this chunk, plus the rows of earlier warps with that key, plus its rank
+// among the warp's equal keys) and stages it in shared memory in sorted order.  The write-out then
+// stores the row-indexed outputs as runs of consecutive rows, so neighbouring lanes write
+// neighbouring addresses instead of one scattered sector per element.
+// Sink interface: at_source(i, p) writes the outputs indexed by element i; payload(i, a, b) gives
+// two ints carried to the sorted side; at_dest(p, key, a, b) writes the outputs indexed by row p.
+// Shared memory: [warps][K] counts, two [K] bases and three [warps * KEYS_PER_WARP] staging arrays.
+__host__ __device__ inline size_t scatter_smem_bytes(int nw, int K) {
+  return (static_cast<size_t>(nw) * K + 2 * static_cast<size_t>(K) + 3 * static_cast<size_t>(nw) * KEYS_PER_WARP) *
+         sizeof(int32_t);
+}
+
 template <class Sink>
 __global__ void chunk_scatter_kernel(const int32_t* __restrict__ keys, long long n, const int32_t* n_dev, int K,
                                      int nchunks, const int32_t* __restrict__ base,
                                      const int32_t* __restrict__ key_offsets, Sink sink) {
-  extern __shared__ int32_t sh[];   // [warps][K]: per-warp counts, then per-warp first rows
+  extern __shared__ int32_t sh[];
+  __shared__ int tmp[32];
+  __shared__ int staged;
   const int nw = blockDim.x >> 5;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x;
-  for (int i = threadIdx.x; i < nw * K; i += blockDim.x) sh[i] = 0;
+  int32_t* cnt = sh;                                   // [nw][K]: counts, then each warp's start in its key's run
+  int32_t* lbase = cnt + static_cast<long long>(nw) * K;   // [K]: first staging slot of each key
+  int32_t* gbase = lbase + K;                          // [K]: first sorted row of each key in this chunk
+  int32_t* skey = gbase + K;                           // [nw * KEYS_PER_WARP]: staged keys, in sorted order
+  int32_t* spa = skey + nw * KEYS_PER_WARP;            // staged payloads
+  int32_t* spb = spa + nw * KEYS_PER_WARP;
+  for (int i = threadIdx.x; i < nw * K; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
   const long long nn = dev_count(n, n_dev);
   const long long b = (static_cast<long long>(chunk) * nw + w) * KEYS_PER_WARP;
-  int32_t* cnt = sh + w * K;
+  int32_t* wcnt = cnt + w * K;
   constexpr int IT = KEYS_PER_WARP / 32;
   int key[IT];
   unsigned peers[IT];
@@ -193,34 +213,65 @@ __global__ void chunk_scatter_kernel(const int32_t* __restrict__ keys, long long
   for (int it = 0; it < IT; ++it) {
     const bool ok = static_cast<unsigned>(key[it]) < static_cast<unsigned>(K);
     peers[it] = __match_any_sync(0xffffffffu, ok ? key[it] : K + lane);
-    if (ok && (peers[it] & ((1u << lane) - 1u)) == 0) cnt[key[it]] += __popc(peers[it]);
+    if (ok && (peers[it] & ((1u << lane) - 1u)) == 0) wcnt[key[it]] += __popc(peers[it]);
     __syncwarp();
   }
   __syncthreads();
-  // exclusive prefix over the warps of this chunk, starting at the chunk's base row of each key
-  if (chunk < nchunks)
-    for (int k = threadIdx.x; k < K; k += blockDim.x) {
-      int run = key_offsets[k] + base[static_cast<long long>(chunk) * K + k];
-      for (int w2 = 0; w2 < nw; ++w2) {
-        const int c = sh[w2 * K + k];
-        sh[w2 * K + k] = run;
-        run += c;
-      }
+  // per key: each warp's start within the key's run of this chunk, the run length, the first row
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+    int run = 0;
+    for (int w2 = 0; w2 < nw; ++w2) {
+      const int c = cnt[w2 * K + k];
+      cnt[w2 * K + k] = run;
+      run += c;
     }
+    lbase[k] = run;
+    gbase[k] = chunk < nchunks ? key_offsets[k] + base[static_cast<long long>(chunk) * K + k] : 0;
+  }
   __syncthreads();
-  // pass 2: rows in key order within the warp
+  // run lengths -> first staging slot of each key (exclusive scan over keys)
+  int carry = 0;
+  for (int k0 = 0; k0 < K; k0 += blockDim.x) {
+    const int k = k0 + threadIdx.x;
+    const int v = k < K ? lbase[k] : 0;
+    int blk;
+    const int ex = block_excl_scan(v, tmp, &blk);
+    if (k < K) lbase[k] = carry + ex;
+    carry += blk;
+  }
+  if (threadIdx.x == 0) staged = carry;
+  __syncthreads();
+  // pass 2: rows in key order within the warp; source-indexed outputs now, the rest staged
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
     const bool ok = static_cast<unsigned>(key[it]) < static_cast<unsigned>(K);
     const int rank = __popc(peers[it] & ((1u << lane) - 1u));
-    const int c0 = ok ? cnt[key[it]] : 0;
+    const int c0 = ok ? wcnt[key[it]] : 0;
     __syncwarp();
-    if (ok && rank == 0) cnt[key[it]] = c0 + __popc(peers[it]);
+    if (ok && rank == 0) wcnt[key[it]] = c0 + __popc(peers[it]);
     __syncwarp();
-    if (ok) sink(b + it * 32 + lane, c0 + rank, key[it]);
+    if (ok) {
+      const long long i = b + it * 32 + lane;
+      const int r = c0 + rank;
+      const int lp = lbase[key[it]] + r;
+      sink.at_source(i, gbase[key[it]] + r);
+      int32_t pa, pb;
+      sink.payload(i, pa, pb);
+      skey[lp] = key[it];
+      spa[lp] = pa;
+      spb[lp] = pb;
+    }
+  }
+  __syncthreads();
+  // write-out in sorted order: consecutive slots of one key are consecutive rows
+  const int nv = staged;
+  for (int lp = threadIdx.x; lp < nv; lp += blockDim.x) {
+    const int k = skey[lp];
+    sink.at_dest(gbase[k] + (lp - lbase[k]), k, spa[lp], spb[lp]);
   }
 }
 
+// PFT: element i = (token i / k, slot i % k) of the t-major assignment list (N < 2^31).
 struct PftSink {
   const float* w;
   int k;
@@ -228,11 +279,15 @@ struct PftSink {
   int32_t* token_ids;
   int32_t* expert_ids;
   float* cw;
-  __device__ void operator()(long long i, int p, int key) const {
-    pos[i] = p;
-    token_ids[p] = static_cast<int32_t>(i / k);
+  __device__ void at_source(long long i, int p) const { pos[i] = p; }
+  __device__ void payload(long long i, int32_t& a, int32_t& b) const {
+    a = static_cast<int32_t>(static_cast<uint32_t>(i) / static_cast<uint32_t>(k));
+    b = __float_as_int(w[i]);
+  }
+  __device__ void at_dest(int p, int key, int32_t a, int32_t b) const {
+    token_ids[p] = a;
     expert_ids[p] = key;
-    cw[p] = w[i];
+    cw[p] = __int_as_float(b);
   }
 };
 
@@ -460,11 +515,15 @@ struct RbdSink {
   int32_t* pilot_node;
   int32_t* rc_sorted;
   int32_t* psorted;
-  __device__ void operator()(long long i, int p, int key) const {
-    pilot_token[p] = ptoken[i];
+  __device__ void at_source(long long i, int p) const { psorted[i] = p; }
+  __device__ void payload(long long i, int32_t& a, int32_t& b) const {
+    a = ptoken[i];
+    b = prc[i];
+  }
+  __device__ void at_dest(int p, int key, int32_t a, int32_t b) const {
+    pilot_token[p] = a;
     pilot_node[p] = key;
-    rc_sorted[p] = prc[i];
-    psorted[i] = p;
+    rc_sorted[p] = b;
   }
 };
 
@@ -524,6 +583,19 @@ int sort_scan(const int32_t* counts, int C, int K, int32_t* totals, int32_t* off
 inline long long long_scan_tiles(long long n_max) { return (n_max + SCAN_TILE - 1) / SCAN_TILE; }
 constexpr long long LONG_SCAN_MIN = 4LL * SCAN_TILE;   // below this one CTA scans the array
 
+// The staged scatter needs up to ~91 KB of shared memory (K = 4096 keys, three warps); opt in once.
+template <class Sink>
+int scatter_smem_attr() {
+  static bool done = false;
+  if (!done) {
+    if (cudaFuncSetAttribute(chunk_scatter_kernel<Sink>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(scatter_smem_bytes(3, 4096) + 4096)) != cudaSuccess)
+      return fail(PFMOE_ERR_CUDA, std::string("cudaFuncSetAttribute failed: ") + cudaGetErrorString(cudaGetLastError()));
+    done = true;
+  }
+  return PFMOE_OK;
+}
+
 }  // namespace
 
 size_t csort_ws_bytes(long long n_max, int K) {
@@ -540,7 +612,8 @@ int pft_build_impl(const int32_t* ids, const float* w, int T, int E, int k, int3
   int32_t* base = counts + static_cast<long long>(C) * E;
   const int wpb = warps_per_block(E);
   const int blocks = C;
-  const size_t sm = static_cast<size_t>(wpb) * E * sizeof(int32_t);
+  const size_t sm = scatter_smem_bytes(wpb, E);
+  PFMOE_TRY(scatter_smem_attr<PftSink>());
   if (C > 0)
     PFMOE_LAUNCH("pft_hist", s,
                  chunk_hist_kernel<<<blocks, wpb * 32, E * sizeof(int32_t), s>>>(ids, N, nullptr, E, C, counts, err));
@@ -600,7 +673,8 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
   PFMOE_RBD_LAUNCH("rbd_emit", rbd_emit_kernel, T, k, s, ids, T, k, E, epd, epn, pbase, pkey, ptoken, prc, err);
   const int wpb = warps_per_block(n_nodes);
   const int blocks = C;
-  const size_t sm = static_cast<size_t>(wpb) * n_nodes * sizeof(int32_t);
+  const size_t sm = scatter_smem_bytes(wpb, n_nodes);
+  PFMOE_TRY(scatter_smem_attr<RbdSink>());
   if (C > 0) {
     PFMOE_LAUNCH("rbd_hist", s,
                  chunk_hist_kernel<<<blocks, wpb * 32, n_nodes * sizeof(int32_t), s>>>(pkey, pmax, counts, n_nodes, C,
