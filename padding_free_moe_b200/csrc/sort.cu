@@ -423,9 +423,11 @@ __device__ __forceinline__ TokView token_view(const int32_t* ids, long long t, b
   v.dev = e / epd;
   int node_before = 0, dev_before = 0, within = 0, same = 0;
   for (int j = 0; j < k; ++j) {
+    // the other lanes' node and device come by shuffle: no division inside the loop
     const int oe = __shfl_sync(0xffffffffu, e, j, G);
+    const int onode = __shfl_sync(0xffffffffu, v.node, j, G);
+    const int odev = __shfl_sync(0xffffffffu, v.dev, j, G);
     const bool earlier = oe < e || (oe == e && j < v.sub);
-    const int onode = oe / epn, odev = oe / epd;
     if (onode == v.node) {
       ++same;
       if (earlier) { ++node_before; ++within; }
