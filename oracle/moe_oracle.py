@@ -17,7 +17,7 @@ Sources (cited by page title and section):
 * [C] Reading notes "【论文】略读笔记90-前沿-可扩展 MoE 训练" (freshwlnd blog),
   sections 需求/创新 (fine-grained experts with large top-k; padding-free training).
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings where the pages are silent:
 
 * Gate: plain linear logits z = x Wg (+ an optional per-expert bias), no noise,
   no temperature.  Selection ranks the logits: descending value, equal values
