@@ -17,6 +17,12 @@ the reported time is the max over ranks.
 
 ``--impl reference`` times the float64 CPU oracle (test infrastructure) on the
 host cores, on bounded token samples of the same workload.
+
+The headline workload is the DeepSeek-V3-like layer (T=8192, d=7168, E=256,
+h=2048, k=8), the largest single-GPU configuration; the DeepSeek-MoE-16B-like,
+skewed DeepSeek-V3-like and fine-grained layers are timed after it and reported
+under ``workloads``.  ``--gpus N`` without a torchrun environment relaunches
+this script under torchrun with N ranks.
 """
 from __future__ import annotations
 
@@ -35,7 +41,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE layer fwd+bwd tokens/s; grouped-GEMM % of BF16 peak; dispatch/combine GB/s"
-DEFAULT_WORKLOAD = "dsmoe16b_bf16"
+DEFAULT_WORKLOAD = "dsv3_bf16"
+EXTRA_WORKLOADS = "dsmoe16b_bf16,dsv3_zipf_bf16,finegrained_bf16"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -48,7 +55,13 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--no-sort-stress", action="store_true", help="skip the PFT / RBD stress-shape timing")
-    ap.add_argument("--cpu-sample-tokens", type=int, default=512)
+    ap.add_argument("--cpu-sample-seconds", type=float, default=12.0,
+                    help="oracle time the cpu_baseline leg spends on token samples")
+    ap.add_argument("--ref-tokens", type=int, default=0,
+                    help="reference arm: tokens per step (0 = sized from the workload)")
+    ap.add_argument("--extra-workloads", default=EXTRA_WORKLOADS,
+                    help="comma-separated workloads timed after the headline one ('' = none)")
+    ap.add_argument("--extra-steps", type=int, default=10)
     return ap.parse_args()
 
 
@@ -162,14 +175,15 @@ def gemm_names():
             "ffn_wgrad_w2"]
 
 
-def traffic_for(kernel):
-    """DRAM bytes per launch from a committed ncu capture, if the kernel source has not changed since."""
+def traffic_for(kernel, workload):
+    """DRAM bytes per launch of `kernel` at `workload` from a committed ncu capture
+    (profiles/traffic.json), if the kernel's source file has not changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         t = json.load(f)
-    ent = t.get(kernel)
+    ent = t.get(workload, {}).get(kernel)
     if not ent:
         return None
     src = os.path.join(ROOT, ent["source"])
@@ -183,19 +197,90 @@ def traffic_for(kernel):
 
 
 # -------------------------------------------------------------- CPU oracle leg
-def oracle_sample(inp_cpu64, cfg, n_tok, seed=0):
-    """Time the float64 oracle's full layer (forward + backward) on n_tok tokens."""
-    import numpy as np
-    import oracle as O
-    rng = np.random.default_rng(seed)
-    toks = np.sort(rng.choice(cfg.T, size=min(n_tok, cfg.T), replace=False))
-    x, wg, bias, w1, w3, w2, dy = inp_cpu64
-    t0 = time.perf_counter()
-    f = O.layer_forward(x[toks], wg, bias, w1, w3, w2, cfg.k)
-    O.layer_backward(f, dy[toks], x[toks], wg, w1, w3, w2)
-    if cfg.has_rbd:
-        O.rbd_plan(f["ids"], cfg.E, cfg.rbd_epd, cfg.rbd_dpn)
-    return len(toks), time.perf_counter() - t0
+class LazyWeights:
+    """Stacked expert weights [E, r, c] (torch, any device) handed to the oracle one expert at a
+    time as float64 numpy: the largest layers' float64 stacks would need tens of GB of host
+    memory.  The conversion time is recorded so that it can be left out of the oracle's time."""
+
+    def __init__(self, t, clock):
+        self.t = t
+        self.shape = tuple(t.shape)
+        self.clock = clock
+
+    def __len__(self):
+        return self.shape[0]
+
+    def __getitem__(self, e):
+        import torch
+        t0 = time.perf_counter()
+        a = self.t[int(e)].detach().to("cpu").to(torch.float64).numpy()
+        self.clock[0] += time.perf_counter() - t0
+        return a
+
+
+class OracleSampler:
+    """The float64 CPU oracle (as it stands) on samples of one workload's tokens.
+
+    One sample = the oracle's gate, routing, PFT, dispatch, expert FFN, combine, the
+    backward of each of those and (with a device map) the RBD plan, on n tokens.  The
+    oracle's own layer_backward keeps weight gradients of all E experts in float64 (30 GB
+    per matrix for the DeepSeek-V3-like layer), so the backward calls its steps directly,
+    one expert at a time, as layer_backward does.  The time reported is the oracle's,
+    without the conversion of the BF16 inputs to float64."""
+
+    def __init__(self, inp, cfg):
+        import torch
+        self.cfg = cfg
+        self.clock = [0.0]
+        cv = lambda t: None if t is None else t.detach().to("cpu").to(torch.float64).numpy()
+        self.x, self.wg, self.bias, self.dy = cv(inp.x), cv(inp.wg), cv(inp.bias), cv(inp.dy)
+        self.w1 = LazyWeights(inp.w1, self.clock)
+        self.w3 = LazyWeights(inp.w3, self.clock)
+        self.w2 = LazyWeights(inp.w2, self.clock)
+
+    def sample(self, n_tok, seed):
+        """(tokens, oracle seconds) of one sample of n_tok random tokens."""
+        import numpy as np
+        import oracle as O
+        cfg = self.cfg
+        rng = np.random.default_rng(seed)
+        toks = np.sort(rng.choice(cfg.T, size=min(n_tok, cfg.T), replace=False))
+        x, dy = self.x[toks], self.dy[toks]
+        self.clock[0] = 0.0
+        t0 = time.perf_counter()
+        f = O.layer_forward(x, self.wg, self.bias, self.w1, self.w3, self.w2, cfg.k)
+        pft = f["pft"]
+        dO, g = O.combine_backward(dy, f["O"], pft["pos"], f["w"])
+        offs = pft["expert_offsets"]
+        dX = np.zeros_like(f["x_pft"])
+        for e in range(cfg.E):
+            r0, r1 = int(offs[e]), int(offs[e + 1])
+            if r1 > r0:
+                gr = O.expert_backward(f["x_pft"][r0:r1], f["H1"][r0:r1], f["H3"][r0:r1], f["A"][r0:r1], dO[r0:r1],
+                                       self.w1[e], self.w3[e], self.w2[e])
+                dX[r0:r1] = gr["dX"]
+        _, _, dx_gate = O.gate_backward(x, self.wg, f["ids"], f["w"], g, cfg.E)
+        O.token_grad(dX, pft["pos"]) + dx_gate
+        if cfg.has_rbd:
+            O.rbd_plan(f["ids"], cfg.E, cfg.rbd_epd, cfg.rbd_dpn)
+        return len(toks), time.perf_counter() - t0 - self.clock[0]
+
+    def tokens_per_second(self, seconds, batch, seed0=0):
+        """Samples of `batch` tokens until the oracle has spent `seconds`: (tokens/s, tokens, seconds)."""
+        tot_n, tot_s, i = 0, 0.0, 0
+        while tot_s < seconds and tot_n < self.cfg.T:
+            n, dt = self.sample(batch, seed0 + i)
+            tot_n += n
+            tot_s += dt
+            i += 1
+        return tot_n / tot_s, tot_n, tot_s
+
+
+def oracle_batch(cfg):
+    """Tokens per oracle sample: about the same oracle work per sample for every workload
+    (a token costs k expert passes over d x h weights)."""
+    per_token = cfg.k * cfg.d * cfg.h
+    return int(max(1, min(256, round(2.0e8 / per_token))))
 
 
 def blas_threads():
@@ -207,41 +292,40 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def inputs_to_cpu64(inp):
-    import torch
-    cv = lambda t: None if t is None else t.detach().to("cpu").to(torch.float64).numpy()
-    return tuple(cv(t) for t in (inp.x, inp.wg, inp.bias, inp.w1, inp.w3, inp.w2, inp.dy))
-
-
 def run_reference(args):
-    """Reference arm: the CPU oracle as it stands, on bounded token samples of the workload."""
+    """Reference arm: the CPU oracle as it stands, on bounded token samples of the workload.
+    The inputs are generated with torch's seeded generator (on the GPU when there is one: the
+    DeepSeek-V3-like weights take minutes to draw on host cores); nothing else uses the GPU."""
     from padding_free_moe_b200 import replicas
     info = replicas.rank_info()
     rank, world = info.rank, info.world
     if rank != 0:
         return 0
+    import torch
     from workloads import get_config, make_inputs
     cfg = get_config(args.workload)
-    inp = make_inputs(cfg, seed=0, device="cpu")
-    cpu = inputs_to_cpu64(inp)
-    n_tok = max(1, min(args.cpu_sample_tokens // 4, cfg.T))
-    for _ in range(args.warmup):
-        oracle_sample(cpu, cfg, n_tok)
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(cfg, seed=0, device=gen_dev)
+    smp = OracleSampler(inp, cfg)
+    n_tok = args.ref_tokens if args.ref_tokens > 0 else oracle_batch(cfg)
+    for i in range(args.warmup):
+        smp.sample(n_tok, 10_000 + i)
     tot_tok, tot_s = 0, 0.0
     for i in range(args.steps):
-        n, s = oracle_sample(cpu, cfg, n_tok, seed=i + 1)
+        n, sec = smp.sample(n_tok, i + 1)
         tot_tok += n
-        tot_s += s
+        tot_s += sec
     value = tot_tok / tot_s
     cores = blas_threads()
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_block(cfg, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"{n_tok} random tokens of {cfg.name} per step through the float64 oracle "
-                                   f"(forward, RBD plan, backward)"},
+                                   f"(forward, RBD plan, backward; expert weights converted to float64 one "
+                                   f"expert at a time, conversion not timed)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -318,13 +402,63 @@ def stress_sort(L, torch, dev, stream, hbm_gbs, reps=20):
     return out
 
 
+def build_layer(cfg, rank, dev):
+    from padding_free_moe_b200.layer import PFTMoELayer, Shape
+    from workloads import make_inputs
+    from workloads.generate import storage_dtype
+    inp = make_inputs(cfg, seed=1000 + rank, device=dev)
+    layer = PFTMoELayer(Shape(cfg.T, cfg.d, cfg.E, cfg.h, cfg.k, storage_dtype(cfg), cfg.rbd_epd, cfg.rbd_dpn), dev)
+    return layer, inp
+
+
+def device_timed(fn, n, stream, torch):
+    """Device milliseconds of n calls of fn() on `stream` (CUDA events on that stream)."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def per_kernel_pass(L, layer, inp, stream, steps, torch, barrier):
+    """The same steps with a CUDA event pair around every kernel launch (on the stream it is
+    launched on): per-kernel durations and launch counts.  The RBD plan runs in line here so
+    that each event pair times one kernel's own work.  Returns (kernels, pass milliseconds)."""
+    L.moe_profile_reset()
+    barrier()
+    torch.cuda.synchronize()
+    L.moe_profile_enable(True)
+    ms = device_timed(lambda: layer.step(inp.x, inp.wg, inp.bias, inp.w1, inp.w3, inp.w2, inp.dy, stream,
+                                         overlap_rbd=False), steps, stream, torch)
+    L.moe_profile_enable(False)
+    barrier()
+    return L.moe_profile_read(), ms
+
+
+def tensor_peak(peaks, peak_src, pass_ms):
+    """The burst GEMM peak for kernels timed in a pass shorter than a second, else the sustained one."""
+    if pass_ms < 1000.0:
+        return float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])), \
+            f"{peak_src} bf16_tflops (burst: the per-kernel pass lasted {pass_ms:.0f} ms)"
+    return float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])), \
+        f"{peak_src} bf16_tflops_sustained (the per-kernel pass lasted {pass_ms:.0f} ms)"
+
+
+def gemm_summary(cfg, kern, steps, tc_peak):
+    gemm_ms = sum(kern[n][1] for n in gemm_names() if n in kern) / steps
+    gemm_flops = 18.0 * cfg.N * cfg.d * cfg.h
+    tf = gemm_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
+    return {"tflops": tf, "frac_of_peak": (tf / tc_peak) if tf else None, "flops_per_step": gemm_flops,
+            "ms_per_step": gemm_ms}
+
+
 def run_ours(args):
     import torch
     from padding_free_moe_b200 import _lib as L
     from padding_free_moe_b200 import replicas
-    from padding_free_moe_b200.layer import PFTMoELayer, Shape
-    from workloads import get_config, make_inputs
-    from workloads.generate import storage_dtype
+    from workloads import get_config
 
     info = replicas.rank_info()
     rank, world, local_rank = info.rank, info.world, info.local_rank
@@ -332,8 +466,7 @@ def run_ours(args):
     dev = torch.device("cuda", local_rank)
     replicas.init(info, "nccl", timeout_s=120, device=dev)
     cfg = get_config(args.workload)
-    inp = make_inputs(cfg, seed=1000 + rank, device=dev)
-    layer = PFTMoELayer(Shape(cfg.T, cfg.d, cfg.E, cfg.h, cfg.k, storage_dtype(cfg), cfg.rbd_epd, cfg.rbd_dpn), dev)
+    layer, inp = build_layer(cfg, rank, dev)
     stream = torch.cuda.current_stream()
 
     def step():
@@ -357,32 +490,13 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize()
     clk.start()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
-    torch.cuda.synchronize()
+    ms_total = device_timed(step, args.steps, stream, torch)
     barrier()
     clocks = clk.stop()
-    ms_total = max_over_ranks(ev0.elapsed_time(ev1))
-    ms_step = ms_total / args.steps
+    ms_step = max_over_ranks(ms_total) / args.steps
     value = world * cfg.T / (ms_step * 1e-3)
 
-    # ---- the same steps again with a CUDA event pair around every kernel launch (on the
-    # stream it is launched on): per-kernel durations for the roofline and launch counts.
-    # Kept out of the headline pass because the events add host-side gaps between kernels;
-    # the RBD plan runs in line here so that each event pair times one kernel's own work.
-    L.moe_profile_reset()
-    barrier()
-    torch.cuda.synchronize()
-    L.moe_profile_enable(True)
-    for _ in range(args.steps):
-        layer.step(inp.x, inp.wg, inp.bias, inp.w1, inp.w3, inp.w2, inp.dy, stream, overlap_rbd=False)
-    torch.cuda.synchronize()
-    L.moe_profile_enable(False)
-    barrier()
-    kern = L.moe_profile_read()
+    kern, pass_ms = per_kernel_pass(L, layer, inp, stream, args.steps, torch, barrier)
 
     # ---- end to end through the public API: every step copies its inputs (x, dY) from pinned
     # host memory and reads its results (y, dx) back to pinned host memory.  Copies run on
@@ -454,11 +568,12 @@ def run_ours(args):
         raise RuntimeError("end-to-end results read back to the host differ from the device results")
     if layer.device_error() != 0:
         raise RuntimeError(f"device error word {layer.device_error():#x}")
+    del x_d, dy_d, y_st, dx_st
 
     # ---- roofline of the dominant kernel + per-kernel table
     peaks, peak_src = load_peaks()
     hbm = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
-    tc_peak = float(peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]))
+    tc_peak, tc_src = tensor_peak(peaks, peak_src, pass_ms)
     kernels = {}
     for nm, (n_launch, ms) in sorted(kern.items(), key=lambda kv: -kv[1][1]):
         per_ms = ms / n_launch
@@ -478,16 +593,13 @@ def run_ours(args):
     if kind == "tensor":
         ach = work / (dom_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": tc_peak, "unit": "TFLOP/s",
-                "frac": ach / tc_peak, "traffic": traffic_for(dom),
-                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
-                "work_per_launch": work}
+                "frac": ach / tc_peak, "traffic": traffic_for(dom, cfg.name), "peak_source": tc_src,
+                "work_per_launch": work, "ms_per_launch": dom_ms}
     else:
         ach = work / (dom_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                "traffic": traffic_for(dom), "peak_source": f"{peak_src} hbm_gbs", "work_per_launch": work}
-    gemm_ms = sum(kern[n][1] for n in gemm_names() if n in kern) / args.steps
-    gemm_flops = 18.0 * cfg.N * cfg.d * cfg.h
-    gemm_tflops = gemm_flops / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
+                "traffic": traffic_for(dom, cfg.name), "peak_source": f"{peak_src} hbm_gbs",
+                "work_per_launch": work, "ms_per_launch": dom_ms}
 
     def gbs(nm):
         return kernels.get(nm, {}).get("gbs")
@@ -502,30 +614,73 @@ def run_ours(args):
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": int(sum(v[0] for v in kern.values())),
         "roofline": roof,
-        "grouped_gemm": {"tflops": gemm_tflops, "pct_of_bf16_peak": (100 * gemm_tflops / tc_peak) if gemm_tflops else None,
-                         "pct_of_burst_peak": (100 * gemm_tflops / float(peaks.get("bf16_tflops", 1590.0)))
-                         if gemm_tflops else None,
-                         "flops_per_step": gemm_flops, "ms_per_step": gemm_ms},
+        "grouped_gemm": gemm_summary(cfg, kern, args.steps, tc_peak),
         "dispatch_gbs": gbs("dispatch"), "combine_gbs": gbs("combine"),
         "sort_stress": None if args.no_sort_stress else stress_sort(L, torch, dev, stream, hbm),
         "kernels": kernels,
     }
 
-    # ---- CPU oracle baseline (rank 0, one GPU only)
+    # ---- CPU oracle baseline (rank 0, one GPU only), on the headline workload's inputs
     if world == 1 and not args.no_cpu_baseline:
-        cpu = inputs_to_cpu64(inp)
-        n, s = oracle_sample(cpu, cfg, args.cpu_sample_tokens)
-        line["cpu_baseline"] = {"value": n / s, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                                "sample": f"{n} random tokens of {cfg.name} through the float64 oracle "
-                                          f"(forward, RBD plan, backward), {s:.1f} s"}
+        smp = OracleSampler(inp, cfg)
+        batch = oracle_batch(cfg)
+        tps, n, sec = smp.tokens_per_second(args.cpu_sample_seconds, batch)
+        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"{n} random tokens of {cfg.name} in samples of {batch} through the "
+                                          f"float64 oracle (forward, RBD plan, backward), {sec:.1f} s of oracle "
+                                          f"time; expert weights converted to float64 one expert at a time, "
+                                          f"conversion not timed"}
+        del smp
+
+    # ---- the other workloads: device-timed steps and their grouped-GEMM rate
+    del layer, inp
+    torch.cuda.empty_cache()
+    extra = {}
+    for name in [w for w in args.extra_workloads.split(",") if w and w != cfg.name]:
+        c2 = get_config(name)
+        lay2, inp2 = build_layer(c2, rank, dev)
+
+        def step2():
+            lay2.step(inp2.x, inp2.wg, inp2.bias, inp2.w1, inp2.w3, inp2.w2, inp2.dy, stream)
+
+        for _ in range(warm):
+            step2()
+        torch.cuda.synchronize()
+        barrier()
+        ms2 = max_over_ranks(device_timed(step2, args.extra_steps, stream, torch)) / args.extra_steps
+        barrier()
+        k2, pass2 = per_kernel_pass(L, lay2, inp2, stream, args.extra_steps, torch, barrier)
+        if lay2.device_error() != 0:
+            raise RuntimeError(f"device error word {lay2.device_error():#x} in {name}")
+        pk, src = tensor_peak(peaks, peak_src, pass2)
+        extra[name] = {"ms_per_step": ms2, "tokens_per_s": world * c2.T / (ms2 * 1e-3), "steps": args.extra_steps,
+                       "grouped_gemm": gemm_summary(c2, k2, args.extra_steps, pk), "peak_source": src,
+                       "config": config_block(c2, world)}
+        del lay2, inp2
+        torch.cuda.empty_cache()
+    line["workloads"] = extra
     if rank == 0:
         print(json.dumps(line), flush=True)
     replicas.finish(info)
     return 0
 
 
+def relaunch_under_torchrun(n: int) -> int:
+    """`--gpus N` from a plain `python bench.py`: run the same command as N torchrun ranks."""
+    import socket
+    sk = socket.socket()
+    sk.bind(("127.0.0.1", 0))
+    port = sk.getsockname()[1]
+    sk.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd, cwd=ROOT)
+
+
 def main():
     args = parse()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch_under_torchrun(args.gpus)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

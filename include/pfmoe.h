@@ -57,7 +57,8 @@ enum {
   PFMOE_DEV_BAD_EXPERT_ID = 1, /* a routed expert id outside [0, E) */
   PFMOE_DEV_BAD_POS = 2,       /* a PFT row index outside [0, T*k) */
   PFMOE_DEV_TIMEOUT = 4,       /* a bounded on-chip wait gave up (the kernel returned early) */
-  PFMOE_DEV_NONFINITE = 8      /* a NaN gate logit was seen (it ranks below every number) */
+  PFMOE_DEV_NONFINITE = 8      /* a NaN gate logit was seen (it ranks below every number), or a
+                                  token's largest logit is +inf or -inf (its weights are undefined) */
 };
 
 /* Rows per grouped-GEMM M tile.  Expert e owns ceil(n_e / PFMOE_TILE_ROWS) tiles. */
@@ -119,7 +120,10 @@ PFMOE_API int pft_build(const int32_t* topk_ids, const float* topk_w, int T, int
  *   PFMOE_PFT_NO_WS_SCRATCH_BYTES (for example T*k up to 260096 with E = 1024, 1046528 with E = 256);
  *   larger shapes return PFMOE_ERR_UNSUPPORTED with a message naming both sizes.
  *   The first call on a device looks up the array's device address (once, with
- *   that device current); make that first call before any stream capture.
+ *   that device current); make that first call before any stream capture (a
+ *   first call on a capturing stream returns PFMOE_ERR_UNSUPPORTED).  The address
+ *   is cached for the life of the process: do not call this entry point on a
+ *   device after cudaDeviceReset of that device.
  *   All calls on a device share the array and it keeps the last call's contents
  *   (nothing has to start at zero); calls that overlap on the GPU race on it.
  */

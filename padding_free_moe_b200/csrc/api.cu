@@ -1,9 +1,12 @@
 // C ABI of libpfmoe: host-side argument checking, workspace layout and the
 // launch sequence of each step.  Every compute step runs in the library's own
 // kernels (gemm_tc.cu, gemm_simt.cu, route.cu, sort.cu, rows.cu).
+#include <atomic>
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <set>
+#include <utility>
 #include <string>
 #include <vector>
 
@@ -29,16 +32,32 @@ int check_launch(const char* what) {
 }
 
 int num_sms() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
-  if (!cached[dev]) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (!n) {
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = n > 0 ? n : 1;
+    n = n > 0 ? n : 1;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
+}
+
+int smem_optin(const void* kernel, int bytes, const char* name) {
+  static std::mutex mu;
+  static std::set<std::pair<int, const void*>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(PFMOE_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  std::lock_guard<std::mutex> lk(mu);
+  if (done.count({dev, kernel})) return PFMOE_OK;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess)
+    return fail(PFMOE_ERR_CUDA, std::string(name) + ": cudaFuncSetAttribute failed: " + cudaGetErrorString(e));
+  done.insert({dev, kernel});
+  return PFMOE_OK;
 }
 
 // ---------------------------------------------------------------- profiler

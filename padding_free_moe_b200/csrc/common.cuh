@@ -24,6 +24,11 @@ int check_launch(const char* what);
 
 int num_sms();
 
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current device.
+// cudaFuncSetAttribute acts on the current device only, so this is done once per
+// (device, kernel) pair; thread-safe.
+int smem_optin(const void* kernel, int bytes, const char* name);
+
 #define PFMOE_TRY(expr)            \
   do {                             \
     int _rc = (expr);              \

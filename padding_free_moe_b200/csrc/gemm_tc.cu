@@ -1516,14 +1516,7 @@ static int launch(Params& p, long long tile_upper_bound, const char* name, cudaS
   p.stages = pick_stages(p.bn, staged, KBK);
   if (p.stages < 2) return fail(PFMOE_ERR_UNSUPPORTED, std::string(name) + ": shared-memory plan needs two stages");
   const size_t smem = smem_bytes(p.bn, p.stages, staged, KBK);
-  static bool attr_done = false;  // per template instance
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(grouped_gemm_kernel<EPI, MODE, KBK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(227 * 1024)) != cudaSuccess)
-      return fail(PFMOE_ERR_CUDA, std::string("cudaFuncSetAttribute failed: ") +
-                                      cudaGetErrorString(cudaGetLastError()));
-    attr_done = true;
-  }
+  PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&grouped_gemm_kernel<EPI, MODE, KBK>), SMEM_LIMIT, name));
   if (tile_upper_bound <= 0) return PFMOE_OK;
   long long grid = num_sms();
   if (tile_upper_bound < grid) grid = tile_upper_bound;
@@ -1534,14 +1527,10 @@ static int launch(Params& p, long long tile_upper_bound, const char* name, cudaS
 }
 
 
-// Two-SM launcher for row-grouped problems.
+// Two-SM launcher for row-grouped problems: one CTA pair per two SMs of the current device.
 static int max_pairs() {
-  static int cached = -1;
-  if (cached < 0) {
-    int n = num_sms() / 2;
-    cached = n > 0 ? n : 1;
-  }
-  return cached;
+  const int n = num_sms() / 2;
+  return n > 0 ? n : 1;
 }
 
 // Token-as-N launcher (expert-segmented rows only).
@@ -1559,14 +1548,7 @@ static int launch_tn(Params& p, long long pair_tile_upper_bound, const char* nam
   if (st < 2) return fail(PFMOE_ERR_UNSUPPORTED, std::string(name) + ": too many experts for the shared-memory plan");
   p.stages = st > MAX_STAGES ? MAX_STAGES : st;
   const size_t smem = fixed + static_cast<size_t>(p.stages) * stage;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(grouped_gemm_tn_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(227 * 1024)) != cudaSuccess)
-      return fail(PFMOE_ERR_CUDA, std::string("cudaFuncSetAttribute failed: ") +
-                                      cudaGetErrorString(cudaGetLastError()));
-    attr_done = true;
-  }
+  PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&grouped_gemm_tn_kernel<EPI>), SMEM_LIMIT, name));
   if (pair_tile_upper_bound <= 0) return PFMOE_OK;
   long long pairs = max_pairs();
   if (pair_tile_upper_bound < pairs) pairs = pair_tile_upper_bound;

@@ -12,7 +12,10 @@
 // address, so the device address is looked up with cudaGetSymbolAddress once
 // per device (with that device current) on the first call made on it, cached,
 // and handed to the kernels.  That first call should therefore come before
-// any stream capture.  Nothing here calls cudaMalloc, cudaFree or any routine
+// any stream capture (a first call on a capturing stream is refused).  The
+// cached address belongs to the device's current context: after
+// cudaDeviceReset the process must not call this entry point on that device
+// again.  Nothing here calls cudaMalloc, cudaFree or any routine
 // that allocates.
 //
 // Every call on a device shares the one array and finds in it whatever the
@@ -36,8 +39,10 @@ __device__ __align__(256) unsigned char g_pft_scratch[PFMOE_PFT_NO_WS_SCRATCH_BY
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_pft_scratch on the current device (looked up once per device).
-int scratch_address(void** out) {
+// Device address of g_pft_scratch on the current device (looked up once per device).  The
+// lookup may load the library's module on the device, which a stream under capture does not
+// allow, so a first call on a capturing stream is refused with a clear message instead.
+int scratch_address(cudaStream_t stream, void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(PFMOE_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
@@ -45,6 +50,13 @@ int scratch_address(void** out) {
     return fail(PFMOE_ERR_UNSUPPORTED, "pft_build_no_ws supports device ordinals below 64");
   std::lock_guard<std::mutex> lk(g_scratch_mu);
   if (!g_scratch_addr[dev]) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(stream, &cs);
+    if (e != cudaSuccess) return fail(PFMOE_ERR_CUDA, std::string("cudaStreamIsCapturing: ") + cudaGetErrorString(e));
+    if (cs != cudaStreamCaptureStatusNone)
+      return fail(PFMOE_ERR_UNSUPPORTED,
+                  "pft_build_no_ws: the first call on a device looks up the built-in scratch array and cannot run "
+                  "during stream capture; make one call on this device before capturing");
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_pft_scratch);
     if (e != cudaSuccess || !p)
@@ -72,7 +84,7 @@ extern "C" int pft_build_no_ws(const int32_t* topk_ids, const float* topk_w, int
                     "array holds " + std::to_string(PFMOE_PFT_NO_WS_SCRATCH_BYTES) +
                     " bytes; use pft_build with a caller workspace");
   void* scratch = nullptr;
-  PFMOE_TRY(scratch_address(&scratch));
+  PFMOE_TRY(scratch_address(static_cast<cudaStream_t>(stream), &scratch));
   return pft_build(topk_ids, topk_w, T, E, k, tokens_per_expert, expert_offsets, token_ids, expert_ids,
                    combine_weights, pos, tile_offsets, scratch, PFMOE_PFT_NO_WS_SCRATCH_BYTES, err, stream);
 }

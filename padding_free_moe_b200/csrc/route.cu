@@ -5,7 +5,8 @@
 // argmax under the order (value descending, index ascending) pick the experts;
 // the weights are the softmax over the picked logits, computed in float32.
 // A NaN logit ranks below every number (including -inf) and raises
-// PFMOE_DEV_NONFINITE.
+// PFMOE_DEV_NONFINITE, as does a token whose largest logit is +inf or -inf
+// (its weights are then undefined).
 #include <climits>
 
 #include "common.cuh"
@@ -82,7 +83,8 @@ __global__ void __launch_bounds__(256) topk_kernel(float* __restrict__ logits, c
       ids[static_cast<long long>(t) * k + lane] = pick_e;
       w[static_cast<long long>(t) * k + lane] = ex / sum;
     }
-    if (__any_sync(0xffffffffu, nan_seen) && lane == 0) dev_error(err, PFMOE_DEV_NONFINITE);
+    // A largest logit of +inf or -inf (every logit -inf or NaN) leaves the weights undefined.
+    if ((__any_sync(0xffffffffu, nan_seen) || !isfinite(m)) && lane == 0) dev_error(err, PFMOE_DEV_NONFINITE);
   }
 }
 

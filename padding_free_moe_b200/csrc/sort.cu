@@ -585,17 +585,12 @@ int sort_scan(const int32_t* counts, int C, int K, int32_t* totals, int32_t* off
 inline long long long_scan_tiles(long long n_max) { return (n_max + SCAN_TILE - 1) / SCAN_TILE; }
 constexpr long long LONG_SCAN_MIN = 4LL * SCAN_TILE;   // below this one CTA scans the array
 
-// The staged scatter needs up to ~91 KB of shared memory (K = 4096 keys, three warps); opt in once.
+// The staged scatter needs up to ~91 KB of shared memory (K = 4096 keys, three warps): opt in
+// once per device.
 template <class Sink>
 int scatter_smem_attr() {
-  static bool done = false;
-  if (!done) {
-    if (cudaFuncSetAttribute(chunk_scatter_kernel<Sink>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(scatter_smem_bytes(3, 4096) + 4096)) != cudaSuccess)
-      return fail(PFMOE_ERR_CUDA, std::string("cudaFuncSetAttribute failed: ") + cudaGetErrorString(cudaGetLastError()));
-    done = true;
-  }
-  return PFMOE_OK;
+  return smem_optin(reinterpret_cast<const void*>(&chunk_scatter_kernel<Sink>),
+                    static_cast<int>(scatter_smem_bytes(3, 4096) + 4096), "chunk_scatter");
 }
 
 }  // namespace

@@ -78,3 +78,45 @@ def check_index_parity(layer: PFTMoELayer, cfg, O):
         assert np.array_equal(i64(layer.replica_expert[:N]), r["replica_expert"])
         assert np.array_equal(i64(layer.assign_pilot), r["assign_pilot"])
     return ids, w
+
+
+class LazyExperts:
+    """Stacked expert weights [E, r, c] kept on the GPU and handed to the oracle one
+    expert at a time as float64 (a full-size stack would need tens of GB of host
+    memory in float64).  The oracle only ever indexes experts that own rows."""
+
+    def __init__(self, t):
+        self.t = t
+        self.shape = tuple(t.shape)
+
+    def __len__(self):
+        return self.shape[0]
+
+    def __getitem__(self, e):
+        return f64(self.t[int(e)])
+
+
+def sampled_layer(O, S, z_gpu, x, wg, w1, w3, w2, dy, k):
+    """The oracle's layer, forward and backward, on the token subset S (tokens are
+    independent in y, dx and dlogits; dWg over S is complete in every column whose
+    routed tokens all lie in S).  Routing uses the GPU's logits, which the tests
+    compare with the oracle's separately.  The backward repeats the oracle's
+    layer_backward step by step, but keeps only dX of each expert: its weight
+    gradients over all E experts would not fit in host memory at full size.
+    w1, w3, w2 are LazyExperts (or arrays); x, wg, dy are float64 arrays."""
+    S = np.asarray(S)
+    xs, dys = x[S], dy[S]
+    fwd = O.layer_forward(xs, wg, None, w1, w3, w2, k, logits=z_gpu[S])
+    pft = fwd["pft"]
+    dO, g = O.combine_backward(dys, fwd["O"], pft["pos"], fwd["w"])
+    offs = pft["expert_offsets"]
+    dX = np.zeros_like(fwd["x_pft"])
+    for e in range(len(offs) - 1):
+        r0, r1 = int(offs[e]), int(offs[e + 1])
+        if r1 > r0:
+            gr = O.expert_backward(fwd["x_pft"][r0:r1], fwd["H1"][r0:r1], fwd["H3"][r0:r1], fwd["A"][r0:r1],
+                                   dO[r0:r1], w1[e], w3[e], w2[e])
+            dX[r0:r1] = gr["dX"]
+    dz, dWg, dx_gate = O.gate_backward(xs, wg, fwd["ids"], fwd["w"], g, wg.shape[1])
+    dx = O.token_grad(dX, pft["pos"]) + dx_gate
+    return {"y": fwd["y"], "dx": dx, "dlogits": dz, "dWg": dWg, "ids": fwd["ids"]}

@@ -1,5 +1,6 @@
 """The bench's reference arm (the float64 oracle on host cores): its JSON line keeps the bench
-contract, and under a multi-rank launch only rank 0 prints."""
+contract, and under a multi-rank launch only rank 0 prints.  `--gpus N` without a torchrun
+environment relaunches the bench as N torchrun ranks (the same path the GPU arm takes)."""
 import json
 import os
 import subprocess
@@ -8,10 +9,12 @@ import sys
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _run(extra_env):
+def _run(extra_env, extra_args=(), drop=()):
     env = dict(os.environ, **extra_env)
+    for k in drop:
+        env.pop(k, None)
     cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny_fp32",
-           "--steps", "2", "--warmup", "1", "--cpu-sample-tokens", "16"]
+           "--steps", "2", "--warmup", "1", "--ref-tokens", "16", *extra_args]
     return subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
 
 
@@ -36,3 +39,12 @@ def test_reference_arm_other_ranks_exit_quietly():
     r = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert not [l for l in r.stdout.splitlines() if l.startswith("{")]
+
+
+def test_gpus_flag_relaunches_as_n_ranks():
+    r = _run({}, extra_args=("--gpus", "2"), drop=("RANK", "WORLD_SIZE", "LOCAL_RANK"))
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["config"]["global_batch"] == 2 * line["config"]["T"]

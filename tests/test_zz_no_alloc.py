@@ -37,9 +37,12 @@ def _run(fn, ids, w, T, E, k, *ws):
 @pytest.mark.gpu
 def test_pft_build_no_ws_matches_pft_build_twice():
     L.lib()
-    # Two calls in a row with different shapes and routings: the second call sees the
-    # first call's leftovers in the built-in scratch array.
-    for T, E, k, seed in ((4096, 64, 6, 11), (1500, 256, 8, 12)):
+    # Calls in a row with different shapes and routings: each call sees the previous call's
+    # leftovers in the built-in scratch array.  The second and fourth shapes have more than 64
+    # chunks of keys, so their chunk counts are scanned per key (the many-chunk path, which
+    # also uses the key-total region of the array), and the fourth runs over the first three's
+    # leftovers in every region it uses.
+    for T, E, k, seed in ((4096, 64, 6, 11), (20000, 1024, 8, 13), (1500, 256, 8, 12), (32768, 256, 8, 14)):
         assert L.pft_build_workspace_size(T, E, k) <= L.PFT_NO_WS_SCRATCH_BYTES
         ids = make_topk_ids(T, E, k, seed=seed, device="cuda")
         w = torch.rand(T, k, device="cuda")
