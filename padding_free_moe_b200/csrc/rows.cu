@@ -1,11 +1,15 @@
 // Row-movement kernels of the padding-free layer: dispatch (PFT.x), combine,
 // combine backward, token-gradient gather-sum with the gate's backward, and a
-// small transpose.  All are HBM-bound and move rows with 16-byte vector
-// loads/stores, so every warp access is a coalesced 512-byte run of one row
-// (BF16).  Dispatch gives a warp one token; the gather-sums give a warp one
-// (token, column chunk) or one PFT row, which keeps many more row loads in
-// flight.  Nothing uses atomics; every sum runs over the k slots in slot
-// order, so results are deterministic.
+// small transpose.  All are HBM-bound.
+//
+// Dispatch and combine move rows through shared memory with 1-D bulk copies
+// (cp.async.bulk, the copy engine of each SM): dispatch loads a piece of a token
+// row once and stores it to the token's k PFT rows straight from shared memory;
+// combine loads the k PFT row pieces of a token into a ring stage and sums them
+// there.  The other kernels move rows with 16-byte vector loads/stores, one warp
+// per (token, column chunk) or PFT row, so every warp access is a coalesced
+// 512-byte run of one row (BF16).  Nothing uses atomics on data; every sum runs
+// over the k slots in slot order, so results are deterministic.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -36,36 +40,237 @@ __device__ __forceinline__ bool load_pos(const int32_t* pos, long long t, int k,
   return true;
 }
 
-// X-MoE article §2.1.2: PFT row r holds token row token_ids[r].  Computed token-major:
-// x[t] is read once and written to its k rows pos[t, j].
-template <typename T, int U>
-__global__ void __launch_bounds__(WARPS * 32) dispatch_kernel(const T* __restrict__ x, const int32_t* __restrict__ pos,
-                                                              int Tn, int k, int d, T* __restrict__ xp, int32_t* err) {
-  constexpr int VN = Vec<T>::n;
-  const int lane = threadIdx.x & 31;
-  const int nw = (gridDim.x * blockDim.x) >> 5;
+// --------------------------------------------------------------- bulk copies
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void bar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void bar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool bar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait (2 s of %globaltimer): false, with PFMOE_DEV_TIMEOUT set, if it gave up.
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, int32_t* err) {
+  if (bar_try(bar, parity)) return true;
+  unsigned long long t0;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  while (true) {
+    if (bar_try(bar, parity)) return true;
+    unsigned long long t1;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
+    if (t1 - t0 > 2000000000ull) {
+      dev_error(err, PFMOE_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+// global -> shared, completing on an mbarrier (both addresses 16-byte aligned, bytes a multiple of 16)
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+// shared -> global, tracked by the issuing thread's bulk groups
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
+               "r"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// X-MoE article §2.1.2: PFT row r holds token row token_ids[r].  Computed token-major with bulk
+// copies: one warp per CTA; lane 0 loads a piece of x[t] into a ring buffer and, once it has
+// landed, stores it to the token's k rows pos[t, j] straight from shared memory.  Work items are
+// (token, piece) pairs; DP_BUFS - 1 loads stay in flight, and a buffer is reloaded once the
+// stores that read it have read it.
+constexpr int DP_BUFS = 4;
+
+__global__ void __launch_bounds__(32) dispatch_bulk_kernel(const char* __restrict__ x, const int32_t* __restrict__ pos,
+                                                           int Tn, int k, int row_bytes, int piece_bytes, int pieces,
+                                                           char* __restrict__ xp, int32_t* err) {
+  extern __shared__ __align__(128) uint8_t dsm[];
+  __shared__ __align__(8) uint64_t bar[DP_BUFS];
+  const int lane = threadIdx.x;
   const long long N = static_cast<long long>(Tn) * k;
-  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < Tn; t += nw) {
-    int my_pos;
-    if (!load_pos(pos, t, k, N, lane, my_pos, err)) continue;
-    const T* src = x + static_cast<long long>(t) * d;
-    for (int base = 0; base < d; base += 32 * VN * U) {   // warp-uniform trip count
-      const int c0 = base + lane * VN;
-      uint4 v[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int c = c0 + u * 32 * VN;
-        if (c < d) v[u] = __ldg(reinterpret_cast<const uint4*>(src + c));
+  const long long items = static_cast<long long>(Tn) * pieces;
+  const long long first = blockIdx.x, stride = gridDim.x;
+  if (first >= items) return;
+  const long long n_my = (items - first + stride - 1) / stride;
+  if (lane == 0) {
+    for (int b = 0; b < DP_BUFS; ++b) bar_init(smem_addr(&bar[b]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  const uint32_t buf0 = smem_addr(dsm);
+  auto piece_of = [&](long long i, long long& t, int& off, int& bytes) {
+    const long long it = first + i * stride;
+    t = it / pieces;
+    const int c = static_cast<int>(it - t * pieces);
+    off = c * piece_bytes;
+    bytes = min(piece_bytes, row_bytes - off);
+  };
+  auto issue_load = [&](long long i) {
+    long long t;
+    int off, bytes;
+    piece_of(i, t, off, bytes);
+    const int b = static_cast<int>(i % DP_BUFS);
+    const uint32_t bb = smem_addr(&bar[b]);
+    bar_expect_tx(bb, bytes);
+    bulk_load(buf0 + b * piece_bytes, x + t * row_bytes + off, bytes, bb);
+  };
+  if (lane == 0)
+    for (long long i = 0; i < DP_BUFS - 1 && i < n_my; ++i) issue_load(i);
+  bool ok = true;
+  long long i = 0;
+  for (; i < n_my && ok; ++i) {
+    long long t;
+    int off, bytes;
+    piece_of(i, t, off, bytes);
+    int my_pos = lane < k ? pos[t * k + lane] : 0;
+    const bool bad = lane < k && (my_pos < 0 || my_pos >= N);
+    const bool any_bad = __any_sync(0xffffffffu, bad);
+    if (any_bad && lane == 0 && off == 0) dev_error(err, PFMOE_DEV_BAD_POS);
+    const int b = static_cast<int>(i % DP_BUFS);
+    ok = __all_sync(0xffffffffu, bar_wait(smem_addr(&bar[b]), static_cast<uint32_t>(i / DP_BUFS) & 1, err));
+    if (!ok) break;
+    for (int j = 0; j < k; ++j) {
+      const long long pj = __shfl_sync(0xffffffffu, my_pos, j);
+      if (lane == 0 && !any_bad) bulk_store(xp + pj * row_bytes + off, buf0 + b * piece_bytes, bytes);
+    }
+    if (lane == 0) {
+      bulk_commit();
+      // the next load goes into the buffer item i - 1 used: its stores (the group before this
+      // one) must have read it
+      if (i + DP_BUFS - 1 < n_my) {
+        bulk_wait_read<1>();
+        issue_load(i + DP_BUFS - 1);
+      }
+    }
+    __syncwarp();
+  }
+  if (lane == 0) {
+    // loads still in flight (after an abort) land before the CTA exits; stores complete
+    for (long long r = i; r < n_my && r < i + DP_BUFS - 1; ++r)
+      bar_wait(smem_addr(&bar[r % DP_BUFS]), static_cast<uint32_t>(r / DP_BUFS) & 1, err);
+    bulk_wait_all();
+  }
+  __syncwarp();
+}
+
+// y[t] = sum_j w[t, j] * O[pos[t, j]] ([A] §2.1.1 combine_weights), with bulk copies: warp 0's
+// lane 0 loads the k PFT row pieces (CB_PIECE bytes each) of a work item (token, piece) into a
+// ring stage; four consumer warps sum the stage in slot order in float32 (one 16-byte vector a
+// thread) and store the piece of y.  A token with an out-of-range row index is flagged and its
+// output row is left unwritten.
+constexpr int CB_PIECE = 2048;
+constexpr int CB_CONSUMERS = 128;
+
+template <typename T>
+__global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const char* __restrict__ O,
+                                                                         const int32_t* __restrict__ pos,
+                                                                         const float* __restrict__ w, int Tn, int k,
+                                                                         int row_bytes, int pieces, int stages,
+                                                                         char* __restrict__ y, int32_t* err) {
+  constexpr int VN = Vec<T>::n;
+  extern __shared__ __align__(128) uint8_t csm[];
+  __shared__ __align__(8) uint64_t full[8];
+  __shared__ __align__(8) uint64_t empty[8];
+  __shared__ int valid[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long N = static_cast<long long>(Tn) * k;
+  const long long items = static_cast<long long>(Tn) * pieces;
+  const uint32_t stage_bytes = static_cast<uint32_t>(k) * CB_PIECE;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      bar_init(smem_addr(&full[s]), 1);
+      bar_init(smem_addr(&empty[s]), CB_CONSUMERS);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  const uint32_t st0 = smem_addr(csm);
+  if (warp == 0) {
+    // ---- producer
+    uint32_t pending = 0, pend_parity = 0;
+    int q = 0;
+    for (long long it = blockIdx.x; it < items; it += gridDim.x, ++q) {
+      const long long t = it / pieces;
+      const int off = static_cast<int>(it - t * pieces) * CB_PIECE;
+      const int bytes = min(CB_PIECE, row_bytes - off);
+      const int s = q % stages;
+      const uint32_t ph = (q / stages) & 1;
+      if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&empty[s]), ph ^ 1, err))) break;
+      const int my_pos = lane < k ? pos[t * k + lane] : 0;
+      const bool bad = lane < k && (my_pos < 0 || my_pos >= N);
+      const bool any_bad = __any_sync(0xffffffffu, bad);
+      if (lane == 0) {
+        valid[s] = any_bad ? 0 : 1;
+        if (any_bad && off == 0) dev_error(err, PFMOE_DEV_BAD_POS);
+      }
+      if (any_bad) {
+        if (lane == 0) bar_arrive(smem_addr(&full[s]));
+        __syncwarp();
+        continue;
+      }
+      const uint32_t fb = smem_addr(&full[s]);
+      if (lane == 0) {
+        bar_expect_tx(fb, static_cast<uint32_t>(k * bytes));
+        pending |= 1u << s;
+        pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
       }
       for (int j = 0; j < k; ++j) {
-        const long long p = __shfl_sync(0xffffffffu, my_pos, j);
-        T* dst = xp + p * d;
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int c = c0 + u * 32 * VN;
-          if (c < d) *reinterpret_cast<uint4*>(dst + c) = v[u];
-        }
+        const long long pj = __shfl_sync(0xffffffffu, my_pos, j);
+        if (lane == 0) bulk_load(st0 + s * stage_bytes + j * CB_PIECE, O + pj * row_bytes + off, bytes, fb);
       }
+      __syncwarp();
+    }
+    if (lane == 0)
+      for (int s = 0; s < stages; ++s)
+        if (pending & (1u << s)) bar_wait(smem_addr(&full[s]), (pend_parity >> s) & 1, err);
+    __syncwarp();
+  } else {
+    // ---- consumers: thread c sums bytes [16 c, 16 c + 16) of the piece
+    const int c = threadIdx.x - 32;
+    int q = 0;
+    for (long long it = blockIdx.x; it < items; it += gridDim.x, ++q) {
+      const long long t = it / pieces;
+      const int off = static_cast<int>(it - t * pieces) * CB_PIECE;
+      const int bytes = min(CB_PIECE, row_bytes - off);
+      const int s = q % stages;
+      if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&full[s]), (q / stages) & 1, err))) break;
+      if (valid[s] && c * 16 < bytes) {
+        float acc[VN];
+#pragma unroll
+        for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+        const uint8_t* sp = csm + s * stage_bytes + c * 16;
+        for (int j = 0; j < k; ++j) {
+          const float wj = __ldg(w + t * k + j);
+          float o[VN];
+          load16(reinterpret_cast<const T*>(sp + j * CB_PIECE), o);
+#pragma unroll
+          for (int i = 0; i < VN; ++i) acc[i] = fmaf(wj, o[i], acc[i]);
+        }
+        store16(reinterpret_cast<T*>(y + t * row_bytes + off + c * 16), acc);
+      }
+      bar_arrive(smem_addr(&empty[s]));
     }
   }
 }
@@ -82,51 +287,6 @@ __host__ __device__ inline int chunk_cols() { return 32 * Vec<T>::n; }
 __host__ __device__ inline int items_per_token(int d, int vn, int U) {
   const int C = (d + 32 * vn - 1) / (32 * vn);
   return (C + U - 1) / U;
-}
-
-// y[t] = sum_j w[t, j] * O[pos[t, j]].  An item covers U consecutive column chunks.
-template <typename T, int U>
-__global__ void __launch_bounds__(WARPS * 32) combine_kernel(const T* __restrict__ O, const int32_t* __restrict__ pos,
-                                                             const float* __restrict__ w, int Tn, int k, int d,
-                                                             T* __restrict__ y, int32_t* err) {
-  constexpr int VN = Vec<T>::n;
-  const int lane = threadIdx.x & 31;
-  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  const long long N = static_cast<long long>(Tn) * k;
-  const int CU = items_per_token(d, VN, U);
-  const long long items = static_cast<long long>(Tn) * CU;
-  for (long long it = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; it < items; it += nw) {
-    const long long t = it / CU;
-    const int cb = static_cast<int>(it - t * CU) * U * chunk_cols<T>() + lane * VN;
-    int my_pos;
-    if (!load_pos(pos, t, k, N, lane, my_pos, err)) continue;
-    const float my_w = lane < k ? w[t * k + lane] : 0.f;
-    float acc[U][VN];
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-#pragma unroll
-      for (int i = 0; i < VN; ++i) acc[u][i] = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < k; ++j) {
-      const long long p = __shfl_sync(0xffffffffu, my_pos, j);
-      const float wj = __shfl_sync(0xffffffffu, my_w, j);
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int c0 = cb + u * chunk_cols<T>();
-        if (c0 < d) {
-          float o[VN];
-          load16(O + p * d + c0, o);
-#pragma unroll
-          for (int i = 0; i < VN; ++i) acc[u][i] = fmaf(wj, o[i], acc[u][i]);
-        }
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int c0 = cb + u * chunk_cols<T>();
-      if (c0 < d) store16(y + t * d + c0, acc[u]);
-    }
-  }
 }
 
 // One warp per PFT row r = (t, j): dO[pos[t, j]] = w[t, j] * dY[t];  g[t, j] = <dY[t], O[pos[t, j]]>.
@@ -278,16 +438,18 @@ __global__ void transpose_kernel(const T* __restrict__ in, int rows, int cols, T
 
 int launch_dispatch(const void* x, const int32_t* pos, int T, int k, int d, int dtype, void* x_pft, int32_t* err,
                     cudaStream_t s) {
-  const int g = token_grid(T);
-  if (dtype == PFMOE_BF16) {
-    PFMOE_LAUNCH("dispatch", s,
-                 (dispatch_kernel<__nv_bfloat16, 4><<<g, WARPS * 32, 0, s>>>(
-                     static_cast<const __nv_bfloat16*>(x), pos, T, k, d, static_cast<__nv_bfloat16*>(x_pft), err)));
-  } else {
-    PFMOE_LAUNCH("dispatch", s,
-                 (dispatch_kernel<float, 4><<<g, WARPS * 32, 0, s>>>(static_cast<const float*>(x), pos, T, k, d,
-                                                                     static_cast<float*>(x_pft), err)));
-  }
+  const int row_bytes = d * (dtype == PFMOE_BF16 ? 2 : 4);
+  // pieces of at most 8 KB (multiples of 16 bytes), as even as the row allows
+  const int pieces = (row_bytes + 8191) / 8192;
+  const int piece_bytes = ((row_bytes + pieces - 1) / pieces + 15) & ~15;
+  const long long items = static_cast<long long>(T) * pieces;
+  long long grid = static_cast<long long>(num_sms()) * 8;
+  if (grid > items) grid = items;
+  const size_t smem = static_cast<size_t>(DP_BUFS) * piece_bytes;
+  PFMOE_LAUNCH("dispatch", s,
+               (dispatch_bulk_kernel<<<static_cast<int>(grid), 32, smem, s>>>(
+                   static_cast<const char*>(x), pos, T, k, row_bytes, piece_bytes, pieces, static_cast<char*>(x_pft),
+                   err)));
   return PFMOE_OK;
 }
 
@@ -297,19 +459,28 @@ static int chunks_per_item(int d, int vn) { return (d + 32 * vn - 1) / (32 * vn)
 
 int launch_combine(const void* out, const int32_t* pos, const float* w, int T, int k, int d, int dtype, void* y,
                    int32_t* err, cudaStream_t s) {
-  const int vn = dtype == PFMOE_BF16 ? 8 : 4;
-  const int U = chunks_per_item(d, vn);
-  const int g = item_grid(static_cast<long long>(T) * items_per_token(d, vn, U));
+  const int row_bytes = d * (dtype == PFMOE_BF16 ? 2 : 4);
+  const int pieces = (row_bytes + CB_PIECE - 1) / CB_PIECE;
+  const int stage_bytes = k * CB_PIECE;
+  int stages = (96 * 1024) / stage_bytes;   // about 96 KB of stages: two CTAs per SM
+  if (stages > 8) stages = 8;
+  if (stages < 2) stages = 2;
+  const size_t smem = static_cast<size_t>(stages) * stage_bytes;
+  const long long items = static_cast<long long>(T) * pieces;
+  long long grid = static_cast<long long>(num_sms()) * 2;
+  if (grid > items) grid = items;
   if (dtype == PFMOE_BF16) {
-    const auto* o = static_cast<const __nv_bfloat16*>(out);
-    auto* yy = static_cast<__nv_bfloat16*>(y);
-    if (U == 4) PFMOE_LAUNCH("combine", s, (combine_kernel<__nv_bfloat16, 4><<<g, WARPS * 32, 0, s>>>(o, pos, w, T, k, d, yy, err)));
-    else PFMOE_LAUNCH("combine", s, (combine_kernel<__nv_bfloat16, 1><<<g, WARPS * 32, 0, s>>>(o, pos, w, T, k, d, yy, err)));
+    PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&combine_bulk_kernel<__nv_bfloat16>), 227 * 1024, "combine"));
+    PFMOE_LAUNCH("combine", s,
+                 (combine_bulk_kernel<__nv_bfloat16><<<static_cast<int>(grid), 32 + CB_CONSUMERS, smem, s>>>(
+                     static_cast<const char*>(out), pos, w, T, k, row_bytes, pieces, stages, static_cast<char*>(y),
+                     err)));
   } else {
-    const auto* o = static_cast<const float*>(out);
-    auto* yy = static_cast<float*>(y);
-    if (U == 4) PFMOE_LAUNCH("combine", s, (combine_kernel<float, 4><<<g, WARPS * 32, 0, s>>>(o, pos, w, T, k, d, yy, err)));
-    else PFMOE_LAUNCH("combine", s, (combine_kernel<float, 1><<<g, WARPS * 32, 0, s>>>(o, pos, w, T, k, d, yy, err)));
+    PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&combine_bulk_kernel<float>), 227 * 1024, "combine"));
+    PFMOE_LAUNCH("combine", s,
+                 (combine_bulk_kernel<float><<<static_cast<int>(grid), 32 + CB_CONSUMERS, smem, s>>>(
+                     static_cast<const char*>(out), pos, w, T, k, row_bytes, pieces, stages, static_cast<char*>(y),
+                     err)));
   }
   return PFMOE_OK;
 }

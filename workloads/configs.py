@@ -92,12 +92,21 @@ SMALL = {
 }
 
 
+# Profiling shapes: slices of a full layer with the same d, h and rows per expert but fewer
+# experts, so that a multi-pass ncu capture holds a few GB on the device instead of ~50 GB.
+# Per-launch traffic scales with the number of experts (each expert's rows, weights and
+# weight gradients are distinct).
+PROFILE = {
+    "dsv3_slice_bf16": LayerConfig("dsv3_slice_bf16", T=512, d=7168, E=16, h=2048, k=8, dtype="bf16",
+                                   note="1/16 of the DeepSeek-V3-like layer: 16 experts, ~256 rows each"),
+}
+
+
 def get_config(name: str) -> LayerConfig:
-    if name in CONFIGS:
-        return CONFIGS[name]
-    if name in SMALL:
-        return SMALL[name]
-    raise KeyError(f"unknown layer config {name!r}; known: {sorted(CONFIGS) + sorted(SMALL)}")
+    for table in (CONFIGS, SMALL, PROFILE):
+        if name in table:
+            return table[name]
+    raise KeyError(f"unknown layer config {name!r}; known: {sorted(CONFIGS) + sorted(SMALL) + sorted(PROFILE)}")
 
 
 def small_configs():
