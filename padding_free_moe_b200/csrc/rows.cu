@@ -16,30 +16,6 @@
 namespace pfmoe {
 namespace {
 
-constexpr int WARPS = 8;   // warps per block
-
-inline int token_grid(long long T) {
-  long long b = (T + WARPS - 1) / WARPS;
-  const long long cap = static_cast<long long>(num_sms()) * 16;
-  if (b > cap) b = cap;
-  return static_cast<int>(b < 1 ? 1 : b);
-}
-
-// Grid for `items` one-warp work items (grid-stride beyond 16 blocks of 8 warps per SM).
-inline int item_grid(long long items) { return token_grid(items); }
-
-// Lane j < k loads pos[t, j]; returns false (and flags) if any row index is out of range.
-__device__ __forceinline__ bool load_pos(const int32_t* pos, long long t, int k, long long N, int lane, int& my_pos,
-                                         int32_t* err) {
-  my_pos = lane < k ? pos[t * k + lane] : 0;
-  const bool bad = lane < k && (my_pos < 0 || my_pos >= N);
-  if (__any_sync(0xffffffffu, bad)) {
-    if (lane == 0) dev_error(err, PFMOE_DEV_BAD_POS);
-    return false;
-  }
-  return true;
-}
-
 // --------------------------------------------------------------- bulk copies
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -180,15 +156,16 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(const char* __restric
 // ring stage; four consumer warps sum the stage in slot order in float32 (one 16-byte vector a
 // thread) and store the piece of y.  A token with an out-of-range row index is flagged and its
 // output row is left unwritten.
-constexpr int CB_PIECE = 2048;
+constexpr int CB_PIECE = 2048;   // largest row piece a ring stage holds per slot: 128 threads x 16 bytes
 constexpr int CB_CONSUMERS = 128;
 
 template <typename T>
 __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const char* __restrict__ O,
                                                                          const int32_t* __restrict__ pos,
                                                                          const float* __restrict__ w, int Tn, int k,
-                                                                         int row_bytes, int pieces, int stages,
-                                                                         char* __restrict__ y, int32_t* err) {
+                                                                         int row_bytes, int piece, int pieces,
+                                                                         int stages, char* __restrict__ y,
+                                                                         int32_t* err) {
   constexpr int VN = Vec<T>::n;
   extern __shared__ __align__(128) uint8_t csm[];
   __shared__ __align__(8) uint64_t full[8];
@@ -197,7 +174,7 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long N = static_cast<long long>(Tn) * k;
   const long long items = static_cast<long long>(Tn) * pieces;
-  const uint32_t stage_bytes = static_cast<uint32_t>(k) * CB_PIECE;
+  const uint32_t stage_bytes = static_cast<uint32_t>(k) * piece;
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       bar_init(smem_addr(&full[s]), 1);
@@ -213,8 +190,8 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const c
     int q = 0;
     for (long long it = blockIdx.x; it < items; it += gridDim.x, ++q) {
       const long long t = it / pieces;
-      const int off = static_cast<int>(it - t * pieces) * CB_PIECE;
-      const int bytes = min(CB_PIECE, row_bytes - off);
+      const int off = static_cast<int>(it - t * pieces) * piece;
+      const int bytes = min(piece, row_bytes - off);
       const int s = q % stages;
       const uint32_t ph = (q / stages) & 1;
       if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&empty[s]), ph ^ 1, err))) break;
@@ -238,7 +215,7 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const c
       }
       for (int j = 0; j < k; ++j) {
         const long long pj = __shfl_sync(0xffffffffu, my_pos, j);
-        if (lane == 0) bulk_load(st0 + s * stage_bytes + j * CB_PIECE, O + pj * row_bytes + off, bytes, fb);
+        if (lane == 0) bulk_load(st0 + s * stage_bytes + j * piece, O + pj * row_bytes + off, bytes, fb);
       }
       __syncwarp();
     }
@@ -252,8 +229,8 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const c
     int q = 0;
     for (long long it = blockIdx.x; it < items; it += gridDim.x, ++q) {
       const long long t = it / pieces;
-      const int off = static_cast<int>(it - t * pieces) * CB_PIECE;
-      const int bytes = min(CB_PIECE, row_bytes - off);
+      const int off = static_cast<int>(it - t * pieces) * piece;
+      const int bytes = min(piece, row_bytes - off);
       const int s = q % stages;
       if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&full[s]), (q / stages) & 1, err))) break;
       if (valid[s] && c * 16 < bytes) {
@@ -264,7 +241,7 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const c
         for (int j = 0; j < k; ++j) {
           const float wj = __ldg(w + t * k + j);
           float o[VN];
-          load16(reinterpret_cast<const T*>(sp + j * CB_PIECE), o);
+          load16(reinterpret_cast<const T*>(sp + j * piece), o);
 #pragma unroll
           for (int i = 0; i < VN; ++i) acc[i] = fmaf(wj, o[i], acc[i]);
         }
@@ -275,145 +252,276 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const c
   }
 }
 
-// The gather-sum kernels below take one work item per warp: a (token, column chunk) pair, the
-// chunk being the 32 * VN columns one warp covers with one 16-byte vector per lane.  Every lane
-// then has all k row loads of its chunk in flight at once, and a token's chunks sit on
-// neighbouring warps (its pos / weight rows stay in L1).  Sums still run over the k slots in
-// slot order with float32 accumulation, so results do not depend on the launch shape.
-template <typename T>
-__host__ __device__ inline int chunk_cols() { return 32 * Vec<T>::n; }
-
-// Items per token when each item covers U column chunks.
-__host__ __device__ inline int items_per_token(int d, int vn, int U) {
-  const int C = (d + 32 * vn - 1) / (32 * vn);
-  return (C + U - 1) / U;
+// The two backward gather kernels below use the same producer / consumer ring as combine: warp 0
+// loads a work item's row pieces (piece bytes each) with bulk copies into a stage and posts the
+// item's per-slot scalars there; four consumer warps (CB_CONSUMERS threads, one 16-byte vector
+// each) read the stage.  KM >= k bounds the per-thread slot arrays so they stay in registers.
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Barrier of the four consumer warps that also ANDs a flag over them: every consumer warp takes the
+// same decision (to go on or to stop), so none is left waiting at a barrier another has left.
+__device__ __forceinline__ bool consumers_all(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred))
+      : "memory");
+  return r != 0;
 }
 
-// One warp per PFT row r = (t, j): dO[pos[t, j]] = w[t, j] * dY[t];  g[t, j] = <dY[t], O[pos[t, j]]>.
-template <typename T>
-__global__ void __launch_bounds__(WARPS * 32) combine_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ O,
-                                                                 const int32_t* __restrict__ pos,
-                                                                 const float* __restrict__ w, int Tn, int k, int d,
-                                                                 T* __restrict__ dO, float* __restrict__ g,
-                                                                 int32_t* err) {
+// Per token t (work items are its row pieces, in order): dO[pos[t, j]] = w[t, j] * dY[t] and
+// g[t, j] = <dY[t], O[pos[t, j]]> (the combine's backward).  Stage: the dY piece, then the k O
+// pieces.  Each consumer thread keeps its partial dot products over the token's pieces; after the
+// last piece they are summed over the thread's warp and then over the four warps in order
+// (deterministic).  A token with an out-of-range row index is flagged and left unwritten.
+template <typename T, int KM>
+__global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bwd_bulk_kernel(
+    const char* __restrict__ dy, const char* __restrict__ O, const int32_t* __restrict__ pos,
+    const float* __restrict__ w, int Tn, int k, int row_bytes, int piece, int pieces, int stages,
+    char* __restrict__ dO, float* __restrict__ g, int32_t* err) {
   constexpr int VN = Vec<T>::n;
-  const int lane = threadIdx.x & 31;
-  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  extern __shared__ __align__(128) uint8_t csm[];
+  __shared__ __align__(8) uint64_t full[8];
+  __shared__ __align__(8) uint64_t empty[8];
+  __shared__ int valid[8];
+  __shared__ int spos[8][32];
+  __shared__ float sw[8][32];
+  __shared__ float red[4][KM];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long N = static_cast<long long>(Tn) * k;
-  for (long long r = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < N; r += nw) {
-    const long long t = r / k;
-    const long long p = pos[r];
-    if (p < 0 || p >= N) {
-      if (lane == 0) dev_error(err, PFMOE_DEV_BAD_POS);
-      continue;
+  const uint32_t stage_bytes = static_cast<uint32_t>(k + 1) * piece;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      bar_init(smem_addr(&full[s]), 1);
+      bar_init(smem_addr(&empty[s]), CB_CONSUMERS);
     }
-    const float wj = w[r];
-    const T* dyr = dy + t * d;
-    const T* orow = O + p * d;
-    T* drow = dO + p * d;
-    float part = 0.f;
-#pragma unroll 2
-    for (int c0 = lane * VN; c0 < d; c0 += 32 * VN) {
-      float a[VN], o[VN];
-      load16(dyr + c0, a);
-      load16(orow + c0, o);
-#pragma unroll
-      for (int i = 0; i < VN; ++i) {
-        part = fmaf(a[i], o[i], part);
-        a[i] *= wj;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  const uint32_t st0 = smem_addr(csm);
+  if (warp == 0) {
+    uint32_t pending = 0, pend_parity = 0;
+    int q = 0;
+    bool ok = true;
+    for (long long t = blockIdx.x; t < Tn && ok; t += gridDim.x) {
+      const int my_pos = lane < k ? pos[t * k + lane] : 0;
+      const bool bad = lane < k && (my_pos < 0 || my_pos >= N);
+      const bool any_bad = __any_sync(0xffffffffu, bad);
+      const float my_w = lane < k ? w[t * k + lane] : 0.f;
+      if (any_bad && lane == 0) dev_error(err, PFMOE_DEV_BAD_POS);
+      for (int c = 0; c < pieces; ++c, ++q) {
+        const int off = c * piece;
+        const int bytes = min(piece, row_bytes - off);
+        const int s = q % stages;
+        const uint32_t ph = (q / stages) & 1;
+        if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&empty[s]), ph ^ 1, err))) { ok = false; break; }
+        spos[s][lane] = my_pos;
+        sw[s][lane] = my_w;
+        if (lane == 0) valid[s] = any_bad ? 0 : 1;
+        __syncwarp();
+        const uint32_t fb = smem_addr(&full[s]);
+        if (any_bad) {
+          if (lane == 0) bar_arrive(fb);
+          continue;
+        }
+        if (lane == 0) {
+          bar_expect_tx(fb, static_cast<uint32_t>((k + 1) * bytes));
+          pending |= 1u << s;
+          pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
+          const uint32_t sb = st0 + s * stage_bytes;
+          bulk_load(sb, dy + t * row_bytes + off, bytes, fb);
+          for (int j = 0; j < k; ++j)
+            bulk_load(sb + (j + 1) * piece, O + static_cast<long long>(spos[s][j]) * row_bytes + off, bytes, fb);
+        }
+        __syncwarp();
       }
-      store16(drow + c0, a);
     }
-    part = warp_sum(part);
-    if (lane == 0) g[r] = part;
+    if (lane == 0)
+      for (int s = 0; s < stages; ++s)
+        if (pending & (1u << s)) bar_wait(smem_addr(&full[s]), (pend_parity >> s) & 1, err);
+    __syncwarp();
+  } else {
+    const int c16 = threadIdx.x - 32;
+    const int cw = warp - 1;
+    int q = 0;
+    bool ok = true;
+    for (long long t = blockIdx.x; t < Tn && ok; t += gridDim.x) {
+      float part[KM];
+#pragma unroll
+      for (int j = 0; j < KM; ++j) part[j] = 0.f;
+      bool tok_valid = true;
+      for (int c = 0; c < pieces; ++c, ++q) {
+        const int off = c * piece;
+        const int bytes = min(piece, row_bytes - off);
+        const int s = q % stages;
+        if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&full[s]), (q / stages) & 1, err))) { ok = false; break; }
+        tok_valid = valid[s] != 0;
+        if (tok_valid && c16 * 16 < bytes) {
+          const uint8_t* sp = csm + s * stage_bytes + c16 * 16;
+          float a[VN];
+          load16(reinterpret_cast<const T*>(sp), a);
+#pragma unroll
+          for (int j = 0; j < KM; ++j) {
+            if (j < k) {
+              float o[VN], dv[VN];
+              load16(reinterpret_cast<const T*>(sp + (j + 1) * piece), o);
+              const float wj = sw[s][j];
+#pragma unroll
+              for (int i = 0; i < VN; ++i) {
+                part[j] = fmaf(a[i], o[i], part[j]);
+                dv[i] = a[i] * wj;
+              }
+              store16(reinterpret_cast<T*>(dO + static_cast<long long>(spos[s][j]) * row_bytes + off + c16 * 16), dv);
+            }
+          }
+        }
+        bar_arrive(smem_addr(&empty[s]));
+      }
+      // every consumer warp takes these two barriers once per token and leaves with the others
+#pragma unroll
+      for (int j = 0; j < KM; ++j) {
+        const float v = warp_sum(part[j]);
+        if (lane == 0) red[cw][j] = v;
+      }
+      const bool all_ok = consumers_all(ok);   // red[] complete
+      if (all_ok && tok_valid && c16 < k) g[t * k + c16] = ((red[0][c16] + red[1][c16]) + red[2][c16]) + red[3][c16];
+      consumers_sync();                        // red[] read before the next token writes it
+      if (!all_ok) break;
+    }
   }
 }
 
-// dz_{t, ids[t,j]} = w_j (g_j - sum_l w_l g_l) (zero elsewhere);
-// dx[t] = sum_j dX_pft[pos[t, j]] + sum_j dz_j * Wg^T[ids[t, j]].
-// The dense dlogits row (and its BF16 copy for the dWg GEMM) is written by the token's chunk-0 item.
-template <typename T, int U>
-__global__ void __launch_bounds__(WARPS * 32) token_grad_kernel(const T* __restrict__ dxp, const int32_t* __restrict__ pos,
-                                                                const float* __restrict__ g, const float* __restrict__ w,
-                                                                const int32_t* __restrict__ ids,
-                                                                const T* __restrict__ wgT, int Tn, int k, int d, int E,
-                                                                T* __restrict__ dx, float* __restrict__ dlogits,
-                                                                __nv_bfloat16* __restrict__ dz_bf16, int32_t* err) {
+// Per token t (work items are its row pieces, in order): dx[t] = sum_j dX_pft[pos[t, j]] +
+// sum_j dz_j Wg^T[ids[t, j]], with dz_j = w_j (g_j - sum_l w_l g_l) the gradient of the selected
+// logits.  Stage: the k dX_pft pieces, then the k Wg^T row pieces; the producer warp computes dz
+// and, after issuing a token's first piece, writes its dense dlogits row (and the BF16 copy the
+// dWg GEMM reads) while the consumers sum.
+template <typename T>
+__global__ void __launch_bounds__(32 + CB_CONSUMERS) token_grad_bulk_kernel(
+    const char* __restrict__ dxp, const int32_t* __restrict__ pos, const float* __restrict__ g,
+    const float* __restrict__ w, const int32_t* __restrict__ ids, const char* __restrict__ wgT, int Tn, int k, int E,
+    int row_bytes, int piece, int pieces, int stages, char* __restrict__ dx, float* __restrict__ dlogits,
+    __nv_bfloat16* __restrict__ dz_bf16, int32_t* err) {
   constexpr int VN = Vec<T>::n;
-  const int lane = threadIdx.x & 31;
-  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  extern __shared__ __align__(128) uint8_t csm[];
+  __shared__ __align__(8) uint64_t full[8];
+  __shared__ __align__(8) uint64_t empty[8];
+  __shared__ int valid[8];
+  __shared__ float sdz[8][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long N = static_cast<long long>(Tn) * k;
-  const int CU = items_per_token(d, VN, U);
-  const long long items = static_cast<long long>(Tn) * CU;
-  for (long long it = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; it < items; it += nw) {
-    const long long t = it / CU;
-    const int ch = static_cast<int>(it - t * CU);
-    const int cb = ch * U * chunk_cols<T>() + lane * VN;
-    int my_pos;
-    if (!load_pos(pos, t, k, N, lane, my_pos, err)) continue;
-    const long long tk = t * k;
-    const float my_w = lane < k ? w[tk + lane] : 0.f;
-    const float my_g = lane < k ? g[tk + lane] : 0.f;
-    int my_id = lane < k ? ids[tk + lane] : 0;
-    if (lane < k && static_cast<unsigned>(my_id) >= static_cast<unsigned>(E)) {
-      dev_error(err, PFMOE_DEV_BAD_EXPERT_ID);
-      my_id = 0;
+  const uint32_t stage_bytes = static_cast<uint32_t>(2 * k) * piece;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      bar_init(smem_addr(&full[s]), 1);
+      bar_init(smem_addr(&empty[s]), CB_CONSUMERS);
     }
-    const float inner = warp_sum(my_w * my_g);
-    const float my_dz = lane < k ? my_w * (my_g - inner) : 0.f;
-    if (ch == 0) {
-      for (int e0 = 0; e0 < E; e0 += 32) {
-        const int e = e0 + lane;
-        float val = 0.f;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  const uint32_t st0 = smem_addr(csm);
+  if (warp == 0) {
+    uint32_t pending = 0, pend_parity = 0;
+    int q = 0;
+    bool ok = true;
+    for (long long t = blockIdx.x; t < Tn && ok; t += gridDim.x) {
+      const long long tk = t * k;
+      const int my_pos = lane < k ? pos[tk + lane] : 0;
+      const bool bad = lane < k && (my_pos < 0 || my_pos >= N);
+      const bool any_bad = __any_sync(0xffffffffu, bad);
+      if (any_bad && lane == 0) dev_error(err, PFMOE_DEV_BAD_POS);
+      const float my_w = lane < k ? w[tk + lane] : 0.f;
+      const float my_g = lane < k ? g[tk + lane] : 0.f;
+      int my_id = lane < k ? ids[tk + lane] : 0;
+      if (lane < k && static_cast<unsigned>(my_id) >= static_cast<unsigned>(E)) {
+        dev_error(err, PFMOE_DEV_BAD_EXPERT_ID);
+        my_id = 0;
+      }
+      const float inner = warp_sum(my_w * my_g);
+      const float my_dz = lane < k ? my_w * (my_g - inner) : 0.f;
+      for (int c = 0; c < pieces; ++c, ++q) {
+        const int off = c * piece;
+        const int bytes = min(piece, row_bytes - off);
+        const int s = q % stages;
+        const uint32_t ph = (q / stages) & 1;
+        if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&empty[s]), ph ^ 1, err))) { ok = false; break; }
+        sdz[s][lane] = my_dz;
+        if (lane == 0) valid[s] = any_bad ? 0 : 1;
+        __syncwarp();
+        const uint32_t fb = smem_addr(&full[s]);
+        if (any_bad) {
+          if (lane == 0) bar_arrive(fb);
+          __syncwarp();
+          continue;
+        }
+        if (lane == 0) {
+          bar_expect_tx(fb, static_cast<uint32_t>(2 * k * bytes));
+          pending |= 1u << s;
+          pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
+        }
+        const uint32_t sb = st0 + s * stage_bytes;
         for (int j = 0; j < k; ++j) {
-          const int idj = __shfl_sync(0xffffffffu, my_id, j);
-          const float dzj = __shfl_sync(0xffffffffu, my_dz, j);
-          if (idj == e) val = dzj;
+          const long long pj = __shfl_sync(0xffffffffu, my_pos, j);
+          const long long ij = __shfl_sync(0xffffffffu, my_id, j);
+          if (lane == 0) {
+            bulk_load(sb + j * piece, dxp + pj * row_bytes + off, bytes, fb);
+            bulk_load(sb + (k + j) * piece, wgT + ij * row_bytes + off, bytes, fb);
+          }
         }
-        if (e < E) {
-          dlogits[t * E + e] = val;
-          if (dz_bf16) dz_bf16[t * E + e] = __float2bfloat16_rn(val);
+        __syncwarp();
+        if (c == 0) {
+          // the dense dlogits row (and its BF16 copy), while the consumers sum the first piece
+          for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            float val = 0.f;
+            for (int j = 0; j < k; ++j) {
+              const int idj = __shfl_sync(0xffffffffu, my_id, j);
+              const float dzj = __shfl_sync(0xffffffffu, my_dz, j);
+              if (idj == e) val = dzj;
+            }
+            if (e < E) {
+              dlogits[t * E + e] = val;
+              if (dz_bf16) dz_bf16[t * E + e] = __float2bfloat16_rn(val);
+            }
+          }
         }
       }
     }
-    float acc[U][VN];
+    if (lane == 0)
+      for (int s = 0; s < stages; ++s)
+        if (pending & (1u << s)) bar_wait(smem_addr(&full[s]), (pend_parity >> s) & 1, err);
+    __syncwarp();
+  } else {
+    const int c16 = threadIdx.x - 32;
+    int q = 0;
+    bool ok = true;
+    for (long long t = blockIdx.x; t < Tn && ok; t += gridDim.x)
+    for (int c = 0; c < pieces; ++c, ++q) {
+      const int off = c * piece;
+      const int bytes = min(piece, row_bytes - off);
+      const int s = q % stages;
+      if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&full[s]), (q / stages) & 1, err))) { ok = false; break; }
+      if (valid[s] && c16 * 16 < bytes) {
+        float acc[VN];
 #pragma unroll
-    for (int u = 0; u < U; ++u)
-#pragma unroll
-      for (int i = 0; i < VN; ++i) acc[u][i] = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < k; ++j) {
-      const long long p = __shfl_sync(0xffffffffu, my_pos, j);
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int c0 = cb + u * chunk_cols<T>();
-        if (c0 < d) {
+        for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+        const uint8_t* sp = csm + s * stage_bytes + c16 * 16;
+        for (int j = 0; j < k; ++j) {
           float v[VN];
-          load16(dxp + p * d + c0, v);
+          load16(reinterpret_cast<const T*>(sp + j * piece), v);
 #pragma unroll
-          for (int i = 0; i < VN; ++i) acc[u][i] += v[i];
+          for (int i = 0; i < VN; ++i) acc[i] += v[i];
         }
-      }
-    }
-#pragma unroll 8
-    for (int j = 0; j < k; ++j) {
-      const long long idj = __shfl_sync(0xffffffffu, my_id, j);
-      const float dzj = __shfl_sync(0xffffffffu, my_dz, j);
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int c0 = cb + u * chunk_cols<T>();
-        if (c0 < d) {
+        for (int j = 0; j < k; ++j) {
           float v[VN];
-          load16(wgT + idj * d + c0, v);
+          load16(reinterpret_cast<const T*>(sp + (k + j) * piece), v);
+          const float dzj = sdz[s][j];
 #pragma unroll
-          for (int i = 0; i < VN; ++i) acc[u][i] = fmaf(dzj, v[i], acc[u][i]);
+          for (int i = 0; i < VN; ++i) acc[i] = fmaf(dzj, v[i], acc[i]);
         }
+        store16(reinterpret_cast<T*>(dx + t * row_bytes + off + c16 * 16), acc);
       }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int c0 = cb + u * chunk_cols<T>();
-      if (c0 < d) store16(dx + t * d + c0, acc[u]);
+      bar_arrive(smem_addr(&empty[s]));
     }
   }
 }
@@ -453,53 +561,77 @@ int launch_dispatch(const void* x, const int32_t* pos, int T, int k, int d, int 
   return PFMOE_OK;
 }
 
-// Column chunks per work item: one for rows of up to 16 chunks (d <= 4096 BF16), else 4, which
-// keeps the per-token prologue (pos / weight loads, dlogits row) off wide rows.
-static int chunks_per_item(int d, int vn) { return (d + 32 * vn - 1) / (32 * vn) > 16 ? 4 : 1; }
+
+// Ring geometry for `slots` row pieces per stage: pieces of CB_PIECE bytes, smaller where a stage
+// of that size would leave room for fewer than two stages in about 200 KB; about 96 KB of
+// stages (two CTAs per SM) where the pieces allow, between 2 and 8 stages.
+struct Ring {
+  int piece, pieces, stages;
+  size_t smem;
+};
+static Ring ring_for(int row_bytes, int slots) {
+  Ring r;
+  r.piece = CB_PIECE;
+  const int cap = (100 * 1024 / slots) & ~15;
+  if (r.piece > cap) r.piece = cap;
+  r.pieces = (row_bytes + r.piece - 1) / r.piece;
+  const int stage = slots * r.piece;
+  r.stages = (96 * 1024) / stage;
+  if (r.stages > 8) r.stages = 8;
+  if (r.stages < 2) r.stages = 2;
+  r.smem = static_cast<size_t>(r.stages) * stage;
+  return r;
+}
 
 int launch_combine(const void* out, const int32_t* pos, const float* w, int T, int k, int d, int dtype, void* y,
                    int32_t* err, cudaStream_t s) {
   const int row_bytes = d * (dtype == PFMOE_BF16 ? 2 : 4);
-  const int pieces = (row_bytes + CB_PIECE - 1) / CB_PIECE;
-  const int stage_bytes = k * CB_PIECE;
-  int stages = (96 * 1024) / stage_bytes;   // about 96 KB of stages: two CTAs per SM
-  if (stages > 8) stages = 8;
-  if (stages < 2) stages = 2;
-  const size_t smem = static_cast<size_t>(stages) * stage_bytes;
-  const long long items = static_cast<long long>(T) * pieces;
+  const Ring r = ring_for(row_bytes, k);
+  const long long items = static_cast<long long>(T) * r.pieces;
   long long grid = static_cast<long long>(num_sms()) * 2;
   if (grid > items) grid = items;
   if (dtype == PFMOE_BF16) {
     PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&combine_bulk_kernel<__nv_bfloat16>), 227 * 1024, "combine"));
     PFMOE_LAUNCH("combine", s,
-                 (combine_bulk_kernel<__nv_bfloat16><<<static_cast<int>(grid), 32 + CB_CONSUMERS, smem, s>>>(
-                     static_cast<const char*>(out), pos, w, T, k, row_bytes, pieces, stages, static_cast<char*>(y),
-                     err)));
+                 (combine_bulk_kernel<__nv_bfloat16><<<static_cast<int>(grid), 32 + CB_CONSUMERS, r.smem, s>>>(
+                     static_cast<const char*>(out), pos, w, T, k, row_bytes, r.piece, r.pieces, r.stages,
+                     static_cast<char*>(y), err)));
   } else {
     PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&combine_bulk_kernel<float>), 227 * 1024, "combine"));
     PFMOE_LAUNCH("combine", s,
-                 (combine_bulk_kernel<float><<<static_cast<int>(grid), 32 + CB_CONSUMERS, smem, s>>>(
-                     static_cast<const char*>(out), pos, w, T, k, row_bytes, pieces, stages, static_cast<char*>(y),
-                     err)));
+                 (combine_bulk_kernel<float><<<static_cast<int>(grid), 32 + CB_CONSUMERS, r.smem, s>>>(
+                     static_cast<const char*>(out), pos, w, T, k, row_bytes, r.piece, r.pieces, r.stages,
+                     static_cast<char*>(y), err)));
   }
+  return PFMOE_OK;
+}
+
+template <typename T, int KM>
+static int launch_cbwd_t(const void* dy, const void* out, const int32_t* pos, const float* w, int T_, int k,
+                         int row_bytes, const Ring& r, int grid, void* dO, float* g, int32_t* err, cudaStream_t s) {
+  PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&combine_bwd_bulk_kernel<T, KM>), 227 * 1024, "combine_bwd"));
+  PFMOE_LAUNCH("combine_bwd", s,
+               (combine_bwd_bulk_kernel<T, KM><<<grid, 32 + CB_CONSUMERS, r.smem, s>>>(
+                   static_cast<const char*>(dy), static_cast<const char*>(out), pos, w, T_, k, row_bytes, r.piece,
+                   r.pieces, r.stages, static_cast<char*>(dO), g, err)));
   return PFMOE_OK;
 }
 
 int launch_combine_bwd(const void* dy, const void* out, const int32_t* pos, const float* w, int T, int k, int d,
                        int dtype, void* dO, float* g, int32_t* err, cudaStream_t s) {
-  const int gr = item_grid(static_cast<long long>(T) * k);
+  const int row_bytes = d * (dtype == PFMOE_BF16 ? 2 : 4);
+  const Ring r = ring_for(row_bytes, k + 1);
+  long long grid = static_cast<long long>(num_sms()) * 2;
+  if (grid > T) grid = T;
+  const int gr = static_cast<int>(grid);
   if (dtype == PFMOE_BF16) {
-    PFMOE_LAUNCH("combine_bwd", s,
-                 combine_bwd_kernel<__nv_bfloat16><<<gr, WARPS * 32, 0, s>>>(
-                     static_cast<const __nv_bfloat16*>(dy), static_cast<const __nv_bfloat16*>(out), pos, w, T, k, d,
-                     static_cast<__nv_bfloat16*>(dO), g, err));
-  } else {
-    PFMOE_LAUNCH("combine_bwd", s,
-                 combine_bwd_kernel<float><<<gr, WARPS * 32, 0, s>>>(static_cast<const float*>(dy),
-                                                                     static_cast<const float*>(out), pos, w, T, k, d,
-                                                                     static_cast<float*>(dO), g, err));
+    if (k <= 8) return launch_cbwd_t<__nv_bfloat16, 8>(dy, out, pos, w, T, k, row_bytes, r, gr, dO, g, err, s);
+    if (k <= 16) return launch_cbwd_t<__nv_bfloat16, 16>(dy, out, pos, w, T, k, row_bytes, r, gr, dO, g, err, s);
+    return launch_cbwd_t<__nv_bfloat16, 32>(dy, out, pos, w, T, k, row_bytes, r, gr, dO, g, err, s);
   }
-  return PFMOE_OK;
+  if (k <= 8) return launch_cbwd_t<float, 8>(dy, out, pos, w, T, k, row_bytes, r, gr, dO, g, err, s);
+  if (k <= 16) return launch_cbwd_t<float, 16>(dy, out, pos, w, T, k, row_bytes, r, gr, dO, g, err, s);
+  return launch_cbwd_t<float, 32>(dy, out, pos, w, T, k, row_bytes, r, gr, dO, g, err, s);
 }
 
 int launch_transpose(const void* in, int rows, int cols, int dtype, void* out, cudaStream_t s) {
@@ -519,30 +651,24 @@ int launch_transpose(const void* in, int rows, int cols, int dtype, void* out, c
 int launch_token_grad(const void* dx_pft, const int32_t* pos, const float* g, const float* w, const int32_t* ids,
                       const void* wgT, int T, int k, int d, int E, int dtype, void* dx, float* dlogits,
                       void* dz_bf16, int32_t* err, cudaStream_t s) {
-  const int vn = dtype == PFMOE_BF16 ? 8 : 4;
-  const int U = chunks_per_item(d, vn);
-  const int gr = item_grid(static_cast<long long>(T) * items_per_token(d, vn, U));
+  const int row_bytes = d * (dtype == PFMOE_BF16 ? 2 : 4);
+  const Ring r = ring_for(row_bytes, 2 * k);
+  long long grid = static_cast<long long>(num_sms()) * 2;
+  if (grid > T) grid = T;
   auto* dzb = static_cast<__nv_bfloat16*>(dz_bf16);
   if (dtype == PFMOE_BF16) {
-    const auto* a = static_cast<const __nv_bfloat16*>(dx_pft);
-    const auto* wt = static_cast<const __nv_bfloat16*>(wgT);
-    auto* o = static_cast<__nv_bfloat16*>(dx);
-    if (U == 4)
-      PFMOE_LAUNCH("token_grad", s, (token_grad_kernel<__nv_bfloat16, 4><<<gr, WARPS * 32, 0, s>>>(
-                                         a, pos, g, w, ids, wt, T, k, d, E, o, dlogits, dzb, err)));
-    else
-      PFMOE_LAUNCH("token_grad", s, (token_grad_kernel<__nv_bfloat16, 1><<<gr, WARPS * 32, 0, s>>>(
-                                         a, pos, g, w, ids, wt, T, k, d, E, o, dlogits, dzb, err)));
+    PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&token_grad_bulk_kernel<__nv_bfloat16>), 227 * 1024,
+                         "token_grad"));
+    PFMOE_LAUNCH("token_grad", s,
+                 (token_grad_bulk_kernel<__nv_bfloat16><<<static_cast<int>(grid), 32 + CB_CONSUMERS, r.smem, s>>>(
+                     static_cast<const char*>(dx_pft), pos, g, w, ids, static_cast<const char*>(wgT), T, k, E,
+                     row_bytes, r.piece, r.pieces, r.stages, static_cast<char*>(dx), dlogits, dzb, err)));
   } else {
-    const auto* a = static_cast<const float*>(dx_pft);
-    const auto* wt = static_cast<const float*>(wgT);
-    auto* o = static_cast<float*>(dx);
-    if (U == 4)
-      PFMOE_LAUNCH("token_grad", s, (token_grad_kernel<float, 4><<<gr, WARPS * 32, 0, s>>>(
-                                         a, pos, g, w, ids, wt, T, k, d, E, o, dlogits, dzb, err)));
-    else
-      PFMOE_LAUNCH("token_grad", s, (token_grad_kernel<float, 1><<<gr, WARPS * 32, 0, s>>>(
-                                         a, pos, g, w, ids, wt, T, k, d, E, o, dlogits, dzb, err)));
+    PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&token_grad_bulk_kernel<float>), 227 * 1024, "token_grad"));
+    PFMOE_LAUNCH("token_grad", s,
+                 (token_grad_bulk_kernel<float><<<static_cast<int>(grid), 32 + CB_CONSUMERS, r.smem, s>>>(
+                     static_cast<const char*>(dx_pft), pos, g, w, ids, static_cast<const char*>(wgT), T, k, E,
+                     row_bytes, r.piece, r.pieces, r.stages, static_cast<char*>(dx), dlogits, dzb, err)));
   }
   return PFMOE_OK;
 }

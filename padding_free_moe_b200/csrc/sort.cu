@@ -17,21 +17,33 @@
 namespace pfmoe {
 namespace {
 
-constexpr int KEYS_PER_WARP = 256;   // 8 per lane
 constexpr int SCAN_THREADS = 1024;
+
+// Keys per warp of a chunk: 256 (8 per lane) while the sort has few chunks, 1024 (32 per lane) once
+// there are enough 1024-key chunks for two CTAs on each of 148 SMs.  Larger chunks amortise each
+// chunk's per-key scans and write the sorted rows as longer runs.  The choice depends only on the
+// shape (never on the device), so workspace sizes are host-computable.
+constexpr int KPW_SMALL = 256;
+constexpr int KPW_LARGE = 1024;
 
 // Warps per chunk CTA: up to 8, while the scatter's per-warp counters (W * K ints) fit in 48 KB.
 inline int warps_per_block(int K) {
   int w = 12288 / (K > 0 ? K : 1);
   return w < 1 ? 1 : (w > 8 ? 8 : w);
 }
-inline long long chunk_keys(int K) { return static_cast<long long>(warps_per_block(K)) * KEYS_PER_WARP; }
+inline int keys_per_warp(long long n_max, int K) {
+  return n_max / (static_cast<long long>(warps_per_block(K)) * KPW_LARGE) >= 296 ? KPW_LARGE : KPW_SMALL;
+}
+inline long long chunk_keys(long long n_max, int K) {
+  return static_cast<long long>(warps_per_block(K)) * keys_per_warp(n_max, K);
+}
 
 __device__ __forceinline__ long long dev_count(long long n, const int32_t* n_dev) {
   return n_dev ? static_cast<long long>(*n_dev) : n;
 }
 
 // One CTA per chunk: shared histogram of the chunk's keys -> counts[chunk][key].
+template <int KPW>
 __global__ void chunk_hist_kernel(const int32_t* __restrict__ keys, long long n, const int32_t* n_dev, int K,
                                   int nchunks, int32_t* __restrict__ counts, int32_t* err) {
   extern __shared__ int32_t sh[];
@@ -39,8 +51,8 @@ __global__ void chunk_hist_kernel(const int32_t* __restrict__ keys, long long n,
   for (int i = threadIdx.x; i < K; i += blockDim.x) sh[i] = 0;
   __syncthreads();
   const long long nn = dev_count(n, n_dev);
-  const long long b = static_cast<long long>(chunk) * blockDim.x / 32 * KEYS_PER_WARP;
-  const long long e = min(b + static_cast<long long>(blockDim.x / 32) * KEYS_PER_WARP, nn);
+  const long long b = static_cast<long long>(chunk) * blockDim.x / 32 * KPW;
+  const long long e = min(b + static_cast<long long>(blockDim.x / 32) * KPW, nn);
   bool bad = false;
   for (long long i = b + threadIdx.x; i < e; i += blockDim.x) {
     const int key = keys[i];
@@ -173,13 +185,13 @@ __global__ void __launch_bounds__(SCAN_THREADS) key_scan_kernel(const int32_t* _
 // neighbouring addresses instead of one scattered sector per element.
 // Sink interface: at_source(i, p) writes the outputs indexed by element i; payload(i, a, b) gives
 // two ints carried to the sorted side; at_dest(p, key, a, b) writes the outputs indexed by row p.
-// Shared memory: [warps][K] counts, two [K] bases and three [warps * KEYS_PER_WARP] staging arrays.
-__host__ __device__ inline size_t scatter_smem_bytes(int nw, int K) {
-  return (static_cast<size_t>(nw) * K + 2 * static_cast<size_t>(K) + 3 * static_cast<size_t>(nw) * KEYS_PER_WARP) *
+// Shared memory: [warps][K] counts, two [K] bases and three [warps * keys per warp] staging arrays.
+__host__ __device__ inline size_t scatter_smem_bytes(int nw, int K, int kpw) {
+  return (static_cast<size_t>(nw) * K + 2 * static_cast<size_t>(K) + 3 * static_cast<size_t>(nw) * kpw) *
          sizeof(int32_t);
 }
 
-template <class Sink>
+template <class Sink, int KPW>
 __global__ void chunk_scatter_kernel(const int32_t* __restrict__ keys, long long n, const int32_t* n_dev, int K,
                                      int nchunks, const int32_t* __restrict__ base,
                                      const int32_t* __restrict__ key_offsets, Sink sink) {
@@ -192,15 +204,15 @@ __global__ void chunk_scatter_kernel(const int32_t* __restrict__ keys, long long
   int32_t* cnt = sh;                                   // [nw][K]: counts, then each warp's start in its key's run
   int32_t* lbase = cnt + static_cast<long long>(nw) * K;   // [K]: first staging slot of each key
   int32_t* gbase = lbase + K;                          // [K]: first sorted row of each key in this chunk
-  int32_t* skey = gbase + K;                           // [nw * KEYS_PER_WARP]: staged keys, in sorted order
-  int32_t* spa = skey + nw * KEYS_PER_WARP;            // staged payloads
-  int32_t* spb = spa + nw * KEYS_PER_WARP;
+  int32_t* skey = gbase + K;                           // [nw * KPW]: staged keys, in sorted order
+  int32_t* spa = skey + nw * KPW;                      // staged payloads
+  int32_t* spb = spa + nw * KPW;
   for (int i = threadIdx.x; i < nw * K; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
   const long long nn = dev_count(n, n_dev);
-  const long long b = (static_cast<long long>(chunk) * nw + w) * KEYS_PER_WARP;
+  const long long b = (static_cast<long long>(chunk) * nw + w) * KPW;
   int32_t* wcnt = cnt + w * K;
-  constexpr int IT = KEYS_PER_WARP / 32;
+  constexpr int IT = KPW / 32;
   int key[IT];
   unsigned peers[IT];
 #pragma unroll
@@ -585,18 +597,49 @@ int sort_scan(const int32_t* counts, int C, int K, int32_t* totals, int32_t* off
 inline long long long_scan_tiles(long long n_max) { return (n_max + SCAN_TILE - 1) / SCAN_TILE; }
 constexpr long long LONG_SCAN_MIN = 4LL * SCAN_TILE;   // below this one CTA scans the array
 
-// The staged scatter needs up to ~91 KB of shared memory (K = 4096 keys, three warps): opt in
-// once per device.
-template <class Sink>
+// The staged scatter needs up to ~116 KB of shared memory (K = 4096 keys, three warps of 1024
+// keys): opt in once per device.
+template <class Sink, int KPW>
 int scatter_smem_attr() {
-  return smem_optin(reinterpret_cast<const void*>(&chunk_scatter_kernel<Sink>),
-                    static_cast<int>(scatter_smem_bytes(3, 4096) + 4096), "chunk_scatter");
+  return smem_optin(reinterpret_cast<const void*>(&chunk_scatter_kernel<Sink, KPW>), 227 * 1024, "chunk_scatter");
+}
+
+// Histogram + scatter launches of one stable counting sort, with the chunk size chosen for n_max.
+template <class Sink>
+int sort_hist(const int32_t* keys, long long n_max, const int32_t* n_dev, int K, int C, int32_t* counts,
+              int32_t* err, const char* name, cudaStream_t s) {
+  const int wpb = warps_per_block(K);
+  if (keys_per_warp(n_max, K) == KPW_LARGE)
+    PFMOE_LAUNCH(name, s, (chunk_hist_kernel<KPW_LARGE><<<C, wpb * 32, K * sizeof(int32_t), s>>>(keys, n_max, n_dev,
+                                                                                              K, C, counts, err)));
+  else
+    PFMOE_LAUNCH(name, s, (chunk_hist_kernel<KPW_SMALL><<<C, wpb * 32, K * sizeof(int32_t), s>>>(keys, n_max, n_dev,
+                                                                                              K, C, counts, err)));
+  return PFMOE_OK;
+}
+
+template <class Sink>
+int sort_scatter(const int32_t* keys, long long n_max, const int32_t* n_dev, int K, int C, const int32_t* base,
+                 const int32_t* key_offsets, const Sink& sink, const char* name, cudaStream_t s) {
+  const int wpb = warps_per_block(K);
+  const int kpw = keys_per_warp(n_max, K);
+  const size_t sm = scatter_smem_bytes(wpb, K, kpw);
+  if (kpw == KPW_LARGE) {
+    PFMOE_TRY((scatter_smem_attr<Sink, KPW_LARGE>()));
+    PFMOE_LAUNCH(name, s, (chunk_scatter_kernel<Sink, KPW_LARGE><<<C, wpb * 32, sm, s>>>(keys, n_max, n_dev, K, C,
+                                                                                       base, key_offsets, sink)));
+  } else {
+    PFMOE_TRY((scatter_smem_attr<Sink, KPW_SMALL>()));
+    PFMOE_LAUNCH(name, s, (chunk_scatter_kernel<Sink, KPW_SMALL><<<C, wpb * 32, sm, s>>>(keys, n_max, n_dev, K, C,
+                                                                                       base, key_offsets, sink)));
+  }
+  return PFMOE_OK;
 }
 
 }  // namespace
 
 size_t csort_ws_bytes(long long n_max, int K) {
-  const long long C = (n_max + chunk_keys(K) - 1) / chunk_keys(K);
+  const long long C = (n_max + chunk_keys(n_max, K) - 1) / chunk_keys(n_max, K);
   return static_cast<size_t>(2 * (C > 0 ? C : 1) * static_cast<long long>(K) + K) * sizeof(int32_t);
 }
 
@@ -604,23 +647,14 @@ int pft_build_impl(const int32_t* ids, const float* w, int T, int E, int k, int3
                    int32_t* token_ids, int32_t* expert_ids, float* cw, int32_t* pos, int32_t* tile_offsets,
                    void* ws, int32_t* err, cudaStream_t s) {
   const long long N = static_cast<long long>(T) * k;
-  const int C = static_cast<int>((N + chunk_keys(E) - 1) / chunk_keys(E));
+  const int C = static_cast<int>((N + chunk_keys(N, E) - 1) / chunk_keys(N, E));
   int32_t* counts = static_cast<int32_t*>(ws);
   int32_t* base = counts + static_cast<long long>(C) * E;
-  const int wpb = warps_per_block(E);
-  const int blocks = C;
-  const size_t sm = scatter_smem_bytes(wpb, E);
-  PFMOE_TRY(scatter_smem_attr<PftSink>());
-  if (C > 0)
-    PFMOE_LAUNCH("pft_hist", s,
-                 chunk_hist_kernel<<<blocks, wpb * 32, E * sizeof(int32_t), s>>>(ids, N, nullptr, E, C, counts, err));
+  if (C > 0) PFMOE_TRY(sort_hist<PftSink>(ids, N, nullptr, E, C, counts, err, "pft_hist", s));
   int32_t* key_tot = base + static_cast<long long>(C) * E;
   PFMOE_TRY(sort_scan(counts, C, E, tpe, offsets, base, tile_offsets, 128, key_tot, "pft_scan", s));
   PftSink sink{w, k, pos, token_ids, expert_ids, cw};
-  if (C > 0)
-    PFMOE_LAUNCH("pft_scatter", s,
-                 chunk_scatter_kernel<PftSink><<<blocks, wpb * 32, sm, s>>>(ids, N, nullptr, E, C, base, offsets,
-                                                                             sink));
+  if (C > 0) PFMOE_TRY(sort_scatter<PftSink>(ids, N, nullptr, E, C, base, offsets, sink, "pft_scatter", s));
   return PFMOE_OK;
 }
 
@@ -651,7 +685,7 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
   int32_t* tsum_a = p; p += lt;
   int32_t* tsum_b = p; p += lt;
   p += 64 - ((p - static_cast<int32_t*>(ws)) & 63);   // keep 256-byte alignment
-  const int C = static_cast<int>((pmax + chunk_keys(n_nodes) - 1) / chunk_keys(n_nodes));
+  const int C = static_cast<int>((pmax + chunk_keys(pmax, n_nodes) - 1) / chunk_keys(pmax, n_nodes));
   int32_t* ccounts = p; p += static_cast<long long>(C > 0 ? C : 1) * n_nodes;
   int32_t* cbase = p;
 
@@ -668,23 +702,13 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
     PFMOE_LAUNCH("rbd_scan_tokens", s, tile_scan_kernel<<<nt, SCAN_THREADS, 0, s>>>(ucount, T, nullptr, tsum_a, pbase));
   }
   PFMOE_RBD_LAUNCH("rbd_emit", rbd_emit_kernel, T, k, s, ids, T, k, E, epd, epn, pbase, pkey, ptoken, prc, err);
-  const int wpb = warps_per_block(n_nodes);
-  const int blocks = C;
-  const size_t sm = scatter_smem_bytes(wpb, n_nodes);
-  PFMOE_TRY(scatter_smem_attr<RbdSink>());
-  if (C > 0) {
-    PFMOE_LAUNCH("rbd_hist", s,
-                 chunk_hist_kernel<<<blocks, wpb * 32, n_nodes * sizeof(int32_t), s>>>(pkey, pmax, counts, n_nodes, C,
-                                                                                     ccounts, err));
-  }
+  if (C > 0) PFMOE_TRY(sort_hist<RbdSink>(pkey, pmax, counts, n_nodes, C, ccounts, err, "rbd_hist", s));
   int32_t* node_tot = cbase + static_cast<long long>(C > 0 ? C : 1) * n_nodes;
   PFMOE_TRY(sort_scan(ccounts, C, n_nodes, pilots_per_node, node_offsets, cbase, nullptr, 0, node_tot,
                       "rbd_scan_nodes", s));
   if (C > 0) {
     RbdSink sink{ptoken, prc, pilot_token, pilot_node, rc_sorted, psorted};
-    PFMOE_LAUNCH("rbd_scatter", s,
-                 chunk_scatter_kernel<RbdSink><<<blocks, wpb * 32, sm, s>>>(pkey, pmax, counts, n_nodes, C, cbase,
-                                                                             node_offsets, sink));
+    PFMOE_TRY(sort_scatter<RbdSink>(pkey, pmax, counts, n_nodes, C, cbase, node_offsets, sink, "rbd_scatter", s));
   }
   if (pmax < LONG_SCAN_MIN) {
     PFMOE_LAUNCH("rbd_scan_replicas", s,

@@ -121,3 +121,52 @@ def test_bounded_wait_gives_up_and_context_survives():
     inp = make_inputs(cfg, seed=3, device="cuda")
     assert run_step(layer, inp) == 0
 
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("E,k,epd,dpn", [(256, 8, 8, 4), (1024, 4, 16, 8)])
+def test_pft_and_rbd_large_chunks_match_oracle(E, k, epd, dpn):
+    # More than 2.4 M assignments: the counting sorts switch to 1024 keys per warp.
+    from workloads.generate import make_topk_ids
+    T = (1 << 22) // k + 123
+    ids = make_topk_ids(T, E, k, seed=9, device="cuda")
+    w = torch.rand(T, k, device="cuda")
+    N = T * k
+    i32 = dict(device="cuda", dtype=torch.int32)
+    tpe, off, tiles = torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(E + 1, **i32)
+    tok, eid, pos = torch.empty(N, **i32), torch.empty(N, **i32), torch.empty(T, k, **i32)
+    cw = torch.empty(N, device="cuda")
+    err = torch.zeros(1, **i32)
+    ws_b = L.pft_build_workspace_size(T, E, k)
+    ws = torch.empty(ws_b, device="cuda", dtype=torch.uint8)
+    L.pft_build(ids, w, T, E, k, tpe, off, tok, eid, cw, pos, tiles, ws, ws_b, err)
+    n_nodes = E // (epd * dpn)
+    pmax = T * min(k, n_nodes)
+    o = dict(ppn=torch.empty(n_nodes, **i32), noff=torch.empty(n_nodes + 1, **i32), ptok=torch.empty(pmax, **i32),
+             pnode=torch.empty(pmax, **i32), pdev=torch.empty(pmax, **i32), roff=torch.empty(pmax + 1, **i32),
+             rexp=torch.empty(N, **i32), ap=torch.empty(T, k, **i32), cnt=torch.empty(2, **i32))
+    rws_b = L.rbd_plan_workspace_size(T, k, E, epd, dpn)
+    rws = torch.empty(rws_b, device="cuda", dtype=torch.uint8)
+    L.rbd_plan(ids, T, k, E, epd, dpn, o["ppn"], o["noff"], o["ptok"], o["pnode"], o["pdev"], o["roff"], o["rexp"],
+               o["ap"], o["cnt"], rws, rws_b, err)
+    torch.cuda.synchronize()
+    assert int(err) == 0
+    ids_h = i64(ids)
+    p = O.pft_build(ids_h, w.cpu().numpy(), E)
+    assert np.array_equal(i64(tpe), p["tokens_per_expert"])
+    assert np.array_equal(i64(off), p["expert_offsets"])
+    assert np.array_equal(i64(tiles), p["tile_offsets"])
+    assert np.array_equal(i64(tok), p["token_ids"])
+    assert np.array_equal(i64(eid), p["expert_ids"])
+    assert np.array_equal(cw.cpu().numpy().astype(np.float64), p["combine_weights"])
+    assert np.array_equal(i64(pos), p["pos"])
+    r = O.rbd_plan(ids_h, E, epd, dpn)
+    P = r["num_pilots"]
+    assert int(o["cnt"][0]) == P and int(o["cnt"][1]) == r["num_token_device_pairs"]
+    assert np.array_equal(i64(o["ppn"]), r["pilots_per_node"])
+    assert np.array_equal(i64(o["ptok"][:P]), r["pilot_token"])
+    assert np.array_equal(i64(o["pnode"][:P]), r["pilot_node"])
+    assert np.array_equal(i64(o["pdev"][:P]), r["pilot_device"])
+    assert np.array_equal(i64(o["roff"][:P + 1]), r["replica_offsets"])
+    assert np.array_equal(i64(o["rexp"]), r["replica_expert"])
+    assert np.array_equal(i64(o["ap"]), r["assign_pilot"])
