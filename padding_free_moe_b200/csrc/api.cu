@@ -53,6 +53,18 @@ int smem_optin(const void* kernel, int bytes, const char* name) {
   if (e != cudaSuccess) return fail(PFMOE_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
   std::lock_guard<std::mutex> lk(mu);
   if (done.count({dev, kernel})) return PFMOE_OK;
+  // The opt-in limit covers dynamic shared memory only: the device's per-block maximum less the
+  // kernel's static shared memory.
+  int optin = 0;
+  e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess)
+    return fail(PFMOE_ERR_CUDA, std::string(name) + ": cudaDeviceGetAttribute: " + cudaGetErrorString(e));
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kernel);
+  if (e != cudaSuccess)
+    return fail(PFMOE_ERR_CUDA, std::string(name) + ": cudaFuncGetAttributes: " + cudaGetErrorString(e));
+  const int cap = optin - static_cast<int>(fa.sharedSizeBytes);
+  if (bytes > cap) bytes = cap;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess)
     return fail(PFMOE_ERR_CUDA, std::string(name) + ": cudaFuncSetAttribute failed: " + cudaGetErrorString(e));

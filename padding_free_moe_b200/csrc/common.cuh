@@ -24,9 +24,10 @@ int check_launch(const char* what);
 
 int num_sms();
 
-// Raise a kernel's dynamic shared-memory limit to `bytes` on the current device.
-// cudaFuncSetAttribute acts on the current device only, so this is done once per
-// (device, kernel) pair; thread-safe.
+// Raise a kernel's dynamic shared-memory limit to `bytes` (at most the device's opt-in limit
+// less the kernel's static shared memory) on the current device.  cudaFuncSetAttribute acts
+// on the current device only, so this is done once per (device, kernel) pair; thread-safe.
+// Every launch then requests no more than the bytes its plan computed from the same limit.
 int smem_optin(const void* kernel, int bytes, const char* name);
 
 #define PFMOE_TRY(expr)            \
