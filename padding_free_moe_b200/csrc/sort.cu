@@ -560,6 +560,208 @@ __global__ void rbd_final_kernel(const int32_t* ids, int T, int k, int E, int ep
   }
 }
 
+
+// ------------------------------------------------ RBD plan for maps of at most 8 nodes
+// Every configured device map has at most 8 nodes; for those the plan needs no sort.  The
+// pilots of node n, in token order, are the tokens that route to n, so pilot (t, n) sits at
+// node_offsets[n] + #{t' < t routing to n}, and its replicas at the node's replica offset +
+// #{replicas on n of tokens t' < t}: per-node prefix counts over tokens.  Three launches, one
+// thread per token:
+//   rbd_fast_count: per 256-token tile, per node: tokens routing to it and replicas on it;
+//   rbd_fast_scan:  per node, exclusive prefix over tiles; node offsets, totals, P;
+//   rbd_fast_emit:  per token, the in-tile prefix by warp scans, then every output.
+constexpr int RF_NODES = 8;
+constexpr int RF_TILE = 256;
+
+template <int KM>
+__device__ __forceinline__ void rf_load(const int32_t* __restrict__ ids, long long t, bool valid, int k, int E, int epn,
+                                        int (&e)[KM], int (&nd)[KM], int32_t* err) {
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    int v = 0;
+    if (valid && j < k) {
+      v = ids[t * k + j];
+      if (static_cast<unsigned>(v) >= static_cast<unsigned>(E)) {
+        dev_error(err, PFMOE_DEV_BAD_EXPERT_ID);
+        v = 0;
+      }
+    }
+    e[j] = v;
+    nd[j] = (valid && j < k) ? v / epn : -1;
+  }
+}
+
+// Packed per-node count of one token: bit 0..15 = 1 if the token routes to the node, 16..31 = its
+// replicas there (sums over a 256-token tile stay below 2^16 in both fields).
+template <int KM>
+__device__ __forceinline__ void rf_counts(const int (&nd)[KM], int (&c)[RF_NODES]) {
+#pragma unroll
+  for (int n = 0; n < RF_NODES; ++n) {
+    int r = 0;
+#pragma unroll
+    for (int j = 0; j < KM; ++j) r += nd[j] == n;
+    c[n] = (r > 0 ? 1 : 0) | (r << 16);
+  }
+}
+
+template <int KM>
+__global__ void __launch_bounds__(RF_TILE) rbd_fast_count_kernel(const int32_t* __restrict__ ids, int T, int k, int E,
+                                                                 int epd, int epn, int32_t* __restrict__ tile_cnt,
+                                                                 int32_t* __restrict__ tile_dev, int32_t* err) {
+  __shared__ int red[RF_TILE / 32][RF_NODES + 1];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long t = static_cast<long long>(blockIdx.x) * RF_TILE + threadIdx.x;
+  const bool valid = t < T;
+  int e[KM], nd[KM], c[RF_NODES];
+  rf_load<KM>(ids, t, valid, k, E, epn, e, nd, err);
+  rf_counts<KM>(nd, c);
+  int dc = 0;   // distinct devices of the token
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    bool first = j < k && valid;
+#pragma unroll
+    for (int i = 0; i < j; ++i) first = first && (e[i] / epd != e[j] / epd);
+    dc += first;
+  }
+#pragma unroll
+  for (int n = 0; n < RF_NODES; ++n) {
+    int v = c[n];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[warp][n] = v;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dc += __shfl_xor_sync(0xffffffffu, dc, o);
+  if (lane == 0) red[warp][RF_NODES] = dc;
+  __syncthreads();
+  if (threadIdx.x <= RF_NODES) {
+    int v = 0;
+    for (int w = 0; w < RF_TILE / 32; ++w) v += red[w][threadIdx.x];
+    if (threadIdx.x < RF_NODES) tile_cnt[static_cast<long long>(blockIdx.x) * RF_NODES + threadIdx.x] = v;
+    else tile_dev[blockIdx.x] = v;
+  }
+}
+
+// One CTA: warp n scans node n's packed tile counts into exclusive token bases (in place) and
+// replica bases (tile_rep_base); then the node offsets, P and the distinct (token, device) total.
+__global__ void __launch_bounds__(256) rbd_fast_scan_kernel(int ntiles, int n_nodes, int32_t* __restrict__ tile_cnt,
+                                                            int32_t* __restrict__ tile_rep_base,
+                                                            const int32_t* __restrict__ tile_dev,
+                                                            int32_t* pilots_per_node, int32_t* node_offsets,
+                                                            int32_t* node_rep_off, int32_t* counts,
+                                                            int32_t* replica_offsets) {
+  __shared__ int tot_tok[RF_NODES], tot_rep[RF_NODES];
+  __shared__ int dsum[8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp < n_nodes) {
+    int ct = 0, cr = 0;   // running totals (unpacked: node totals can exceed 16 bits)
+    for (int i0 = 0; i0 < ntiles; i0 += 32) {
+      const int i = i0 + lane;
+      const int v = i < ntiles ? tile_cnt[static_cast<long long>(i) * RF_NODES + warp] : 0;
+      int a = v & 0xffff, b = v >> 16;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int ya = __shfl_up_sync(0xffffffffu, a, o);
+        const int yb = __shfl_up_sync(0xffffffffu, b, o);
+        if (lane >= o) { a += ya; b += yb; }
+      }
+      const int ea = a - (v & 0xffff), eb = b - (v >> 16);
+      if (i < ntiles) {   // exclusive bases, unpacked (node totals exceed 16 bits)
+        tile_cnt[static_cast<long long>(i) * RF_NODES + warp] = ct + ea;
+        tile_rep_base[static_cast<long long>(i) * RF_NODES + warp] = cr + eb;
+      }
+      ct += __shfl_sync(0xffffffffu, a, 31);
+      cr += __shfl_sync(0xffffffffu, b, 31);
+    }
+    if (lane == 0) { tot_tok[warp] = ct; tot_rep[warp] = cr; }
+  }
+  int ds = 0;
+  for (int i = threadIdx.x; i < ntiles; i += blockDim.x) ds += tile_dev[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
+  if (lane == 0) dsum[warp] = ds;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int off = 0, roff = 0, dtot = 0;
+    for (int w = 0; w < 8; ++w) dtot += dsum[w];
+    for (int n = 0; n < n_nodes; ++n) {
+      node_offsets[n] = off;
+      pilots_per_node[n] = tot_tok[n];
+      node_rep_off[n] = roff;
+      off += tot_tok[n];
+      roff += tot_rep[n];
+    }
+    node_offsets[n_nodes] = off;
+    counts[0] = off;
+    counts[1] = dtot;
+    replica_offsets[off] = roff;
+  }
+}
+
+template <int KM>
+__global__ void __launch_bounds__(RF_TILE) rbd_fast_emit_kernel(
+    const int32_t* __restrict__ ids, int T, int k, int E, int epd, int epn, int n_nodes,
+    const int32_t* __restrict__ tile_tok_base, const int32_t* __restrict__ tile_rep_base,
+    const int32_t* __restrict__ node_offsets, const int32_t* __restrict__ node_rep_off, int32_t* __restrict__ pilot_token,
+    int32_t* __restrict__ pilot_node, int32_t* __restrict__ pilot_device, int32_t* __restrict__ replica_offsets,
+    int32_t* __restrict__ replica_expert, int32_t* __restrict__ assign_pilot, int32_t* err) {
+  __shared__ int wsum[RF_TILE / 32][RF_NODES];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long t = static_cast<long long>(blockIdx.x) * RF_TILE + threadIdx.x;
+  const bool valid = t < T;
+  int e[KM], nd[KM], c[RF_NODES], ex[RF_NODES];
+  rf_load<KM>(ids, t, valid, k, E, epn, e, nd, nullptr);   // rbd_fast_count flagged bad ids
+  rf_counts<KM>(nd, c);
+  // in-warp exclusive prefix of the packed counts, per node
+#pragma unroll
+  for (int n = 0; n < RF_NODES; ++n) {
+    int a = c[n];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, a, o);
+      if (lane >= o) a += y;
+    }
+    ex[n] = a - c[n];
+    if (lane == 31) wsum[warp][n] = a;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int n = 0; n < RF_NODES; ++n)
+    for (int w = 0; w < warp; ++w) ex[n] += wsum[w][n];
+  if (!valid) return;
+  (void)err;
+  int idx[RF_NODES], rs[RF_NODES];
+  const long long tb = static_cast<long long>(blockIdx.x) * RF_NODES;
+#pragma unroll
+  for (int n = 0; n < RF_NODES; ++n) {
+    idx[n] = 0;
+    rs[n] = 0;
+    if (n < n_nodes && (c[n] & 0xffff)) {
+      idx[n] = node_offsets[n] + tile_tok_base[tb + n] + (ex[n] & 0xffff);
+      rs[n] = node_rep_off[n] + tile_rep_base[tb + n] + (ex[n] >> 16);
+      pilot_token[idx[n]] = static_cast<int32_t>(t);
+      pilot_node[idx[n]] = n;
+      replica_offsets[idx[n]] = rs[n];
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    if (j < k) {
+      int within = 0;
+#pragma unroll
+      for (int i = 0; i < KM; ++i)
+        within += (i < k) && nd[i] == nd[j] && (e[i] < e[j] || (e[i] == e[j] && i < j));
+      int pj = 0, rj = 0;
+#pragma unroll
+      for (int n = 0; n < RF_NODES; ++n)
+        if (nd[j] == n) { pj = idx[n]; rj = rs[n]; }
+      replica_expert[rj + within] = e[j];
+      assign_pilot[t * k + j] = pj;
+      if (within == 0) pilot_device[pj] = e[j] / epd;
+    }
+  }
+}
+
 // Launch one of the per-token RBD kernels with the smallest lane group that holds k experts.
 #define PFMOE_RBD_LAUNCH(NAME, KERNEL, T_, k_, s_, ...)                                                       \
   do {                                                                                                       \
@@ -636,6 +838,46 @@ int sort_scatter(const int32_t* keys, long long n_max, const int32_t* n_dev, int
   return PFMOE_OK;
 }
 
+
+template <int KM>
+static int rbd_fast_launch(const int32_t* ids, int T, int k, int E, int epd, int epn, int n_nodes, int32_t* ppn,
+                           int32_t* noff, int32_t* ptok, int32_t* pnode, int32_t* pdev, int32_t* roff, int32_t* rexp,
+                           int32_t* ap, int32_t* counts, int32_t* tile_cnt, int32_t* tile_rep, int32_t* tile_dev,
+                           int32_t* node_rep_off, int32_t* err, cudaStream_t s) {
+  const int ntiles = (T + RF_TILE - 1) / RF_TILE;
+  if (ntiles > 0)
+    PFMOE_LAUNCH("rbd_count", s,
+                 (rbd_fast_count_kernel<KM><<<ntiles, RF_TILE, 0, s>>>(ids, T, k, E, epd, epn, tile_cnt, tile_dev,
+                                                                      err)));
+  PFMOE_LAUNCH("rbd_scan_nodes", s,
+               (rbd_fast_scan_kernel<<<1, 256, 0, s>>>(ntiles, n_nodes, tile_cnt, tile_rep, tile_dev, ppn, noff,
+                                                       node_rep_off, counts, roff)));
+  if (ntiles > 0)
+    PFMOE_LAUNCH("rbd_emit", s,
+               (rbd_fast_emit_kernel<KM><<<ntiles, RF_TILE, 0, s>>>(ids, T, k, E, epd, epn, n_nodes, tile_cnt, tile_rep,
+                                                                    noff, node_rep_off, ptok, pnode, pdev, roff, rexp,
+                                                                    ap, err)));
+  return PFMOE_OK;
+}
+
+static int rbd_fast_impl(const int32_t* ids, int T, int k, int E, int epd, int epn, int n_nodes, int32_t* ppn,
+                         int32_t* noff, int32_t* ptok, int32_t* pnode, int32_t* pdev, int32_t* roff, int32_t* rexp,
+                         int32_t* ap, int32_t* counts, void* ws, int32_t* err, cudaStream_t s) {
+  const size_t tiles = (static_cast<size_t>(T) + RF_TILE - 1) / RF_TILE;
+  int32_t* tile_cnt = static_cast<int32_t*>(ws);
+  int32_t* tile_rep = tile_cnt + tiles * RF_NODES;
+  int32_t* tile_dev = tile_rep + tiles * RF_NODES;
+  int32_t* node_rep_off = tile_dev + tiles;
+  if (k <= 8)
+    return rbd_fast_launch<8>(ids, T, k, E, epd, epn, n_nodes, ppn, noff, ptok, pnode, pdev, roff, rexp, ap, counts,
+                              tile_cnt, tile_rep, tile_dev, node_rep_off, err, s);
+  if (k <= 16)
+    return rbd_fast_launch<16>(ids, T, k, E, epd, epn, n_nodes, ppn, noff, ptok, pnode, pdev, roff, rexp, ap, counts,
+                               tile_cnt, tile_rep, tile_dev, node_rep_off, err, s);
+  return rbd_fast_launch<32>(ids, T, k, E, epd, epn, n_nodes, ppn, noff, ptok, pnode, pdev, roff, rexp, ap, counts,
+                             tile_cnt, tile_rep, tile_dev, node_rep_off, err, s);
+}
+
 }  // namespace
 
 size_t csort_ws_bytes(long long n_max, int K) {
@@ -658,7 +900,14 @@ int pft_build_impl(const int32_t* ids, const float* w, int T, int E, int k, int3
   return PFMOE_OK;
 }
 
+// Workspace of the plan for maps of at most RF_NODES nodes: two [tiles][RF_NODES] arrays, one [tiles].
+static size_t rbd_fast_ws_bytes(int T) {
+  const size_t tiles = (static_cast<size_t>(T) + RF_TILE - 1) / RF_TILE;
+  return (2 * tiles * RF_NODES + tiles + 64) * sizeof(int32_t);
+}
+
 size_t rbd_ws_bytes(int T, int k, int n_nodes) {
+  if (n_nodes <= RF_NODES) return rbd_fast_ws_bytes(T);
   const long long pmax = static_cast<long long>(T) * (k < n_nodes ? k : n_nodes);
   const long long lt = long_scan_tiles(pmax > T ? pmax : T);
   const size_t ints = 3 * static_cast<size_t>(T) + 5 * static_cast<size_t>(pmax) + 2 * static_cast<size_t>(lt) + 128;
@@ -671,6 +920,9 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
                   void* ws, int32_t* err, cudaStream_t s) {
   const int epn = epd * dpn;
   const int n_nodes = E / epn;
+  if (n_nodes <= RF_NODES) return rbd_fast_impl(ids, T, k, E, epd, epn, n_nodes, pilots_per_node, node_offsets,
+                                                pilot_token, pilot_node, pilot_device, replica_offsets, replica_expert,
+                                                assign_pilot, counts, ws, err, s);
   const long long pmax = static_cast<long long>(T) * (k < n_nodes ? k : n_nodes);
   int32_t* p = static_cast<int32_t*>(ws);
   int32_t* ucount = p; p += T;

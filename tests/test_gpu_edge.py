@@ -170,3 +170,35 @@ def test_pft_and_rbd_large_chunks_match_oracle(E, k, epd, dpn):
     assert np.array_equal(i64(o["roff"][:P + 1]), r["replica_offsets"])
     assert np.array_equal(i64(o["rexp"]), r["replica_expert"])
     assert np.array_equal(i64(o["ap"]), r["assign_pilot"])
+
+
+@pytest.mark.gpu
+def test_rbd_many_nodes_general_path():
+    # 64 nodes: more than the per-token fast plan handles, so the sort-based plan runs.
+    from workloads.generate import make_topk_ids
+    T, E, k, epd, dpn = 5000, 256, 8, 2, 2
+    ids = make_topk_ids(T, E, k, seed=13, device="cuda")
+    n_nodes = E // (epd * dpn)
+    pmax = T * min(k, n_nodes)
+    i32 = dict(device="cuda", dtype=torch.int32)
+    o = dict(ppn=torch.empty(n_nodes, **i32), noff=torch.empty(n_nodes + 1, **i32), ptok=torch.empty(pmax, **i32),
+             pnode=torch.empty(pmax, **i32), pdev=torch.empty(pmax, **i32), roff=torch.empty(pmax + 1, **i32),
+             rexp=torch.empty(T * k, **i32), ap=torch.empty(T, k, **i32), cnt=torch.empty(2, **i32))
+    ws_b = L.rbd_plan_workspace_size(T, k, E, epd, dpn)
+    ws = torch.empty(ws_b, device="cuda", dtype=torch.uint8)
+    err = torch.zeros(1, **i32)
+    L.rbd_plan(ids, T, k, E, epd, dpn, o["ppn"], o["noff"], o["ptok"], o["pnode"], o["pdev"], o["roff"], o["rexp"],
+               o["ap"], o["cnt"], ws, ws_b, err)
+    torch.cuda.synchronize()
+    assert int(err) == 0
+    r = O.rbd_plan(i64(ids), E, epd, dpn)
+    P = r["num_pilots"]
+    assert int(o["cnt"][0]) == P and int(o["cnt"][1]) == r["num_token_device_pairs"]
+    assert np.array_equal(i64(o["ppn"]), r["pilots_per_node"])
+    assert np.array_equal(i64(o["noff"]), r["node_offsets"])
+    assert np.array_equal(i64(o["ptok"][:P]), r["pilot_token"])
+    assert np.array_equal(i64(o["pnode"][:P]), r["pilot_node"])
+    assert np.array_equal(i64(o["pdev"][:P]), r["pilot_device"])
+    assert np.array_equal(i64(o["roff"][:P + 1]), r["replica_offsets"])
+    assert np.array_equal(i64(o["rexp"]), r["replica_expert"])
+    assert np.array_equal(i64(o["ap"]), r["assign_pilot"])
