@@ -1529,8 +1529,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 // operands, one item per (column tile, row step), the B blocks cycling through the same
 // slots as a ring.  An expert with no rows gets NT items whose epilogue writes zeros.
 //
-// Roles (224 threads): warp 0 producer (lane 0: A, lane 1: B), warp 1 MMA issuer (even
-// CTA), warps 2..5 epilogue, warp 6 K-tail zeroing.  Every load lands on a barrier of its
+// Roles (256 threads): warp 0 A producer, warp 7 B producer, warp 1 MMA issuer (even CTA),
+// warps 2..5 epilogue, warp 6 K-tail zeroing.  Every load lands on a barrier of its
 // own CTA; each CTA's zeroing warp clears the rows past n_g of a segment's last 16-row
 // step and then arrives on the even CTA's ready barrier (two arrivals per phase), which
 // the MMA issuer waits on.  MMA commits reach both CTAs (free A stage / B slot, full
@@ -1583,8 +1583,10 @@ __device__ __forceinline__ void wg_zero_tail(uint32_t blk, int tail, int zero_ro
   asm volatile("fence.proxy.async;" ::: "memory");
 }
 
+constexpr int WG_THREADS = 256;   // 8 warps: A producer, MMA, 4 epilogue, K-tail zeroing, B producer
+
 template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS_KG, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(WG_THREADS, 1)
     wgrad_pair_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1629,7 +1631,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS_KG, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&acc_full[b]), 1);
-      mbar_init(smem_u32(&acc_empty[b]), 2 * 4 * 32);
+      mbar_init(smem_u32(&acc_empty[b]), 2 * 4);   // one arrival per epilogue warp of each CTA
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
@@ -1672,20 +1674,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS_KG, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int total = item_off[p.G];
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer (both CTAs)
-    if (lane < 2) {
-      uint32_t pending = 0, pend_parity = 0;   // A stages (lane 0) or B slots (lane 1) with a load issued
-      int q = 0;                               // loads issued by this lane
+  if (warp == 0 || warp == 7) {
+    // ------------------------------------------------------------ producers (both CTAs)
+    // Lane 0 of warp 0 loads the A blocks, lane 0 of warp 7 the B blocks.  The two walk different
+    // sequences (A every step, B once per resident item) and wait at different times, so they sit
+    // in different warps: spin-waits of two lanes of one warp on different barriers can starve one.
+    const bool is_a = warp == 0;
+    if (lane == 0) {
+      uint32_t pending = 0, pend_parity = 0;   // A stages or B slots with a load issued
+      int q = 0;                               // loads issued by this thread
       bool ok = true;
-      const int S = lane == 0 ? SA : SB;
-      uint64_t* fullv = lane == 0 ? full_a : full_b;
-      uint64_t* emptyv = lane == 0 ? empty_a : empty_b;
+      const int S = is_a ? SA : SB;
+      uint64_t* fullv = is_a ? full_a : full_b;
+      uint64_t* emptyv = is_a ? empty_a : empty_b;
       for (int t = pair; t < total && ok; t += npairs) {
         const WgItem it = wg_decode(p, item_off, t);
         if (it.n == 0) continue;
-        // lane 1: B blocks (once per resident item, per row step otherwise); lane 0: A blocks
-        const int reps = lane == 1 && it.resident ? 1 : it.p1 - it.p0;
+        // B blocks once per resident item, per row step otherwise; A blocks every row step
+        const int reps = !is_a && it.resident ? 1 : it.p1 - it.p0;
         for (int r = 0; r < reps && ok; ++r) {
           const int pstep = it.p0 + r;
           for (int kb = 0; kb < it.nkb; ++kb, ++q) {
@@ -1697,7 +1703,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS_KG, 1)
             pending |= 1u << s;
             pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
             const int krow = it.s0 + kb * BK;
-            if (lane == 0) {
+            if (is_a) {
               const uint32_t dst = smem_u32(a_area + s * WG_BLK);
               const int m0 = pstep * 2 * BM + static_cast<int>(rank) * BM;
               if (p.a_merged) {
@@ -1720,7 +1726,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS_KG, 1)
           }
         }
       }
-      // Drain: every load this lane issued has landed before the CTA may exit.
+      // Drain: every load this thread issued has landed before the CTA may exit.
       for (int s = 0; s < S; ++s)
         if (pending & (1u << s)) wait_bar2(smem_u32(&fullv[s]), (pend_parity >> s) & 1, abort_flag, p.err, false);
     }
@@ -1863,7 +1869,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS_KG, 1)
         const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * (2 * BM);
         epilogue_tile<EPI>(p, tl, tacc, q, lane, stg);
         tc_fence_before();
-        mbar_arrive_cluster(acc_empty_leader0 + 8u * buf);
+        __syncwarp();   // every lane's TMEM reads are done (tcgen05.wait::ld) before lane 0 frees the buffer
+        if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8u * buf);
       }
     }
     emit_drain(lane);
@@ -1947,7 +1954,7 @@ static int launch_wgrad_pair(Params& p, long long item_upper_bound, const char* 
   if (item_upper_bound <= 0) return PFMOE_OK;
   long long pairs = max_pairs();
   if (item_upper_bound < pairs) pairs = item_upper_bound;
-  PFMOE_LAUNCH(name, stream, (wgrad_pair_kernel<EPI><<<static_cast<int>(2 * pairs), THREADS_KG, smem, stream>>>(p)));
+  PFMOE_LAUNCH(name, stream, (wgrad_pair_kernel<EPI><<<static_cast<int>(2 * pairs), WG_THREADS, smem, stream>>>(p)));
   return PFMOE_OK;
 }
 

@@ -152,11 +152,12 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(const char* __restric
 }
 
 // y[t] = sum_j w[t, j] * O[pos[t, j]] ([A] §2.1.1 combine_weights), with bulk copies: warp 0's
-// lane 0 loads the k PFT row pieces (CB_PIECE bytes each) of a work item (token, piece) into a
-// ring stage; four consumer warps sum the stage in slot order in float32 (one 16-byte vector a
-// thread) and store the piece of y.  A token with an out-of-range row index is flagged and its
+// lane 0 loads the k PFT row pieces (at most CB_PIECE bytes each) of a work item (token, piece)
+// into a ring stage, and the warp posts the token's k weights beside it (a global load on the
+// consumers' path would stall every item); four consumer warps sum the stage in slot order in
+// float32 (one 16-byte vector a thread) and store the piece of y.  A token with an out-of-range row index is flagged and its
 // output row is left unwritten.
-constexpr int CB_PIECE = 2048;   // largest row piece a ring stage holds per slot: 128 threads x 16 bytes
+constexpr int CB_PIECE = 8192;   // largest row piece a ring stage holds per slot
 constexpr int CB_CONSUMERS = 128;
 
 template <typename T>
@@ -171,6 +172,7 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const c
   __shared__ __align__(8) uint64_t full[8];
   __shared__ __align__(8) uint64_t empty[8];
   __shared__ int valid[8];
+  __shared__ float sw[8][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long N = static_cast<long long>(Tn) * k;
   const long long items = static_cast<long long>(Tn) * pieces;
@@ -198,10 +200,12 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const c
       const int my_pos = lane < k ? pos[t * k + lane] : 0;
       const bool bad = lane < k && (my_pos < 0 || my_pos >= N);
       const bool any_bad = __any_sync(0xffffffffu, bad);
+      sw[s][lane] = lane < k ? w[t * k + lane] : 0.f;   // the weights travel with the stage
       if (lane == 0) {
         valid[s] = any_bad ? 0 : 1;
         if (any_bad && off == 0) dev_error(err, PFMOE_DEV_BAD_POS);
       }
+      __syncwarp();
       if (any_bad) {
         if (lane == 0) bar_arrive(smem_addr(&full[s]));
         __syncwarp();
@@ -224,7 +228,7 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const c
         if (pending & (1u << s)) bar_wait(smem_addr(&full[s]), (pend_parity >> s) & 1, err);
     __syncwarp();
   } else {
-    // ---- consumers: thread c sums bytes [16 c, 16 c + 16) of the piece
+    // ---- consumers: thread c sums the 16-byte vectors c, c + 128, ... of the piece
     const int c = threadIdx.x - 32;
     int q = 0;
     for (long long it = blockIdx.x; it < items; it += gridDim.x, ++q) {
@@ -233,19 +237,21 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const c
       const int bytes = min(piece, row_bytes - off);
       const int s = q % stages;
       if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&full[s]), (q / stages) & 1, err))) break;
-      if (valid[s] && c * 16 < bytes) {
-        float acc[VN];
+      if (valid[s]) {
+        for (int v = c; v * 16 < bytes; v += CB_CONSUMERS) {
+          float acc[VN];
 #pragma unroll
-        for (int i = 0; i < VN; ++i) acc[i] = 0.f;
-        const uint8_t* sp = csm + s * stage_bytes + c * 16;
-        for (int j = 0; j < k; ++j) {
-          const float wj = __ldg(w + t * k + j);
-          float o[VN];
-          load16(reinterpret_cast<const T*>(sp + j * piece), o);
+          for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+          const uint8_t* sp = csm + s * stage_bytes + v * 16;
+          for (int j = 0; j < k; ++j) {
+            const float wj = sw[s][j];
+            float o[VN];
+            load16(reinterpret_cast<const T*>(sp + j * piece), o);
 #pragma unroll
-          for (int i = 0; i < VN; ++i) acc[i] = fmaf(wj, o[i], acc[i]);
+            for (int i = 0; i < VN; ++i) acc[i] = fmaf(wj, o[i], acc[i]);
+          }
+          store16(reinterpret_cast<T*>(y + t * row_bytes + off + v * 16), acc);
         }
-        store16(reinterpret_cast<T*>(y + t * row_bytes + off + c * 16), acc);
       }
       bar_arrive(smem_addr(&empty[s]));
     }
@@ -356,22 +362,24 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bwd_bulk_kernel(
         const int s = q % stages;
         if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&full[s]), (q / stages) & 1, err))) { ok = false; break; }
         tok_valid = valid[s] != 0;
-        if (tok_valid && c16 * 16 < bytes) {
-          const uint8_t* sp = csm + s * stage_bytes + c16 * 16;
-          float a[VN];
-          load16(reinterpret_cast<const T*>(sp), a);
+        if (tok_valid) {
+          for (int v = c16; v * 16 < bytes; v += CB_CONSUMERS) {
+            const uint8_t* sp = csm + s * stage_bytes + v * 16;
+            float a[VN];
+            load16(reinterpret_cast<const T*>(sp), a);
 #pragma unroll
-          for (int j = 0; j < KM; ++j) {
-            if (j < k) {
-              float o[VN], dv[VN];
-              load16(reinterpret_cast<const T*>(sp + (j + 1) * piece), o);
-              const float wj = sw[s][j];
+            for (int j = 0; j < KM; ++j) {
+              if (j < k) {
+                float o[VN], dv[VN];
+                load16(reinterpret_cast<const T*>(sp + (j + 1) * piece), o);
+                const float wj = sw[s][j];
 #pragma unroll
-              for (int i = 0; i < VN; ++i) {
-                part[j] = fmaf(a[i], o[i], part[j]);
-                dv[i] = a[i] * wj;
+                for (int i = 0; i < VN; ++i) {
+                  part[j] = fmaf(a[i], o[i], part[j]);
+                  dv[i] = a[i] * wj;
+                }
+                store16(reinterpret_cast<T*>(dO + static_cast<long long>(spos[s][j]) * row_bytes + off + v * 16), dv);
               }
-              store16(reinterpret_cast<T*>(dO + static_cast<long long>(spos[s][j]) * row_bytes + off + c16 * 16), dv);
             }
           }
         }
@@ -501,25 +509,27 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) token_grad_bulk_kernel(
       const int bytes = min(piece, row_bytes - off);
       const int s = q % stages;
       if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&full[s]), (q / stages) & 1, err))) { ok = false; break; }
-      if (valid[s] && c16 * 16 < bytes) {
-        float acc[VN];
+      if (valid[s]) {
+        for (int vv = c16; vv * 16 < bytes; vv += CB_CONSUMERS) {
+          float acc[VN];
 #pragma unroll
-        for (int i = 0; i < VN; ++i) acc[i] = 0.f;
-        const uint8_t* sp = csm + s * stage_bytes + c16 * 16;
-        for (int j = 0; j < k; ++j) {
-          float v[VN];
-          load16(reinterpret_cast<const T*>(sp + j * piece), v);
+          for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+          const uint8_t* sp = csm + s * stage_bytes + vv * 16;
+          for (int j = 0; j < k; ++j) {
+            float v[VN];
+            load16(reinterpret_cast<const T*>(sp + j * piece), v);
 #pragma unroll
-          for (int i = 0; i < VN; ++i) acc[i] += v[i];
+            for (int i = 0; i < VN; ++i) acc[i] += v[i];
+          }
+          for (int j = 0; j < k; ++j) {
+            float v[VN];
+            load16(reinterpret_cast<const T*>(sp + (k + j) * piece), v);
+            const float dzj = sdz[s][j];
+#pragma unroll
+            for (int i = 0; i < VN; ++i) acc[i] = fmaf(dzj, v[i], acc[i]);
+          }
+          store16(reinterpret_cast<T*>(dx + t * row_bytes + off + vv * 16), acc);
         }
-        for (int j = 0; j < k; ++j) {
-          float v[VN];
-          load16(reinterpret_cast<const T*>(sp + (k + j) * piece), v);
-          const float dzj = sdz[s][j];
-#pragma unroll
-          for (int i = 0; i < VN; ++i) acc[i] = fmaf(dzj, v[i], acc[i]);
-        }
-        store16(reinterpret_cast<T*>(dx + t * row_bytes + off + c16 * 16), acc);
       }
       bar_arrive(smem_addr(&empty[s]));
     }
@@ -562,24 +572,27 @@ int launch_dispatch(const void* x, const int32_t* pos, int T, int k, int d, int 
 }
 
 
-// Ring geometry for `slots` row pieces per stage: pieces of CB_PIECE bytes, smaller where a stage
-// of that size would leave room for fewer than two stages in about 200 KB; about 96 KB of
-// stages (two CTAs per SM) where the pieces allow, between 2 and 8 stages.
+// Ring geometry for `slots` row pieces per stage.  The copy engine's cost per copy favours large
+// pieces, so a CTA takes about 200 KB (one per SM) in at least three stages, with pieces of up to
+// CB_PIECE bytes; rows narrower than a piece make smaller stages, and then up to eight of them.
 struct Ring {
-  int piece, pieces, stages;
+  int piece, pieces, stages, ctas_per_sm;
   size_t smem;
 };
 static Ring ring_for(int row_bytes, int slots) {
+  constexpr int kBudget = 200 * 1024;
   Ring r;
-  r.piece = CB_PIECE;
-  const int cap = (100 * 1024 / slots) & ~15;
-  if (r.piece > cap) r.piece = cap;
+  int cap = (kBudget / (3 * slots)) & ~15;
+  if (cap < 16) cap = 16;
+  r.piece = CB_PIECE < cap ? CB_PIECE : cap;
+  if (r.piece > row_bytes) r.piece = row_bytes;     // row_bytes is a multiple of 16
   r.pieces = (row_bytes + r.piece - 1) / r.piece;
   const int stage = slots * r.piece;
-  r.stages = (96 * 1024) / stage;
+  r.stages = kBudget / stage;
   if (r.stages > 8) r.stages = 8;
   if (r.stages < 2) r.stages = 2;
   r.smem = static_cast<size_t>(r.stages) * stage;
+  r.ctas_per_sm = r.smem <= 100 * 1024 ? 2 : 1;
   return r;
 }
 
@@ -588,7 +601,7 @@ int launch_combine(const void* out, const int32_t* pos, const float* w, int T, i
   const int row_bytes = d * (dtype == PFMOE_BF16 ? 2 : 4);
   const Ring r = ring_for(row_bytes, k);
   const long long items = static_cast<long long>(T) * r.pieces;
-  long long grid = static_cast<long long>(num_sms()) * 2;
+  long long grid = static_cast<long long>(num_sms()) * r.ctas_per_sm;
   if (grid > items) grid = items;
   if (dtype == PFMOE_BF16) {
     PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&combine_bulk_kernel<__nv_bfloat16>), 227 * 1024, "combine"));
@@ -621,7 +634,7 @@ int launch_combine_bwd(const void* dy, const void* out, const int32_t* pos, cons
                        int dtype, void* dO, float* g, int32_t* err, cudaStream_t s) {
   const int row_bytes = d * (dtype == PFMOE_BF16 ? 2 : 4);
   const Ring r = ring_for(row_bytes, k + 1);
-  long long grid = static_cast<long long>(num_sms()) * 2;
+  long long grid = static_cast<long long>(num_sms()) * r.ctas_per_sm;
   if (grid > T) grid = T;
   const int gr = static_cast<int>(grid);
   if (dtype == PFMOE_BF16) {
@@ -653,7 +666,7 @@ int launch_token_grad(const void* dx_pft, const int32_t* pos, const float* g, co
                       void* dz_bf16, int32_t* err, cudaStream_t s) {
   const int row_bytes = d * (dtype == PFMOE_BF16 ? 2 : 4);
   const Ring r = ring_for(row_bytes, 2 * k);
-  long long grid = static_cast<long long>(num_sms()) * 2;
+  long long grid = static_cast<long long>(num_sms()) * r.ctas_per_sm;
   if (grid > T) grid = T;
   auto* dzb = static_cast<__nv_bfloat16*>(dz_bf16);
   if (dtype == PFMOE_BF16) {
