@@ -573,14 +573,24 @@ __global__ void rbd_final_kernel(const int32_t* ids, int T, int k, int E, int ep
 constexpr int RF_NODES = 8;
 constexpr int RF_TILE = 256;
 
+// The tile's ids ([RF_TILE][k] consecutive ints) are staged in shared memory with coalesced loads;
+// each thread then reads its token's k ids from there.
+__device__ __forceinline__ void rf_stage_ids(const int32_t* __restrict__ ids, int T, int k, int32_t* sids) {
+  const long long base = static_cast<long long>(blockIdx.x) * RF_TILE * k;
+  const long long end = static_cast<long long>(T) * k;
+  for (int i = threadIdx.x; i < RF_TILE * k; i += blockDim.x)
+    sids[i] = base + i < end ? ids[base + i] : 0;
+  __syncthreads();
+}
+
 template <int KM>
-__device__ __forceinline__ void rf_load(const int32_t* __restrict__ ids, long long t, bool valid, int k, int E, int epn,
+__device__ __forceinline__ void rf_load(const int32_t* __restrict__ sids, bool valid, int k, int E, int epn,
                                         int (&e)[KM], int (&nd)[KM], int32_t* err) {
 #pragma unroll
   for (int j = 0; j < KM; ++j) {
     int v = 0;
     if (valid && j < k) {
-      v = ids[t * k + j];
+      v = sids[threadIdx.x * k + j];
       if (static_cast<unsigned>(v) >= static_cast<unsigned>(E)) {
         dev_error(err, PFMOE_DEV_BAD_EXPERT_ID);
         v = 0;
@@ -609,11 +619,13 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_count_kernel(const int32_t* 
                                                                  int epd, int epn, int32_t* __restrict__ tile_cnt,
                                                                  int32_t* __restrict__ tile_dev, int32_t* err) {
   __shared__ int red[RF_TILE / 32][RF_NODES + 1];
+  __shared__ int32_t sids[RF_TILE * KM];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long t = static_cast<long long>(blockIdx.x) * RF_TILE + threadIdx.x;
   const bool valid = t < T;
   int e[KM], nd[KM], c[RF_NODES];
-  rf_load<KM>(ids, t, valid, k, E, epn, e, nd, err);
+  rf_stage_ids(ids, T, k, sids);
+  rf_load<KM>(sids, valid, k, E, epn, e, nd, err);
   rf_counts<KM>(nd, c);
   int dc = 0;   // distinct devices of the token
 #pragma unroll
@@ -642,54 +654,99 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_count_kernel(const int32_t* 
   }
 }
 
-// One CTA: warp n scans node n's packed tile counts into exclusive token bases (in place) and
-// replica bases (tile_rep_base); then the node offsets, P and the distinct (token, device) total.
-__global__ void __launch_bounds__(256) rbd_fast_scan_kernel(int ntiles, int n_nodes, int32_t* __restrict__ tile_cnt,
-                                                            int32_t* __restrict__ tile_rep_base,
-                                                            const int32_t* __restrict__ tile_dev,
-                                                            int32_t* pilots_per_node, int32_t* node_offsets,
-                                                            int32_t* node_rep_off, int32_t* counts,
-                                                            int32_t* replica_offsets) {
-  __shared__ int tot_tok[RF_NODES], tot_rep[RF_NODES];
-  __shared__ int dsum[8];
+// One CTA of 512 threads: thread i takes a run of consecutive tiles (all loaded up front), the
+// runs are scanned per node across the block, and each thread writes its tiles' exclusive token
+// bases (in place) and replica bases (tile_rep_base); then the node offsets, P and the distinct
+// (token, device) total.  Tiles beyond 512 runs' worth are handled in further passes.
+constexpr int RF_SCAN_THREADS = 512;
+constexpr int RF_RUN = 4;   // tiles per thread per pass
+
+__global__ void __launch_bounds__(RF_SCAN_THREADS) rbd_fast_scan_kernel(int ntiles, int n_nodes,
+                                                                        int32_t* __restrict__ tile_cnt,
+                                                                        int32_t* __restrict__ tile_rep_base,
+                                                                        const int32_t* __restrict__ tile_dev,
+                                                                        int32_t* pilots_per_node, int32_t* node_offsets,
+                                                                        int32_t* node_rep_off, int32_t* counts,
+                                                                        int32_t* replica_offsets) {
+  __shared__ int wt[RF_SCAN_THREADS / 32][RF_NODES], wr[RF_SCAN_THREADS / 32][RF_NODES];
+  __shared__ int carry_t[RF_NODES], carry_r[RF_NODES];
+  __shared__ int dsum[RF_SCAN_THREADS / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (warp < n_nodes) {
-    int ct = 0, cr = 0;   // running totals (unpacked: node totals can exceed 16 bits)
-    for (int i0 = 0; i0 < ntiles; i0 += 32) {
-      const int i = i0 + lane;
-      const int v = i < ntiles ? tile_cnt[static_cast<long long>(i) * RF_NODES + warp] : 0;
-      int a = v & 0xffff, b = v >> 16;
+  if (threadIdx.x < RF_NODES) { carry_t[threadIdx.x] = 0; carry_r[threadIdx.x] = 0; }
+  int ds = 0;
+  __syncthreads();
+  for (int base = 0; base < ntiles; base += RF_SCAN_THREADS * RF_RUN) {
+    const int t0 = base + threadIdx.x * RF_RUN;
+    int v[RF_RUN][RF_NODES];
+#pragma unroll
+    for (int r = 0; r < RF_RUN; ++r) {
+      const bool ok = t0 + r < ntiles;
+#pragma unroll
+      for (int n = 0; n < RF_NODES; ++n)
+        v[r][n] = ok && n < n_nodes ? tile_cnt[static_cast<long long>(t0 + r) * RF_NODES + n] : 0;
+      if (ok) ds += tile_dev[t0 + r];
+    }
+    int run_t[RF_NODES], run_r[RF_NODES], ex_t[RF_NODES], ex_r[RF_NODES];
+#pragma unroll
+    for (int n = 0; n < RF_NODES; ++n) {
+      run_t[n] = 0;
+      run_r[n] = 0;
+#pragma unroll
+      for (int r = 0; r < RF_RUN; ++r) { run_t[n] += v[r][n] & 0xffff; run_r[n] += v[r][n] >> 16; }
+      int a = run_t[n], b = run_r[n];
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int ya = __shfl_up_sync(0xffffffffu, a, o);
         const int yb = __shfl_up_sync(0xffffffffu, b, o);
         if (lane >= o) { a += ya; b += yb; }
       }
-      const int ea = a - (v & 0xffff), eb = b - (v >> 16);
-      if (i < ntiles) {   // exclusive bases, unpacked (node totals exceed 16 bits)
-        tile_cnt[static_cast<long long>(i) * RF_NODES + warp] = ct + ea;
-        tile_rep_base[static_cast<long long>(i) * RF_NODES + warp] = cr + eb;
-      }
-      ct += __shfl_sync(0xffffffffu, a, 31);
-      cr += __shfl_sync(0xffffffffu, b, 31);
+      ex_t[n] = a - run_t[n];
+      ex_r[n] = b - run_r[n];
+      if (lane == 31) { wt[warp][n] = a; wr[warp][n] = b; }
     }
-    if (lane == 0) { tot_tok[warp] = ct; tot_rep[warp] = cr; }
+    __syncthreads();
+    // warp totals -> warp offsets (warp 0, one lane per node), plus the carry from earlier passes
+    if (warp == 0 && lane < RF_NODES) {
+      int st = carry_t[lane], sr = carry_r[lane];
+      for (int w = 0; w < RF_SCAN_THREADS / 32; ++w) {
+        const int xt = wt[w][lane], xr = wr[w][lane];
+        wt[w][lane] = st;
+        wr[w][lane] = sr;
+        st += xt;
+        sr += xr;
+      }
+      carry_t[lane] = st;
+      carry_r[lane] = sr;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int n = 0; n < RF_NODES; ++n) {
+      int at = wt[warp][n] + ex_t[n], ar = wr[warp][n] + ex_r[n];
+#pragma unroll
+      for (int r = 0; r < RF_RUN; ++r) {
+        if (t0 + r < ntiles && n < n_nodes) {
+          tile_cnt[static_cast<long long>(t0 + r) * RF_NODES + n] = at;
+          tile_rep_base[static_cast<long long>(t0 + r) * RF_NODES + n] = ar;
+        }
+        at += v[r][n] & 0xffff;
+        ar += v[r][n] >> 16;
+      }
+    }
+    __syncthreads();   // wt / wr are rewritten by the next pass
   }
-  int ds = 0;
-  for (int i = threadIdx.x; i < ntiles; i += blockDim.x) ds += tile_dev[i];
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
   if (lane == 0) dsum[warp] = ds;
   __syncthreads();
   if (threadIdx.x == 0) {
     int off = 0, roff = 0, dtot = 0;
-    for (int w = 0; w < 8; ++w) dtot += dsum[w];
+    for (int w = 0; w < RF_SCAN_THREADS / 32; ++w) dtot += dsum[w];
     for (int n = 0; n < n_nodes; ++n) {
       node_offsets[n] = off;
-      pilots_per_node[n] = tot_tok[n];
+      pilots_per_node[n] = carry_t[n];
       node_rep_off[n] = roff;
-      off += tot_tok[n];
-      roff += tot_rep[n];
+      off += carry_t[n];
+      roff += carry_r[n];
     }
     node_offsets[n_nodes] = off;
     counts[0] = off;
@@ -706,11 +763,13 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_emit_kernel(
     int32_t* __restrict__ pilot_node, int32_t* __restrict__ pilot_device, int32_t* __restrict__ replica_offsets,
     int32_t* __restrict__ replica_expert, int32_t* __restrict__ assign_pilot, int32_t* err) {
   __shared__ int wsum[RF_TILE / 32][RF_NODES];
+  __shared__ int32_t sids[RF_TILE * KM];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long t = static_cast<long long>(blockIdx.x) * RF_TILE + threadIdx.x;
   const bool valid = t < T;
   int e[KM], nd[KM], c[RF_NODES], ex[RF_NODES];
-  rf_load<KM>(ids, t, valid, k, E, epn, e, nd, nullptr);   // rbd_fast_count flagged bad ids
+  rf_stage_ids(ids, T, k, sids);
+  rf_load<KM>(sids, valid, k, E, epn, e, nd, nullptr);   // rbd_fast_count flagged bad ids
   rf_counts<KM>(nd, c);
   // in-warp exclusive prefix of the packed counts, per node
 #pragma unroll
@@ -850,8 +909,8 @@ static int rbd_fast_launch(const int32_t* ids, int T, int k, int E, int epd, int
                  (rbd_fast_count_kernel<KM><<<ntiles, RF_TILE, 0, s>>>(ids, T, k, E, epd, epn, tile_cnt, tile_dev,
                                                                       err)));
   PFMOE_LAUNCH("rbd_scan_nodes", s,
-               (rbd_fast_scan_kernel<<<1, 256, 0, s>>>(ntiles, n_nodes, tile_cnt, tile_rep, tile_dev, ppn, noff,
-                                                       node_rep_off, counts, roff)));
+               (rbd_fast_scan_kernel<<<1, RF_SCAN_THREADS, 0, s>>>(ntiles, n_nodes, tile_cnt, tile_rep, tile_dev, ppn,
+                                                                   noff, node_rep_off, counts, roff)));
   if (ntiles > 0)
     PFMOE_LAUNCH("rbd_emit", s,
                (rbd_fast_emit_kernel<KM><<<ntiles, RF_TILE, 0, s>>>(ids, T, k, E, epd, epn, n_nodes, tile_cnt, tile_rep,
