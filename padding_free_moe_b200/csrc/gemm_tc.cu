@@ -81,7 +81,6 @@ struct Params {
   int G;
   int dense_len;
   int stages;
-  int sb_slots;      // pair weight-gradient kernel: 64-row B blocks each CTA holds (resident or ring)
   int ksplit;        // dense problems only: K is cut into ksplit parts, part s writes output slice s
   int kchunk;        // KG dense: K rows per part (multiple of KG_BK)
   void* D0;
@@ -1511,380 +1510,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 }
 
 
-// ============================================================================
-// Weight gradients on CTA pairs (cta_group::2) with a resident B operand.
-//
-// dW_g[M, Nout] = XA_g^T XB_g, the reduction running over expert g's PFT rows
-// [seg[g], seg[g+1]) (n_g rows; X-MoE article §2.1.2: one GEMM per expert over its
-// unpadded rows).  XA [rows, M] and XB [rows, Nout] are both MN-major operands.  A pair
-// tile is 256 output rows (128 per CTA: TMEM lanes) by 256 output columns; each CTA
-// holds 128 of the columns of XB_g in shared memory (with nsplit: CTA 0 the dH1
-// columns, CTA 1 the dH3 columns of the same 128-column tile).
-//
-// Work items: an expert whose rows fit the B region (sb_slots blocks of 64 rows) is cut
-// into NT items, one per 256-column tile; such an item loads its XB_g columns once and
-// keeps them while XA_g^T streams through the A ring for every 256-row step of M.  Per
-// output byte a CTA then reads about n_g / 256 bytes of XA_g instead of three times that
-// with both operands streamed per output tile.  An expert with more rows streams both
-// operands, one item per (column tile, row step), the B blocks cycling through the same
-// slots as a ring.  An expert with no rows gets NT items whose epilogue writes zeros.
-//
-// Roles (256 threads): warp 0 A producer, warp 7 B producer, warp 1 MMA issuer (even CTA),
-// warps 2..5 epilogue, warp 6 K-tail zeroing.  Every load lands on a barrier of its
-// own CTA; each CTA's zeroing warp clears the rows past n_g of a segment's last 16-row
-// step and then arrives on the even CTA's ready barrier (two arrivals per phase), which
-// the MMA issuer waits on.  MMA commits reach both CTAs (free A stage / B slot, full
-// accumulator); both CTAs' epilogues arrive on the even CTA's acc_empty.  Items are
-// handed to pairs round-robin in expert order, so the pairs working on one expert at the
-// same time share its XA rows in L2.
-constexpr int WG_BLK = 128 * BK * 2;   // one 64-row block of 128 MN-major columns (two 64-wide boxes): 16 KB
-constexpr int WG_MAX_A = 8;
-constexpr int WG_MAX_B = 16;
-
-struct WgItem {
-  int g, j, p0, p1, s0, n, nkb;
-  bool resident;
-};
-
-__device__ __forceinline__ int wg_col_tiles(const Params& p) { return (p.Nout + n_step(p) - 1) / n_step(p); }
-__device__ __forceinline__ int wg_row_steps(const Params& p) { return (p.M + 2 * BM - 1) / (2 * BM); }
-
-__device__ __forceinline__ WgItem wg_decode(const Params& p, const int* item_off, int t) {
-  int lo = 0, hi = p.G - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (item_off[mid] <= t) lo = mid; else hi = mid - 1;
-  }
-  WgItem it;
-  it.g = lo;
-  it.s0 = p.seg[lo];
-  it.n = max(0, p.seg[lo + 1] - it.s0);
-  it.nkb = (it.n + BK - 1) / BK;
-  it.resident = it.nkb <= p.sb_slots;   // also true for an empty expert
-  const int local = t - item_off[lo];
-  const int MP = wg_row_steps(p);
-  if (it.resident) {
-    it.j = local;
-    it.p0 = 0;
-    it.p1 = MP;
-  } else {
-    it.j = local / MP;
-    it.p0 = local - it.j * MP;
-    it.p1 = it.p0 + 1;
-  }
-  return it;
-}
-
-// Rows past the segment end in the last 16-row step of a block: [tail, tail + zero_rows).
-__device__ __forceinline__ void wg_zero_tail(uint32_t blk, int tail, int zero_rows, int lane) {
-  const int chunks = zero_rows * 8;   // 16-byte chunks per 64-wide box
-  for (int b = 0; b < 2; ++b)
-    for (int i = lane; i < chunks; i += 32) st_shared16(blk + b * (BK * 128) + tail * 128 + i * 16, make_uint4(0, 0, 0, 0));
-  asm volatile("fence.proxy.async;" ::: "memory");
-}
-
-constexpr int WG_THREADS = 256;   // 8 warps: A producer, MMA, 4 epilogue, K-tail zeroing, B producer
-
-template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(WG_THREADS, 1)
-    wgrad_pair_kernel(const __grid_constant__ Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int SA = p.stages, SB = p.sb_slots;
-  uint8_t* a_area = smem;
-  uint8_t* b_area = a_area + SA * WG_BLK;
-  uint8_t* stage_area = b_area + SB * WG_BLK;
-  int* item_off = reinterpret_cast<int*>(stage_area + 4 * STAGE_BUFS * STAGE_BYTES_PER_WARP);
-  const int ioff_ints = (p.G + 1 + 63) & ~63;
-  uint64_t* full_a = reinterpret_cast<uint64_t*>(item_off + ioff_ints);
-  uint64_t* empty_a = full_a + WG_MAX_A;
-  uint64_t* ready_a = empty_a + WG_MAX_A;
-  uint64_t* full_b = ready_a + WG_MAX_A;
-  uint64_t* empty_b = full_b + WG_MAX_B;
-  uint64_t* ready_b = empty_b + WG_MAX_B;
-  uint64_t* acc_full = ready_b + WG_MAX_B;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_rank();
-  const bool leader = rank == 0;
-  const int pair = blockIdx.x >> 1;
-  const int npairs = gridDim.x >> 1;
-  constexpr uint32_t tmem_cols = 512;   // two 256-column accumulators
-  const int NT = wg_col_tiles(p);
-  const int MP = wg_row_steps(p);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < WG_MAX_A; ++s) {
-      mbar_init(smem_u32(&full_a[s]), 1);
-      mbar_init(smem_u32(&empty_a[s]), 1);
-      mbar_init(smem_u32(&ready_a[s]), 2);
-    }
-    for (int s = 0; s < WG_MAX_B; ++s) {
-      mbar_init(smem_u32(&full_b[s]), 1);
-      mbar_init(smem_u32(&empty_b[s]), 1);
-      mbar_init(smem_u32(&ready_b[s]), 2);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&acc_full[b]), 1);
-      mbar_init(smem_u32(&acc_empty[b]), 2 * 4);   // one arrival per epilogue warp of each CTA
-    }
-    mbar_init(smem_u32(drain), 1);
-    *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  }
-  // Prefix over experts of their work items (NT, or NT * MP when both operands stream).
-  if (warp == 0) {
-    int carry = 0;
-    for (int base = 0; base < p.G; base += 32) {
-      const int e = base + lane;
-      int ni = 0;
-      if (e < p.G) {
-        const int n = max(0, p.seg[e + 1] - p.seg[e]);
-        ni = (n + BK - 1) / BK <= p.sb_slots ? NT : NT * MP;
-      }
-      int x = ni;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      if (e < p.G) item_off[e] = carry + x - ni;
-      carry += __shfl_sync(0xffffffffu, x, 31);
-    }
-    if (lane == 0) item_off[p.G] = carry;
-    if (lane == 0) {
-      prefetch_tmap(&p.tmA[0]);
-      prefetch_tmap(&p.tmB[0]);
-    }
-  }
-  if (warp == 1) {
-    tmem_alloc2(smem_u32(tmem_slot), tmem_cols);
-    tmem_relinquish2();
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  const int total = item_off[p.G];
-
-  if (warp == 0 || warp == 7) {
-    // ------------------------------------------------------------ producers (both CTAs)
-    // Lane 0 of warp 0 loads the A blocks, lane 0 of warp 7 the B blocks.  The two walk different
-    // sequences (A every step, B once per resident item) and wait at different times, so they sit
-    // in different warps: spin-waits of two lanes of one warp on different barriers can starve one.
-    const bool is_a = warp == 0;
-    if (lane == 0) {
-      uint32_t pending = 0, pend_parity = 0;   // A stages or B slots with a load issued
-      int q = 0;                               // loads issued by this thread
-      bool ok = true;
-      const int S = is_a ? SA : SB;
-      uint64_t* fullv = is_a ? full_a : full_b;
-      uint64_t* emptyv = is_a ? empty_a : empty_b;
-      for (int t = pair; t < total && ok; t += npairs) {
-        const WgItem it = wg_decode(p, item_off, t);
-        if (it.n == 0) continue;
-        // B blocks once per resident item, per row step otherwise; A blocks every row step
-        const int reps = !is_a && it.resident ? 1 : it.p1 - it.p0;
-        for (int r = 0; r < reps && ok; ++r) {
-          const int pstep = it.p0 + r;
-          for (int kb = 0; kb < it.nkb; ++kb, ++q) {
-            const int s = q % S;
-            const uint32_t ph = (q / S) & 1;
-            if (!wait_bar2(smem_u32(&emptyv[s]), ph ^ 1, abort_flag, p.err)) { ok = false; break; }
-            const uint32_t fb = smem_u32(&fullv[s]);
-            mbar_expect_tx(fb, WG_BLK);
-            pending |= 1u << s;
-            pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
-            const int krow = it.s0 + kb * BK;
-            if (is_a) {
-              const uint32_t dst = smem_u32(a_area + s * WG_BLK);
-              const int m0 = pstep * 2 * BM + static_cast<int>(rank) * BM;
-              if (p.a_merged) {
-                tma_load_4d(dst, &p.tmA[0], fb, 0, krow, m0 / 64, 0);
-              } else {
-                tma_load_3d(dst, &p.tmA[0], fb, m0, krow, 0);
-                tma_load_3d(dst + BK * 128, &p.tmA[0], fb, m0 + 64, krow, 0);
-              }
-            } else {
-              const uint32_t dst = smem_u32(b_area + s * WG_BLK);
-              const CUtensorMap* tb = &p.tmB[p.nsplit ? rank : 0];
-              const int c0 = p.nsplit ? it.j * BM : it.j * 2 * BM + static_cast<int>(rank) * BM;
-              if (p.b_merged) {
-                tma_load_4d(dst, tb, fb, 0, krow, c0 / 64, 0);
-              } else {
-                tma_load_3d(dst, tb, fb, c0, krow, 0);
-                tma_load_3d(dst + BK * 128, tb, fb, c0 + 64, krow, 0);
-              }
-            }
-          }
-        }
-      }
-      // Drain: every load this thread issued has landed before the CTA may exit.
-      for (int s = 0; s < S; ++s)
-        if (pending & (1u << s)) wait_bar2(smem_u32(&fullv[s]), (pend_parity >> s) & 1, abort_flag, p.err, false);
-    }
-  } else if (warp == 6) {
-    // ------------------------------------------------------------ K-tail zeroing (both CTAs)
-    int qa = 0, qb = 0;
-    bool ok = true;
-    const uint32_t ready_a0 = mapa_shared(smem_u32(&ready_a[0]), 0);
-    const uint32_t ready_b0 = mapa_shared(smem_u32(&ready_b[0]), 0);
-    auto pass = [&](bool is_b, int kb, const WgItem& it) -> bool {
-      const int S = is_b ? SB : SA;
-      int& qq = is_b ? qb : qa;
-      const int s = qq % S;
-      const uint32_t ph = (qq / S) & 1;
-      ++qq;
-      if (!__all_sync(0xffffffffu, wait_bar2(smem_u32(is_b ? &full_b[s] : &full_a[s]), ph, abort_flag, p.err)))
-        return false;
-      const int tail = it.n - (it.nkb - 1) * BK;          // rows of the last block, 1..64
-      const int zero_rows = ((tail + 15) & ~15) - tail;
-      if (kb == it.nkb - 1 && zero_rows > 0)
-        wg_zero_tail(smem_u32((is_b ? b_area : a_area) + s * WG_BLK), tail, zero_rows, lane);
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster((is_b ? ready_b0 : ready_a0) + 8u * s);
-      return true;
-    };
-    for (int t = pair; t < total && ok; t += npairs) {
-      const WgItem it = wg_decode(p, item_off, t);
-      if (it.n == 0) continue;
-      if (it.resident)
-        for (int kb = 0; kb < it.nkb && ok; ++kb) ok = pass(true, kb, it);
-      for (int ps = it.p0; ps < it.p1 && ok; ++ps)
-        for (int kb = 0; kb < it.nkb && ok; ++kb) {
-          if (!it.resident) ok = pass(true, kb, it);
-          if (ok) ok = pass(false, kb, it);
-        }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (even CTA)
-    if (leader) {
-      const uint32_t idesc = idesc_bf16(2 * BM, 2 * BM, 1, 1);
-      int qa = 0, qb = 0, acc = 0;
-      bool ok = true;
-      for (int t = pair; t < total && ok; t += npairs) {
-        const WgItem it = wg_decode(p, item_off, t);
-        if (it.n == 0) {
-          for (int ps = it.p0; ps < it.p1 && ok; ++ps, ++acc) {
-            const int buf = acc & 1;
-            ok = __all_sync(0xffffffffu, wait_bar2(smem_u32(&acc_empty[buf]), ((acc >> 1) & 1) ^ 1, abort_flag, p.err));
-            if (!ok) break;
-            if (lane == 0) tc_commit2_both(smem_u32(&acc_full[buf]));   // nothing to wait for: zeros
-            __syncwarp();
-          }
-          continue;
-        }
-        const int tail = it.n - (it.nkb - 1) * BK;
-        const int last_kk = ((tail + 15) & ~15) / 16;
-        const int qb0 = qb;
-        if (it.resident) {
-          for (int kb = 0; kb < it.nkb && ok; ++kb) {
-            const int sl = (qb0 + kb) % SB;
-            ok = __all_sync(0xffffffffu, wait_bar2(smem_u32(&ready_b[sl]), ((qb0 + kb) / SB) & 1, abort_flag, p.err));
-          }
-          qb += it.nkb;
-        }
-        for (int ps = it.p0; ps < it.p1 && ok; ++ps, ++acc) {
-          const int buf = acc & 1;
-          ok = __all_sync(0xffffffffu, wait_bar2(smem_u32(&acc_empty[buf]), ((acc >> 1) & 1) ^ 1, abort_flag, p.err));
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t tmem_d = tmem_base + buf * (2 * BM);
-          const bool last_step = ps == it.p1 - 1;
-          for (int kb = 0; kb < it.nkb; ++kb) {
-            int sl;
-            if (it.resident) {
-              sl = (qb0 + kb) % SB;
-            } else {
-              sl = qb % SB;
-              ok = __all_sync(0xffffffffu, wait_bar2(smem_u32(&ready_b[sl]), (qb / SB) & 1, abort_flag, p.err));
-              ++qb;
-              if (!ok) break;
-            }
-            const int s = qa % SA;
-            ok = __all_sync(0xffffffffu, wait_bar2(smem_u32(&ready_a[s]), (qa / SA) & 1, abort_flag, p.err));
-            ++qa;
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t sa = smem_u32(a_area + s * WG_BLK);
-            const uint32_t sb = smem_u32(b_area + sl * WG_BLK);
-            const int kk_count = kb == it.nkb - 1 ? last_kk : BK / 16;
-            if (lane == 0) {
-              for (int kk = 0; kk < kk_count; ++kk) {
-                const uint64_t ad = sdesc(sa + kk * 2048, BK * 128, 1024);
-                const uint64_t bd = sdesc(sb + kk * 2048, BK * 128, 1024);
-                tc_mma2(tmem_d, ad, bd, idesc, (kb | kk) != 0);
-              }
-              tc_commit2_both(smem_u32(&empty_a[s]));
-              // A streamed B block is free after its own MMAs; a resident one after the item's
-              // last row step has used it (so the next item's B can load during that step).
-              if (!it.resident || last_step) tc_commit2_both(smem_u32(&empty_b[sl]));
-            }
-            __syncwarp();
-          }
-          if (!ok) break;
-          if (lane == 0) tc_commit2_both(smem_u32(&acc_full[buf]));
-          __syncwarp();
-        }
-      }
-      if (lane == 0) {
-        tc_commit2_both(smem_u32(drain));
-        wait_bar2(smem_u32(drain), 0, abort_flag, p.err, false);
-      }
-      __syncwarp();
-    }
-  } else {
-    // ------------------------------------------------------------ epilogue (both CTAs)
-    const int q = warp & 3;
-    const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
-    Stager stg{smem_u32(stage_area + (warp - 2) * STAGE_BUFS * STAGE_BYTES_PER_WARP), 0};
-    int acc = 0;
-    bool ok = true;
-    for (int t = pair; t < total && ok; t += npairs) {
-      const WgItem it = wg_decode(p, item_off, t);
-      for (int ps = it.p0; ps < it.p1; ++ps, ++acc) {
-        const int buf = acc & 1;
-        if (!__all_sync(0xffffffffu, wait_bar2(smem_u32(&acc_full[buf]), (acc >> 1) & 1, abort_flag, p.err))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        Tile tl;
-        tl.g = it.g;
-        tl.row0 = ps * 2 * BM + static_cast<int>(rank) * BM;
-        tl.rows = min(BM, p.M - tl.row0);
-        tl.n0 = it.j * n_step(p);
-        tl.nk = it.n > 0 ? 1 : 0;
-        tl.krow0 = it.s0;
-        tl.kvalid = 0;
-        tl.kb0 = 0;
-        tl.split = 0;
-        const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * (2 * BM);
-        epilogue_tile<EPI>(p, tl, tacc, q, lane, stg);
-        tc_fence_before();
-        __syncwarp();   // every lane's TMEM reads are done (tcgen05.wait::ld) before lane 0 frees the buffer
-        if (lane == 0) mbar_arrive_cluster(acc_empty_leader0 + 8u * buf);
-      }
-    }
-    emit_drain(lane);
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc2(tmem_base, tmem_cols);
-  }
-}
-
 template <int EPI, int MODE, int KBK = BK>
 static int launch(Params& p, long long tile_upper_bound, const char* name, cudaStream_t stream) {
   p.mode = MODE;
@@ -1933,30 +1558,6 @@ static int launch_tn(Params& p, long long pair_tile_upper_bound, const char* nam
   return PFMOE_OK;
 }
 
-
-// Pair weight-gradient launcher: four 16 KB A stages and as many 16 KB B blocks as the rest of
-// shared memory holds (seven at 227 KB), at most WG_MAX_B.
-template <int EPI>
-static int launch_wgrad_pair(Params& p, long long item_upper_bound, const char* name, cudaStream_t stream) {
-  p.mode = KG;
-  p.bn = 2 * BM;
-  const int ioff = ((p.G + 1 + 63) & ~63) * 4;
-  const int bars = (3 * WG_MAX_A + 3 * WG_MAX_B + 5) * 8 + 16;
-  const int fixed = 1024 + ioff + ((bars + 127) & ~127) + 4 * STAGE_BUFS * STAGE_BYTES_PER_WARP;
-  int sa = 4;
-  int sb = (SMEM_LIMIT - fixed) / WG_BLK - sa;
-  if (sb > WG_MAX_B) sb = WG_MAX_B;
-  if (sb < 2) return fail(PFMOE_ERR_UNSUPPORTED, std::string(name) + ": too many experts for the shared-memory plan");
-  p.stages = sa;
-  p.sb_slots = sb;
-  const size_t smem = fixed + static_cast<size_t>(sa + sb) * WG_BLK;
-  PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&wgrad_pair_kernel<EPI>), SMEM_LIMIT, name));
-  if (item_upper_bound <= 0) return PFMOE_OK;
-  long long pairs = max_pairs();
-  if (item_upper_bound < pairs) pairs = item_upper_bound;
-  PFMOE_LAUNCH(name, stream, (wgrad_pair_kernel<EPI><<<static_cast<int>(2 * pairs), WG_THREADS, smem, stream>>>(p)));
-  return PFMOE_OK;
-}
 
 // Token-tile upper bound of the token-as-N kernel: sum_e ceil(n_e / 256) <= N / 256 + E.
 static long long tn_tiles_ub(int N, int E, int F, int fstep) {
@@ -2120,11 +1721,13 @@ int tc_ffn_dgrad_x(const void* dh1, const void* dh3, const int* seg, const int* 
   return launch_tn<EPI_STORE_BF16>(p, tn_tiles_ub(N, E, d, p.fstep), "ffn_dgrad_x", s);
 }
 
-// dW1_e = X_e^T dH1_e, dW3_e = X_e^T dH3_e (reduction over the expert's PFT rows), on CTA pairs:
-// 256 rows of d by 128 columns of dH1 (even CTA) and the same 128 of dH3 (odd CTA).
+// dW1_e = X_e^T dH1_e, dW3_e = X_e^T dH3_e (K-grouped over the expert's PFT rows).
 int tc_ffn_wgrad13(const void* x_pft, const void* dh1, const void* dh3, const int* seg, int N, int E, int d, int h,
                    void* dw1, void* dw3, int32_t* err, cudaStream_t s) {
   Params p = base_params(err);
+  p.mode = KG;
+  p.b_major = 1;
+  p.bn = h > 64 ? 256 : 128;
   p.nsplit = 1;
   p.M = d;
   p.Nout = h;
@@ -2132,11 +1735,12 @@ int tc_ffn_wgrad13(const void* x_pft, const void* dh1, const void* dh3, const in
   p.D0 = dw1; p.D1 = dw3; p.ldd = h; p.d_gstride = static_cast<long long>(d) * h;
   p.a_merged = d % 64 == 0;
   p.b_merged = h % 64 == 0;
+  const uint32_t bblk = (p.bn / 2) / 64;
   if (p.a_merged) PFMOE_TRY(make_tmap_mn(&p.tmA[0], x_pft, d, N, 1, BK, 2, "x_pft^T"));
   else PFMOE_TRY(make_tmap(&p.tmA[0], x_pft, d, N, 1, 64, BK, "x_pft^T"));
   if (p.b_merged) {
-    PFMOE_TRY(make_tmap_mn(&p.tmB[0], dh1, h, N, 1, BK, 2, "dh1"));
-    PFMOE_TRY(make_tmap_mn(&p.tmB[1], dh3, h, N, 1, BK, 2, "dh3"));
+    PFMOE_TRY(make_tmap_mn(&p.tmB[0], dh1, h, N, 1, BK, bblk, "dh1"));
+    PFMOE_TRY(make_tmap_mn(&p.tmB[1], dh3, h, N, 1, BK, bblk, "dh3"));
   } else {
     PFMOE_TRY(make_tmap(&p.tmB[0], dh1, h, N, 1, 64, BK, "dh1"));
     PFMOE_TRY(make_tmap(&p.tmB[1], dh3, h, N, 1, 64, BK, "dh3"));
@@ -2144,14 +1748,17 @@ int tc_ffn_wgrad13(const void* x_pft, const void* dh1, const void* dh3, const in
   PFMOE_TRY(make_out_map(&p.tmD[0], dw1, h, d, E, "dw1 out"));
   PFMOE_TRY(make_out_map(&p.tmD[1], dw3, h, d, E, "dw3 out"));
   p.tma_store = 1;
-  const long long ub = static_cast<long long>(E) * ((h + BM - 1) / BM) * ((d + 2 * BM - 1) / (2 * BM));
-  return launch_wgrad_pair<EPI_SPLIT_BF16>(p, ub, "ffn_wgrad_w1w3", s);
+  const long long ub = static_cast<long long>(E) * ((d + BM - 1) / BM) * ((h + p.bn / 2 - 1) / (p.bn / 2));
+  return launch<EPI_SPLIT_BF16, KG>(p, ub, "ffn_wgrad_w1w3", s);
 }
 
-// dW2_e = A_e^T dO_e on CTA pairs: 256 rows of h by 256 columns of d (128 per CTA).
+// dW2_e = A_e^T dO_e.
 int tc_ffn_wgrad2(const void* a, const void* dO, const int* seg, int N, int E, int d, int h, void* dw2,
                   int32_t* err, cudaStream_t s) {
   Params p = base_params(err);
+  p.mode = KG;
+  p.b_major = 1;
+  p.bn = round_bn(d);
   p.M = h;
   p.Nout = d;
   p.seg = seg; p.G = E;
@@ -2160,12 +1767,12 @@ int tc_ffn_wgrad2(const void* a, const void* dO, const int* seg, int N, int E, i
   p.b_merged = d % 64 == 0;
   if (p.a_merged) PFMOE_TRY(make_tmap_mn(&p.tmA[0], a, h, N, 1, BK, 2, "a^T"));
   else PFMOE_TRY(make_tmap(&p.tmA[0], a, h, N, 1, 64, BK, "a^T"));
-  if (p.b_merged) PFMOE_TRY(make_tmap_mn(&p.tmB[0], dO, d, N, 1, BK, 2, "dO"));
+  if (p.b_merged) PFMOE_TRY(make_tmap_mn(&p.tmB[0], dO, d, N, 1, BK, p.bn / 64, "dO"));
   else PFMOE_TRY(make_tmap(&p.tmB[0], dO, d, N, 1, 64, BK, "dO"));
   PFMOE_TRY(make_out_map(&p.tmD[0], dw2, d, h, E, "dw2 out"));
   p.tma_store = 1;
-  const long long ub = static_cast<long long>(E) * ((d + 2 * BM - 1) / (2 * BM)) * ((h + 2 * BM - 1) / (2 * BM));
-  return launch_wgrad_pair<EPI_STORE_BF16>(p, ub, "ffn_wgrad_w2", s);
+  const long long ub = static_cast<long long>(E) * ((h + BM - 1) / BM) * ((d + p.bn - 1) / p.bn);
+  return launch<EPI_STORE_BF16, KG>(p, ub, "ffn_wgrad_w2", s);
 }
 
 static int gate_logits_split(int T, int d, int E) {

@@ -154,11 +154,12 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(const char* __restric
 // y[t] = sum_j w[t, j] * O[pos[t, j]] ([A] §2.1.1 combine_weights), with bulk copies: warp 0's
 // lane 0 loads the k PFT row pieces (at most CB_PIECE bytes each) of a work item (token, piece)
 // into a ring stage, and the warp posts the token's k weights beside it (a global load on the
-// consumers' path would stall every item); four consumer warps sum the stage in slot order in
+// consumers' path would stall every item); eight consumer warps sum the stage in slot order in
 // float32 (one 16-byte vector a thread) and store the piece of y.  A token with an out-of-range row index is flagged and its
 // output row is left unwritten.
 constexpr int CB_PIECE = 8192;   // largest row piece a ring stage holds per slot
-constexpr int CB_CONSUMERS = 128;
+constexpr int CB_CONSUMERS = 256;   // eight consumer warps per CTA
+constexpr int CB_CWARPS = CB_CONSUMERS / 32;
 
 template <typename T>
 __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const char* __restrict__ O,
@@ -260,17 +261,17 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const c
 
 // The two backward gather kernels below use the same producer / consumer ring as combine: warp 0
 // loads a work item's row pieces (piece bytes each) with bulk copies into a stage and posts the
-// item's per-slot scalars there; four consumer warps (CB_CONSUMERS threads, one 16-byte vector
+// item's per-slot scalars there; eight consumer warps (CB_CONSUMERS threads, one 16-byte vector
 // each) read the stage.  KM >= k bounds the per-thread slot arrays so they stay in registers.
-__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-// Barrier of the four consumer warps that also ANDs a flag over them: every consumer warp takes the
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(CB_CONSUMERS) : "memory"); }
+// Barrier of the consumer warps that also ANDs a flag over them: every consumer warp takes the
 // same decision (to go on or to stop), so none is left waiting at a barrier another has left.
 __device__ __forceinline__ bool consumers_all(bool pred) {
   uint32_t r;
   asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred))
+      : "r"(static_cast<uint32_t>(pred)), "n"(CB_CONSUMERS)
       : "memory");
   return r != 0;
 }
@@ -278,7 +279,7 @@ __device__ __forceinline__ bool consumers_all(bool pred) {
 // Per token t (work items are its row pieces, in order): dO[pos[t, j]] = w[t, j] * dY[t] and
 // g[t, j] = <dY[t], O[pos[t, j]]> (the combine's backward).  Stage: the dY piece, then the k O
 // pieces.  Each consumer thread keeps its partial dot products over the token's pieces; after the
-// last piece they are summed over the thread's warp and then over the four warps in order
+// last piece they are summed over the thread's warp and then over the consumer warps in order
 // (deterministic).  A token with an out-of-range row index is flagged and left unwritten.
 template <typename T, int KM>
 __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bwd_bulk_kernel(
@@ -292,7 +293,7 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bwd_bulk_kernel(
   __shared__ int valid[8];
   __shared__ int spos[8][32];
   __shared__ float sw[8][32];
-  __shared__ float red[4][KM];
+  __shared__ float red[CB_CWARPS][KM];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long N = static_cast<long long>(Tn) * k;
   const uint32_t stage_bytes = static_cast<uint32_t>(k + 1) * piece;
@@ -392,7 +393,12 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bwd_bulk_kernel(
         if (lane == 0) red[cw][j] = v;
       }
       const bool all_ok = consumers_all(ok);   // red[] complete
-      if (all_ok && tok_valid && c16 < k) g[t * k + c16] = ((red[0][c16] + red[1][c16]) + red[2][c16]) + red[3][c16];
+      if (all_ok && tok_valid && c16 < k) {
+        float gs = red[0][c16];
+#pragma unroll
+        for (int w = 1; w < CB_CWARPS; ++w) gs += red[w][c16];   // warps in order: deterministic
+        g[t * k + c16] = gs;
+      }
       consumers_sync();                        // red[] read before the next token writes it
       if (!all_ok) break;
     }
