@@ -19,31 +19,20 @@ namespace {
 
 constexpr int SCAN_THREADS = 1024;
 
-// Keys per warp of a chunk: 256 (8 per lane) while the sort has few chunks, 1024 (32 per lane) once
-// there are enough 1024-key chunks for two CTAs on each of 148 SMs.  Larger chunks amortise each
-// chunk's per-key scans and write the sorted rows as longer runs.  The choice depends only on the
-// shape (never on the device), so workspace sizes are host-computable.
-constexpr int KPW_SMALL = 256;
-constexpr int KPW_LARGE = 1024;
+constexpr int KPW = 256;   // keys per warp of a chunk (8 per lane)
 
 // Warps per chunk CTA: up to 8, while the scatter's per-warp counters (W * K ints) fit in 48 KB.
 inline int warps_per_block(int K) {
   int w = 12288 / (K > 0 ? K : 1);
   return w < 1 ? 1 : (w > 8 ? 8 : w);
 }
-inline int keys_per_warp(long long n_max, int K) {
-  return n_max / (static_cast<long long>(warps_per_block(K)) * KPW_LARGE) >= 296 ? KPW_LARGE : KPW_SMALL;
-}
-inline long long chunk_keys(long long n_max, int K) {
-  return static_cast<long long>(warps_per_block(K)) * keys_per_warp(n_max, K);
-}
+inline long long chunk_keys(int K) { return static_cast<long long>(warps_per_block(K)) * KPW; }
 
 __device__ __forceinline__ long long dev_count(long long n, const int32_t* n_dev) {
   return n_dev ? static_cast<long long>(*n_dev) : n;
 }
 
 // One CTA per chunk: shared histogram of the chunk's keys -> counts[chunk][key].
-template <int KPW>
 __global__ void chunk_hist_kernel(const int32_t* __restrict__ keys, long long n, const int32_t* n_dev, int K,
                                   int nchunks, int32_t* __restrict__ counts, int32_t* err) {
   extern __shared__ int32_t sh[];
@@ -185,13 +174,13 @@ __global__ void __launch_bounds__(SCAN_THREADS) key_scan_kernel(const int32_t* _
 // neighbouring addresses instead of one scattered sector per element.
 // Sink interface: at_source(i, p) writes the outputs indexed by element i; payload(i, a, b) gives
 // two ints carried to the sorted side; at_dest(p, key, a, b) writes the outputs indexed by row p.
-// Shared memory: [warps][K] counts, two [K] bases and three [warps * keys per warp] staging arrays.
-__host__ __device__ inline size_t scatter_smem_bytes(int nw, int K, int kpw) {
-  return (static_cast<size_t>(nw) * K + 2 * static_cast<size_t>(K) + 3 * static_cast<size_t>(nw) * kpw) *
+// Shared memory: [warps][K] counts, two [K] bases and three [warps * KPW] staging arrays.
+__host__ __device__ inline size_t scatter_smem_bytes(int nw, int K) {
+  return (static_cast<size_t>(nw) * K + 2 * static_cast<size_t>(K) + 3 * static_cast<size_t>(nw) * KPW) *
          sizeof(int32_t);
 }
 
-template <class Sink, int KPW>
+template <class Sink>
 __global__ void chunk_scatter_kernel(const int32_t* __restrict__ keys, long long n, const int32_t* n_dev, int K,
                                      int nchunks, const int32_t* __restrict__ base,
                                      const int32_t* __restrict__ key_offsets, Sink sink) {
@@ -858,24 +847,19 @@ int sort_scan(const int32_t* counts, int C, int K, int32_t* totals, int32_t* off
 inline long long long_scan_tiles(long long n_max) { return (n_max + SCAN_TILE - 1) / SCAN_TILE; }
 constexpr long long LONG_SCAN_MIN = 4LL * SCAN_TILE;   // below this one CTA scans the array
 
-// The staged scatter needs up to ~116 KB of shared memory (K = 4096 keys, three warps of 1024
-// keys): opt in once per device.
-template <class Sink, int KPW>
+// The staged scatter needs up to ~95 KB of shared memory (K = 4096 keys, three warps): opt in
+// once per device.
+template <class Sink>
 int scatter_smem_attr() {
-  return smem_optin(reinterpret_cast<const void*>(&chunk_scatter_kernel<Sink, KPW>), 227 * 1024, "chunk_scatter");
+  return smem_optin(reinterpret_cast<const void*>(&chunk_scatter_kernel<Sink>), 227 * 1024, "chunk_scatter");
 }
 
-// Histogram + scatter launches of one stable counting sort, with the chunk size chosen for n_max.
-template <class Sink>
+// Histogram + scatter launches of one stable counting sort.
 int sort_hist(const int32_t* keys, long long n_max, const int32_t* n_dev, int K, int C, int32_t* counts,
               int32_t* err, const char* name, cudaStream_t s) {
   const int wpb = warps_per_block(K);
-  if (keys_per_warp(n_max, K) == KPW_LARGE)
-    PFMOE_LAUNCH(name, s, (chunk_hist_kernel<KPW_LARGE><<<C, wpb * 32, K * sizeof(int32_t), s>>>(keys, n_max, n_dev,
-                                                                                              K, C, counts, err)));
-  else
-    PFMOE_LAUNCH(name, s, (chunk_hist_kernel<KPW_SMALL><<<C, wpb * 32, K * sizeof(int32_t), s>>>(keys, n_max, n_dev,
-                                                                                              K, C, counts, err)));
+  PFMOE_LAUNCH(name, s, (chunk_hist_kernel<<<C, wpb * 32, K * sizeof(int32_t), s>>>(keys, n_max, n_dev, K, C, counts,
+                                                                                   err)));
   return PFMOE_OK;
 }
 
@@ -883,20 +867,11 @@ template <class Sink>
 int sort_scatter(const int32_t* keys, long long n_max, const int32_t* n_dev, int K, int C, const int32_t* base,
                  const int32_t* key_offsets, const Sink& sink, const char* name, cudaStream_t s) {
   const int wpb = warps_per_block(K);
-  const int kpw = keys_per_warp(n_max, K);
-  const size_t sm = scatter_smem_bytes(wpb, K, kpw);
-  if (kpw == KPW_LARGE) {
-    PFMOE_TRY((scatter_smem_attr<Sink, KPW_LARGE>()));
-    PFMOE_LAUNCH(name, s, (chunk_scatter_kernel<Sink, KPW_LARGE><<<C, wpb * 32, sm, s>>>(keys, n_max, n_dev, K, C,
-                                                                                       base, key_offsets, sink)));
-  } else {
-    PFMOE_TRY((scatter_smem_attr<Sink, KPW_SMALL>()));
-    PFMOE_LAUNCH(name, s, (chunk_scatter_kernel<Sink, KPW_SMALL><<<C, wpb * 32, sm, s>>>(keys, n_max, n_dev, K, C,
-                                                                                       base, key_offsets, sink)));
-  }
+  PFMOE_TRY(scatter_smem_attr<Sink>());
+  PFMOE_LAUNCH(name, s, (chunk_scatter_kernel<Sink><<<C, wpb * 32, scatter_smem_bytes(wpb, K), s>>>(
+                            keys, n_max, n_dev, K, C, base, key_offsets, sink)));
   return PFMOE_OK;
 }
-
 
 template <int KM>
 static int rbd_fast_launch(const int32_t* ids, int T, int k, int E, int epd, int epn, int n_nodes, int32_t* ppn,
@@ -940,7 +915,7 @@ static int rbd_fast_impl(const int32_t* ids, int T, int k, int E, int epd, int e
 }  // namespace
 
 size_t csort_ws_bytes(long long n_max, int K) {
-  const long long C = (n_max + chunk_keys(n_max, K) - 1) / chunk_keys(n_max, K);
+  const long long C = (n_max + chunk_keys(K) - 1) / chunk_keys(K);
   return static_cast<size_t>(2 * (C > 0 ? C : 1) * static_cast<long long>(K) + K) * sizeof(int32_t);
 }
 
@@ -948,10 +923,10 @@ int pft_build_impl(const int32_t* ids, const float* w, int T, int E, int k, int3
                    int32_t* token_ids, int32_t* expert_ids, float* cw, int32_t* pos, int32_t* tile_offsets,
                    void* ws, int32_t* err, cudaStream_t s) {
   const long long N = static_cast<long long>(T) * k;
-  const int C = static_cast<int>((N + chunk_keys(N, E) - 1) / chunk_keys(N, E));
+  const int C = static_cast<int>((N + chunk_keys(E) - 1) / chunk_keys(E));
   int32_t* counts = static_cast<int32_t*>(ws);
   int32_t* base = counts + static_cast<long long>(C) * E;
-  if (C > 0) PFMOE_TRY(sort_hist<PftSink>(ids, N, nullptr, E, C, counts, err, "pft_hist", s));
+  if (C > 0) PFMOE_TRY(sort_hist(ids, N, nullptr, E, C, counts, err, "pft_hist", s));
   int32_t* key_tot = base + static_cast<long long>(C) * E;
   PFMOE_TRY(sort_scan(counts, C, E, tpe, offsets, base, tile_offsets, 128, key_tot, "pft_scan", s));
   PftSink sink{w, k, pos, token_ids, expert_ids, cw};
@@ -996,7 +971,7 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
   int32_t* tsum_a = p; p += lt;
   int32_t* tsum_b = p; p += lt;
   p += 64 - ((p - static_cast<int32_t*>(ws)) & 63);   // keep 256-byte alignment
-  const int C = static_cast<int>((pmax + chunk_keys(pmax, n_nodes) - 1) / chunk_keys(pmax, n_nodes));
+  const int C = static_cast<int>((pmax + chunk_keys(n_nodes) - 1) / chunk_keys(n_nodes));
   int32_t* ccounts = p; p += static_cast<long long>(C > 0 ? C : 1) * n_nodes;
   int32_t* cbase = p;
 
@@ -1013,7 +988,7 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
     PFMOE_LAUNCH("rbd_scan_tokens", s, tile_scan_kernel<<<nt, SCAN_THREADS, 0, s>>>(ucount, T, nullptr, tsum_a, pbase));
   }
   PFMOE_RBD_LAUNCH("rbd_emit", rbd_emit_kernel, T, k, s, ids, T, k, E, epd, epn, pbase, pkey, ptoken, prc, err);
-  if (C > 0) PFMOE_TRY(sort_hist<RbdSink>(pkey, pmax, counts, n_nodes, C, ccounts, err, "rbd_hist", s));
+  if (C > 0) PFMOE_TRY(sort_hist(pkey, pmax, counts, n_nodes, C, ccounts, err, "rbd_hist", s));
   int32_t* node_tot = cbase + static_cast<long long>(C > 0 ? C : 1) * n_nodes;
   PFMOE_TRY(sort_scan(ccounts, C, n_nodes, pilots_per_node, node_offsets, cbase, nullptr, 0, node_tot,
                       "rbd_scan_nodes", s));

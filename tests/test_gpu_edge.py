@@ -125,8 +125,8 @@ def test_bounded_wait_gives_up_and_context_survives():
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("E,k,epd,dpn", [(256, 8, 8, 4), (1024, 4, 16, 8)])
-def test_pft_and_rbd_large_chunks_match_oracle(E, k, epd, dpn):
-    # More than 2.4 M assignments: the counting sorts switch to 1024 keys per warp.
+def test_pft_and_rbd_four_million_assignments_match_oracle(E, k, epd, dpn):
+    # About 4.2 M assignments (2000+ sort chunks; RBD tiles past the scan's first pass).
     from workloads.generate import make_topk_ids
     T = (1 << 22) // k + 123
     ids = make_topk_ids(T, E, k, seed=9, device="cuda")
