@@ -44,7 +44,13 @@ constexpr int BM = 128;          // MMA M (one CTA)
 constexpr int BK = 64;           // K elements per stage (one 128-byte swizzle row of BF16)
 constexpr int MAX_STAGES = 8;
 constexpr int THREADS = 192;
-constexpr int THREADS_KG = 224;          // K-grouped launches add a seventh warp: the K-tail zeroing warp
+// K-grouped (weight-gradient) launches: 8 epilogue warps, two per TMEM lane quarter, each writing
+// half of a tile's 64-column blocks (their reduction over one expert's rows is short, so the
+// epilogue, not the MMA, sets the pace), and a K-tail zeroing warp after them.
+constexpr int KG_EPI_WARPS = 8;
+constexpr int KG_STAGE_BUFS = 1;         // staging slabs per KG epilogue warp
+constexpr int KG_ZERO_WARP = 2 + KG_EPI_WARPS;
+constexpr int THREADS_KG = (KG_ZERO_WARP + 1) * 32;
 constexpr int BOX_BYTES = 64 * 128;      // one 64 x 64 BF16 box (MN-major block)
 constexpr int A_BYTES = BM * BK * 2;     // 16 KB
 
@@ -348,7 +354,6 @@ __device__ __forceinline__ void epilogue_tile_direct(const Params& p, const Tile
 // segment.  Every global store is then part of a full 128-byte line.  Used for
 // K-grouped (weight-gradient) tiles, whose short K loops leave the epilogue exposed.
 constexpr int STAGE_BYTES_PER_WARP = 32 * 128;   // one 32-row x 128-byte slab
-constexpr int STAGE_BUFS = 2;                     // per warp: ping-pong so a TMA store overlaps the next slab
 
 __device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t* r) {
   asm volatile(
@@ -425,7 +430,7 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* tm, uint32_t src
                : "memory");
 }
 
-// Per-warp staging state: two 4 KB slabs used alternately.
+// Per-warp staging state: KG_STAGE_BUFS 4 KB slabs used in turn.
 struct Stager {
   uint32_t base;
   int seq;
@@ -434,13 +439,14 @@ struct Stager {
 // Stage one 32-row x 128-byte slab and write it out: a full slab goes out as one TMA store
 // (the staging layout is the TMA 128-byte swizzle; the store clips at the tensor bounds);
 // a slab with missing rows goes out with masked vector stores.  One bulk group is committed
-// per slab, so "at most one group pending" means the slab about to be reused is free.
+// per slab, so "at most KG_STAGE_BUFS - 1 groups pending" means the slab about to be reused is free.
 template <typename T>
 __device__ __forceinline__ void emit(Stager& st, int lane, const float* v, const CUtensorMap* tm, int c0, int c1,
                                      int c2, T* dst_row0, long long ldd, int rows_valid, int cols_valid) {
-  const uint32_t buf = st.base + (st.seq & 1) * STAGE_BYTES_PER_WARP;
+  const uint32_t buf = st.base + (st.seq % KG_STAGE_BUFS) * STAGE_BYTES_PER_WARP;
   ++st.seq;
-  if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+  // the slab about to be written was last read by the store KG_STAGE_BUFS groups ago
+  if (lane == 0) asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(KG_STAGE_BUFS - 1) : "memory");
   __syncwarp();
   stage_row<T>(buf, lane, v);
   if (tm && rows_valid == 32) {
@@ -465,9 +471,11 @@ __device__ __forceinline__ const CUtensorMap* tmd(const Params& p, int i) {
   return p.tma_store ? &p.tmD[i] : nullptr;
 }
 
+// Warp (q, half) of nhalves warps per lane quarter writes the 64-column blocks b (32-column chunks
+// for FP32) with b % nhalves == half.
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, uint32_t tacc, int q, int lane,
-                                              Stager& stg) {
+                                              Stager& stg, int half, int nhalves) {
   const int slab0 = q * 32;
   const int rows_valid = max(0, min(32, tl.rows - slab0));
   const long long grow0 = static_cast<long long>(tl.row0) + slab0;
@@ -482,6 +490,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, u
       for (int c = 0; c < width; c += 64) {
         const int col = tl.n0 + c;
         if (col >= p.Nout) break;
+        if (((part * width + c) / 64) % nhalves != half) continue;
         float v[64];
         if (!zero) tmem_ld64(tacc + part * width + c, v);
         else {
@@ -497,6 +506,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, u
     for (int c = 0; c < p.bn; c += 32) {
       const int col = tl.n0 + c;
       if (col >= p.Nout) break;
+      if ((c / 32) % nhalves != half) continue;
       float v[32];
       if (!zero) {
         uint32_t r[32];
@@ -530,7 +540,7 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
   const uint32_t b_bytes = static_cast<uint32_t>(p.bn) * KBK * 2;
   const uint32_t stage_bytes = a_bytes + b_bytes;
   uint8_t* stage_area = smem + S * stage_bytes;                       // epilogue staging (K-grouped only)
-  uint8_t* bar_area = stage_area + (MODE == KG ? 4 * STAGE_BUFS * STAGE_BYTES_PER_WARP : 0);
+  uint8_t* bar_area = stage_area + (MODE == KG ? KG_EPI_WARPS * KG_STAGE_BUFS * STAGE_BYTES_PER_WARP : 0);
   uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
   uint64_t* empty = full + MAX_STAGES;
   uint64_t* acc_full = empty + MAX_STAGES;
@@ -551,7 +561,7 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&acc_full[b]), 1);
-      mbar_init(smem_u32(&acc_empty[b]), 4 * 32);
+      mbar_init(smem_u32(&acc_empty[b]), (MODE == KG ? KG_EPI_WARPS : 4) * 32);
     }
     mbar_init(smem_u32(drain), 1);
     for (int z = 0; z < MAX_STAGES; ++z) mbar_init(smem_u32(&ready[z]), 1);
@@ -690,7 +700,7 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
       wait_bar(smem_u32(drain), 0, abort_flag, p.err, false);
     }
     __syncwarp();
-  } else if (MODE == KG && warp == 6) {
+  } else if (MODE == KG && warp == KG_ZERO_WARP) {
     // ---------------------------------------------------- K-tail zeroing (K-grouped only)
     // Walks every K block in ring order: waits for it to land (full[s]), clears the rows of a
     // segment's last 16-row step past the segment end in every box (A: 2, B: bn/64), and hands
@@ -720,7 +730,8 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
   } else {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;           // TMEM lane quarter this warp may access: rows 32q .. 32q+31
-    Stager stg{smem_u32(stage_area + (warp - 2) * STAGE_BUFS * STAGE_BYTES_PER_WARP), 0};
+    const int half = (warp - 2) / 4;  // K-grouped: which of the two warps of the quarter
+    Stager stg{smem_u32(stage_area + (warp - 2) * KG_STAGE_BUFS * STAGE_BYTES_PER_WARP), 0};
     int tcount = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tcount) {
       const Tile tl = decode<MODE, KBK>(p, t);
@@ -729,7 +740,7 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
       if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&acc_full[buf]), aph, abort_flag, p.err))) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * p.bn;
-      if constexpr (MODE == KG) epilogue_tile<EPI>(p, tl, tacc, q, lane, stg);
+      if constexpr (MODE == KG) epilogue_tile<EPI>(p, tl, tacc, q, lane, stg, half, KG_EPI_WARPS / 4);
       else epilogue_tile_direct<EPI>(p, tl, tacc, q * 32 + lane);
       tc_fence_before();
       mbar_arrive(smem_u32(&acc_empty[buf]));
@@ -827,7 +838,9 @@ static int round_bn(int n) {
 
 constexpr int SMEM_LIMIT = 227 * 1024;
 // Alignment slack + barriers (512 B), plus the epilogue staging buffers when the launch uses them (K-grouped).
-static int smem_fixed(bool staged) { return 1024 + 512 + (staged ? 4 * STAGE_BUFS * STAGE_BYTES_PER_WARP : 0); }
+static int smem_fixed(bool staged) {
+  return 1024 + 512 + (staged ? KG_EPI_WARPS * KG_STAGE_BUFS * STAGE_BYTES_PER_WARP : 0);
+}
 
 static int stage_size(int bn, int kbk) { return (BM + bn) * kbk * 2; }
 
