@@ -44,11 +44,11 @@ constexpr int BM = 128;          // MMA M (one CTA)
 constexpr int BK = 64;           // K elements per stage (one 128-byte swizzle row of BF16)
 constexpr int MAX_STAGES = 8;
 constexpr int THREADS = 192;
-// K-grouped (weight-gradient) launches: 8 epilogue warps, two per TMEM lane quarter, each writing
-// half of a tile's 64-column blocks (their reduction over one expert's rows is short, so the
-// epilogue, not the MMA, sets the pace), and a K-tail zeroing warp after them.
-constexpr int KG_EPI_WARPS = 8;
-constexpr int KG_STAGE_BUFS = 1;         // staging slabs per KG epilogue warp
+// K-grouped (weight-gradient) launches: KG_EPI_WARPS epilogue warps (a multiple of 4; with 8, two
+// per TMEM lane quarter each write half of a tile's column blocks) and a K-tail zeroing warp after
+// them.  Four warps with two staging slabs each measured as fast as eight with one or two.
+constexpr int KG_EPI_WARPS = 4;
+constexpr int KG_STAGE_BUFS = 2;         // staging slabs per KG epilogue warp
 constexpr int KG_ZERO_WARP = 2 + KG_EPI_WARPS;
 constexpr int THREADS_KG = (KG_ZERO_WARP + 1) * 32;
 constexpr int BOX_BYTES = 64 * 128;      // one 64 x 64 BF16 box (MN-major block)

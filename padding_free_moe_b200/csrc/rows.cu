@@ -158,8 +158,11 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(const char* __restric
 // float32 (one 16-byte vector a thread) and store the piece of y.  A token with an out-of-range row index is flagged and its
 // output row is left unwritten.
 constexpr int CB_PIECE = 8192;   // largest row piece a ring stage holds per slot
-constexpr int CB_CONSUMERS = 256;   // eight consumer warps per CTA
-constexpr int CB_CWARPS = CB_CONSUMERS / 32;
+constexpr int CB_CONSUMERS = 256;   // combine: eight consumer warps per CTA
+// combine_bwd and token_grad: four consumer warps per CTA, two CTAs per SM (measured faster for
+// them than one CTA of eight consumer warps with larger pieces)
+constexpr int GB_CONSUMERS = 128;
+constexpr int GB_CWARPS = GB_CONSUMERS / 32;
 
 template <typename T>
 __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const char* __restrict__ O,
@@ -261,9 +264,9 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const c
 
 // The two backward gather kernels below use the same producer / consumer ring as combine: warp 0
 // loads a work item's row pieces (piece bytes each) with bulk copies into a stage and posts the
-// item's per-slot scalars there; eight consumer warps (CB_CONSUMERS threads, one 16-byte vector
+// item's per-slot scalars there; four consumer warps (GB_CONSUMERS threads, one 16-byte vector
 // each) read the stage.  KM >= k bounds the per-thread slot arrays so they stay in registers.
-__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(CB_CONSUMERS) : "memory"); }
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(GB_CONSUMERS) : "memory"); }
 // Barrier of the consumer warps that also ANDs a flag over them: every consumer warp takes the
 // same decision (to go on or to stop), so none is left waiting at a barrier another has left.
 __device__ __forceinline__ bool consumers_all(bool pred) {
@@ -271,7 +274,7 @@ __device__ __forceinline__ bool consumers_all(bool pred) {
   asm volatile(
       "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred)), "n"(CB_CONSUMERS)
+      : "r"(static_cast<uint32_t>(pred)), "n"(GB_CONSUMERS)
       : "memory");
   return r != 0;
 }
@@ -282,7 +285,7 @@ __device__ __forceinline__ bool consumers_all(bool pred) {
 // last piece they are summed over the thread's warp and then over the consumer warps in order
 // (deterministic).  A token with an out-of-range row index is flagged and left unwritten.
 template <typename T, int KM>
-__global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bwd_bulk_kernel(
+__global__ void __launch_bounds__(32 + GB_CONSUMERS) combine_bwd_bulk_kernel(
     const char* __restrict__ dy, const char* __restrict__ O, const int32_t* __restrict__ pos,
     const float* __restrict__ w, int Tn, int k, int row_bytes, int piece, int pieces, int stages,
     char* __restrict__ dO, float* __restrict__ g, int32_t* err) {
@@ -293,14 +296,14 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bwd_bulk_kernel(
   __shared__ int valid[8];
   __shared__ int spos[8][32];
   __shared__ float sw[8][32];
-  __shared__ float red[CB_CWARPS][KM];
+  __shared__ float red[GB_CWARPS][KM];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long N = static_cast<long long>(Tn) * k;
   const uint32_t stage_bytes = static_cast<uint32_t>(k + 1) * piece;
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       bar_init(smem_addr(&full[s]), 1);
-      bar_init(smem_addr(&empty[s]), CB_CONSUMERS);
+      bar_init(smem_addr(&empty[s]), GB_CONSUMERS);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -364,7 +367,7 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bwd_bulk_kernel(
         if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&full[s]), (q / stages) & 1, err))) { ok = false; break; }
         tok_valid = valid[s] != 0;
         if (tok_valid) {
-          for (int v = c16; v * 16 < bytes; v += CB_CONSUMERS) {
+          for (int v = c16; v * 16 < bytes; v += GB_CONSUMERS) {
             const uint8_t* sp = csm + s * stage_bytes + v * 16;
             float a[VN];
             load16(reinterpret_cast<const T*>(sp), a);
@@ -396,7 +399,7 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bwd_bulk_kernel(
       if (all_ok && tok_valid && c16 < k) {
         float gs = red[0][c16];
 #pragma unroll
-        for (int w = 1; w < CB_CWARPS; ++w) gs += red[w][c16];   // warps in order: deterministic
+        for (int w = 1; w < GB_CWARPS; ++w) gs += red[w][c16];   // warps in order: deterministic
         g[t * k + c16] = gs;
       }
       consumers_sync();                        // red[] read before the next token writes it
@@ -411,7 +414,7 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bwd_bulk_kernel(
 // and, after issuing a token's first piece, writes its dense dlogits row (and the BF16 copy the
 // dWg GEMM reads) while the consumers sum.
 template <typename T>
-__global__ void __launch_bounds__(32 + CB_CONSUMERS) token_grad_bulk_kernel(
+__global__ void __launch_bounds__(32 + GB_CONSUMERS) token_grad_bulk_kernel(
     const char* __restrict__ dxp, const int32_t* __restrict__ pos, const float* __restrict__ g,
     const float* __restrict__ w, const int32_t* __restrict__ ids, const char* __restrict__ wgT, int Tn, int k, int E,
     int row_bytes, int piece, int pieces, int stages, char* __restrict__ dx, float* __restrict__ dlogits,
@@ -428,7 +431,7 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) token_grad_bulk_kernel(
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       bar_init(smem_addr(&full[s]), 1);
-      bar_init(smem_addr(&empty[s]), CB_CONSUMERS);
+      bar_init(smem_addr(&empty[s]), GB_CONSUMERS);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -516,7 +519,7 @@ __global__ void __launch_bounds__(32 + CB_CONSUMERS) token_grad_bulk_kernel(
       const int s = q % stages;
       if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&full[s]), (q / stages) & 1, err))) { ok = false; break; }
       if (valid[s]) {
-        for (int vv = c16; vv * 16 < bytes; vv += CB_CONSUMERS) {
+        for (int vv = c16; vv * 16 < bytes; vv += GB_CONSUMERS) {
           float acc[VN];
 #pragma unroll
           for (int i = 0; i < VN; ++i) acc[i] = 0.f;
@@ -578,23 +581,23 @@ int launch_dispatch(const void* x, const int32_t* pos, int T, int k, int d, int 
 }
 
 
-// Ring geometry for `slots` row pieces per stage.  The copy engine's cost per copy favours large
-// pieces, so a CTA takes about 200 KB (one per SM) in at least three stages, with pieces of up to
-// CB_PIECE bytes; rows narrower than a piece make smaller stages, and then up to eight of them.
+// Ring geometry for `slots` row pieces per stage: pieces of at most `piece_cap` bytes (smaller where
+// fewer than three stages of them fit the CTA's `budget`), then as many stages of them as the
+// budget holds (2 to 8), and how many such CTAs share an SM.  The copy engine's cost per copy
+// favours large pieces; the consumers' share of the work per piece favours more CTAs per SM.
 struct Ring {
   int piece, pieces, stages, ctas_per_sm;
   size_t smem;
 };
-static Ring ring_for(int row_bytes, int slots) {
-  constexpr int kBudget = 200 * 1024;
+static Ring ring_for(int row_bytes, int slots, int budget, int piece_cap) {
   Ring r;
-  int cap = (kBudget / (3 * slots)) & ~15;
+  int cap = (budget / (3 * slots)) & ~15;
   if (cap < 16) cap = 16;
-  r.piece = CB_PIECE < cap ? CB_PIECE : cap;
+  r.piece = piece_cap < cap ? piece_cap : cap;
   if (r.piece > row_bytes) r.piece = row_bytes;     // row_bytes is a multiple of 16
   r.pieces = (row_bytes + r.piece - 1) / r.piece;
   const int stage = slots * r.piece;
-  r.stages = kBudget / stage;
+  r.stages = budget / stage;
   if (r.stages > 8) r.stages = 8;
   if (r.stages < 2) r.stages = 2;
   r.smem = static_cast<size_t>(r.stages) * stage;
@@ -605,7 +608,7 @@ static Ring ring_for(int row_bytes, int slots) {
 int launch_combine(const void* out, const int32_t* pos, const float* w, int T, int k, int d, int dtype, void* y,
                    int32_t* err, cudaStream_t s) {
   const int row_bytes = d * (dtype == PFMOE_BF16 ? 2 : 4);
-  const Ring r = ring_for(row_bytes, k);
+  const Ring r = ring_for(row_bytes, k, 200 * 1024, CB_PIECE);
   const long long items = static_cast<long long>(T) * r.pieces;
   long long grid = static_cast<long long>(num_sms()) * r.ctas_per_sm;
   if (grid > items) grid = items;
@@ -630,7 +633,7 @@ static int launch_cbwd_t(const void* dy, const void* out, const int32_t* pos, co
                          int row_bytes, const Ring& r, int grid, void* dO, float* g, int32_t* err, cudaStream_t s) {
   PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&combine_bwd_bulk_kernel<T, KM>), 227 * 1024, "combine_bwd"));
   PFMOE_LAUNCH("combine_bwd", s,
-               (combine_bwd_bulk_kernel<T, KM><<<grid, 32 + CB_CONSUMERS, r.smem, s>>>(
+               (combine_bwd_bulk_kernel<T, KM><<<grid, 32 + GB_CONSUMERS, r.smem, s>>>(
                    static_cast<const char*>(dy), static_cast<const char*>(out), pos, w, T_, k, row_bytes, r.piece,
                    r.pieces, r.stages, static_cast<char*>(dO), g, err)));
   return PFMOE_OK;
@@ -639,7 +642,7 @@ static int launch_cbwd_t(const void* dy, const void* out, const int32_t* pos, co
 int launch_combine_bwd(const void* dy, const void* out, const int32_t* pos, const float* w, int T, int k, int d,
                        int dtype, void* dO, float* g, int32_t* err, cudaStream_t s) {
   const int row_bytes = d * (dtype == PFMOE_BF16 ? 2 : 4);
-  const Ring r = ring_for(row_bytes, k + 1);
+  const Ring r = ring_for(row_bytes, k + 1, 96 * 1024, 2048);
   long long grid = static_cast<long long>(num_sms()) * r.ctas_per_sm;
   if (grid > T) grid = T;
   const int gr = static_cast<int>(grid);
@@ -671,7 +674,7 @@ int launch_token_grad(const void* dx_pft, const int32_t* pos, const float* g, co
                       const void* wgT, int T, int k, int d, int E, int dtype, void* dx, float* dlogits,
                       void* dz_bf16, int32_t* err, cudaStream_t s) {
   const int row_bytes = d * (dtype == PFMOE_BF16 ? 2 : 4);
-  const Ring r = ring_for(row_bytes, 2 * k);
+  const Ring r = ring_for(row_bytes, 2 * k, 96 * 1024, 2048);
   long long grid = static_cast<long long>(num_sms()) * r.ctas_per_sm;
   if (grid > T) grid = T;
   auto* dzb = static_cast<__nv_bfloat16*>(dz_bf16);
@@ -679,13 +682,13 @@ int launch_token_grad(const void* dx_pft, const int32_t* pos, const float* g, co
     PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&token_grad_bulk_kernel<__nv_bfloat16>), 227 * 1024,
                          "token_grad"));
     PFMOE_LAUNCH("token_grad", s,
-                 (token_grad_bulk_kernel<__nv_bfloat16><<<static_cast<int>(grid), 32 + CB_CONSUMERS, r.smem, s>>>(
+                 (token_grad_bulk_kernel<__nv_bfloat16><<<static_cast<int>(grid), 32 + GB_CONSUMERS, r.smem, s>>>(
                      static_cast<const char*>(dx_pft), pos, g, w, ids, static_cast<const char*>(wgT), T, k, E,
                      row_bytes, r.piece, r.pieces, r.stages, static_cast<char*>(dx), dlogits, dzb, err)));
   } else {
     PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&token_grad_bulk_kernel<float>), 227 * 1024, "token_grad"));
     PFMOE_LAUNCH("token_grad", s,
-                 (token_grad_bulk_kernel<float><<<static_cast<int>(grid), 32 + CB_CONSUMERS, r.smem, s>>>(
+                 (token_grad_bulk_kernel<float><<<static_cast<int>(grid), 32 + GB_CONSUMERS, r.smem, s>>>(
                      static_cast<const char*>(dx_pft), pos, g, w, ids, static_cast<const char*>(wgT), T, k, E,
                      row_bytes, r.piece, r.pieces, r.stages, static_cast<char*>(dx), dlogits, dzb, err)));
   }
