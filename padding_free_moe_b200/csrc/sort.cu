@@ -11,6 +11,8 @@
 //      their keys per key, take an exclusive prefix over warps, then walk their keys in
 //      order, 32 at a time; lanes holding the same key find each other with
 //      __match_any_sync and take consecutive rows in lane order -> the sort is stable.
+#include <climits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -744,6 +746,9 @@ __global__ void __launch_bounds__(RF_SCAN_THREADS) rbd_fast_scan_kernel(int ntil
   }
 }
 
+// Per token: the in-tile prefix by warp scans, then the outputs.  The pilot rows of one node in a
+// tile are consecutive, so the per-node pilot stores are coalesced; the replica lists and
+// assign_pilot are staged in shared memory (the ids' buffer, reused) and leave as contiguous runs.
 template <int KM>
 __global__ void __launch_bounds__(RF_TILE) rbd_fast_emit_kernel(
     const int32_t* __restrict__ ids, int T, int k, int E, int epd, int epn, int n_nodes,
@@ -752,13 +757,15 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_emit_kernel(
     int32_t* __restrict__ pilot_node, int32_t* __restrict__ pilot_device, int32_t* __restrict__ replica_offsets,
     int32_t* __restrict__ replica_expert, int32_t* __restrict__ assign_pilot, int32_t* err) {
   __shared__ int wsum[RF_TILE / 32][RF_NODES];
-  __shared__ int32_t sids[RF_TILE * KM];
+  __shared__ int node_loc[RF_NODES + 1];   // replicas of earlier nodes in this tile
+  __shared__ int32_t sbuf[RF_TILE * KM];   // the tile's ids, then its replica lists, then assign_pilot
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long t = static_cast<long long>(blockIdx.x) * RF_TILE + threadIdx.x;
   const bool valid = t < T;
   int e[KM], nd[KM], c[RF_NODES], ex[RF_NODES];
-  rf_stage_ids(ids, T, k, sids);
-  rf_load<KM>(sids, valid, k, E, epn, e, nd, nullptr);   // rbd_fast_count flagged bad ids
+  rf_stage_ids(ids, T, k, sbuf);
+  rf_load<KM>(sbuf, valid, k, E, epn, e, nd, nullptr);   // rbd_fast_count flagged bad ids
+  (void)err;
   rf_counts<KM>(nd, c);
   // in-warp exclusive prefix of the packed counts, per node
 #pragma unroll
@@ -772,42 +779,77 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_emit_kernel(
     ex[n] = a - c[n];
     if (lane == 31) wsum[warp][n] = a;
   }
-  __syncthreads();
+  __syncthreads();   // wsum complete; every thread has read its ids from sbuf
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int n = 0; n < RF_NODES; ++n) {
+      node_loc[n] = run;
+      for (int w = 0; w < RF_TILE / 32; ++w) run += wsum[w][n] >> 16;
+    }
+    node_loc[RF_NODES] = run;
+  }
 #pragma unroll
   for (int n = 0; n < RF_NODES; ++n)
     for (int w = 0; w < warp; ++w) ex[n] += wsum[w][n];
-  if (!valid) return;
-  (void)err;
-  int idx[RF_NODES], rs[RF_NODES];
+  __syncthreads();   // node_loc ready
   const long long tb = static_cast<long long>(blockIdx.x) * RF_NODES;
+  int idx[RF_NODES];
 #pragma unroll
   for (int n = 0; n < RF_NODES; ++n) {
     idx[n] = 0;
-    rs[n] = 0;
-    if (n < n_nodes && (c[n] & 0xffff)) {
+    if (valid && n < n_nodes && (c[n] & 0xffff)) {
       idx[n] = node_offsets[n] + tile_tok_base[tb + n] + (ex[n] & 0xffff);
-      rs[n] = node_rep_off[n] + tile_rep_base[tb + n] + (ex[n] >> 16);
+      int emin = INT_MAX;
+#pragma unroll
+      for (int j = 0; j < KM; ++j)
+        if (nd[j] == n && e[j] < emin) emin = e[j];
       pilot_token[idx[n]] = static_cast<int32_t>(t);
       pilot_node[idx[n]] = n;
-      replica_offsets[idx[n]] = rs[n];
+      pilot_device[idx[n]] = emin / epd;
+      replica_offsets[idx[n]] = node_rep_off[n] + tile_rep_base[tb + n] + (ex[n] >> 16);
     }
   }
+  // replica lists, node by node in this tile's part of replica_expert
+  if (valid) {
 #pragma unroll
-  for (int j = 0; j < KM; ++j) {
-    if (j < k) {
-      int within = 0;
+    for (int j = 0; j < KM; ++j) {
+      if (j < k) {
+        int within = 0;
 #pragma unroll
-      for (int i = 0; i < KM; ++i)
-        within += (i < k) && nd[i] == nd[j] && (e[i] < e[j] || (e[i] == e[j] && i < j));
-      int pj = 0, rj = 0;
+        for (int i = 0; i < KM; ++i)
+          within += (i < k) && nd[i] == nd[j] && (e[i] < e[j] || (e[i] == e[j] && i < j));
+        int loc = 0;
 #pragma unroll
-      for (int n = 0; n < RF_NODES; ++n)
-        if (nd[j] == n) { pj = idx[n]; rj = rs[n]; }
-      replica_expert[rj + within] = e[j];
-      assign_pilot[t * k + j] = pj;
-      if (within == 0) pilot_device[pj] = e[j] / epd;
+        for (int n = 0; n < RF_NODES; ++n)
+          if (nd[j] == n) loc = node_loc[n] + (ex[n] >> 16);
+        sbuf[loc + within] = e[j];
+      }
     }
   }
+  __syncthreads();
+  for (int n = 0; n < n_nodes; ++n) {
+    const int cnt = node_loc[n + 1] - node_loc[n];
+    const long long g0 = static_cast<long long>(node_rep_off[n]) + tile_rep_base[tb + n];
+    for (int i = threadIdx.x; i < cnt; i += RF_TILE) replica_expert[g0 + i] = sbuf[node_loc[n] + i];
+  }
+  __syncthreads();
+  // assign_pilot: the tile's [tokens][k] block is contiguous
+  if (valid) {
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      if (j < k) {
+        int pj = 0;
+#pragma unroll
+        for (int n = 0; n < RF_NODES; ++n)
+          if (nd[j] == n) pj = idx[n];
+        sbuf[threadIdx.x * k + j] = pj;
+      }
+    }
+  }
+  __syncthreads();
+  const long long a0 = static_cast<long long>(blockIdx.x) * RF_TILE * k;
+  const long long a_end = static_cast<long long>(T) * k;
+  for (int i = threadIdx.x; i < RF_TILE * k && a0 + i < a_end; i += RF_TILE) assign_pilot[a0 + i] = sbuf[i];
 }
 
 // Launch one of the per-token RBD kernels with the smallest lane group that holds k experts.
