@@ -2,14 +2,18 @@
 // combine backward, token-gradient gather-sum with the gate's backward, and a
 // small transpose.  All are HBM-bound.
 //
-// Dispatch and combine move rows through shared memory with 1-D bulk copies
-// (cp.async.bulk, the copy engine of each SM): dispatch loads a piece of a token
-// row once and stores it to the token's k PFT rows straight from shared memory;
-// combine loads the k PFT row pieces of a token into a ring stage and sums them
-// there.  The other kernels move rows with 16-byte vector loads/stores, one warp
-// per (token, column chunk) or PFT row, so every warp access is a coalesced
-// 512-byte run of one row (BF16).  Nothing uses atomics on data; every sum runs
-// over the k slots in slot order, so results are deterministic.
+// Dispatch and the combine's backward move rows through shared memory with 1-D
+// bulk copies (cp.async.bulk, the copy engine of each SM): dispatch loads a piece
+// of a token row once and stores it to the token's k PFT rows straight from
+// shared memory; the combine's backward loads dY and the k PFT row pieces of a
+// token into a ring stage and reads both there.  The two gather-sums (combine,
+// token gradient) keep their k row loads in registers instead: one warp per
+// (token, column chunk), 16-byte vector loads, every warp access a coalesced
+// 512-byte run of one row (BF16), all k loads of a lane in flight at once.  At
+// d = 7168, k = 8 that measured faster than a staged ring, whose consumers wait
+// on each stage while the register form keeps 8 loads per lane outstanding.
+// Nothing uses atomics on data; every sum runs over the k slots in slot order,
+// so results are deterministic.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -151,121 +155,15 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(const char* __restric
   __syncwarp();
 }
 
-// y[t] = sum_j w[t, j] * O[pos[t, j]] ([A] §2.1.1 combine_weights), with bulk copies: warp 0's
-// lane 0 loads the k PFT row pieces (at most CB_PIECE bytes each) of a work item (token, piece)
-// into a ring stage, and the warp posts the token's k weights beside it (a global load on the
-// consumers' path would stall every item); eight consumer warps sum the stage in slot order in
-// float32 (one 16-byte vector a thread) and store the piece of y.  A token with an out-of-range row index is flagged and its
-// output row is left unwritten.
-constexpr int CB_PIECE = 8192;   // largest row piece a ring stage holds per slot
-constexpr int CB_CONSUMERS = 256;   // combine: eight consumer warps per CTA
-// combine_bwd and token_grad: four consumer warps per CTA, two CTAs per SM (measured faster for
-// them than one CTA of eight consumer warps with larger pieces)
+// Consumer warps of the combine's backward: four per CTA, two CTAs per SM (measured faster than
+// one CTA of eight consumer warps with larger pieces).
 constexpr int GB_CONSUMERS = 128;
 constexpr int GB_CWARPS = GB_CONSUMERS / 32;
 
-template <typename T>
-__global__ void __launch_bounds__(32 + CB_CONSUMERS) combine_bulk_kernel(const char* __restrict__ O,
-                                                                         const int32_t* __restrict__ pos,
-                                                                         const float* __restrict__ w, int Tn, int k,
-                                                                         int row_bytes, int piece, int pieces,
-                                                                         int stages, char* __restrict__ y,
-                                                                         int32_t* err) {
-  constexpr int VN = Vec<T>::n;
-  extern __shared__ __align__(128) uint8_t csm[];
-  __shared__ __align__(8) uint64_t full[8];
-  __shared__ __align__(8) uint64_t empty[8];
-  __shared__ int valid[8];
-  __shared__ float sw[8][32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long N = static_cast<long long>(Tn) * k;
-  const long long items = static_cast<long long>(Tn) * pieces;
-  const uint32_t stage_bytes = static_cast<uint32_t>(k) * piece;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < stages; ++s) {
-      bar_init(smem_addr(&full[s]), 1);
-      bar_init(smem_addr(&empty[s]), CB_CONSUMERS);
-    }
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
-  const uint32_t st0 = smem_addr(csm);
-  if (warp == 0) {
-    // ---- producer
-    uint32_t pending = 0, pend_parity = 0;
-    int q = 0;
-    for (long long it = blockIdx.x; it < items; it += gridDim.x, ++q) {
-      const long long t = it / pieces;
-      const int off = static_cast<int>(it - t * pieces) * piece;
-      const int bytes = min(piece, row_bytes - off);
-      const int s = q % stages;
-      const uint32_t ph = (q / stages) & 1;
-      if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&empty[s]), ph ^ 1, err))) break;
-      const int my_pos = lane < k ? pos[t * k + lane] : 0;
-      const bool bad = lane < k && (my_pos < 0 || my_pos >= N);
-      const bool any_bad = __any_sync(0xffffffffu, bad);
-      sw[s][lane] = lane < k ? w[t * k + lane] : 0.f;   // the weights travel with the stage
-      if (lane == 0) {
-        valid[s] = any_bad ? 0 : 1;
-        if (any_bad && off == 0) dev_error(err, PFMOE_DEV_BAD_POS);
-      }
-      __syncwarp();
-      if (any_bad) {
-        if (lane == 0) bar_arrive(smem_addr(&full[s]));
-        __syncwarp();
-        continue;
-      }
-      const uint32_t fb = smem_addr(&full[s]);
-      if (lane == 0) {
-        bar_expect_tx(fb, static_cast<uint32_t>(k * bytes));
-        pending |= 1u << s;
-        pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
-      }
-      for (int j = 0; j < k; ++j) {
-        const long long pj = __shfl_sync(0xffffffffu, my_pos, j);
-        if (lane == 0) bulk_load(st0 + s * stage_bytes + j * piece, O + pj * row_bytes + off, bytes, fb);
-      }
-      __syncwarp();
-    }
-    if (lane == 0)
-      for (int s = 0; s < stages; ++s)
-        if (pending & (1u << s)) bar_wait(smem_addr(&full[s]), (pend_parity >> s) & 1, err);
-    __syncwarp();
-  } else {
-    // ---- consumers: thread c sums the 16-byte vectors c, c + 128, ... of the piece
-    const int c = threadIdx.x - 32;
-    int q = 0;
-    for (long long it = blockIdx.x; it < items; it += gridDim.x, ++q) {
-      const long long t = it / pieces;
-      const int off = static_cast<int>(it - t * pieces) * piece;
-      const int bytes = min(piece, row_bytes - off);
-      const int s = q % stages;
-      if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&full[s]), (q / stages) & 1, err))) break;
-      if (valid[s]) {
-        for (int v = c; v * 16 < bytes; v += CB_CONSUMERS) {
-          float acc[VN];
-#pragma unroll
-          for (int i = 0; i < VN; ++i) acc[i] = 0.f;
-          const uint8_t* sp = csm + s * stage_bytes + v * 16;
-          for (int j = 0; j < k; ++j) {
-            const float wj = sw[s][j];
-            float o[VN];
-            load16(reinterpret_cast<const T*>(sp + j * piece), o);
-#pragma unroll
-            for (int i = 0; i < VN; ++i) acc[i] = fmaf(wj, o[i], acc[i]);
-          }
-          store16(reinterpret_cast<T*>(y + t * row_bytes + off + v * 16), acc);
-        }
-      }
-      bar_arrive(smem_addr(&empty[s]));
-    }
-  }
-}
-
-// The two backward gather kernels below use the same producer / consumer ring as combine: warp 0
-// loads a work item's row pieces (piece bytes each) with bulk copies into a stage and posts the
-// item's per-slot scalars there; four consumer warps (GB_CONSUMERS threads, one 16-byte vector
-// each) read the stage.  KM >= k bounds the per-thread slot arrays so they stay in registers.
+// The combine's backward below runs a producer / consumer ring: warp 0 loads a work item's row
+// pieces (piece bytes each) with bulk copies into a stage and posts the item's per-slot scalars
+// there; four consumer warps (GB_CONSUMERS threads, one 16-byte vector each) read the stage.
+// KM >= k bounds the per-thread slot arrays so they stay in registers.
 __device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(GB_CONSUMERS) : "memory"); }
 // Barrier of the consumer warps that also ANDs a flag over them: every consumer warp takes the
 // same decision (to go on or to stop), so none is left waiting at a barrier another has left.
@@ -408,139 +306,174 @@ __global__ void __launch_bounds__(32 + GB_CONSUMERS) combine_bwd_bulk_kernel(
   }
 }
 
-// Per token t (work items are its row pieces, in order): dx[t] = sum_j dX_pft[pos[t, j]] +
-// sum_j dz_j Wg^T[ids[t, j]], with dz_j = w_j (g_j - sum_l w_l g_l) the gradient of the selected
-// logits.  Stage: the k dX_pft pieces, then the k Wg^T row pieces; the producer warp computes dz
-// and, after issuing a token's first piece, writes its dense dlogits row (and the BF16 copy the
-// dWg GEMM reads) while the consumers sum.
-template <typename T>
-__global__ void __launch_bounds__(32 + GB_CONSUMERS) token_grad_bulk_kernel(
-    const char* __restrict__ dxp, const int32_t* __restrict__ pos, const float* __restrict__ g,
-    const float* __restrict__ w, const int32_t* __restrict__ ids, const char* __restrict__ wgT, int Tn, int k, int E,
-    int row_bytes, int piece, int pieces, int stages, char* __restrict__ dx, float* __restrict__ dlogits,
-    __nv_bfloat16* __restrict__ dz_bf16, int32_t* err) {
-  constexpr int VN = Vec<T>::n;
-  extern __shared__ __align__(128) uint8_t csm[];
-  __shared__ __align__(8) uint64_t full[8];
-  __shared__ __align__(8) uint64_t empty[8];
-  __shared__ int valid[8];
-  __shared__ float sdz[8][32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long N = static_cast<long long>(Tn) * k;
-  const uint32_t stage_bytes = static_cast<uint32_t>(2 * k) * piece;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < stages; ++s) {
-      bar_init(smem_addr(&full[s]), 1);
-      bar_init(smem_addr(&empty[s]), GB_CONSUMERS);
-    }
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+constexpr int WARPS = 8;   // warps per block
+
+inline int token_grid(long long T) {
+  long long b = (T + WARPS - 1) / WARPS;
+  const long long cap = static_cast<long long>(num_sms()) * 16;
+  if (b > cap) b = cap;
+  return static_cast<int>(b < 1 ? 1 : b);
+}
+
+// Grid for `items` one-warp work items (grid-stride beyond 16 blocks of 8 warps per SM).
+inline int item_grid(long long items) { return token_grid(items); }
+
+// Lane j < k loads pos[t, j]; returns false (and flags) if any row index is out of range.
+__device__ __forceinline__ bool load_pos(const int32_t* pos, long long t, int k, long long N, int lane, int& my_pos,
+                                         int32_t* err) {
+  my_pos = lane < k ? pos[t * k + lane] : 0;
+  const bool bad = lane < k && (my_pos < 0 || my_pos >= N);
+  if (__any_sync(0xffffffffu, bad)) {
+    if (lane == 0) dev_error(err, PFMOE_DEV_BAD_POS);
+    return false;
   }
-  __syncthreads();
-  const uint32_t st0 = smem_addr(csm);
-  if (warp == 0) {
-    uint32_t pending = 0, pend_parity = 0;
-    int q = 0;
-    bool ok = true;
-    for (long long t = blockIdx.x; t < Tn && ok; t += gridDim.x) {
-      const long long tk = t * k;
-      const int my_pos = lane < k ? pos[tk + lane] : 0;
-      const bool bad = lane < k && (my_pos < 0 || my_pos >= N);
-      const bool any_bad = __any_sync(0xffffffffu, bad);
-      if (any_bad && lane == 0) dev_error(err, PFMOE_DEV_BAD_POS);
-      const float my_w = lane < k ? w[tk + lane] : 0.f;
-      const float my_g = lane < k ? g[tk + lane] : 0.f;
-      int my_id = lane < k ? ids[tk + lane] : 0;
-      if (lane < k && static_cast<unsigned>(my_id) >= static_cast<unsigned>(E)) {
-        dev_error(err, PFMOE_DEV_BAD_EXPERT_ID);
-        my_id = 0;
-      }
-      const float inner = warp_sum(my_w * my_g);
-      const float my_dz = lane < k ? my_w * (my_g - inner) : 0.f;
-      for (int c = 0; c < pieces; ++c, ++q) {
-        const int off = c * piece;
-        const int bytes = min(piece, row_bytes - off);
-        const int s = q % stages;
-        const uint32_t ph = (q / stages) & 1;
-        if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&empty[s]), ph ^ 1, err))) { ok = false; break; }
-        sdz[s][lane] = my_dz;
-        if (lane == 0) valid[s] = any_bad ? 0 : 1;
-        __syncwarp();
-        const uint32_t fb = smem_addr(&full[s]);
-        if (any_bad) {
-          if (lane == 0) bar_arrive(fb);
-          __syncwarp();
-          continue;
-        }
-        if (lane == 0) {
-          bar_expect_tx(fb, static_cast<uint32_t>(2 * k * bytes));
-          pending |= 1u << s;
-          pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
-        }
-        const uint32_t sb = st0 + s * stage_bytes;
-        for (int j = 0; j < k; ++j) {
-          const long long pj = __shfl_sync(0xffffffffu, my_pos, j);
-          const long long ij = __shfl_sync(0xffffffffu, my_id, j);
-          if (lane == 0) {
-            bulk_load(sb + j * piece, dxp + pj * row_bytes + off, bytes, fb);
-            bulk_load(sb + (k + j) * piece, wgT + ij * row_bytes + off, bytes, fb);
-          }
-        }
-        __syncwarp();
-        if (c == 0) {
-          // the dense dlogits row (and its BF16 copy), while the consumers sum the first piece
-          for (int e0 = 0; e0 < E; e0 += 32) {
-            const int e = e0 + lane;
-            float val = 0.f;
-            for (int j = 0; j < k; ++j) {
-              const int idj = __shfl_sync(0xffffffffu, my_id, j);
-              const float dzj = __shfl_sync(0xffffffffu, my_dz, j);
-              if (idj == e) val = dzj;
-            }
-            if (e < E) {
-              dlogits[t * E + e] = val;
-              if (dz_bf16) dz_bf16[t * E + e] = __float2bfloat16_rn(val);
-            }
-          }
+  return true;
+}
+
+// The gather-sum kernels below take one work item per warp: a (token, column chunk) pair, the
+// chunk being the 32 * VN columns one warp covers with one 16-byte vector per lane.  Every lane
+// then has all k row loads of its chunk in flight at once, and a token's chunks sit on
+// neighbouring warps (its pos / weight rows stay in L1).  Sums still run over the k slots in
+// slot order with float32 accumulation, so results do not depend on the launch shape.
+template <typename T>
+__host__ __device__ inline int chunk_cols() { return 32 * Vec<T>::n; }
+
+// Items per token when each item covers U column chunks.
+__host__ __device__ inline int items_per_token(int d, int vn, int U) {
+  const int C = (d + 32 * vn - 1) / (32 * vn);
+  return (C + U - 1) / U;
+}
+
+// y[t] = sum_j w[t, j] * O[pos[t, j]].  An item covers U consecutive column chunks.
+template <typename T, int U>
+__global__ void __launch_bounds__(WARPS * 32) combine_kernel(const T* __restrict__ O, const int32_t* __restrict__ pos,
+                                                             const float* __restrict__ w, int Tn, int k, int d,
+                                                             T* __restrict__ y, int32_t* err) {
+  constexpr int VN = Vec<T>::n;
+  const int lane = threadIdx.x & 31;
+  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  const long long N = static_cast<long long>(Tn) * k;
+  const int CU = items_per_token(d, VN, U);
+  const long long items = static_cast<long long>(Tn) * CU;
+  for (long long it = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; it < items; it += nw) {
+    const long long t = it / CU;
+    const int cb = static_cast<int>(it - t * CU) * U * chunk_cols<T>() + lane * VN;
+    int my_pos;
+    if (!load_pos(pos, t, k, N, lane, my_pos, err)) continue;
+    const float my_w = lane < k ? w[t * k + lane] : 0.f;
+    float acc[U][VN];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int i = 0; i < VN; ++i) acc[u][i] = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < k; ++j) {
+      const long long p = __shfl_sync(0xffffffffu, my_pos, j);
+      const float wj = __shfl_sync(0xffffffffu, my_w, j);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c0 = cb + u * chunk_cols<T>();
+        if (c0 < d) {
+          float o[VN];
+          load16(O + p * d + c0, o);
+#pragma unroll
+          for (int i = 0; i < VN; ++i) acc[u][i] = fmaf(wj, o[i], acc[u][i]);
         }
       }
     }
-    if (lane == 0)
-      for (int s = 0; s < stages; ++s)
-        if (pending & (1u << s)) bar_wait(smem_addr(&full[s]), (pend_parity >> s) & 1, err);
-    __syncwarp();
-  } else {
-    const int c16 = threadIdx.x - 32;
-    int q = 0;
-    bool ok = true;
-    for (long long t = blockIdx.x; t < Tn && ok; t += gridDim.x)
-    for (int c = 0; c < pieces; ++c, ++q) {
-      const int off = c * piece;
-      const int bytes = min(piece, row_bytes - off);
-      const int s = q % stages;
-      if (!__all_sync(0xffffffffu, bar_wait(smem_addr(&full[s]), (q / stages) & 1, err))) { ok = false; break; }
-      if (valid[s]) {
-        for (int vv = c16; vv * 16 < bytes; vv += GB_CONSUMERS) {
-          float acc[VN];
 #pragma unroll
-          for (int i = 0; i < VN; ++i) acc[i] = 0.f;
-          const uint8_t* sp = csm + s * stage_bytes + vv * 16;
-          for (int j = 0; j < k; ++j) {
-            float v[VN];
-            load16(reinterpret_cast<const T*>(sp + j * piece), v);
-#pragma unroll
-            for (int i = 0; i < VN; ++i) acc[i] += v[i];
-          }
-          for (int j = 0; j < k; ++j) {
-            float v[VN];
-            load16(reinterpret_cast<const T*>(sp + (k + j) * piece), v);
-            const float dzj = sdz[s][j];
-#pragma unroll
-            for (int i = 0; i < VN; ++i) acc[i] = fmaf(dzj, v[i], acc[i]);
-          }
-          store16(reinterpret_cast<T*>(dx + t * row_bytes + off + vv * 16), acc);
+    for (int u = 0; u < U; ++u) {
+      const int c0 = cb + u * chunk_cols<T>();
+      if (c0 < d) store16(y + t * d + c0, acc[u]);
+    }
+  }
+}
+
+// dz_{t, ids[t,j]} = w_j (g_j - sum_l w_l g_l) (zero elsewhere);
+// dx[t] = sum_j dX_pft[pos[t, j]] + sum_j dz_j * Wg^T[ids[t, j]].
+// The dense dlogits row (and its BF16 copy for the dWg GEMM) is written by the token's chunk-0 item.
+template <typename T, int U>
+__global__ void __launch_bounds__(WARPS * 32) token_grad_kernel(const T* __restrict__ dxp, const int32_t* __restrict__ pos,
+                                                                const float* __restrict__ g, const float* __restrict__ w,
+                                                                const int32_t* __restrict__ ids,
+                                                                const T* __restrict__ wgT, int Tn, int k, int d, int E,
+                                                                T* __restrict__ dx, float* __restrict__ dlogits,
+                                                                __nv_bfloat16* __restrict__ dz_bf16, int32_t* err) {
+  constexpr int VN = Vec<T>::n;
+  const int lane = threadIdx.x & 31;
+  const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  const long long N = static_cast<long long>(Tn) * k;
+  const int CU = items_per_token(d, VN, U);
+  const long long items = static_cast<long long>(Tn) * CU;
+  for (long long it = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; it < items; it += nw) {
+    const long long t = it / CU;
+    const int ch = static_cast<int>(it - t * CU);
+    const int cb = ch * U * chunk_cols<T>() + lane * VN;
+    int my_pos;
+    if (!load_pos(pos, t, k, N, lane, my_pos, err)) continue;
+    const long long tk = t * k;
+    const float my_w = lane < k ? w[tk + lane] : 0.f;
+    const float my_g = lane < k ? g[tk + lane] : 0.f;
+    int my_id = lane < k ? ids[tk + lane] : 0;
+    if (lane < k && static_cast<unsigned>(my_id) >= static_cast<unsigned>(E)) {
+      dev_error(err, PFMOE_DEV_BAD_EXPERT_ID);
+      my_id = 0;
+    }
+    const float inner = warp_sum(my_w * my_g);
+    const float my_dz = lane < k ? my_w * (my_g - inner) : 0.f;
+    if (ch == 0) {
+      for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        float val = 0.f;
+        for (int j = 0; j < k; ++j) {
+          const int idj = __shfl_sync(0xffffffffu, my_id, j);
+          const float dzj = __shfl_sync(0xffffffffu, my_dz, j);
+          if (idj == e) val = dzj;
+        }
+        if (e < E) {
+          dlogits[t * E + e] = val;
+          if (dz_bf16) dz_bf16[t * E + e] = __float2bfloat16_rn(val);
         }
       }
-      bar_arrive(smem_addr(&empty[s]));
+    }
+    float acc[U][VN];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int i = 0; i < VN; ++i) acc[u][i] = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < k; ++j) {
+      const long long p = __shfl_sync(0xffffffffu, my_pos, j);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c0 = cb + u * chunk_cols<T>();
+        if (c0 < d) {
+          float v[VN];
+          load16(dxp + p * d + c0, v);
+#pragma unroll
+          for (int i = 0; i < VN; ++i) acc[u][i] += v[i];
+        }
+      }
+    }
+#pragma unroll 8
+    for (int j = 0; j < k; ++j) {
+      const long long idj = __shfl_sync(0xffffffffu, my_id, j);
+      const float dzj = __shfl_sync(0xffffffffu, my_dz, j);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c0 = cb + u * chunk_cols<T>();
+        if (c0 < d) {
+          float v[VN];
+          load16(wgT + idj * d + c0, v);
+#pragma unroll
+          for (int i = 0; i < VN; ++i) acc[u][i] = fmaf(dzj, v[i], acc[u][i]);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c0 = cb + u * chunk_cols<T>();
+      if (c0 < d) store16(dx + t * d + c0, acc[u]);
     }
   }
 }
@@ -605,29 +538,6 @@ static Ring ring_for(int row_bytes, int slots, int budget, int piece_cap) {
   return r;
 }
 
-int launch_combine(const void* out, const int32_t* pos, const float* w, int T, int k, int d, int dtype, void* y,
-                   int32_t* err, cudaStream_t s) {
-  const int row_bytes = d * (dtype == PFMOE_BF16 ? 2 : 4);
-  const Ring r = ring_for(row_bytes, k, 200 * 1024, CB_PIECE);
-  const long long items = static_cast<long long>(T) * r.pieces;
-  long long grid = static_cast<long long>(num_sms()) * r.ctas_per_sm;
-  if (grid > items) grid = items;
-  if (dtype == PFMOE_BF16) {
-    PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&combine_bulk_kernel<__nv_bfloat16>), 227 * 1024, "combine"));
-    PFMOE_LAUNCH("combine", s,
-                 (combine_bulk_kernel<__nv_bfloat16><<<static_cast<int>(grid), 32 + CB_CONSUMERS, r.smem, s>>>(
-                     static_cast<const char*>(out), pos, w, T, k, row_bytes, r.piece, r.pieces, r.stages,
-                     static_cast<char*>(y), err)));
-  } else {
-    PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&combine_bulk_kernel<float>), 227 * 1024, "combine"));
-    PFMOE_LAUNCH("combine", s,
-                 (combine_bulk_kernel<float><<<static_cast<int>(grid), 32 + CB_CONSUMERS, r.smem, s>>>(
-                     static_cast<const char*>(out), pos, w, T, k, row_bytes, r.piece, r.pieces, r.stages,
-                     static_cast<char*>(y), err)));
-  }
-  return PFMOE_OK;
-}
-
 template <typename T, int KM>
 static int launch_cbwd_t(const void* dy, const void* out, const int32_t* pos, const float* w, int T_, int k,
                          int row_bytes, const Ring& r, int grid, void* dO, float* g, int32_t* err, cudaStream_t s) {
@@ -670,27 +580,56 @@ int launch_transpose(const void* in, int rows, int cols, int dtype, void* out, c
   return PFMOE_OK;
 }
 
+// Column chunks per work item: one for rows of up to 16 chunks (d <= 4096 BF16), else 4, which
+// keeps the per-token prologue (pos / weight loads, dlogits row) off wide rows.
+static int chunks_per_item(int d, int vn) { return (d + 32 * vn - 1) / (32 * vn) > 16 ? 4 : 1; }
+
+int launch_combine(const void* out, const int32_t* pos, const float* w, int T, int k, int d, int dtype, void* y,
+                   int32_t* err, cudaStream_t s) {
+  const int vn = dtype == PFMOE_BF16 ? 8 : 4;
+  const int U = chunks_per_item(d, vn);
+  const int g = item_grid(static_cast<long long>(T) * items_per_token(d, vn, U));
+  if (dtype == PFMOE_BF16) {
+    const auto* o = static_cast<const __nv_bfloat16*>(out);
+    auto* yy = static_cast<__nv_bfloat16*>(y);
+    if (U == 4) PFMOE_LAUNCH("combine", s, (combine_kernel<__nv_bfloat16, 4><<<g, WARPS * 32, 0, s>>>(o, pos, w, T, k, d, yy, err)));
+    else PFMOE_LAUNCH("combine", s, (combine_kernel<__nv_bfloat16, 1><<<g, WARPS * 32, 0, s>>>(o, pos, w, T, k, d, yy, err)));
+  } else {
+    const auto* o = static_cast<const float*>(out);
+    auto* yy = static_cast<float*>(y);
+    if (U == 4) PFMOE_LAUNCH("combine", s, (combine_kernel<float, 4><<<g, WARPS * 32, 0, s>>>(o, pos, w, T, k, d, yy, err)));
+    else PFMOE_LAUNCH("combine", s, (combine_kernel<float, 1><<<g, WARPS * 32, 0, s>>>(o, pos, w, T, k, d, yy, err)));
+  }
+  return PFMOE_OK;
+}
+
 int launch_token_grad(const void* dx_pft, const int32_t* pos, const float* g, const float* w, const int32_t* ids,
                       const void* wgT, int T, int k, int d, int E, int dtype, void* dx, float* dlogits,
                       void* dz_bf16, int32_t* err, cudaStream_t s) {
-  const int row_bytes = d * (dtype == PFMOE_BF16 ? 2 : 4);
-  const Ring r = ring_for(row_bytes, 2 * k, 96 * 1024, 2048);
-  long long grid = static_cast<long long>(num_sms()) * r.ctas_per_sm;
-  if (grid > T) grid = T;
+  const int vn = dtype == PFMOE_BF16 ? 8 : 4;
+  const int U = chunks_per_item(d, vn);
+  const int gr = item_grid(static_cast<long long>(T) * items_per_token(d, vn, U));
   auto* dzb = static_cast<__nv_bfloat16*>(dz_bf16);
   if (dtype == PFMOE_BF16) {
-    PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&token_grad_bulk_kernel<__nv_bfloat16>), 227 * 1024,
-                         "token_grad"));
-    PFMOE_LAUNCH("token_grad", s,
-                 (token_grad_bulk_kernel<__nv_bfloat16><<<static_cast<int>(grid), 32 + GB_CONSUMERS, r.smem, s>>>(
-                     static_cast<const char*>(dx_pft), pos, g, w, ids, static_cast<const char*>(wgT), T, k, E,
-                     row_bytes, r.piece, r.pieces, r.stages, static_cast<char*>(dx), dlogits, dzb, err)));
+    const auto* a = static_cast<const __nv_bfloat16*>(dx_pft);
+    const auto* wt = static_cast<const __nv_bfloat16*>(wgT);
+    auto* o = static_cast<__nv_bfloat16*>(dx);
+    if (U == 4)
+      PFMOE_LAUNCH("token_grad", s, (token_grad_kernel<__nv_bfloat16, 4><<<gr, WARPS * 32, 0, s>>>(
+                                         a, pos, g, w, ids, wt, T, k, d, E, o, dlogits, dzb, err)));
+    else
+      PFMOE_LAUNCH("token_grad", s, (token_grad_kernel<__nv_bfloat16, 1><<<gr, WARPS * 32, 0, s>>>(
+                                         a, pos, g, w, ids, wt, T, k, d, E, o, dlogits, dzb, err)));
   } else {
-    PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&token_grad_bulk_kernel<float>), 227 * 1024, "token_grad"));
-    PFMOE_LAUNCH("token_grad", s,
-                 (token_grad_bulk_kernel<float><<<static_cast<int>(grid), 32 + GB_CONSUMERS, r.smem, s>>>(
-                     static_cast<const char*>(dx_pft), pos, g, w, ids, static_cast<const char*>(wgT), T, k, E,
-                     row_bytes, r.piece, r.pieces, r.stages, static_cast<char*>(dx), dlogits, dzb, err)));
+    const auto* a = static_cast<const float*>(dx_pft);
+    const auto* wt = static_cast<const float*>(wgT);
+    auto* o = static_cast<float*>(dx);
+    if (U == 4)
+      PFMOE_LAUNCH("token_grad", s, (token_grad_kernel<float, 4><<<gr, WARPS * 32, 0, s>>>(
+                                         a, pos, g, w, ids, wt, T, k, d, E, o, dlogits, dzb, err)));
+    else
+      PFMOE_LAUNCH("token_grad", s, (token_grad_kernel<float, 1><<<gr, WARPS * 32, 0, s>>>(
+                                         a, pos, g, w, ids, wt, T, k, d, E, o, dlogits, dzb, err)));
   }
   return PFMOE_OK;
 }
