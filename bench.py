@@ -592,9 +592,10 @@ def run_ours(args):
     dom_ms = kern[dom][1] / kern[dom][0]
     if kind == "tensor":
         ach = work / (dom_ms * 1e-3) / 1e12
+        burst = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
         roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": tc_peak, "unit": "TFLOP/s",
                 "frac": ach / tc_peak, "traffic": traffic_for(dom, cfg.name), "peak_source": tc_src,
-                "work_per_launch": work, "ms_per_launch": dom_ms}
+                "frac_of_burst": ach / burst, "work_per_launch": work, "ms_per_launch": dom_ms}
     else:
         ach = work / (dom_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
