@@ -681,10 +681,15 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
         const uint32_t sb = sa + a_bytes;
         tc_fence_after();
         if (lane == 0) {
-          for (int kk = 0; kk < kk_count; ++kk) {
-            const uint64_t ad = sdesc(sa + kk * a_step, a_lbo, 1024);
-            const uint64_t bd = sdesc(sb + kk * b_step, b_lbo, 1024);
-            tc_mma(tmem_d, ad, bd, idesc, (kb | kk) != 0);
+          // Unrolled with a predicate: one thread issues these, and a rolled loop over a runtime
+          // count measured 2-5 % slower on the weight-gradient kernels at d = 7168.
+#pragma unroll
+          for (int kk = 0; kk < KBK / 16; ++kk) {
+            if (kk < kk_count) {
+              const uint64_t ad = sdesc(sa + kk * a_step, a_lbo, 1024);
+              const uint64_t bd = sdesc(sb + kk * b_step, b_lbo, 1024);
+              tc_mma(tmem_d, ad, bd, idesc, (kb | kk) != 0);
+            }
           }
           tc_commit(smem_u32(&empty[s]));
         }
