@@ -154,6 +154,21 @@ PFMOE_API int moe_expert_ffn(const void* x_pft, const int32_t* expert_offsets, c
                    void* h1, void* h3, void* a, void* out, int32_t* err, void* stream);
 
 /*
+ * moe_expert_ffn_gathered -- moe_expert_ffn with the dispatch gather fused into the
+ *   first expert GEMM ([A] §2.1.2: the expert reads its rows by token id; [A] §1 and
+ *   §2.1.1: dispatch buffers dominate activation memory).  Row r of the expert input
+ *   is x[token_ids[r]] (x [T,d]; token_ids [N] from pft_build), read straight into the
+ *   GEMM's operand ring: no [N,d] copy of x is written.  Same outputs, layout and
+ *   tolerance as moe_expert_ffn.  BF16 only (PFMOE_ERR_UNSUPPORTED otherwise); d and
+ *   h multiples of 8.  token_ids must hold valid token indices (< T) for all N rows:
+ *   the kernel does not check them.
+ */
+PFMOE_API int moe_expert_ffn_gathered(const void* x, const int32_t* token_ids, const int32_t* expert_offsets,
+                            const int32_t* tile_offsets, int N, int E, int d, int h, int dtype, const void* w1,
+                            const void* w3, const void* w2, void* h1, void* h3, void* a, void* out, int32_t* err,
+                            void* stream);
+
+/*
  * moe_combine -- y[t] = sum_{j<k} topk_w[t,j] * out[pos[t,j]] ([A] §2.1.1
  *   combine_weights; [B] 训练流程 step d), summed in slot order in float32 and
  *   rounded once.  Deterministic (no atomics).  y [T,d] out.

@@ -36,6 +36,7 @@ SIGNATURES = {
     "pft_build_no_ws": (_I, [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "moe_expert_ffn": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_expert_ffn_gathered": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "moe_backward_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
     "moe_backward": (_I, [_P] * 16 + [_I] * 6 + [_P] * 7 + [_Z, _P, _P]),
@@ -152,6 +153,14 @@ def moe_expert_ffn(x_pft, expert_offsets, tile_offsets, N, E, d, h, dtype, w1, w
     _check("moe_expert_ffn", lib().moe_expert_ffn(_ptr(x_pft), _ptr(expert_offsets), _ptr(tile_offsets), N, E, d, h,
                                                   dtype, _ptr(w1), _ptr(w3), _ptr(w2), _ptr(h1), _ptr(h3), _ptr(a),
                                                   _ptr(out), _ptr(err), _stream(stream)))
+
+
+def moe_expert_ffn_gathered(x, token_ids, expert_offsets, tile_offsets, N, E, d, h, dtype, w1, w3, w2, h1, h3, a, out,
+                            err=None, stream=None):
+    _check("moe_expert_ffn_gathered",
+           lib().moe_expert_ffn_gathered(_ptr(x), _ptr(token_ids), _ptr(expert_offsets), _ptr(tile_offsets), N, E, d,
+                                         h, dtype, _ptr(w1), _ptr(w3), _ptr(w2), _ptr(h1), _ptr(h3), _ptr(a),
+                                         _ptr(out), _ptr(err), _stream(stream)))
 
 
 def moe_combine(out, pos, topk_w, T, k, d, dtype, y, err=None, stream=None):

@@ -291,6 +291,33 @@ int moe_dispatch(const void* x, const int32_t* pos, int T, int k, int d, int dty
   return launch_dispatch(x, pos, T, k, d, dtype, x_pft, err, st(stream));
 }
 
+int moe_expert_ffn_gathered(const void* x, const int32_t* token_ids, const int32_t* expert_offsets,
+                            const int32_t* tile_offsets, int N, int E, int d, int h, int dtype, const void* w1,
+                            const void* w3, const void* w2, void* h1, void* h3, void* a, void* out, int32_t* err,
+                            void* stream) {
+  set_error("");
+  PFMOE_TRY(need_dtype(dtype));
+  if (dtype != PFMOE_BF16) return fail(PFMOE_ERR_UNSUPPORTED, "moe_expert_ffn_gathered: BF16 only");
+  if (N < 0 || E <= 0) return fail(PFMOE_ERR_ARG, "need N >= 0 and E > 0");
+  PFMOE_TRY(need_width(d, "d", dtype));
+  PFMOE_TRY(need_width(h, "h", dtype));
+  if (N == 0) return PFMOE_OK;
+  PFMOE_TRY(need_ptr(x, "x"));
+  PFMOE_TRY(need_ptr(token_ids, "token_ids"));
+  PFMOE_TRY(need_ptr(expert_offsets, "expert_offsets"));
+  PFMOE_TRY(need_ptr(tile_offsets, "tile_offsets"));
+  PFMOE_TRY(need_ptr(w1, "w1"));
+  PFMOE_TRY(need_ptr(w3, "w3"));
+  PFMOE_TRY(need_ptr(w2, "w2"));
+  PFMOE_TRY(need_ptr(h1, "h1"));
+  PFMOE_TRY(need_ptr(h3, "h3"));
+  PFMOE_TRY(need_ptr(a, "a"));
+  PFMOE_TRY(need_ptr(out, "out"));
+  cudaStream_t s = st(stream);
+  PFMOE_TRY(tc_ffn_gemm1_gather(x, token_ids, expert_offsets, tile_offsets, N, E, d, h, w1, w3, h1, h3, a, err, s));
+  return tc_ffn_gemm2(a, expert_offsets, tile_offsets, N, E, d, h, w2, out, err, s);
+}
+
 int moe_expert_ffn(const void* x_pft, const int32_t* expert_offsets, const int32_t* tile_offsets, int N, int E, int d,
                    int h, int dtype, const void* w1, const void* w3, const void* w2, void* h1, void* h3, void* a,
                    void* out, int32_t* err, void* stream) {

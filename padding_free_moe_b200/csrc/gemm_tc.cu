@@ -44,6 +44,11 @@ constexpr int BM = 128;          // MMA M (one CTA)
 constexpr int BK = 64;           // K elements per stage (one 128-byte swizzle row of BF16)
 constexpr int MAX_STAGES = 8;
 constexpr int THREADS = 192;
+// Token-as-N kernel with the token rows gathered into the B ring (no PFT copy of x): four more
+// warps copy the rows with 16-byte cp.async (TMA tile::gather4 moves 512 bytes per copy and
+// measured 16 GB/s per SM on this part, against 83 GB/s for four warps of cp.async).
+constexpr int GATHER_WARPS = 4;
+constexpr int THREADS_GATHER = THREADS + 32 * (GATHER_WARPS + 1);   // + one relay warp
 // K-grouped (weight-gradient) launches: KG_EPI_WARPS epilogue warps (a multiple of 4; with 8, two
 // per TMEM lane quarter each write half of a tile's column blocks) and a K-tail zeroing warp after
 // them.  Four warps with two staging slabs each measured as fast as eight with one or two.
@@ -97,6 +102,9 @@ struct Params {
   const float* bias; // STORE_F32: optional per-column bias
   long long ldd;     // output row stride (elements)
   long long d_gstride;  // KG: elements between consecutive groups' outputs
+  const int32_t* gather_ids;  // token-as-N with gathered B: PFT row -> token (token_ids)
+  const void* gather_src;      // token rows [T, gather_ld] the B operand is gathered from
+  long long gather_ld;
   int32_t* err;
 };
 
@@ -880,6 +888,11 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
+// 16-byte global -> shared copy (cp.async, L2 only); bytes past src_bytes (0 or 16) are zero-filled.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
@@ -1312,8 +1325,8 @@ __device__ __forceinline__ void epilogue_tn(const Params& p, const TnTile& tl, u
   }
 }
 
-template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+template <int EPI, bool GATHER = false>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GATHER ? THREADS_GATHER : THREADS, 1)
     grouped_gemm_tn_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1328,7 +1341,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint64_t* acc_full = empty + MAX_STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* landed = drain + 1;   // gathered B: stage s's copies of this CTA have landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(landed + MAX_STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -1341,8 +1355,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(smem_u32(&full[s]), 1);
+      // with gathered rows: the producer's expect_tx plus the relay of each CTA of the pair
+      mbar_init(smem_u32(&full[s]), GATHER ? 3 : 1);
       mbar_init(smem_u32(&empty[s]), 1);
+      if (GATHER) mbar_init(smem_u32(&landed[s]), 32 * GATHER_WARPS);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&acc_full[b]), 1);
@@ -1371,7 +1387,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (lane == 0) pair_off[p.G] = carry;
     if (lane == 0) {
       prefetch_tmap(&p.tmA[0]);
-      prefetch_tmap(&p.tmB[0]);
+      if (!GATHER) prefetch_tmap(&p.tmB[0]);   // gathered B has no tensor map
     }
   }
   if (warp == 1) {
@@ -1399,7 +1415,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // them are not read by the MMA).  Smaller boxes for ragged tiles measured slower: TMA
         // delivery per copy has a fixed cost.
         const int tokc = tl.tok0 + static_cast<int>(rank) * (tl.nmma / 2);
-        const uint32_t tx = 2 * stage_bytes;
+        const uint32_t tx = GATHER ? 2 * (2 * TN_SUB) : 2 * stage_bytes;   // gathered: A only
         for (int kb = 0; kb < tl.nk; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
@@ -1413,6 +1429,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           const int kk = (src == 0 ? kb : kb - p.k0_blocks) * TN_BK;
           pending |= 1u << s;
           pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
+          if (lane == 1 && GATHER) continue;   // the gather warps fill B
           if (lane == 1) {
             const CUtensorMap* tb = &p.tmB[p.nsplit ? 0 : src];
             tma_load_3d_pair(sb, tb, fb, kk, tokc, 0);
@@ -1494,6 +1511,70 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
       __syncwarp();
     }
+  } else if (GATHER && warp >= THREADS / 32 && warp < THREADS / 32 + GATHER_WARPS) {
+    // ------------------------------------------------------------ token-row gather (both CTAs)
+    // The dispatch gather of the X-MoE article (§2.1.2) fused into the operand ring: row r of this
+    // CTA's B block is token row gather_src[gather_ids[tokc + r]], so no PFT copy of x exists.
+    // Thread gt copies 16-byte chunk (gt & 7) of 64-column half ((gt >> 3) & 1) of rows
+    // (gt >> 4) + 2 GATHER_WARPS i into the same 128-byte-swizzled layout a TMA box load writes (a
+    // warp covers two whole rows per step: 512 contiguous bytes of x), then hands the
+    // stage's completion to landed[s] (cp.async.mbarrier.arrive) and moves on: like the TMA
+    // producer it runs up to a full ring ahead of the MMA.
+    constexpr int RPT = 128 * 16 / (32 * GATHER_WARPS);   // rows per thread
+    const int gt = threadIdx.x - THREADS;
+    const int half = (gt >> 3) & 1, chunk = gt & 7, row_lo = gt >> 4;
+    const __nv_bfloat16* xs = static_cast<const __nv_bfloat16*>(p.gather_src);
+    int it = 0;
+    bool ok = true;
+    int wave = 0;
+    TnTile tl;
+    while (ok && tn_next(p, pair_off, npairs, pair, wave, tl)) {
+      const int rows = tl.nmma / 2;                          // B rows this CTA's half of the MMA reads
+      const int tokc = tl.tok0 + static_cast<int>(rank) * rows;
+      const int last = p.seg[p.G] - 1;                       // rows past the segment repeat a valid row
+      long long src_row[RPT];
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) {
+        const int r = max(0, min(tokc + i * (2 * GATHER_WARPS) + row_lo, last));
+        src_row[i] = static_cast<long long>(p.gather_ids[r]) * p.gather_ld;
+      }
+      for (int kb = 0; kb < tl.nk; ++kb, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1;
+        ok = __all_sync(0xffffffffu, wait_bar2(smem_u32(&empty[s]), ph ^ 1, abort_flag, p.err));
+        if (!ok) break;
+        const uint32_t sb = smem_u32(smem + s * stage_bytes) + 2 * TN_SUB + half * TN_SUB;
+        const long long col = static_cast<long long>(kb) * TN_BK + half * BK + chunk * 8;
+        const bool in = col < p.gather_ld;                   // columns past d read as zeros
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+          const int row = i * (2 * GATHER_WARPS) + row_lo;
+          if (row < rows) cp_async16(sb + row * 128 + ((chunk ^ (row & 7)) << 4), xs + src_row[i] + (in ? col : 0),
+                                     in ? 16 : 0);
+        }
+        // arrives on landed[s] once every copy this thread issued so far has landed
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&landed[s])) : "memory");
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");   // no copy in flight at exit
+  } else if (GATHER && warp == THREADS / 32 + GATHER_WARPS) {
+    // ------------------------------------------------------------ gather relay (both CTAs)
+    // Waits until a stage's gathered rows have landed, makes them visible to the tensor core's
+    // (async-proxy) reads with a proxy fence, and arrives on the leader's full barrier.
+    int it = 0;
+    bool ok = true;
+    int wave = 0;
+    TnTile tl;
+    while (ok && tn_next(p, pair_off, npairs, pair, wave, tl)) {
+      for (int kb = 0; kb < tl.nk; ++kb, ++it) {
+        const int s = it % S;
+        ok = __all_sync(0xffffffffu, wait_bar2(smem_u32(&landed[s]), (it / S) & 1, abort_flag, p.err));
+        if (!ok) break;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&full[s]), 0));
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;
@@ -1553,7 +1634,7 @@ static int max_pairs() {
 }
 
 // Token-as-N launcher (expert-segmented rows only).
-template <int EPI>
+template <int EPI, bool GATHER = false>
 static int launch_tn(Params& p, long long pair_tile_upper_bound, const char* name, cudaStream_t stream) {
   p.mode = RG;
   const int stage = TN_STAGE;
@@ -1567,12 +1648,13 @@ static int launch_tn(Params& p, long long pair_tile_upper_bound, const char* nam
   if (st < 2) return fail(PFMOE_ERR_UNSUPPORTED, std::string(name) + ": too many experts for the shared-memory plan");
   p.stages = st > MAX_STAGES ? MAX_STAGES : st;
   const size_t smem = fixed + static_cast<size_t>(p.stages) * stage;
-  PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&grouped_gemm_tn_kernel<EPI>), SMEM_LIMIT, name));
+  PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&grouped_gemm_tn_kernel<EPI, GATHER>), SMEM_LIMIT, name));
   if (pair_tile_upper_bound <= 0) return PFMOE_OK;
   long long pairs = max_pairs();
   if (pair_tile_upper_bound < pairs) pairs = pair_tile_upper_bound;
   PFMOE_LAUNCH(name, stream,
-               (grouped_gemm_tn_kernel<EPI><<<static_cast<int>(2 * pairs), THREADS, smem, stream>>>(p)));
+               (grouped_gemm_tn_kernel<EPI, GATHER><<<static_cast<int>(2 * pairs), GATHER ? THREADS_GATHER : THREADS, smem,
+                                                     stream>>>(p)));
   return PFMOE_OK;
 }
 
@@ -1680,6 +1762,29 @@ int tc_ffn_gemm1(const void* x_pft, const int* seg, const int* tiles, int N, int
   PFMOE_TRY(make_out_map_tn(&p.tmD[2], a, h, N, "a out"));
   p.tma_store = 1;
   return launch_tn<EPI_SWIGLU_FWD>(p, tn_tiles_ub(N, E, h, p.fstep), "ffn_gemm1_swiglu", s);
+}
+
+// The same with the expert rows gathered from x by token_ids inside the GEMM (X_pft[r] =
+// x[token_ids[r]], X-MoE article §2.1.2): the forward writes no PFT copy of x.
+int tc_ffn_gemm1_gather(const void* x, const int* token_ids, const int* seg, const int* tiles, int N, int E, int d,
+                        int h, const void* w1, const void* w3, void* h1, void* h3, void* a, int32_t* err,
+                        cudaStream_t s) {
+  Params p = base_params(err);
+  p.nsplit = 1;
+  p.Nout = h;
+  p.k0_blocks = (d + TN_BK - 1) / TN_BK;
+  p.seg = seg; p.tiles = tiles; p.G = E;
+  p.D0 = h1; p.D1 = h3; p.D2 = a; p.ldd = h;
+  p.a_major = 1;
+  p.fstep = 128;
+  p.gather_ids = token_ids; p.gather_src = x; p.gather_ld = d;
+  PFMOE_TRY(make_tmap(&p.tmA[0], w1, h, d, E, 64, TN_BK, "w1"));
+  PFMOE_TRY(make_tmap(&p.tmA[1], w3, h, d, E, 64, TN_BK, "w3"));
+  PFMOE_TRY(make_out_map_tn(&p.tmD[0], h1, h, N, "h1 out"));
+  PFMOE_TRY(make_out_map_tn(&p.tmD[1], h3, h, N, "h3 out"));
+  PFMOE_TRY(make_out_map_tn(&p.tmD[2], a, h, N, "a out"));
+  p.tma_store = 1;
+  return launch_tn<EPI_SWIGLU_FWD, true>(p, tn_tiles_ub(N, E, h, p.fstep), "ffn_gemm1_swiglu", s);
 }
 
 // O = A W2_e.

@@ -3,6 +3,13 @@
 Host plumbing only -- torch allocates the device buffers once, every compute
 step is a libpfmoe kernel.  Forward: moe_route -> pft_build -> moe_dispatch ->
 moe_expert_ffn -> moe_combine.  Backward: moe_backward.  RBD: rbd_plan.
+
+fused_gather=True (BF16 only) runs the forward as moe_route -> pft_build ->
+moe_expert_ffn_gathered (the first expert GEMM reads its rows from x by token id,
+so the forward writes no [N, d] copy of x) -> moe_combine, and the backward as
+moe_dispatch (the PFT copy of x, needed only by the weight gradients) ->
+moe_backward.  Same results bit for bit; it is off by default because the
+gathered GEMM is slower on B200 than dispatch plus the TMA-fed GEMM.
 """
 from __future__ import annotations
 
@@ -33,10 +40,11 @@ class Shape:
 class PFTMoELayer:
     """Buffers for one layer shape on one device; inputs/weights are passed per call."""
 
-    def __init__(self, shape: Shape, device="cuda"):
+    def __init__(self, shape: Shape, device="cuda", fused_gather=False):
         self.s = s = shape
         self.device = torch.device(device)
         self.code = L.dtype_code(s.dtype)
+        self.fused_gather = bool(fused_gather) and s.dtype == torch.bfloat16
         dev, f32, i32, dt = self.device, torch.float32, torch.int32, s.dtype
         T, d, E, h, k, N = s.T, s.d, s.E, s.h, s.k, s.N
         e = lambda *shape_, dtype=dt: torch.empty(*shape_, device=dev, dtype=dtype)
@@ -118,6 +126,11 @@ class PFTMoELayer:
         L.moe_expert_ffn(self.x_pft, self.expert_offsets, self.tile_offsets, s.N, s.E, s.d, s.h, self.code, w1, w3,
                          w2, self.h1, self.h3, self.a, self.out, self.err, stream)
 
+    def experts_gathered(self, x, w1, w3, w2, stream=None):
+        s = self.s
+        L.moe_expert_ffn_gathered(x, self.token_ids, self.expert_offsets, self.tile_offsets, s.N, s.E, s.d, s.h,
+                                  self.code, w1, w3, w2, self.h1, self.h3, self.a, self.out, self.err, stream)
+
     def combine(self, stream=None):
         s = self.s
         L.moe_combine(self.out, self.pos, self.topk_w, s.T, s.k, s.d, self.code, self.y, self.err, stream)
@@ -125,13 +138,18 @@ class PFTMoELayer:
     def forward(self, x, wg, bias, w1, w3, w2, stream=None):
         self.route(x, wg, bias, stream)
         self.build_pft(stream)
-        self.dispatch(x, stream)
-        self.experts(w1, w3, w2, stream)
+        if self.fused_gather:
+            self.experts_gathered(x, w1, w3, w2, stream)
+        else:
+            self.dispatch(x, stream)
+            self.experts(w1, w3, w2, stream)
         self.combine(stream)
         return self.y
 
     def backward(self, dy, x, wg, w1, w3, w2, stream=None):
         s = self.s
+        if self.fused_gather:
+            self.dispatch(x, stream)   # the PFT copy of x, for the weight gradients only
         L.moe_backward(dy, x, wg, self.topk_w, self.topk_ids, self.pos, self.expert_offsets, self.tile_offsets,
                        self.x_pft, self.h1, self.h3, self.a, self.out, w1, w3, w2, s.T, s.d, s.E, s.h, s.k, self.code,
                        self.dx, self.dwg, self.dw1, self.dw3, self.dw2, self.dlogits, self.bwd_ws, self.bwd_ws_bytes,
@@ -162,8 +180,11 @@ class PFTMoELayer:
             self.rbd(self.side)
             self.ev_rbd_done.record(self.side)
         self.build_pft(main)
-        self.dispatch(x, main)
-        self.experts(w1, w3, w2, main)
+        if self.fused_gather:
+            self.experts_gathered(x, w1, w3, w2, main)
+        else:
+            self.dispatch(x, main)
+            self.experts(w1, w3, w2, main)
         self.combine(main)
         self.backward(dy, x, wg, w1, w3, w2, main)
         if self.has_rbd and overlap_rbd:
