@@ -62,6 +62,8 @@ def parse():
     ap.add_argument("--extra-workloads", default=EXTRA_WORKLOADS,
                     help="comma-separated workloads timed after the headline one ('' = none)")
     ap.add_argument("--extra-steps", type=int, default=10)
+    ap.add_argument("--no-gathered", action="store_true",
+                    help="skip the timing of the step with the gather fused into the first expert GEMM")
     return ap.parse_args()
 
 
@@ -660,6 +662,32 @@ def run_ours(args):
         del lay2, inp2
         torch.cuda.empty_cache()
     line["workloads"] = extra
+
+    # ---- the same step with the dispatch gather fused into the first expert GEMM (no x_pft in the forward)
+    if cfg.dtype == "bf16" and not args.no_gathered:
+        lay3, inp3 = build_layer(cfg, rank, dev)
+        lay3.fused_gather = True
+
+        def step3():
+            lay3.step(inp3.x, inp3.wg, inp3.bias, inp3.w1, inp3.w3, inp3.w2, inp3.dy, stream)
+
+        for _ in range(warm):
+            step3()
+        torch.cuda.synchronize()
+        barrier()
+        ms3 = max_over_ranks(device_timed(step3, args.extra_steps, stream, torch)) / args.extra_steps
+        barrier()
+        k3, _ = per_kernel_pass(L, lay3, inp3, stream, args.extra_steps, torch, barrier)
+        if lay3.device_error() != 0:
+            raise RuntimeError(f"device error word {lay3.device_error():#x} in the gathered step")
+        per = {nm: k3[nm][1] / k3[nm][0] for nm in ("ffn_gemm1_swiglu", "dispatch") if nm in k3}
+        line["gathered_forward"] = {
+            "workload": cfg.name, "ms_per_step": ms3, "tokens_per_s": world * cfg.T / (ms3 * 1e-3),
+            "steps": args.extra_steps, "ffn_gemm1_swiglu_ms": per.get("ffn_gemm1_swiglu"),
+            "dispatch_ms_in_backward": per.get("dispatch"),
+            "note": "moe_expert_ffn_gathered: the forward writes no [N, d] copy of x; the backward dispatches it"}
+        del lay3, inp3
+        torch.cuda.empty_cache()
     if rank == 0:
         print(json.dumps(line), flush=True)
     replicas.finish(info)
