@@ -161,6 +161,8 @@ def kernel_work(cfg, name):
         "pft_scan": 8 * E,
         "pft_scatter": 8 * N + 16 * N,
         "transpose": 2 * d * E * b,
+        # dense dz rows x Wg^T reduce-added into dx: dz and Wg^T read, dx read and written (in L2/HBM)
+        "gate_dx": 2 * T * d * b + T * E * b + d * E * b,
     }
     if cfg.has_rbd:   # RBD plan kernels: ids in, pilot / replica lists out (P <= N)
         P = T * min(k, E // (cfg.rbd_epd * cfg.rbd_dpn))

@@ -67,7 +67,8 @@ enum Mode { RG = 0, KG = 1 };
 // issuer's barrier handshakes; 64 for the 256-wide expert weight-gradient tiles, where a
 // 128-deep stage leaves room for only two stages and measured slower.
 constexpr int KG_BK = 2 * BK;
-enum Epi { EPI_STORE_BF16 = 0, EPI_STORE_F32 = 1, EPI_SWIGLU_FWD = 2, EPI_SWIGLU_BWD = 3, EPI_SPLIT_BF16 = 4 };
+enum Epi { EPI_STORE_BF16 = 0, EPI_STORE_F32 = 1, EPI_SWIGLU_FWD = 2, EPI_SWIGLU_BWD = 3, EPI_SPLIT_BF16 = 4,
+           EPI_REDADD_BF16 = 5 };   // REDADD: D += acc (BF16), full slabs by TMA reduce-add
 
 struct Params {
   CUtensorMap tmA[2];
@@ -437,6 +438,37 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* tm, uint32_t src
                "r"(src), "r"(c0), "r"(c1), "r"(c2)
                : "memory");
 }
+// Element-wise add of the staged box into global memory (the reduction runs in L2; one add per element).
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* tm, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tm)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
+// Staged BF16 slab added to global rows (read, add in float32, round, write); rows >= rows_valid and
+// bytes >= bytes_valid are skipped.  Every element has one owner, so there is no race.
+__device__ __forceinline__ void copy_out_add_bf16(uint32_t stg, int lane, char* base, long long stride, int rows_valid,
+                                                  int bytes_valid) {
+  const int chunk = lane & 7;
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int row = it * 4 + (lane >> 3);
+    const uint4 u = ld_shared16(stg_addr(stg, row, chunk));
+    if (row < rows_valid && chunk * 16 < bytes_valid) {
+      uint4* g = reinterpret_cast<uint4*>(base + row * stride + chunk * 16);
+      uint4 o = *g;
+      const __nv_bfloat162* a = reinterpret_cast<const __nv_bfloat162*>(&u);
+      __nv_bfloat162* b = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 fa = __bfloat1622float2(a[i]), fb = __bfloat1622float2(b[i]);
+        b[i] = __floats2bfloat162_rn(fa.x + fb.x, fa.y + fb.y);
+      }
+      *g = o;
+    }
+  }
+}
 
 // Per-warp staging state: KG_STAGE_BUFS 4 KB slabs used in turn.
 struct Stager {
@@ -448,7 +480,7 @@ struct Stager {
 // (the staging layout is the TMA 128-byte swizzle; the store clips at the tensor bounds);
 // a slab with missing rows goes out with masked vector stores.  One bulk group is committed
 // per slab, so "at most KG_STAGE_BUFS - 1 groups pending" means the slab about to be reused is free.
-template <typename T>
+template <typename T, bool ADD = false>
 __device__ __forceinline__ void emit(Stager& st, int lane, const float* v, const CUtensorMap* tm, int c0, int c1,
                                      int c2, T* dst_row0, long long ldd, int rows_valid, int cols_valid) {
   const uint32_t buf = st.base + (st.seq % KG_STAGE_BUFS) * STAGE_BYTES_PER_WARP;
@@ -460,11 +492,18 @@ __device__ __forceinline__ void emit(Stager& st, int lane, const float* v, const
   if (tm && rows_valid == 32) {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncwarp();
-    if (lane == 0) tma_store_3d(tm, buf, c0, c1, c2);
+    if (lane == 0) {
+      if constexpr (ADD) tma_reduce_add_3d(tm, buf, c0, c1, c2);
+      else tma_store_3d(tm, buf, c0, c1, c2);
+    }
   } else {
     __syncwarp();
-    copy_out(buf, lane, reinterpret_cast<char*>(dst_row0), ldd * static_cast<long long>(sizeof(T)), rows_valid,
-             min(128, cols_valid * static_cast<int>(sizeof(T))));
+    if constexpr (ADD)
+      copy_out_add_bf16(buf, lane, reinterpret_cast<char*>(dst_row0), ldd * static_cast<long long>(sizeof(T)),
+                        rows_valid, min(128, cols_valid * static_cast<int>(sizeof(T))));
+    else
+      copy_out(buf, lane, reinterpret_cast<char*>(dst_row0), ldd * static_cast<long long>(sizeof(T)), rows_valid,
+               min(128, cols_valid * static_cast<int>(sizeof(T))));
   }
   if (lane == 0) asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -489,7 +528,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, u
   const long long grow0 = static_cast<long long>(tl.row0) + slab0;
   const bool zero = tl.nk == 0;
   const int tz = p.mode == KG ? tl.g : 0;   // third output coordinate: expert / split part
-  if constexpr (EPI == EPI_STORE_BF16 || EPI == EPI_SPLIT_BF16) {
+  if constexpr (EPI == EPI_STORE_BF16 || EPI == EPI_SPLIT_BF16 || EPI == EPI_REDADD_BF16) {
     const int nparts = EPI == EPI_SPLIT_BF16 ? 2 : 1;
     const int width = EPI == EPI_SPLIT_BF16 ? p.bn / 2 : p.bn;
     const long long goff = p.mode == KG ? tl.g * p.d_gstride : 0;
@@ -505,8 +544,8 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& tl, u
 #pragma unroll
           for (int i = 0; i < 64; ++i) v[i] = 0.f;
         }
-        emit(stg, lane, v, tmd(p, part), col, static_cast<int>(grow0), tz, D + grow0 * p.ldd + col, p.ldd, rows_valid,
-             p.Nout - col);
+        emit<__nv_bfloat16, EPI == EPI_REDADD_BF16>(stg, lane, v, tmd(p, part), col, static_cast<int>(grow0), tz,
+                                                   D + grow0 * p.ldd + col, p.ldd, rows_valid, p.Nout - col);
       }
     }
   } else if constexpr (EPI == EPI_STORE_F32) {
@@ -548,7 +587,8 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
   const uint32_t b_bytes = static_cast<uint32_t>(p.bn) * KBK * 2;
   const uint32_t stage_bytes = a_bytes + b_bytes;
   uint8_t* stage_area = smem + S * stage_bytes;                       // epilogue staging (K-grouped only)
-  uint8_t* bar_area = stage_area + (MODE == KG ? KG_EPI_WARPS * KG_STAGE_BUFS * STAGE_BYTES_PER_WARP : 0);
+  constexpr bool STAGED = MODE == KG || EPI == EPI_REDADD_BF16;   // staged epilogue (slabs + TMA stores)
+  uint8_t* bar_area = stage_area + (STAGED ? KG_EPI_WARPS * KG_STAGE_BUFS * STAGE_BYTES_PER_WARP : 0);
   uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
   uint64_t* empty = full + MAX_STAGES;
   uint64_t* acc_full = empty + MAX_STAGES;
@@ -753,7 +793,7 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
       if (!__all_sync(0xffffffffu, wait_bar(smem_u32(&acc_full[buf]), aph, abort_flag, p.err))) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * p.bn;
-      if constexpr (MODE == KG) epilogue_tile<EPI>(p, tl, tacc, q, lane, stg, half, KG_EPI_WARPS / 4);
+      if constexpr (STAGED) epilogue_tile<EPI>(p, tl, tacc, q, lane, stg, half, KG_EPI_WARPS / 4);
       else epilogue_tile_direct<EPI>(p, tl, tacc, q * 32 + lane);
       tc_fence_before();
       mbar_arrive(smem_u32(&acc_empty[buf]));
@@ -1612,7 +1652,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GATHER ? THREADS_GAT
 template <int EPI, int MODE, int KBK = BK>
 static int launch(Params& p, long long tile_upper_bound, const char* name, cudaStream_t stream) {
   p.mode = MODE;
-  const bool staged = p.mode == KG;
+  const bool staged = p.mode == KG || EPI == EPI_REDADD_BF16;
   p.stages = pick_stages(p.bn, staged, KBK);
   if (p.stages < 2) return fail(PFMOE_ERR_UNSUPPORTED, std::string(name) + ": shared-memory plan needs two stages");
   const size_t smem = smem_bytes(p.bn, p.stages, staged, KBK);
@@ -1945,6 +1985,30 @@ int tc_gate_logits(const void* x, const void* wg, const float* bias, int T, int 
   PFMOE_TRY((launch<EPI_STORE_F32, RG>(p, ub, "gate_logits", s)));
   *nparts = ks;   // ks > 1: the top-k kernel sums the parts (and adds the bias)
   return PFMOE_OK;
+}
+
+// Gate term of the token gradient: dx[t] += sum_e dz[t, e] Wg^T[e] ([B] 训练流程, the gate's backward),
+// as a dense tensor-core GEMM of the BF16 dz rows (A [T, E], K-major) against Wg^T (B [E, d], rows of
+// d).  The epilogue adds the product into the BF16 dx the token-gradient kernel wrote, with TMA
+// reduce-add stores: every element is added once, in L2.
+int tc_gate_dx(const void* dz_bf16, const void* wgT, int T, int d, int E, void* dx, int32_t* err, cudaStream_t s) {
+  Params p = base_params(err);
+  p.mode = RG;
+  p.b_major = 1;              // Wg^T [E, d]: K rows, d contiguous
+  p.bn = round_bn(d);
+  p.Nout = d;
+  p.k0_blocks = (E + BK - 1) / BK;
+  p.G = 1;
+  p.dense_len = T;
+  p.ldd = d;
+  p.ksplit = 1;
+  p.D0 = dx;
+  PFMOE_TRY(make_tmap(&p.tmA[0], dz_bf16, E, T, 1, BK, BM, "dz"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], wgT, d, E, 1, 64, 64, "wg^T"));
+  PFMOE_TRY(make_out_map(&p.tmD[0], dx, d, T, 1, "dx"));
+  p.tma_store = 1;
+  const long long ub = static_cast<long long>((T + BM - 1) / BM) * ((d + p.bn - 1) / p.bn);
+  return launch<EPI_REDADD_BF16, RG>(p, ub, "gate_dx", s);
 }
 
 int tc_gate_wgrad(const void* x, const void* dz_bf16, int T, int d, int E, float* dwg, void* ws, size_t ws_bytes,

@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(WARPS * 32) combine_kernel(const T* __restrict
 }
 
 // dz_{t, ids[t,j]} = w_j (g_j - sum_l w_l g_l) (zero elsewhere);
-// dx[t] = sum_j dX_pft[pos[t, j]] + sum_j dz_j * Wg^T[ids[t, j]].
+// dx[t] = sum_j dX_pft[pos[t, j]] + sum_j dz_j * Wg^T[ids[t, j]] (the second sum only when wgT is given).
 // The dense dlogits row (and its BF16 copy for the dWg GEMM) is written by the token's chunk-0 item.
 template <typename T, int U>
 __global__ void __launch_bounds__(WARPS * 32) token_grad_kernel(const T* __restrict__ dxp, const int32_t* __restrict__ pos,
@@ -455,18 +455,22 @@ __global__ void __launch_bounds__(WARPS * 32) token_grad_kernel(const T* __restr
         }
       }
     }
+    // The gate term; with wgT null the caller adds it afterwards (BF16: a tensor-core GEMM of the
+    // dense dz rows against Wg^T that reduce-adds into dx).
+    if (wgT != nullptr) {
 #pragma unroll 8
-    for (int j = 0; j < k; ++j) {
-      const long long idj = __shfl_sync(0xffffffffu, my_id, j);
-      const float dzj = __shfl_sync(0xffffffffu, my_dz, j);
+      for (int j = 0; j < k; ++j) {
+        const long long idj = __shfl_sync(0xffffffffu, my_id, j);
+        const float dzj = __shfl_sync(0xffffffffu, my_dz, j);
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int c0 = cb + u * chunk_cols<T>();
-        if (c0 < d) {
-          float v[VN];
-          load16(wgT + idj * d + c0, v);
+        for (int u = 0; u < U; ++u) {
+          const int c0 = cb + u * chunk_cols<T>();
+          if (c0 < d) {
+            float v[VN];
+            load16(wgT + idj * d + c0, v);
 #pragma unroll
-          for (int i = 0; i < VN; ++i) acc[u][i] = fmaf(dzj, v[i], acc[u][i]);
+            for (int i = 0; i < VN; ++i) acc[u][i] = fmaf(dzj, v[i], acc[u][i]);
+          }
         }
       }
     }
