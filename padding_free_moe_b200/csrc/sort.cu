@@ -566,6 +566,18 @@ __global__ void rbd_final_kernel(const int32_t* ids, int T, int k, int E, int ep
 constexpr int RF_NODES = 8;
 constexpr int RF_TILE = 256;
 
+// Division of an expert id (< 2^16) by a divisor d < 2^16 as a multiply-high: with m = ceil(2^32 / d),
+// floor(v m / 2^32) = floor(v / d) whenever v, d < 2^16 (the error v (m - 2^32 / d) / 2^32 stays below
+// 1 / d).  Replaces the per-id integer divisions of the per-token kernels.
+struct FastDiv {
+  unsigned m;
+  int d;
+  __device__ __forceinline__ explicit FastDiv(int d_) : m(d_ > 1 ? 0xffffffffu / static_cast<unsigned>(d_) + 1u : 0u), d(d_) {}
+  __device__ __forceinline__ int operator()(int v) const {
+    return d > 1 ? static_cast<int>(__umulhi(static_cast<unsigned>(v), m)) : v;
+  }
+};
+
 // The tile's ids ([RF_TILE][k] consecutive ints) are staged in shared memory with coalesced loads;
 // each thread then reads its token's k ids from there.
 __device__ __forceinline__ void rf_stage_ids(const int32_t* __restrict__ ids, int T, int k, int32_t* sids) {
@@ -577,7 +589,7 @@ __device__ __forceinline__ void rf_stage_ids(const int32_t* __restrict__ ids, in
 }
 
 template <int KM>
-__device__ __forceinline__ void rf_load(const int32_t* __restrict__ sids, bool valid, int k, int E, int epn,
+__device__ __forceinline__ void rf_load(const int32_t* __restrict__ sids, bool valid, int k, int E, const FastDiv& node_of,
                                         int (&e)[KM], int (&nd)[KM], int32_t* err) {
 #pragma unroll
   for (int j = 0; j < KM; ++j) {
@@ -590,7 +602,7 @@ __device__ __forceinline__ void rf_load(const int32_t* __restrict__ sids, bool v
       }
     }
     e[j] = v;
-    nd[j] = (valid && j < k) ? v / epn : -1;
+    nd[j] = (valid && j < k) ? node_of(v) : -1;
   }
 }
 
@@ -618,14 +630,18 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_count_kernel(const int32_t* 
   const bool valid = t < T;
   int e[KM], nd[KM], c[RF_NODES];
   rf_stage_ids(ids, T, k, sids);
-  rf_load<KM>(sids, valid, k, E, epn, e, nd, err);
+  const FastDiv node_of(epn), dev_of(epd);
+  rf_load<KM>(sids, valid, k, E, node_of, e, nd, err);
   rf_counts<KM>(nd, c);
+  int dv[KM];
+#pragma unroll
+  for (int j = 0; j < KM; ++j) dv[j] = dev_of(e[j]);
   int dc = 0;   // distinct devices of the token
 #pragma unroll
   for (int j = 0; j < KM; ++j) {
     bool first = j < k && valid;
 #pragma unroll
-    for (int i = 0; i < j; ++i) first = first && (e[i] / epd != e[j] / epd);
+    for (int i = 0; i < j; ++i) first = first && (dv[i] != dv[j]);
     dc += first;
   }
 #pragma unroll
@@ -647,12 +663,16 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_count_kernel(const int32_t* 
   }
 }
 
-// One CTA of 512 threads: thread i takes a run of consecutive tiles (all loaded up front), the
-// runs are scanned per node across the block, and each thread writes its tiles' exclusive token
-// bases (in place) and replica bases (tile_rep_base); then the node offsets, P and the distinct
-// (token, device) total.  Tiles beyond 512 runs' worth are handled in further passes.
+// One CTA of 512 threads: thread i takes a run of RF_RUN consecutive tiles, the runs are scanned per
+// node across the block, and each thread writes its tiles' exclusive token bases (in place) and
+// replica bases (tile_rep_base); then the node offsets, P and the distinct (token, device) total.
+// The [tile][node] rows go through shared memory: read and written with coalesced accesses, each
+// thread's run of RF_RUN * RF_NODES ints padded by one int so that the per-thread reads are free of
+// bank conflicts.  Tiles beyond one block's worth are handled in further passes.
 constexpr int RF_SCAN_THREADS = 512;
-constexpr int RF_RUN = 4;   // tiles per thread per pass
+constexpr int RF_RUN = 4;                              // tiles per thread per pass
+constexpr int RF_ROW = RF_RUN * RF_NODES + 1;          // padded ints per thread run
+constexpr int RF_SCAN_SMEM = 2 * RF_SCAN_THREADS * RF_ROW * 4;
 
 __global__ void __launch_bounds__(RF_SCAN_THREADS) rbd_fast_scan_kernel(int ntiles, int n_nodes,
                                                                         int32_t* __restrict__ tile_cnt,
@@ -661,6 +681,9 @@ __global__ void __launch_bounds__(RF_SCAN_THREADS) rbd_fast_scan_kernel(int ntil
                                                                         int32_t* pilots_per_node, int32_t* node_offsets,
                                                                         int32_t* node_rep_off, int32_t* counts,
                                                                         int32_t* replica_offsets) {
+  extern __shared__ int32_t scan_sm[];
+  int32_t* s_tok = scan_sm;                            // [thread][RF_ROW]: counts in, token bases out
+  int32_t* s_rep = scan_sm + RF_SCAN_THREADS * RF_ROW; // replica bases out
   __shared__ int wt[RF_SCAN_THREADS / 32][RF_NODES], wr[RF_SCAN_THREADS / 32][RF_NODES];
   __shared__ int carry_t[RF_NODES], carry_r[RF_NODES];
   __shared__ int dsum[RF_SCAN_THREADS / 32];
@@ -669,6 +692,12 @@ __global__ void __launch_bounds__(RF_SCAN_THREADS) rbd_fast_scan_kernel(int ntil
   int ds = 0;
   __syncthreads();
   for (int base = 0; base < ntiles; base += RF_SCAN_THREADS * RF_RUN) {
+    const int nt = min(RF_SCAN_THREADS * RF_RUN, ntiles - base);   // tiles in this pass
+    const long long g0 = static_cast<long long>(base) * RF_NODES;
+    for (int i = threadIdx.x; i < nt * RF_NODES; i += RF_SCAN_THREADS)
+      s_tok[(i / (RF_RUN * RF_NODES)) * RF_ROW + i % (RF_RUN * RF_NODES)] = tile_cnt[g0 + i];
+    for (int i = threadIdx.x; i < nt; i += RF_SCAN_THREADS) ds += tile_dev[base + i];
+    __syncthreads();
     const int t0 = base + threadIdx.x * RF_RUN;
     int v[RF_RUN][RF_NODES];
 #pragma unroll
@@ -676,8 +705,7 @@ __global__ void __launch_bounds__(RF_SCAN_THREADS) rbd_fast_scan_kernel(int ntil
       const bool ok = t0 + r < ntiles;
 #pragma unroll
       for (int n = 0; n < RF_NODES; ++n)
-        v[r][n] = ok && n < n_nodes ? tile_cnt[static_cast<long long>(t0 + r) * RF_NODES + n] : 0;
-      if (ok) ds += tile_dev[t0 + r];
+        v[r][n] = ok && n < n_nodes ? s_tok[threadIdx.x * RF_ROW + r * RF_NODES + n] : 0;
     }
     int run_t[RF_NODES], run_r[RF_NODES], ex_t[RF_NODES], ex_r[RF_NODES];
 #pragma unroll
@@ -717,15 +745,20 @@ __global__ void __launch_bounds__(RF_SCAN_THREADS) rbd_fast_scan_kernel(int ntil
       int at = wt[warp][n] + ex_t[n], ar = wr[warp][n] + ex_r[n];
 #pragma unroll
       for (int r = 0; r < RF_RUN; ++r) {
-        if (t0 + r < ntiles && n < n_nodes) {
-          tile_cnt[static_cast<long long>(t0 + r) * RF_NODES + n] = at;
-          tile_rep_base[static_cast<long long>(t0 + r) * RF_NODES + n] = ar;
-        }
+        s_tok[threadIdx.x * RF_ROW + r * RF_NODES + n] = at;
+        s_rep[threadIdx.x * RF_ROW + r * RF_NODES + n] = ar;
         at += v[r][n] & 0xffff;
         ar += v[r][n] >> 16;
       }
     }
-    __syncthreads();   // wt / wr are rewritten by the next pass
+    __syncthreads();
+    // columns n >= n_nodes are written too (zero counts, so the bases repeat): the rows stay whole
+    for (int i = threadIdx.x; i < nt * RF_NODES; i += RF_SCAN_THREADS) {
+      const int si = (i / (RF_RUN * RF_NODES)) * RF_ROW + i % (RF_RUN * RF_NODES);
+      tile_cnt[g0 + i] = s_tok[si];
+      tile_rep_base[g0 + i] = s_rep[si];
+    }
+    __syncthreads();   // the buffers and wt / wr are rewritten by the next pass
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
@@ -766,7 +799,8 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_emit_kernel(
   const bool valid = t < T;
   int e[KM], nd[KM], c[RF_NODES], ex[RF_NODES];
   rf_stage_ids(ids, T, k, sbuf);
-  rf_load<KM>(sbuf, valid, k, E, epn, e, nd, nullptr);   // rbd_fast_count flagged bad ids
+  const FastDiv node_of(epn), dev_of(epd);
+  rf_load<KM>(sbuf, valid, k, E, node_of, e, nd, nullptr);   // rbd_fast_count flagged bad ids
   (void)err;
   rf_counts<KM>(nd, c);
   // in-warp exclusive prefix of the packed counts, per node
@@ -807,7 +841,7 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_emit_kernel(
         if (nd[j] == n && e[j] < emin) emin = e[j];
       pilot_token[idx[n]] = static_cast<int32_t>(t);
       pilot_node[idx[n]] = n;
-      pilot_device[idx[n]] = emin / epd;
+      pilot_device[idx[n]] = dev_of(emin);
       replica_offsets[idx[n]] = node_rep_off[n] + tile_rep_base[tb + n] + (ex[n] >> 16);
     }
   }
@@ -927,9 +961,11 @@ static int rbd_fast_launch(const int32_t* ids, int T, int k, int E, int epd, int
     PFMOE_LAUNCH("rbd_count", s,
                  (rbd_fast_count_kernel<KM><<<ntiles, RF_TILE, 0, s>>>(ids, T, k, E, epd, epn, tile_cnt, tile_dev,
                                                                       err)));
+  PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&rbd_fast_scan_kernel), RF_SCAN_SMEM, "rbd_scan_nodes"));
   PFMOE_LAUNCH("rbd_scan_nodes", s,
-               (rbd_fast_scan_kernel<<<1, RF_SCAN_THREADS, 0, s>>>(ntiles, n_nodes, tile_cnt, tile_rep, tile_dev, ppn,
-                                                                   noff, node_rep_off, counts, roff)));
+               (rbd_fast_scan_kernel<<<1, RF_SCAN_THREADS, RF_SCAN_SMEM, s>>>(ntiles, n_nodes, tile_cnt, tile_rep,
+                                                                              tile_dev, ppn, noff, node_rep_off,
+                                                                              counts, roff)));
   if (ntiles > 0)
     PFMOE_LAUNCH("rbd_emit", s,
                (rbd_fast_emit_kernel<KM><<<ntiles, RF_TILE, 0, s>>>(ids, T, k, E, epd, epn, n_nodes, tile_cnt, tile_rep,
