@@ -816,18 +816,35 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_emit_kernel(
     if (lane == 31) wsum[warp][n] = a;
   }
   __syncthreads();   // wsum complete; every thread has read its ids from sbuf
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int n = 0; n < RF_NODES; ++n) {
-      node_loc[n] = run;
-      for (int w = 0; w < RF_TILE / 32; ++w) run += wsum[w][n] >> 16;
+  if (warp == 0) {
+    // lane n < RF_NODES: column n of wsum -> exclusive prefix over the warps (the packed fields add
+    // independently); the node's replica total -> node_loc by a scan over lanes 0 .. RF_NODES - 1
+    int tot = 0;
+    if (lane < RF_NODES) {
+      int run = 0;
+      for (int w = 0; w < RF_TILE / 32; ++w) {
+        const int x = wsum[w][lane];
+        wsum[w][lane] = run;
+        run += x;
+      }
+      tot = run >> 16;
     }
-    node_loc[RF_NODES] = run;
-  }
+    int x = tot;
 #pragma unroll
-  for (int n = 0; n < RF_NODES; ++n)
-    for (int w = 0; w < warp; ++w) ex[n] += wsum[w][n];
-  __syncthreads();   // node_loc ready
+    for (int o = 1; o < RF_NODES; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane < RF_NODES) node_loc[lane] = x - tot;
+    if (lane == RF_NODES - 1) node_loc[RF_NODES] = x;
+  }
+  __syncthreads();   // node_loc and the warp prefixes ready
+  int rep_base[RF_NODES];   // this token's first slot in the tile's replica staging, per node
+#pragma unroll
+  for (int n = 0; n < RF_NODES; ++n) {
+    ex[n] += wsum[warp][n];
+    rep_base[n] = node_loc[n] + (ex[n] >> 16);
+  }
   const long long tb = static_cast<long long>(blockIdx.x) * RF_NODES;
   int idx[RF_NODES];
 #pragma unroll
@@ -857,7 +874,7 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_emit_kernel(
         int loc = 0;
 #pragma unroll
         for (int n = 0; n < RF_NODES; ++n)
-          if (nd[j] == n) loc = node_loc[n] + (ex[n] >> 16);
+          if (nd[j] == n) loc = rep_base[n];
         sbuf[loc + within] = e[j];
       }
     }
