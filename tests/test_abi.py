@@ -73,6 +73,18 @@ def test_other_argument_errors(lib):
     assert lib.moe_combine(FAKE, None, FAKE, 4, 2, 64, L.PFMOE_BF16, FAKE, None, None) == L.PFMOE_ERR_ARG
     assert lib.moe_expert_ffn(FAKE, FAKE, FAKE, 8, 4, 64, 60, L.PFMOE_BF16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
                               FAKE, None, None) == L.PFMOE_ERR_UNSUPPORTED
+    # the gathered expert FFN: BF16 only, 16-byte rows, every pointer given
+    def gathered(**kw):
+        a = dict(x=FAKE, ids=FAKE, N=8, E=4, d=64, h=64, dtype=L.PFMOE_BF16)
+        a.update(kw)
+        return lib.moe_expert_ffn_gathered(a["x"], a["ids"], FAKE, FAKE, a["N"], a["E"], a["d"], a["h"], a["dtype"],
+                                           FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None)
+    assert gathered(dtype=L.PFMOE_F32) == L.PFMOE_ERR_UNSUPPORTED
+    assert b"BF16" in lib.moe_last_error()
+    assert gathered(h=60) == L.PFMOE_ERR_UNSUPPORTED
+    assert gathered(ids=None) == L.PFMOE_ERR_ARG
+    assert gathered(x=FAKE + 4) == L.PFMOE_ERR_ARG
+    assert gathered(N=-1) == L.PFMOE_ERR_ARG
     # RBD map must tile the experts
     assert lib.rbd_plan(FAKE, 4, 2, 12, 4, 2, *([FAKE] * 10), 1 << 20, None, None) == L.PFMOE_ERR_ARG
     assert lib.rbd_plan_workspace_size(4, 2, 12, 4, 2) == 0
@@ -91,6 +103,8 @@ def test_empty_inputs_are_noops(lib):
     assert lib.moe_combine(None, None, None, 0, 2, 64, L.PFMOE_BF16, None, None, None) == L.PFMOE_OK
     assert lib.moe_expert_ffn(None, None, None, 0, 4, 64, 64, L.PFMOE_BF16, None, None, None, None, None, None,
                               None, None, None) == L.PFMOE_OK
+    assert lib.moe_expert_ffn_gathered(None, None, None, None, 0, 4, 64, 64, L.PFMOE_BF16, None, None, None, None,
+                                       None, None, None, None, None) == L.PFMOE_OK
 
 
 def test_workspace_sizes(lib):
