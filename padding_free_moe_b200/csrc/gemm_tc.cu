@@ -1713,16 +1713,19 @@ static Params base_params(int32_t* err) {
   return p;
 }
 
-// Split-K for the dense gate GEMMs, which have too few output tiles to fill the GPU:
-// enough parts for about one wave on a 148-SM B200, at least 4 K blocks per part,
-// every part non-empty.  Depends only on the shape, so workspace sizes are host-computable.
+// Split-K for the dense gate GEMMs, which have too few output tiles to fill the GPU: the part
+// count (at most 8, at least 4 K blocks per part, every part non-empty) with the fewest waves of
+// work on a 148-SM B200.  Depends only on the shape, so workspace sizes are host-computable.
 static int choose_ksplit(long long tiles, int nk) {
-  long long ks = (148 + tiles - 1) / tiles;
-  if (ks > 8) ks = 8;
-  const long long cap = nk / 4 > 1 ? nk / 4 : 1;
-  if (ks > cap) ks = cap;
-  if (ks < 1) ks = 1;
-  const long long kbs = (nk + ks - 1) / ks;
+  // The part count that minimises waves x K blocks per part (ties: fewer parts, less to reduce).
+  const long long cap = nk / 4 > 1 ? (nk / 4 < 8 ? nk / 4 : 8) : 1;
+  long long best = 1, best_cost = -1;
+  for (long long ks = 1; ks <= cap; ++ks) {
+    const long long kbs = (nk + ks - 1) / ks;
+    const long long cost = ((tiles * ks + 147) / 148) * kbs;
+    if (best_cost < 0 || cost < best_cost) { best = ks; best_cost = cost; }
+  }
+  const long long kbs = (nk + best - 1) / best;
   return static_cast<int>((nk + kbs - 1) / kbs);
 }
 
