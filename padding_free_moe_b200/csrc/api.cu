@@ -418,11 +418,10 @@ int moe_backward(const void* dy, const void* x, const void* wg, const float* top
     PFMOE_TRY(tc_ffn_dgrad_x(w.dh1, w.dh3, expert_offsets, tile_offsets, N, E, d, h, w1, w3, w.dx_pft, err, s));
     PFMOE_TRY(tc_ffn_wgrad13(x_pft, w.dh1, w.dh3, expert_offsets, N, E, d, h, dw1, dw3, err, s));
     PFMOE_TRY(tc_ffn_wgrad2(a, w.dO, expert_offsets, N, E, d, h, dw2, err, s));
-    PFMOE_TRY(launch_transpose(wg, d, E, dtype, w.wgT, s));
     // dx = sum of the token's dX_pft rows (and dz, dlogits); then the gate term on the tensor cores
     PFMOE_TRY(launch_token_grad(w.dx_pft, pos, w.g, topk_w, topk_ids, nullptr, T, k, d, E, dtype, dx, dlogits,
                                 w.dz_bf16, err, s));
-    PFMOE_TRY(tc_gate_dx(w.dz_bf16, w.wgT, T, d, E, dx, err, s));
+    PFMOE_TRY(tc_gate_dx(w.dz_bf16, wg, T, d, E, dx, err, s));
     return tc_gate_wgrad(x, w.dz_bf16, T, d, E, dwg, w.dwg_parts, w.dwg_parts_bytes, err, s);
   }
   // FP32 path on the CUDA cores.

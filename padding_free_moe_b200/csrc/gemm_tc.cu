@@ -655,9 +655,11 @@ __global__ void __launch_bounds__(MODE == KG ? THREADS_KG : THREADS, 1) grouped_
           pending |= 1u << s;
           pend_parity = (pend_parity & ~(1u << s)) | (ph << s);
           if constexpr (MODE == RG) {
-            // dense gate GEMM: A = X rows (K-major), B = Wg [K, N] (MN-major 64-column boxes)
+            // dense gate GEMMs: A rows K-major; B MN-major ([K, N], 64-column boxes) or K-major
+            // ([N, K], one box of bn rows)
             const int kk = (tl.kb0 + kb) * BK;
             if (lane == 0) tma_load_3d(sa, &p.tmA[0], fb, kk, tl.row0, 0);
+            else if (!p.b_major) tma_load_3d(sb, &p.tmB[0], fb, kk, tl.n0, 0);
             else for (int j = 0; j < nb; ++j) tma_load_3d(sb + j * BOX_BYTES, &p.tmB[0], fb, tl.n0 + 64 * j, kk, 0);
           } else {
             const int krow = tl.krow0 + kb * KBK;
@@ -1990,14 +1992,14 @@ int tc_gate_logits(const void* x, const void* wg, const float* bias, int T, int 
   return PFMOE_OK;
 }
 
-// Gate term of the token gradient: dx[t] += sum_e dz[t, e] Wg^T[e] ([B] 训练流程, the gate's backward),
-// as a dense tensor-core GEMM of the BF16 dz rows (A [T, E], K-major) against Wg^T (B [E, d], rows of
-// d).  The epilogue adds the product into the BF16 dx the token-gradient kernel wrote, with TMA
-// reduce-add stores: every element is added once, in L2.
-int tc_gate_dx(const void* dz_bf16, const void* wgT, int T, int d, int E, void* dx, int32_t* err, cudaStream_t s) {
+// Gate term of the token gradient: dx[t] += sum_e dz[t, e] Wg[:, e] ([B] 训练流程, the gate's backward),
+// as a dense tensor-core GEMM of the BF16 dz rows (A [T, E], K-major) against Wg (B [d, E]: N rows of
+// K, read K-major, so no transpose).  The epilogue adds the product into the BF16 dx the
+// token-gradient kernel wrote, with TMA reduce-add stores: every element is added once, in L2.
+int tc_gate_dx(const void* dz_bf16, const void* wg, int T, int d, int E, void* dx, int32_t* err, cudaStream_t s) {
   Params p = base_params(err);
   p.mode = RG;
-  p.b_major = 1;              // Wg^T [E, d]: K rows, d contiguous
+  p.b_major = 0;              // Wg [d, E]: rows of K
   p.bn = round_bn(d);
   p.Nout = d;
   p.k0_blocks = (E + BK - 1) / BK;
@@ -2007,7 +2009,7 @@ int tc_gate_dx(const void* dz_bf16, const void* wgT, int T, int d, int E, void* 
   p.ksplit = 1;
   p.D0 = dx;
   PFMOE_TRY(make_tmap(&p.tmA[0], dz_bf16, E, T, 1, BK, BM, "dz"));
-  PFMOE_TRY(make_tmap(&p.tmB[0], wgT, d, E, 1, 64, 64, "wg^T"));
+  PFMOE_TRY(make_tmap(&p.tmB[0], wg, E, d, 1, BK, p.bn, "wg"));
   PFMOE_TRY(make_out_map(&p.tmD[0], dx, d, T, 1, "dx"));
   p.tma_store = 1;
   const long long ub = static_cast<long long>((T + BM - 1) / BM) * ((d + p.bn - 1) / p.bn);

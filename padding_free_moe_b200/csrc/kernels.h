@@ -13,7 +13,7 @@ int tc_ffn_gemm1(const void* x_pft, const int* seg, const int* tiles, int N, int
 int tc_ffn_gemm1_gather(const void* x, const int* token_ids, const int* seg, const int* tiles, int N, int E, int d,
                         int h, const void* w1, const void* w3, void* h1, void* h3, void* a, int32_t* err,
                         cudaStream_t s);
-int tc_gate_dx(const void* dz_bf16, const void* wgT, int T, int d, int E, void* dx, int32_t* err, cudaStream_t s);
+int tc_gate_dx(const void* dz_bf16, const void* wg, int T, int d, int E, void* dx, int32_t* err, cudaStream_t s);
 int tc_ffn_gemm2(const void* a, const int* seg, const int* tiles, int N, int E, int d, int h, const void* w2,
                  void* out, int32_t* err, cudaStream_t s);
 int tc_ffn_dgrad_act(const void* dO, const int* seg, const int* tiles, int N, int E, int d, int h, const void* w2,
