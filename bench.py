@@ -62,6 +62,8 @@ def parse():
     ap.add_argument("--extra-workloads", default=EXTRA_WORKLOADS,
                     help="comma-separated workloads timed after the headline one ('' = none)")
     ap.add_argument("--extra-steps", type=int, default=10)
+    ap.add_argument("--sort-stress-only", action="store_true",
+                    help="time only the PFT build and RBD plan on the stress shape (T = 2^20, E = 256, k = 8)")
     ap.add_argument("--no-gathered", action="store_true",
                     help="skip the timing of the step with the gather fused into the first expert GEMM")
     return ap.parse_args()
@@ -708,8 +710,21 @@ def relaunch_under_torchrun(n: int) -> int:
     return subprocess.call(cmd, cwd=ROOT)
 
 
+def run_sort_stress_only(args):
+    """The PFT build and RBD plan on the stress shape alone (one GPU): one JSON object."""
+    import torch
+    from padding_free_moe_b200 import _lib as L
+    dev = torch.device("cuda", 0)
+    peaks, _ = load_peaks()
+    out = stress_sort(L, torch, dev, torch.cuda.current_stream(), float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])))
+    print(json.dumps({"sort_stress": out}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    if args.sort_stress_only:
+        return run_sort_stress_only(args)
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         return relaunch_under_torchrun(args.gpus)
     if args.impl == "reference":
