@@ -123,23 +123,53 @@ __global__ void __launch_bounds__(SCAN_THREADS) chunk_scan_kernel(const int32_t*
   }
 }
 
-// Many chunks: one CTA per key scans that key's column of chunk counts (exclusive, relative
-// bases) and writes the key's total; key_scan_kernel then forms the key offsets.
-__global__ void __launch_bounds__(SCAN_THREADS) col_scan_kernel(const int32_t* __restrict__ counts, int C, int K,
-                                                                int32_t* __restrict__ base, int32_t* totals) {
-  __shared__ int tmp[32];
-  const int key = blockIdx.x;
-  int carry = 0;
-  for (int c0 = 0; c0 < C; c0 += SCAN_THREADS) {
-    const int c = c0 + threadIdx.x;
-    const long long idx = static_cast<long long>(c) * K + key;
-    const int v = c < C ? counts[idx] : 0;
-    int blk;
-    const int ex = block_excl_scan(v, tmp, &blk);
-    if (c < C) base[idx] = carry + ex;
-    carry += blk;
+// Many chunks: the [C][K] chunk counts scanned down their columns, for strips of STRIP_KEYS keys (one
+// 32-byte sector of a row) per CTA; its 32 warps take consecutive row segments, a warp instruction
+// covering 4 rows of the strip.  Pass 1 sums each warp's segment per key, the segment sums are scanned
+// per key across the warps, and pass 2 writes each element's exclusive prefix (relative base) in the
+// same order.  Every access is a whole sector (a CTA per key used one int per sector).
+constexpr int STRIP_KEYS = 8;
+
+__global__ void __launch_bounds__(SCAN_THREADS) strip_scan_kernel(const int32_t* __restrict__ counts, int C, int K,
+                                                                  int32_t* __restrict__ base, int32_t* totals) {
+  __shared__ int wsum[SCAN_THREADS / 32][STRIP_KEYS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kk = lane % STRIP_KEYS, rsub = lane / STRIP_KEYS;   // key of the strip, row of a 4-row step
+  const int key = blockIdx.x * STRIP_KEYS + kk;
+  const bool kok = key < K;
+  const int R = (C + SCAN_THREADS / 32 - 1) / (SCAN_THREADS / 32);   // rows per warp
+  const int r0 = min(C, warp * R), r1 = min(C, r0 + R);
+  int sum = 0;
+  for (int c = r0 + rsub; c < r1; c += 4)
+    if (kok) sum += counts[static_cast<long long>(c) * K + key];
+  sum += __shfl_xor_sync(0xffffffffu, sum, 8);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 16);
+  if (rsub == 0) wsum[warp][kk] = sum;
+  __syncthreads();
+  if (warp == 0 && lane < STRIP_KEYS) {
+    int run = 0;
+    for (int w = 0; w < SCAN_THREADS / 32; ++w) {
+      const int x = wsum[w][lane];
+      wsum[w][lane] = run;
+      run += x;
+    }
+    if (blockIdx.x * STRIP_KEYS + lane < K) totals[blockIdx.x * STRIP_KEYS + lane] = run;
   }
-  if (threadIdx.x == 0) totals[key] = carry;
+  __syncthreads();
+  int carry = wsum[warp][kk];
+  for (int c0 = r0; c0 < r1; c0 += 4) {
+    const int c = c0 + rsub;
+    const bool ok = c < r1 && kok;
+    const long long idx = static_cast<long long>(c) * K + key;
+    const int v = ok ? counts[idx] : 0;
+    int x = v;   // inclusive prefix over the step's rows of this key (lanes kk, kk + 8, kk + 16, kk + 24)
+    int y = __shfl_up_sync(0xffffffffu, x, 8);
+    if (rsub >= 1) x += y;
+    y = __shfl_up_sync(0xffffffffu, x, 16);
+    if (rsub >= 2) x += y;
+    if (ok) base[idx] = carry + x - v;
+    carry += __shfl_sync(0xffffffffu, x, 3 * STRIP_KEYS + kk);
+  }
 }
 
 // Key totals -> offsets [K+1], optional tiles [K+1] (prefix of ceil(total/tile_rows)), optional copy of totals.
@@ -923,7 +953,7 @@ int rows_grid(long long rows, int warps_per_blk = 8) {
 }
 
 // Chunk counts -> relative bases + key totals/offsets/tiles: one CTA while the chunks are few, else a
-// CTA per key (col_scan) and a key scan.  key_tot receives the totals on the many-chunk path.
+// CTA per strip of keys (strip_scan) and a key scan.  key_tot receives the totals on the many-chunk path.
 constexpr int SMALL_CHUNKS = 64;
 
 int sort_scan(const int32_t* counts, int C, int K, int32_t* totals, int32_t* offsets, int32_t* base, int32_t* tiles,
@@ -933,7 +963,8 @@ int sort_scan(const int32_t* counts, int C, int K, int32_t* totals, int32_t* off
                  chunk_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(counts, C, K, totals, offsets, base, tiles, tile_rows));
     return PFMOE_OK;
   }
-  PFMOE_LAUNCH(name, s, col_scan_kernel<<<K, SCAN_THREADS, 0, s>>>(counts, C, K, base, key_tot));
+  PFMOE_LAUNCH(name, s, strip_scan_kernel<<<(K + STRIP_KEYS - 1) / STRIP_KEYS, SCAN_THREADS, 0, s>>>(counts, C, K, base,
+                                                                                            key_tot));
   PFMOE_LAUNCH(name, s, key_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(key_tot, K, totals, offsets, tiles, tile_rows));
   return PFMOE_OK;
 }
