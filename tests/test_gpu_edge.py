@@ -202,3 +202,25 @@ def test_rbd_many_nodes_general_path():
     assert np.array_equal(i64(o["roff"][:P + 1]), r["replica_offsets"])
     assert np.array_equal(i64(o["rexp"]), r["replica_expert"])
     assert np.array_equal(i64(o["ap"]), r["assign_pilot"])
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("fused", [False, True])
+def test_largest_routing_shape_matches_oracle(fused):
+    # The routing limits: E = 1024 experts, k = 32 (RBD map of 8 nodes: the per-token plan at its
+    # widest lane group), the whole layer forward and backward against the oracle.
+    from tests.parity import TOL, check_index_parity, f64, rel_err
+    cfg = get_config("small_bf16").with_(name="largest_routing", T=160, d=64, E=1024, h=64, k=32, rbd_epd=32,
+                                         rbd_dpn=4)
+    inp = make_inputs(cfg, seed=21, device="cuda")
+    layer = make_layer(cfg)
+    layer.fused_gather = fused
+    assert run_step(layer, inp) == 0
+    check_index_parity(layer, cfg, O)
+    x, wg, bias, w1, w3, w2, dy = map(f64, (inp.x, inp.wg, inp.bias, inp.w1, inp.w3, inp.w2, inp.dy))
+    fwd = O.layer_forward(x, wg, bias, w1, w3, w2, cfg.k, logits=layer.logits.cpu().numpy())
+    assert rel_err(f64(layer.y), fwd["y"]) <= TOL[cfg.dtype]
+    bwd = O.layer_backward(fwd, dy, x, wg, w1, w3, w2)
+    for nm, t in (("dx", layer.dx), ("dWg", layer.dwg), ("dW1", layer.dw1), ("dW3", layer.dw3),
+                  ("dW2", layer.dw2), ("dlogits", layer.dlogits)):
+        assert rel_err(f64(t), bwd[nm]) <= TOL[cfg.dtype], nm
