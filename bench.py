@@ -21,8 +21,12 @@ host cores, on bounded token samples of the same workload.
 The headline workload is the DeepSeek-V3-like layer (T=8192, d=7168, E=256,
 h=2048, k=8), the largest single-GPU configuration; the DeepSeek-MoE-16B-like,
 skewed DeepSeek-V3-like and fine-grained layers are timed after it and reported
-under ``workloads``.  ``--gpus N`` without a torchrun environment relaunches
-this script under torchrun with N ranks.
+under ``workloads``; the headline layer's step with the dispatch gather fused into
+the first expert GEMM (PFTMoELayer(fused_gather=True)) is reported under
+``gathered_forward`` (``--no-gathered`` skips it), and ``sort_stress`` times the PFT
+build and the RBD plan on a 2^20-token shape (``--sort-stress-only`` runs just that).
+``--gpus N`` without a torchrun environment relaunches this script under torchrun
+with N ranks.
 """
 from __future__ import annotations
 
