@@ -15,16 +15,34 @@
 namespace pfmoe {
 namespace {
 
-// Does (va, ea) come before (vb, eb) in selection order?  ea/eb == INT_MAX means "none".
-__device__ __forceinline__ bool before(float va, int ea, float vb, int eb) {
-  if (ea == INT_MAX) return false;
-  if (eb == INT_MAX) return true;
-  return va > vb || (va == vb && ea < eb);
+// Selection key of (value, expert): larger keys come first.  The float's bits are made monotonic
+// as an unsigned integer (NaN is mapped to -inf before, -0 to +0), and the low half holds ~e, so
+// equal values order by lower expert id: the tie rule of the selection.  Key 0 (below every real
+// key) is "none".
+__device__ __forceinline__ unsigned long long sel_key(float v, int e) {
+  uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);   // -0 and +0 compare equal: one key
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (static_cast<unsigned long long>(u) << 32) | static_cast<uint32_t>(~e);
+}
+__device__ __forceinline__ float key_value(unsigned long long key) {
+  uint32_t u = static_cast<uint32_t>(key >> 32);
+  u = (u & 0x80000000u) ? (u & 0x7fffffffu) : ~u;
+  return __uint_as_float(u);
+}
+__device__ __forceinline__ int key_expert(unsigned long long key) {
+  return static_cast<int>(~static_cast<uint32_t>(key));
+}
+__device__ __forceinline__ void cswap(unsigned long long& a, unsigned long long& b) {   // a >= b after
+  const unsigned long long hi = a > b ? a : b, lo = a > b ? b : a;
+  a = hi;
+  b = lo;
 }
 
 // With parts != null the logits row is first formed from the split-K parts of the gate GEMM
 // (sum in part order, then the bias: the same float operations as a separate reduce) and
-// written out, so the logits take one pass instead of two.
+// written out, so the logits take one pass instead of two.  Each lane sorts its VPT keys once
+// (descending); the k rounds then take the warp maximum of the lanes' heads, and the lane that
+// held it pops its head.
 template <int VPT>
 __global__ void __launch_bounds__(256) topk_kernel(float* __restrict__ logits, const float* __restrict__ parts,
                                                    int nparts, const float* __restrict__ bias, int T, int E, int k,
@@ -35,12 +53,12 @@ __global__ void __launch_bounds__(256) topk_kernel(float* __restrict__ logits, c
   const long long pstride = static_cast<long long>(T) * E;
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
     float* z = logits + static_cast<long long>(t) * E;
-    float v[VPT];
-    uint32_t taken = 0;
+    unsigned long long key[VPT];
     bool nan_seen = false;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int e = lane + 32 * i;
+      key[i] = 0ull;
       if (e < E) {
         float x;
         if (parts) {
@@ -53,29 +71,31 @@ __global__ void __launch_bounds__(256) topk_kernel(float* __restrict__ logits, c
           x = z[e];
         }
         if (x != x) { nan_seen = true; x = -INFINITY; }
-        v[i] = x;
-      } else {
-        v[i] = -INFINITY;
-        taken |= 1u << i;
+        key[i] = sel_key(x, e);
       }
     }
-    float pick_v = -INFINITY;
-    int pick_e = 0;
-    for (int r = 0; r < k; ++r) {
-      float bv = -INFINITY;
-      int be = INT_MAX;
+    // descending sort of the lane's keys (odd-even transposition: VPT rounds)
 #pragma unroll
-      for (int i = 0; i < VPT; ++i)
-        if (!((taken >> i) & 1u) && before(v[i], lane + 32 * i, bv, be)) { bv = v[i]; be = lane + 32 * i; }
+    for (int r = 0; r < VPT; ++r)
+#pragma unroll
+      for (int i = r & 1; i + 1 < VPT; i += 2) cswap(key[i], key[i + 1]);
+    unsigned long long pick = 0ull;
+    for (int r = 0; r < k; ++r) {
+      unsigned long long best = key[0];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (before(ov, oe, bv, be)) { bv = ov; be = oe; }
+        const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+        best = other > best ? other : best;
       }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      if (lane == r) { pick_v = bv; pick_e = be; }
+      if (key[0] == best) {   // keys are distinct per expert: exactly one lane pops
+#pragma unroll
+        for (int i = 0; i + 1 < VPT; ++i) key[i] = key[i + 1];
+        key[VPT - 1] = 0ull;
+      }
+      if (lane == r) pick = best;
     }
+    const float pick_v = key_value(pick);
+    const int pick_e = key_expert(pick);
     const float m = __shfl_sync(0xffffffffu, pick_v, 0);
     const float ex = lane < k ? expf(pick_v - m) : 0.f;
     const float sum = warp_sum(ex);
