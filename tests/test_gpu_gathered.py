@@ -71,7 +71,8 @@ def test_gathered_forward_full_size_matches_materialised_path():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("name", ["small_ragged_bf16", "small_pairs_bf16", "dsv3_bf16"])
+@pytest.mark.parametrize("name", ["small_ragged_bf16", "small_pairs_bf16", "small_skew_bf16", "dsv3_bf16",
+                                  "dsv3_zipf_bf16"])
 def test_gathered_step_equals_materialised_step(name):
     # forward, RBD plan and backward: every output bit for bit
     cfg = get_config(name)
