@@ -478,7 +478,7 @@ size_t rbd_plan_workspace_size(int T, int k, int E, int experts_per_device, int 
   if (T < 0 || k <= 0 || E <= 0 || experts_per_device <= 0 || devices_per_node <= 0) return 0;
   const long long epn = static_cast<long long>(experts_per_device) * devices_per_node;
   if (epn > E || E % epn) return 0;
-  return align256(rbd_ws_bytes(T, k, static_cast<int>(E / epn)));
+  return align256(rbd_ws_bytes(T, k, E, static_cast<int>(E / epn)));
 }
 
 int rbd_plan(const int32_t* topk_ids, int T, int k, int E, int experts_per_device, int devices_per_node,

@@ -69,7 +69,7 @@ size_t csort_ws_bytes(long long n_max, int K);
 int pft_build_impl(const int32_t* ids, const float* w, int T, int E, int k, int32_t* tpe, int32_t* offsets,
                    int32_t* token_ids, int32_t* expert_ids, float* cw, int32_t* pos, int32_t* tile_offsets,
                    void* ws, int32_t* err, cudaStream_t s);
-size_t rbd_ws_bytes(int T, int k, int n_nodes);
+size_t rbd_ws_bytes(int T, int k, int E, int n_nodes);
 int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int32_t* pilots_per_node,
                   int32_t* node_offsets, int32_t* pilot_token, int32_t* pilot_node, int32_t* pilot_device,
                   int32_t* replica_offsets, int32_t* replica_expert, int32_t* assign_pilot, int32_t* counts,

@@ -5,12 +5,14 @@
 // Sort = three launches over chunks of W * 256 consecutive keys (one CTA of W warps
 // per chunk, W = 8 unless the per-warp counters would not fit in shared memory):
 //   1. chunk histograms counts[c][key];
-//   2. one-CTA scan in (key, chunk) order -> per-key totals, key offsets and
-//      every chunk's base row for every key (plus the grouped-GEMM tile prefix);
+//   2. scan in (key, chunk) order -> per-key totals, key offsets and every chunk's base
+//      row for every key (plus the grouped-GEMM tile prefix): one CTA for few chunks, else
+//      a CTA per strip of keys and a key scan;
 //   3. scatter: warp w of a chunk owns keys [256w, 256w + 256) of it; the warps count
 //      their keys per key, take an exclusive prefix over warps, then walk their keys in
-//      order, 32 at a time; lanes holding the same key find each other with
-//      __match_any_sync and take consecutive rows in lane order -> the sort is stable.
+//      order, 32 at a time; lanes holding the same key find each other (one ballot per
+//      key bit, or __match_any_sync for wide keys) and take consecutive rows in lane
+//      order -> the sort is stable.
 #include <climits>
 
 #include "common.cuh"
@@ -43,11 +45,33 @@ __global__ void chunk_hist_kernel(const int32_t* __restrict__ keys, long long n,
   __syncthreads();
   const long long nn = dev_count(n, n_dev);
   const long long b = static_cast<long long>(chunk) * blockDim.x / 32 * KPW;
-  const long long e = min(b + static_cast<long long>(blockDim.x / 32) * KPW, nn);
+  // a chunk is blockDim.x * IT keys: every load of the thread is issued before its first atomic
+  // (16-byte vectors for a whole chunk of 16-byte aligned keys)
+  constexpr int IT = KPW / 32;
+  int key[IT];
+  const bool whole = b + static_cast<long long>(blockDim.x) * IT <= nn;
+  if (whole && (reinterpret_cast<uintptr_t>(keys) & 15) == 0) {
+    const int4* kv = reinterpret_cast<const int4*>(keys + b);
+#pragma unroll
+    for (int h = 0; h < IT / 4; ++h) {
+      const int4 q = kv[h * blockDim.x + threadIdx.x];
+      key[4 * h] = q.x;
+      key[4 * h + 1] = q.y;
+      key[4 * h + 2] = q.z;
+      key[4 * h + 3] = q.w;
+    }
+  } else {
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const long long i = b + static_cast<long long>(it) * blockDim.x + threadIdx.x;
+      key[it] = i < nn ? keys[i] : 0;
+    }
+  }
   bool bad = false;
-  for (long long i = b + threadIdx.x; i < e; i += blockDim.x) {
-    const int key = keys[i];
-    if (static_cast<unsigned>(key) < static_cast<unsigned>(K)) atomicAdd(&sh[key], 1);
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    if (!whole && b + static_cast<long long>(it) * blockDim.x + threadIdx.x >= nn) break;
+    if (static_cast<unsigned>(key[it]) < static_cast<unsigned>(K)) atomicAdd(&sh[key[it]], 1);
     else bad = true;
   }
   if (bad) dev_error(err, PFMOE_DEV_BAD_EXPERT_ID);
@@ -123,27 +147,38 @@ __global__ void __launch_bounds__(SCAN_THREADS) chunk_scan_kernel(const int32_t*
   }
 }
 
-// Many chunks: the [C][K] chunk counts scanned down their columns, for strips of STRIP_KEYS keys (one
-// 32-byte sector of a row) per CTA; its 32 warps take consecutive row segments, a warp instruction
-// covering 4 rows of the strip.  Pass 1 sums each warp's segment per key, the segment sums are scanned
-// per key across the warps, and pass 2 writes each element's exclusive prefix (relative base) in the
-// same order.  Every access is a whole sector (a CTA per key used one int per sector).
-constexpr int STRIP_KEYS = 8;
+// Many chunks: the [C][K] chunk counts scanned down their columns, for strips of STRIP_KEYS keys per
+// CTA; its 32 warps take consecutive row segments, a warp instruction covering 32 / STRIP_KEYS rows of
+// the strip.  Pass 1 sums each warp's segment per key, the segment sums are scanned per key across the
+// warps, and pass 2 writes each element's exclusive prefix (relative base) in the same order.  A narrow
+// strip spreads the scan over more SMs (K / STRIP_KEYS CTAs); the partly used sectors it reads are L2
+// hits, the counts having just been written.
+constexpr int STRIP_KEYS = 2;
+constexpr int STRIP_ROWS = 32 / STRIP_KEYS;   // rows per warp step
 
 __global__ void __launch_bounds__(SCAN_THREADS) strip_scan_kernel(const int32_t* __restrict__ counts, int C, int K,
                                                                   int32_t* __restrict__ base, int32_t* totals) {
   __shared__ int wsum[SCAN_THREADS / 32][STRIP_KEYS];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kk = lane % STRIP_KEYS, rsub = lane / STRIP_KEYS;   // key of the strip, row of a 4-row step
+  const int kk = lane % STRIP_KEYS, rsub = lane / STRIP_KEYS;   // key of the strip, row of a step
   const int key = blockIdx.x * STRIP_KEYS + kk;
   const bool kok = key < K;
   const int R = (C + SCAN_THREADS / 32 - 1) / (SCAN_THREADS / 32);   // rows per warp
   const int r0 = min(C, warp * R), r1 = min(C, r0 + R);
+  constexpr int U = 8;   // row steps whose loads are in flight together
   int sum = 0;
-  for (int c = r0 + rsub; c < r1; c += 4)
-    if (kok) sum += counts[static_cast<long long>(c) * K + key];
-  sum += __shfl_xor_sync(0xffffffffu, sum, 8);
-  sum += __shfl_xor_sync(0xffffffffu, sum, 16);
+  for (int c0 = r0 + rsub; c0 < r1; c0 += STRIP_ROWS * U) {
+    int v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + STRIP_ROWS * u;
+      v[u] = kok && c < r1 ? counts[static_cast<long long>(c) * K + key] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) sum += v[u];
+  }
+#pragma unroll
+  for (int o = STRIP_KEYS; o < 32; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   if (rsub == 0) wsum[warp][kk] = sum;
   __syncthreads();
   if (warp == 0 && lane < STRIP_KEYS) {
@@ -157,18 +192,25 @@ __global__ void __launch_bounds__(SCAN_THREADS) strip_scan_kernel(const int32_t*
   }
   __syncthreads();
   int carry = wsum[warp][kk];
-  for (int c0 = r0; c0 < r1; c0 += 4) {
-    const int c = c0 + rsub;
-    const bool ok = c < r1 && kok;
-    const long long idx = static_cast<long long>(c) * K + key;
-    const int v = ok ? counts[idx] : 0;
-    int x = v;   // inclusive prefix over the step's rows of this key (lanes kk, kk + 8, kk + 16, kk + 24)
-    int y = __shfl_up_sync(0xffffffffu, x, 8);
-    if (rsub >= 1) x += y;
-    y = __shfl_up_sync(0xffffffffu, x, 16);
-    if (rsub >= 2) x += y;
-    if (ok) base[idx] = carry + x - v;
-    carry += __shfl_sync(0xffffffffu, x, 3 * STRIP_KEYS + kk);
+  for (int c0 = r0; c0 < r1; c0 += STRIP_ROWS * U) {
+    int v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + STRIP_ROWS * u + rsub;
+      v[u] = c < r1 && kok ? counts[static_cast<long long>(c) * K + key] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + STRIP_ROWS * u + rsub;
+      int x = v[u];   // inclusive prefix over the step's rows of this key (lanes kk, kk + STRIP_KEYS, ...)
+#pragma unroll
+      for (int o = 1; o < STRIP_ROWS; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o * STRIP_KEYS);
+        if (rsub >= o) x += y;
+      }
+      if (c < r1 && kok) base[static_cast<long long>(c) * K + key] = carry + x - v[u];
+      carry += __shfl_sync(0xffffffffu, x, (STRIP_ROWS - 1) * STRIP_KEYS + kk);
+    }
   }
 }
 
@@ -204,18 +246,38 @@ __global__ void __launch_bounds__(SCAN_THREADS) key_scan_kernel(const int32_t* _
 // among the warp's equal keys) and stages it in shared memory in sorted order.  The write-out then
 // stores the row-indexed outputs as runs of consecutive rows, so neighbouring lanes write
 // neighbouring addresses instead of one scattered sector per element.
-// Sink interface: at_source(i, p) writes the outputs indexed by element i; payload(i, a, b) gives
-// two ints carried to the sorted side; at_dest(p, key, a, b) writes the outputs indexed by row p.
+// Sink interface: preload(i) is read with the keys, before the passes (one int); at_source(i, p)
+// writes the outputs indexed by element i; payload(i, pre, a, b) gives two ints carried to the sorted
+// side; at_dest(p, key, a, b) writes the outputs indexed by row p.
+// Lanes holding equal keys (peers) are found with __match_any_sync, or for keys of at most KEY_BITS
+// bits with one ballot per key bit.
 // Shared memory: [warps][K] counts, two [K] bases and three [warps * KPW] staging arrays.
 __host__ __device__ inline size_t scatter_smem_bytes(int nw, int K) {
   return (static_cast<size_t>(nw) * K + 2 * static_cast<size_t>(K) + 3 * static_cast<size_t>(nw) * KPW) *
          sizeof(int32_t);
 }
 
-// Six blocks per SM: with the default register allocation (64) only four fit, and the scatter,
-// bound by shared-memory latency, ran 19 % slower on the 2^23-key stress shape.
-template <class Sink>
-__global__ void __launch_bounds__(256, 6) chunk_scatter_kernel(const int32_t* __restrict__ keys, long long n, const int32_t* n_dev, int K,
+template <int KEY_BITS>
+__device__ __forceinline__ unsigned key_peers(bool ok, int key) {
+  const unsigned valid = __ballot_sync(0xffffffffu, ok);
+  if constexpr (KEY_BITS == 0) {
+    return __match_any_sync(0xffffffffu, ok ? key : -1 - static_cast<int>(threadIdx.x & 31)) & valid;
+  } else {
+    unsigned peers = valid;
+#pragma unroll
+    for (int bit = 0; bit < KEY_BITS; ++bit) {
+      const bool set = (key >> bit) & 1;
+      const unsigned bal = __ballot_sync(0xffffffffu, set);
+      peers &= set ? bal : ~bal;
+    }
+    return peers;
+  }
+}
+
+// Five blocks per SM (48 registers): the key, preload and peer registers of a thread's eight
+// elements stay live across the passes; with 64 registers only four blocks fit, with 40 they spill.
+template <class Sink, int KEY_BITS>
+__global__ void __launch_bounds__(256, 5) chunk_scatter_kernel(const int32_t* __restrict__ keys, long long n, const int32_t* n_dev, int K,
                                      int nchunks, const int32_t* __restrict__ base,
                                      const int32_t* __restrict__ key_offsets, Sink sink) {
   extern __shared__ int32_t sh[];
@@ -230,27 +292,28 @@ __global__ void __launch_bounds__(256, 6) chunk_scatter_kernel(const int32_t* __
   int32_t* skey = gbase + K;                           // [nw * KPW]: staged keys, in sorted order
   int32_t* spa = skey + nw * KPW;                      // staged payloads
   int32_t* spb = spa + nw * KPW;
-  for (int i = threadIdx.x; i < nw * K; i += blockDim.x) cnt[i] = 0;
-  __syncthreads();
   const long long nn = dev_count(n, n_dev);
   const long long b = (static_cast<long long>(chunk) * nw + w) * KPW;
-  int32_t* wcnt = cnt + w * K;
   constexpr int IT = KPW / 32;
-  int key[IT];
-  unsigned peers[IT];
+  // every global load of the CTA is issued here: the keys, the sink's preload, and the first row of
+  // key threadIdx.x in this chunk
+  int key[IT], pre[IT];
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
     const long long i = b + it * 32 + lane;
     key[it] = i < nn ? keys[i] : -1;
+    pre[it] = i < nn ? sink.preload(i) : 0;
   }
-  // pass 1: per-warp counts (one shared update per distinct key per 32 keys)
+  const int gfirst = threadIdx.x < K && chunk < nchunks
+                         ? key_offsets[threadIdx.x] + base[static_cast<long long>(chunk) * K + threadIdx.x]
+                         : 0;
+  for (int i = threadIdx.x; i < nw * K; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  int32_t* wcnt = cnt + w * K;
+  // pass 1: per-warp counts by shared atomics (a count does not depend on the order of equal keys)
 #pragma unroll
-  for (int it = 0; it < IT; ++it) {
-    const bool ok = static_cast<unsigned>(key[it]) < static_cast<unsigned>(K);
-    peers[it] = __match_any_sync(0xffffffffu, ok ? key[it] : K + lane);
-    if (ok && (peers[it] & ((1u << lane) - 1u)) == 0) wcnt[key[it]] += __popc(peers[it]);
-    __syncwarp();
-  }
+  for (int it = 0; it < IT; ++it)
+    if (static_cast<unsigned>(key[it]) < static_cast<unsigned>(K)) atomicAdd(&wcnt[key[it]], 1);
   __syncthreads();
   // per key: each warp's start within the key's run of this chunk, the run length, the first row
   for (int k = threadIdx.x; k < K; k += blockDim.x) {
@@ -261,7 +324,8 @@ __global__ void __launch_bounds__(256, 6) chunk_scatter_kernel(const int32_t* __
       run += c;
     }
     lbase[k] = run;
-    gbase[k] = chunk < nchunks ? key_offsets[k] + base[static_cast<long long>(chunk) * K + k] : 0;
+    gbase[k] = k == threadIdx.x ? gfirst
+                                : (chunk < nchunks ? key_offsets[k] + base[static_cast<long long>(chunk) * K + k] : 0);
   }
   __syncthreads();
   // run lengths -> first staging slot of each key (exclusive scan over keys)
@@ -271,7 +335,10 @@ __global__ void __launch_bounds__(256, 6) chunk_scatter_kernel(const int32_t* __
     const int v = k < K ? lbase[k] : 0;
     int blk;
     const int ex = block_excl_scan(v, tmp, &blk);
-    if (k < K) lbase[k] = carry + ex;
+    if (k < K) {
+      lbase[k] = carry + ex;
+      gbase[k] -= carry + ex;   // from here: sorted row - staging slot, for every slot of key k
+    }
     carry += blk;
   }
   if (threadIdx.x == 0) staged = carry;
@@ -280,18 +347,19 @@ __global__ void __launch_bounds__(256, 6) chunk_scatter_kernel(const int32_t* __
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
     const bool ok = static_cast<unsigned>(key[it]) < static_cast<unsigned>(K);
-    const int rank = __popc(peers[it] & ((1u << lane) - 1u));
+    const unsigned peers = key_peers<KEY_BITS>(ok, key[it]);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
     const int c0 = ok ? wcnt[key[it]] : 0;
     __syncwarp();
-    if (ok && rank == 0) wcnt[key[it]] = c0 + __popc(peers[it]);
+    if (ok && rank == 0) wcnt[key[it]] = c0 + __popc(peers);
     __syncwarp();
     if (ok) {
       const long long i = b + it * 32 + lane;
       const int r = c0 + rank;
       const int lp = lbase[key[it]] + r;
-      sink.at_source(i, gbase[key[it]] + r);
+      sink.at_source(i, gbase[key[it]] + lp);
       int32_t pa, pb;
-      sink.payload(i, pa, pb);
+      sink.payload(i, pre[it], pa, pb);
       skey[lp] = key[it];
       spa[lp] = pa;
       spb[lp] = pb;
@@ -302,7 +370,7 @@ __global__ void __launch_bounds__(256, 6) chunk_scatter_kernel(const int32_t* __
   const int nv = staged;
   for (int lp = threadIdx.x; lp < nv; lp += blockDim.x) {
     const int k = skey[lp];
-    sink.at_dest(gbase[k] + (lp - lbase[k]), k, spa[lp], spb[lp]);
+    sink.at_dest(gbase[k] + lp, k, spa[lp], spb[lp]);
   }
 }
 
@@ -310,14 +378,16 @@ __global__ void __launch_bounds__(256, 6) chunk_scatter_kernel(const int32_t* __
 struct PftSink {
   const float* w;
   int k;
+  unsigned long long kinv;   // 2^64 / k rounded up (k > 1): i / k = high word of i * kinv for any 32-bit i
   int32_t* pos;
   int32_t* token_ids;
   int32_t* expert_ids;
   float* cw;
+  __device__ int32_t preload(long long i) const { return __float_as_int(w[i]); }
   __device__ void at_source(long long i, int p) const { pos[i] = p; }
-  __device__ void payload(long long i, int32_t& a, int32_t& b) const {
-    a = static_cast<int32_t>(static_cast<uint32_t>(i) / static_cast<uint32_t>(k));
-    b = __float_as_int(w[i]);
+  __device__ void payload(long long i, int32_t pre, int32_t& a, int32_t& b) const {
+    a = k > 1 ? static_cast<int32_t>(__umul64hi(static_cast<unsigned long long>(i), kinv)) : static_cast<int32_t>(i);
+    b = pre;
   }
   __device__ void at_dest(int p, int key, int32_t a, int32_t b) const {
     token_ids[p] = a;
@@ -552,10 +622,11 @@ struct RbdSink {
   int32_t* pilot_node;
   int32_t* rc_sorted;
   int32_t* psorted;
+  __device__ int32_t preload(long long i) const { return prc[i]; }
   __device__ void at_source(long long i, int p) const { psorted[i] = p; }
-  __device__ void payload(long long i, int32_t& a, int32_t& b) const {
+  __device__ void payload(long long i, int32_t pre, int32_t& a, int32_t& b) const {
     a = ptoken[i];
-    b = prc[i];
+    b = pre;
   }
   __device__ void at_dest(int p, int key, int32_t a, int32_t b) const {
     pilot_token[p] = a;
@@ -608,45 +679,85 @@ struct FastDiv {
   }
 };
 
-// The tile's ids ([RF_TILE][k] consecutive ints) are staged in shared memory with coalesced loads;
-// each thread then reads its token's k ids from there.
-__device__ __forceinline__ void rf_stage_ids(const int32_t* __restrict__ ids, int T, int k, int32_t* sids) {
+// The tile's ids are staged in shared memory with coalesced loads, one padded row of KM + 1 ints per
+// token (row r holds token r's k ids), so that each thread's reads of its own row are free of bank
+// conflicts for every k.
+template <int KM>
+__device__ __forceinline__ void rf_stage_rows(const int32_t* __restrict__ ids, int T, int k, int32_t* rows) {
   const long long base = static_cast<long long>(blockIdx.x) * RF_TILE * k;
   const long long end = static_cast<long long>(T) * k;
-  for (int i = threadIdx.x; i < RF_TILE * k; i += blockDim.x)
-    sids[i] = base + i < end ? ids[base + i] : 0;
+  const FastDiv row_of(k);
+  int v[KM];
+#pragma unroll
+  for (int it = 0; it < KM; ++it) {
+    const long long g = base + it * RF_TILE + threadIdx.x;
+    v[it] = it < k && g < end ? ids[g] : 0;
+  }
+#pragma unroll
+  for (int it = 0; it < KM; ++it)
+    if (it < k) {
+      const int i = it * RF_TILE + threadIdx.x;   // below RF_TILE * KM <= 2^13, so the division is exact
+      const int r = row_of(i);
+      rows[r * (KM + 1) + (i - r * k)] = v[it];
+    }
   __syncthreads();
 }
 
+// The token's ids as sort keys id * 256 + slot, in ascending order (slots k .. KM - 1 and tokens past
+// T hold INT_MAX).  Ids outside [0, E) are flagged (when err is given) and read as 0.  Node and device
+// are monotone in the id, so each node's replicas form one run of the sorted keys, in (id, slot) order,
+// and the run's first key is the node's lowest id.  Bitonic sorting network, unrolled over KM.
 template <int KM>
-__device__ __forceinline__ void rf_load(const int32_t* __restrict__ sids, bool valid, int k, int E, const FastDiv& node_of,
-                                        int (&e)[KM], int (&nd)[KM], int32_t* err) {
+__device__ __forceinline__ void rf_sorted_keys(const int32_t* row, bool valid, int k, int E, int32_t* err,
+                                               int (&key)[KM]) {
 #pragma unroll
   for (int j = 0; j < KM; ++j) {
-    int v = 0;
+    int x = INT_MAX;
     if (valid && j < k) {
-      v = sids[threadIdx.x * k + j];
+      int v = row[j];
       if (static_cast<unsigned>(v) >= static_cast<unsigned>(E)) {
-        dev_error(err, PFMOE_DEV_BAD_EXPERT_ID);
+        if (err) dev_error(err, PFMOE_DEV_BAD_EXPERT_ID);
         v = 0;
       }
+      x = (v << 8) | j;
     }
-    e[j] = v;
-    nd[j] = (valid && j < k) ? node_of(v) : -1;
+    key[j] = x;
   }
+#pragma unroll
+  for (int size = 2; size <= KM; size <<= 1)
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1)
+#pragma unroll
+      for (int i = 0; i < KM; ++i) {
+        const int p = i ^ stride;
+        if (p > i) {
+          const int lo = min(key[i], key[p]), hi = max(key[i], key[p]);
+          const bool up = (i & size) == 0;
+          key[i] = up ? lo : hi;
+          key[p] = up ? hi : lo;
+        }
+      }
+}
+
+// The token's replicas per node, 8 bits per node (k <= 32 < 256; nodes < RF_NODES = 8).
+template <int KM>
+__device__ __forceinline__ unsigned long long rf_node_counts(const int (&key)[KM], const FastDiv& node_of) {
+  unsigned long long cnt = 0;
+#pragma unroll
+  for (int s = 0; s < KM; ++s)
+    if (key[s] != INT_MAX) cnt += 1ull << (8 * node_of(key[s] >> 8));
+  return cnt;
+}
+
+__device__ __forceinline__ int rf_node_field(unsigned long long packed, int n) {
+  return static_cast<int>((packed >> (8 * n)) & 0xffu);
 }
 
 // Packed per-node count of one token: bit 0..15 = 1 if the token routes to the node, 16..31 = its
 // replicas there (sums over a 256-token tile stay below 2^16 in both fields).
-template <int KM>
-__device__ __forceinline__ void rf_counts(const int (&nd)[KM], int (&c)[RF_NODES]) {
-#pragma unroll
-  for (int n = 0; n < RF_NODES; ++n) {
-    int r = 0;
-#pragma unroll
-    for (int j = 0; j < KM; ++j) r += nd[j] == n;
-    c[n] = (r > 0 ? 1 : 0) | (r << 16);
-  }
+__device__ __forceinline__ int rf_packed(unsigned long long cnt, int n) {
+  const int r = rf_node_field(cnt, n);
+  return (r > 0 ? 1 : 0) | (r << 16);
 }
 
 template <int KM>
@@ -654,29 +765,26 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_count_kernel(const int32_t* 
                                                                  int epd, int epn, int32_t* __restrict__ tile_cnt,
                                                                  int32_t* __restrict__ tile_dev, int32_t* err) {
   __shared__ int red[RF_TILE / 32][RF_NODES + 1];
-  __shared__ int32_t sids[RF_TILE * KM];
+  __shared__ int32_t rows[RF_TILE * (KM + 1)];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long t = static_cast<long long>(blockIdx.x) * RF_TILE + threadIdx.x;
   const bool valid = t < T;
-  int e[KM], nd[KM], c[RF_NODES];
-  rf_stage_ids(ids, T, k, sids);
+  rf_stage_rows<KM>(ids, T, k, rows);
   const FastDiv node_of(epn), dev_of(epd);
-  rf_load<KM>(sids, valid, k, E, node_of, e, nd, err);
-  rf_counts<KM>(nd, c);
-  int dv[KM];
+  int key[KM];
+  rf_sorted_keys<KM>(rows + threadIdx.x * (KM + 1), valid, k, E, err, key);
+  const unsigned long long cnt = rf_node_counts<KM>(key, node_of);
+  int dc = 0, prev = -1;   // distinct devices of the token: the device changes along the sorted ids
 #pragma unroll
-  for (int j = 0; j < KM; ++j) dv[j] = dev_of(e[j]);
-  int dc = 0;   // distinct devices of the token
-#pragma unroll
-  for (int j = 0; j < KM; ++j) {
-    bool first = j < k && valid;
-#pragma unroll
-    for (int i = 0; i < j; ++i) first = first && (dv[i] != dv[j]);
-    dc += first;
-  }
+  for (int s = 0; s < KM; ++s)
+    if (key[s] != INT_MAX) {
+      const int dv = dev_of(key[s] >> 8);
+      dc += dv != prev;
+      prev = dv;
+    }
 #pragma unroll
   for (int n = 0; n < RF_NODES; ++n) {
-    int v = c[n];
+    int v = rf_packed(cnt, n);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) red[warp][n] = v;
@@ -813,7 +921,12 @@ __global__ void __launch_bounds__(RF_SCAN_THREADS) rbd_fast_scan_kernel(int ntil
 
 // Per token: the in-tile prefix by warp scans, then the outputs.  The pilot rows of one node in a
 // tile are consecutive, so the per-node pilot stores are coalesced; the replica lists and
-// assign_pilot are staged in shared memory (the ids' buffer, reused) and leave as contiguous runs.
+// assign_pilot are staged in shared memory and leave as contiguous runs.  Each thread keeps its
+// token's sorted keys in its own padded row and reads a node's run back from there.
+// Dynamic shared memory: RF_TILE rows of KM + 1 ints, then the RF_TILE * KM staging ints.
+template <int KM>
+constexpr int rf_emit_smem() { return (RF_TILE * (KM + 1) + RF_TILE * KM) * 4; }
+
 template <int KM>
 __global__ void __launch_bounds__(RF_TILE) rbd_fast_emit_kernel(
     const int32_t* __restrict__ ids, int T, int k, int E, int epd, int epn, int n_nodes,
@@ -821,21 +934,40 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_emit_kernel(
     const int32_t* __restrict__ node_offsets, const int32_t* __restrict__ node_rep_off, int32_t* __restrict__ pilot_token,
     int32_t* __restrict__ pilot_node, int32_t* __restrict__ pilot_device, int32_t* __restrict__ replica_offsets,
     int32_t* __restrict__ replica_expert, int32_t* __restrict__ assign_pilot, int32_t* err) {
+  extern __shared__ int32_t rf_sm[];
   __shared__ int wsum[RF_TILE / 32][RF_NODES];
   __shared__ int node_loc[RF_NODES + 1];   // replicas of earlier nodes in this tile
-  __shared__ int32_t sbuf[RF_TILE * KM];   // the tile's ids, then its replica lists, then assign_pilot
+  __shared__ int tok_base[RF_NODES];       // per node: the tile's first pilot row
+  __shared__ int rep_gbase[RF_NODES];      // per node: the tile's first replica row
+  int32_t* rows = rf_sm;                   // [RF_TILE][KM + 1]: the tile's ids, then each token's sorted keys
+  int32_t* sbuf = rf_sm + RF_TILE * (KM + 1);   // [RF_TILE * KM]: replica lists, then assign_pilot
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long t = static_cast<long long>(blockIdx.x) * RF_TILE + threadIdx.x;
   const bool valid = t < T;
-  int e[KM], nd[KM], c[RF_NODES], ex[RF_NODES];
-  rf_stage_ids(ids, T, k, sbuf);
+  const long long tb = static_cast<long long>(blockIdx.x) * RF_NODES;
+  if (threadIdx.x < n_nodes) {
+    tok_base[threadIdx.x] = node_offsets[threadIdx.x] + tile_tok_base[tb + threadIdx.x];
+    rep_gbase[threadIdx.x] = node_rep_off[threadIdx.x] + tile_rep_base[tb + threadIdx.x];
+  }
+  rf_stage_rows<KM>(ids, T, k, rows);
+  (void)err;   // rbd_fast_count flagged bad ids
   const FastDiv node_of(epn), dev_of(epd);
-  rf_load<KM>(sbuf, valid, k, E, node_of, e, nd, nullptr);   // rbd_fast_count flagged bad ids
-  (void)err;
-  rf_counts<KM>(nd, c);
+  int32_t* row = rows + threadIdx.x * (KM + 1);
+  unsigned long long cnt;
+  {
+    int key[KM];
+    rf_sorted_keys<KM>(row, valid, k, E, nullptr, key);
+#pragma unroll
+    for (int s = 0; s < KM; ++s) row[s] = key[s];
+    cnt = rf_node_counts<KM>(key, node_of);
+  }
+  // byte n: the token's replicas on nodes before n = the sorted position of node n's run
+  const unsigned long long first = cnt * 0x0101010101010101ull - cnt;
+  int c[RF_NODES], ex[RF_NODES];
   // in-warp exclusive prefix of the packed counts, per node
 #pragma unroll
   for (int n = 0; n < RF_NODES; ++n) {
+    c[n] = rf_packed(cnt, n);
     int a = c[n];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -845,7 +977,7 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_emit_kernel(
     ex[n] = a - c[n];
     if (lane == 31) wsum[warp][n] = a;
   }
-  __syncthreads();   // wsum complete; every thread has read its ids from sbuf
+  __syncthreads();   // wsum complete
   if (warp == 0) {
     // lane n < RF_NODES: column n of wsum -> exclusive prefix over the warps (the packed fields add
     // independently); the node's replica total -> node_loc by a scan over lanes 0 .. RF_NODES - 1
@@ -869,64 +1001,41 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_emit_kernel(
     if (lane == RF_NODES - 1) node_loc[RF_NODES] = x;
   }
   __syncthreads();   // node_loc and the warp prefixes ready
-  int rep_base[RF_NODES];   // this token's first slot in the tile's replica staging, per node
-#pragma unroll
-  for (int n = 0; n < RF_NODES; ++n) {
-    ex[n] += wsum[warp][n];
-    rep_base[n] = node_loc[n] + (ex[n] >> 16);
-  }
-  const long long tb = static_cast<long long>(blockIdx.x) * RF_NODES;
   int idx[RF_NODES];
 #pragma unroll
   for (int n = 0; n < RF_NODES; ++n) {
+    ex[n] += wsum[warp][n];
     idx[n] = 0;
     if (valid && n < n_nodes && (c[n] & 0xffff)) {
-      idx[n] = node_offsets[n] + tile_tok_base[tb + n] + (ex[n] & 0xffff);
-      int emin = INT_MAX;
-#pragma unroll
-      for (int j = 0; j < KM; ++j)
-        if (nd[j] == n && e[j] < emin) emin = e[j];
+      idx[n] = tok_base[n] + (ex[n] & 0xffff);
       pilot_token[idx[n]] = static_cast<int32_t>(t);
       pilot_node[idx[n]] = n;
-      pilot_device[idx[n]] = dev_of(emin);
-      replica_offsets[idx[n]] = node_rep_off[n] + tile_rep_base[tb + n] + (ex[n] >> 16);
+      pilot_device[idx[n]] = dev_of(row[rf_node_field(first, n)] >> 8);   // the node's lowest id
+      replica_offsets[idx[n]] = rep_gbase[n] + (ex[n] >> 16);
     }
   }
-  // replica lists, node by node in this tile's part of replica_expert
+  // replica lists: node n's run of sorted keys at this token's slots of the tile's staging
   if (valid) {
 #pragma unroll
-    for (int j = 0; j < KM; ++j) {
-      if (j < k) {
-        int within = 0;
-#pragma unroll
-        for (int i = 0; i < KM; ++i)
-          within += (i < k) && nd[i] == nd[j] && (e[i] < e[j] || (e[i] == e[j] && i < j));
-        int loc = 0;
-#pragma unroll
-        for (int n = 0; n < RF_NODES; ++n)
-          if (nd[j] == n) loc = rep_base[n];
-        sbuf[loc + within] = e[j];
-      }
+    for (int n = 0; n < RF_NODES; ++n) {
+      const int cn = rf_node_field(cnt, n), f = rf_node_field(first, n);
+      const int at = node_loc[n] + (ex[n] >> 16);
+      for (int w = 0; w < cn; ++w) sbuf[at + w] = row[f + w] >> 8;
     }
   }
   __syncthreads();
   for (int n = 0; n < n_nodes; ++n) {
-    const int cnt = node_loc[n + 1] - node_loc[n];
-    const long long g0 = static_cast<long long>(node_rep_off[n]) + tile_rep_base[tb + n];
-    for (int i = threadIdx.x; i < cnt; i += RF_TILE) replica_expert[g0 + i] = sbuf[node_loc[n] + i];
+    const int cn = node_loc[n + 1] - node_loc[n];
+    const long long g0 = rep_gbase[n];
+    for (int i = threadIdx.x; i < cn; i += RF_TILE) replica_expert[g0 + i] = sbuf[node_loc[n] + i];
   }
   __syncthreads();
-  // assign_pilot: the tile's [tokens][k] block is contiguous
+  // assign_pilot: the tile's [tokens][k] block is contiguous; slot j of a key is its low byte
   if (valid) {
 #pragma unroll
-    for (int j = 0; j < KM; ++j) {
-      if (j < k) {
-        int pj = 0;
-#pragma unroll
-        for (int n = 0; n < RF_NODES; ++n)
-          if (nd[j] == n) pj = idx[n];
-        sbuf[threadIdx.x * k + j] = pj;
-      }
+    for (int n = 0; n < RF_NODES; ++n) {
+      const int cn = rf_node_field(cnt, n), f = rf_node_field(first, n);
+      for (int w = 0; w < cn; ++w) sbuf[threadIdx.x * k + (row[f + w] & 0xff)] = idx[n];
     }
   }
   __syncthreads();
@@ -975,9 +1084,10 @@ constexpr long long LONG_SCAN_MIN = 4LL * SCAN_TILE;   // below this one CTA sca
 
 // The staged scatter needs up to ~95 KB of shared memory (K = 4096 keys, three warps): opt in
 // once per device.
-template <class Sink>
+template <class Sink, int KEY_BITS>
 int scatter_smem_attr() {
-  return smem_optin(reinterpret_cast<const void*>(&chunk_scatter_kernel<Sink>), 227 * 1024, "chunk_scatter");
+  return smem_optin(reinterpret_cast<const void*>(&chunk_scatter_kernel<Sink, KEY_BITS>), 227 * 1024,
+                    "chunk_scatter");
 }
 
 // Histogram + scatter launches of one stable counting sort.
@@ -989,14 +1099,23 @@ int sort_hist(const int32_t* keys, long long n_max, const int32_t* n_dev, int K,
   return PFMOE_OK;
 }
 
+template <class Sink, int KEY_BITS>
+int sort_scatter_as(const int32_t* keys, long long n_max, const int32_t* n_dev, int K, int C, const int32_t* base,
+                    const int32_t* key_offsets, const Sink& sink, const char* name, cudaStream_t s) {
+  const int wpb = warps_per_block(K);
+  PFMOE_TRY((scatter_smem_attr<Sink, KEY_BITS>()));
+  PFMOE_LAUNCH(name, s, (chunk_scatter_kernel<Sink, KEY_BITS><<<C, wpb * 32, scatter_smem_bytes(wpb, K), s>>>(
+                            keys, n_max, n_dev, K, C, base, key_offsets, sink)));
+  return PFMOE_OK;
+}
+
+// Equal keys found by ballots over their bits up to 1024 keys, else by __match_any_sync.
 template <class Sink>
 int sort_scatter(const int32_t* keys, long long n_max, const int32_t* n_dev, int K, int C, const int32_t* base,
                  const int32_t* key_offsets, const Sink& sink, const char* name, cudaStream_t s) {
-  const int wpb = warps_per_block(K);
-  PFMOE_TRY(scatter_smem_attr<Sink>());
-  PFMOE_LAUNCH(name, s, (chunk_scatter_kernel<Sink><<<C, wpb * 32, scatter_smem_bytes(wpb, K), s>>>(
-                            keys, n_max, n_dev, K, C, base, key_offsets, sink)));
-  return PFMOE_OK;
+  if (K <= 256) return sort_scatter_as<Sink, 8>(keys, n_max, n_dev, K, C, base, key_offsets, sink, name, s);
+  if (K <= 1024) return sort_scatter_as<Sink, 10>(keys, n_max, n_dev, K, C, base, key_offsets, sink, name, s);
+  return sort_scatter_as<Sink, 0>(keys, n_max, n_dev, K, C, base, key_offsets, sink, name, s);
 }
 
 template <int KM>
@@ -1014,9 +1133,10 @@ static int rbd_fast_launch(const int32_t* ids, int T, int k, int E, int epd, int
                (rbd_fast_scan_kernel<<<1, RF_SCAN_THREADS, RF_SCAN_SMEM, s>>>(ntiles, n_nodes, tile_cnt, tile_rep,
                                                                               tile_dev, ppn, noff, node_rep_off,
                                                                               counts, roff)));
+  PFMOE_TRY(smem_optin(reinterpret_cast<const void*>(&rbd_fast_emit_kernel<KM>), rf_emit_smem<KM>(), "rbd_emit"));
   if (ntiles > 0)
     PFMOE_LAUNCH("rbd_emit", s,
-               (rbd_fast_emit_kernel<KM><<<ntiles, RF_TILE, 0, s>>>(ids, T, k, E, epd, epn, n_nodes, tile_cnt, tile_rep,
+               (rbd_fast_emit_kernel<KM><<<ntiles, RF_TILE, rf_emit_smem<KM>(), s>>>(ids, T, k, E, epd, epn, n_nodes, tile_cnt, tile_rep,
                                                                     noff, node_rep_off, ptok, pnode, pdev, roff, rexp,
                                                                     ap, err)));
   return PFMOE_OK;
@@ -1057,7 +1177,7 @@ int pft_build_impl(const int32_t* ids, const float* w, int T, int E, int k, int3
   if (C > 0) PFMOE_TRY(sort_hist(ids, N, nullptr, E, C, counts, err, "pft_hist", s));
   int32_t* key_tot = base + static_cast<long long>(C) * E;
   PFMOE_TRY(sort_scan(counts, C, E, tpe, offsets, base, tile_offsets, 128, key_tot, "pft_scan", s));
-  PftSink sink{w, k, pos, token_ids, expert_ids, cw};
+  PftSink sink{w, k, k > 1 ? ~0ull / static_cast<unsigned>(k) + 1 : 0ull, pos, token_ids, expert_ids, cw};
   if (C > 0) PFMOE_TRY(sort_scatter<PftSink>(ids, N, nullptr, E, C, base, offsets, sink, "pft_scatter", s));
   return PFMOE_OK;
 }
@@ -1068,8 +1188,12 @@ static size_t rbd_fast_ws_bytes(int T) {
   return (2 * tiles * RF_NODES + tiles + 64) * sizeof(int32_t);
 }
 
-size_t rbd_ws_bytes(int T, int k, int n_nodes) {
-  if (n_nodes <= RF_NODES) return rbd_fast_ws_bytes(T);
+// The plan without a sort serves maps of at most RF_NODES nodes whose ids fit the 16-bit fast division
+// and the id * 256 + slot sort keys.
+static bool rbd_fast_ok(int E, int n_nodes) { return n_nodes <= RF_NODES && E <= (1 << 16); }
+
+size_t rbd_ws_bytes(int T, int k, int E, int n_nodes) {
+  if (rbd_fast_ok(E, n_nodes)) return rbd_fast_ws_bytes(T);
   const long long pmax = static_cast<long long>(T) * (k < n_nodes ? k : n_nodes);
   const long long lt = long_scan_tiles(pmax > T ? pmax : T);
   const size_t ints = 3 * static_cast<size_t>(T) + 5 * static_cast<size_t>(pmax) + 2 * static_cast<size_t>(lt) + 128;
@@ -1082,7 +1206,7 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
                   void* ws, int32_t* err, cudaStream_t s) {
   const int epn = epd * dpn;
   const int n_nodes = E / epn;
-  if (n_nodes <= RF_NODES) return rbd_fast_impl(ids, T, k, E, epd, epn, n_nodes, pilots_per_node, node_offsets,
+  if (rbd_fast_ok(E, n_nodes)) return rbd_fast_impl(ids, T, k, E, epd, epn, n_nodes, pilots_per_node, node_offsets,
                                                 pilot_token, pilot_node, pilot_device, replica_offsets, replica_expert,
                                                 assign_pilot, counts, ws, err, s);
   const long long pmax = static_cast<long long>(T) * (k < n_nodes ? k : n_nodes);
