@@ -708,8 +708,7 @@ __device__ __forceinline__ void rf_stage_rows(const int32_t* __restrict__ ids, i
 // are monotone in the id, so each node's replicas form one run of the sorted keys, in (id, slot) order,
 // and the run's first key is the node's lowest id.  Bitonic sorting network, unrolled over KM.
 template <int KM>
-__device__ __forceinline__ void rf_sorted_keys(const int32_t* row, bool valid, int k, int E, int32_t* err,
-                                               int (&key)[KM]) {
+__device__ __forceinline__ void rf_keys(const int32_t* row, bool valid, int k, int E, int32_t* err, int (&key)[KM]) {
 #pragma unroll
   for (int j = 0; j < KM; ++j) {
     int x = INT_MAX;
@@ -723,6 +722,12 @@ __device__ __forceinline__ void rf_sorted_keys(const int32_t* row, bool valid, i
     }
     key[j] = x;
   }
+}
+
+template <int KM>
+__device__ __forceinline__ void rf_sorted_keys(const int32_t* row, bool valid, int k, int E, int32_t* err,
+                                               int (&key)[KM]) {
+  rf_keys<KM>(row, valid, k, E, err, key);
 #pragma unroll
   for (int size = 2; size <= KM; size <<= 1)
 #pragma unroll
@@ -772,16 +777,26 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_count_kernel(const int32_t* 
   rf_stage_rows<KM>(ids, T, k, rows);
   const FastDiv node_of(epn), dev_of(epd);
   int key[KM];
-  rf_sorted_keys<KM>(rows + threadIdx.x * (KM + 1), valid, k, E, err, key);
-  const unsigned long long cnt = rf_node_counts<KM>(key, node_of);
-  int dc = 0, prev = -1;   // distinct devices of the token: the device changes along the sorted ids
+  int dc = 0;   // distinct devices of the token
+  if (E <= 64 * epd) {   // at most 64 devices: a bit per device, the ids need no order
+    rf_keys<KM>(rows + threadIdx.x * (KM + 1), valid, k, E, err, key);
+    unsigned long long seen = 0;
 #pragma unroll
-  for (int s = 0; s < KM; ++s)
-    if (key[s] != INT_MAX) {
-      const int dv = dev_of(key[s] >> 8);
-      dc += dv != prev;
-      prev = dv;
-    }
+    for (int s = 0; s < KM; ++s)
+      if (key[s] != INT_MAX) seen |= 1ull << dev_of(key[s] >> 8);
+    dc = __popcll(seen);
+  } else {   // the device changes along the sorted ids
+    rf_sorted_keys<KM>(rows + threadIdx.x * (KM + 1), valid, k, E, err, key);
+    int prev = -1;
+#pragma unroll
+    for (int s = 0; s < KM; ++s)
+      if (key[s] != INT_MAX) {
+        const int dv = dev_of(key[s] >> 8);
+        dc += dv != prev;
+        prev = dv;
+      }
+  }
+  const unsigned long long cnt = rf_node_counts<KM>(key, node_of);
 #pragma unroll
   for (int n = 0; n < RF_NODES; ++n) {
     int v = rf_packed(cnt, n);
@@ -832,8 +847,20 @@ __global__ void __launch_bounds__(RF_SCAN_THREADS) rbd_fast_scan_kernel(int ntil
   for (int base = 0; base < ntiles; base += RF_SCAN_THREADS * RF_RUN) {
     const int nt = min(RF_SCAN_THREADS * RF_RUN, ntiles - base);   // tiles in this pass
     const long long g0 = static_cast<long long>(base) * RF_NODES;
-    for (int i = threadIdx.x; i < nt * RF_NODES; i += RF_SCAN_THREADS)
-      s_tok[(i / (RF_RUN * RF_NODES)) * RF_ROW + i % (RF_RUN * RF_NODES)] = tile_cnt[g0 + i];
+    constexpr int PASS_INTS = RF_SCAN_THREADS * RF_RUN * RF_NODES;
+    if (nt == RF_SCAN_THREADS * RF_RUN) {   // a whole pass: every load of the thread in flight at once
+      int x[PASS_INTS / RF_SCAN_THREADS];
+#pragma unroll
+      for (int q = 0; q < PASS_INTS / RF_SCAN_THREADS; ++q) x[q] = tile_cnt[g0 + q * RF_SCAN_THREADS + threadIdx.x];
+#pragma unroll
+      for (int q = 0; q < PASS_INTS / RF_SCAN_THREADS; ++q) {
+        const int i = q * RF_SCAN_THREADS + threadIdx.x;
+        s_tok[(i / (RF_RUN * RF_NODES)) * RF_ROW + i % (RF_RUN * RF_NODES)] = x[q];
+      }
+    } else {
+      for (int i = threadIdx.x; i < nt * RF_NODES; i += RF_SCAN_THREADS)
+        s_tok[(i / (RF_RUN * RF_NODES)) * RF_ROW + i % (RF_RUN * RF_NODES)] = tile_cnt[g0 + i];
+    }
     for (int i = threadIdx.x; i < nt; i += RF_SCAN_THREADS) ds += tile_dev[base + i];
     __syncthreads();
     const int t0 = base + threadIdx.x * RF_RUN;

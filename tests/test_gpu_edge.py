@@ -123,14 +123,8 @@ def test_bounded_wait_gives_up_and_context_survives():
 
 
 
-@pytest.mark.gpu
-@pytest.mark.parametrize("E,k,epd,dpn", [(256, 8, 8, 4), (1024, 4, 16, 8)])
-def test_pft_and_rbd_four_million_assignments_match_oracle(E, k, epd, dpn):
-    # About 4.2 M assignments (2000+ sort chunks; RBD tiles past the scan's first pass).
-    from workloads.generate import make_topk_ids
-    T = (1 << 22) // k + 123
-    ids = make_topk_ids(T, E, k, seed=9, device="cuda")
-    w = torch.rand(T, k, device="cuda")
+def _pft_and_rbd_match_oracle(ids, w, E, k, epd, dpn):
+    T = ids.shape[0]
     N = T * k
     i32 = dict(device="cuda", dtype=torch.int32)
     tpe, off, tiles = torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(E + 1, **i32)
@@ -164,12 +158,40 @@ def test_pft_and_rbd_four_million_assignments_match_oracle(E, k, epd, dpn):
     P = r["num_pilots"]
     assert int(o["cnt"][0]) == P and int(o["cnt"][1]) == r["num_token_device_pairs"]
     assert np.array_equal(i64(o["ppn"]), r["pilots_per_node"])
+    assert np.array_equal(i64(o["noff"]), r["node_offsets"])
     assert np.array_equal(i64(o["ptok"][:P]), r["pilot_token"])
     assert np.array_equal(i64(o["pnode"][:P]), r["pilot_node"])
     assert np.array_equal(i64(o["pdev"][:P]), r["pilot_device"])
     assert np.array_equal(i64(o["roff"][:P + 1]), r["replica_offsets"])
     assert np.array_equal(i64(o["rexp"]), r["replica_expert"])
     assert np.array_equal(i64(o["ap"]), r["assign_pilot"])
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("E,k,epd,dpn", [(256, 8, 8, 4), (1024, 4, 16, 8), (1024, 16, 2, 64)])
+def test_pft_and_rbd_four_million_assignments_match_oracle(E, k, epd, dpn):
+    # About 4.2 M assignments (2000+ sort chunks; RBD tiles past the scan's first pass).  The last map
+    # has 8 nodes of 64 devices each: the per-token plan with more than 64 devices.
+    from workloads.generate import make_topk_ids
+    T = (1 << 22) // k + 123
+    ids = make_topk_ids(T, E, k, seed=9, device="cuda")
+    w = torch.rand(T, k, device="cuda")
+    _pft_and_rbd_match_oracle(ids, w, E, k, epd, dpn)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("E,k,epd,dpn", [(64, 8, 2, 4), (64, 8, 1, 16), (64, 8, 1, 1), (512, 32, 1, 64)])
+def test_pft_and_rbd_with_repeated_ids_match_oracle(E, k, epd, dpn):
+    # Ids drawn with repetition, so a token can name one expert in several slots: the PFT keeps the
+    # slots in order, and the RBD plan lists the repeats as separate replicas of one pilot, after
+    # equal ids in slot order (the oracle's stable sort).  Maps: 8 nodes (per-token plan, up to 64
+    # devices), 4 nodes of 16 devices, 64 nodes (the sort-based plan), 8 nodes of 64 devices.
+    T = 20000 + 7
+    g = torch.Generator(device="cuda").manual_seed(17)
+    ids = torch.randint(0, E, (T, k), generator=g, device="cuda", dtype=torch.int32)
+    ids[:, 1] = ids[:, 0]   # at least one repeat in every token
+    w = torch.rand(T, k, device="cuda", generator=g)
+    _pft_and_rbd_match_oracle(ids, w, E, k, epd, dpn)
 
 
 @pytest.mark.gpu
