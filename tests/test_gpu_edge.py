@@ -195,6 +195,19 @@ def test_pft_and_rbd_with_repeated_ids_match_oracle(E, k, epd, dpn):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("E,k,epd,dpn", [(2048, 8, 32, 8), (4096, 6, 16, 16), (4096, 8, 4, 2)])
+def test_pft_and_rbd_wide_expert_ids_match_oracle(E, k, epd, dpn):
+    # More than 1024 experts: the PFT scatter finds equal keys with __match_any_sync (not ballots) and
+    # runs fewer warps per chunk; hundreds of chunks, so the chunk counts take the many-chunk scan.
+    # Maps: 8 nodes of 8 devices (per-token plan), 16 nodes and 512 nodes (sort-based plan).
+    T = 40000 + 3
+    g = torch.Generator(device="cuda").manual_seed(19)
+    ids = torch.randint(0, E, (T, k), generator=g, device="cuda", dtype=torch.int32)
+    w = torch.rand(T, k, device="cuda", generator=g)
+    _pft_and_rbd_match_oracle(ids, w, E, k, epd, dpn)
+
+
+@pytest.mark.gpu
 def test_rbd_many_nodes_general_path():
     # 64 nodes: more than the per-token fast plan handles, so the sort-based plan runs.
     from workloads.generate import make_topk_ids
