@@ -7,7 +7,7 @@
 //   1. chunk histograms counts[c][key];
 //   2. scan in (key, chunk) order -> per-key totals, key offsets and every chunk's base
 //      row for every key (plus the grouped-GEMM tile prefix): one CTA for few chunks, else
-//      a CTA per strip of keys and a key scan;
+//      a CTA per strip of keys, the last of which scans the key totals;
 //   3. scatter: warp w of a chunk owns keys [256w, 256w + 256) of it; the warps count
 //      their keys per key, take an exclusive prefix over warps, then walk their keys in
 //      order, 32 at a time; lanes holding the same key find each other (one ballot per
@@ -37,10 +37,12 @@ __device__ __forceinline__ long long dev_count(long long n, const int32_t* n_dev
 }
 
 // One CTA per chunk: shared histogram of the chunk's keys -> counts[chunk][key].
+// It also zeroes the strip scan's ticket counter.
 __global__ void chunk_hist_kernel(const int32_t* __restrict__ keys, long long n, const int32_t* n_dev, int K,
-                                  int nchunks, int32_t* __restrict__ counts, int32_t* err) {
+                                  int nchunks, int32_t* __restrict__ counts, unsigned* ticket, int32_t* err) {
   extern __shared__ int32_t sh[];
   const int chunk = blockIdx.x;
+  if (chunk == 0 && threadIdx.x == 0) *ticket = 0u;
   for (int i = threadIdx.x; i < K; i += blockDim.x) sh[i] = 0;
   __syncthreads();
   const long long nn = dev_count(n, n_dev);
@@ -147,18 +149,49 @@ __global__ void __launch_bounds__(SCAN_THREADS) chunk_scan_kernel(const int32_t*
   }
 }
 
+// Key totals -> offsets [K+1], optional tiles [K+1] (prefix of ceil(total/tile_rows)), optional copy of
+// totals: all threads of one CTA.  The totals are read from L2 (other CTAs wrote them).
+__device__ void key_scan_body(const int32_t* totals, int K, int32_t* totals_out, int32_t* offsets, int32_t* tiles,
+                              int tile_rows, int* tmp /*[32]*/) {
+  int carry = 0, tcarry = 0;
+  for (int k0 = 0; k0 < K; k0 += blockDim.x) {
+    const int key = k0 + threadIdx.x;
+    const int tot = key < K ? __ldcg(totals + key) : 0;
+    int blk, tblk;
+    const int excl = block_excl_scan(tot, tmp, &blk) + carry;
+    const int nt = tile_rows > 0 ? (tot + tile_rows - 1) / tile_rows : 0;
+    const int texcl = block_excl_scan(nt, tmp, &tblk) + tcarry;
+    if (key < K) {
+      if (totals_out) totals_out[key] = tot;
+      offsets[key] = excl;
+      if (tiles) tiles[key] = texcl;
+    }
+    carry += blk;
+    tcarry += tblk;
+  }
+  if (threadIdx.x == 0) {
+    offsets[K] = carry;
+    if (tiles) tiles[K] = tcarry;
+  }
+}
+
 // Many chunks: the [C][K] chunk counts scanned down their columns, for strips of STRIP_KEYS keys per
 // CTA; its 32 warps take consecutive row segments, a warp instruction covering 32 / STRIP_KEYS rows of
 // the strip.  Pass 1 sums each warp's segment per key, the segment sums are scanned per key across the
 // warps, and pass 2 writes each element's exclusive prefix (relative base) in the same order.  A narrow
 // strip spreads the scan over more SMs (K / STRIP_KEYS CTAs); the partly used sectors it reads are L2
-// hits, the counts having just been written.
+// hits, the counts having just been written.  The last CTA to finish (a ticket counter that the
+// histogram launch zeroed) turns the key totals into key offsets and tile offsets, which saves a launch.
 constexpr int STRIP_KEYS = 2;
 constexpr int STRIP_ROWS = 32 / STRIP_KEYS;   // rows per warp step
 
 __global__ void __launch_bounds__(SCAN_THREADS) strip_scan_kernel(const int32_t* __restrict__ counts, int C, int K,
-                                                                  int32_t* __restrict__ base, int32_t* totals) {
+                                                                  int32_t* __restrict__ base, int32_t* totals,
+                                                                  unsigned* ticket, int32_t* totals_out,
+                                                                  int32_t* offsets, int32_t* tiles, int tile_rows) {
   __shared__ int wsum[SCAN_THREADS / 32][STRIP_KEYS];
+  __shared__ int tmp[32];
+  __shared__ bool last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kk = lane % STRIP_KEYS, rsub = lane / STRIP_KEYS;   // key of the strip, row of a step
   const int key = blockIdx.x * STRIP_KEYS + kk;
@@ -189,6 +222,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) strip_scan_kernel(const int32_t*
       run += x;
     }
     if (blockIdx.x * STRIP_KEYS + lane < K) totals[blockIdx.x * STRIP_KEYS + lane] = run;
+    __threadfence();   // the totals are visible to the CTA that takes the last ticket
   }
   __syncthreads();
   int carry = wsum[warp][kk];
@@ -212,33 +246,12 @@ __global__ void __launch_bounds__(SCAN_THREADS) strip_scan_kernel(const int32_t*
       carry += __shfl_sync(0xffffffffu, x, (STRIP_ROWS - 1) * STRIP_KEYS + kk);
     }
   }
-}
-
-// Key totals -> offsets [K+1], optional tiles [K+1] (prefix of ceil(total/tile_rows)), optional copy of totals.
-__global__ void __launch_bounds__(SCAN_THREADS) key_scan_kernel(const int32_t* __restrict__ totals, int K,
-                                                                int32_t* totals_out, int32_t* offsets, int32_t* tiles,
-                                                                int tile_rows) {
-  __shared__ int tmp[32];
-  int carry = 0, tcarry = 0;
-  for (int k0 = 0; k0 < K; k0 += SCAN_THREADS) {
-    const int key = k0 + threadIdx.x;
-    const int tot = key < K ? totals[key] : 0;
-    int blk, tblk;
-    const int excl = block_excl_scan(tot, tmp, &blk) + carry;
-    const int nt = tile_rows > 0 ? (tot + tile_rows - 1) / tile_rows : 0;
-    const int texcl = block_excl_scan(nt, tmp, &tblk) + tcarry;
-    if (key < K) {
-      if (totals_out) totals_out[key] = tot;
-      offsets[key] = excl;
-      if (tiles) tiles[key] = texcl;
-    }
-    carry += blk;
-    tcarry += tblk;
-  }
-  if (threadIdx.x == 0) {
-    offsets[K] = carry;
-    if (tiles) tiles[K] = tcarry;
-  }
+  if (threadIdx.x == 0) last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  key_scan_body(totals, K, totals_out, offsets, tiles, tile_rows, tmp);
+  if (threadIdx.x == 0) *ticket = 0u;
 }
 
 // Stable scatter.  Pass 1 counts each warp's keys.  Pass 2 gives every element its sorted row p
@@ -286,7 +299,7 @@ __global__ void __launch_bounds__(256, 5) chunk_scatter_kernel(const int32_t* __
   const int nw = blockDim.x >> 5;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x;
-  int32_t* cnt = sh;                                   // [nw][K]: counts, then each warp's start in its key's run
+  int32_t* cnt = sh;                                   // [nw][K]: counts, then each warp's first staging slot
   int32_t* lbase = cnt + static_cast<long long>(nw) * K;   // [K]: first staging slot of each key
   int32_t* gbase = lbase + K;                          // [K]: first sorted row of each key in this chunk
   int32_t* skey = gbase + K;                           // [nw * KPW]: staged keys, in sorted order
@@ -315,14 +328,18 @@ __global__ void __launch_bounds__(256, 5) chunk_scatter_kernel(const int32_t* __
   for (int it = 0; it < IT; ++it)
     if (static_cast<unsigned>(key[it]) < static_cast<unsigned>(K)) atomicAdd(&wcnt[key[it]], 1);
   __syncthreads();
-  // per key: each warp's start within the key's run of this chunk, the run length, the first row
+  // per key: the run length in this chunk and its first row (a thread keeps its key's warp counts
+  // in registers when it has one key)
+  const bool one_key = K <= static_cast<int>(blockDim.x);
+  int wc[8];   // nw <= 8
   for (int k = threadIdx.x; k < K; k += blockDim.x) {
     int run = 0;
-    for (int w2 = 0; w2 < nw; ++w2) {
-      const int c = cnt[w2 * K + k];
-      cnt[w2 * K + k] = run;
-      run += c;
-    }
+#pragma unroll
+    for (int w2 = 0; w2 < 8; ++w2)
+      if (w2 < nw) {
+        wc[w2] = cnt[w2 * K + k];
+        run += wc[w2];
+      }
     lbase[k] = run;
     gbase[k] = k == threadIdx.x ? gfirst
                                 : (chunk < nchunks ? key_offsets[k] + base[static_cast<long long>(chunk) * K + k] : 0);
@@ -342,6 +359,27 @@ __global__ void __launch_bounds__(256, 5) chunk_scatter_kernel(const int32_t* __
     carry += blk;
   }
   if (threadIdx.x == 0) staged = carry;
+  // each warp's first staging slot of each key
+  if (one_key) {
+    if (static_cast<int>(threadIdx.x) < K) {
+      int run = lbase[threadIdx.x];
+#pragma unroll
+      for (int w2 = 0; w2 < 8; ++w2)
+        if (w2 < nw) {
+          cnt[w2 * K + threadIdx.x] = run;
+          run += wc[w2];
+        }
+    }
+  } else {
+    for (int k = threadIdx.x; k < K; k += blockDim.x) {
+      int run = lbase[k];
+      for (int w2 = 0; w2 < nw; ++w2) {
+        const int c = cnt[w2 * K + k];
+        cnt[w2 * K + k] = run;
+        run += c;
+      }
+    }
+  }
   __syncthreads();
   // pass 2: rows in key order within the warp; source-indexed outputs now, the rest staged
 #pragma unroll
@@ -355,8 +393,7 @@ __global__ void __launch_bounds__(256, 5) chunk_scatter_kernel(const int32_t* __
     __syncwarp();
     if (ok) {
       const long long i = b + it * 32 + lane;
-      const int r = c0 + rank;
-      const int lp = lbase[key[it]] + r;
+      const int lp = c0 + rank;   // staging slot
       sink.at_source(i, gbase[key[it]] + lp);
       int32_t pa, pb;
       sink.payload(i, pre[it], pa, pb);
@@ -1089,19 +1126,19 @@ int rows_grid(long long rows, int warps_per_blk = 8) {
 }
 
 // Chunk counts -> relative bases + key totals/offsets/tiles: one CTA while the chunks are few, else a
-// CTA per strip of keys (strip_scan) and a key scan.  key_tot receives the totals on the many-chunk path.
+// CTA per strip of keys (strip_scan, whose last CTA scans the keys).  key_tot [K] and the ticket
+// (zeroed by the histogram launch) serve the many-chunk path.
 constexpr int SMALL_CHUNKS = 64;
 
 int sort_scan(const int32_t* counts, int C, int K, int32_t* totals, int32_t* offsets, int32_t* base, int32_t* tiles,
-              int tile_rows, int32_t* key_tot, const char* name, cudaStream_t s) {
+              int tile_rows, int32_t* key_tot, unsigned* ticket, const char* name, cudaStream_t s) {
   if (C <= SMALL_CHUNKS) {
     PFMOE_LAUNCH(name, s,
                  chunk_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(counts, C, K, totals, offsets, base, tiles, tile_rows));
     return PFMOE_OK;
   }
-  PFMOE_LAUNCH(name, s, strip_scan_kernel<<<(K + STRIP_KEYS - 1) / STRIP_KEYS, SCAN_THREADS, 0, s>>>(counts, C, K, base,
-                                                                                            key_tot));
-  PFMOE_LAUNCH(name, s, key_scan_kernel<<<1, SCAN_THREADS, 0, s>>>(key_tot, K, totals, offsets, tiles, tile_rows));
+  PFMOE_LAUNCH(name, s, strip_scan_kernel<<<(K + STRIP_KEYS - 1) / STRIP_KEYS, SCAN_THREADS, 0, s>>>(
+                            counts, C, K, base, key_tot, ticket, totals, offsets, tiles, tile_rows));
   return PFMOE_OK;
 }
 
@@ -1119,10 +1156,10 @@ int scatter_smem_attr() {
 
 // Histogram + scatter launches of one stable counting sort.
 int sort_hist(const int32_t* keys, long long n_max, const int32_t* n_dev, int K, int C, int32_t* counts,
-              int32_t* err, const char* name, cudaStream_t s) {
+              unsigned* ticket, int32_t* err, const char* name, cudaStream_t s) {
   const int wpb = warps_per_block(K);
   PFMOE_LAUNCH(name, s, (chunk_hist_kernel<<<C, wpb * 32, K * sizeof(int32_t), s>>>(keys, n_max, n_dev, K, C, counts,
-                                                                                   err)));
+                                                                                   ticket, err)));
   return PFMOE_OK;
 }
 
@@ -1189,9 +1226,10 @@ static int rbd_fast_impl(const int32_t* ids, int T, int k, int E, int epd, int e
 
 }  // namespace
 
+// Counts and bases ([C][K] each), key totals [K], the strip scan's ticket.
 size_t csort_ws_bytes(long long n_max, int K) {
   const long long C = (n_max + chunk_keys(K) - 1) / chunk_keys(K);
-  return static_cast<size_t>(2 * (C > 0 ? C : 1) * static_cast<long long>(K) + K) * sizeof(int32_t);
+  return static_cast<size_t>(2 * (C > 0 ? C : 1) * static_cast<long long>(K) + K + 1) * sizeof(int32_t);
 }
 
 int pft_build_impl(const int32_t* ids, const float* w, int T, int E, int k, int32_t* tpe, int32_t* offsets,
@@ -1201,9 +1239,10 @@ int pft_build_impl(const int32_t* ids, const float* w, int T, int E, int k, int3
   const int C = static_cast<int>((N + chunk_keys(E) - 1) / chunk_keys(E));
   int32_t* counts = static_cast<int32_t*>(ws);
   int32_t* base = counts + static_cast<long long>(C) * E;
-  if (C > 0) PFMOE_TRY(sort_hist(ids, N, nullptr, E, C, counts, err, "pft_hist", s));
   int32_t* key_tot = base + static_cast<long long>(C) * E;
-  PFMOE_TRY(sort_scan(counts, C, E, tpe, offsets, base, tile_offsets, 128, key_tot, "pft_scan", s));
+  unsigned* ticket = reinterpret_cast<unsigned*>(key_tot + E);
+  if (C > 0) PFMOE_TRY(sort_hist(ids, N, nullptr, E, C, counts, ticket, err, "pft_hist", s));
+  PFMOE_TRY(sort_scan(counts, C, E, tpe, offsets, base, tile_offsets, 128, key_tot, ticket, "pft_scan", s));
   PftSink sink{w, k, k > 1 ? ~0ull / static_cast<unsigned>(k) + 1 : 0ull, pos, token_ids, expert_ids, cw};
   if (C > 0) PFMOE_TRY(sort_scatter<PftSink>(ids, N, nullptr, E, C, base, offsets, sink, "pft_scatter", s));
   return PFMOE_OK;
@@ -1267,9 +1306,10 @@ int rbd_plan_impl(const int32_t* ids, int T, int k, int E, int epd, int dpn, int
     PFMOE_LAUNCH("rbd_scan_tokens", s, tile_scan_kernel<<<nt, SCAN_THREADS, 0, s>>>(ucount, T, nullptr, tsum_a, pbase));
   }
   PFMOE_RBD_LAUNCH("rbd_emit", rbd_emit_kernel, T, k, s, ids, T, k, E, epd, epn, pbase, pkey, ptoken, prc, err);
-  if (C > 0) PFMOE_TRY(sort_hist(pkey, pmax, counts, n_nodes, C, ccounts, err, "rbd_hist", s));
   int32_t* node_tot = cbase + static_cast<long long>(C > 0 ? C : 1) * n_nodes;
-  PFMOE_TRY(sort_scan(ccounts, C, n_nodes, pilots_per_node, node_offsets, cbase, nullptr, 0, node_tot,
+  unsigned* ticket = reinterpret_cast<unsigned*>(node_tot + n_nodes);
+  if (C > 0) PFMOE_TRY(sort_hist(pkey, pmax, counts, n_nodes, C, ccounts, ticket, err, "rbd_hist", s));
+  PFMOE_TRY(sort_scan(ccounts, C, n_nodes, pilots_per_node, node_offsets, cbase, nullptr, 0, node_tot, ticket,
                       "rbd_scan_nodes", s));
   if (C > 0) {
     RbdSink sink{ptoken, prc, pilot_token, pilot_node, rc_sorted, psorted};
