@@ -740,31 +740,57 @@ __device__ __forceinline__ void rf_stage_rows(const int32_t* __restrict__ ids, i
   __syncthreads();
 }
 
-// The token's ids as sort keys id * 256 + slot, in ascending order (slots k .. KM - 1 and tokens past
-// T hold INT_MAX).  Ids outside [0, E) are flagged (when err is given) and read as 0.  Node and device
-// are monotone in the id, so each node's replicas form one run of the sorted keys, in (id, slot) order,
-// and the run's first key is the node's lowest id.  Bitonic sorting network, unrolled over KM.
+// The token's k ids, from its padded row of the staged tile, or, for k = KM and 16-byte aligned ids,
+// straight from global memory as KM / 4 16-byte vectors: a warp's loads then cover its 32 tokens'
+// ids contiguously, and the staging round trip through shared memory (and its barrier) is skipped.
 template <int KM>
-__device__ __forceinline__ void rf_keys(const int32_t* row, bool valid, int k, int E, int32_t* err, int (&key)[KM]) {
+__device__ __forceinline__ bool rf_direct(const int32_t* ids, int k) {
+  return k == KM && (reinterpret_cast<uintptr_t>(ids) & 15) == 0;
+}
+
+template <int KM>
+__device__ __forceinline__ void rf_ids_direct(const int32_t* __restrict__ ids, long long t, bool valid, int (&v)[KM]) {
+  const int4* src = reinterpret_cast<const int4*>(ids + t * KM);
+#pragma unroll
+  for (int q = 0; q < KM / 4; ++q) {
+    const int4 x = valid ? src[q] : make_int4(0, 0, 0, 0);
+    v[4 * q] = x.x;
+    v[4 * q + 1] = x.y;
+    v[4 * q + 2] = x.z;
+    v[4 * q + 3] = x.w;
+  }
+}
+
+template <int KM>
+__device__ __forceinline__ void rf_ids_row(const int32_t* row, bool valid, int k, int (&v)[KM]) {
+#pragma unroll
+  for (int j = 0; j < KM; ++j) v[j] = valid && j < k ? row[j] : 0;
+}
+
+// The token's ids as sort keys id * 256 + slot (slots k .. KM - 1 and tokens past T hold INT_MAX).
+// Ids outside [0, E) are flagged (when err is given) and read as 0.
+template <int KM>
+__device__ __forceinline__ void rf_keys(const int (&v)[KM], bool valid, int k, int E, int32_t* err, int (&key)[KM]) {
 #pragma unroll
   for (int j = 0; j < KM; ++j) {
     int x = INT_MAX;
     if (valid && j < k) {
-      int v = row[j];
-      if (static_cast<unsigned>(v) >= static_cast<unsigned>(E)) {
+      int id = v[j];
+      if (static_cast<unsigned>(id) >= static_cast<unsigned>(E)) {
         if (err) dev_error(err, PFMOE_DEV_BAD_EXPERT_ID);
-        v = 0;
+        id = 0;
       }
-      x = (v << 8) | j;
+      x = (id << 8) | j;
     }
     key[j] = x;
   }
 }
 
+// Keys in ascending order.  Node and device are monotone in the id, so each node's replicas then form
+// one run of the sorted keys, in (id, slot) order, and the run's first key is the node's lowest id.
+// Bitonic sorting network, unrolled over KM.
 template <int KM>
-__device__ __forceinline__ void rf_sorted_keys(const int32_t* row, bool valid, int k, int E, int32_t* err,
-                                               int (&key)[KM]) {
-  rf_keys<KM>(row, valid, k, E, err, key);
+__device__ __forceinline__ void rf_sort(int (&key)[KM]) {
 #pragma unroll
   for (int size = 2; size <= KM; size <<= 1)
 #pragma unroll
@@ -811,19 +837,25 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_count_kernel(const int32_t* 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long t = static_cast<long long>(blockIdx.x) * RF_TILE + threadIdx.x;
   const bool valid = t < T;
-  rf_stage_rows<KM>(ids, T, k, rows);
+  int v[KM];
+  if (rf_direct<KM>(ids, k)) {
+    rf_ids_direct<KM>(ids, t, valid, v);
+  } else {
+    rf_stage_rows<KM>(ids, T, k, rows);
+    rf_ids_row<KM>(rows + threadIdx.x * (KM + 1), valid, k, v);
+  }
   const FastDiv node_of(epn), dev_of(epd);
   int key[KM];
+  rf_keys<KM>(v, valid, k, E, err, key);
   int dc = 0;   // distinct devices of the token
   if (E <= 64 * epd) {   // at most 64 devices: a bit per device, the ids need no order
-    rf_keys<KM>(rows + threadIdx.x * (KM + 1), valid, k, E, err, key);
     unsigned long long seen = 0;
 #pragma unroll
     for (int s = 0; s < KM; ++s)
       if (key[s] != INT_MAX) seen |= 1ull << dev_of(key[s] >> 8);
     dc = __popcll(seen);
   } else {   // the device changes along the sorted ids
-    rf_sorted_keys<KM>(rows + threadIdx.x * (KM + 1), valid, k, E, err, key);
+    rf_sort<KM>(key);
     int prev = -1;
 #pragma unroll
     for (int s = 0; s < KM; ++s)
@@ -1013,14 +1045,21 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_emit_kernel(
     tok_base[threadIdx.x] = node_offsets[threadIdx.x] + tile_tok_base[tb + threadIdx.x];
     rep_gbase[threadIdx.x] = node_rep_off[threadIdx.x] + tile_rep_base[tb + threadIdx.x];
   }
-  rf_stage_rows<KM>(ids, T, k, rows);
-  (void)err;   // rbd_fast_count flagged bad ids
-  const FastDiv node_of(epn), dev_of(epd);
   int32_t* row = rows + threadIdx.x * (KM + 1);
   unsigned long long cnt;
+  (void)err;   // rbd_fast_count flagged bad ids
+  const FastDiv node_of(epn), dev_of(epd);
   {
+    int v[KM];
+    if (rf_direct<KM>(ids, k)) {
+      rf_ids_direct<KM>(ids, t, valid, v);
+    } else {
+      rf_stage_rows<KM>(ids, T, k, rows);
+      rf_ids_row<KM>(row, valid, k, v);
+    }
     int key[KM];
-    rf_sorted_keys<KM>(row, valid, k, E, nullptr, key);
+    rf_keys<KM>(v, valid, k, E, nullptr, key);
+    rf_sort<KM>(key);
 #pragma unroll
     for (int s = 0; s < KM; ++s) row[s] = key[s];
     cnt = rf_node_counts<KM>(key, node_of);
