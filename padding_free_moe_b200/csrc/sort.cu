@@ -866,15 +866,13 @@ __global__ void __launch_bounds__(RF_TILE) rbd_fast_count_kernel(const int32_t* 
       }
   }
   const unsigned long long cnt = rf_node_counts<KM>(key, node_of);
+  // warp sums by the hardware reduction (the packed fields stay below 2^16: 32 flags, 32 k replicas)
 #pragma unroll
   for (int n = 0; n < RF_NODES; ++n) {
-    int v = rf_packed(cnt, n);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int v = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(rf_packed(cnt, n))));
     if (lane == 0) red[warp][n] = v;
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) dc += __shfl_xor_sync(0xffffffffu, dc, o);
+  dc = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(dc)));
   if (lane == 0) red[warp][RF_NODES] = dc;
   __syncthreads();
   if (threadIdx.x <= RF_NODES) {
