@@ -163,6 +163,30 @@ def test_pft_against_buckets_and_invariants(seed):
     assert p["tile_offsets"].tolist() == [0] + list(np.cumsum(tiles))
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_pft_with_repeated_ids_keeps_slot_order(seed):
+    # A token may name one expert in several slots (the entry points accept any ids in [0, E)):
+    # the stable sort then keeps those slots in slot order, next to each other.
+    r = rng(40 + seed)
+    T = int(r.integers(1, 40)); E = int(r.integers(1, 6)); k = int(r.integers(2, 9))
+    ids = r.integers(0, E, size=(T, k))
+    ids[:, 1] = ids[:, 0]
+    w = r.random((T, k))
+    p = O.pft_build(ids, w, E)
+    counts, order = _bucket_sort_reference(ids, E)
+    assert p["tokens_per_expert"].tolist() == counts
+    assert p["token_ids"].tolist() == [t for t, _ in order]
+    np.testing.assert_array_equal(p["combine_weights"], [w[t, j] for t, j in order])
+    for t in range(T):
+        for j in range(k):
+            q = p["pos"][t, j]
+            assert p["token_ids"][q] == t and p["expert_ids"][q] == ids[t, j]
+        for j in range(1, k):   # equal ids of one token: rows in slot order
+            for i in range(j):
+                if ids[t, i] == ids[t, j]:
+                    assert p["pos"][t, i] < p["pos"][t, j]
+
+
 def test_pft_rejects_bad_ids():
     with pytest.raises(ValueError):
         O.pft_build(np.array([[0, 5]]), np.ones((1, 2)), 4)
@@ -426,6 +450,33 @@ def test_rbd_bruteforce_tiny():
                     assert got["pilots_per_node"].tolist() == cnt
                     n_cases += 1
     assert n_cases > 100
+
+
+def test_rbd_bruteforce_repeated_ids():
+    # Ids drawn with repetition: one pilot per (token, node) still, the repeats listed as separate
+    # replicas of it, every repeated slot assigned to that pilot, one (token, device) pair per device.
+    r = rng(71)
+    n_cases = 0
+    for E in (2, 4, 8, 12):
+        for epd in (1, 2):
+            for dpn in (1, 2):
+                if E % (epd * dpn):
+                    continue
+                for k in (2, 3, 5, 8):
+                    T = int(r.integers(1, 9))
+                    ids = r.integers(0, E, size=(T, k))
+                    got = O.rbd_plan(ids, E, epd, dpn)
+                    pilots, assign, npairs = _rbd_bruteforce(ids, E, epd, dpn)
+                    assert got["num_pilots"] == len(pilots)
+                    assert got["pilot_token"].tolist() == [p[0] for p in pilots]
+                    assert got["pilot_node"].tolist() == [p[1] for p in pilots]
+                    assert got["replica_expert"].tolist() == [e for p in pilots for e in p[2]]
+                    assert got["replica_offsets"].tolist() == [0] + list(np.cumsum([len(p[2]) for p in pilots]))
+                    assert got["pilot_device"].tolist() == [p[2][0] // epd for p in pilots]
+                    assert got["assign_pilot"].tolist() == assign.tolist()
+                    assert got["num_token_device_pairs"] == npairs
+                    n_cases += 1
+    assert n_cases > 40
 
 
 @pytest.mark.parametrize("E,k,epd,dpn,expect", [
